@@ -1,0 +1,270 @@
+/*
+ * Sparse-BitLinear forward: CPU ORACLE.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the plain, slow, literal restatement of
+ * what the Sparse-BitLinear forward computes.  It is used by the test-suite, by the
+ * smoke check and by the benchmark's CPU-baseline leg, and by nothing else.  It
+ * shares no code, header, table or helper with the CUDA library; neither side
+ * includes or links the other.
+ *
+ * Sources (web pages; cited by title and section):
+ *   [SBN-es]  "Sparse-BitNet: 1.58-bit LLMs are Naturally Friendly to Semi-Structured
+ *             Sparsity", gist.science technical summary (Spanish), section
+ *             "2. Metodología: Sparse-BitNet" (Sparse-BitLinear, mask generation,
+ *             quant-then-mask order, dynamic recomputation).
+ *   [SBN-ar]  Same paper, gist.science technical summary (Arabic), section 2
+ *             "Methodology: Sparse-BitNet" (items 1-3 of the Sparse-BitLinear
+ *             architecture; "mask generation" and "quant-then-mask order").
+ *   [BitNet.cpp] "Marco de inferencia de Microsoft lleva modelos de lenguaje grande de
+ *             1 bit a dispositivos locales" (unite.ai), section "Fundamento
+ *             matemático", items 2 (activation quantisation) and 3 (BitLinear op).
+ *   [BitNet-proj] "Introducción Detallada al Proyecto BitNet" (aibars.net), section
+ *             "Especificaciones Técnicas" (W1.58A8, absmean weights, 8-bit activations,
+ *             no bias).
+ *
+ * Readings where the pages are silent (each one is listed in the design notes):
+ *   - gamma is per tensor, over all masters before masking, and the mean |W| is taken
+ *     as an exact integer sum of trunc(|W| * 2^24) so that it does not depend on the
+ *     summation order; eps is added in fp32.
+ *   - round() is round-half-to-even; W/g and 127*x/s are IEEE fp32 divisions, because
+ *     fp32 is the precision in which the GPU takes the same integer decisions.
+ *   - M-groups run along the input dimension K inside one output row; the top-N rule
+ *     ranks |W_master| and the lower index wins a tie.
+ *   - Qb = 127, symmetric clip to [-127, 127]; the per-token scale is
+ *     max(max|x|, 1e-5).
+ *   - y = acc * g * s / 127 is evaluated in fp64 here (no rounding order is fixed by
+ *     the pages); the GPU's fp32 result is compared to it with a relative tolerance.
+ *
+ * Build: gcc -O2 -ffp-contract=off -fno-fast-math -fopenmp -shared -fPIC.
+ */
+#include <fenv.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_ERR_W_NONFINITE 1
+#define ORACLE_ERR_W_RANGE 2
+#define ORACLE_ERR_X_NONFINITE 4
+#define ORACLE_ERR_ACC_OVERFLOW 8
+
+static float bf16_bits_to_float(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+/* 1 when the host FPU rounds to nearest-even (every decision below assumes it). */
+int oracle_rounding_is_nearest(void) { return fegetround() == FE_TONEAREST; }
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/*
+ * S1: per-tensor absmean scale [SBN-ar §2 item 1: gamma is the mean absolute value of
+ * the weights; BitNet-proj: "absmean" weight quantisation].
+ *   S     = sum_i trunc(|W_i| * 2^24)                 (exact, unsigned 64-bit)
+ *   gamma = fp32( fp64(S) / (fp64(n) * 2^24) )
+ *   g     = fp32( gamma + eps )
+ * Elements that are NaN/Inf set ORACLE_ERR_W_NONFINITE, elements with |W| >= 256 set
+ * ORACLE_ERR_W_RANGE; such elements are left out of S (the outputs are then
+ * unspecified).  Returns the error bits.
+ */
+int oracle_weight_gamma(const uint16_t *W, int64_t n, float eps, uint64_t *S_out,
+                        float *gamma_out, float *g_out) {
+  uint64_t S = 0;
+  int err = 0;
+#pragma omp parallel for reduction(+ : S) reduction(| : err) schedule(static)
+  for (int64_t i = 0; i < n; ++i) {
+    float a = fabsf(bf16_bits_to_float(W[i]));
+    if (!isfinite(a)) {
+      err |= ORACLE_ERR_W_NONFINITE;
+      continue;
+    }
+    if (a >= 256.0f) {
+      err |= ORACLE_ERR_W_RANGE;
+      continue;
+    }
+    double scaled = (double)a * 16777216.0; /* exact: 8-bit significand times 2^24 */
+    S += (uint64_t)scaled;                  /* C conversion truncates toward zero */
+  }
+  float gamma = (float)((double)S / ((double)n * 16777216.0));
+  float g = gamma + eps;
+  if (S_out) *S_out = S;
+  if (gamma_out) *gamma_out = gamma;
+  if (g_out) *g_out = g;
+  return err;
+}
+
+/*
+ * S2: ternary code of one master weight [SBN-ar §2 item 1; BitNet-proj "Especificaciones
+ * Técnicas"]: t = clamp(round(w / g), -1, 1) with an fp32 division and round-half-even.
+ * A NaN quotient (only 0/0, when g == 0 and w == +-0) gives 0.
+ */
+static int8_t ternary_code(float w, float g) {
+  float q = w / g;
+  float r = rintf(q);
+  if (r >= 1.0f) return 1;
+  if (r <= -1.0f) return -1;
+  return 0;
+}
+
+/*
+ * S2 + S3 + S4(apply): codes, N:M mask and masked codes for a [O, K] master matrix.
+ * Mask [SBN-es §2 "Generación de Máscara"; SBN-ar §2 "mask generation"]: inside each
+ * group of M consecutive weights along K (aligned at multiples of M) keep position i iff
+ *   #{ j in group : |W_j| > |W_i|  or  (|W_j| == |W_i| and j < i) }  <  N,
+ * i.e. the N largest master magnitudes, lower index first on ties.
+ * Order [SBN-es §2 "Orden de Operaciones"; SBN-ar §2 quant-then-mask]: the codes are
+ * computed from all masters first, then the mask zeroes the pruned positions:
+ *   ws = keep ? t : 0.
+ * Outputs are [O, K] int8 / uint8 arrays (t, keep in {0,1}, ws); any may be NULL.
+ */
+void oracle_ternary_mask(const uint16_t *W, int64_t O, int64_t K, int N, int M, float g,
+                         int8_t *t_out, uint8_t *keep_out, int8_t *ws_out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < O; ++r) {
+    for (int64_t base = 0; base < K; base += M) {
+      float mag[8];
+      for (int i = 0; i < M; ++i) mag[i] = fabsf(bf16_bits_to_float(W[r * K + base + i]));
+      for (int i = 0; i < M; ++i) {
+        int rank = 0;
+        for (int j = 0; j < M; ++j) {
+          if (j == i) continue;
+          if (mag[j] > mag[i] || (mag[j] == mag[i] && j < i)) ++rank;
+        }
+        int64_t idx = r * K + base + i;
+        uint8_t keep = (uint8_t)(rank < N);
+        int8_t t = ternary_code(bf16_bits_to_float(W[idx]), g);
+        if (t_out) t_out[idx] = t;
+        if (keep_out) keep_out[idx] = keep;
+        if (ws_out) ws_out[idx] = keep ? t : 0;
+      }
+    }
+  }
+}
+
+/*
+ * S4 (pack): the hardware format of the masked ternary matrix.  The pages ask for
+ * "well-defined N:M metadata on the discrete weights" [SBN-ar §2 quant-then-mask]; the
+ * layout below is this library's reading of it:
+ *   codes plane, row r: the kept positions of the row in ascending K order, 2 bits each
+ *     (0 -> 00, +1 -> 01, -1 -> 11), kept element e at bits 2*(e%4) of byte e/4;
+ *   meta plane, row r: one M-bit mask per group (bit i = position i of the group kept);
+ *     M == 8: one byte per group; M == 4: group 2h in the low nibble of byte h, group
+ *     2h+1 in the high nibble;
+ *   rows are ldc / ldm bytes apart; every byte past a row's data is zero.
+ * Returns 0, or -1 if some group does not keep exactly N positions.
+ */
+int oracle_pack(const int8_t *t, const uint8_t *keep, int64_t O, int64_t K, int N, int M,
+                uint8_t *codes, int64_t ldc, uint8_t *meta, int64_t ldm) {
+  int bad = 0;
+  memset(codes, 0, (size_t)(O * ldc));
+  memset(meta, 0, (size_t)(O * ldm));
+#pragma omp parallel for reduction(| : bad) schedule(static)
+  for (int64_t r = 0; r < O; ++r) {
+    int64_t e = 0;
+    for (int64_t k = 0; k < K; ++k) {
+      if (!keep[r * K + k]) continue;
+      int8_t v = t[r * K + k];
+      uint8_t code = (v == 0) ? 0u : (v == 1 ? 1u : 3u);
+      if (e / 4 >= ldc) { /* more kept positions than the plane holds */
+        bad = 1;
+        break;
+      }
+      codes[r * ldc + e / 4] |= (uint8_t)(code << (2 * (e % 4)));
+      ++e;
+    }
+    if (e != K / M * N) bad = 1;
+    for (int64_t gi = 0; gi < K / M; ++gi) {
+      unsigned bits = 0;
+      int kept = 0;
+      for (int i = 0; i < M; ++i) {
+        if (keep[r * K + gi * M + i]) {
+          bits |= 1u << i;
+          ++kept;
+        }
+      }
+      if (kept != N) bad = 1;
+      if (M == 8)
+        meta[r * ldm + gi] = (uint8_t)bits;
+      else
+        meta[r * ldm + gi / 2] |= (uint8_t)(bits << (4 * (gi % 2)));
+    }
+  }
+  return bad ? -1 : 0;
+}
+
+/*
+ * S5: per-token absmax int8 activations [BitNet.cpp "Fundamento matemático" item 2:
+ * x_q = Clip(x * Qb / gamma_x, -Qb + eps, Qb - eps), gamma_x = max |x|; BitNet-proj
+ * W1.58A8].  With Qb = 127:
+ *   s = max(max_k |x_k|, 1e-5)                         (fp32)
+ *   q = clamp(round_half_even((127 * x) / s), -127, 127)  (fp32 product is exact)
+ * X is [T, K] bf16 bits; Xq is [T, K] int8; s_out is [T] fp32.  Returns error bits.
+ */
+int oracle_quant_acts(const uint16_t *X, int64_t T, int64_t K, int8_t *Xq, float *s_out) {
+  int err = 0;
+#pragma omp parallel for reduction(| : err) schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
+    float a = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+      float v = fabsf(bf16_bits_to_float(X[t * K + k]));
+      if (!isfinite(v)) {
+        err |= ORACLE_ERR_X_NONFINITE;
+        continue;
+      }
+      if (v > a) a = v;
+    }
+    float s = (a < 1e-5f) ? 1e-5f : a;
+    s_out[t] = s;
+    for (int64_t k = 0; k < K; ++k) {
+      float x = bf16_bits_to_float(X[t * K + k]);
+      float r = rintf((127.0f * x) / s);
+      if (r > 127.0f) r = 127.0f;
+      if (r < -127.0f) r = -127.0f;
+      if (r != r) r = 0.0f; /* only reachable for non-finite x (flagged above) */
+      Xq[t * K + k] = (int8_t)r;
+    }
+  }
+  return err;
+}
+
+/*
+ * S6: exact integer contraction [BitNet.cpp item 3; the ternary product is a signed sum]:
+ *   acc[t, o] = sum_k Xq[t, k] * Ws[o, k]   (accumulated in int64, stored as int32)
+ * Returns ORACLE_ERR_ACC_OVERFLOW if any sum leaves the int32 range.
+ */
+int oracle_contract(const int8_t *Xq, const int8_t *Ws, int64_t T, int64_t O, int64_t K,
+                    int32_t *acc) {
+  int err = 0;
+#pragma omp parallel for reduction(| : err) schedule(static)
+  for (int64_t o = 0; o < O; ++o) {
+    for (int64_t t = 0; t < T; ++t) {
+      int64_t sum = 0;
+      for (int64_t k = 0; k < K; ++k) sum += (int64_t)Xq[t * K + k] * (int64_t)Ws[o * K + k];
+      if (sum > INT32_MAX || sum < INT32_MIN) err |= ORACLE_ERR_ACC_OVERFLOW;
+      acc[t * O + o] = (int32_t)sum;
+    }
+  }
+  return err;
+}
+
+/*
+ * S7: dequantising rescale [BitNet.cpp item 3: y = W x (beta * gamma / Qb)], here
+ *   y[t, o] = acc[t, o] * g * s[t] / 127    evaluated in fp64.
+ */
+void oracle_rescale(const int32_t *acc, const float *s, float g, int64_t T, int64_t O,
+                    double *y) {
+  for (int64_t t = 0; t < T; ++t)
+    for (int64_t o = 0; o < O; ++o)
+      y[t * O + o] = (double)acc[t * O + o] * (double)g * (double)s[t] / 127.0;
+}

@@ -1,0 +1,285 @@
+"""Checks that pin the CPU oracle to something other than itself.
+
+Each check raises AssertionError on a mismatch.  They are run against the real oracle
+(tests/test_oracle_pins.py) and against deliberately broken copies of it
+(tests/test_oracle_mutants.py), which must each fail at least one check.
+
+What pins what:
+  hand_example        every stage, against values worked out by hand (golden file)
+  mask_bruteforce     the top-N rule, against exhaustive search over all N-subsets
+  gamma_closed_form   S1, against the exact rational mean |W| (fractions.Fraction)
+  rounding_ties       round-half-to-even and the clip, on constructed exact ties
+  dense_pattern       n == m reduces to the plain (unmasked) b1.58 BitLinear
+  constant_magnitude  codes == sign(W) when all |W| are equal
+  act_absmax          the absmax element of every token maps to +-127; 0-token -> 0
+  contract_bruteforce S6, against an int64 sum written as a Python loop / numpy
+  unpack_roundtrip    the packed planes decode (independent decoder) to the masked codes
+  invariants          code range, no 0b10 pattern, N bits per group, zero padding
+  scale_invariance    W -> 2W leaves the mask and codes unchanged and doubles gamma
+  rescale_closed_form S7, against acc * g * s / 127 recomputed with Fraction
+"""
+import itertools
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_golden(name):
+    d = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            k, *v = line.split()
+            d[k] = v
+    return d
+
+
+def _f32(bits):
+    return workloads.bf16_bits_to_f32(bits)
+
+
+def hand_example(o):
+    g = _read_golden("hand_example_2of4.txt")
+    n, m = int(g["n"][0]), int(g["m"][0])
+    W = workloads.to_bf16_bits(np.array([[float(v) for v in g["W"]]], np.float32))
+    X = workloads.to_bf16_bits(np.array([[float(v) for v in g["x"]]], np.float32))
+    assert np.array_equal(_f32(W)[0], np.array([float(v) for v in g["W"]], np.float32))
+    r = o.linear(X, W, n, m, eps=float(g["eps"][0]))
+    assert r["err"] == 0 and r["xerr"] == 0
+    assert r["S"] == int(g["S"][0]), r["S"]
+    assert r["gamma"] == np.float32(float(g["gamma"][0])), r["gamma"]
+    assert r["t"][0].tolist() == [int(v) for v in g["t"]], r["t"]
+    assert r["keep"][0].tolist() == [int(v) for v in g["keep"]], r["keep"]
+    assert r["ws"][0].tolist() == [int(v) for v in g["ws"]], r["ws"]
+    assert r["codes"][0].tolist() == [int(v, 0) for v in g["codes"]], r["codes"]
+    assert r["meta"][0].tolist() == [int(v, 0) for v in g["meta"]], r["meta"]
+    assert r["s"][0] == np.float32(float(g["s"][0])), r["s"]
+    assert r["Xq"][0].tolist() == [int(v) for v in g["q"]], r["Xq"]
+    assert int(r["acc"][0, 0]) == int(g["acc"][0]), r["acc"]
+    y_exact = float(g["y_num"][0]) / float(g["y_den"][0])
+    assert abs(r["y"][0, 0] - y_exact) <= 1e-12 * abs(y_exact), r["y"]
+    # eps = 1e-5 moves g but no code: y follows acc * fp32(gamma + eps) * s / 127.
+    r2 = o.linear(X, W, n, m, eps=1e-5)
+    assert r2["ws"][0].tolist() == [int(v) for v in g["ws"]]
+    g2 = float(np.float32(np.float32(0.23046875) + np.float32(1e-5)))
+    y2 = float(Fraction(-119) * Fraction(g2) * 8 / 127)
+    assert abs(r2["y"][0, 0] - y2) <= 1e-12 * abs(y2), (r2["y"], y2)
+
+
+def _tie_heavy_masters(rows, K, seed):
+    rng = np.random.default_rng(seed)
+    vals = np.array([0.0, -0.0, 0.25, -0.25, 0.5, -0.5, 0.0625, 1.0, -1.0], np.float32)
+    a = rng.choice(vals, size=(rows, K))
+    # sprinkle distinct magnitudes so groups mix ties and non-ties
+    a += np.where(rng.random((rows, K)) < 0.3, rng.standard_normal((rows, K)) * 0.02, 0)
+    return workloads.to_bf16_bits(a.astype(np.float32))
+
+
+def mask_bruteforce(o):
+    for (n, m) in [(1, 4), (2, 4), (3, 4), (4, 4), (1, 8), (2, 8), (4, 8), (6, 8), (7, 8)]:
+        W = _tie_heavy_masters(6, 4 * m, seed=17 * n + m)
+        _, keep, _ = o.ternary_mask(W, n, m, np.float32(0.1))
+        mags = np.abs(_f32(W))
+        for r in range(W.shape[0]):
+            for base in range(0, W.shape[1], m):
+                grp = mags[r, base:base + m]
+                best = None
+                for sub in itertools.combinations(range(m), n):
+                    key = (sorted((float(grp[i]) for i in sub), reverse=True), [-i for i in sub])
+                    if best is None or key > best[0]:
+                        best = (key, sub)
+                want = np.zeros(m, np.uint8)
+                want[list(best[1])] = 1
+                got = keep[r, base:base + m]
+                assert np.array_equal(got, want), (n, m, r, base, grp, got, want)
+
+
+def gamma_closed_form(o):
+    for seed, (O, K) in enumerate([(7, 64), (64, 256), (33, 448)]):
+        W = workloads.masters(O, K, seed=100 + seed)
+        a = np.abs(_f32(W)).astype(np.float64)
+        exact = sum((Fraction(float(v)) for v in a.ravel() if v >= 2.0 ** -17), Fraction(0))
+        tiny = [float(v) for v in a.ravel() if 0 < v < 2.0 ** -17]
+        # values below 2^-17 are truncated at 2^-24 by the stated definition
+        exact += sum((Fraction(math.floor(v * 2 ** 24), 2 ** 24) for v in tiny), Fraction(0))
+        mean = exact / W.size
+        S, gamma, g, err = o.weight_gamma(W, 0.0)
+        assert err == 0
+        assert Fraction(S, 2 ** 24) == exact, (S, exact)
+        # gamma is fp32(fp64(S) / (n 2^24)): within one fp32 ulp of the exact mean
+        ulp = np.spacing(np.float32(float(mean)))
+        assert abs(Fraction(float(gamma)) - mean) <= Fraction(float(ulp)), (gamma, float(mean))
+        assert g == gamma
+        S2, gamma2, g2, _ = o.weight_gamma(W, 1e-5)
+        assert g2 == np.float32(gamma2 + np.float32(1e-5))
+    # a mean that is exactly representable comes out exactly
+    W = workloads.to_bf16_bits(np.array([[0.25, -0.75, 0.5, -0.5] * 16], np.float32))
+    S, gamma, g, err = o.weight_gamma(W, 0.0)
+    assert gamma == np.float32(0.5) and S == 32 * 2 ** 24
+    # the stated truncation: magnitudes below 2^-24 contribute nothing
+    W = workloads.to_bf16_bits(np.full((1, 64), 2.0 ** -30, np.float32))
+    assert o.weight_gamma(W, 0.0)[0] == 0
+
+
+def rounding_ties(o):
+    # mean |W| = 0.5 exactly; 0.25/0.5 = 0.5 -> 0 (even), 0.75/0.5 = 1.5 -> 2 -> clip 1
+    row = np.array([0.25, 0.75, 0.5, 0.5, -0.25, -0.75, -0.5, -0.5], np.float32)
+    W = workloads.to_bf16_bits(np.tile(row, (2, 8)))
+    S, gamma, g, _ = o.weight_gamma(W, 0.0)
+    assert g == np.float32(0.5)
+    t, keep, ws = o.ternary_mask(W, 8, 8, g)
+    assert t[0, :8].tolist() == [0, 1, 1, 1, 0, -1, -1, -1], t[0, :8]
+    # activations: absmax 127 -> q = x exactly; absmax 2 -> 127 x / 2 at exact .5 ties
+    x = np.array([[1.0, 0.5, -0.5, 1.5, -1.5, 2.0, 0.0, -2.0]], np.float32)
+    Xq, s, _ = o.quant_acts(workloads.to_bf16_bits(x))
+    # 127*[1,.5,-.5,1.5,-1.5,2,0,-2]/2 = 63.5 31.75 -31.75 95.25 -95.25 127 0 -127
+    assert Xq[0].tolist() == [64, 32, -32, 95, -95, 127, 0, -127], Xq
+    x = np.array([[0.5, 127.0, 62.5, -62.5, 61.5, -0.5, 1.5, 2.5]], np.float32)
+    Xq, s, _ = o.quant_acts(workloads.to_bf16_bits(x))
+    assert s[0] == 127 and Xq[0].tolist() == [0, 127, 62, -62, 62, 0, 2, 2], Xq
+
+
+def dense_pattern(o):
+    W = workloads.masters(5, 128, seed=5)
+    for m in (4, 8):
+        r = o.quantize_mask_pack(W, m, m, eps=1e-5)
+        assert r["keep"].all()
+        assert np.array_equal(r["ws"], r["t"])
+        ldm = r["meta"].shape[1]
+        assert (r["meta"][:, :128 // 8] == 0xFF).all() and (r["meta"][:, 128 // 8:ldm] == 0).all()
+        # plain b1.58: codes = clip(round(W / g)) with no mask
+        w = _f32(W)
+        want = np.clip(np.rint(w / r["g"]), -1, 1).astype(np.int8)
+        assert np.array_equal(r["t"], want)
+
+
+def constant_magnitude(o):
+    rng = np.random.default_rng(3)
+    sign = np.where(rng.random((4, 64)) < 0.5, -1.0, 1.0).astype(np.float32)
+    W = workloads.to_bf16_bits(sign * np.float32(0.0234375))
+    for n, m in [(2, 4), (6, 8)]:
+        r = o.quantize_mask_pack(W, n, m, eps=1e-5)
+        assert np.array_equal(r["t"], sign.astype(np.int8))
+        # all magnitudes tie: the first n positions of every group are kept
+        assert (r["keep"].reshape(4, -1, m)[:, :, :n] == 1).all()
+        assert (r["keep"].reshape(4, -1, m)[:, :, n:] == 0).all()
+
+
+def act_absmax(o):
+    X = workloads.activations(9, 256, seed=4)
+    X[3] = 0  # an all-zero token
+    Xq, s, err = o.quant_acts(X)
+    x = _f32(X)
+    assert err == 0
+    for t in range(9):
+        if t == 3:
+            assert s[t] == np.float32(1e-5) and (Xq[t] == 0).all()
+            continue
+        j = int(np.argmax(np.abs(x[t])))
+        assert s[t] == np.abs(x[t]).max()
+        assert Xq[t, j] == (127 if x[t, j] > 0 else -127)
+        assert np.abs(Xq[t]).max() == 127
+
+
+def contract_bruteforce(o):
+    rng = np.random.default_rng(9)
+    Xq = rng.integers(-127, 128, size=(5, 96), dtype=np.int64).astype(np.int8)
+    Ws = rng.integers(-1, 2, size=(7, 96), dtype=np.int64).astype(np.int8)
+    acc = o.contract(Xq, Ws)
+    for t in range(5):
+        for j in range(7):
+            want = 0
+            for k in range(96):
+                want += int(Xq[t, k]) * int(Ws[j, k])
+            assert int(acc[t, j]) == want, (t, j)
+    # a larger case against numpy's int64 matmul (operand order: tokens x outputs)
+    Xq = rng.integers(-127, 128, size=(33, 640), dtype=np.int64).astype(np.int8)
+    Ws = rng.integers(-1, 2, size=(65, 640), dtype=np.int64).astype(np.int8)
+    assert np.array_equal(o.contract(Xq, Ws), Xq.astype(np.int64) @ Ws.astype(np.int64).T)
+
+
+def unpack_planes(codes, meta, K, n, m):
+    """Independent decoder of the packed format, written from its description."""
+    O = codes.shape[0]
+    ws = np.zeros((O, K), np.int8)
+    for r in range(O):
+        e = 0
+        for gi in range(K // m):
+            if m == 8:
+                bits = int(meta[r, gi])
+            else:
+                bits = (int(meta[r, gi // 2]) >> (4 * (gi % 2))) & 0xF
+            for i in range(m):
+                if bits >> i & 1:
+                    c = (int(codes[r, e // 4]) >> (2 * (e % 4))) & 3
+                    assert c != 2, "code 0b10 is never written"
+                    ws[r, gi * m + i] = {0: 0, 1: 1, 3: -1}[c]
+                    e += 1
+    return ws
+
+
+def unpack_roundtrip(o):
+    for n, m, K in [(2, 4, 256), (6, 8, 192), (1, 8, 64), (3, 4, 64)]:
+        W = workloads.masters(9, K, seed=K + n)
+        r = o.quantize_mask_pack(W, n, m)
+        assert np.array_equal(unpack_planes(r["codes"], r["meta"], K, n, m), r["ws"])
+
+
+def invariants(o):
+    for n, m in [(2, 4), (6, 8)]:
+        W = workloads.masters(64, 320, seed=n * m)
+        r = o.quantize_mask_pack(W, n, m)
+        K = 320
+        assert set(np.unique(r["t"]).tolist()) <= {-1, 0, 1}
+        keep = r["keep"].reshape(64, -1, m)
+        assert (keep.sum(-1) == n).all()
+        assert ((r["ws"] != 0).reshape(64, -1, m).sum(-1) <= n).all()
+        assert np.array_equal(r["ws"], r["t"] * r["keep"])
+        used_c = K // m * n * 2 // 8
+        used_m = K // 8
+        assert (r["codes"][:, used_c:] == 0).all() and (r["meta"][:, used_m:] == 0).all()
+        c = r["codes"][:, :used_c]
+        for sh in (0, 2, 4, 6):
+            assert ((c >> sh) & 3 != 2).all()
+        if m == 4:
+            nib = np.concatenate([r["meta"][:, :used_m] & 0xF, r["meta"][:, :used_m] >> 4])
+        else:
+            nib = r["meta"][:, :used_m]
+        pop = np.unpackbits(nib.astype(np.uint8)[..., None], axis=-1).sum(-1)
+        assert (pop == n).all()
+
+
+def scale_invariance(o):
+    W = workloads.masters(16, 256, seed=21)
+    W2 = workloads.to_bf16_bits(_f32(W) * 2)
+    for n, m in [(2, 4), (6, 8)]:
+        a = o.quantize_mask_pack(W, n, m, eps=0.0)
+        b = o.quantize_mask_pack(W2, n, m, eps=0.0)
+        assert np.array_equal(a["keep"], b["keep"])
+        assert np.array_equal(a["ws"], b["ws"])
+        assert b["gamma"] == 2 * a["gamma"]
+
+
+def rescale_closed_form(o):
+    rng = np.random.default_rng(2)
+    acc = rng.integers(-2 ** 20, 2 ** 20, size=(3, 5)).astype(np.int32)
+    s = np.array([0.5, 3.25, 117.0], np.float32)
+    g = np.float32(0.0171875)
+    y = o.rescale(acc, s, g)
+    for t in range(3):
+        for j in range(5):
+            want = Fraction(int(acc[t, j])) * Fraction(float(g)) * Fraction(float(s[t])) / 127
+            assert abs(Fraction(float(y[t, j])) - want) <= abs(want) * Fraction(1, 2 ** 50)
+
+
+ALL = [hand_example, mask_bruteforce, gamma_closed_form, rounding_ties, dense_pattern,
+       constant_magnitude, act_absmax, contract_bruteforce, unpack_roundtrip, invariants,
+       scale_invariance, rescale_closed_form]

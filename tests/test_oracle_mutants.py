@@ -1,0 +1,63 @@
+"""Plants plausible mistakes in copies of the CPU oracle and checks that the pins catch
+each one (no GPU).  A mutant that passes every pin would mean a hole in the pins."""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import oracle_pins
+from oracle import build as oracle_build
+
+# (name, original text, mutated text): each original must occur exactly once.
+# Not listed: widening the activation clip to -128.  It is an equivalent mutant: with
+# s = max|x| (or the 1e-5 floor above it) |127 x / s| <= 127 always holds, so the clip
+# never binds.
+MUTANTS = [
+    ("tie_higher_index_wins", "(mag[j] == mag[i] && j < i)", "(mag[j] == mag[i] && j > i)"),
+    ("keeps_n_plus_one", "(uint8_t)(rank < N)", "(uint8_t)(rank <= N)"),
+    ("mask_not_applied", "ws_out[idx] = keep ? t : 0;", "ws_out[idx] = t;"),
+    ("mask_from_codes", "mag[i] = fabsf(bf16_bits_to_float(W[r * K + base + i]));",
+     "mag[i] = fabsf((float)ternary_code(bf16_bits_to_float(W[r * K + base + i]), g));"),
+    ("code_signs_swapped", "(v == 1 ? 1u : 3u)", "(v == 1 ? 3u : 1u)"),
+    ("code_bit_order", "(code << (2 * (e % 4)))", "(code << (2 * (3 - e % 4)))"),
+    ("meta_nibble_order", "(bits << (4 * (gi % 2)))", "(bits << (4 * (1 - gi % 2)))"),
+    ("gamma_wrong_count", "((double)n * 16777216.0)", "((double)(n + 1) * 16777216.0)"),
+    ("gamma_drops_eps", "float g = gamma + eps;", "float g = gamma;"),
+    ("round_half_away", "float r = rintf(q);", "float r = roundf(q);"),
+    ("act_qb_128", "rintf((127.0f * x) / s)", "rintf((128.0f * x) / s)"),
+    ("act_round_half_away", "rintf((127.0f * x) / s)", "roundf((127.0f * x) / s)"),
+    ("act_scale_floor_missing", "(a < 1e-5f) ? 1e-5f : a", "a"),
+    ("acc_transposed", "acc[t * O + o] = (int32_t)sum;", "acc[o * T + t] = (int32_t)sum;"),
+    ("rescale_qb_128", "(double)s[t] / 127.0", "(double)s[t] / 128.0"),
+    ("rescale_drops_g", "(double)acc[t * O + o] * (double)g * (double)s[t]",
+     "(double)acc[t * O + o] * (double)s[t]"),
+]
+
+
+@pytest.fixture(scope="module")
+def source():
+    with open(oracle_build.SRC) as f:
+        return f.read()
+
+
+@pytest.mark.parametrize("name,orig,mut", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, source, name, orig, mut):
+    assert source.count(orig) == 1, f"mutation site for {name} not unique/present"
+    src = tmp_path / f"{name}.c"
+    src.write_text(source.replace(orig, mut))
+    lib_path = str(tmp_path / f"lib{name}.so")
+    subprocess.check_call(["gcc", *oracle_build.CFLAGS, str(src), "-o", lib_path, "-lm"])
+    lib = oracle.load_library(lib_path)
+    oracle.use_library(lib)
+    failed = []
+    try:
+        for check in oracle_pins.ALL:
+            try:
+                check(oracle)
+            except (AssertionError, OverflowError, IndexError, ValueError):
+                failed.append(check.__name__)
+    finally:
+        oracle.use_library(None)
+    assert failed, f"mutant {name} passed every pin"
+    os.environ.setdefault("SBN_LAST_MUTANT_CAUGHT_BY", ",".join(failed))
