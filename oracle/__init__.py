@@ -82,10 +82,12 @@ def _bits(a):
 
 
 def plane_dims(K: int, n: int, m: int):
-    """Row strides (bytes) of the codes and meta planes: each row's data rounded up to
-    16 bytes.  codes: K*n/m kept elements x 2 bits; meta: K/m groups x m bits."""
-    codes_bytes = -(-(K // m * n * 2) // 8)
-    meta_bytes = -(-(K // m * m) // 8)
+    """Row strides (bytes) of the codes and meta planes, each row's data rounded up to 16
+    bytes.  codes: 2 bits per stored element (K/2 kept elements for 2:4, K positions
+    otherwise); meta: 4 bits per group for m == 4, 8 bits per group for m == 8."""
+    stored = K // 2 if (n, m) == (2, 4) else K
+    codes_bytes = -(-(stored * 2) // 8)
+    meta_bytes = -(-((K // m) * (4 if m == 4 else 8)) // 8)
     return (-(-codes_bytes // 16) * 16, -(-meta_bytes // 16) * 16)
 
 

@@ -153,43 +153,57 @@ void oracle_ternary_mask(const uint16_t *W, int64_t O, int64_t K, int N, int M, 
 }
 
 /*
- * S4 (pack): the hardware format of the masked ternary matrix.  The pages ask for
- * "well-defined N:M metadata on the discrete weights" [SBN-ar §2 quant-then-mask]; the
- * layout below is this library's reading of it:
- *   codes plane, row r: the kept positions of the row in ascending K order, 2 bits each
- *     (0 -> 00, +1 -> 01, -1 -> 11), kept element e at bits 2*(e%4) of byte e/4;
- *   meta plane, row r: one M-bit mask per group (bit i = position i of the group kept);
- *     M == 8: one byte per group; M == 4: group 2h in the low nibble of byte h, group
- *     2h+1 in the high nibble;
- *   rows are ldc / ldm bytes apart; every byte past a row's data is zero.
+ * S4 (pack): the hardware format of the masked ternary matrix.  The pages ask for "2-bit
+ * codes" with "well-defined N:M metadata on the discrete weights" [SBN-ar §2
+ * quant-then-mask]; the layout below is this library's reading of it.
+ *
+ * Which positions the codes plane stores:
+ *   pattern 2:4 (the pattern the sparse tensor cores consume): only the kept positions of
+ *     each row, in ascending K order (K/2 stored elements per row);
+ *   every other pattern: every position of the row in ascending K order, pruned positions
+ *     holding the code of 0 (K stored elements per row).
+ * Codes plane, row r: stored element e sits in the little-endian 32-bit word e/16 of the
+ *   row; inside that word, with j = (e%16)/4 and k = e%4, it occupies bits
+ *   [8k + 6 - 2j, 8k + 7 - 2j] (byte k, bit 6 - 2j).  A code is the 2-bit two's complement
+ *   of the ternary value: 0 -> 00, +1 -> 01, -1 -> 11 (10 is never written).
+ * Meta plane, row r, group g (M consecutive positions):
+ *   pattern 2:4: the two kept positions i0 < i1 of the group as the nibble i0 | i1 << 2;
+ *   other M == 4 patterns: the 4-bit keep mask (bit i = position i kept);
+ *   M == 8: the 8-bit keep mask, one byte per group;
+ *   nibbles: group 2h in the low nibble of byte h, group 2h+1 in the high nibble.
+ * Rows are ldc / ldm bytes apart; every byte past a row's data is zero.
  * Returns 0, or -1 if some group does not keep exactly N positions.
  */
 int oracle_pack(const int8_t *t, const uint8_t *keep, int64_t O, int64_t K, int N, int M,
                 uint8_t *codes, int64_t ldc, uint8_t *meta, int64_t ldm) {
   int bad = 0;
+  int compact = (N == 2 && M == 4);
   memset(codes, 0, (size_t)(O * ldc));
   memset(meta, 0, (size_t)(O * ldm));
 #pragma omp parallel for reduction(| : bad) schedule(static)
   for (int64_t r = 0; r < O; ++r) {
     int64_t e = 0;
     for (int64_t k = 0; k < K; ++k) {
-      if (!keep[r * K + k]) continue;
-      int8_t v = t[r * K + k];
+      int kept = keep[r * K + k];
+      if (compact && !kept) continue;
+      int8_t v = kept ? t[r * K + k] : 0;
       uint8_t code = (v == 0) ? 0u : (v == 1 ? 1u : 3u);
-      if (e / 4 >= ldc) { /* more kept positions than the plane holds */
+      int64_t byte = 4 * (e / 16) + e % 4;
+      int shift = 6 - 2 * (int)((e % 16) / 4);
+      if (byte >= ldc) { /* more stored elements than the plane holds */
         bad = 1;
         break;
       }
-      codes[r * ldc + e / 4] |= (uint8_t)(code << (2 * (e % 4)));
+      codes[r * ldc + byte] |= (uint8_t)(code << shift);
       ++e;
     }
-    if (e != K / M * N) bad = 1;
     for (int64_t gi = 0; gi < K / M; ++gi) {
-      unsigned bits = 0;
+      unsigned bits = 0, idx = 0;
       int kept = 0;
       for (int i = 0; i < M; ++i) {
         if (keep[r * K + gi * M + i]) {
           bits |= 1u << i;
+          if (kept < 2) idx |= (unsigned)i << (2 * kept);
           ++kept;
         }
       }
@@ -197,7 +211,7 @@ int oracle_pack(const int8_t *t, const uint8_t *keep, int64_t O, int64_t K, int 
       if (M == 8)
         meta[r * ldm + gi] = (uint8_t)bits;
       else
-        meta[r * ldm + gi / 2] |= (uint8_t)(bits << (4 * (gi % 2)));
+        meta[r * ldm + gi / 2] |= (uint8_t)((compact ? idx : bits) << (4 * (gi % 2)));
     }
   }
   return bad ? -1 : 0;

@@ -207,54 +207,80 @@ def contract_bruteforce(o):
 
 
 def unpack_planes(codes, meta, K, n, m):
-    """Independent decoder of the packed format, written from its description."""
+    """Independent decoder of the packed format, written from its description: returns
+    (ws, keep) with ws the masked ternary matrix and keep the mask."""
     O = codes.shape[0]
+    compact = (n, m) == (2, 4)
     ws = np.zeros((O, K), np.int8)
+    keep = np.zeros((O, K), np.uint8)
+
+    def code_at(r, e):
+        word = int.from_bytes(bytes(codes[r, 4 * (e // 16):4 * (e // 16) + 4]), "little")
+        c = (word >> (8 * (e % 4) + 6 - 2 * ((e % 16) // 4))) & 3
+        assert c != 2, "code 0b10 is never written"
+        return {0: 0, 1: 1, 3: -1}[c]
+
     for r in range(O):
-        e = 0
         for gi in range(K // m):
             if m == 8:
-                bits = int(meta[r, gi])
+                field = int(meta[r, gi])
             else:
-                bits = (int(meta[r, gi // 2]) >> (4 * (gi % 2))) & 0xF
-            for i in range(m):
-                if bits >> i & 1:
-                    c = (int(codes[r, e // 4]) >> (2 * (e % 4))) & 3
-                    assert c != 2, "code 0b10 is never written"
-                    ws[r, gi * m + i] = {0: 0, 1: 1, 3: -1}[c]
+                field = (int(meta[r, gi // 2]) >> (4 * (gi % 2))) & 0xF
+            if compact:
+                i0, i1 = field & 3, field >> 2
+                assert i0 < i1, "2:4 indices are stored in ascending order"
+                kept = [i0, i1]
+            else:
+                kept = [i for i in range(m) if field >> i & 1]
+            for i in kept:
+                keep[r, gi * m + i] = 1
+        e = 0
+        for k in range(K):
+            if compact:
+                if keep[r, k]:
+                    ws[r, k] = code_at(r, e)
                     e += 1
-    return ws
+            else:
+                v = code_at(r, k)
+                assert keep[r, k] or v == 0, "pruned positions hold the code of 0"
+                ws[r, k] = v
+    return ws, keep
 
 
 def unpack_roundtrip(o):
     for n, m, K in [(2, 4, 256), (6, 8, 192), (1, 8, 64), (3, 4, 64)]:
         W = workloads.masters(9, K, seed=K + n)
         r = o.quantize_mask_pack(W, n, m)
-        assert np.array_equal(unpack_planes(r["codes"], r["meta"], K, n, m), r["ws"])
+        ws, keep = unpack_planes(r["codes"], r["meta"], K, n, m)
+        assert np.array_equal(ws, r["ws"]) and np.array_equal(keep, r["keep"])
 
 
 def invariants(o):
-    for n, m in [(2, 4), (6, 8)]:
-        W = workloads.masters(64, 320, seed=n * m)
-        r = o.quantize_mask_pack(W, n, m)
+    for n, m in [(2, 4), (6, 8), (3, 4), (4, 8)]:
         K = 320
+        W = workloads.masters(64, K, seed=n * m)
+        r = o.quantize_mask_pack(W, n, m)
         assert set(np.unique(r["t"]).tolist()) <= {-1, 0, 1}
         keep = r["keep"].reshape(64, -1, m)
         assert (keep.sum(-1) == n).all()
         assert ((r["ws"] != 0).reshape(64, -1, m).sum(-1) <= n).all()
         assert np.array_equal(r["ws"], r["t"] * r["keep"])
-        used_c = K // m * n * 2 // 8
+        stored = K // 2 if (n, m) == (2, 4) else K
+        used_c = stored * 2 // 8
         used_m = K // 8
         assert (r["codes"][:, used_c:] == 0).all() and (r["meta"][:, used_m:] == 0).all()
         c = r["codes"][:, :used_c]
         for sh in (0, 2, 4, 6):
             assert ((c >> sh) & 3 != 2).all()
+        mm = r["meta"][:, :used_m]
         if m == 4:
-            nib = np.concatenate([r["meta"][:, :used_m] & 0xF, r["meta"][:, :used_m] >> 4])
+            nib = np.concatenate([mm & 0xF, mm >> 4])
+            if n == 2:
+                assert ((nib & 3) < (nib >> 2)).all()
+            else:
+                assert (np.unpackbits(nib[..., None], axis=-1).sum(-1) == n).all()
         else:
-            nib = r["meta"][:, :used_m]
-        pop = np.unpackbits(nib.astype(np.uint8)[..., None], axis=-1).sum(-1)
-        assert (pop == n).all()
+            assert (np.unpackbits(mm[..., None], axis=-1).sum(-1) == n).all()
 
 
 def scale_invariance(o):

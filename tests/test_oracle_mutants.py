@@ -20,8 +20,14 @@ MUTANTS = [
     ("mask_from_codes", "mag[i] = fabsf(bf16_bits_to_float(W[r * K + base + i]));",
      "mag[i] = fabsf((float)ternary_code(bf16_bits_to_float(W[r * K + base + i]), g));"),
     ("code_signs_swapped", "(v == 1 ? 1u : 3u)", "(v == 1 ? 3u : 1u)"),
-    ("code_bit_order", "(code << (2 * (e % 4)))", "(code << (2 * (3 - e % 4)))"),
-    ("meta_nibble_order", "(bits << (4 * (gi % 2)))", "(bits << (4 * (1 - gi % 2)))"),
+    ("code_bit_order", "int shift = 6 - 2 * (int)((e % 16) / 4);",
+     "int shift = 2 * (int)((e % 16) / 4);"),
+    ("code_byte_order", "int64_t byte = 4 * (e / 16) + e % 4;",
+     "int64_t byte = 4 * (e / 16) + 3 - e % 4;"),
+    ("pruned_not_zeroed_dense", "int8_t v = kept ? t[r * K + k] : 0;", "int8_t v = t[r * K + k];"),
+    ("meta_nibble_order", "<< (4 * (gi % 2)));", "<< (4 * (1 - gi % 2)));"),
+    ("index_order_swapped", "idx |= (unsigned)i << (2 * kept);",
+     "idx |= (unsigned)i << (2 - 2 * kept);"),
     ("gamma_wrong_count", "((double)n * 16777216.0)", "((double)(n + 1) * 16777216.0)"),
     ("gamma_drops_eps", "float g = gamma + eps;", "float g = gamma;"),
     ("round_half_away", "float r = rintf(q);", "float r = roundf(q);"),
