@@ -1,0 +1,431 @@
+"""Benchmark of the Sparse-BitLinear forward hot path on B200.
+
+One step = the whole forward for one synthetic batch: pack the bf16 master weights
+(absmean gamma, ternary codes, N:M mask, 2-bit pack), quantise the activations to int8,
+contract and rescale.  Default workload: decode GEMV, W [6912 x 2560] 6:8, one token.
+
+Timing: the K timed steps are captured in one CUDA graph (after W warm-up steps) and
+replayed between a barrier + synchronize on both sides; the device time is the max over
+ranks.  Inputs rotate over R sets whose total exceeds the 126 MB L2, so every step reads
+its weights from HBM.  CUDA events recorded inside the graph bracket every C-ABI call and
+give the per-call durations used for the roofline.  nvidia-smi clocks are sampled during
+the timed region.
+
+`--impl reference` times the CPU oracle (test infrastructure) on a bounded sample of the
+same workload instead.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "Sparse-BitLinear TOPS & packed-weight GB/s vs roofline; quant+mask GB/s"
+L2_BYTES = 126 * 1024 * 1024
+
+WORKLOADS = {
+    "decode": workloads.DECODE_GEMV,
+    "prefill": workloads.PREFILL_GEMM,
+    "tiny": workloads.TINY,
+}
+
+
+# ---- algorithmic bytes / ops (per step) --------------------------------------------------
+
+def packed_bytes(O, K, n, m):
+    """Bytes of the packed planes without row padding: codes + metadata."""
+    stored = K // 2 if (n, m) == (2, 4) else K
+    return O * (stored // 4), O * (K // 8)
+
+
+def step_accounting(cfg):
+    O, K, T, n, m = cfg["O"], cfg["K"], cfg["T"], cfg["n"], cfg["m"]
+    codes_b, meta_b = packed_bytes(O, K, n, m)
+    # the contraction reads the codes, and the metadata only for 2:4
+    linear_w = codes_b + (meta_b if (n, m) == (2, 4) else 0)
+    pack = 2 * O * K + codes_b + meta_b
+    act = 2 * T * K + T * K + 4 * T
+    linear = linear_w + T * K + 4 * T + 4 * T * O
+    return dict(pack=pack, act=act, linear=linear, linear_weight=linear_w,
+                ops=2 * T * O * K * n // m, total=pack + act + linear)
+
+
+# ---- helpers -----------------------------------------------------------------------------
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"],
+                    bf16_sustained=d.get("bf16_tflops_sustained"), source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---- the CUDA arm ------------------------------------------------------------------------
+
+def run_cuda(args, cfg):
+    import sparse_linear_layers_absmean_b200 as sbn
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    O, K, T, n, m = cfg["O"], cfg["K"], cfg["T"], cfg["n"], cfg["m"]
+    acct = step_accounting(cfg)
+    set_bytes = 2 * O * K + 2 * T * K
+    R = max(2, -(-2 * L2_BYTES // set_bytes)) if set_bytes < 2 * L2_BYTES else 1
+    R = min(R, 64)
+
+    # R rotating input sets generated on the host (seeded, same recipe as the tests);
+    # a rank draws its own sets (tensor id offset by the rank).
+    sets = []
+    for r in range(R):
+        Wb = workloads.masters(O, K, seed=0, config=1, tensor=2 * (r + R * rank))
+        Xb = workloads.activations(T, K, seed=0, config=1, tensor=2 * (r + R * rank) + 1)
+        W = workloads.torch_bf16(Wb, dev)
+        X = workloads.torch_bf16(Xb, dev)
+        d = sbn.sbn_linear_ref_dims(O, K, n, m)
+        sets.append(dict(
+            W=W, X=X,
+            codes=torch.empty((O, d.codes_ld), dtype=torch.uint8, device=dev),
+            meta=torch.empty((O, d.meta_ld), dtype=torch.uint8, device=dev),
+            g=torch.empty(1, dtype=torch.float32, device=dev),
+            Xq=torch.empty((T, K), dtype=torch.int8, device=dev),
+            s=torch.empty((T,), dtype=torch.float32, device=dev),
+            Y=torch.empty((T, O), dtype=torch.float32, device=dev)))
+    ws = sbn.new_workspace(O, K, n, m, dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step(st, ev=None):
+        if ev is not None:
+            ev[0].record()
+        sbn.sbn_quantize_mask_pack_weights(st["W"], n, m, 1e-5, st["codes"], st["meta"], st["g"],
+                                           ws, None, err)
+        if ev is not None:
+            ev[1].record()
+        sbn.sbn_quantize_acts(st["X"], st["Xq"], st["s"], err)
+        if ev is not None:
+            ev[2].record()
+        sbn.sbn_linear(st["Xq"], st["s"], st["codes"], st["meta"], st["g"], O, K, n, m, st["Y"],
+                       None, err)
+        if ev is not None:
+            ev[3].record()
+
+    kernels_per_step = 4  # abs-sum reduction, quant/mask/pack, act quant, contraction
+    stream = torch.cuda.Stream(device=dev)
+    # warm-up (also loads the module and sets kernel attributes outside capture)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(sets[i % R])
+    torch.cuda.synchronize()
+
+    # external events: recorded by the graph replay itself, readable afterwards
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+           for _ in range(args.steps)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(args.steps):
+            step(sets[i % R], evs[i])
+    wg = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(wg, stream=stream):
+        for i in range(max(args.warmup, 3)):
+            step(sets[i % R])
+    wg.replay()
+    torch.cuda.synchronize()
+
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            t0.record()
+            g.replay()
+            t1.record()
+        torch.cuda.synchronize()
+        # keep sampling briefly if the timed region was shorter than the sampling period
+        if t0.elapsed_time(t1) < 300:
+            with torch.cuda.stream(stream):
+                for _ in range(max(1, int(300 / max(t0.elapsed_time(t1), 1e-3)))):
+                    g.replay()
+            torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(t0.elapsed_time(t1), world)
+    flag = int(err.item())
+
+    per = {"pack": [], "act": [], "linear": []}
+    for e in evs:
+        per["pack"].append(e[0].elapsed_time(e[1]))
+        per["act"].append(e[1].elapsed_time(e[2]))
+        per["linear"].append(e[2].elapsed_time(e[3]))
+    avg = {k: sum(v) / len(v) for k, v in per.items()}
+
+    # e2e through the public API with host buffers (pinned), copies in the timed region
+    e2e = None
+    if True:
+        hostW = [sets[r]["W"].cpu().pin_memory() for r in range(R)]
+        hostX = [sets[r]["X"].cpu().pin_memory() for r in range(R)]
+        hostY = torch.empty((T, O), dtype=torch.float32).pin_memory()
+        Wd = torch.empty_like(sets[0]["W"])
+        Xd = torch.empty_like(sets[0]["X"])
+        ke = min(args.steps, 20)
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                Wd.copy_(hostW[i % R], non_blocking=True)
+                Xd.copy_(hostX[i % R], non_blocking=True)
+                Y = sbn.forward(Xd, Wd, n, m, workspace=ws)
+                hostY.copy_(Y, non_blocking=True)
+            torch.cuda.synchronize()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            for i in range(ke):
+                Wd.copy_(hostW[i % R], non_blocking=True)
+                Xd.copy_(hostX[i % R], non_blocking=True)
+                Y = sbn.forward(Xd, Wd, n, m, workspace=ws)
+                hostY.copy_(Y, non_blocking=True)
+                torch.cuda.current_stream().synchronize()  # the step's result is on the host
+            b.record()
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / ke, world)
+        e2e = {"value": acct["total"] * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": 2 * O * K + 2 * T * K, "d2h_bytes_per_step": 4 * T * O,
+               "ms_per_step": e2e_ms}
+
+    peaks = load_peaks()
+    total_s = ms * 1e-3
+    value = acct["total"] * args.steps * world / total_s / 1e9
+    # dominant C-ABI call by time share
+    dom = max(avg, key=avg.get)
+    dom_bytes = {"pack": acct["pack"], "act": acct["act"], "linear": acct["linear"]}[dom]
+    achieved = dom_bytes / (avg[dom] * 1e-3) / 1e9
+    traffic = load_traffic(cfg["name"], dom)
+    result = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8xternary->int32, fp32 out",
+        "data": "synthetic (seeded N(0,0.02) bf16 masters; N(0,1) activations, 0.5% x20 outliers)",
+        "config": {"workload": cfg["name"], "O": O, "K": K, "tokens": T, "pattern": f"{n}:{m}",
+                   "step": "pack(S1-S4) + act quant(S5) + contract/rescale(S6-S7)",
+                   "l2": f"{R} rotating input sets ({R * set_bytes / 1e6:.0f} MB > 126 MB L2)",
+                   "parallelism": f"replicas x{world} (independent problems)"},
+        "kernels": {
+            "pack": {"ms": avg["pack"], "GB/s": acct["pack"] / (avg["pack"] * 1e-3) / 1e9,
+                     "launches": 2},
+            "act_quant": {"ms": avg["act"], "GB/s": acct["act"] / (avg["act"] * 1e-3) / 1e9},
+            "linear": {"ms": avg["linear"],
+                       "packed_weight_GB/s": acct["linear_weight"] / (avg["linear"] * 1e-3) / 1e9,
+                       "TOPS": acct["ops"] / (avg["linear"] * 1e-3) / 1e12},
+        },
+        "roofline": {"bound": "hbm", "kernel": {"pack": "quant_mask_pack (abs-sum + pack)",
+                                                "act": "act_quant", "linear": "contraction"}[dom],
+                     "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm"], "traffic": traffic,
+                     "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, burst)"},
+        "gpu_launches": kernels_per_step * args.steps,
+        "err_flag": flag,
+        "e2e": e2e,
+    }
+    if rank == 0:
+        result["clocks"] = clk.summary()
+        if world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_seconds)
+        print(json.dumps(result))
+    if world > 1:
+        del g, wg
+        torch.distributed.destroy_process_group()
+
+
+def load_traffic(workload, dom):
+    """DRAM bytes per launch of the dominant call from the committed ncu summary, if any."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    return d.get(workload, {}).get(dom)
+
+
+# ---- the oracle (CPU baseline / reference arm) -------------------------------------------
+
+def oracle_step(cfg, Wb, Xb):
+    import oracle
+    w = oracle.quantize_mask_pack(Wb, cfg["n"], cfg["m"], 1e-5)
+    Xq, s, _ = oracle.quant_acts(Xb)
+    acc = oracle.contract(Xq, w["ws"])
+    return oracle.rescale(acc, s, w["g"])
+
+
+def cpu_baseline(cfg, budget_s=10.0, steps=None):
+    """Times the oracle as it stands on this host's cores on whole steps of the workload
+    (bounded: stops after `budget_s` seconds or `steps` steps)."""
+    import oracle
+    acct = step_accounting(cfg)
+    Wb = workloads.masters(cfg["O"], cfg["K"], seed=0, config=1, tensor=0)
+    Xb = workloads.activations(cfg["T"], cfg["K"], seed=0, config=1, tensor=1)
+    oracle_step(cfg, Wb, Xb)  # load / build outside the timing
+    done, t0 = 0, time.perf_counter()
+    while True:
+        oracle_step(cfg, Wb, Xb)
+        done += 1
+        el = time.perf_counter() - t0
+        if (steps is not None and done >= steps) or (steps is None and el >= budget_s):
+            break
+    return {"value": acct["total"] * done / el / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{done} whole steps of {cfg['name']} ({el:.1f} s)",
+            "ms_per_step": el / done * 1e3}
+
+
+def run_reference(args, cfg):
+    """The oracle as the reference arm: W warm-up steps, then K timed steps on the host cores.
+    Each step is the whole forward on a bounded sample of the workload (a slice of output
+    rows, all tokens) sized so that the whole run stays within about two minutes."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    O = cfg["O"]
+    Wb = workloads.masters(O, cfg["K"], seed=0, config=1, tensor=0)
+    Xb = workloads.activations(cfg["T"], cfg["K"], seed=0, config=1, tensor=1)
+    t0 = time.perf_counter()
+    oracle_step(cfg, Wb, Xb)
+    full = time.perf_counter() - t0
+    frac = min(1.0, 100.0 / max(full * (args.steps + args.warmup), 1e-9))
+    rows = max(8, int(O * frac) // 8 * 8)
+    sub = dict(cfg, O=rows)
+    Ws = np.ascontiguousarray(Wb[:rows])
+    for _ in range(args.warmup):
+        oracle_step(sub, Ws, Xb)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(sub, Ws, Xb)
+    el = time.perf_counter() - t0
+    value = step_accounting(sub)["total"] * args.steps / el / 1e9
+    sample = f"{args.steps} steps, each {rows} of {O} output rows x all tokens of {cfg['name']}"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8xternary->int64, fp64 out", "data": "synthetic",
+        "config": {"workload": cfg["name"], "O": O, "K": cfg["K"], "tokens": cfg["T"],
+                   "pattern": f"{cfg['n']}:{cfg['m']}"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    cfg = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_cuda(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,161 @@
+/*
+ * sbn.h -- C ABI of the Sparse-BitLinear forward on NVIDIA B200 (sm_100a).
+ *
+ * The operation (Sparse-BitNet, "1.58-bit LLMs are Naturally Friendly to Semi-Structured
+ * Sparsity", technical summaries on gist.science, section 2 "Methodology":
+ * Sparse-BitLinear layer):
+ *   1. gamma = mean |W| over the bf16 master weights of one tensor; g = gamma + eps;
+ *   2. ternary codes t = clip(round(W / g), -1, 1)       (absmean quantisation);
+ *   3. N:M mask = in every group of M consecutive inputs of a row, the N largest master
+ *      magnitudes (ties: lower index), applied AFTER quantisation (quant-then-mask);
+ *   4. the masked codes are packed as 2-bit codes plus per-group metadata;
+ *   5. activations are quantised per token to int8 by absmax with Qb = 127
+ *      ("Marco de inferencia de Microsoft lleva modelos de lenguaje grande de 1 bit a
+ *      dispositivos locales", unite.ai, "Fundamento matemático", item 2);
+ *   6. acc = Xq . Ws^T in exact int32; y = acc * g * s / 127 (same article, item 3:
+ *      the BitLinear output is rescaled by the weight and activation scales over Qb).
+ * Rounding of round() is half-to-even; W/g and 127*x/s are IEEE fp32 divisions.
+ *
+ * Conventions for every call below:
+ *   - All tensor arguments are DEVICE pointers owned by the caller; the library keeps no
+ *     state and allocates no memory.  Layouts are row-major and dense.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only enqueues
+ *     work on it and returns without synchronising.
+ *   - Argument errors are detected on the host, before anything is launched, and
+ *     returned as an sbn_status; nothing is written in that case.
+ *   - Data errors (NaN/Inf or |W| >= 256 in the inputs) are found by the kernels, which
+ *     OR the SBN_FLAG_* bits into *err_flag (an int32 in device memory that the caller
+ *     zeroes; err_flag may be NULL to not report them).  Outputs are unspecified when a
+ *     flag is raised.
+ *   - Supported patterns: m in {4, 8}, 1 <= n <= m (n == m is the unmasked b1.58 layer).
+ *     `in` (K) must be a positive multiple of 64; `out` (O) positive; tokens >= 0.
+ *   - Device pointers must be 16-byte aligned.
+ */
+#ifndef SBN_H_
+#define SBN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SBN_API __attribute__((visibility("default")))
+#else
+#define SBN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sbn_status {
+  SBN_OK = 0,
+  SBN_ERR_NULL = 1,    /* a required pointer is NULL */
+  SBN_ERR_SHAPE = 2,   /* out <= 0, in <= 0, in % 64 != 0, tokens < 0, or too large */
+  SBN_ERR_PATTERN = 3, /* m not in {4, 8} or n not in [1, m] */
+  SBN_ERR_ALIGN = 4,   /* a device pointer is not 16-byte aligned */
+  SBN_ERR_CUDA = 5,    /* a CUDA runtime call or a launch failed */
+  SBN_ERR_ARG = 6      /* eps negative or not finite */
+} sbn_status;
+
+/* Data-error bits OR-ed into *err_flag by the kernels. */
+#define SBN_FLAG_W_NONFINITE 1 /* a master weight is NaN or Inf */
+#define SBN_FLAG_W_RANGE 2     /* a master weight has |W| >= 256 */
+#define SBN_FLAG_X_NONFINITE 4 /* an activation is NaN or Inf */
+#define SBN_FLAG_TIMEOUT 8     /* a tensor-core pipeline wait gave up (~1 s); Y unspecified */
+
+/*
+ * Packed weight format (sizes from sbn_linear_ref_dims).  Row r of each plane starts at
+ * byte r * ld; bytes past a row's data up to ld are written as zero.
+ *   codes plane: 2-bit codes (0 -> 00, +1 -> 01, -1 -> 11) of the row's stored elements:
+ *     pattern 2:4 stores the kept positions only (K/2 per row, ascending K); every other
+ *     pattern stores all K positions, pruned ones as 0.  Stored element e lives in the
+ *     little-endian 32-bit word e/16 of the row, at bits [8k + 6 - 2j, 8k + 7 - 2j] with
+ *     j = (e % 16) / 4 and k = e % 4, so (word << 2j) & 0xC0C0C0C0 holds 64 * code of
+ *     elements 4j..4j+3 as four int8 lanes.
+ *   meta plane: per group g of M inputs: 2:4 -> nibble i0 | i1 << 2 (the two kept
+ *     positions, i0 < i1); other M == 4 -> 4-bit keep mask; M == 8 -> 8-bit keep mask
+ *     (one byte per group).  Group 2h is the low nibble of byte h, 2h+1 the high one.
+ */
+typedef struct sbn_dims {
+  int64_t codes_ld;             /* bytes between rows of the codes plane (multiple of 16) */
+  int64_t meta_ld;              /* bytes between rows of the meta plane (multiple of 16) */
+  int64_t codes_row_bytes;      /* data bytes per codes row (the rest is zero padding) */
+  int64_t meta_row_bytes;       /* data bytes per meta row */
+  int64_t codes_bytes;          /* out * codes_ld: size of the codes buffer */
+  int64_t meta_bytes;           /* out * meta_ld: size of the meta buffer */
+  int64_t pack_workspace_bytes; /* device workspace sbn_quantize_mask_pack_weights needs */
+} sbn_dims;
+
+/*
+ * Host only, no CUDA call: validates (out, in, n, m) and fills *d with the plane sizes
+ * and the workspace size.  Returns SBN_ERR_NULL / SHAPE / PATTERN on bad arguments.
+ */
+SBN_API sbn_status sbn_linear_ref_dims(int64_t out, int64_t in, int n, int m, sbn_dims *d);
+
+/*
+ * Steps 1-4 for one master tensor (Sparse-BitNet section 2: absmean ternary
+ * quantisation, mask from the master magnitudes, quant-then-mask, packing).
+ *   W          bf16 [out, in] master weights (bits of __nv_bfloat16), read only.
+ *   eps        added to gamma in fp32 (finite, >= 0; 1e-5 is the usual value).
+ *   codes      uint8 [dims.codes_bytes], written (including the zero padding).
+ *   meta       uint8 [dims.meta_bytes], written.
+ *   gamma_eff  one fp32: g = fp32(gamma + eps), where
+ *              gamma = fp32( fp64(S) / (fp64(out * in) * 2^24) ),
+ *              S = sum over all weights of trunc(|W| * 2^24)  (exact 64-bit integer sum,
+ *              so the result does not depend on the order of summation).
+ *   workspace  dims.pack_workspace_bytes of device memory, zero-filled before its first
+ *              use.  It holds per-CTA partial sums and an arrival counter; every call
+ *              returns the counter to zero, so the same workspace can be reused by later
+ *              calls without clearing it again.  Calls that share one workspace must not
+ *              run concurrently.
+ *   dense_dbg  optional int8 [out, in]: the masked ternary matrix (NULL to skip).
+ *   err_flag   optional: SBN_FLAG_W_NONFINITE / SBN_FLAG_W_RANGE.
+ * out * in must be below 2^31.
+ */
+SBN_API sbn_status sbn_quantize_mask_pack_weights(const void *W, int64_t out, int64_t in, int n,
+                                          int m, float eps, uint8_t *codes, uint8_t *meta,
+                                          float *gamma_eff, void *workspace,
+                                          int8_t *dense_dbg, int32_t *err_flag,
+                                          void *stream);
+
+/*
+ * Step 5: per-token absmax int8 activations (bitnet.cpp article, "Fundamento
+ * matemático", item 2, with Qb = 127):
+ *   s[t] = max(max_k |X[t,k]|, 1e-5);  Xq[t,k] = clamp(rint((127 * X[t,k]) / s[t]), +-127).
+ *   X       bf16 [tokens, in], read only.
+ *   Xq      int8 [tokens, in], written.
+ *   absmax  fp32 [tokens], written (s, after the 1e-5 floor).
+ *   err_flag optional: SBN_FLAG_X_NONFINITE.
+ * tokens == 0 is a no-op that returns SBN_OK before any pointer is checked (empty
+ * tensors may have NULL data pointers).
+ */
+SBN_API sbn_status sbn_quantize_acts(const void *X, int64_t tokens, int64_t in, int8_t *Xq,
+                             float *absmax, int32_t *err_flag, void *stream);
+
+/*
+ * Step 6: y[t, o] = (sum_k Xq[t,k] * Ws[o,k]) * c_t,  c_t = fp32(fp32(g * s[t]) / 127),
+ * where Ws is the masked ternary matrix held by (codes, meta) and g = *gamma_eff.  The
+ * sum is exact (int32).  The product acc * c_t is one fp32 multiply (no FMA); with
+ * y_is_bf16 it is then rounded to bf16 (nearest-even).
+ *   Xq, absmax       from sbn_quantize_acts (int8 [tokens, in], fp32 [tokens]).
+ *   codes, meta      from sbn_quantize_mask_pack_weights for the same (out, in, n, m).
+ *   gamma_eff        one fp32 on the device.
+ *   Y                fp32 or bf16 [tokens, out], written.
+ *   acc_dbg          optional int32 [tokens, out]: the exact integer sums (NULL to skip).
+ *   err_flag         optional: SBN_FLAG_TIMEOUT if the tensor-core pipeline stalled.
+ * tokens == 0 is a no-op that returns SBN_OK once the shapes and pattern are valid, before
+ * any pointer is checked.
+ */
+SBN_API sbn_status sbn_linear(const int8_t *Xq, const float *absmax, const uint8_t *codes,
+                      const uint8_t *meta, const float *gamma_eff, int64_t tokens,
+                      int64_t out, int64_t in, int n, int m, void *Y, int y_is_bf16,
+                      int32_t *acc_dbg, int32_t *err_flag, void *stream);
+
+/* A static, human-readable name for a status code. */
+SBN_API const char *sbn_status_string(sbn_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SBN_H_ */

@@ -1,0 +1,182 @@
+"""Sparse-BitLinear forward on B200 (sm_100a): thin Python binding of libsbn.so.
+
+The C ABI (include/sbn.h) does all the work in CUDA kernels; this module only marshals
+arguments.  PyTorch provides device memory and streams.  The functions named like the
+C entry points take torch tensors and forward their data pointers; the helpers at the end
+(`pack_weights`, `quantize_acts`, `linear`, `forward`) allocate the output tensors with
+torch and call them.
+
+There is no CPU fallback: if libsbn.so cannot be loaded, or a tensor is not on a CUDA
+device, the call raises.
+"""
+import ctypes
+import os
+from typing import NamedTuple, Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsbn.so")
+
+SBN_OK = 0
+STATUS = {0: "SBN_OK", 1: "SBN_ERR_NULL", 2: "SBN_ERR_SHAPE", 3: "SBN_ERR_PATTERN",
+          4: "SBN_ERR_ALIGN", 5: "SBN_ERR_CUDA", 6: "SBN_ERR_ARG"}
+FLAG_W_NONFINITE = 1
+FLAG_W_RANGE = 2
+FLAG_X_NONFINITE = 4
+FLAG_TIMEOUT = 8
+
+EXPORTED = ("sbn_linear_ref_dims", "sbn_quantize_mask_pack_weights", "sbn_quantize_acts",
+            "sbn_linear", "sbn_status_string")
+
+
+class SbnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class SbnDims(ctypes.Structure):
+    _fields_ = [("codes_ld", ctypes.c_int64), ("meta_ld", ctypes.c_int64),
+                ("codes_row_bytes", ctypes.c_int64), ("meta_row_bytes", ctypes.c_int64),
+                ("codes_bytes", ctypes.c_int64), ("meta_bytes", ctypes.c_int64),
+                ("pack_workspace_bytes", ctypes.c_int64)]
+
+
+_LIB = None
+
+
+def lib():
+    """Load libsbn.so (built in-tree by ``build.py``); raises if it is missing."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built; run sparse_linear_layers_absmean_b200/"
+                               "build.py (or __graft_entry__.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        L.sbn_linear_ref_dims.argtypes = [i64, i64, i32, i32, ctypes.POINTER(SbnDims)]
+        L.sbn_linear_ref_dims.restype = i32
+        L.sbn_quantize_mask_pack_weights.argtypes = [p, i64, i64, i32, i32, ctypes.c_float, p, p,
+                                                     p, p, p, p, p]
+        L.sbn_quantize_mask_pack_weights.restype = i32
+        L.sbn_quantize_acts.argtypes = [p, i64, i64, p, p, p, p]
+        L.sbn_quantize_acts.restype = i32
+        L.sbn_linear.argtypes = [p, p, p, p, p, i64, i64, i64, i32, i32, p, i32, p, p, p]
+        L.sbn_linear.restype = i32
+        L.sbn_status_string.argtypes = [i32]
+        L.sbn_status_string.restype = ctypes.c_char_p
+        _LIB = L
+    return _LIB
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("sbn kernels take CUDA tensors only (no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError("sbn kernels take contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(status: int, what: str):
+    if status != SBN_OK:
+        raise SbnError(status, what)
+
+
+# ---- the C entry points ------------------------------------------------------------------
+
+def sbn_linear_ref_dims(out: int, in_: int, n: int, m: int) -> SbnDims:
+    d = SbnDims()
+    _check(lib().sbn_linear_ref_dims(out, in_, n, m, ctypes.byref(d)), "sbn_linear_ref_dims")
+    return d
+
+
+def sbn_quantize_mask_pack_weights(W, n, m, eps, codes, meta, gamma_eff, workspace,
+                                   dense_dbg=None, err_flag=None, stream=None):
+    out, in_ = W.shape
+    _check(lib().sbn_quantize_mask_pack_weights(
+        _ptr(W), out, in_, n, m, ctypes.c_float(eps), _ptr(codes), _ptr(meta), _ptr(gamma_eff),
+        _ptr(workspace), _ptr(dense_dbg), _ptr(err_flag), _stream(stream)),
+        "sbn_quantize_mask_pack_weights")
+
+
+def sbn_quantize_acts(X, Xq, absmax, err_flag=None, stream=None):
+    tokens, in_ = X.shape
+    _check(lib().sbn_quantize_acts(_ptr(X), tokens, in_, _ptr(Xq), _ptr(absmax), _ptr(err_flag),
+                                   _stream(stream)), "sbn_quantize_acts")
+
+
+def sbn_linear(Xq, absmax, codes, meta, gamma_eff, out, in_, n, m, Y, acc_dbg=None,
+               err_flag=None, stream=None):
+    tokens = Xq.shape[0]
+    y_is_bf16 = 1 if Y.dtype == torch.bfloat16 else 0
+    if Y.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("Y must be float32 or bfloat16")
+    _check(lib().sbn_linear(_ptr(Xq), _ptr(absmax), _ptr(codes), _ptr(meta), _ptr(gamma_eff),
+                            tokens, out, in_, n, m, _ptr(Y), y_is_bf16, _ptr(acc_dbg),
+                            _ptr(err_flag), _stream(stream)), "sbn_linear")
+
+
+# ---- allocation helpers --------------------------------------------------------------------
+
+class PackedWeights(NamedTuple):
+    codes: torch.Tensor      # uint8 [out, codes_ld]
+    meta: torch.Tensor       # uint8 [out, meta_ld]
+    gamma_eff: torch.Tensor  # fp32 [1]
+    out: int
+    in_: int
+    n: int
+    m: int
+
+
+def new_workspace(out: int, in_: int, n: int, m: int, device="cuda") -> torch.Tensor:
+    """Zero-filled pack workspace (reusable by later calls on the same stream)."""
+    d = sbn_linear_ref_dims(out, in_, n, m)
+    return torch.zeros(d.pack_workspace_bytes, dtype=torch.uint8, device=device)
+
+
+def pack_weights(W: torch.Tensor, n: int, m: int, eps: float = 1e-5,
+                 workspace: Optional[torch.Tensor] = None, dense_dbg: Optional[torch.Tensor] = None,
+                 err_flag: Optional[torch.Tensor] = None, stream=None) -> PackedWeights:
+    out, in_ = W.shape
+    d = sbn_linear_ref_dims(out, in_, n, m)
+    codes = torch.empty((out, d.codes_ld), dtype=torch.uint8, device=W.device)
+    meta = torch.empty((out, d.meta_ld), dtype=torch.uint8, device=W.device)
+    gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    if workspace is None:
+        workspace = new_workspace(out, in_, n, m, W.device)
+    sbn_quantize_mask_pack_weights(W, n, m, eps, codes, meta, gamma, workspace, dense_dbg,
+                                   err_flag, stream)
+    return PackedWeights(codes, meta, gamma, out, in_, n, m)
+
+
+def quantize_acts(X: torch.Tensor, err_flag=None, stream=None):
+    tokens, in_ = X.shape
+    Xq = torch.empty((tokens, in_), dtype=torch.int8, device=X.device)
+    s = torch.empty((tokens,), dtype=torch.float32, device=X.device)
+    sbn_quantize_acts(X, Xq, s, err_flag, stream)
+    return Xq, s
+
+
+def linear(Xq: torch.Tensor, s: torch.Tensor, w: PackedWeights, out_dtype=torch.float32,
+           acc_dbg=None, err_flag=None, stream=None) -> torch.Tensor:
+    Y = torch.empty((Xq.shape[0], w.out), dtype=out_dtype, device=Xq.device)
+    sbn_linear(Xq, s, w.codes, w.meta, w.gamma_eff, w.out, w.in_, w.n, w.m, Y, acc_dbg, err_flag,
+               stream)
+    return Y
+
+
+def forward(X: torch.Tensor, W: torch.Tensor, n: int, m: int, eps: float = 1e-5,
+            out_dtype=torch.float32, workspace=None, stream=None) -> torch.Tensor:
+    """The whole Sparse-BitLinear forward: pack W, quantise X, contract and rescale."""
+    w = pack_weights(W, n, m, eps, workspace=workspace, stream=stream)
+    Xq, s = quantize_acts(X, stream=stream)
+    return linear(Xq, s, w, out_dtype, stream=stream)

@@ -1,0 +1,103 @@
+// Per-token absmax int8 activation quantisation ("Marco de inferencia de Microsoft lleva
+// modelos de lenguaje grande de 1 bit a dispositivos locales", unite.ai, "Fundamento
+// matemático" item 2; Qb = 127):
+//   s = max(max_k |x_k|, 1e-5),  q_k = clamp(rint((127 * x_k) / s), -127, 127).
+// One CTA per token.  Rows of up to 16384 inputs stay in registers between the max pass
+// and the quantise pass (one HBM read); longer rows are read twice.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace sbn {
+
+constexpr int kAqThreads = 256;
+
+__device__ __forceinline__ uint32_t quant_pair(uint32_t w, float s) {
+  // two bf16 values -> two int8 codes in the low 16 bits
+  float xl = bf16_lo_to_float(w), xh = bf16_hi_to_float(w);
+  int ql = __float2int_rn(__fdiv_rn(__fmul_rn(127.0f, xl), s));
+  int qh = __float2int_rn(__fdiv_rn(__fmul_rn(127.0f, xh), s));
+  ql = min(127, max(-127, ql));
+  qh = min(127, max(-127, qh));
+  return ((uint32_t)ql & 0xffu) | (((uint32_t)qh & 0xffu) << 8);
+}
+
+__device__ __forceinline__ uint2 quant_vec8(uint4 v, float s) {
+  uint32_t a = quant_pair(v.x, s) | (quant_pair(v.y, s) << 16);
+  uint32_t b = quant_pair(v.z, s) | (quant_pair(v.w, s) << 16);
+  return make_uint2(a, b);
+}
+
+__device__ __forceinline__ uint32_t vec8_absmax_bits(uint4 v, uint32_t mx) {
+  mx = __vmaxu2(mx, v.x & 0x7fff7fffu);
+  mx = __vmaxu2(mx, v.y & 0x7fff7fffu);
+  mx = __vmaxu2(mx, v.z & 0x7fff7fffu);
+  mx = __vmaxu2(mx, v.w & 0x7fff7fffu);
+  return mx;
+}
+
+// Block-wide max of the per-thread packed magnitudes; returns the token's scale s.
+__device__ __forceinline__ float block_scale(uint32_t mx, int32_t *err_flag) {
+  __shared__ uint32_t s_mx[kAqThreads / 32];
+  uint32_t m = warp_max_u32(max(mx & 0xffffu, mx >> 16));
+  if ((threadIdx.x & 31) == 0) s_mx[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = 0;
+#pragma unroll
+  for (int w = 0; w < kAqThreads / 32; ++w) m = max(m, s_mx[w]);
+  if (m >= kBf16InfBits && threadIdx.x == 0 && err_flag) atomicOr(err_flag, SBN_FLAG_X_NONFINITE);
+  return fmaxf(__uint_as_float(m << 16), 1e-5f);
+}
+
+template <int R>
+__global__ void __launch_bounds__(kAqThreads)
+    k_act_quant_reg(const uint4 *__restrict__ X, int64_t nv, int8_t *__restrict__ Xq,
+                    float *__restrict__ absmax, int32_t *err_flag) {
+  const int64_t t = blockIdx.x;
+  const uint4 *row = X + t * nv;
+  uint4 v[R];
+  uint32_t mx = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    int64_t i = threadIdx.x + (int64_t)r * kAqThreads;
+    v[r] = i < nv ? __ldg(row + i) : make_uint4(0u, 0u, 0u, 0u);
+    mx = vec8_absmax_bits(v[r], mx);
+  }
+  const float s = block_scale(mx, err_flag);
+  if (threadIdx.x == 0) absmax[t] = s;
+  uint2 *qrow = reinterpret_cast<uint2 *>(Xq + t * nv * 8);
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    int64_t i = threadIdx.x + (int64_t)r * kAqThreads;
+    if (i < nv) qrow[i] = quant_vec8(v[r], s);
+  }
+}
+
+__global__ void __launch_bounds__(kAqThreads)
+    k_act_quant_loop(const uint4 *__restrict__ X, int64_t nv, int8_t *__restrict__ Xq,
+                     float *__restrict__ absmax, int32_t *err_flag) {
+  const int64_t t = blockIdx.x;
+  const uint4 *row = X + t * nv;
+  uint32_t mx = 0;
+  for (int64_t i = threadIdx.x; i < nv; i += kAqThreads) mx = vec8_absmax_bits(__ldg(row + i), mx);
+  const float s = block_scale(mx, err_flag);
+  if (threadIdx.x == 0) absmax[t] = s;
+  uint2 *qrow = reinterpret_cast<uint2 *>(Xq + t * nv * 8);
+  for (int64_t i = threadIdx.x; i < nv; i += kAqThreads) qrow[i] = quant_vec8(__ldg(row + i), s);
+}
+
+sbn_status launch_act_quant(const void *X, int64_t tokens, int64_t in, int8_t *Xq,
+                            float *absmax, int32_t *err_flag, cudaStream_t st) {
+  const int64_t nv = in / 8;
+  const uint4 *X4 = reinterpret_cast<const uint4 *>(X);
+  const unsigned grid = (unsigned)tokens;
+  if (nv <= 2 * kAqThreads)
+    k_act_quant_reg<2><<<grid, kAqThreads, 0, st>>>(X4, nv, Xq, absmax, err_flag);
+  else if (nv <= 8 * kAqThreads)
+    k_act_quant_reg<8><<<grid, kAqThreads, 0, st>>>(X4, nv, Xq, absmax, err_flag);
+  else
+    k_act_quant_loop<<<grid, kAqThreads, 0, st>>>(X4, nv, Xq, absmax, err_flag);
+  SBN_LAUNCH_CHECK();
+  return SBN_OK;
+}
+
+}  // namespace sbn

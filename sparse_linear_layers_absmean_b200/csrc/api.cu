@@ -1,0 +1,121 @@
+// The C ABI of sbn.h: host-side validation, buffer geometry and dispatch to the kernels.
+// Nothing here allocates device memory or synchronises.
+#include <cmath>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace {
+
+constexpr int64_t kMaxIn = 131072;           // keeps 64 * 127 * in below 2^31
+constexpr int64_t kMaxElems = (1ll << 31) - 1;  // out * in (one tensor)
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+sbn_status check_pattern(int n, int m) {
+  if (m != 4 && m != 8) return SBN_ERR_PATTERN;
+  if (n < 1 || n > m) return SBN_ERR_PATTERN;
+  return SBN_OK;
+}
+
+sbn_status check_in(int64_t in) {
+  if (in <= 0 || in % 64 != 0 || in > kMaxIn) return SBN_ERR_SHAPE;
+  return SBN_OK;
+}
+
+void fill_dims(int64_t out, int64_t in, int n, int m, sbn_dims *d) {
+  const bool compact = (n == 2 && m == 4);
+  const int64_t stored = compact ? in / 2 : in;
+  d->codes_row_bytes = stored / 4;
+  d->meta_row_bytes = in / 8;
+  d->codes_ld = (d->codes_row_bytes + 15) / 16 * 16;
+  d->meta_ld = (d->meta_row_bytes + 15) / 16 * 16;
+  d->codes_bytes = out * d->codes_ld;
+  d->meta_bytes = out * d->meta_ld;
+  d->pack_workspace_bytes = (int64_t)((sizeof(sbn::PackWorkspace) + 255) / 256 * 256);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *sbn_status_string(sbn_status s) {
+  switch (s) {
+    case SBN_OK: return "ok";
+    case SBN_ERR_NULL: return "null pointer";
+    case SBN_ERR_SHAPE: return "bad shape";
+    case SBN_ERR_PATTERN: return "unsupported N:M pattern";
+    case SBN_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case SBN_ERR_CUDA: return "CUDA error";
+    case SBN_ERR_ARG: return "bad argument";
+  }
+  return "unknown status";
+}
+
+sbn_status sbn_linear_ref_dims(int64_t out, int64_t in, int n, int m, sbn_dims *d) {
+  if (!d) return SBN_ERR_NULL;
+  sbn_status st = check_pattern(n, m);
+  if (st != SBN_OK) return st;
+  if ((st = check_in(in)) != SBN_OK) return st;
+  if (out <= 0 || out > kMaxElems / in) return SBN_ERR_SHAPE;
+  fill_dims(out, in, n, m, d);
+  return SBN_OK;
+}
+
+sbn_status sbn_quantize_mask_pack_weights(const void *W, int64_t out, int64_t in, int n, int m,
+                                          float eps, uint8_t *codes, uint8_t *meta,
+                                          float *gamma_eff, void *workspace, int8_t *dense_dbg,
+                                          int32_t *err_flag, void *stream) {
+  sbn_dims d;
+  sbn_status st = sbn_linear_ref_dims(out, in, n, m, &d);
+  if (st != SBN_OK) return st;
+  if (!W || !codes || !meta || !gamma_eff || !workspace) return SBN_ERR_NULL;
+  if (!std::isfinite(eps) || eps < 0.0f) return SBN_ERR_ARG;
+  if (!aligned16(W) || !aligned16(codes) || !aligned16(meta) || !aligned16(workspace) ||
+      (dense_dbg && !aligned16(dense_dbg)))
+    return SBN_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(gamma_eff) & 3u) || (reinterpret_cast<uintptr_t>(err_flag) & 3u))
+    return SBN_ERR_ALIGN;
+  return sbn::launch_pack(W, out, in, n, m, eps, codes, d.codes_ld, d.codes_row_bytes, meta,
+                          d.meta_ld, d.meta_row_bytes, gamma_eff,
+                          static_cast<sbn::PackWorkspace *>(workspace), dense_dbg, err_flag,
+                          static_cast<cudaStream_t>(stream));
+}
+
+sbn_status sbn_quantize_acts(const void *X, int64_t tokens, int64_t in, int8_t *Xq,
+                             float *absmax, int32_t *err_flag, void *stream) {
+  sbn_status st = check_in(in);
+  if (st != SBN_OK) return st;
+  if (tokens < 0 || tokens > (1ll << 31) - 1) return SBN_ERR_SHAPE;
+  if (tokens == 0) return SBN_OK;  // empty batch: nothing to read or write
+  if (!X || !Xq || !absmax) return SBN_ERR_NULL;
+  if (!aligned16(X) || !aligned16(Xq) || (reinterpret_cast<uintptr_t>(absmax) & 3u) ||
+      (reinterpret_cast<uintptr_t>(err_flag) & 3u))
+    return SBN_ERR_ALIGN;
+  return sbn::launch_act_quant(X, tokens, in, Xq, absmax, err_flag,
+                               static_cast<cudaStream_t>(stream));
+}
+
+sbn_status sbn_linear(const int8_t *Xq, const float *absmax, const uint8_t *codes,
+                      const uint8_t *meta, const float *gamma_eff, int64_t tokens, int64_t out,
+                      int64_t in, int n, int m, void *Y, int y_is_bf16, int32_t *acc_dbg,
+                      int32_t *err_flag, void *stream) {
+  sbn_dims d;
+  sbn_status st = sbn_linear_ref_dims(out, in, n, m, &d);
+  if (st != SBN_OK) return st;
+  if (tokens < 0 || tokens > (1ll << 31) - 1) return SBN_ERR_SHAPE;
+  if (tokens == 0) return SBN_OK;  // empty batch: nothing to read or write
+  if (!Xq || !absmax || !codes || !meta || !gamma_eff || !Y) return SBN_ERR_NULL;
+  if (!aligned16(Xq) || !aligned16(codes) || !aligned16(meta) || !aligned16(Y) ||
+      (acc_dbg && !aligned16(acc_dbg)) || (reinterpret_cast<uintptr_t>(absmax) & 3u) ||
+      (reinterpret_cast<uintptr_t>(gamma_eff) & 3u) || (reinterpret_cast<uintptr_t>(err_flag) & 3u))
+    return SBN_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (tokens <= sbn::kGemvMaxTokens && tokens * in <= sbn::kGemvMaxSmemBytes)
+    return sbn::launch_gemv(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, n, m, d.codes_ld,
+                            d.meta_ld, Y, y_is_bf16, acc_dbg, s);
+  return sbn::launch_gemm_tc(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, n, m,
+                             d.codes_ld, d.meta_ld, Y, y_is_bf16, acc_dbg, err_flag, s);
+}
+
+}  // extern "C"

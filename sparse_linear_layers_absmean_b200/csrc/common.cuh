@@ -1,0 +1,57 @@
+// Shared device helpers of the Sparse-BitLinear kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sbn.h"
+
+namespace sbn {
+
+constexpr int kWarp = 32;
+
+// Magnitude bits of bf16 values: NaN/Inf have all exponent bits set (>= 0x7f80);
+// 256.0 is 0x4380, the first magnitude outside the supported weight range.
+constexpr uint32_t kBf16InfBits = 0x7f80u;
+constexpr uint32_t kBf16Mag256Bits = 0x4380u;
+
+__device__ __forceinline__ float bf16_lo_to_float(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi_to_float(uint32_t w) {
+  return __uint_as_float(w & 0xffff0000u);
+}
+
+__device__ __forceinline__ uint4 ldg_v4(const void *p) {
+  return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
+  return __reduce_max_sync(0xffffffffu, v);
+}
+
+__device__ __forceinline__ uint32_t warp_or_u32(uint32_t v) {
+  return __reduce_or_sync(0xffffffffu, v);
+}
+
+// Per-token activation scale and weight scale combined as the rescale factor
+// c = fp32(fp32(g * s) / 127), then y = fp32(acc * c); no FMA contraction anywhere.
+__device__ __forceinline__ float rescale_factor(float g, float s) {
+  return __fdiv_rn(__fmul_rn(g, s), 127.0f);
+}
+
+}  // namespace sbn
+
+// Host-side launch check shared by the entry points.
+#define SBN_LAUNCH_CHECK()                                         \
+  do {                                                             \
+    if (cudaPeekAtLastError() != cudaSuccess) {                    \
+      (void)cudaGetLastError();                                    \
+      return SBN_ERR_CUDA;                                         \
+    }                                                              \
+  } while (0)

@@ -1,0 +1,347 @@
+// Tensor-core contraction (prefill): Y[t, o] = (sum_k Xq[t,k] * Ws[o,k]) * c_t on the
+// 5th-generation tensor cores (tcgen05.mma kind::i8, int32 accumulators in TMEM).
+//
+// One CTA computes a 128 (outputs) x BN (tokens) tile with a multi-stage shared-memory
+// pipeline over K in blocks of 128:
+//   warp 4     TMA producer: per K block, the int8 activation tile (128-byte swizzle,
+//              K-major) and the packed weight tile (codes, plus the 2:4 metadata) of the
+//              CTA's 128 rows.
+//   warps 0-3  weight expanders: thread r owns tile row r, reads its packed bytes from
+//              shared memory, expands them to int8 lanes of 64 * t (one shift and one AND
+//              per four weights; 2:4 codes are placed at their kept positions with a byte
+//              permute) and stores them in the swizzled K-major layout the MMA reads;
+//              then the epilogue.
+//   warp 5     TMEM allocation and the single MMA-issuing thread.
+// The accumulator carries 64 * acc; the epilogue divides by 64 exactly, multiplies by
+// c_t = fp32(fp32(g * s_t) / 127) and stores fp32 or bf16.
+// Every mbarrier wait gives up after about one second and raises SBN_FLAG_TIMEOUT.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace sbn {
+
+constexpr int kTcThreads = 192;
+constexpr int kBM = 128;
+constexpr int kBK = 128;
+constexpr uint64_t kWaitNs = 1000000000ull;  // give up a wait after ~1 s
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait on an mbarrier phase; false on timeout.
+__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    for (int i = 0; i < 256; ++i)
+      if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitNs) return false;
+  }
+}
+
+template <int BN, bool kCompact>
+struct TcCfg {
+  static constexpr int kABytes = kBM * kBK;
+  static constexpr int kBBytes = BN * kBK;
+  // packed weight bytes per row and K block: 2:4 -> 16 code + 16 meta, others -> 32 code
+  static constexpr int kPackRow = kCompact ? 16 : 32;
+  static constexpr int kPBytes = kBM * 32;
+  static constexpr int kStageBytes = kABytes + kBBytes + kPBytes;
+  static constexpr int kBudget = 225 * 1024 - BN * 4 - 512;
+  static constexpr int kStages = (kBudget / kStageBytes) > 8 ? 8 : (kBudget / kStageBytes);
+  static constexpr int kTmemCols = BN < 32 ? 32 : BN;
+  static constexpr uint32_t kTxBytes = kBBytes + kPBytes;
+  static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes +
+                                  (size_t)(3 * kStages + 1) * 8 + 16 + (size_t)BN * 4;
+};
+
+// prmt selector placing the two kept 64*t bytes (bytes `b0`, `b0+1` of the code word) of a
+// 2:4 group at positions i0 and i1 of a 4-byte word, zeros elsewhere (selector 4 picks a
+// byte of the zero operand).
+__device__ __forceinline__ uint32_t scatter_selector(uint32_t nib, uint32_t b0) {
+  const uint32_t i0 = nib & 3u, i1 = nib >> 2;
+  uint32_t sel = 0x4444u;
+  sel = (sel & ~(0xfu << (4 * i0))) | (b0 << (4 * i0));
+  sel = (sel & ~(0xfu << (4 * i1))) | ((b0 + 1u) << (4 * i1));
+  return sel;
+}
+
+template <int BN, bool kCompact>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_c,
+              const __grid_constant__ CUtensorMap tmap_m, const float *__restrict__ absmax,
+              const float *__restrict__ gamma_eff, int64_t T, int64_t O, int64_t K,
+              void *__restrict__ Y, int y_is_bf16, int32_t *__restrict__ acc_dbg,
+              int32_t *err_flag) {
+  using Cfg = TcCfg<BN, kCompact>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + S * Cfg::kABytes;
+  uint8_t *sP = sB + S * Cfg::kBBytes;
+  uint64_t *full_a = reinterpret_cast<uint64_t *>(sP + S * Cfg::kPBytes);
+  uint64_t *full_t = full_a + S;  // activation tile + packed weight tile landed
+  uint64_t *empty = full_t + S;
+  uint64_t *done = empty + S;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+  float *s_scale = reinterpret_cast<float *>(tmem_slot + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t o0 = (int64_t)blockIdx.x * kBM;
+  const int64_t t0 = (int64_t)blockIdx.y * BN;
+  const int nkb = (int)((K + kBK - 1) / kBK);
+  bool timed_out = false;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      ptx::mbar_init(&full_a[s], 4);
+      ptx::mbar_init(&full_t[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    ptx::mbar_init(done, 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 5) {
+    ptx::tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i < BN; i += kTcThreads) {
+    const int64_t t = t0 + i;
+    s_scale[i] = t < T ? rescale_factor(__ldg(gamma_eff), __ldg(absmax + t)) : 0.0f;
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < 4) {
+    // ---------------- weight expanders ----------------
+    const int r = threadIdx.x;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % S;
+      const uint32_t ph = (uint32_t)(kb / S) & 1u;
+      if ((kb >= S && !wait_phase(&empty[s], ph ^ 1u)) || !wait_phase(&full_t[s], ph)) {
+        timed_out = true;
+        break;
+      }
+      const uint8_t *prow = sP + s * Cfg::kPBytes;
+      uint4 chunk[8];
+      if constexpr (!kCompact) {
+        const uint4 c0 = *reinterpret_cast<const uint4 *>(prow + r * 32);
+        const uint4 c1 = *reinterpret_cast<const uint4 *>(prow + r * 32 + 16);
+        const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          chunk[c] = make_uint4(w[c] & 0xC0C0C0C0u, (w[c] << 2) & 0xC0C0C0C0u,
+                                (w[c] << 4) & 0xC0C0C0C0u, (w[c] << 6) & 0xC0C0C0C0u);
+      } else {
+        const uint4 cw = *reinterpret_cast<const uint4 *>(prow + r * 16);
+        const uint4 mw4 = *reinterpret_cast<const uint4 *>(prow + kBM * 16 + r * 16);
+        const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+        const uint32_t mw[4] = {mw4.x, mw4.y, mw4.z, mw4.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t out[8];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t z = (w[q] << (2 * j)) & 0xC0C0C0C0u;
+            const uint32_t m8 = (mw[q] >> (8 * j)) & 0xffu;
+            out[2 * j] = __byte_perm(z, 0u, scatter_selector(m8 & 15u, 0u));
+            out[2 * j + 1] = __byte_perm(z, 0u, scatter_selector(m8 >> 4, 2u));
+          }
+          chunk[2 * q] = make_uint4(out[0], out[1], out[2], out[3]);
+          chunk[2 * q + 1] = make_uint4(out[4], out[5], out[6], out[7]);
+        }
+      }
+      uint8_t *dst = sA + s * Cfg::kABytes + r * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4 *>(dst + ((c ^ (r & 7)) << 4)) = chunk[c];
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&full_a[s]);
+    }
+  } else if (warp == 4) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmap_x);
+      ptx::prefetch_tmap(&tmap_c);
+      if constexpr (kCompact) ptx::prefetch_tmap(&tmap_m);
+      int issued = 0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (uint32_t)(kb / S) & 1u;
+        if (kb >= S && !wait_phase(&empty[s], ph ^ 1u)) {
+          timed_out = true;
+          break;
+        }
+        ptx::mbar_arrive_expect_tx(&full_t[s], Cfg::kTxBytes);
+        ptx::tma_load_2d(sB + s * Cfg::kBBytes, &tmap_x, &full_t[s], kb * kBK, (int32_t)t0);
+        uint8_t *p = sP + s * Cfg::kPBytes;
+        ptx::tma_load_2d(p, &tmap_c, &full_t[s], kb * Cfg::kPackRow, (int32_t)o0);
+        if constexpr (kCompact)
+          ptx::tma_load_2d(p + kBM * 16, &tmap_m, &full_t[s], kb * 16, (int32_t)o0);
+        issued = kb + 1;
+      }
+      // let every issued copy land before the CTA can exit (bounded)
+      for (int kb = issued - S < 0 ? 0 : issued - S; kb < issued; ++kb)
+        if (!wait_phase(&full_t[kb % S], (uint32_t)(kb / S) & 1u)) timed_out = true;
+    }
+  } else {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = ptx::idesc_i8(kBM, BN);
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (uint32_t)(kb / S) & 1u;
+        if (!wait_phase(&full_a[s], ph) || !wait_phase(&full_t[s], ph)) {
+          timed_out = true;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t a_addr = ptx::smem_u32(sA + s * Cfg::kABytes);
+        const uint32_t b_addr = ptx::smem_u32(sB + s * Cfg::kBBytes);
+#pragma unroll
+        for (int k = 0; k < kBK / 32; ++k)
+          ptx::mma_i8(tmem, ptx::smem_desc_sw128(a_addr + 32 * k),
+                      ptx::smem_desc_sw128(b_addr + 32 * k), idesc, (kb | k) != 0);
+        ptx::mma_commit(&empty[s]);
+      }
+      ptx::mma_commit(done);
+    }
+  }
+
+  if (warp < 4) {
+    // ---------------- epilogue ----------------
+    __syncwarp();
+    if (!timed_out && !wait_phase(done, 0)) timed_out = true;
+    ptx::tc_fence_after();
+    const int64_t o = o0 + warp * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll 1
+    for (int cb = 0; cb < BN / 16; ++cb) {
+      uint32_t v[16];
+      ptx::tmem_ld_16(trow + cb * 16, v);
+      ptx::tmem_ld_wait();
+      if (!timed_out && o < O) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int64_t t = t0 + cb * 16 + i;
+          if (t < T) {
+            const int a = ((int)v[i]) >> 6;
+            const float y = __fmul_rn((float)a, s_scale[cb * 16 + i]);
+            if (y_is_bf16)
+              reinterpret_cast<__nv_bfloat16 *>(Y)[t * O + o] = __float2bfloat16_rn(y);
+            else
+              reinterpret_cast<float *>(Y)[t * O + o] = y;
+            if (acc_dbg) acc_dbg[t * O + o] = a;
+          }
+        }
+      }
+    }
+  }
+  if (timed_out && err_flag) atomicOr(err_flag, SBN_FLAG_TIMEOUT);
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void *p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D tensor map over a row-major uint8 matrix [rows, cols] with row stride `ld` bytes.
+static bool encode_u8(CUtensorMap *map, const void *base, int64_t cols, int64_t rows, int64_t ld,
+                      uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  auto encode = get_encode_fn();
+  if (!encode) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, bool kCompact>
+static sbn_status gemm_tc_t(const int8_t *Xq, const float *absmax, const uint8_t *codes,
+                            const uint8_t *meta, const float *gamma_eff, int64_t T, int64_t O,
+                            int64_t K, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
+                            int32_t *acc_dbg, int32_t *err_flag, cudaStream_t st) {
+  using Cfg = TcCfg<BN, kCompact>;
+  CUtensorMap tx, tc, tm;
+  const int64_t crow = kCompact ? K / 8 : K / 4;  // data bytes of a codes row
+  if (!encode_u8(&tx, Xq, K, T, K, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_u8(&tc, codes, crow, O, ldc, Cfg::kPackRow, kBM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_u8(&tm, meta, K / 8, O, ldm, 16, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return SBN_ERR_CUDA;
+  auto kern = k_gemm_tc<BN, kCompact>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::kSmem) !=
+      cudaSuccess)
+    return SBN_ERR_CUDA;
+  dim3 grid((unsigned)((O + kBM - 1) / kBM), (unsigned)((T + BN - 1) / BN));
+  kern<<<grid, kTcThreads, Cfg::kSmem, st>>>(tx, tc, tm, absmax, gamma_eff, T, O, K, Y, y_is_bf16,
+                                             acc_dbg, err_flag);
+  SBN_LAUNCH_CHECK();
+  return SBN_OK;
+}
+
+template <int BN>
+static sbn_status gemm_tc_bn(bool compact, const int8_t *Xq, const float *absmax,
+                             const uint8_t *codes, const uint8_t *meta, const float *gamma_eff,
+                             int64_t T, int64_t O, int64_t K, int64_t ldc, int64_t ldm, void *Y,
+                             int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag, cudaStream_t st) {
+  return compact ? gemm_tc_t<BN, true>(Xq, absmax, codes, meta, gamma_eff, T, O, K, ldc, ldm, Y,
+                                       y_is_bf16, acc_dbg, err_flag, st)
+                 : gemm_tc_t<BN, false>(Xq, absmax, codes, meta, gamma_eff, T, O, K, ldc, ldm, Y,
+                                        y_is_bf16, acc_dbg, err_flag, st);
+}
+
+sbn_status launch_gemm_tc(const int8_t *Xq, const float *absmax, const uint8_t *codes,
+                          const uint8_t *meta, const float *gamma_eff, int64_t tokens,
+                          int64_t out, int64_t in, int n, int m, int64_t ldc, int64_t ldm,
+                          void *Y, int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag,
+                          cudaStream_t st) {
+  const bool compact = (n == 2 && m == 4);
+  if (tokens > 128)
+    return gemm_tc_bn<256>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc,
+                           ldm, Y, y_is_bf16, acc_dbg, err_flag, st);
+  if (tokens > 64)
+    return gemm_tc_bn<128>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc,
+                           ldm, Y, y_is_bf16, acc_dbg, err_flag, st);
+  if (tokens > 32)
+    return gemm_tc_bn<64>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc,
+                          ldm, Y, y_is_bf16, acc_dbg, err_flag, st);
+  if (tokens > 16)
+    return gemm_tc_bn<32>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc,
+                          ldm, Y, y_is_bf16, acc_dbg, err_flag, st);
+  return gemm_tc_bn<16>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc, ldm,
+                        Y, y_is_bf16, acc_dbg, err_flag, st);
+}
+
+}  // namespace sbn

@@ -1,0 +1,51 @@
+// Internal launchers behind the C ABI (sbn.h).  Every launcher assumes its arguments were
+// validated by the entry point and enqueues work on `st` without synchronising.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sbn.h"
+
+namespace sbn {
+
+// Device workspace of the weight pack: one partial sum per CTA of the reduction, the
+// arrival ticket (zero between calls), and the values the last CTA publishes.
+constexpr int kPackMaxParts = 1024;
+struct PackWorkspace {
+  unsigned long long part[kPackMaxParts];
+  unsigned int ticket;  // CTAs of k_abs_sum that finished; the last one resets it to 0
+  unsigned int thr;     // smallest bf16 magnitude (bits) whose ternary code is non-zero
+  float g;              // gamma + eps
+  unsigned int pad;
+};
+
+int num_sms();
+
+sbn_status launch_pack(const void *W, int64_t out, int64_t in, int n, int m, float eps,
+                       uint8_t *codes, int64_t ldc, int64_t crow, uint8_t *meta, int64_t ldm,
+                       int64_t mrow, float *gamma_eff, PackWorkspace *ws, int8_t *dense_dbg,
+                       int32_t *err_flag, cudaStream_t st);
+
+sbn_status launch_act_quant(const void *X, int64_t tokens, int64_t in, int8_t *Xq,
+                            float *absmax, int32_t *err_flag, cudaStream_t st);
+
+// CUDA-core contraction for few tokens.
+sbn_status launch_gemv(const int8_t *Xq, const float *absmax, const uint8_t *codes,
+                       const uint8_t *meta, const float *gamma_eff, int64_t tokens,
+                       int64_t out, int64_t in, int n, int m, int64_t ldc, int64_t ldm,
+                       void *Y, int y_is_bf16, int32_t *acc_dbg, cudaStream_t st);
+
+// Tensor-core (tcgen05, int8) contraction.
+sbn_status launch_gemm_tc(const int8_t *Xq, const float *absmax, const uint8_t *codes,
+                          const uint8_t *meta, const float *gamma_eff, int64_t tokens,
+                          int64_t out, int64_t in, int n, int m, int64_t ldc, int64_t ldm,
+                          void *Y, int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag,
+                          cudaStream_t st);
+
+// Largest token count routed to the CUDA-core kernel, and the largest activation block
+// (tokens * in bytes) it stages in shared memory; larger calls use the tensor cores.
+constexpr int64_t kGemvMaxTokens = 4;
+constexpr int64_t kGemvMaxSmemBytes = 192 * 1024;
+
+}  // namespace sbn

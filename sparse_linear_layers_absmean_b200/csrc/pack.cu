@@ -1,0 +1,404 @@
+// Weight path of the Sparse-BitLinear forward: absmean scale, ternary codes, N:M mask
+// from the master magnitudes applied after quantisation, and the 2-bit + metadata pack.
+// (Sparse-BitNet technical summaries, section 2 "Methodology": Sparse-BitLinear items 1-2,
+// mask generation from the BF16 masters, quant-then-mask order.)
+//
+// Two launches on the caller's stream:
+//   k_abs_sum          exact integer sum S = sum trunc(|W| * 2^24) (one partial per CTA);
+//                      the last CTA to finish turns S into gamma, g = gamma + eps and the
+//                      code threshold, and re-arms the workspace.
+//   k_quant_mask_pack  one pass over W: each lane owns 8 consecutive weights (one 16-byte
+//                      load), computes the keep mask of its group(s), the codes, and the
+//                      lanes of a 64-weight block assemble their packed words by shuffles.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace sbn {
+
+// ---------------------------------------------------------------------------------------
+// S1: per-tensor absmean scale.
+// ---------------------------------------------------------------------------------------
+
+// Smallest bf16 magnitude (as bits) whose ternary code is non-zero for this g:
+// round_half_even(x / g) != 0  <=>  fl(x / g) > 0.5, and fl(x / g) is non-decreasing in x,
+// so the set of non-zero magnitudes is an up-set found by bisection over the bit patterns
+// (positive bf16 values are ordered like their bits).  Every division is IEEE fp32.
+__device__ uint32_t code_threshold(float g) {
+  uint32_t lo = 0, hi = kBf16InfBits;  // predicate false at 0 (0/g), true at +Inf
+  while (hi - lo > 1) {
+    uint32_t mid = (lo + hi) >> 1;
+    if (__fdiv_rn(__uint_as_float(mid << 16), g) > 0.5f)
+      hi = mid;
+    else
+      lo = mid;
+  }
+  return hi;
+}
+
+__global__ void __launch_bounds__(256) k_abs_sum(const uint4 *__restrict__ W, int64_t nvec,
+                                                 int64_t n, float eps, PackWorkspace *ws,
+                                                 float *gamma_eff, int32_t *err_flag) {
+  unsigned long long acc = 0;
+  uint32_t mx_all = 0, mx_fin = 0;
+  auto consume = [&](const uint4 &v) {
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t a = w4[q] & 0x7fff7fffu;  // |W| of both halves
+      mx_all = __vmaxu2(mx_all, a);
+      const uint32_t nonfin = __vcmpgeu2(a, 0x7f807f80u);
+      mx_fin = __vmaxu2(mx_fin, a & ~nonfin);
+      // |W| * 2^24 is exact in fp32; the conversion truncates toward zero.
+      const float lo = __fmul_rn(__uint_as_float(a << 16), 16777216.0f);
+      const float hi = __fmul_rn(__uint_as_float(a & 0xffff0000u), 16777216.0f);
+      acc += (unsigned long long)__float2uint_rz(lo) + (unsigned long long)__float2uint_rz(hi);
+    }
+  };
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < nvec; i += 4 * stride) {  // four 16-byte loads in flight
+    const uint4 v0 = __ldg(W + i), v1 = __ldg(W + i + stride), v2 = __ldg(W + i + 2 * stride),
+                v3 = __ldg(W + i + 3 * stride);
+    consume(v0);
+    consume(v1);
+    consume(v2);
+    consume(v3);
+  }
+  for (; i < nvec; i += stride) consume(__ldg(W + i));
+  __shared__ unsigned long long s_sum[8];
+  __shared__ uint32_t s_all[8], s_fin[8];
+  __shared__ int s_last;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  acc = warp_sum_u64(acc);
+  uint32_t ma = warp_max_u32(max(mx_all & 0xffffu, mx_all >> 16));
+  uint32_t mf = warp_max_u32(max(mx_fin & 0xffffu, mx_fin >> 16));
+  if (lane == 0) {
+    s_sum[warp] = acc;
+    s_all[warp] = ma;
+    s_fin[warp] = mf;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long sum = 0;
+    uint32_t a = 0, f = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+      sum += s_sum[w];
+      a = max(a, s_all[w]);
+      f = max(f, s_fin[w]);
+    }
+    ws->part[blockIdx.x] = sum;
+    int flags = 0;
+    if (a >= kBf16InfBits) flags |= SBN_FLAG_W_NONFINITE;
+    if (f >= kBf16Mag256Bits) flags |= SBN_FLAG_W_RANGE;
+    if (flags && err_flag) atomicOr(err_flag, flags);
+    __threadfence();
+    unsigned int ticket = atomicAdd(&ws->ticket, 1u);
+    s_last = (ticket == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  // Last CTA: every other CTA's partial is visible (fence before each ticket).
+  __threadfence();
+  unsigned long long S = 0;
+  for (int i = threadIdx.x; i < (int)gridDim.x; i += blockDim.x) S += __ldcg(&ws->part[i]);
+  S = warp_sum_u64(S);
+  if (lane == 0) s_sum[warp] = S;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long tot = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += s_sum[w];
+    double mean = __ddiv_rn(__ull2double_rn(tot), (double)n * 16777216.0);
+    float gamma = __double2float_rn(mean);
+    float g = __fadd_rn(gamma, eps);
+    *gamma_eff = g;
+    ws->g = g;
+    ws->thr = code_threshold(g);
+    ws->ticket = 0;  // re-arm for the next call on this stream
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// S2-S4: codes, mask, pack.
+// ---------------------------------------------------------------------------------------
+
+// Keep mask of one group of M magnitudes: the N largest, the lower index winning ties.
+// Keys (mag << 3) | (M-1-i) are distinct and order exactly like that rule.
+template <int N, int M>
+__device__ __forceinline__ uint32_t group_keep(const uint32_t *mag) {
+  if constexpr (N == M) {
+    return (1u << M) - 1u;
+  } else {
+    uint32_t key[M];
+#pragma unroll
+    for (int i = 0; i < M; ++i) key[i] = (mag[i] << 3) | (uint32_t)(M - 1 - i);
+    uint32_t keep = 0;
+    if constexpr (M - N <= N) {
+      // drop the M-N smallest keys: tau = (M-N)-th smallest
+      constexpr int D = M - N;
+      uint32_t s[D];
+#pragma unroll
+      for (int d = 0; d < D; ++d) s[d] = 0xffffffffu;
+#pragma unroll
+      for (int i = 0; i < M; ++i) {
+        uint32_t x = key[i];
+#pragma unroll
+        for (int d = 0; d < D; ++d) {
+          uint32_t lo = min(s[d], x);
+          x = max(s[d], x);
+          s[d] = lo;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < M; ++i) keep |= (uint32_t)(key[i] > s[D - 1]) << i;
+    } else {
+      // keep the N largest keys: tau = N-th largest
+      uint32_t s[N];
+#pragma unroll
+      for (int d = 0; d < N; ++d) s[d] = 0u;
+#pragma unroll
+      for (int i = 0; i < M; ++i) {
+        uint32_t x = key[i];
+#pragma unroll
+        for (int d = 0; d < N; ++d) {
+          uint32_t hi = max(s[d], x);
+          x = min(s[d], x);
+          s[d] = hi;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < M; ++i) keep |= (uint32_t)(key[i] >= s[N - 1]) << i;
+    }
+    return keep;
+  }
+}
+
+// bits 0..3 of x -> bit 0 of bytes 0..3
+__device__ __forceinline__ uint32_t spread4_to_bytes(uint32_t x) {
+  return (x * 0x00204081u) & 0x01010101u;
+}
+
+// For a 2:4 keep nibble with exactly two bits set: the meta nibble i0 | i1 << 2.
+// Table indexed by the keep nibble (4 bits per entry); other entries are unused.
+constexpr unsigned long long kPairNibbleLut =
+    (4ull << (4 * 0x3)) | (8ull << (4 * 0x5)) | (9ull << (4 * 0x6)) | (12ull << (4 * 0x9)) |
+    (13ull << (4 * 0xA)) | (14ull << (4 * 0xC));
+
+// Exact b / d for b < 2^25 and 1 <= d <= 2^11: with L = ceil(log2 d) and
+// M = ceil(2^(31+L) / d) < 2^32, b / d == (b * M) >> (31 + L) (the error term b*(M*d - 2^(31+L))
+// stays below 2^(31+L) because b < 2^31).
+struct FastDiv {
+  uint32_t mul, shift;  // shift = L - 1, or 0xffffffff for d == 1
+};
+
+__device__ __forceinline__ uint32_t fast_div(uint32_t b, FastDiv f) {
+  return f.shift == 0xffffffffu ? b : (__umulhi(b, f.mul) >> f.shift);
+}
+
+template <int N, int M>
+struct QmpArgs {
+  const uint4 *W;
+  int64_t nblocks;
+  uint32_t bpr;
+  FastDiv div_bpr;
+  const PackWorkspace *ws;
+  uint8_t *codes;
+  int64_t ldc, codes_row_bytes;
+  uint8_t *meta;
+  int64_t ldm, meta_row_bytes;
+  int8_t *dense_dbg;
+};
+
+// One 64-weight block per 8 lanes: lane `sub` owns weights 8*sub .. 8*sub+7 of block b.
+template <int N, int M>
+__device__ __forceinline__ void qmp_block(const QmpArgs<N, M> &a, uint4 v, int64_t b, int sub,
+                                          uint32_t thr) {
+  constexpr bool kCompact = (N == 2 && M == 4);
+  constexpr int kCodeBytesPerBlock = kCompact ? 8 : 16;  // 32 or 64 stored elements
+  const bool valid = b < a.nblocks;
+  const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+  uint32_t mag[8];
+  uint32_t neg = 0;
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const uint32_t h = (w4[p >> 1] >> (16 * (p & 1))) & 0xffffu;
+    mag[p] = h & 0x7fffu;
+    neg |= (h >> 15) << p;
+  }
+  uint32_t keep;
+  if constexpr (M == 8) {
+    keep = group_keep<N, 8>(mag);
+  } else {
+    keep = group_keep<N, 4>(mag) | (group_keep<N, 4>(mag + 4) << 4);
+  }
+  uint32_t nz = 0;
+#pragma unroll
+  for (int p = 0; p < 8; ++p) nz |= (uint32_t)(mag[p] >= thr) << p;
+  const uint32_t nzneg = nz & neg;
+
+  uint32_t word, meta_byte;
+  if constexpr (kCompact) {
+    // stored elements 4*sub .. 4*sub+3 = (group A kept i0, i1, group B kept i0, i1);
+    // they are j = sub % 4 of word sub / 4, bytes 0..3, bit 6 - 2j.
+    const uint32_t nibA = (uint32_t)(kPairNibbleLut >> (4 * (keep & 15u))) & 15u;
+    const uint32_t nibB = (uint32_t)(kPairNibbleLut >> (4 * (keep >> 4))) & 15u;
+    const uint32_t pos0 = nibA & 3u, pos1 = nibA >> 2, pos2 = 4u + (nibB & 3u),
+                   pos3 = 4u + (nibB >> 2);
+    // bit 0 of byte k <- "non-zero" at the k-th kept position; bit 1 <- "negative"
+    const uint32_t lo = ((nz >> pos0) & 1u) | (((nz >> pos1) & 1u) << 8) |
+                        (((nz >> pos2) & 1u) << 16) | (((nz >> pos3) & 1u) << 24);
+    const uint32_t hi = ((nzneg >> pos0) & 1u) | (((nzneg >> pos1) & 1u) << 8) |
+                        (((nzneg >> pos2) & 1u) << 16) | (((nzneg >> pos3) & 1u) << 24);
+    word = (lo | (hi << 1)) << (6 - 2 * (sub & 3));
+    meta_byte = nibA | (nibB << 4);
+    word |= __shfl_xor_sync(0xffffffffu, word, 1);
+    word |= __shfl_xor_sync(0xffffffffu, word, 2);
+  } else {
+    // stored elements 8*sub + p: word sub/2, j = 2*(sub&1) + p/4, byte p%4;
+    // pruned positions hold the code of 0
+    const int jb = 2 * (sub & 1);
+    const uint32_t kn = nz & keep, kneg = nzneg & keep;
+    const uint32_t c_lo = spread4_to_bytes(kn & 15u) | (spread4_to_bytes(kneg & 15u) << 1);
+    const uint32_t c_hi = spread4_to_bytes(kn >> 4) | (spread4_to_bytes(kneg >> 4) << 1);
+    word = (c_lo << (6 - 2 * jb)) | (c_hi << (4 - 2 * jb));
+    meta_byte = keep;  // M == 8: one group; M == 4: group A low nibble, B high nibble
+    word |= __shfl_xor_sync(0xffffffffu, word, 1);
+  }
+  uint32_t mword = meta_byte << (8 * (sub & 3));
+  mword |= __shfl_xor_sync(0xffffffffu, mword, 1);
+  mword |= __shfl_xor_sync(0xffffffffu, mword, 2);
+  if (!valid) return;
+  const uint32_t row = fast_div((uint32_t)b, a.div_bpr);
+  const uint32_t col = (uint32_t)b - row * a.bpr;
+  uint8_t *crow = a.codes + (int64_t)row * a.ldc + col * kCodeBytesPerBlock;
+  if constexpr (kCompact) {
+    if ((sub & 3) == 0) reinterpret_cast<uint32_t *>(crow)[sub >> 2] = word;
+  } else {
+    if ((sub & 1) == 0) reinterpret_cast<uint32_t *>(crow)[sub >> 1] = word;
+  }
+  uint8_t *mrow = a.meta + (int64_t)row * a.ldm + col * 8;
+  if ((sub & 3) == 0) reinterpret_cast<uint32_t *>(mrow)[sub >> 2] = mword;
+  if (col == a.bpr - 1 && sub == 0) {
+    // zero padding up to the 16-byte row stride (0 or 8 bytes)
+    if (a.ldc > a.codes_row_bytes)
+      *reinterpret_cast<uint2 *>(a.codes + (int64_t)row * a.ldc + a.codes_row_bytes) =
+          make_uint2(0u, 0u);
+    if (a.ldm > a.meta_row_bytes)
+      *reinterpret_cast<uint2 *>(a.meta + (int64_t)row * a.ldm + a.meta_row_bytes) =
+          make_uint2(0u, 0u);
+  }
+  if (a.dense_dbg) {
+    // masked ternary values, one int8 per position
+    const uint32_t kn = keep & nz, kneg = keep & nzneg;
+    const uint32_t lo4 = spread4_to_bytes(kn & 15u) | (spread4_to_bytes(kneg & 15u) * 0xfeu);
+    const uint32_t hi4 = spread4_to_bytes(kn >> 4) | (spread4_to_bytes(kneg >> 4) * 0xfeu);
+    *reinterpret_cast<uint2 *>(a.dense_dbg + b * 64 + sub * 8) = make_uint2(lo4, hi4);
+  }
+}
+
+template <int N, int M>
+__global__ void __launch_bounds__(256) k_quant_mask_pack(const QmpArgs<N, M> a) {
+  const uint32_t thr = a.ws->thr;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane & 7;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t nquads = (a.nblocks + 3) >> 2;
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+  // each warp takes quads q and q + nwarps per iteration: two 16-byte loads in flight
+  for (int64_t q = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; q < nquads;
+       q += 2 * nwarps) {
+    const int64_t b0 = 4 * q + (lane >> 3);
+    const int64_t b1 = b0 + 4 * nwarps;
+    const uint4 v0 = b0 < a.nblocks ? __ldg(a.W + b0 * 8 + sub) : zero;
+    const uint4 v1 = b1 < a.nblocks ? __ldg(a.W + b1 * 8 + sub) : zero;
+    qmp_block<N, M>(a, v0, b0, sub, thr);
+    if (q + nwarps < nquads) qmp_block<N, M>(a, v1, b1, sub, thr);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Host launchers
+// ---------------------------------------------------------------------------------------
+
+int num_sms() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 148;
+  }
+  return sms;
+}
+
+static FastDiv make_fast_div(uint32_t d) {
+  FastDiv f;
+  if (d == 1) {
+    f.mul = 0;
+    f.shift = 0xffffffffu;
+    return f;
+  }
+  uint32_t L = 0;
+  while ((1u << L) < d) ++L;
+  f.mul = (uint32_t)(((1ull << (31 + L)) + d - 1) / d);
+  f.shift = L - 1;
+  return f;
+}
+
+template <int N, int M>
+static void launch_qmp(const uint4 *W, int64_t nblocks, int64_t bpr, const PackWorkspace *ws,
+                       uint8_t *codes, int64_t ldc, int64_t crow, uint8_t *meta, int64_t ldm,
+                       int64_t mrow, int8_t *dense_dbg, cudaStream_t st) {
+  const int threads = 256;
+  const int64_t nquads = (nblocks + 3) / 4;
+  int64_t grid = (nquads + 15) / 16;  // 8 warps x 2 quads per CTA iteration
+  const int64_t cap = (int64_t)num_sms() * 8;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  QmpArgs<N, M> a{W, nblocks, (uint32_t)bpr, make_fast_div((uint32_t)bpr), ws, codes, ldc, crow,
+                  meta, ldm, mrow, dense_dbg};
+  k_quant_mask_pack<N, M><<<(unsigned)grid, threads, 0, st>>>(a);
+}
+
+sbn_status launch_pack(const void *W, int64_t out, int64_t in, int n, int m, float eps,
+                       uint8_t *codes, int64_t ldc, int64_t crow, uint8_t *meta, int64_t ldm,
+                       int64_t mrow, float *gamma_eff, PackWorkspace *ws, int8_t *dense_dbg,
+                       int32_t *err_flag, cudaStream_t st) {
+  const int64_t nel = out * in;
+  const int64_t nvec = nel / 8;
+  int64_t grid = (nvec + 256 * 4 - 1) / (256 * 4);
+  const int64_t cap = (int64_t)num_sms() * 4;
+  if (grid > cap) grid = cap;
+  if (grid > kPackMaxParts) grid = kPackMaxParts;
+  if (grid < 1) grid = 1;
+  k_abs_sum<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint4 *>(W), nvec, nel, eps,
+                                           ws, gamma_eff, err_flag);
+  SBN_LAUNCH_CHECK();
+  const uint4 *W4 = reinterpret_cast<const uint4 *>(W);
+  const int64_t nblocks = nel / 64, bpr = in / 64;
+#define SBN_QMP(NN, MM)                                                                    \
+  case (NN * 16 + MM):                                                                     \
+    launch_qmp<NN, MM>(W4, nblocks, bpr, ws, codes, ldc, crow, meta, ldm, mrow, dense_dbg, \
+                       st);                                                                \
+    break;
+  switch (n * 16 + m) {
+    SBN_QMP(1, 4)
+    SBN_QMP(2, 4)
+    SBN_QMP(3, 4)
+    SBN_QMP(4, 4)
+    SBN_QMP(1, 8)
+    SBN_QMP(2, 8)
+    SBN_QMP(3, 8)
+    SBN_QMP(4, 8)
+    SBN_QMP(5, 8)
+    SBN_QMP(6, 8)
+    SBN_QMP(7, 8)
+    SBN_QMP(8, 8)
+    default:
+      return SBN_ERR_PATTERN;
+  }
+#undef SBN_QMP
+  SBN_LAUNCH_CHECK();
+  return SBN_OK;
+}
+
+}  // namespace sbn

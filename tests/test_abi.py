@@ -1,0 +1,98 @@
+"""The C ABI library loads, exports every entry point its header declares, and rejects bad
+arguments on the host before touching a GPU (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+import sparse_linear_layers_absmean_b200 as sbn
+from sparse_linear_layers_absmean_b200 import build as sbn_build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "sbn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    sbn_build.build()
+    return sbn.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SBN_API\s+[\w\s\*]+?\b(sbn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    assert set(sbn.EXPORTED) <= set(declared_symbols())
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8), (1, 4), (3, 4), (4, 4), (1, 8), (5, 8), (8, 8)])
+@pytest.mark.parametrize("out,in_", [(1, 64), (37, 192), (256, 256), (6912, 2560), (300, 3200),
+                                     (7, 8640)])
+def test_dims_match_the_oracle_geometry(L, n, m, out, in_):
+    d = sbn.sbn_linear_ref_dims(out, in_, n, m)
+    ldc, ldm = oracle.plane_dims(in_, n, m)
+    assert (d.codes_ld, d.meta_ld) == (ldc, ldm)
+    assert d.codes_bytes == out * ldc and d.meta_bytes == out * ldm
+    stored = in_ // 2 if (n, m) == (2, 4) else in_
+    assert d.codes_row_bytes == stored // 4 and d.meta_row_bytes == in_ // 8
+    assert d.pack_workspace_bytes >= 8 * 1024 and d.pack_workspace_bytes % 256 == 0
+
+
+@pytest.mark.parametrize("args,status", [
+    ((0, 64, 2, 4), 2), ((-1, 64, 2, 4), 2), ((8, 0, 2, 4), 2), ((8, 96, 2, 4), 2),
+    ((8, 32, 2, 4), 2), ((8, 64 * 3000, 2, 4), 2), ((2 ** 20, 4096, 2, 4), 2),
+    ((8, 64, 2, 3), 3), ((8, 64, 0, 4), 3), ((8, 64, 5, 4), 3), ((8, 64, 9, 8), 3),
+    ((8, 64, 2, 16), 3)])
+def test_dims_rejects_bad_arguments(L, args, status):
+    d = sbn.SbnDims()
+    assert L.sbn_linear_ref_dims(*args, ctypes.byref(d)) == status
+    assert L.sbn_linear_ref_dims(*args[:4], None) in (1, status)
+
+
+def _p(v):
+    return ctypes.c_void_p(v)
+
+
+def test_entry_points_validate_before_launching(L):
+    # Every call below fails validation on the host and returns before any CUDA call.
+    A = _p(0x10000)   # a 16-byte aligned placeholder address, never dereferenced
+    U = _p(0x10008)   # misaligned
+    f = ctypes.c_float
+    q = L.sbn_quantize_mask_pack_weights
+    assert q(None, 8, 64, 2, 4, f(1e-5), A, A, A, A, None, None, None) == 1
+    assert q(A, 8, 64, 2, 4, f(1e-5), None, A, A, A, None, None, None) == 1
+    assert q(A, 8, 64, 2, 4, f(1e-5), A, A, A, None, None, None, None) == 1
+    assert q(A, 8, 96, 2, 4, f(1e-5), A, A, A, A, None, None, None) == 2
+    assert q(A, 8, 64, 3, 5, f(1e-5), A, A, A, A, None, None, None) == 3
+    assert q(U, 8, 64, 2, 4, f(1e-5), A, A, A, A, None, None, None) == 4
+    assert q(A, 8, 64, 2, 4, f(1e-5), A, A, A, A, U, None, None) == 4
+    assert q(A, 8, 64, 2, 4, f(-1.0), A, A, A, A, None, None, None) == 6
+    assert q(A, 8, 64, 2, 4, f(float("nan")), A, A, A, A, None, None, None) == 6
+    assert q(A, 8, 64, 2, 4, f(float("inf")), A, A, A, A, None, None, None) == 6
+    a = L.sbn_quantize_acts
+    assert a(None, 4, 64, A, A, None, None) == 1
+    assert a(A, 4, 65, A, A, None, None) == 2
+    assert a(A, -1, 64, A, A, None, None) == 2
+    assert a(U, 4, 64, A, A, None, None) == 4
+    assert a(A, 0, 64, A, A, None, None) == 0  # empty: a valid no-op, nothing launched
+    ln = L.sbn_linear
+    assert ln(A, A, A, A, A, 4, 8, 64, 2, 4, None, 0, None, None, None) == 1
+    assert ln(A, A, A, A, A, 4, 8, 64, 2, 7, A, 0, None, None, None) == 3
+    assert ln(A, A, A, A, A, -2, 8, 64, 2, 4, A, 0, None, None, None) == 2
+    assert ln(A, A, A, A, A, 4, 8, 64, 2, 4, U, 0, None, None, None) == 4
+    assert ln(A, A, A, A, A, 0, 8, 64, 2, 4, A, 0, None, None, None) == 0
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert L.sbn_status_string(s)

@@ -1,0 +1,148 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI (needs a B200).
+
+Bit-exact: gamma (as fp32 bits), codes and meta planes including the zero padding, the
+masked ternary matrix, int8 activations, per-token scales, int32 accumulators.
+Float: fp32 y within 1e-5 relative of the oracle's fp64 y; bf16 y within 8e-3."""
+import numpy as np
+import pytest
+import torch
+
+import gpu_path
+import oracle
+import workloads
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+PATTERNS = [(2, 4), (6, 8), (1, 4), (3, 4), (4, 4), (1, 8), (2, 8), (3, 8), (4, 8), (5, 8),
+            (7, 8), (8, 8)]
+
+
+def check_pack(W_bits, n, m, eps=1e-5):
+    got = gpu_path.pack(W_bits, n, m, eps)
+    ref = oracle.quantize_mask_pack(W_bits, n, m, eps)
+    assert got["err"] == ref["err"] == 0
+    assert got["g"].view(np.uint32) == np.float32(ref["g"]).view(np.uint32), (got["g"], ref["g"])
+    assert np.array_equal(got["ws"], ref["ws"])
+    assert np.array_equal(got["meta"], ref["meta"])
+    assert np.array_equal(got["codes"], ref["codes"])
+    return got, ref
+
+
+@pytest.mark.parametrize("n,m", PATTERNS)
+@pytest.mark.parametrize("O,K", [(1, 64), (37, 192), (130, 320), (9, 3200)])
+def test_pack_small(n, m, O, K):
+    check_pack(workloads.masters(O, K, seed=O * K + n * 8 + m), n, m)
+
+
+def test_pack_ties_and_signed_zeros():
+    rng = np.random.default_rng(0)
+    vals = np.array([0.0, -0.0, 0.015625, -0.015625, 0.03125, -0.03125], np.float32)
+    W = workloads.to_bf16_bits(rng.choice(vals, size=(64, 256)))
+    for n, m in [(2, 4), (6, 8), (3, 8), (1, 4)]:
+        check_pack(W, n, m)
+
+
+def test_pack_exact_half_ties():
+    # mean |W| = 0.5 exactly with eps = 0: 0.25 / 0.5 = 0.5 -> 0, 0.75 / 0.5 = 1.5 -> 1
+    row = np.array([0.25, 0.75, 0.5, 0.5, -0.25, -0.75, -0.5, -0.5], np.float32)
+    W = workloads.to_bf16_bits(np.tile(row, (16, 8)))
+    got, ref = check_pack(W, 8, 8, eps=0.0)
+    assert got["g"] == np.float32(0.5)
+
+
+def test_pack_all_zero_with_zero_eps():
+    W = np.zeros((8, 128), np.uint16)
+    got, ref = check_pack(W, 2, 4, eps=0.0)
+    assert got["g"] == 0 and not got["ws"].any()
+
+
+def test_pack_workspace_is_rearmed():
+    W1 = workloads.masters(64, 256, seed=1)
+    W2 = workloads.masters(64, 256, seed=2)
+    import sparse_linear_layers_absmean_b200 as sbn
+    ws = sbn.new_workspace(64, 256, 2, 4)
+    for W in (W1, W2, W1):
+        got = gpu_path.pack(W, 2, 4, workspace=ws)
+        ref = oracle.quantize_mask_pack(W, 2, 4)
+        assert got["g"] == ref["g"] and np.array_equal(got["codes"], ref["codes"])
+    # the arrival counter (first word after the 1024 partial sums) is back at zero
+    assert ws[8192:8196].cpu().numpy().view(np.uint32)[0] == 0
+
+
+@pytest.mark.parametrize("bad,flag", [(np.nan, 1), (np.inf, 1), (-np.inf, 1), (300.0, 2),
+                                      (-256.0, 2)])
+def test_pack_flags_bad_weights(bad, flag):
+    W = workloads.masters(16, 128, seed=3)
+    W[5, 77] = workloads.to_bf16_bits(np.array([bad], np.float32))[0]
+    got = gpu_path.pack(W, 2, 4)
+    assert got["err"] == flag
+
+
+@pytest.mark.parametrize("T,K", [(1, 64), (3, 256), (8, 2560), (37, 4096), (5, 11008),
+                                 (2, 20480)])
+def test_act_quant(T, K):
+    X = workloads.activations(T, K, seed=T * K)
+    X[0, :7] = workloads.to_bf16_bits(np.array([0.5, -0.5, 1.5, 2.5, -2.5, 0, -0.0], np.float32))
+    if T > 2:
+        X[1] = 0
+    got = gpu_path.quant(X)
+    Xq, s, err = oracle.quant_acts(X)
+    assert got["err"] == err == 0
+    assert np.array_equal(got["s"].view(np.uint32), s.view(np.uint32))
+    assert np.array_equal(got["Xq"], Xq)
+
+
+def test_act_quant_flags_nonfinite():
+    X = workloads.activations(4, 256, seed=5)
+    X[2, 9] = workloads.to_bf16_bits(np.array([np.nan], np.float32))[0]
+    assert gpu_path.quant(X)["err"] == 4
+
+
+def check_linear(T, O, K, n, m, seed, out_dtype=torch.float32, eps=1e-5):
+    W = workloads.masters(O, K, seed=seed)
+    X = workloads.activations(T, K, seed=seed + 1)
+    got = gpu_path.linear(X, W, n, m, eps, out_dtype)
+    ref = oracle.linear(X, W, n, m, eps)
+    assert got["err"] == 0
+    assert np.array_equal(got["quant"]["Xq"], ref["Xq"])
+    assert np.array_equal(got["pack"]["codes"], ref["codes"])
+    assert np.array_equal(got["acc"], ref["acc"]), np.argwhere(got["acc"] != ref["acc"])[:8]
+    gpu_path.assert_y_close(got["y"], ref["y"], bf16=out_dtype == torch.bfloat16)
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8), (4, 4), (1, 8)])
+@pytest.mark.parametrize("T", [1, 2, 3, 4])
+@pytest.mark.parametrize("O,K", [(37, 192), (300, 640)])
+def test_linear_cuda_cores(T, O, K, n, m):
+    check_linear(T, O, K, n, m, seed=T + O + K + n)
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8), (8, 8), (3, 4)])
+@pytest.mark.parametrize("T", [5, 16, 17, 40, 100, 129, 300])
+@pytest.mark.parametrize("O,K", [(300, 192), (130, 640)])
+def test_linear_tensor_cores(T, O, K, n, m):
+    check_linear(T, O, K, n, m, seed=T * 7 + O + K + n)
+
+
+@pytest.mark.parametrize("T", [1, 3, 9, 300])
+def test_linear_bf16_output(T):
+    check_linear(T, 260, 256, 2, 4, seed=11, out_dtype=torch.bfloat16)
+    check_linear(T, 260, 256, 6, 8, seed=12, out_dtype=torch.bfloat16)
+
+
+def test_linear_zero_tokens_is_noop():
+    import sparse_linear_layers_absmean_b200 as sbn
+    w = sbn.pack_weights(workloads.torch_bf16(workloads.masters(8, 64), "cuda"), 2, 4)
+    Xq = torch.empty((0, 64), dtype=torch.int8, device="cuda")
+    s = torch.empty((0,), dtype=torch.float32, device="cuda")
+    Y = sbn.linear(Xq, s, w)
+    assert Y.shape == (0, 8)
+
+
+def test_linear_zero_token_row_gives_zero():
+    W = workloads.masters(140, 256, seed=4)
+    X = workloads.activations(20, 256, seed=5)
+    X[3] = 0
+    got = gpu_path.linear(X, W, 2, 4)
+    assert (got["y"][3] == 0).all() and (got["acc"][3] == 0).all()
