@@ -119,6 +119,31 @@ SBN_API sbn_status sbn_quantize_mask_pack_weights(const void *W, int64_t out, in
                                           void *stream);
 
 /*
+ * The same computation as sbn_quantize_mask_pack_weights, for callers that cannot give
+ * this library any device memory: plugin hosts that own every allocation and hand an
+ * operator no workspace, or serving loops that forbid cudaMalloc/cudaFree on their hot
+ * path because those calls can synchronise the device and fragment its memory.  (The
+ * pages have no counterpart: this is an interface convenience, not part of the method.)
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.  The pack's
+ *     scratch (absmean partial sums and an arrival counter) is a fixed 8448-byte array in
+ *     the library's own device memory; every GPU that loads the library holds it until
+ *     the process exits.
+ *   - Sizes: the same limits as sbn_quantize_mask_pack_weights (out * in < 2^31,
+ *     in <= 131072); anything larger is refused with SBN_ERR_SHAPE.
+ *   - The first call on a device looks up the array's device address (with that device
+ *     current) and caches it; make that first call before any stream capture.
+ *   - Each call clears the arrival counter on `stream` before its kernels run.  All calls
+ *     in the process share the one array per device: calls that overlap on the GPU (for
+ *     instance on two streams) race and give wrong results.
+ * Arguments and outputs are those of sbn_quantize_mask_pack_weights without `workspace`.
+ */
+SBN_API sbn_status sbn_quantize_mask_pack_weights_noalloc(const void *W, int64_t out,
+                                                          int64_t in, int n, int m, float eps,
+                                                          uint8_t *codes, uint8_t *meta,
+                                                          float *gamma_eff, int8_t *dense_dbg,
+                                                          int32_t *err_flag, void *stream);
+
+/*
  * Step 5: per-token absmax int8 activations (bitnet.cpp article, "Fundamento
  * matemático", item 2, with Qb = 127):
  *   s[t] = max(max_k |X[t,k]|, 1e-5);  Xq[t,k] = clamp(rint((127 * X[t,k]) / s[t]), +-127).

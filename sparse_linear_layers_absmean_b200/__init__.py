@@ -27,7 +27,7 @@ FLAG_X_NONFINITE = 4
 FLAG_TIMEOUT = 8
 
 EXPORTED = ("sbn_linear_ref_dims", "sbn_quantize_mask_pack_weights", "sbn_quantize_acts",
-            "sbn_linear", "sbn_status_string")
+            "sbn_linear", "sbn_status_string", "sbn_quantize_mask_pack_weights_noalloc")
 
 
 class SbnError(RuntimeError):
@@ -60,6 +60,9 @@ def lib():
         L.sbn_quantize_mask_pack_weights.argtypes = [p, i64, i64, i32, i32, ctypes.c_float, p, p,
                                                      p, p, p, p, p]
         L.sbn_quantize_mask_pack_weights.restype = i32
+        L.sbn_quantize_mask_pack_weights_noalloc.argtypes = [p, i64, i64, i32, i32,
+                                                             ctypes.c_float, p, p, p, p, p, p]
+        L.sbn_quantize_mask_pack_weights_noalloc.restype = i32
         L.sbn_quantize_acts.argtypes = [p, i64, i64, p, p, p, p]
         L.sbn_quantize_acts.restype = i32
         L.sbn_linear.argtypes = [p, p, p, p, p, i64, i64, i64, i32, i32, p, i32, p, p, p]
@@ -106,6 +109,17 @@ def sbn_quantize_mask_pack_weights(W, n, m, eps, codes, meta, gamma_eff, workspa
         _ptr(W), out, in_, n, m, ctypes.c_float(eps), _ptr(codes), _ptr(meta), _ptr(gamma_eff),
         _ptr(workspace), _ptr(dense_dbg), _ptr(err_flag), _stream(stream)),
         "sbn_quantize_mask_pack_weights")
+
+
+def sbn_quantize_mask_pack_weights_noalloc(W, n, m, eps, codes, meta, gamma_eff, dense_dbg=None,
+                                           err_flag=None, stream=None):
+    """Same outputs as sbn_quantize_mask_pack_weights, with no workspace argument: for
+    callers that cannot provide device memory (the library uses a fixed array of its own;
+    calls overlapping on the GPU race)."""
+    out, in_ = W.shape
+    _check(lib().sbn_quantize_mask_pack_weights_noalloc(
+        _ptr(W), out, in_, n, m, ctypes.c_float(eps), _ptr(codes), _ptr(meta), _ptr(gamma_eff),
+        _ptr(dense_dbg), _ptr(err_flag), _stream(stream)), "sbn_quantize_mask_pack_weights_noalloc")
 
 
 def sbn_quantize_acts(X, Xq, absmax, err_flag=None, stream=None):
