@@ -47,6 +47,55 @@ __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity) {
   }
 }
 
+// Epilogue of the tensor-core kernels: warp w (0..3) owns accumulator lanes 32w..32w+31
+// (output rows o), TMEM column j is token t0 + j and holds 64 * acc.  s_scale[j] holds
+// c_t = fp32(fp32(g * s_t) / 127).  y = fp32(acc * c_t): acc is converted exactly (the
+// magic-number addition is exact for |acc| < 2^22, a plain conversion is used otherwise)
+// and multiplied once, the same rounding as acc * c_t.
+template <int BN>
+__device__ __forceinline__ void store_tile(uint32_t trow, const float *s_scale, int64_t o,
+                                           int64_t O, int64_t t0, int64_t T, bool small_acc,
+                                           void *Y, int y_is_bf16, int32_t *acc_dbg) {
+  constexpr int kCols = BN < 32 ? BN : 32;
+  const bool row_ok = o < O;
+#pragma unroll 1
+  for (int cb = 0; cb < BN; cb += 2 * kCols) {
+    uint32_t va[32], vb[32];
+    if constexpr (kCols == 32) {
+      ptx::tmem_ld_32(trow + cb, va);
+      if (cb + 32 < BN) ptx::tmem_ld_32(trow + cb + 32, vb);
+    } else {
+      uint32_t v16[16];
+      ptx::tmem_ld_16(trow + cb, v16);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) va[i] = v16[i];
+    }
+    ptx::tmem_ld_wait();
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int c0 = cb + half * kCols;
+      if (c0 >= BN || !row_ok) continue;
+      const uint32_t *v = half ? vb : va;
+      const int64_t nt = T - (t0 + c0);  // columns of this chunk that are real tokens
+      float *yf = reinterpret_cast<float *>(Y) + (t0 + c0) * O + o;
+      __nv_bfloat16 *yb = reinterpret_cast<__nv_bfloat16 *>(Y) + (t0 + c0) * O + o;
+#pragma unroll
+      for (int i = 0; i < kCols; ++i) {
+        if (i >= nt) break;
+        const int a = ((int)v[i]) >> 6;
+        const float fa = small_acc ? __fsub_rn(__int_as_float(a + 0x4B400000), 12582912.0f)
+                                   : __int2float_rn(a);
+        const float y = __fmul_rn(fa, s_scale[c0 + i]);
+        if (y_is_bf16)
+          yb[(int64_t)i * O] = __float2bfloat16_rn(y);
+        else
+          yf[(int64_t)i * O] = y;
+        if (acc_dbg) acc_dbg[(t0 + c0 + i) * O + o] = a;
+      }
+    }
+  }
+}
+
 template <int BN, bool kCompact>
 struct TcCfg {
   static constexpr int kABytes = kBM * kBK;
@@ -228,27 +277,192 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     ptx::tc_fence_after();
     const int64_t o = o0 + warp * 32 + lane;
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-#pragma unroll 1
-    for (int cb = 0; cb < BN / 16; ++cb) {
-      uint32_t v[16];
-      ptx::tmem_ld_16(trow + cb * 16, v);
-      ptx::tmem_ld_wait();
-      if (!timed_out && o < O) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int64_t t = t0 + cb * 16 + i;
-          if (t < T) {
-            const int a = ((int)v[i]) >> 6;
-            const float y = __fmul_rn((float)a, s_scale[cb * 16 + i]);
-            if (y_is_bf16)
-              reinterpret_cast<__nv_bfloat16 *>(Y)[t * O + o] = __float2bfloat16_rn(y);
-            else
-              reinterpret_cast<float *>(Y)[t * O + o] = y;
-            if (acc_dbg) acc_dbg[t * O + o] = a;
-          }
-        }
-      }
+    // |acc| <= 127 * K < 2^22 for K <= 32768
+    if (!timed_out)
+      store_tile<BN>(trow, s_scale, o, O, t0, T, K <= 32768, Y, y_is_bf16, acc_dbg);
+  }
+  if (timed_out && err_flag) atomicOr(err_flag, SBN_FLAG_TIMEOUT);
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// 2:4 on the sparse tensor cores (tcgen05.mma.sp kind::i8).
+//
+// A is the compressed weight tile: per row the 64 kept codes of a 128-wide K block, expanded
+// to int8 lanes of 64 * t (no scatter: the kept codes are stored in order) into a 64-byte
+// swizzled K-major tile.  The 2-bit metadata of the packed format (i0 | i1 << 2 per group,
+// group 2h in the low nibble of byte h) is the sparse MMA's metadata as it stands: the TMA
+// brings the 128 x 16-byte tile into shared memory and tcgen05.cp moves it to 4 TMEM
+// columns; each K=64 MMA reads 2 of them.
+// ---------------------------------------------------------------------------------------
+
+template <int BN>
+struct SpCfg {
+  static constexpr int kKL = 128;                 // logical K per stage
+  static constexpr int kABytes = kBM * kKL / 2;   // compressed int8: 64 bytes per row
+  static constexpr int kBBytes = BN * kKL;        // activations: 128 bytes per token
+  static constexpr int kPBytes = kBM * 16 * 2;    // packed codes + metadata, 16 B each per row
+  static constexpr int kStageBytes = kABytes + kBBytes + kPBytes;
+  static constexpr int kBudget = 225 * 1024 - BN * 4 - 512;
+  static constexpr int kStages = (kBudget / kStageBytes) > 8 ? 8 : (kBudget / kStageBytes);
+  static constexpr int kMetaCol = BN < 32 ? 32 : BN;  // first TMEM column of the metadata
+  static constexpr int kNeedCols = kMetaCol + 4 * kStages;
+  static constexpr int kTmemCols = kNeedCols <= 32 ? 32 : kNeedCols <= 64 ? 64
+                                   : kNeedCols <= 128 ? 128 : kNeedCols <= 256 ? 256 : 512;
+  static constexpr uint32_t kTxBytes = kBBytes + kPBytes;
+  static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes +
+                                  (size_t)(3 * kStages + 1) * 8 + 16 + (size_t)BN * 4;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    k_gemm_sp24(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_c,
+                const __grid_constant__ CUtensorMap tmap_m, const float *__restrict__ absmax,
+                const float *__restrict__ gamma_eff, int64_t T, int64_t O, int64_t K,
+                void *__restrict__ Y, int y_is_bf16, int32_t *__restrict__ acc_dbg,
+                int32_t *err_flag) {
+  using Cfg = SpCfg<BN>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sB = smem;                        // 1024-aligned stages (128-byte swizzle)
+  uint8_t *sA = sB + S * Cfg::kBBytes;       // 512-aligned stages (64-byte swizzle)
+  uint8_t *sP = sA + S * Cfg::kABytes;       // packed codes [128][16] then metadata [128][16]
+  uint64_t *full_a = reinterpret_cast<uint64_t *>(sP + S * Cfg::kPBytes);
+  uint64_t *full_t = full_a + S;
+  uint64_t *empty = full_t + S;
+  uint64_t *done = empty + S;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+  float *s_scale = reinterpret_cast<float *>(tmem_slot + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t o0 = (int64_t)blockIdx.x * kBM;
+  const int64_t t0 = (int64_t)blockIdx.y * BN;
+  const int nkb = (int)((K + Cfg::kKL - 1) / Cfg::kKL);
+  bool timed_out = false;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      ptx::mbar_init(&full_a[s], 4);
+      ptx::mbar_init(&full_t[s], 1);
+      ptx::mbar_init(&empty[s], 1);
     }
+    ptx::mbar_init(done, 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 5) {
+    ptx::tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i < BN; i += kTcThreads) {
+    const int64_t t = t0 + i;
+    s_scale[i] = t < T ? rescale_factor(__ldg(gamma_eff), __ldg(absmax + t)) : 0.0f;
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < 4) {
+    // ---------------- compressed-weight expanders ----------------
+    const int r = threadIdx.x;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % S;
+      const uint32_t ph = (uint32_t)(kb / S) & 1u;
+      if ((kb >= S && !wait_phase(&empty[s], ph ^ 1u)) || !wait_phase(&full_t[s], ph)) {
+        timed_out = true;
+        break;
+      }
+      const uint4 cw = *reinterpret_cast<const uint4 *>(sP + s * Cfg::kPBytes + r * 16);
+      const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+      // Groups past the matrix (rows >= O, or the second half of the last block when
+      // K % 128 == 64) were zero-filled by the TMA; give them the valid index pair (0, 1)
+      // so the MMA never sees a malformed metadata nibble (their codes are zero anyway).
+      if (o0 + r >= O) {
+        *reinterpret_cast<uint4 *>(sP + s * Cfg::kPBytes + kBM * 16 + r * 16) =
+            make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+      } else if ((int64_t)kb * Cfg::kKL + 64 >= K) {
+        *reinterpret_cast<uint2 *>(sP + s * Cfg::kPBytes + kBM * 16 + r * 16 + 8) =
+            make_uint2(0x44444444u, 0x44444444u);
+      }
+      uint8_t *dst = sA + s * Cfg::kABytes + r * 64;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)  // 16 kept codes -> 16 int8 lanes, in order
+        *reinterpret_cast<uint4 *>(dst + ((c ^ ((r >> 1) & 3)) << 4)) =
+            make_uint4(w[c] & 0xC0C0C0C0u, (w[c] << 2) & 0xC0C0C0C0u,
+                       (w[c] << 4) & 0xC0C0C0C0u, (w[c] << 6) & 0xC0C0C0C0u);
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&full_a[s]);
+    }
+  } else if (warp == 4) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmap_x);
+      ptx::prefetch_tmap(&tmap_c);
+      ptx::prefetch_tmap(&tmap_m);
+      int issued = 0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (uint32_t)(kb / S) & 1u;
+        if (kb >= S && !wait_phase(&empty[s], ph ^ 1u)) {
+          timed_out = true;
+          break;
+        }
+        ptx::mbar_arrive_expect_tx(&full_t[s], Cfg::kTxBytes);
+        ptx::tma_load_2d(sB + s * Cfg::kBBytes, &tmap_x, &full_t[s], kb * Cfg::kKL, (int32_t)t0);
+        uint8_t *p = sP + s * Cfg::kPBytes;
+        ptx::tma_load_2d(p, &tmap_c, &full_t[s], kb * 16, (int32_t)o0);
+        ptx::tma_load_2d(p + kBM * 16, &tmap_m, &full_t[s], kb * 16, (int32_t)o0);
+        issued = kb + 1;
+      }
+      for (int kb = issued - S < 0 ? 0 : issued - S; kb < issued; ++kb)
+        if (!wait_phase(&full_t[kb % S], (uint32_t)(kb / S) & 1u)) timed_out = true;
+    }
+  } else {
+    // ---------------- metadata copy + sparse MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = ptx::idesc_i8_sparse(kBM, BN);
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (uint32_t)(kb / S) & 1u;
+        if (!wait_phase(&full_a[s], ph) || !wait_phase(&full_t[s], ph)) {
+          timed_out = true;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t e_col = tmem + Cfg::kMetaCol + 4 * s;
+        ptx::tmem_cp_128x128b(e_col, ptx::smem_desc_rows16(ptx::smem_u32(sP + s * Cfg::kPBytes +
+                                                                        kBM * 16)));
+        const uint32_t a_addr = ptx::smem_u32(sA + s * Cfg::kABytes);
+        const uint32_t b_addr = ptx::smem_u32(sB + s * Cfg::kBBytes);
+#pragma unroll
+        for (int k = 0; k < 2; ++k)  // logical K 64 per MMA: 32 bytes of A, 64 of B
+          ptx::mma_sp_i8(tmem, ptx::smem_desc_sw64(a_addr + 32 * k),
+                         ptx::smem_desc_sw128(b_addr + 64 * k), e_col + 2 * k, idesc,
+                         (kb | k) != 0);
+        ptx::mma_commit(&empty[s]);
+      }
+      ptx::mma_commit(done);
+    }
+  }
+
+  if (warp < 4) {
+    // ---------------- epilogue ----------------
+    __syncwarp();
+    if (!timed_out && !wait_phase(done, 0)) timed_out = true;
+    ptx::tc_fence_after();
+    const int64_t o = o0 + warp * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    // |acc| <= 127 * K < 2^22 for K <= 32768
+    if (!timed_out)
+      store_tile<BN>(trow, s_scale, o, O, t0, T, K <= 32768, Y, y_is_bf16, acc_dbg);
   }
   if (timed_out && err_flag) atomicOr(err_flag, SBN_FLAG_TIMEOUT);
   ptx::tc_fence_before();
@@ -312,14 +526,37 @@ static sbn_status gemm_tc_t(const int8_t *Xq, const float *absmax, const uint8_t
 }
 
 template <int BN>
+static sbn_status gemm_sp24_t(const int8_t *Xq, const float *absmax, const uint8_t *codes,
+                              const uint8_t *meta, const float *gamma_eff, int64_t T, int64_t O,
+                              int64_t K, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
+                              int32_t *acc_dbg, int32_t *err_flag, cudaStream_t st) {
+  using Cfg = SpCfg<BN>;
+  CUtensorMap tx, tc, tm;
+  if (!encode_u8(&tx, Xq, K, T, K, Cfg::kKL, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_u8(&tc, codes, K / 8, O, ldc, 16, kBM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_u8(&tm, meta, K / 8, O, ldm, 16, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return SBN_ERR_CUDA;
+  auto kern = k_gemm_sp24<BN>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::kSmem) !=
+      cudaSuccess)
+    return SBN_ERR_CUDA;
+  dim3 grid((unsigned)((O + kBM - 1) / kBM), (unsigned)((T + BN - 1) / BN));
+  kern<<<grid, kTcThreads, Cfg::kSmem, st>>>(tx, tc, tm, absmax, gamma_eff, T, O, K, Y, y_is_bf16,
+                                             acc_dbg, err_flag);
+  SBN_LAUNCH_CHECK();
+  return SBN_OK;
+}
+
+template <int BN>
 static sbn_status gemm_tc_bn(bool compact, const int8_t *Xq, const float *absmax,
                              const uint8_t *codes, const uint8_t *meta, const float *gamma_eff,
                              int64_t T, int64_t O, int64_t K, int64_t ldc, int64_t ldm, void *Y,
                              int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag, cudaStream_t st) {
-  return compact ? gemm_tc_t<BN, true>(Xq, absmax, codes, meta, gamma_eff, T, O, K, ldc, ldm, Y,
-                                       y_is_bf16, acc_dbg, err_flag, st)
-                 : gemm_tc_t<BN, false>(Xq, absmax, codes, meta, gamma_eff, T, O, K, ldc, ldm, Y,
-                                        y_is_bf16, acc_dbg, err_flag, st);
+  if (compact)
+    return gemm_sp24_t<BN>(Xq, absmax, codes, meta, gamma_eff, T, O, K, ldc, ldm, Y, y_is_bf16,
+                           acc_dbg, err_flag, st);
+  return gemm_tc_t<BN, false>(Xq, absmax, codes, meta, gamma_eff, T, O, K, ldc, ldm, Y,
+                              y_is_bf16, acc_dbg, err_flag, st);
 }
 
 sbn_status launch_gemm_tc(const int8_t *Xq, const float *absmax, const uint8_t *codes,

@@ -5,8 +5,7 @@
 // multiplications become additions and subtractions).  The int32 sum is divided by 64
 // exactly at the end; y = acc * fp32(fp32(g * s) / 127).
 //
-// Work split: 8 lanes per output row (a warp owns 4 rows), lane i of a row takes the
-// 64-weight chunks i, i+8, ...; the activations of all tokens sit in shared memory.
+// Work split: one warp per output row; see k_gemv.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -21,106 +20,151 @@ __device__ __forceinline__ uint32_t pair_selector(uint32_t mb) {
          ((((mb >> 6) & 3u) + 4u) << 12);
 }
 
-template <int T, bool kCompact>
+// One warp per output row: lane l takes the 64-weight chunks l, l+32, ..., at most CPL of
+// them, and issues every chunk load of the row before any arithmetic.  When T * CPL <= 4
+// the lane's activation words stay in registers for the whole kernel (the lane always sees
+// the same chunks); otherwise they are read from shared memory.
+template <int T, int CPL, bool kCompact>
 __global__ void __launch_bounds__(kGvThreads)
     k_gemv(const int8_t *__restrict__ Xq, const float *__restrict__ absmax,
            const uint8_t *__restrict__ codes, const uint8_t *__restrict__ meta,
            const float *__restrict__ gamma_eff, int64_t out, int64_t in, int64_t ldc,
            int64_t ldm, void *__restrict__ Y, int y_is_bf16, int32_t *__restrict__ acc_dbg) {
-  extern __shared__ __align__(16) uint32_t xs[];  // [T][in/4] int8 words
+  // registers hold the activations only when one pass covers the row (CPL chosen >= the
+  // chunks per lane, which the launcher guarantees for CPL <= 4)
+  constexpr bool kXReg = T * CPL <= 4;
+  extern __shared__ __align__(16) uint32_t xs[];  // [T][in/4] int8 words (shared mode)
   const int64_t kw = in / 4;
-  for (int64_t i = threadIdx.x; i < T * kw / 4; i += blockDim.x)
-    reinterpret_cast<uint4 *>(xs)[i] = __ldg(reinterpret_cast<const uint4 *>(Xq) + i);
-  __syncthreads();
-
   const int lane = threadIdx.x & 31;
-  const int sub = lane & 7;
-  const int64_t nchunks = in / 64;
+  const int nchunks = (int)(in / 64);
+  uint32_t xr[kXReg ? T * CPL * 16 : 1];
+  if constexpr (kXReg) {
+#pragma unroll
+    for (int t = 0; t < T; ++t)
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) {
+        const int c = lane + 32 * i;
+        const uint4 *src = reinterpret_cast<const uint4 *>(Xq + t * in + (int64_t)c * 64);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 x4 = c < nchunks ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
+          uint32_t *d = xr + (t * CPL + i) * 16 + 4 * v;
+          d[0] = x4.x;
+          d[1] = x4.y;
+          d[2] = x4.z;
+          d[3] = x4.w;
+        }
+      }
+  } else {
+    for (int64_t i = threadIdx.x; i < T * kw / 4; i += blockDim.x)
+      reinterpret_cast<uint4 *>(xs)[i] = __ldg(reinterpret_cast<const uint4 *>(Xq) + i);
+    __syncthreads();
+  }
+  auto xword = [&](int t, int i, int c, int word) -> uint32_t {
+    if constexpr (kXReg)
+      return xr[(t * CPL + i) * 16 + word];
+    else
+      return xs[t * kw + (int64_t)c * 16 + word];
+  };
+
   const float g = __ldg(gamma_eff);
-  const int64_t rows_per_pass = (int64_t)gridDim.x * (blockDim.x / 8);
-  // all lanes of a warp iterate together (shuffles below); rows past the end do no loads
-  for (int64_t row0 = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5) * 4; row0 < out;
-       row0 += rows_per_pass) {
-    const int64_t row = row0 + (lane >> 3);
-    const bool valid = row < out;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  // the next row's first chunk is requested before the current row is reduced
+  for (int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < out;
+       row += nwarps) {
+    if (row + nwarps < out && lane * 16 < ldc)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(codes + (row + nwarps) * ldc + lane * 16));
     int acc[T];
 #pragma unroll
     for (int t = 0; t < T; ++t) acc[t] = 0;
-    if (valid) {
-      if constexpr (!kCompact) {
-        const uint4 *crow = reinterpret_cast<const uint4 *>(codes + row * ldc);
-        for (int64_t c = sub; c < nchunks; c += 8) {
-          uint4 cw = __ldg(crow + c);  // 64 positions
-          uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
+    for (int c0 = 0; c0 < nchunks; c0 += 32 * CPL) {  // one pass unless K > 2048 * CPL
+    if constexpr (!kCompact) {
+      const uint4 *crow = reinterpret_cast<const uint4 *>(codes + row * ldc);
+      uint4 cw[CPL];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+      for (int i = 0; i < CPL; ++i)
+        cw[i] = c0 + lane + 32 * i < nchunks ? __ldg(crow + c0 + lane + 32 * i)
+                                             : make_uint4(0, 0, 0, 0);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              int z = (int)((w4[q] << (2 * j)) & 0xC0C0C0C0u);
+      for (int i = 0; i < CPL; ++i) {
+        const int c = c0 + lane + 32 * i;
+        if (c >= nchunks) continue;
+        const uint32_t w4[4] = {cw[i].x, cw[i].y, cw[i].z, cw[i].w};
 #pragma unroll
-              for (int t = 0; t < T; ++t)
-                acc[t] = __dp4a(z, (int)xs[t * kw + c * 16 + q * 4 + j], acc[t]);
-            }
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int z = (int)((w4[q] << (2 * j)) & 0xC0C0C0C0u);
+#pragma unroll
+            for (int t = 0; t < T; ++t) acc[t] = __dp4a(z, (int)xword(t, i, c, q * 4 + j), acc[t]);
           }
-        }
-      } else {
-        const uint2 *crow = reinterpret_cast<const uint2 *>(codes + row * ldc);
-        const uint2 *mrow = reinterpret_cast<const uint2 *>(meta + row * ldm);
-        for (int64_t c = sub; c < nchunks; c += 8) {
-          uint2 cw = __ldg(crow + c);  // 32 stored codes = 64 positions
-          uint2 mw = __ldg(mrow + c);  // 16 groups
-          uint32_t w2[2] = {cw.x, cw.y}, m2[2] = {mw.x, mw.y};
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              int z = (int)((w2[q] << (2 * j)) & 0xC0C0C0C0u);
-              uint32_t sel = pair_selector((m2[q] >> (8 * j)) & 0xffu);
-              const int64_t xw = c * 16 + q * 8 + 2 * j;  // x words of the two groups
-#pragma unroll
-              for (int t = 0; t < T; ++t) {
-                uint32_t xk = __byte_perm(xs[t * kw + xw], xs[t * kw + xw + 1], sel);
-                acc[t] = __dp4a(z, (int)xk, acc[t]);
-              }
-            }
-          }
-        }
       }
+    } else {
+      const uint2 *crow = reinterpret_cast<const uint2 *>(codes + row * ldc);
+      const uint2 *mrow = reinterpret_cast<const uint2 *>(meta + row * ldm);
+      uint2 cw[CPL], mw[CPL];
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) {
+        const bool ok = c0 + lane + 32 * i < nchunks;
+        cw[i] = ok ? __ldg(crow + c0 + lane + 32 * i) : make_uint2(0, 0);
+        mw[i] = ok ? __ldg(mrow + c0 + lane + 32 * i) : make_uint2(0, 0);
+      }
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) {
+        const int c = c0 + lane + 32 * i;
+        if (c >= nchunks) continue;
+        const uint32_t w2[2] = {cw[i].x, cw[i].y}, m2[2] = {mw[i].x, mw[i].y};
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int z = (int)((w2[q] << (2 * j)) & 0xC0C0C0C0u);
+            const uint32_t sel = pair_selector((m2[q] >> (8 * j)) & 0xffu);
+            const int xw = q * 8 + 2 * j;  // x words of the two groups
+#pragma unroll
+            for (int t = 0; t < T; ++t) {
+              const uint32_t xk = __byte_perm(xword(t, i, c, xw), xword(t, i, c, xw + 1), sel);
+              acc[t] = __dp4a(z, (int)xk, acc[t]);
+            }
+          }
+      }
+    }
     }
 #pragma unroll
     for (int t = 0; t < T; ++t) {
-      acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 1);
-      acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 2);
-      acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 4);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
     }
-    if (valid && sub < T) {
-      // lane `sub` writes token `sub` (T <= 8)
+    if (lane < T) {
+      // lane t writes token t
       int a = 0;
 #pragma unroll
       for (int t = 0; t < T; ++t)
-        if (t == sub) a = acc[t];
+        if (t == lane) a = acc[t];
       a >>= 6;  // the code lanes carry 64 * t; the sum is an exact multiple of 64
-      const float y = __fmul_rn((float)a, rescale_factor(g, __ldg(absmax + sub)));
+      const float y = __fmul_rn((float)a, rescale_factor(g, __ldg(absmax + lane)));
       if (y_is_bf16)
-        reinterpret_cast<__nv_bfloat16 *>(Y)[sub * out + row] = __float2bfloat16_rn(y);
+        reinterpret_cast<__nv_bfloat16 *>(Y)[lane * out + row] = __float2bfloat16_rn(y);
       else
-        reinterpret_cast<float *>(Y)[sub * out + row] = y;
-      if (acc_dbg) acc_dbg[sub * out + row] = a;
+        reinterpret_cast<float *>(Y)[lane * out + row] = y;
+      if (acc_dbg) acc_dbg[lane * out + row] = a;
     }
   }
 }
 
-template <int T>
-static sbn_status gemv_t(const int8_t *Xq, const float *absmax, const uint8_t *codes,
-                         const uint8_t *meta, const float *gamma_eff, int64_t out, int64_t in,
-                         bool compact, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
-                         int32_t *acc_dbg, cudaStream_t st) {
-  const size_t smem = (size_t)T * (size_t)in;
-  const int64_t rows_per_cta = kGvThreads / 8;
+template <int T, int CPL>
+static sbn_status gemv_tc(const int8_t *Xq, const float *absmax, const uint8_t *codes,
+                          const uint8_t *meta, const float *gamma_eff, int64_t out, int64_t in,
+                          bool compact, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
+                          int32_t *acc_dbg, cudaStream_t st) {
+  constexpr bool kXReg = T * CPL <= 4;
+  const size_t smem = kXReg ? 0 : (size_t)T * (size_t)in;
+  const int64_t rows_per_cta = kGvThreads / 32;
   int64_t grid = (out + rows_per_cta - 1) / rows_per_cta;
-  const int64_t cap = (int64_t)num_sms() * 8;
+  // persistent grid: activations are loaded once per warp (registers) or per CTA (shared)
+  const int64_t cap = (int64_t)num_sms() * (kXReg ? 4 : 2);
   if (grid > cap) grid = cap;
-  auto kern = compact ? k_gemv<T, true> : k_gemv<T, false>;
+  auto kern = compact ? k_gemv<T, CPL, true> : k_gemv<T, CPL, false>;
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
           cudaSuccess)
@@ -129,6 +173,25 @@ static sbn_status gemv_t(const int8_t *Xq, const float *absmax, const uint8_t *c
                                                  ldc, ldm, Y, y_is_bf16, acc_dbg);
   SBN_LAUNCH_CHECK();
   return SBN_OK;
+}
+
+template <int T>
+static sbn_status gemv_t(const int8_t *Xq, const float *absmax, const uint8_t *codes,
+                         const uint8_t *meta, const float *gamma_eff, int64_t out, int64_t in,
+                         bool compact, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
+                         int32_t *acc_dbg, cudaStream_t st) {
+  const int64_t cpl = (in / 64 + 31) / 32;
+  if (cpl <= 1)
+    return gemv_tc<T, 1>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
+                         y_is_bf16, acc_dbg, st);
+  if (cpl <= 2)
+    return gemv_tc<T, 2>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
+                         y_is_bf16, acc_dbg, st);
+  if (cpl <= 4)
+    return gemv_tc<T, 4>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
+                         y_is_bf16, acc_dbg, st);
+  return gemv_tc<T, 8>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
+                       y_is_bf16, acc_dbg, st);
 }
 
 sbn_status launch_gemv(const int8_t *Xq, const float *absmax, const uint8_t *codes,

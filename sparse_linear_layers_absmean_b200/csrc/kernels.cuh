@@ -22,6 +22,36 @@ struct PackWorkspace {
 
 int num_sms();
 
+// Exact b / d for b < 2^25 and 1 <= d <= 2^11: with L = ceil(log2 d) and
+// M = ceil(2^(31+L) / d) < 2^32, b / d == (b * M) >> (31 + L): the error term
+// b * (M*d - 2^(31+L)) stays below 2^(31+L) because b < 2^31.
+struct FastDiv {
+  uint32_t mul, shift;  // shift = L - 1, or 0xffffffff for d == 1
+};
+
+__device__ __forceinline__ uint32_t fast_div(uint32_t b, FastDiv f) {
+  return f.shift == 0xffffffffu ? b : (__umulhi(b, f.mul) >> f.shift);
+}
+
+FastDiv make_fast_div(uint32_t d);
+
+// Arguments of the 6:8 and 2:4 quant/mask/pack kernels (64-weight blocks, K % 64 == 0).
+struct FastPackArgs {
+  const uint4 *W;
+  int64_t nblocks;
+  uint32_t bpr;  // blocks per row
+  FastDiv div_bpr;
+  const PackWorkspace *ws;
+  uint8_t *codes;
+  int64_t ldc, codes_row_bytes;
+  uint8_t *meta;
+  int64_t ldm, meta_row_bytes;
+  int8_t *dense_dbg;
+};
+
+__global__ void k_qmp_6of8(const FastPackArgs a);
+__global__ void k_qmp_2of4(const FastPackArgs a);
+
 sbn_status launch_pack(const void *W, int64_t out, int64_t in, int n, int m, float eps,
                        uint8_t *codes, int64_t ldc, int64_t crow, uint8_t *meta, int64_t ldm,
                        int64_t mrow, float *gamma_eff, PackWorkspace *ws, int8_t *dense_dbg,

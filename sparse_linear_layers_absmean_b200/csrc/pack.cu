@@ -39,23 +39,22 @@ __global__ void __launch_bounds__(256) k_abs_sum(const uint4 *__restrict__ W, in
                                                  int64_t n, float eps, PackWorkspace *ws,
                                                  float *gamma_eff, int32_t *err_flag) {
   unsigned long long acc = 0;
-  uint32_t mx_all = 0, mx_fin = 0;
+  uint32_t mx = 0;  // largest magnitude bits seen, per 16-bit half
   auto consume = [&](const uint4 &v) {
     const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const uint32_t a = w4[q] & 0x7fff7fffu;  // |W| of both halves
-      mx_all = __vmaxu2(mx_all, a);
-      const uint32_t nonfin = __vcmpgeu2(a, 0x7f807f80u);
-      mx_fin = __vmaxu2(mx_fin, a & ~nonfin);
+      asm("max.u16x2 %0, %0, %1;" : "+r"(mx) : "r"(a));
       // |W| * 2^24 is exact in fp32; the conversion truncates toward zero.
       const float lo = __fmul_rn(__uint_as_float(a << 16), 16777216.0f);
       const float hi = __fmul_rn(__uint_as_float(a & 0xffff0000u), 16777216.0f);
-      acc += (unsigned long long)__float2uint_rz(lo) + (unsigned long long)__float2uint_rz(hi);
+      acc += (unsigned long long)__float2uint_rz(lo) + __float2uint_rz(hi);
     }
   };
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  int64_t i = i0;
   for (; i + 3 * stride < nvec; i += 4 * stride) {  // four 16-byte loads in flight
     const uint4 v0 = __ldg(W + i), v1 = __ldg(W + i + stride), v2 = __ldg(W + i + 2 * stride),
                 v3 = __ldg(W + i + 3 * stride);
@@ -65,13 +64,28 @@ __global__ void __launch_bounds__(256) k_abs_sum(const uint4 *__restrict__ W, in
     consume(v3);
   }
   for (; i < nvec; i += stride) consume(__ldg(W + i));
+  // Rare path: some |W| >= 256 (or NaN/Inf).  Re-read this thread's weights to tell the
+  // two error kinds apart.
+  uint32_t mx_all = 0, mx_fin = 0;
+  if (max(mx & 0xffffu, mx >> 16) >= kBf16Mag256Bits) {
+    for (int64_t j = i0; j < nvec; j += stride) {
+      const uint4 v = __ldg(W + j);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      for (int q = 0; q < 4; ++q)
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t m = (w4[q] >> (16 * h)) & 0x7fffu;
+          mx_all = max(mx_all, m);
+          if (m < kBf16InfBits) mx_fin = max(mx_fin, m);
+        }
+    }
+  }
   __shared__ unsigned long long s_sum[8];
   __shared__ uint32_t s_all[8], s_fin[8];
   __shared__ int s_last;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   acc = warp_sum_u64(acc);
-  uint32_t ma = warp_max_u32(max(mx_all & 0xffffu, mx_all >> 16));
-  uint32_t mf = warp_max_u32(max(mx_fin & 0xffffu, mx_fin >> 16));
+  uint32_t ma = warp_max_u32(mx_all);
+  uint32_t mf = warp_max_u32(mx_fin);
   if (lane == 0) {
     s_sum[warp] = acc;
     s_all[warp] = ma;
@@ -182,17 +196,6 @@ __device__ __forceinline__ uint32_t spread4_to_bytes(uint32_t x) {
 constexpr unsigned long long kPairNibbleLut =
     (4ull << (4 * 0x3)) | (8ull << (4 * 0x5)) | (9ull << (4 * 0x6)) | (12ull << (4 * 0x9)) |
     (13ull << (4 * 0xA)) | (14ull << (4 * 0xC));
-
-// Exact b / d for b < 2^25 and 1 <= d <= 2^11: with L = ceil(log2 d) and
-// M = ceil(2^(31+L) / d) < 2^32, b / d == (b * M) >> (31 + L) (the error term b*(M*d - 2^(31+L))
-// stays below 2^(31+L) because b < 2^31).
-struct FastDiv {
-  uint32_t mul, shift;  // shift = L - 1, or 0xffffffff for d == 1
-};
-
-__device__ __forceinline__ uint32_t fast_div(uint32_t b, FastDiv f) {
-  return f.shift == 0xffffffffu ? b : (__umulhi(b, f.mul) >> f.shift);
-}
 
 template <int N, int M>
 struct QmpArgs {
@@ -330,7 +333,7 @@ int num_sms() {
   return sms;
 }
 
-static FastDiv make_fast_div(uint32_t d) {
+FastDiv make_fast_div(uint32_t d) {
   FastDiv f;
   if (d == 1) {
     f.mul = 0;
@@ -366,7 +369,7 @@ sbn_status launch_pack(const void *W, int64_t out, int64_t in, int n, int m, flo
   const int64_t nel = out * in;
   const int64_t nvec = nel / 8;
   int64_t grid = (nvec + 256 * 4 - 1) / (256 * 4);
-  const int64_t cap = (int64_t)num_sms() * 4;
+  const int64_t cap = (int64_t)num_sms() * 7;  // ~56 resident warps per SM
   if (grid > cap) grid = cap;
   if (grid > kPackMaxParts) grid = kPackMaxParts;
   if (grid < 1) grid = 1;
@@ -375,6 +378,20 @@ sbn_status launch_pack(const void *W, int64_t out, int64_t in, int n, int m, flo
   SBN_LAUNCH_CHECK();
   const uint4 *W4 = reinterpret_cast<const uint4 *>(W);
   const int64_t nblocks = nel / 64, bpr = in / 64;
+  if ((n == 6 && m == 8) || (n == 2 && m == 4)) {
+    FastPackArgs fa{W4,   nblocks, (uint32_t)bpr, make_fast_div((uint32_t)bpr), ws,   codes,
+                    ldc,  crow,    meta,          ldm,                          mrow, dense_dbg};
+    int64_t g = (nblocks + 63) / 64;  // 8 warps x 8 blocks per CTA pass
+    const int64_t capq = (int64_t)num_sms() * 8;
+    if (g > capq) g = capq;
+    if (g < 1) g = 1;
+    if (n == 6)
+      k_qmp_6of8<<<(unsigned)g, 256, 0, st>>>(fa);
+    else
+      k_qmp_2of4<<<(unsigned)g, 256, 0, st>>>(fa);
+    SBN_LAUNCH_CHECK();
+    return SBN_OK;
+  }
 #define SBN_QMP(NN, MM)                                                                    \
   case (NN * 16 + MM):                                                                     \
     launch_qmp<NN, MM>(W4, nblocks, bpr, ws, codes, ldc, crow, meta, ldm, mrow, dense_dbg, \
