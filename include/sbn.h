@@ -103,11 +103,9 @@ SBN_API sbn_status sbn_linear_ref_dims(int64_t out, int64_t in, int n, int m, sb
  *              gamma = fp32( fp64(S) / (fp64(out * in) * 2^24) ),
  *              S = sum over all weights of trunc(|W| * 2^24)  (exact 64-bit integer sum,
  *              so the result does not depend on the order of summation).
- *   workspace  dims.pack_workspace_bytes of device memory, zero-filled before its first
- *              use.  It holds per-CTA partial sums and an arrival counter; every call
- *              returns the counter to zero, so the same workspace can be reused by later
- *              calls without clearing it again.  Calls that share one workspace must not
- *              run concurrently.
+ *   workspace  dims.pack_workspace_bytes of device memory for the reduction's per-CTA
+ *              partial sums.  Its contents need no initialisation and may be reused by
+ *              later calls; calls that share one workspace must not run concurrently.
  *   dense_dbg  optional int8 [out, in]: the masked ternary matrix (NULL to skip).
  *   err_flag   optional: SBN_FLAG_W_NONFINITE / SBN_FLAG_W_RANGE.
  * out * in must be below 2^31.

@@ -152,7 +152,7 @@ class PackedWeights(NamedTuple):
 
 
 def new_workspace(out: int, in_: int, n: int, m: int, device="cuda") -> torch.Tensor:
-    """Zero-filled pack workspace (reusable by later calls on the same stream)."""
+    """Pack workspace (reusable by later calls on the same stream)."""
     d = sbn_linear_ref_dims(out, in_, n, m)
     return torch.zeros(d.pack_workspace_bytes, dtype=torch.uint8, device=device)
 

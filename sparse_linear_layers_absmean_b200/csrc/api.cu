@@ -111,7 +111,7 @@ sbn_status sbn_linear(const int8_t *Xq, const float *absmax, const uint8_t *code
       (reinterpret_cast<uintptr_t>(gamma_eff) & 3u) || (reinterpret_cast<uintptr_t>(err_flag) & 3u))
     return SBN_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (tokens <= sbn::kGemvMaxTokens && tokens * in <= sbn::kGemvMaxSmemBytes)
+  if (tokens <= sbn::kGemvMaxTokens)
     return sbn::launch_gemv(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, n, m, d.codes_ld,
                             d.meta_ld, Y, y_is_bf16, acc_dbg, s);
   return sbn::launch_gemm_tc(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, n, m,

@@ -62,8 +62,24 @@ __device__ __forceinline__ void store_tile(uint32_t trow, const float *s_scale, 
   for (int cb = 0; cb < BN; cb += 2 * kCols) {
     uint32_t va[32], vb[32];
     if constexpr (kCols == 32) {
-      ptx::tmem_ld_32(trow + cb, va);
-      if (cb + 32 < BN) ptx::tmem_ld_32(trow + cb + 32, vb);
+      // BN is a multiple of 16: a chunk of 16 columns at the end is loaded at its own width,
+      // so no load reads past the tile's accumulator columns
+      if (BN - cb >= 32) {
+        ptx::tmem_ld_32(trow + cb, va);
+      } else {
+        uint32_t v16[16];
+        ptx::tmem_ld_16(trow + cb, v16);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) va[i] = v16[i];
+      }
+      if (BN - cb - 32 >= 32) {
+        ptx::tmem_ld_32(trow + cb + 32, vb);
+      } else if (BN - cb - 32 > 0) {
+        uint32_t v16[16];
+        ptx::tmem_ld_16(trow + cb + 32, v16);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) vb[i] = v16[i];
+      }
     } else {
       uint32_t v16[16];
       ptx::tmem_ld_16(trow + cb, v16);
@@ -76,7 +92,8 @@ __device__ __forceinline__ void store_tile(uint32_t trow, const float *s_scale, 
       const int c0 = cb + half * kCols;
       if (c0 >= BN || !row_ok) continue;
       const uint32_t *v = half ? vb : va;
-      const int64_t nt = T - (t0 + c0);  // columns of this chunk that are real tokens
+      // columns of this chunk that are real tokens of this tile
+      const int64_t nt = min(T - (t0 + c0), (int64_t)(BN - c0));
       float *yf = reinterpret_cast<float *>(Y) + (t0 + c0) * O + o;
       __nv_bfloat16 *yb = reinterpret_cast<__nv_bfloat16 *>(Y) + (t0 + c0) * O + o;
 #pragma unroll
@@ -474,6 +491,259 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------------
+// Persistent 2:4 kernel for large token counts.  Each CTA loops over output tiles
+// (128 weight rows x BN tokens); the TMEM holds two accumulators so that four dedicated
+// epilogue warps drain tile i while the MMA already accumulates tile i+1.
+//   warps 0-3  expanders (compressed A tiles), warp 4 TMA, warp 5 TMEM + MMA issue,
+//   warps 6-9  epilogue (warp w reads accumulator lanes 32*(w%4) .. +31).
+// Every wait is bounded; a timeout anywhere raises a shared abort flag that ends all loops.
+// ---------------------------------------------------------------------------------------
+
+constexpr int kPsThreads = 320;
+
+template <int BN>
+struct PsCfg {
+  static constexpr int kKL = 128;
+  static constexpr int kABytes = kBM * kKL / 2;
+  static constexpr int kBBytes = BN * kKL;
+  static constexpr int kPBytes = kBM * 16 * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes + kPBytes;
+  static constexpr int kBudget = 225 * 1024 - BN * 4 - 1024;
+  static constexpr int kStages = (kBudget / kStageBytes) > 8 ? 8 : (kBudget / kStageBytes);
+  // accumulator b at TMEM columns 256 * b .. 256 * b + BN - 1; each stage's 4 metadata
+  // columns sit in the gaps after the accumulators
+  static constexpr int kAccStride = 256;
+  static constexpr int kGap = (256 - BN) / 4;  // metadata slots after one accumulator
+  static_assert(BN <= 256 && BN % 16 == 0, "tile width");
+  static_assert(2 * kGap >= kStages, "two accumulators and the metadata must fit in TMEM");
+  static constexpr int kTmemCols = 512;
+  __device__ static constexpr uint32_t meta_col(int s) {
+    return s < kGap ? (uint32_t)(BN + 4 * s) : (uint32_t)(kAccStride + BN + 4 * (s - kGap));
+  }
+  static constexpr uint32_t kTxBytes = kBBytes + kPBytes;
+  static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes +
+                                  (size_t)(3 * kStages + 4 + 1) * 8 + 32 + (size_t)BN * 4;
+};
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    for (int i = 0; i < 64; ++i)
+      if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_ns() - t0 > kWaitNs) {
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// bar.red.or over the `n` threads of named barrier `id`: every participant learns whether
+// any of them passed true.
+__device__ __forceinline__ bool bar_any(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kPsThreads, 1)
+    k_gemm_sp24_persist(const __grid_constant__ CUtensorMap tmap_x,
+                        const __grid_constant__ CUtensorMap tmap_c,
+                        const __grid_constant__ CUtensorMap tmap_m,
+                        const float *__restrict__ absmax, const float *__restrict__ gamma_eff,
+                        int64_t T, int64_t O, int64_t K, void *__restrict__ Y, int y_is_bf16,
+                        int32_t *__restrict__ acc_dbg, int32_t *err_flag) {
+  using Cfg = PsCfg<BN>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sB = smem;
+  uint8_t *sA = sB + S * Cfg::kBBytes;
+  uint8_t *sP = sA + S * Cfg::kABytes;
+  uint64_t *full_a = reinterpret_cast<uint64_t *>(sP + S * Cfg::kPBytes);
+  uint64_t *full_t = full_a + S;
+  uint64_t *empty = full_t + S;
+  uint64_t *acc_full = empty + S;   // [2]
+  uint64_t *acc_empty = acc_full + 2;  // [2]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+  volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_slot + 2);
+  float *s_scale = reinterpret_cast<float *>(tmem_slot + 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nkb = (int)((K + Cfg::kKL - 1) / Cfg::kKL);
+  const int64_t n_o = (O + kBM - 1) / kBM, n_t = (T + BN - 1) / BN;
+  const int64_t ntiles = n_o * n_t;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      ptx::mbar_init(&full_a[s], 4);
+      ptx::mbar_init(&full_t[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&acc_full[b], 1);
+      ptx::mbar_init(&acc_empty[b], 4);
+    }
+    *s_abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 5) {
+    ptx::tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < 4) {
+    // ---------------- compressed-weight expanders ----------------
+    const int r = threadIdx.x;
+    int64_t kg = 0;
+    for (int64_t tile = blockIdx.x;
+         tile < ntiles && !__any_sync(0xffffffffu, *s_abort != 0); tile += gridDim.x) {
+      const int64_t o0 = (tile % n_o) * kBM;
+      for (int kb = 0; kb < nkb; ++kb, ++kg) {
+        const int s = (int)(kg % S);
+        const uint32_t ph = (uint32_t)(kg / S) & 1u;
+        const bool ok = (kg < S || wait_or_abort(&empty[s], ph ^ 1u, s_abort)) &&
+                        wait_or_abort(&full_t[s], ph, s_abort);
+        if (!__all_sync(0xffffffffu, ok)) break;  // the whole warp leaves together
+        const uint4 cw = *reinterpret_cast<const uint4 *>(sP + s * Cfg::kPBytes + r * 16);
+        const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+        if (o0 + r >= O) {
+          *reinterpret_cast<uint4 *>(sP + s * Cfg::kPBytes + kBM * 16 + r * 16) =
+              make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+        } else if ((int64_t)kb * Cfg::kKL + 64 >= K) {
+          *reinterpret_cast<uint2 *>(sP + s * Cfg::kPBytes + kBM * 16 + r * 16 + 8) =
+              make_uint2(0x44444444u, 0x44444444u);
+        }
+        uint8_t *dst = sA + s * Cfg::kABytes + r * 64;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4 *>(dst + ((c ^ ((r >> 1) & 3)) << 4)) =
+              make_uint4(w[c] & 0xC0C0C0C0u, (w[c] << 2) & 0xC0C0C0C0u,
+                         (w[c] << 4) & 0xC0C0C0C0u, (w[c] << 6) & 0xC0C0C0C0u);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&full_a[s]);
+      }
+    }
+  } else if (warp == 4) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmap_x);
+      ptx::prefetch_tmap(&tmap_c);
+      ptx::prefetch_tmap(&tmap_m);
+      int64_t kg = 0, issued = 0;
+      for (int64_t tile = blockIdx.x; tile < ntiles && !*s_abort; tile += gridDim.x) {
+        const int64_t o0 = (tile % n_o) * kBM, t0 = (tile / n_o) * BN;
+        for (int kb = 0; kb < nkb; ++kb, ++kg) {
+          const int s = (int)(kg % S);
+          const uint32_t ph = (uint32_t)(kg / S) & 1u;
+          if (kg >= S && !wait_or_abort(&empty[s], ph ^ 1u, s_abort)) break;
+          ptx::mbar_arrive_expect_tx(&full_t[s], Cfg::kTxBytes);
+          ptx::tma_load_2d(sB + s * Cfg::kBBytes, &tmap_x, &full_t[s], kb * Cfg::kKL,
+                           (int32_t)t0);
+          uint8_t *p = sP + s * Cfg::kPBytes;
+          ptx::tma_load_2d(p, &tmap_c, &full_t[s], kb * 16, (int32_t)o0);
+          ptx::tma_load_2d(p + kBM * 16, &tmap_m, &full_t[s], kb * 16, (int32_t)o0);
+          issued = kg + 1;
+        }
+      }
+      // every issued copy lands before the CTA can exit (bounded, even after an abort)
+      for (int64_t q = issued - S < 0 ? 0 : issued - S; q < issued; ++q)
+        if (!wait_phase(&full_t[q % S], (uint32_t)(q / S) & 1u)) *s_abort = 1;
+    }
+  } else if (warp == 5) {
+    // ---------------- metadata copy + sparse MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = ptx::idesc_i8_sparse(kBM, BN);
+      int64_t kg = 0;
+      int i = 0;
+      for (int64_t tile = blockIdx.x; tile < ntiles && !*s_abort; tile += gridDim.x, ++i) {
+        const int buf = i & 1;
+        if (i >= 2 && !wait_or_abort(&acc_empty[buf], ((uint32_t)(i >> 1) & 1u) ^ 1u, s_abort))
+          break;
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(buf * Cfg::kAccStride);
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb, ++kg) {
+          const int s = (int)(kg % S);
+          const uint32_t ph = (uint32_t)(kg / S) & 1u;
+          if (!wait_or_abort(&full_a[s], ph, s_abort) || !wait_or_abort(&full_t[s], ph, s_abort)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t e_col = tmem + Cfg::meta_col(s);
+          ptx::tmem_cp_128x128b(
+              e_col, ptx::smem_desc_rows16(ptx::smem_u32(sP + s * Cfg::kPBytes + kBM * 16)));
+          const uint32_t a_addr = ptx::smem_u32(sA + s * Cfg::kABytes);
+          const uint32_t b_addr = ptx::smem_u32(sB + s * Cfg::kBBytes);
+#pragma unroll
+          for (int k = 0; k < 2; ++k)
+            ptx::mma_sp_i8(d_tmem, ptx::smem_desc_sw64(a_addr + 32 * k),
+                           ptx::smem_desc_sw128(b_addr + 64 * k), e_col + 2 * k, idesc,
+                           (kb | k) != 0);
+          ptx::mma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        ptx::mma_commit(&acc_full[buf]);
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 6-9) ----------------
+    const int q = warp & 3;  // TMEM lane quadrant this warp may read
+    const int et = threadIdx.x - 6 * 32;  // 0..127
+    const float g = __ldg(gamma_eff);
+    bool failed = false;
+    int i = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+      const int buf = i & 1;
+      const int64_t o0 = (tile % n_o) * kBM, t0 = (tile / n_o) * BN;
+      // all four warps are done with the previous tile's scales, and all of them stop
+      // together if any wait of the previous tile gave up
+      if (bar_any(1, 128, failed)) break;
+      for (int c = et; c < BN; c += 128) {
+        const int64_t t = t0 + c;
+        s_scale[c] = t < T ? rescale_factor(g, __ldg(absmax + t)) : 0.0f;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      failed = !__all_sync(0xffffffffu, !*s_abort && wait_or_abort(&acc_full[buf],
+                                                                   (uint32_t)(i >> 1) & 1u,
+                                                                   s_abort));
+      ptx::tc_fence_after();
+      if (!failed) {
+        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * Cfg::kAccStride);
+        store_tile<BN>(trow, s_scale, o0 + q * 32 + lane, O, t0, T, K <= 32768, Y, y_is_bf16,
+                       acc_dbg);
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *s_abort && err_flag) atomicOr(err_flag, SBN_FLAG_TIMEOUT);
+  if (warp == 5) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
 
 static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -548,6 +818,31 @@ static sbn_status gemm_sp24_t(const int8_t *Xq, const float *absmax, const uint8
 }
 
 template <int BN>
+static sbn_status gemm_sp24_persist_t(const int8_t *Xq, const float *absmax, const uint8_t *codes,
+                                      const uint8_t *meta, const float *gamma_eff, int64_t T,
+                                      int64_t O, int64_t K, int64_t ldc, int64_t ldm, void *Y,
+                                      int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag,
+                                      cudaStream_t st) {
+  using Cfg = PsCfg<BN>;
+  CUtensorMap tx, tc, tm;
+  if (!encode_u8(&tx, Xq, K, T, K, Cfg::kKL, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_u8(&tc, codes, K / 8, O, ldc, 16, kBM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_u8(&tm, meta, K / 8, O, ldm, 16, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return SBN_ERR_CUDA;
+  auto kern = k_gemm_sp24_persist<BN>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::kSmem) !=
+      cudaSuccess)
+    return SBN_ERR_CUDA;
+  const int64_t ntiles = ((O + kBM - 1) / kBM) * ((T + BN - 1) / BN);
+  int64_t grid = num_sms();
+  if (grid > ntiles) grid = ntiles;
+  kern<<<(unsigned)grid, kPsThreads, Cfg::kSmem, st>>>(tx, tc, tm, absmax, gamma_eff, T, O, K, Y,
+                                                       y_is_bf16, acc_dbg, err_flag);
+  SBN_LAUNCH_CHECK();
+  return SBN_OK;
+}
+
+template <int BN>
 static sbn_status gemm_tc_bn(bool compact, const int8_t *Xq, const float *absmax,
                              const uint8_t *codes, const uint8_t *meta, const float *gamma_eff,
                              int64_t T, int64_t O, int64_t K, int64_t ldc, int64_t ldm, void *Y,
@@ -565,6 +860,9 @@ sbn_status launch_gemm_tc(const int8_t *Xq, const float *absmax, const uint8_t *
                           void *Y, int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag,
                           cudaStream_t st) {
   const bool compact = (n == 2 && m == 4);
+  if (compact && tokens > 128)
+    return gemm_sp24_persist_t<240>(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc, ldm,
+                                    Y, y_is_bf16, acc_dbg, err_flag, st);
   if (tokens > 128)
     return gemm_tc_bn<256>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc,
                            ldm, Y, y_is_bf16, acc_dbg, err_flag, st);

@@ -11,7 +11,7 @@
 
 namespace sbn {
 
-constexpr int kGvThreads = 256;
+constexpr int kGvThreads = 128;
 
 // prmt selector that gathers the kept activations of two 2:4 groups: meta byte
 // (i0A | i1A << 2 | i0B << 4 | i1B << 6) -> byte selectors i0A, i1A, 4 + i0B, 4 + i1B.
@@ -20,64 +20,25 @@ __device__ __forceinline__ uint32_t pair_selector(uint32_t mb) {
          ((((mb >> 6) & 3u) + 4u) << 12);
 }
 
-// One warp per output row: lane l takes the 64-weight chunks l, l+32, ..., at most CPL of
-// them, and issues every chunk load of the row before any arithmetic.  When T * CPL <= 4
-// the lane's activation words stay in registers for the whole kernel (the lane always sees
-// the same chunks); otherwise they are read from shared memory.
+// One warp per output row, every row in one round (enough CTAs for all rows): lane l takes
+// the 64-weight chunks l, l+32, ... (at most CPL per pass).  The row's code (and 2:4
+// metadata) loads are issued first, then the activation words are read through L1 (each
+// SM touches the few-KB activation block once, every other warp hits L1), then the dp4a
+// sums; the warp reduces with shuffles and lane t writes token t.
 template <int T, int CPL, bool kCompact>
 __global__ void __launch_bounds__(kGvThreads)
     k_gemv(const int8_t *__restrict__ Xq, const float *__restrict__ absmax,
            const uint8_t *__restrict__ codes, const uint8_t *__restrict__ meta,
            const float *__restrict__ gamma_eff, int64_t out, int64_t in, int64_t ldc,
            int64_t ldm, void *__restrict__ Y, int y_is_bf16, int32_t *__restrict__ acc_dbg) {
-  // registers hold the activations only when one pass covers the row (CPL chosen >= the
-  // chunks per lane, which the launcher guarantees for CPL <= 4)
-  constexpr bool kXReg = T * CPL <= 4;
-  extern __shared__ __align__(16) uint32_t xs[];  // [T][in/4] int8 words (shared mode)
-  const int64_t kw = in / 4;
   const int lane = threadIdx.x & 31;
+  const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (row >= out) return;  // whole warps leave together
   const int nchunks = (int)(in / 64);
-  uint32_t xr[kXReg ? T * CPL * 16 : 1];
-  if constexpr (kXReg) {
+  int acc[T];
 #pragma unroll
-    for (int t = 0; t < T; ++t)
-#pragma unroll
-      for (int i = 0; i < CPL; ++i) {
-        const int c = lane + 32 * i;
-        const uint4 *src = reinterpret_cast<const uint4 *>(Xq + t * in + (int64_t)c * 64);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const uint4 x4 = c < nchunks ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
-          uint32_t *d = xr + (t * CPL + i) * 16 + 4 * v;
-          d[0] = x4.x;
-          d[1] = x4.y;
-          d[2] = x4.z;
-          d[3] = x4.w;
-        }
-      }
-  } else {
-    for (int64_t i = threadIdx.x; i < T * kw / 4; i += blockDim.x)
-      reinterpret_cast<uint4 *>(xs)[i] = __ldg(reinterpret_cast<const uint4 *>(Xq) + i);
-    __syncthreads();
-  }
-  auto xword = [&](int t, int i, int c, int word) -> uint32_t {
-    if constexpr (kXReg)
-      return xr[(t * CPL + i) * 16 + word];
-    else
-      return xs[t * kw + (int64_t)c * 16 + word];
-  };
-
-  const float g = __ldg(gamma_eff);
-  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  // the next row's first chunk is requested before the current row is reduced
-  for (int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < out;
-       row += nwarps) {
-    if (row + nwarps < out && lane * 16 < ldc)
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(codes + (row + nwarps) * ldc + lane * 16));
-    int acc[T];
-#pragma unroll
-    for (int t = 0; t < T; ++t) acc[t] = 0;
-    for (int c0 = 0; c0 < nchunks; c0 += 32 * CPL) {  // one pass unless K > 2048 * CPL
+  for (int t = 0; t < T; ++t) acc[t] = 0;
+  for (int c0 = 0; c0 < nchunks; c0 += 32 * CPL) {  // one pass unless in > 2048 * CPL
     if constexpr (!kCompact) {
       const uint4 *crow = reinterpret_cast<const uint4 *>(codes + row * ldc);
       uint4 cw[CPL];
@@ -91,13 +52,17 @@ __global__ void __launch_bounds__(kGvThreads)
         if (c >= nchunks) continue;
         const uint32_t w4[4] = {cw[i].x, cw[i].y, cw[i].z, cw[i].w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int t = 0; t < T; ++t) {
+          const uint4 *xs = reinterpret_cast<const uint4 *>(Xq + t * in + (int64_t)c * 64);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int z = (int)((w4[q] << (2 * j)) & 0xC0C0C0C0u);
+          for (int q = 0; q < 4; ++q) {
+            const uint4 x4 = __ldg(xs + q);
+            const uint32_t xw[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
-            for (int t = 0; t < T; ++t) acc[t] = __dp4a(z, (int)xword(t, i, c, q * 4 + j), acc[t]);
+            for (int j = 0; j < 4; ++j)
+              acc[t] = __dp4a((int)((w4[q] << (2 * j)) & 0xC0C0C0C0u), (int)xw[j], acc[t]);
           }
+        }
       }
     } else {
       const uint2 *crow = reinterpret_cast<const uint2 *>(codes + row * ldc);
@@ -115,40 +80,40 @@ __global__ void __launch_bounds__(kGvThreads)
         if (c >= nchunks) continue;
         const uint32_t w2[2] = {cw[i].x, cw[i].y}, m2[2] = {mw[i].x, mw[i].y};
 #pragma unroll
-        for (int q = 0; q < 2; ++q)
+        for (int t = 0; t < T; ++t) {
+          const uint4 *xs = reinterpret_cast<const uint4 *>(Xq + t * in + (int64_t)c * 64);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int z = (int)((w2[q] << (2 * j)) & 0xC0C0C0C0u);
-            const uint32_t sel = pair_selector((m2[q] >> (8 * j)) & 0xffu);
-            const int xw = q * 8 + 2 * j;  // x words of the two groups
+          for (int q = 0; q < 2; ++q) {  // 32 stored codes = 8 groups = 32 positions
+            const uint4 xa = __ldg(xs + 2 * q), xb = __ldg(xs + 2 * q + 1);
+            const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
 #pragma unroll
-            for (int t = 0; t < T; ++t) {
-              const uint32_t xk = __byte_perm(xword(t, i, c, xw), xword(t, i, c, xw + 1), sel);
-              acc[t] = __dp4a(z, (int)xk, acc[t]);
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t sel = pair_selector((m2[q] >> (8 * j)) & 0xffu);
+              const uint32_t xk = __byte_perm(xw[2 * j], xw[2 * j + 1], sel);
+              acc[t] = __dp4a((int)((w2[q] << (2 * j)) & 0xC0C0C0C0u), (int)xk, acc[t]);
             }
           }
+        }
       }
     }
-    }
+  }
 #pragma unroll
-    for (int t = 0; t < T; ++t) {
+  for (int t = 0; t < T; ++t) {
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
-    }
-    if (lane < T) {
-      // lane t writes token t
-      int a = 0;
+    for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+  }
+  if (lane < T) {
+    int a = 0;
 #pragma unroll
-      for (int t = 0; t < T; ++t)
-        if (t == lane) a = acc[t];
-      a >>= 6;  // the code lanes carry 64 * t; the sum is an exact multiple of 64
-      const float y = __fmul_rn((float)a, rescale_factor(g, __ldg(absmax + lane)));
-      if (y_is_bf16)
-        reinterpret_cast<__nv_bfloat16 *>(Y)[lane * out + row] = __float2bfloat16_rn(y);
-      else
-        reinterpret_cast<float *>(Y)[lane * out + row] = y;
-      if (acc_dbg) acc_dbg[lane * out + row] = a;
-    }
+    for (int t = 0; t < T; ++t)
+      if (t == lane) a = acc[t];
+    a >>= 6;  // the code lanes carry 64 * t; the sum is an exact multiple of 64
+    const float y = __fmul_rn((float)a, rescale_factor(__ldg(gamma_eff), __ldg(absmax + lane)));
+    if (y_is_bf16)
+      reinterpret_cast<__nv_bfloat16 *>(Y)[lane * out + row] = __float2bfloat16_rn(y);
+    else
+      reinterpret_cast<float *>(Y)[lane * out + row] = y;
+    if (acc_dbg) acc_dbg[lane * out + row] = a;
   }
 }
 
@@ -157,20 +122,11 @@ static sbn_status gemv_tc(const int8_t *Xq, const float *absmax, const uint8_t *
                           const uint8_t *meta, const float *gamma_eff, int64_t out, int64_t in,
                           bool compact, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
                           int32_t *acc_dbg, cudaStream_t st) {
-  constexpr bool kXReg = T * CPL <= 4;
-  const size_t smem = kXReg ? 0 : (size_t)T * (size_t)in;
   const int64_t rows_per_cta = kGvThreads / 32;
-  int64_t grid = (out + rows_per_cta - 1) / rows_per_cta;
-  // persistent grid: activations are loaded once per warp (registers) or per CTA (shared)
-  const int64_t cap = (int64_t)num_sms() * (kXReg ? 4 : 2);
-  if (grid > cap) grid = cap;
+  const int64_t grid = (out + rows_per_cta - 1) / rows_per_cta;
   auto kern = compact ? k_gemv<T, CPL, true> : k_gemv<T, CPL, false>;
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-          cudaSuccess)
-    return SBN_ERR_CUDA;
-  kern<<<(unsigned)grid, kGvThreads, smem, st>>>(Xq, absmax, codes, meta, gamma_eff, out, in,
-                                                 ldc, ldm, Y, y_is_bf16, acc_dbg);
+  kern<<<(unsigned)grid, kGvThreads, 0, st>>>(Xq, absmax, codes, meta, gamma_eff, out, in, ldc,
+                                              ldm, Y, y_is_bf16, acc_dbg);
   SBN_LAUNCH_CHECK();
   return SBN_OK;
 }

@@ -9,14 +9,15 @@
 
 namespace sbn {
 
-// Device workspace of the weight pack: one partial sum per CTA of the reduction, the
-// arrival ticket (zero between calls), and the values the last CTA publishes.
+// Device workspace of the weight pack: one partial sum per CTA of the reduction.  The
+// quant/mask/pack kernel that follows on the same stream reads them; nothing in the
+// workspace needs clearing between calls.
 constexpr int kPackMaxParts = 1024;
 struct PackWorkspace {
-  unsigned long long part[kPackMaxParts];
-  unsigned int ticket;  // CTAs of k_abs_sum that finished; the last one resets it to 0
-  unsigned int thr;     // smallest bf16 magnitude (bits) whose ternary code is non-zero
-  float g;              // gamma + eps
+  unsigned long long part[kPackMaxParts];  // one exact partial sum per k_abs_sum CTA
+  unsigned int ticket;  // reserved (kept at zero)
+  unsigned int thr;     // reserved
+  float g;              // reserved
   unsigned int pad;
 };
 
@@ -47,6 +48,10 @@ struct FastPackArgs {
   uint8_t *meta;
   int64_t ldm, meta_row_bytes;
   int8_t *dense_dbg;
+  int nparts;       // partial sums left by k_abs_sum
+  int64_t n;        // weights in the tensor
+  float eps;
+  float *gamma_eff;  // written by CTA 0
 };
 
 __global__ void k_qmp_6of8(const FastPackArgs a);
@@ -73,9 +78,7 @@ sbn_status launch_gemm_tc(const int8_t *Xq, const float *absmax, const uint8_t *
                           void *Y, int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag,
                           cudaStream_t st);
 
-// Largest token count routed to the CUDA-core kernel, and the largest activation block
-// (tokens * in bytes) it stages in shared memory; larger calls use the tensor cores.
+// Largest token count routed to the CUDA-core kernel; larger calls use the tensor cores.
 constexpr int64_t kGemvMaxTokens = 4;
-constexpr int64_t kGemvMaxSmemBytes = 192 * 1024;
 
 }  // namespace sbn

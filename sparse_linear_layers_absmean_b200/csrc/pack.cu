@@ -4,14 +4,16 @@
 // mask generation from the BF16 masters, quant-then-mask order.)
 //
 // Two launches on the caller's stream:
-//   k_abs_sum          exact integer sum S = sum trunc(|W| * 2^24) (one partial per CTA);
-//                      the last CTA to finish turns S into gamma, g = gamma + eps and the
-//                      code threshold, and re-arms the workspace.
-//   k_quant_mask_pack  one pass over W: each lane owns 8 consecutive weights (one 16-byte
-//                      load), computes the keep mask of its group(s), the codes, and the
-//                      lanes of a 64-weight block assemble their packed words by shuffles.
+//   k_abs_sum          exact integer sum S = sum trunc(|W| * 2^24), one partial per CTA in
+//                      the workspace (eight 16-byte loads in flight per thread).
+//   k_quant_mask_pack  (generic N:M; 6:8 and 2:4 use pack_fast.cu) every CTA first turns the
+//                      partials into g and the code threshold (pack_common.cuh), then one
+//                      pass over W: each lane owns 8 consecutive weights, computes the keep
+//                      mask of its group(s) and the codes, and the lanes of a 64-weight
+//                      block assemble their packed words by shuffles.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "pack_common.cuh"
 
 namespace sbn {
 
@@ -19,25 +21,8 @@ namespace sbn {
 // S1: per-tensor absmean scale.
 // ---------------------------------------------------------------------------------------
 
-// Smallest bf16 magnitude (as bits) whose ternary code is non-zero for this g:
-// round_half_even(x / g) != 0  <=>  fl(x / g) > 0.5, and fl(x / g) is non-decreasing in x,
-// so the set of non-zero magnitudes is an up-set found by bisection over the bit patterns
-// (positive bf16 values are ordered like their bits).  Every division is IEEE fp32.
-__device__ uint32_t code_threshold(float g) {
-  uint32_t lo = 0, hi = kBf16InfBits;  // predicate false at 0 (0/g), true at +Inf
-  while (hi - lo > 1) {
-    uint32_t mid = (lo + hi) >> 1;
-    if (__fdiv_rn(__uint_as_float(mid << 16), g) > 0.5f)
-      hi = mid;
-    else
-      lo = mid;
-  }
-  return hi;
-}
-
 __global__ void __launch_bounds__(256) k_abs_sum(const uint4 *__restrict__ W, int64_t nvec,
-                                                 int64_t n, float eps, PackWorkspace *ws,
-                                                 float *gamma_eff, int32_t *err_flag) {
+                                                 PackWorkspace *ws, int32_t *err_flag) {
   unsigned long long acc = 0;
   uint32_t mx = 0;  // largest magnitude bits seen, per 16-bit half
   auto consume = [&](const uint4 &v) {
@@ -55,15 +40,14 @@ __global__ void __launch_bounds__(256) k_abs_sum(const uint4 *__restrict__ W, in
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   int64_t i = i0;
-  for (; i + 3 * stride < nvec; i += 4 * stride) {  // four 16-byte loads in flight
-    const uint4 v0 = __ldg(W + i), v1 = __ldg(W + i + stride), v2 = __ldg(W + i + 2 * stride),
-                v3 = __ldg(W + i + 3 * stride);
-    consume(v0);
-    consume(v1);
-    consume(v2);
-    consume(v3);
+  for (; i < nvec; i += 8 * stride) {  // up to eight 16-byte loads in flight per round
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      v[u] = i + u * stride < nvec ? __ldg(W + i + u * stride) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) consume(v[u]);  // zero words add nothing
   }
-  for (; i < nvec; i += stride) consume(__ldg(W + i));
   // Rare path: some |W| >= 256 (or NaN/Inf).  Re-read this thread's weights to tell the
   // two error kinds apart.
   uint32_t mx_all = 0, mx_fin = 0;
@@ -81,7 +65,6 @@ __global__ void __launch_bounds__(256) k_abs_sum(const uint4 *__restrict__ W, in
   }
   __shared__ unsigned long long s_sum[8];
   __shared__ uint32_t s_all[8], s_fin[8];
-  __shared__ int s_last;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   acc = warp_sum_u64(acc);
   uint32_t ma = warp_max_u32(mx_all);
@@ -105,29 +88,6 @@ __global__ void __launch_bounds__(256) k_abs_sum(const uint4 *__restrict__ W, in
     if (a >= kBf16InfBits) flags |= SBN_FLAG_W_NONFINITE;
     if (f >= kBf16Mag256Bits) flags |= SBN_FLAG_W_RANGE;
     if (flags && err_flag) atomicOr(err_flag, flags);
-    __threadfence();
-    unsigned int ticket = atomicAdd(&ws->ticket, 1u);
-    s_last = (ticket == gridDim.x - 1);
-  }
-  __syncthreads();
-  if (!s_last) return;
-  // Last CTA: every other CTA's partial is visible (fence before each ticket).
-  __threadfence();
-  unsigned long long S = 0;
-  for (int i = threadIdx.x; i < (int)gridDim.x; i += blockDim.x) S += __ldcg(&ws->part[i]);
-  S = warp_sum_u64(S);
-  if (lane == 0) s_sum[warp] = S;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    unsigned long long tot = 0;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += s_sum[w];
-    double mean = __ddiv_rn(__ull2double_rn(tot), (double)n * 16777216.0);
-    float gamma = __double2float_rn(mean);
-    float g = __fadd_rn(gamma, eps);
-    *gamma_eff = g;
-    ws->g = g;
-    ws->thr = code_threshold(g);
-    ws->ticket = 0;  // re-arm for the next call on this stream
   }
 }
 
@@ -209,6 +169,10 @@ struct QmpArgs {
   uint8_t *meta;
   int64_t ldm, meta_row_bytes;
   int8_t *dense_dbg;
+  int nparts;
+  int64_t n;
+  float eps;
+  float *gamma_eff;
 };
 
 // One 64-weight block per 8 lanes: lane `sub` owns weights 8*sub .. 8*sub+7 of block b.
@@ -300,7 +264,7 @@ __device__ __forceinline__ void qmp_block(const QmpArgs<N, M> &a, uint4 v, int64
 
 template <int N, int M>
 __global__ void __launch_bounds__(256) k_quant_mask_pack(const QmpArgs<N, M> a) {
-  const uint32_t thr = a.ws->thr;
+  const uint32_t thr = pack_prologue(a.ws, a.nparts, a.n, a.eps, a.gamma_eff);
   const int lane = threadIdx.x & 31;
   const int sub = lane & 7;
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -350,15 +314,17 @@ FastDiv make_fast_div(uint32_t d) {
 template <int N, int M>
 static void launch_qmp(const uint4 *W, int64_t nblocks, int64_t bpr, const PackWorkspace *ws,
                        uint8_t *codes, int64_t ldc, int64_t crow, uint8_t *meta, int64_t ldm,
-                       int64_t mrow, int8_t *dense_dbg, cudaStream_t st) {
+                       int64_t mrow, int8_t *dense_dbg, int nparts, int64_t n, float eps,
+                       float *gamma_eff, cudaStream_t st) {
   const int threads = 256;
   const int64_t nquads = (nblocks + 3) / 4;
   int64_t grid = (nquads + 15) / 16;  // 8 warps x 2 quads per CTA iteration
   const int64_t cap = (int64_t)num_sms() * 8;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  QmpArgs<N, M> a{W, nblocks, (uint32_t)bpr, make_fast_div((uint32_t)bpr), ws, codes, ldc, crow,
-                  meta, ldm, mrow, dense_dbg};
+  QmpArgs<N, M> a{W,    nblocks,   (uint32_t)bpr, make_fast_div((uint32_t)bpr), ws, codes, ldc,
+                  crow, meta,      ldm,           mrow,          dense_dbg,    nparts, n,
+                  eps,  gamma_eff};
   k_quant_mask_pack<N, M><<<(unsigned)grid, threads, 0, st>>>(a);
 }
 
@@ -368,21 +334,24 @@ sbn_status launch_pack(const void *W, int64_t out, int64_t in, int n, int m, flo
                        int32_t *err_flag, cudaStream_t st) {
   const int64_t nel = out * in;
   const int64_t nvec = nel / 8;
-  int64_t grid = (nvec + 256 * 4 - 1) / (256 * 4);
-  const int64_t cap = (int64_t)num_sms() * 7;  // ~56 resident warps per SM
+  int64_t grid = (nvec + 256 * 8 - 1) / (256 * 8);
+  const int64_t cap = (int64_t)num_sms() * 4;  // 32 resident warps per SM, 8 loads each
   if (grid > cap) grid = cap;
   if (grid > kPackMaxParts) grid = kPackMaxParts;
   if (grid < 1) grid = 1;
-  k_abs_sum<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint4 *>(W), nvec, nel, eps,
-                                           ws, gamma_eff, err_flag);
+  const int nparts = (int)grid;
+  k_abs_sum<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint4 *>(W), nvec, ws,
+                                           err_flag);
   SBN_LAUNCH_CHECK();
   const uint4 *W4 = reinterpret_cast<const uint4 *>(W);
   const int64_t nblocks = nel / 64, bpr = in / 64;
   if ((n == 6 && m == 8) || (n == 2 && m == 4)) {
-    FastPackArgs fa{W4,   nblocks, (uint32_t)bpr, make_fast_div((uint32_t)bpr), ws,   codes,
-                    ldc,  crow,    meta,          ldm,                          mrow, dense_dbg};
+    FastPackArgs fa{W4,  nblocks, (uint32_t)bpr, make_fast_div((uint32_t)bpr),
+                    ws,  codes,   ldc,           crow,
+                    meta, ldm,    mrow,          dense_dbg,
+                    nparts, nel,  eps,           gamma_eff};
     int64_t g = (nblocks + 63) / 64;  // 8 warps x 8 blocks per CTA pass
-    const int64_t capq = (int64_t)num_sms() * 8;
+    const int64_t capq = (int64_t)num_sms() * 4;
     if (g > capq) g = capq;
     if (g < 1) g = 1;
     if (n == 6)
@@ -395,7 +364,7 @@ sbn_status launch_pack(const void *W, int64_t out, int64_t in, int n, int m, flo
 #define SBN_QMP(NN, MM)                                                                    \
   case (NN * 16 + MM):                                                                     \
     launch_qmp<NN, MM>(W4, nblocks, bpr, ws, codes, ldc, crow, meta, ldm, mrow, dense_dbg, \
-                       st);                                                                \
+                       nparts, nel, eps, gamma_eff, st);                                   \
     break;
   switch (n * 16 + m) {
     SBN_QMP(1, 4)

@@ -1,0 +1,57 @@
+// Finishing the absmean scale, shared by the quant/mask/pack kernels (pack.cu,
+// pack_fast.cu).  k_abs_sum leaves one exact partial sum per CTA in the workspace; every
+// CTA of the next kernel turns them into gamma, g = gamma + eps and the code threshold.
+#pragma once
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace sbn {
+
+// Smallest bf16 magnitude (as bits) whose ternary code is non-zero for this g.
+// round_half_even(x / g) != 0  <=>  fl(x / g) > 0.5, and fl(x / g) is non-decreasing in x,
+// so the set of non-zero magnitudes is an up-set over the bit patterns (positive bf16
+// values are ordered like their bits).  One warp searches it 32-ary: the predicate is
+// false at 0 (0/g) and true at +Inf; each round keeps the sub-interval where it switches.
+// Every division is an IEEE fp32 division.
+__device__ __forceinline__ uint32_t code_threshold_warp(float g, int lane) {
+  uint32_t lo = 0, hi = kBf16InfBits;
+  while (hi - lo > 1) {
+    const uint32_t step = (hi - lo + 31) / 32;
+    uint32_t cand = lo + (uint32_t)(lane + 1) * step;
+    if (cand > hi) cand = hi;
+    const bool p = __fdiv_rn(__uint_as_float(cand << 16), g) > 0.5f;
+    const uint32_t ballot = __ballot_sync(0xffffffffu, p || cand == hi);
+    const int f = __ffs(ballot) - 1;  // first candidate where the predicate holds
+    const uint32_t new_hi = __shfl_sync(0xffffffffu, cand, f);
+    const uint32_t new_lo = f == 0 ? lo : __shfl_sync(0xffffffffu, cand, f > 0 ? f - 1 : 0);
+    hi = new_hi;
+    lo = new_lo;
+  }
+  return hi;
+}
+
+// Run by every thread of a CTA at the start of a quant/mask/pack kernel.  Returns the code
+// threshold; CTA 0 also publishes g = fp32(gamma + eps) to *gamma_eff, where
+// gamma = fp32(fp64(S) / (fp64(n) * 2^24)) and S is the exact sum of the partials.
+__device__ __forceinline__ uint32_t pack_prologue(const PackWorkspace *ws, int nparts,
+                                                  int64_t n, float eps, float *gamma_eff) {
+  __shared__ uint32_t s_thr;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    unsigned long long S = 0;
+    for (int i = lane; i < nparts; i += 32) S += ws->part[i];
+    S = warp_sum_u64(S);
+    const double mean = __ddiv_rn(__ull2double_rn(S), (double)n * 16777216.0);
+    const float g = __fadd_rn(__double2float_rn(mean), eps);
+    const uint32_t thr = code_threshold_warp(g, lane);
+    if (lane == 0) {
+      s_thr = thr;
+      if (blockIdx.x == 0) *gamma_eff = g;
+    }
+  }
+  __syncthreads();
+  return s_thr;
+}
+
+}  // namespace sbn

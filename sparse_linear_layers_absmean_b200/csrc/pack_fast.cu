@@ -14,6 +14,7 @@
 //     weight i in bit 8i+7) and shifted straight into the packed code layout.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "pack_common.cuh"
 
 namespace sbn {
 
@@ -129,18 +130,36 @@ __device__ uint32_t pair_entry(uint32_t keep8) {
   return meta | (sel << 8);
 }
 
+// This lane's 32 bytes of warp iteration q (zeros past the end).
+__device__ __forceinline__ void load_lane(const FastPackArgs &a, int64_t q, int lane, uint4 &v0,
+                                          uint4 &v1) {
+  const int64_t b = 8 * q + (lane >> 2);
+  if (b < a.nblocks) {
+    const uint4 *src = a.W + b * 8 + 2 * (lane & 3);
+    v0 = __ldg(src);
+    v1 = __ldg(src + 1);
+  } else {
+    v0 = v1 = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 __global__ void __launch_bounds__(256) k_qmp_6of8(const FastPackArgs a) {
-  const uint32_t thr = a.ws->thr;
-  const uint32_t thr2 = thr | (thr << 16);
   const int lane = threadIdx.x & 31;
   const int s = lane & 3;  // lane inside its 64-weight block
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int64_t noct = (a.nblocks + 7) >> 3;  // 8 blocks per warp iteration
-  for (int64_t q = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; q < noct; q += nwarps) {
+  const int64_t q0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  // the first weights are requested before the scale is finished, the next iteration's
+  // before the current one is processed
+  uint4 n0, n1;
+  load_lane(a, q0, lane, n0, n1);
+  const uint32_t thr = pack_prologue(a.ws, a.nparts, a.n, a.eps, a.gamma_eff);
+  const uint32_t thr2 = thr | (thr << 16);
+  for (int64_t q = q0; q < noct; q += nwarps) {
+    const uint4 v0 = n0, v1 = n1;
+    load_lane(a, q + nwarps, lane, n0, n1);
     const int64_t b = 8 * q + (lane >> 2);
     if (b >= a.nblocks) continue;  // no cross-lane exchange in this kernel
-    const uint4 *src = a.W + b * 8 + 2 * s;
-    const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
     uint32_t KGA, KGB, KHA, KHB;
     keep_6of8(w, KGA, KGB);
@@ -177,19 +196,21 @@ __global__ void __launch_bounds__(256) k_qmp_6of8(const FastPackArgs a) {
 __global__ void __launch_bounds__(256) k_qmp_2of4(const FastPackArgs a) {
   __shared__ uint32_t s_pair[256];
   s_pair[threadIdx.x] = pair_entry(threadIdx.x);
-  __syncthreads();
-  const uint32_t thr = a.ws->thr;
-  const uint32_t thr2 = thr | (thr << 16);
   const int lane = threadIdx.x & 31;
   const int s = lane & 3;
   const int js = 4 * (s & 1);  // 2j of stored elements 8s..8s+3 (j = 2*(s&1))
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int64_t noct = (a.nblocks + 7) >> 3;
-  for (int64_t q = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; q < noct; q += nwarps) {
+  const int64_t q0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  uint4 n0, n1;
+  load_lane(a, q0, lane, n0, n1);
+  const uint32_t thr = pack_prologue(a.ws, a.nparts, a.n, a.eps, a.gamma_eff);  // syncs
+  const uint32_t thr2 = thr | (thr << 16);
+  for (int64_t q = q0; q < noct; q += nwarps) {
+    const uint4 v0 = n0, v1 = n1;
+    load_lane(a, q + nwarps, lane, n0, n1);
     const int64_t b = 8 * q + (lane >> 2);
     const bool valid = b < a.nblocks;  // all lanes stay for the shuffle below
-    const uint4 *src = a.W + (valid ? b : 0) * 8 + 2 * s;
-    const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
     const uint32_t KA = keep_2of4(w[0], w[1]), KB = keep_2of4(w[2], w[3]);
     const uint32_t KC = keep_2of4(w[4], w[5]), KD = keep_2of4(w[6], w[7]);

@@ -57,7 +57,7 @@ def test_pack_all_zero_with_zero_eps():
     assert got["g"] == 0 and not got["ws"].any()
 
 
-def test_pack_workspace_is_rearmed():
+def test_pack_workspace_is_reusable():
     W1 = workloads.masters(64, 256, seed=1)
     W2 = workloads.masters(64, 256, seed=2)
     import sparse_linear_layers_absmean_b200 as sbn
@@ -66,7 +66,7 @@ def test_pack_workspace_is_rearmed():
         got = gpu_path.pack(W, 2, 4, workspace=ws)
         ref = oracle.quantize_mask_pack(W, 2, 4)
         assert got["g"] == ref["g"] and np.array_equal(got["codes"], ref["codes"])
-    # the arrival counter (first word after the 1024 partial sums) is back at zero
+    # the reserved word after the 1024 partial sums is never written
     assert ws[8192:8196].cpu().numpy().view(np.uint32)[0] == 0
 
 
@@ -123,6 +123,14 @@ def test_linear_cuda_cores(T, O, K, n, m):
 @pytest.mark.parametrize("O,K", [(300, 192), (130, 640)])
 def test_linear_tensor_cores(T, O, K, n, m):
     check_linear(T, O, K, n, m, seed=T * 7 + O + K + n)
+
+
+@pytest.mark.parametrize("T,O,K", [(1500, 6000, 320), (1000, 8000, 128), (500, 12000, 64)])
+def test_linear_many_tiles_per_cta(T, O, K):
+    """Enough 128 x 240 output tiles that the persistent 2:4 kernel gives each CTA several,
+    so both TMEM accumulators and the stage ring wrap across tiles (ragged rows, tokens
+    and K in each case)."""
+    check_linear(T, O, K, 2, 4, seed=T + O + K)
 
 
 @pytest.mark.parametrize("T", [1, 3, 9, 300])
