@@ -3,14 +3,15 @@
 // (Sparse-BitNet technical summaries, section 2 "Methodology": Sparse-BitLinear items 1-2,
 // mask generation from the BF16 masters, quant-then-mask order.)
 //
-// Two launches on the caller's stream:
+// Two launches on the caller's stream.  6:8 and 2:4 use pack_fast.cu (keep masks and the
+// sum in the first launch, codes in the second); every other N:M pattern uses:
 //   k_abs_sum          exact integer sum S = sum trunc(|W| * 2^24), one partial per CTA in
 //                      the workspace (eight 16-byte loads in flight per thread).
-//   k_quant_mask_pack  (generic N:M; 6:8 and 2:4 use pack_fast.cu) every CTA first turns the
-//                      partials into g and the code threshold (pack_common.cuh), then one
-//                      pass over W: each lane owns 8 consecutive weights, computes the keep
-//                      mask of its group(s) and the codes, and the lanes of a 64-weight
-//                      block assemble their packed words by shuffles.
+//   k_quant_mask_pack  every CTA first turns the partials into g and the code threshold
+//                      (pack_common.cuh), then one pass over W: each lane owns 8
+//                      consecutive weights, computes the keep mask of its group(s) and the
+//                      codes, and the lanes of a 64-weight block assemble their packed
+//                      words by shuffles.
 #include "common.cuh"
 #include "kernels.cuh"
 #include "pack_common.cuh"
@@ -333,6 +334,16 @@ sbn_status launch_pack(const void *W, int64_t out, int64_t in, int n, int m, flo
                        int64_t mrow, float *gamma_eff, PackWorkspace *ws, int8_t *dense_dbg,
                        int32_t *err_flag, cudaStream_t st) {
   const int64_t nel = out * in;
+  const uint4 *W4 = reinterpret_cast<const uint4 *>(W);
+  const int64_t nblocks = nel / 64, bpr = in / 64;
+  if ((n == 6 && m == 8) || (n == 2 && m == 4)) {
+    FastPackArgs fa{W4,  nblocks, (uint32_t)bpr, make_fast_div((uint32_t)bpr),
+                    ws,  codes,   ldc,           crow,
+                    meta, ldm,    mrow,          dense_dbg,
+                    0,   nel,     eps,           gamma_eff};
+    fa.nparts = (int)fast_pack_parts(fa);
+    return launch_fast_pack(fa, n == 2, err_flag, st);
+  }
   const int64_t nvec = nel / 8;
   int64_t grid = (nvec + 256 * 8 - 1) / (256 * 8);
   const int64_t cap = (int64_t)num_sms() * 4;  // 32 resident warps per SM, 8 loads each
@@ -340,27 +351,8 @@ sbn_status launch_pack(const void *W, int64_t out, int64_t in, int n, int m, flo
   if (grid > kPackMaxParts) grid = kPackMaxParts;
   if (grid < 1) grid = 1;
   const int nparts = (int)grid;
-  k_abs_sum<<<(unsigned)grid, 256, 0, st>>>(reinterpret_cast<const uint4 *>(W), nvec, ws,
-                                           err_flag);
+  k_abs_sum<<<(unsigned)grid, 256, 0, st>>>(W4, nvec, ws, err_flag);
   SBN_LAUNCH_CHECK();
-  const uint4 *W4 = reinterpret_cast<const uint4 *>(W);
-  const int64_t nblocks = nel / 64, bpr = in / 64;
-  if ((n == 6 && m == 8) || (n == 2 && m == 4)) {
-    FastPackArgs fa{W4,  nblocks, (uint32_t)bpr, make_fast_div((uint32_t)bpr),
-                    ws,  codes,   ldc,           crow,
-                    meta, ldm,    mrow,          dense_dbg,
-                    nparts, nel,  eps,           gamma_eff};
-    int64_t g = (nblocks + 63) / 64;  // 8 warps x 8 blocks per CTA pass
-    const int64_t capq = (int64_t)num_sms() * 4;
-    if (g > capq) g = capq;
-    if (g < 1) g = 1;
-    if (n == 6)
-      k_qmp_6of8<<<(unsigned)g, 256, 0, st>>>(fa);
-    else
-      k_qmp_2of4<<<(unsigned)g, 256, 0, st>>>(fa);
-    SBN_LAUNCH_CHECK();
-    return SBN_OK;
-  }
 #define SBN_QMP(NN, MM)                                                                    \
   case (NN * 16 + MM):                                                                     \
     launch_qmp<NN, MM>(W4, nblocks, bpr, ws, codes, ldc, crow, meta, ldm, mrow, dense_dbg, \

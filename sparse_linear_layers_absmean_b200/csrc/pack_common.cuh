@@ -33,14 +33,21 @@ __device__ __forceinline__ uint32_t code_threshold_warp(float g, int lane) {
 
 // Run by every thread of a CTA at the start of a quant/mask/pack kernel.  Returns the code
 // threshold; CTA 0 also publishes g = fp32(gamma + eps) to *gamma_eff, where
-// gamma = fp32(fp64(S) / (fp64(n) * 2^24)) and S is the exact sum of the partials.
+// gamma = fp32(fp64(S) / (fp64(n) * 2^24)) and S is the exact sum of the partials.  All
+// threads load the partials (a few each, in one round of loads), warp 0 finishes.
 __device__ __forceinline__ uint32_t pack_prologue(const PackWorkspace *ws, int nparts,
                                                   int64_t n, float eps, float *gamma_eff) {
+  __shared__ unsigned long long s_part[32];
   __shared__ uint32_t s_thr;
+  unsigned long long S = 0;
+#pragma unroll 4
+  for (int i = threadIdx.x; i < nparts; i += blockDim.x) S += ws->part[i];
+  S = warp_sum_u64(S);
+  if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = S;
+  __syncthreads();
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
-    unsigned long long S = 0;
-    for (int i = lane; i < nparts; i += 32) S += ws->part[i];
+    S = lane < (int)(blockDim.x >> 5) ? s_part[lane] : 0ull;
     S = warp_sum_u64(S);
     const double mean = __ddiv_rn(__ull2double_rn(S), (double)n * 16777216.0);
     const float g = __fadd_rn(__double2float_rn(mean), eps);

@@ -1,13 +1,20 @@
 // Quant/mask/pack for the two patterns the pages use most, 6:8 and 2:4, with far fewer
 // instructions per weight than the generic kernel (pack.cu).  Same results, bit for bit.
 //
+// Two passes over W.  The N:M selection does not depend on the scale, so it runs in the
+// pass that must read all of W anyway for the absmean sum: k_mask_sum streams W from HBM,
+// writes the metadata plane and the per-CTA partial sums, and its selection arithmetic
+// overlaps the loads.  k_codes finishes the scale and then needs only a compare per
+// weight: it re-reads W (from L2 where W fits there) with the metadata and writes the
+// codes plane.
+//
 // Each lane owns 16 consecutive weights (two 16-byte loads).  The arithmetic runs on the
 // bf16 words as they are loaded (two weights per 32-bit register):
 //   * N:M selection: the values of the M-N smallest magnitudes come from a min/max network
 //     on both 16-bit halves at once (min.u16x2 / max.u16x2); a weight is pruned iff its
 //     magnitude is <= the (M-N)-th smallest.  That set has exactly M-N members unless
-//     magnitudes tie at the boundary; those groups (rare) take the exact rank rule with
-//     the lower index winning, the same rule as everywhere else.
+//     magnitudes tie at the boundary; those groups (about one in a hundred) resolve the
+//     tie inline with the rank rule's order (the lower index wins).
 //   * code non-zero test: mag >= thr for both halves with one OR and one subtract
 //     ((w | 0x80008000) - thr2 leaves each half's answer in its top bit, no borrow crosses).
 //   * per-weight flags are collected with byte permutes into "byte-top" words (flag of
@@ -15,6 +22,7 @@
 #include "common.cuh"
 #include "kernels.cuh"
 #include "pack_common.cuh"
+#include "ptx.cuh"
 
 namespace sbn {
 
@@ -50,22 +58,21 @@ __device__ __forceinline__ uint32_t flags_to_i8(uint32_t lo, uint32_t hi) {
   return (lo >> 7) | ((hi >> 7) * 0xfeu);
 }
 
-// Exact rank rule for one group (the fallback when magnitudes tie at the boundary).
-template <int N, int M>
-__device__ __noinline__ uint32_t exact_keep(const uint32_t *w) {
-  uint32_t key[M];
-#pragma unroll
-  for (int i = 0; i < M; ++i)
-    key[i] = ((((w[i >> 1] >> (16 * (i & 1))) & 0x7fffu)) << 3) | (uint32_t)(M - 1 - i);
-  uint32_t keep = 0;
-#pragma unroll
-  for (int i = 0; i < M; ++i) {
-    int rank = 0;
-#pragma unroll
-    for (int j = 0; j < M; ++j) rank += (j != i) && (key[j] > key[i]);
-    keep |= (uint32_t)(rank < N) << i;
-  }
-  return keep;
+// Highest set bit of x (x != 0) as a mask; 0 for x == 0.
+__device__ __forceinline__ uint32_t top_bit(uint32_t x) {
+  return x ? (0x80000000u >> __clz(x)) : 0u;
+}
+
+// Boundary ties.  With m2 the second smallest magnitude of a group, the pruned set is
+// every weight below m2 (LT, at most one) plus, of the weights equal to m2 (EQ), the ones
+// with the highest indices until two are pruned: the lower index wins a tie, as in the
+// rank rule.  LE / LT / EQ are bit masks ordered like the weights, so the highest index
+// is the highest set bit.
+__device__ __forceinline__ uint32_t prune_with_ties(uint32_t le, uint32_t lt) {
+  const uint32_t eq = le ^ lt;
+  const uint32_t h1 = top_bit(eq);
+  const uint32_t h2 = top_bit(eq ^ h1);
+  return lt | h1 | (lt ? 0u : h2);
 }
 
 // 6:8 keep flags of one group (w[0..3]); KA/KB: byte-top flags of weights 0-3 / 4-7.
@@ -78,14 +85,19 @@ __device__ __forceinline__ void keep_6of8(const uint32_t *w, uint32_t &KA, uint3
   // second smallest of all eight, in both halves
   const uint32_t m2 = vmin16(vmax16(c0, swap16(c0)), vmin16(c1, swap16(c1)));
   const uint32_t h = m2 | kHalf;
-  // top bit of each half: mag <= m2 (pruned when the boundary has no tie)
+  // top bit of each half: mag <= m2 (exactly the pruned pair when the boundary has no tie)
   const uint32_t LA = __byte_perm(h - M0, h - M1, 0x7531) & kTop;
   const uint32_t LB = __byte_perm(h - M2, h - M3, 0x7531) & kTop;
   if (__popc(LA | (LB >> 1)) == 2) {
     KA = LA ^ kTop;
     KB = LB ^ kTop;
   } else {
-    const uint32_t keep = exact_keep<6, 8>(w);
+    // mag <= m2 - 1 (nothing when m2 == 0: each half of hl is then 0x7fff)
+    const uint32_t hl = h - 0x00010001u;
+    const uint32_t TA = __byte_perm(hl - M0, hl - M1, 0x7531) & kTop;
+    const uint32_t TB = __byte_perm(hl - M2, hl - M3, 0x7531) & kTop;
+    const uint32_t keep =
+        ~prune_with_ties(top_bits_to_byte(LA, LB), top_bits_to_byte(TA, TB)) & 0xffu;
     KA = nibble_to_top_bits(keep);
     KB = nibble_to_top_bits(keep >> 4);
   }
@@ -99,8 +111,9 @@ __device__ __forceinline__ uint32_t keep_2of4(uint32_t wa, uint32_t wb) {
   const uint32_t h = m2 | kHalf;
   const uint32_t L = __byte_perm(h - Ma, h - Mb, 0x7531) & kTop;
   if (__popc(L) == 2) return L ^ kTop;
-  const uint32_t w2[2] = {wa, wb};
-  return nibble_to_top_bits(exact_keep<2, 4>(w2));
+  const uint32_t hl = h - 0x00010001u;
+  const uint32_t T = __byte_perm(hl - Ma, hl - Mb, 0x7531) & kTop;
+  return prune_with_ties(L, T) ^ kTop;  // byte-top flags are ordered like the weights too
 }
 
 __device__ __forceinline__ uint32_t nonzero_flags(uint32_t w, uint32_t thr2) {
@@ -108,6 +121,7 @@ __device__ __forceinline__ uint32_t nonzero_flags(uint32_t w, uint32_t thr2) {
 }
 
 }  // namespace
+
 
 // For a keep byte (two 2:4 groups, 4 bits each): the meta byte (i0 | i1 << 2 per group)
 // in bits 0-7, and in bits 8-23 the byte-permute selector that compacts the kept weights
@@ -130,12 +144,41 @@ __device__ uint32_t pair_entry(uint32_t keep8) {
   return meta | (sel << 8);
 }
 
-// This lane's 32 bytes of warp iteration q (zeros past the end).
-__device__ __forceinline__ void load_lane(const FastPackArgs &a, int64_t q, int lane, uint4 &v0,
-                                          uint4 &v1) {
-  const int64_t b = 8 * q + (lane >> 2);
-  if (b < a.nblocks) {
-    const uint4 *src = a.W + b * 8 + 2 * (lane & 3);
+// ---------------------------------------------------------------------------------------
+// Exact absmean sum S = sum trunc(|W| * 2^24) with one fp64 add per weight.
+// ((h << 13) & 0x0fffe000) | 0x40000000, for the 15 magnitude bits h of a bf16 value, is
+// the high word of the fp64 number |W| * 2^128 (bf16 exponent e -> fp64 exponent field
+// e + 1024, the seven mantissa bits after it; zero and subnormals give values below 4).
+// The accumulator starts at 2^156, where the fp64 spacing is 2^104, and every add rounds
+// toward zero: with acc on that grid and 0 <= v, floor(acc + v) = acc + floor(v), so each
+// add contributes exactly floor(|W| * 2^128 / 2^104) = trunc(|W| * 2^24).  The low 52 bits
+// of the final accumulator are the sum (below 2^52 for any one thread's share).  Exact for
+// |W| < 256, the supported range.
+// ---------------------------------------------------------------------------------------
+constexpr double kAccBias = 9.1343852333181432e46;  // 2^156
+
+__device__ __forceinline__ double mag_lo_x2p128(uint32_t w) {
+  return __hiloint2double((int)(((w << 13) & 0x0fffe000u) | 0x40000000u), 0);
+}
+__device__ __forceinline__ double mag_hi_x2p128(uint32_t w) {
+  return __hiloint2double((int)(((w >> 3) & 0x0fffe000u) | 0x40000000u), 0);
+}
+__device__ __forceinline__ unsigned long long acc_value(double acc) {
+  return (unsigned long long)__double_as_longlong(acc) & ((1ull << 52) - 1);
+}
+
+// Work split of both passes: warp-iteration q covers 64-weight blocks 8q .. 8q+7 (1 KB of
+// W); lane l owns weights 16 (l & 3) .. +15 of block 8q + (l >> 2), loaded as two 16-byte
+// words.  Warps stride over q; four 256-thread CTAs per SM keep about 64 KB of loads in
+// flight per SM (the next iteration's words are requested before the current ones are
+// used), enough for the full HBM bandwidth.
+constexpr int kPkThreads = 256;
+constexpr int kPkCtasPerSm = 4;
+
+__device__ __forceinline__ void pk_load(const uint4 *W, uint32_t nb, uint32_t b, int s, uint4 &v0,
+                                        uint4 &v1) {
+  if (b < nb) {
+    const uint4 *src = W + (uint64_t)b * 8 + 2 * s;
     v0 = __ldg(src);
     v1 = __ldg(src + 1);
   } else {
@@ -143,114 +186,248 @@ __device__ __forceinline__ void load_lane(const FastPackArgs &a, int64_t q, int 
   }
 }
 
-__global__ void __launch_bounds__(256) k_qmp_6of8(const FastPackArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int s = lane & 3;  // lane inside its 64-weight block
-  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  const int64_t noct = (a.nblocks + 7) >> 3;  // 8 blocks per warp iteration
-  const int64_t q0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  // the first weights are requested before the scale is finished, the next iteration's
-  // before the current one is processed
+// ---------------------------------------------------------------------------------------
+// Pass 1: keep masks and the exact absmean sum, in one read of W.  The metadata plane is
+// written here (6:8: the keep bits of each group of 8; 2:4: i0 | i1 << 2 per group of 4);
+// each CTA leaves its partial sum in the workspace and raises the weight error flags.
+// ---------------------------------------------------------------------------------------
+template <bool kCompact>
+__global__ void __launch_bounds__(kPkThreads, kPkCtasPerSm)
+    k_mask_sum(const FastPackArgs a, int32_t *err_flag) {
+  __shared__ uint32_t s_meta[256];  // 2:4: keep byte of two groups -> their meta byte
+  __shared__ unsigned long long s_sum[kPkThreads / 32];
+  __shared__ uint32_t s_all[kPkThreads / 32], s_fin[kPkThreads / 32];
+  // the codes pass may start launching; its CTAs find room only as these ones leave
+  ptx::grid_dep_launch();
+  if (kCompact) s_meta[threadIdx.x] = pair_entry(threadIdx.x) & 0xffu;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int s = lane & 3;
+  const uint32_t nb = (uint32_t)a.nblocks;
+  const uint32_t nwarps = gridDim.x * (kPkThreads / 32);
+  const uint32_t bstep = 8 * nwarps;
+  uint32_t b = 8 * (blockIdx.x * (kPkThreads / 32) + warp) + (lane >> 2);
+  double acc0 = kAccBias, acc1 = kAccBias;
+  uint32_t mx = 0;  // largest magnitude bits seen, per 16-bit half
   uint4 n0, n1;
-  load_lane(a, q0, lane, n0, n1);
-  const uint32_t thr = pack_prologue(a.ws, a.nparts, a.n, a.eps, a.gamma_eff);
-  const uint32_t thr2 = thr | (thr << 16);
-  for (int64_t q = q0; q < noct; q += nwarps) {
+  pk_load(a.W, nb, b, s, n0, n1);
+  for (; b - (lane >> 2) < nb; b += bstep) {  // warp-uniform: the warp's first block
     const uint4 v0 = n0, v1 = n1;
-    load_lane(a, q + nwarps, lane, n0, n1);
-    const int64_t b = 8 * q + (lane >> 2);
-    if (b >= a.nblocks) continue;  // no cross-lane exchange in this kernel
+    pk_load(a.W, nb, b + bstep, s, n0, n1);
+    if (b >= nb) continue;
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    uint32_t KGA, KGB, KHA, KHB;
-    keep_6of8(w, KGA, KGB);
-    keep_6of8(w + 4, KHA, KHB);
-    const uint32_t NGA = __byte_perm(nonzero_flags(w[0], thr2), nonzero_flags(w[1], thr2), 0x7531);
-    const uint32_t NGB = __byte_perm(nonzero_flags(w[2], thr2), nonzero_flags(w[3], thr2), 0x7531);
-    const uint32_t NHA = __byte_perm(nonzero_flags(w[4], thr2), nonzero_flags(w[5], thr2), 0x7531);
-    const uint32_t NHB = __byte_perm(nonzero_flags(w[6], thr2), nonzero_flags(w[7], thr2), 0x7531);
-    const uint32_t LGA = NGA & KGA, LGB = NGB & KGB, LHA = NHA & KHA, LHB = NHB & KHB;
-    const uint32_t HGA = LGA & __byte_perm(w[0], w[1], 0x7531);
-    const uint32_t HGB = LGB & __byte_perm(w[2], w[3], 0x7531);
-    const uint32_t HHA = LHA & __byte_perm(w[4], w[5], 0x7531);
-    const uint32_t HHB = LHB & __byte_perm(w[6], w[7], 0x7531);
-    // weights e = 0..15 of this lane are elements 16s+e of the block: word s, byte e%4,
-    // bits (7,6) - 2*(e/4) for (negative, non-zero)
-    const uint32_t word = HGA | (LGA >> 1) | (HGB >> 2) | (LGB >> 3) | (HHA >> 4) | (LHA >> 5) |
-                          (HHB >> 6) | (LHB >> 7);
-    const uint32_t meta16 = top_bits_to_byte(KGA, KGB) | (top_bits_to_byte(KHA, KHB) << 8);
-    const uint32_t row = fast_div((uint32_t)b, a.div_bpr);
-    const uint32_t col = (uint32_t)b - row * a.bpr;
-    uint8_t *crow = a.codes + (int64_t)row * a.ldc;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      mx = vmax16(mx, w[k] & kMag);
+      acc0 = __dadd_rz(acc0, mag_lo_x2p128(w[k]));
+      acc1 = __dadd_rz(acc1, mag_hi_x2p128(w[k]));
+    }
+    uint32_t meta16;
+    if constexpr (kCompact) {
+      const uint32_t KA = keep_2of4(w[0], w[1]), KB = keep_2of4(w[2], w[3]);
+      const uint32_t KC = keep_2of4(w[4], w[5]), KD = keep_2of4(w[6], w[7]);
+      meta16 = s_meta[top_bits_to_byte(KA, KB)] | (s_meta[top_bits_to_byte(KC, KD)] << 8);
+    } else {
+      uint32_t KGA, KGB, KHA, KHB;
+      keep_6of8(w, KGA, KGB);
+      keep_6of8(w + 4, KHA, KHB);
+      meta16 = top_bits_to_byte(KGA, KGB) | (top_bits_to_byte(KHA, KHB) << 8);
+    }
+    const uint32_t row = fast_div(b, a.div_bpr);
+    const uint32_t col = b - row * a.bpr;
     uint8_t *mrow = a.meta + (int64_t)row * a.ldm;
-    reinterpret_cast<uint32_t *>(crow + col * 16)[s] = word;
     reinterpret_cast<uint16_t *>(mrow + col * 8)[s] = (uint16_t)meta16;
-    if (col == a.bpr - 1 && s == 0 && a.ldm > a.meta_row_bytes)
+    if (s == 0 && col == a.bpr - 1 && a.ldm > a.meta_row_bytes)
       *reinterpret_cast<uint2 *>(mrow + a.meta_row_bytes) = make_uint2(0u, 0u);
-    if (a.dense_dbg)
-      *reinterpret_cast<uint4 *>(a.dense_dbg + b * 64 + 16 * s) =
-          make_uint4(flags_to_i8(LGA, HGA), flags_to_i8(LGB, HGB), flags_to_i8(LHA, HHA),
-                     flags_to_i8(LHB, HHB));
+  }
+  unsigned long long sum = acc_value(acc0) + acc_value(acc1);
+  // Rare path: some |W| >= 256 (or NaN/Inf).  Re-read this lane's weights to tell the two
+  // error kinds apart.
+  uint32_t mx_all = 0, mx_fin = 0;
+  if (max(mx & 0xffffu, mx >> 16) >= kBf16Mag256Bits) {
+    for (uint32_t bb = 8 * (blockIdx.x * (kPkThreads / 32) + warp) + (lane >> 2); bb < nb;
+         bb += bstep) {
+      uint4 v0, v1;
+      pk_load(a.W, nb, bb, s, v0, v1);
+      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      for (int k = 0; k < 16; ++k) {
+        const uint32_t m = (w[k >> 1] >> (16 * (k & 1))) & 0x7fffu;
+        mx_all = max(mx_all, m);
+        if (m < kBf16InfBits) mx_fin = max(mx_fin, m);
+      }
+    }
+  }
+  sum = warp_sum_u64(sum);
+  const uint32_t ma = warp_max_u32(mx_all), mf = warp_max_u32(mx_fin);
+  if (lane == 0) {
+    s_sum[warp] = sum;
+    s_all[warp] = ma;
+    s_fin[warp] = mf;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long tot = 0;
+    uint32_t am = 0, fm = 0;
+    for (int i = 0; i < kPkThreads / 32; ++i) {
+      tot += s_sum[i];
+      am = max(am, s_all[i]);
+      fm = max(fm, s_fin[i]);
+    }
+    const_cast<PackWorkspace *>(a.ws)->part[blockIdx.x] = tot;
+    int flags = 0;
+    if (am >= kBf16InfBits) flags |= SBN_FLAG_W_NONFINITE;
+    if (fm >= kBf16Mag256Bits) flags |= SBN_FLAG_W_RANGE;
+    if (flags && err_flag) atomicOr(err_flag, flags);
   }
 }
 
-__global__ void __launch_bounds__(256) k_qmp_2of4(const FastPackArgs a) {
-  __shared__ uint32_t s_pair[256];
-  s_pair[threadIdx.x] = pair_entry(threadIdx.x);
-  const int lane = threadIdx.x & 31;
+// prmt selector that compacts the kept weights of two 2:4 groups: meta byte
+// (i0A | i1A << 2 | i0B << 4 | i1B << 6) -> byte selectors i0A, i1A, 4 + i0B, 4 + i1B.
+__device__ __forceinline__ uint32_t compact_selector(uint32_t mb) {
+  return (mb & 3u) | (((mb >> 2) & 3u) << 4) | ((((mb >> 4) & 3u) + 4u) << 8) |
+         ((((mb >> 6) & 3u) + 4u) << 12);
+}
+
+// Meta bits of this lane for block b (pass 1's output), 0 past the end.
+__device__ __forceinline__ uint32_t meta_of(const FastPackArgs &a, uint32_t nb, uint32_t b, int s) {
+  if (b >= nb) return 0u;
+  const uint32_t row = fast_div(b, a.div_bpr);
+  const uint32_t col = b - row * a.bpr;
+  return reinterpret_cast<const uint16_t *>(a.meta + (int64_t)row * a.ldm + col * 8)[s];
+}
+
+// ---------------------------------------------------------------------------------------
+// Pass 2: codes.  Each lane requests its first W words at once (W does not depend on
+// pass 1; after pass 1 they are mostly L2 hits), then the CTA waits for pass 1 to
+// complete, finishes the scale (pack_prologue) and stores the 2-bit codes of the kept
+// weights, with the next iteration's W words and metadata requested ahead.
+// ---------------------------------------------------------------------------------------
+template <bool kCompact>
+__global__ void __launch_bounds__(kPkThreads, kPkCtasPerSm) k_codes(const FastPackArgs a) {
+  __shared__ uint32_t s_sel[256];  // 2:4: meta byte -> compaction selector
+  if (kCompact) s_sel[threadIdx.x] = compact_selector(threadIdx.x);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int s = lane & 3;
-  const int js = 4 * (s & 1);  // 2j of stored elements 8s..8s+3 (j = 2*(s&1))
-  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  const int64_t noct = (a.nblocks + 7) >> 3;
-  const int64_t q0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int js = 4 * (s & 1);  // 2:4: 2j of stored elements 8s..8s+3 (j = 2*(s&1))
+  const uint32_t nb = (uint32_t)a.nblocks;
+  const uint32_t bstep = 8 * gridDim.x * (kPkThreads / 32);
+  uint32_t b = 8 * (blockIdx.x * (kPkThreads / 32) + warp) + (lane >> 2);
   uint4 n0, n1;
-  load_lane(a, q0, lane, n0, n1);
+  pk_load(a.W, nb, b, s, n0, n1);
+  ptx::grid_dep_wait();  // pass 1 complete: partial sums and metadata visible
   const uint32_t thr = pack_prologue(a.ws, a.nparts, a.n, a.eps, a.gamma_eff);  // syncs
   const uint32_t thr2 = thr | (thr << 16);
-  for (int64_t q = q0; q < noct; q += nwarps) {
+  uint32_t nm = meta_of(a, nb, b, s);
+  for (; b - (lane >> 2) < nb; b += bstep) {  // warp-uniform: the warp's first block
     const uint4 v0 = n0, v1 = n1;
-    load_lane(a, q + nwarps, lane, n0, n1);
-    const int64_t b = 8 * q + (lane >> 2);
-    const bool valid = b < a.nblocks;  // all lanes stay for the shuffle below
+    const uint32_t m16 = nm;
+    pk_load(a.W, nb, b + bstep, s, n0, n1);
+    nm = meta_of(a, nb, b + bstep, s);
+    const bool valid = b < nb;  // both lanes of a shuffle pair share the block
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    const uint32_t KA = keep_2of4(w[0], w[1]), KB = keep_2of4(w[2], w[3]);
-    const uint32_t KC = keep_2of4(w[4], w[5]), KD = keep_2of4(w[6], w[7]);
-    const uint32_t eAB = s_pair[top_bits_to_byte(KA, KB)];
-    const uint32_t eCD = s_pair[top_bits_to_byte(KC, KD)];
-    const uint32_t NA = __byte_perm(nonzero_flags(w[0], thr2), nonzero_flags(w[1], thr2), 0x7531);
-    const uint32_t NB = __byte_perm(nonzero_flags(w[2], thr2), nonzero_flags(w[3], thr2), 0x7531);
-    const uint32_t NC = __byte_perm(nonzero_flags(w[4], thr2), nonzero_flags(w[5], thr2), 0x7531);
-    const uint32_t ND = __byte_perm(nonzero_flags(w[6], thr2), nonzero_flags(w[7], thr2), 0x7531);
-    const uint32_t SA = __byte_perm(w[0], w[1], 0x7531), SB = __byte_perm(w[2], w[3], 0x7531);
-    const uint32_t SC = __byte_perm(w[4], w[5], 0x7531), SD = __byte_perm(w[6], w[7], 0x7531);
-    // kept weights in order: stored elements 8s..8s+7 = (A.first, A.second, B.first,
-    // B.second | C.first, ..., D.second): j = 2*(s&1) (+1 for C, D), byte k = position
-    const uint32_t selAB = eAB >> 8, selCD = eCD >> 8;
-    const uint32_t LAB = __byte_perm(NA, NB, selAB) & kTop;
-    const uint32_t HAB = LAB & __byte_perm(SA, SB, selAB);
-    const uint32_t LCD = __byte_perm(NC, ND, selCD) & kTop;
-    const uint32_t HCD = LCD & __byte_perm(SC, SD, selCD);
-    uint32_t word = (HAB >> js) | (LAB >> (1 + js)) | (HCD >> (2 + js)) | (LCD >> (3 + js));
-    word |= __shfl_xor_sync(0xffffffffu, word, 1);
-    if (!valid) continue;
-    const uint32_t row = fast_div((uint32_t)b, a.div_bpr);
-    const uint32_t col = (uint32_t)b - row * a.bpr;
-    uint8_t *crow = a.codes + (int64_t)row * a.ldc;
-    uint8_t *mrow = a.meta + (int64_t)row * a.ldm;
-    if ((s & 1) == 0) reinterpret_cast<uint32_t *>(crow + col * 8)[s >> 1] = word;
-    reinterpret_cast<uint16_t *>(mrow + col * 8)[s] = (uint16_t)((eAB & 0xffu) | ((eCD & 0xffu) << 8));
-    if (col == a.bpr - 1 && s == 0) {
-      if (a.ldc > a.codes_row_bytes)
-        *reinterpret_cast<uint2 *>(crow + a.codes_row_bytes) = make_uint2(0u, 0u);
-      if (a.ldm > a.meta_row_bytes)
-        *reinterpret_cast<uint2 *>(mrow + a.meta_row_bytes) = make_uint2(0u, 0u);
+    const uint32_t N0 = __byte_perm(nonzero_flags(w[0], thr2), nonzero_flags(w[1], thr2), 0x7531);
+    const uint32_t N1 = __byte_perm(nonzero_flags(w[2], thr2), nonzero_flags(w[3], thr2), 0x7531);
+    const uint32_t N2 = __byte_perm(nonzero_flags(w[4], thr2), nonzero_flags(w[5], thr2), 0x7531);
+    const uint32_t N3 = __byte_perm(nonzero_flags(w[6], thr2), nonzero_flags(w[7], thr2), 0x7531);
+    const uint32_t S0 = __byte_perm(w[0], w[1], 0x7531), S1 = __byte_perm(w[2], w[3], 0x7531);
+    const uint32_t S2 = __byte_perm(w[4], w[5], 0x7531), S3 = __byte_perm(w[6], w[7], 0x7531);
+    uint32_t word;
+    if constexpr (kCompact) {
+      // kept weights in order: stored elements 8s..8s+7 = (A.first, A.second, B.first,
+      // B.second | C.first, ..., D.second): j = 2*(s&1) (+1 for C, D), byte k = position
+      const uint32_t selAB = s_sel[m16 & 0xffu], selCD = s_sel[(m16 >> 8) & 0xffu];
+      const uint32_t LAB = __byte_perm(N0, N1, selAB) & kTop;
+      const uint32_t HAB = LAB & __byte_perm(S0, S1, selAB);
+      const uint32_t LCD = __byte_perm(N2, N3, selCD) & kTop;
+      const uint32_t HCD = LCD & __byte_perm(S2, S3, selCD);
+      word = (HAB >> js) | (LAB >> (1 + js)) | (HCD >> (2 + js)) | (LCD >> (3 + js));
+      word |= __shfl_xor_sync(0xffffffffu, word, 1);
+    } else {
+      const uint32_t L0 = N0 & nibble_to_top_bits(m16), L1 = N1 & nibble_to_top_bits(m16 >> 4);
+      const uint32_t L2 = N2 & nibble_to_top_bits(m16 >> 8),
+                     L3 = N3 & nibble_to_top_bits(m16 >> 12);
+      const uint32_t H0 = L0 & S0, H1 = L1 & S1, H2 = L2 & S2, H3 = L3 & S3;
+      // weights e = 0..15 of this lane are elements 16s+e of the block: word s, byte e%4,
+      // bits (7,6) - 2*(e/4) for (negative, non-zero)
+      word = H0 | (L0 >> 1) | (H1 >> 2) | (L1 >> 3) | (H2 >> 4) | (L2 >> 5) | (H3 >> 6) |
+             (L3 >> 7);
     }
+    if (!valid) continue;
+    const uint32_t row = fast_div(b, a.div_bpr);
+    const uint32_t col = b - row * a.bpr;
+    uint8_t *crow = a.codes + (int64_t)row * a.ldc;
+    if constexpr (kCompact) {
+      if ((s & 1) == 0) reinterpret_cast<uint32_t *>(crow + col * 8)[s >> 1] = word;
+    } else {
+      reinterpret_cast<uint32_t *>(crow + col * 16)[s] = word;
+    }
+    if (col == a.bpr - 1 && s == 0 && a.ldc > a.codes_row_bytes)
+      *reinterpret_cast<uint2 *>(crow + a.codes_row_bytes) = make_uint2(0u, 0u);
     if (a.dense_dbg) {
-      const uint32_t la = NA & KA, lb = NB & KB, lc = NC & KC, ld = ND & KD;
-      *reinterpret_cast<uint4 *>(a.dense_dbg + b * 64 + 16 * s) =
-          make_uint4(flags_to_i8(la, la & SA), flags_to_i8(lb, lb & SB), flags_to_i8(lc, lc & SC),
-                     flags_to_i8(ld, ld & SD));
+      uint32_t K0, K1, K2, K3;
+      if constexpr (kCompact) {
+        auto keep_of = [](uint32_t nib) {
+          return (0x80u << (8 * (nib & 3u))) | (0x80u << (8 * ((nib >> 2) & 3u)));
+        };
+        K0 = keep_of(m16);
+        K1 = keep_of(m16 >> 4);
+        K2 = keep_of(m16 >> 8);
+        K3 = keep_of(m16 >> 12);
+      } else {
+        K0 = nibble_to_top_bits(m16);
+        K1 = nibble_to_top_bits(m16 >> 4);
+        K2 = nibble_to_top_bits(m16 >> 8);
+        K3 = nibble_to_top_bits(m16 >> 12);
+      }
+      const uint32_t l0 = N0 & K0, l1 = N1 & K1, l2 = N2 & K2, l3 = N3 & K3;
+      *reinterpret_cast<uint4 *>(a.dense_dbg + (uint64_t)b * 64 + 16 * s) =
+          make_uint4(flags_to_i8(l0, l0 & S0), flags_to_i8(l1, l1 & S1),
+                     flags_to_i8(l2, l2 & S2), flags_to_i8(l3, l3 & S3));
     }
   }
+}
+
+template <bool kCompact>
+static sbn_status launch_two_pass(const FastPackArgs &a, int64_t grid, int32_t *err_flag,
+                                  cudaStream_t st) {
+  k_mask_sum<kCompact><<<(unsigned)grid, kPkThreads, 0, st>>>(a, err_flag);
+  SBN_LAUNCH_CHECK();
+  // pass 2 may launch while pass 1 drains (programmatic dependent launch); it waits for
+  // pass 1's completion before reading anything pass 1 wrote
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kPkThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k_codes<kCompact>, a) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  return SBN_OK;
+}
+
+// Grid of both passes: one wave of kPkCtasPerSm CTAs per SM (fewer for small tensors:
+// one warp-iteration per warp at least).
+int64_t fast_pack_parts(const FastPackArgs &a) {
+  const int64_t warp_iters = (a.nblocks + 7) / 8;
+  int64_t g = (warp_iters + kPkThreads / 32 - 1) / (kPkThreads / 32);
+  const int64_t cap = (int64_t)num_sms() * kPkCtasPerSm;
+  if (g > cap) g = cap;
+  if (g > kPackMaxParts) g = kPackMaxParts;
+  return g < 1 ? 1 : g;
+}
+
+sbn_status launch_fast_pack(const FastPackArgs &a, bool compact, int32_t *err_flag,
+                            cudaStream_t st) {
+  const int64_t g = fast_pack_parts(a);
+  if (a.nparts != g) return SBN_ERR_ARG;
+  return compact ? launch_two_pass<true>(a, g, err_flag, st)
+                 : launch_two_pass<false>(a, g, err_flag, st);
 }
 
 }  // namespace sbn

@@ -28,7 +28,7 @@ def _check_pack(W, n, m):
 
 def _linear_sampled(X, W, n, m, sample_tokens):
     got = gpu_path.linear(X, W, n, m)
-    assert got["err"] == 0
+    assert got["err"] == got["pack"]["err"] == got["quant"]["err"] == 0
     Xq, s, _ = oracle.quant_acts(X)
     assert np.array_equal(got["quant"]["Xq"], Xq)
     assert np.array_equal(got["quant"]["s"].view(np.uint32), s.view(np.uint32))

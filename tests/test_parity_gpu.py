@@ -51,6 +51,22 @@ def test_pack_exact_half_ties():
     assert got["g"] == np.float32(0.5)
 
 
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8), (3, 8)])
+def test_pack_large_magnitudes(n, m):
+    """Weights up to 255 (inside the supported range): 16 consecutive terms of
+    trunc(|W| * 2^24) overflow 32 bits, so the exact sum must not depend on a narrow
+    partial.  Rows of large values next to rows of ordinary ones, plus scattered 16.0 and
+    15.9375 (the two sides of the narrow-partial bound)."""
+    rng = np.random.default_rng(7)
+    Wf = rng.normal(0.0, 0.02, size=(300, 512)).astype(np.float32)
+    Wf[5] = rng.uniform(100.0, 255.0, size=512) * rng.choice([-1.0, 1.0], size=512)
+    Wf[200, :64] = 255.0
+    idx = rng.integers(0, Wf.size, size=40)
+    Wf.flat[idx[:20]] = 16.0
+    Wf.flat[idx[20:]] = -15.9375
+    check_pack(workloads.to_bf16_bits(Wf), n, m)
+
+
 def test_pack_all_zero_with_zero_eps():
     W = np.zeros((8, 128), np.uint16)
     got, ref = check_pack(W, 2, 4, eps=0.0)
@@ -104,7 +120,7 @@ def check_linear(T, O, K, n, m, seed, out_dtype=torch.float32, eps=1e-5):
     X = workloads.activations(T, K, seed=seed + 1)
     got = gpu_path.linear(X, W, n, m, eps, out_dtype)
     ref = oracle.linear(X, W, n, m, eps)
-    assert got["err"] == 0
+    assert got["err"] == got["pack"]["err"] == got["quant"]["err"] == 0
     assert np.array_equal(got["quant"]["Xq"], ref["Xq"])
     assert np.array_equal(got["pack"]["codes"], ref["codes"])
     assert np.array_equal(got["acc"], ref["acc"]), np.argwhere(got["acc"] != ref["acc"])[:8]
