@@ -188,9 +188,32 @@ def linear(Xq: torch.Tensor, s: torch.Tensor, w: PackedWeights, out_dtype=torch.
     return Y
 
 
+_SIDE_STREAMS = {}
+
+
+def _side_stream(device: torch.device):
+    """One auxiliary stream per device, for work that may overlap the weight pack."""
+    key = device.index if device.index is not None else torch.cuda.current_device()
+    if key not in _SIDE_STREAMS:
+        _SIDE_STREAMS[key] = torch.cuda.Stream(device=key)
+    return _SIDE_STREAMS[key]
+
+
 def forward(X: torch.Tensor, W: torch.Tensor, n: int, m: int, eps: float = 1e-5,
             out_dtype=torch.float32, workspace=None, stream=None) -> torch.Tensor:
-    """The whole Sparse-BitLinear forward: pack W, quantise X, contract and rescale."""
-    w = pack_weights(W, n, m, eps, workspace=workspace, stream=stream)
-    Xq, s = quantize_acts(X, stream=stream)
-    return linear(Xq, s, w, out_dtype, stream=stream)
+    """The whole Sparse-BitLinear forward: pack W, quantise X, contract and rescale.
+
+    The activation quantiser does not depend on the weights: it runs on an auxiliary
+    stream while the pack runs on `stream` (the current stream by default), and the
+    contraction waits for both."""
+    main = stream if stream is not None else torch.cuda.current_stream(X.device)
+    side = _side_stream(X.device)
+    side.wait_stream(main)  # X is ready on `main`
+    with torch.cuda.stream(side):
+        Xq, s = quantize_acts(X, stream=side)
+    X.record_stream(side)
+    w = pack_weights(W, n, m, eps, workspace=workspace, stream=main)
+    main.wait_stream(side)
+    Xq.record_stream(main)
+    s.record_stream(main)
+    return linear(Xq, s, w, out_dtype, stream=main)

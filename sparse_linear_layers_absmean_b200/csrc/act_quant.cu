@@ -2,8 +2,9 @@
 // modelos de lenguaje grande de 1 bit a dispositivos locales", unite.ai, "Fundamento
 // matemático" item 2; Qb = 127):
 //   s = max(max_k |x_k|, 1e-5),  q_k = clamp(rint((127 * x_k) / s), -127, 127).
-// One CTA per token.  Rows of up to 16384 inputs stay in registers between the max pass
-// and the quantise pass (one HBM read); longer rows are read twice.
+// Few tokens: one CTA per token; rows of up to 16384 inputs stay in registers between the
+// max pass and the quantise pass (one HBM read), longer rows are read twice.  Many tokens
+// with rows of up to 4096 inputs: one warp per token (k_act_quant_warp).
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -85,11 +86,55 @@ __global__ void __launch_bounds__(kAqThreads)
   for (int64_t i = threadIdx.x; i < nv; i += kAqThreads) qrow[i] = quant_vec8(__ldg(row + i), s);
 }
 
+// One warp per token for rows of up to 32 * 8 * R inputs: the whole row stays in the
+// lane's registers (R 16-byte words each, all requested at once), the max is a shuffle
+// reduction, and no CTA barrier is involved.
+template <int R>
+__global__ void __launch_bounds__(kAqThreads)
+    k_act_quant_warp(const uint4 *__restrict__ X, int64_t tokens, int64_t nv,
+                     int8_t *__restrict__ Xq, float *__restrict__ absmax, int32_t *err_flag) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * (kAqThreads / 32) + (threadIdx.x >> 5);
+  if (t >= tokens) return;  // whole warps leave together
+  const uint4 *row = X + t * nv;
+  uint4 v[R];
+  uint32_t mx = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int64_t i = lane + 32 * r;
+    v[r] = i < nv ? __ldg(row + i) : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int r = 0; r < R; ++r) mx = vec8_absmax_bits(v[r], mx);
+  const uint32_t m = warp_max_u32(max(mx & 0xffffu, mx >> 16));
+  if (m >= kBf16InfBits && lane == 0 && err_flag) atomicOr(err_flag, SBN_FLAG_X_NONFINITE);
+  const float s = fmaxf(__uint_as_float(m << 16), 1e-5f);
+  if (lane == 0) absmax[t] = s;
+  uint2 *qrow = reinterpret_cast<uint2 *>(Xq + t * nv * 8);
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int64_t i = lane + 32 * r;
+    if (i < nv) qrow[i] = quant_vec8(v[r], s);
+  }
+}
+
 sbn_status launch_act_quant(const void *X, int64_t tokens, int64_t in, int8_t *Xq,
                             float *absmax, int32_t *err_flag, cudaStream_t st) {
   const int64_t nv = in / 8;
   const uint4 *X4 = reinterpret_cast<const uint4 *>(X);
   const unsigned grid = (unsigned)tokens;
+  if (tokens > 16 && nv <= 32 * 16) {
+    // many tokens: one warp each (a CTA-wide reduction per token costs more than the row)
+    const unsigned wgrid = (unsigned)((tokens + kAqThreads / 32 - 1) / (kAqThreads / 32));
+    if (nv <= 32 * 4)
+      k_act_quant_warp<4><<<wgrid, kAqThreads, 0, st>>>(X4, tokens, nv, Xq, absmax, err_flag);
+    else if (nv <= 32 * 8)
+      k_act_quant_warp<8><<<wgrid, kAqThreads, 0, st>>>(X4, tokens, nv, Xq, absmax, err_flag);
+    else
+      k_act_quant_warp<16><<<wgrid, kAqThreads, 0, st>>>(X4, tokens, nv, Xq, absmax, err_flag);
+    SBN_LAUNCH_CHECK();
+    return SBN_OK;
+  }
   if (nv <= 2 * kAqThreads)
     k_act_quant_reg<2><<<grid, kAqThreads, 0, st>>>(X4, nv, Xq, absmax, err_flag);
   else if (nv <= 8 * kAqThreads)

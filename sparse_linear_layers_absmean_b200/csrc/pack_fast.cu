@@ -192,6 +192,37 @@ __device__ __forceinline__ void pk_load(const uint4 *W, uint32_t nb, uint32_t b,
 // each CTA leaves its partial sum in the workspace and raises the weight error flags.
 // ---------------------------------------------------------------------------------------
 template <bool kCompact>
+__device__ __forceinline__ void mask_sum_unit(const FastPackArgs &a, const uint32_t *s_meta,
+                                              uint4 v0, uint4 v1, uint32_t b, int s, double &acc0,
+                                              double &acc1, uint32_t &mx) {
+  if (b >= (uint32_t)a.nblocks) return;
+  const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    mx = vmax16(mx, w[k] & kMag);
+    acc0 = __dadd_rz(acc0, mag_lo_x2p128(w[k]));
+    acc1 = __dadd_rz(acc1, mag_hi_x2p128(w[k]));
+  }
+  uint32_t meta16;
+  if constexpr (kCompact) {
+    const uint32_t KA = keep_2of4(w[0], w[1]), KB = keep_2of4(w[2], w[3]);
+    const uint32_t KC = keep_2of4(w[4], w[5]), KD = keep_2of4(w[6], w[7]);
+    meta16 = s_meta[top_bits_to_byte(KA, KB)] | (s_meta[top_bits_to_byte(KC, KD)] << 8);
+  } else {
+    uint32_t KGA, KGB, KHA, KHB;
+    keep_6of8(w, KGA, KGB);
+    keep_6of8(w + 4, KHA, KHB);
+    meta16 = top_bits_to_byte(KGA, KGB) | (top_bits_to_byte(KHA, KHB) << 8);
+  }
+  const uint32_t row = fast_div(b, a.div_bpr);
+  const uint32_t col = b - row * a.bpr;
+  uint8_t *mrow = a.meta + (int64_t)row * a.ldm;
+  reinterpret_cast<uint16_t *>(mrow + col * 8)[s] = (uint16_t)meta16;
+  if (s == 0 && col == a.bpr - 1 && a.ldm > a.meta_row_bytes)
+    *reinterpret_cast<uint2 *>(mrow + a.meta_row_bytes) = make_uint2(0u, 0u);
+}
+
+template <bool kCompact>
 __global__ void __launch_bounds__(kPkThreads, kPkCtasPerSm)
     k_mask_sum(const FastPackArgs a, int32_t *err_flag) {
   __shared__ uint32_t s_meta[256];  // 2:4: keep byte of two groups -> their meta byte
@@ -204,49 +235,25 @@ __global__ void __launch_bounds__(kPkThreads, kPkCtasPerSm)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int s = lane & 3;
   const uint32_t nb = (uint32_t)a.nblocks;
-  const uint32_t nwarps = gridDim.x * (kPkThreads / 32);
-  const uint32_t bstep = 8 * nwarps;
-  uint32_t b = 8 * (blockIdx.x * (kPkThreads / 32) + warp) + (lane >> 2);
+  const uint32_t bstep = 8 * gridDim.x * (kPkThreads / 32);
+  const uint32_t first = 8 * (blockIdx.x * (kPkThreads / 32) + warp);  // warp-uniform
+  const uint32_t sub = lane >> 2;
   double acc0 = kAccBias, acc1 = kAccBias;
   uint32_t mx = 0;  // largest magnitude bits seen, per 16-bit half
-  uint4 n0, n1;
-  pk_load(a.W, nb, b, s, n0, n1);
-  for (; b - (lane >> 2) < nb; b += bstep) {  // warp-uniform: the warp's first block
-    const uint4 v0 = n0, v1 = n1;
-    pk_load(a.W, nb, b + bstep, s, n0, n1);
-    if (b >= nb) continue;
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      mx = vmax16(mx, w[k] & kMag);
-      acc0 = __dadd_rz(acc0, mag_lo_x2p128(w[k]));
-      acc1 = __dadd_rz(acc1, mag_hi_x2p128(w[k]));
-    }
-    uint32_t meta16;
-    if constexpr (kCompact) {
-      const uint32_t KA = keep_2of4(w[0], w[1]), KB = keep_2of4(w[2], w[3]);
-      const uint32_t KC = keep_2of4(w[4], w[5]), KD = keep_2of4(w[6], w[7]);
-      meta16 = s_meta[top_bits_to_byte(KA, KB)] | (s_meta[top_bits_to_byte(KC, KD)] << 8);
-    } else {
-      uint32_t KGA, KGB, KHA, KHB;
-      keep_6of8(w, KGA, KGB);
-      keep_6of8(w + 4, KHA, KHB);
-      meta16 = top_bits_to_byte(KGA, KGB) | (top_bits_to_byte(KHA, KHB) << 8);
-    }
-    const uint32_t row = fast_div(b, a.div_bpr);
-    const uint32_t col = b - row * a.bpr;
-    uint8_t *mrow = a.meta + (int64_t)row * a.ldm;
-    reinterpret_cast<uint16_t *>(mrow + col * 8)[s] = (uint16_t)meta16;
-    if (s == 0 && col == a.bpr - 1 && a.ldm > a.meta_row_bytes)
-      *reinterpret_cast<uint2 *>(mrow + a.meta_row_bytes) = make_uint2(0u, 0u);
+  // two warp-iterations per loop trip: four 16-byte loads in flight per lane
+  for (uint32_t base = first; base < nb; base += 2 * bstep) {
+    uint4 p0, p1, q0, q1;
+    pk_load(a.W, nb, base + sub, s, p0, p1);
+    pk_load(a.W, nb, base + bstep + sub, s, q0, q1);
+    mask_sum_unit<kCompact>(a, s_meta, p0, p1, base + sub, s, acc0, acc1, mx);
+    mask_sum_unit<kCompact>(a, s_meta, q0, q1, base + bstep + sub, s, acc0, acc1, mx);
   }
   unsigned long long sum = acc_value(acc0) + acc_value(acc1);
   // Rare path: some |W| >= 256 (or NaN/Inf).  Re-read this lane's weights to tell the two
   // error kinds apart.
   uint32_t mx_all = 0, mx_fin = 0;
   if (max(mx & 0xffffu, mx >> 16) >= kBf16Mag256Bits) {
-    for (uint32_t bb = 8 * (blockIdx.x * (kPkThreads / 32) + warp) + (lane >> 2); bb < nb;
-         bb += bstep) {
+    for (uint32_t bb = first + sub; bb < nb; bb += bstep) {
       uint4 v0, v1;
       pk_load(a.W, nb, bb, s, v0, v1);
       const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
@@ -300,90 +307,99 @@ __device__ __forceinline__ uint32_t meta_of(const FastPackArgs &a, uint32_t nb, 
 // Pass 2: codes.  Each lane requests its first W words at once (W does not depend on
 // pass 1; after pass 1 they are mostly L2 hits), then the CTA waits for pass 1 to
 // complete, finishes the scale (pack_prologue) and stores the 2-bit codes of the kept
-// weights, with the next iteration's W words and metadata requested ahead.
+// weights.
 // ---------------------------------------------------------------------------------------
+template <bool kCompact>
+__device__ __forceinline__ void codes_unit(const FastPackArgs &a, const uint32_t *s_sel, uint4 v0,
+                                           uint4 v1, uint32_t m16, uint32_t b, int s,
+                                           uint32_t thr2) {
+  const bool valid = b < (uint32_t)a.nblocks;  // both lanes of a shuffle pair share the block
+  const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  const uint32_t N0 = __byte_perm(nonzero_flags(w[0], thr2), nonzero_flags(w[1], thr2), 0x7531);
+  const uint32_t N1 = __byte_perm(nonzero_flags(w[2], thr2), nonzero_flags(w[3], thr2), 0x7531);
+  const uint32_t N2 = __byte_perm(nonzero_flags(w[4], thr2), nonzero_flags(w[5], thr2), 0x7531);
+  const uint32_t N3 = __byte_perm(nonzero_flags(w[6], thr2), nonzero_flags(w[7], thr2), 0x7531);
+  const uint32_t S0 = __byte_perm(w[0], w[1], 0x7531), S1 = __byte_perm(w[2], w[3], 0x7531);
+  const uint32_t S2 = __byte_perm(w[4], w[5], 0x7531), S3 = __byte_perm(w[6], w[7], 0x7531);
+  uint32_t word;
+  if constexpr (kCompact) {
+    // kept weights in order: stored elements 8s..8s+7 = (A.first, A.second, B.first,
+    // B.second | C.first, ..., D.second): j = 2*(s&1) (+1 for C, D), byte k = position
+    const int js = 4 * (s & 1);
+    const uint32_t selAB = s_sel[m16 & 0xffu], selCD = s_sel[(m16 >> 8) & 0xffu];
+    const uint32_t LAB = __byte_perm(N0, N1, selAB) & kTop;
+    const uint32_t HAB = LAB & __byte_perm(S0, S1, selAB);
+    const uint32_t LCD = __byte_perm(N2, N3, selCD) & kTop;
+    const uint32_t HCD = LCD & __byte_perm(S2, S3, selCD);
+    word = (HAB >> js) | (LAB >> (1 + js)) | (HCD >> (2 + js)) | (LCD >> (3 + js));
+    word |= __shfl_xor_sync(0xffffffffu, word, 1);
+  } else {
+    const uint32_t L0 = N0 & nibble_to_top_bits(m16), L1 = N1 & nibble_to_top_bits(m16 >> 4);
+    const uint32_t L2 = N2 & nibble_to_top_bits(m16 >> 8), L3 = N3 & nibble_to_top_bits(m16 >> 12);
+    const uint32_t H0 = L0 & S0, H1 = L1 & S1, H2 = L2 & S2, H3 = L3 & S3;
+    // weights e = 0..15 of this lane are elements 16s+e of the block: word s, byte e%4,
+    // bits (7,6) - 2*(e/4) for (negative, non-zero)
+    word = H0 | (L0 >> 1) | (H1 >> 2) | (L1 >> 3) | (H2 >> 4) | (L2 >> 5) | (H3 >> 6) | (L3 >> 7);
+  }
+  if (!valid) return;
+  const uint32_t row = fast_div(b, a.div_bpr);
+  const uint32_t col = b - row * a.bpr;
+  uint8_t *crow = a.codes + (int64_t)row * a.ldc;
+  if constexpr (kCompact) {
+    if ((s & 1) == 0) reinterpret_cast<uint32_t *>(crow + col * 8)[s >> 1] = word;
+  } else {
+    reinterpret_cast<uint32_t *>(crow + col * 16)[s] = word;
+  }
+  if (col == a.bpr - 1 && s == 0 && a.ldc > a.codes_row_bytes)
+    *reinterpret_cast<uint2 *>(crow + a.codes_row_bytes) = make_uint2(0u, 0u);
+  if (a.dense_dbg) {
+    uint32_t K0, K1, K2, K3;
+    if constexpr (kCompact) {
+      auto keep_of = [](uint32_t nib) {
+        return (0x80u << (8 * (nib & 3u))) | (0x80u << (8 * ((nib >> 2) & 3u)));
+      };
+      K0 = keep_of(m16);
+      K1 = keep_of(m16 >> 4);
+      K2 = keep_of(m16 >> 8);
+      K3 = keep_of(m16 >> 12);
+    } else {
+      K0 = nibble_to_top_bits(m16);
+      K1 = nibble_to_top_bits(m16 >> 4);
+      K2 = nibble_to_top_bits(m16 >> 8);
+      K3 = nibble_to_top_bits(m16 >> 12);
+    }
+    const uint32_t l0 = N0 & K0, l1 = N1 & K1, l2 = N2 & K2, l3 = N3 & K3;
+    *reinterpret_cast<uint4 *>(a.dense_dbg + (uint64_t)b * 64 + 16 * s) =
+        make_uint4(flags_to_i8(l0, l0 & S0), flags_to_i8(l1, l1 & S1), flags_to_i8(l2, l2 & S2),
+                   flags_to_i8(l3, l3 & S3));
+  }
+}
+
 template <bool kCompact>
 __global__ void __launch_bounds__(kPkThreads, kPkCtasPerSm) k_codes(const FastPackArgs a) {
   __shared__ uint32_t s_sel[256];  // 2:4: meta byte -> compaction selector
   if (kCompact) s_sel[threadIdx.x] = compact_selector(threadIdx.x);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int s = lane & 3;
-  const int js = 4 * (s & 1);  // 2:4: 2j of stored elements 8s..8s+3 (j = 2*(s&1))
   const uint32_t nb = (uint32_t)a.nblocks;
   const uint32_t bstep = 8 * gridDim.x * (kPkThreads / 32);
-  uint32_t b = 8 * (blockIdx.x * (kPkThreads / 32) + warp) + (lane >> 2);
-  uint4 n0, n1;
-  pk_load(a.W, nb, b, s, n0, n1);
+  const uint32_t first = 8 * (blockIdx.x * (kPkThreads / 32) + warp);  // warp-uniform
+  const uint32_t sub = lane >> 2;
+  uint4 p0, p1, q0, q1;
+  pk_load(a.W, nb, first + sub, s, p0, p1);
+  pk_load(a.W, nb, first + bstep + sub, s, q0, q1);
   ptx::grid_dep_wait();  // pass 1 complete: partial sums and metadata visible
   const uint32_t thr = pack_prologue(a.ws, a.nparts, a.n, a.eps, a.gamma_eff);  // syncs
   const uint32_t thr2 = thr | (thr << 16);
-  uint32_t nm = meta_of(a, nb, b, s);
-  for (; b - (lane >> 2) < nb; b += bstep) {  // warp-uniform: the warp's first block
-    const uint4 v0 = n0, v1 = n1;
-    const uint32_t m16 = nm;
-    pk_load(a.W, nb, b + bstep, s, n0, n1);
-    nm = meta_of(a, nb, b + bstep, s);
-    const bool valid = b < nb;  // both lanes of a shuffle pair share the block
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    const uint32_t N0 = __byte_perm(nonzero_flags(w[0], thr2), nonzero_flags(w[1], thr2), 0x7531);
-    const uint32_t N1 = __byte_perm(nonzero_flags(w[2], thr2), nonzero_flags(w[3], thr2), 0x7531);
-    const uint32_t N2 = __byte_perm(nonzero_flags(w[4], thr2), nonzero_flags(w[5], thr2), 0x7531);
-    const uint32_t N3 = __byte_perm(nonzero_flags(w[6], thr2), nonzero_flags(w[7], thr2), 0x7531);
-    const uint32_t S0 = __byte_perm(w[0], w[1], 0x7531), S1 = __byte_perm(w[2], w[3], 0x7531);
-    const uint32_t S2 = __byte_perm(w[4], w[5], 0x7531), S3 = __byte_perm(w[6], w[7], 0x7531);
-    uint32_t word;
-    if constexpr (kCompact) {
-      // kept weights in order: stored elements 8s..8s+7 = (A.first, A.second, B.first,
-      // B.second | C.first, ..., D.second): j = 2*(s&1) (+1 for C, D), byte k = position
-      const uint32_t selAB = s_sel[m16 & 0xffu], selCD = s_sel[(m16 >> 8) & 0xffu];
-      const uint32_t LAB = __byte_perm(N0, N1, selAB) & kTop;
-      const uint32_t HAB = LAB & __byte_perm(S0, S1, selAB);
-      const uint32_t LCD = __byte_perm(N2, N3, selCD) & kTop;
-      const uint32_t HCD = LCD & __byte_perm(S2, S3, selCD);
-      word = (HAB >> js) | (LAB >> (1 + js)) | (HCD >> (2 + js)) | (LCD >> (3 + js));
-      word |= __shfl_xor_sync(0xffffffffu, word, 1);
-    } else {
-      const uint32_t L0 = N0 & nibble_to_top_bits(m16), L1 = N1 & nibble_to_top_bits(m16 >> 4);
-      const uint32_t L2 = N2 & nibble_to_top_bits(m16 >> 8),
-                     L3 = N3 & nibble_to_top_bits(m16 >> 12);
-      const uint32_t H0 = L0 & S0, H1 = L1 & S1, H2 = L2 & S2, H3 = L3 & S3;
-      // weights e = 0..15 of this lane are elements 16s+e of the block: word s, byte e%4,
-      // bits (7,6) - 2*(e/4) for (negative, non-zero)
-      word = H0 | (L0 >> 1) | (H1 >> 2) | (L1 >> 3) | (H2 >> 4) | (L2 >> 5) | (H3 >> 6) |
-             (L3 >> 7);
-    }
-    if (!valid) continue;
-    const uint32_t row = fast_div(b, a.div_bpr);
-    const uint32_t col = b - row * a.bpr;
-    uint8_t *crow = a.codes + (int64_t)row * a.ldc;
-    if constexpr (kCompact) {
-      if ((s & 1) == 0) reinterpret_cast<uint32_t *>(crow + col * 8)[s >> 1] = word;
-    } else {
-      reinterpret_cast<uint32_t *>(crow + col * 16)[s] = word;
-    }
-    if (col == a.bpr - 1 && s == 0 && a.ldc > a.codes_row_bytes)
-      *reinterpret_cast<uint2 *>(crow + a.codes_row_bytes) = make_uint2(0u, 0u);
-    if (a.dense_dbg) {
-      uint32_t K0, K1, K2, K3;
-      if constexpr (kCompact) {
-        auto keep_of = [](uint32_t nib) {
-          return (0x80u << (8 * (nib & 3u))) | (0x80u << (8 * ((nib >> 2) & 3u)));
-        };
-        K0 = keep_of(m16);
-        K1 = keep_of(m16 >> 4);
-        K2 = keep_of(m16 >> 8);
-        K3 = keep_of(m16 >> 12);
-      } else {
-        K0 = nibble_to_top_bits(m16);
-        K1 = nibble_to_top_bits(m16 >> 4);
-        K2 = nibble_to_top_bits(m16 >> 8);
-        K3 = nibble_to_top_bits(m16 >> 12);
-      }
-      const uint32_t l0 = N0 & K0, l1 = N1 & K1, l2 = N2 & K2, l3 = N3 & K3;
-      *reinterpret_cast<uint4 *>(a.dense_dbg + (uint64_t)b * 64 + 16 * s) =
-          make_uint4(flags_to_i8(l0, l0 & S0), flags_to_i8(l1, l1 & S1),
-                     flags_to_i8(l2, l2 & S2), flags_to_i8(l3, l3 & S3));
-    }
+  // two warp-iterations per loop trip: four 16-byte loads in flight per lane
+  for (uint32_t base = first;;) {
+    const uint32_t mp = meta_of(a, nb, base + sub, s), mq = meta_of(a, nb, base + bstep + sub, s);
+    codes_unit<kCompact>(a, s_sel, p0, p1, mp, base + sub, s, thr2);
+    codes_unit<kCompact>(a, s_sel, q0, q1, mq, base + bstep + sub, s, thr2);
+    base += 2 * bstep;
+    if (base >= nb) break;
+    pk_load(a.W, nb, base + sub, s, p0, p1);
+    pk_load(a.W, nb, base + bstep + sub, s, q0, q1);
   }
 }
 

@@ -96,8 +96,11 @@ def test_pack_flags_bad_weights(bad, flag):
 
 
 @pytest.mark.parametrize("T,K", [(1, 64), (3, 256), (8, 2560), (37, 4096), (5, 11008),
-                                 (2, 20480)])
+                                 (2, 20480), (17, 64), (300, 1024), (101, 2048), (40, 4160),
+                                 (1000, 3200)])
 def test_act_quant(T, K):
+    """Few tokens take the one-CTA-per-token kernel, many tokens with rows up to 4096 the
+    one-warp-per-token kernel (ragged last CTA in each case)."""
     X = workloads.activations(T, K, seed=T * K)
     X[0, :7] = workloads.to_bf16_bits(np.array([0.5, -0.5, 1.5, 2.5, -2.5, 0, -0.0], np.float32))
     if T > 2:
@@ -109,9 +112,13 @@ def test_act_quant(T, K):
     assert np.array_equal(got["Xq"], Xq)
 
 
-def test_act_quant_flags_nonfinite():
-    X = workloads.activations(4, 256, seed=5)
+@pytest.mark.parametrize("T", [4, 100])
+def test_act_quant_flags_nonfinite(T):
+    X = workloads.activations(T, 256, seed=5)
     X[2, 9] = workloads.to_bf16_bits(np.array([np.nan], np.float32))[0]
+    assert gpu_path.quant(X)["err"] == 4
+    X = workloads.activations(T, 256, seed=6)
+    X[T - 1, 200] = workloads.to_bf16_bits(np.array([-np.inf], np.float32))[0]
     assert gpu_path.quant(X)["err"] == 4
 
 
@@ -170,3 +177,22 @@ def test_linear_zero_token_row_gives_zero():
     X[3] = 0
     got = gpu_path.linear(X, W, 2, 4)
     assert (got["y"][3] == 0).all() and (got["acc"][3] == 0).all()
+
+
+@pytest.mark.parametrize("T,n,m", [(1, 6, 8), (8, 2, 4), (300, 2, 4), (40, 6, 8)])
+def test_forward_public_api(T, n, m):
+    """sbn.forward (activation quantiser on a side stream, pack on the caller's stream)
+    against the oracle, on a non-default caller stream."""
+    import sparse_linear_layers_absmean_b200 as sbn
+    O, K = 300, 512
+    W_bits = workloads.masters(O, K, seed=T + n)
+    X_bits = workloads.activations(T, K, seed=T + m)
+    ref = oracle.linear(X_bits, W_bits, n, m, 1e-5)
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):
+        W = workloads.torch_bf16(W_bits, "cuda")
+        X = workloads.torch_bf16(X_bits, "cuda")
+        Y = sbn.forward(X, W, n, m)
+        del W, X  # freed while the side stream may still read X: record_stream keeps it
+        y = Y.cpu().numpy()
+    gpu_path.assert_y_close(y, ref["y"])
