@@ -13,22 +13,32 @@ namespace sbn {
 
 constexpr int kGvThreads = 128;
 
-// prmt selector that gathers the kept activations of two 2:4 groups: meta byte
-// (i0A | i1A << 2 | i0B << 4 | i1B << 6) -> byte selectors i0A, i1A, 4 + i0B, 4 + i1B.
-__device__ __forceinline__ uint32_t pair_selector(uint32_t mb) {
-  return (mb & 3u) | (((mb >> 2) & 3u) << 4) | ((((mb >> 4) & 3u) + 4u) << 8) |
-         ((((mb >> 6) & 3u) + 4u) << 12);
+// prmt selectors that gather the kept activations of 2:4 groups, two at a time: each meta
+// byte (i0A | i1A << 2 | i0B << 4 | i1B << 6) becomes the 16-bit selector with nibbles
+// i0A, i1A, 4 + i0B, 4 + i1B.  For meta bytes b0, b1 in the low 16 bits of m, the result
+// holds the selector of b0 in bits 0-15 and that of b1 in bits 16-31 (prmt reads the low
+// 16 bits of its selector): every 2-bit field is spread to its own nibble.
+__device__ __forceinline__ uint32_t pair_selectors(uint32_t m) {
+  uint32_t x = m & 0xffffu;
+  x = (x | (x << 8)) & 0x00ff00ffu;
+  x = (x | (x << 4)) & 0x0f0f0f0fu;
+  x = (x | (x << 2)) & 0x33333333u;
+  return x + 0x44004400u;
 }
 
 // Two output rows per warp (rows 2w and 2w + 1), every row in one round: enough CTAs for
-// all rows at once, so the whole codes plane is requested in one wave.  Lane l takes the
-// 64-weight chunks l, l+32, ... (at most CPL per pass) of both rows; the per-token scales
-// are requested first, then both rows' code (and 2:4 metadata) words, then the activation
-// words (through L1: every warp of an SM reads the same few KB), each used for both rows.
-// The warp reduces with shuffles and lane t writes token t of each row.
+// all rows at once, so the whole codes plane is requested in one wave.  The row is cut
+// into segments of 32 code words (one per lane): for 6:8 / dense codes a word holds 16
+// weights and the lane's activations are the 16 bytes at 16 l of the 512-input segment;
+// for 2:4 a word holds the 16 kept codes of 32 inputs with one metadata word beside it,
+// and the lane's activations are the 32 bytes at 32 l of the 1024-input segment.  Both
+// code and activation loads are contiguous across the warp.  SPL segments are requested
+// per pass (the per-token scales first, then both rows' code and metadata words, then the
+// activations, each used for both rows); the warp reduces with shuffles and lane t writes
+// token t of each row.
 constexpr int kGvRows = 2;
 
-template <int T, int CPL, bool kCompact>
+template <int T, int SPL, bool kCompact>
 __global__ void __launch_bounds__(kGvThreads)
     k_gemv(const int8_t *__restrict__ Xq, const float *__restrict__ absmax,
            const uint8_t *__restrict__ codes, const uint8_t *__restrict__ meta,
@@ -39,78 +49,56 @@ __global__ void __launch_bounds__(kGvThreads)
   if (row0 >= out) return;  // whole warps leave together
   const bool two = row0 + 1 < out;
   const float c = lane < T ? rescale_factor(__ldg(gamma_eff), __ldg(absmax + lane)) : 0.0f;
-  const int nchunks = (int)(in / 64);
+  const int nwords = (int)(in / (kCompact ? 32 : 16));  // code words per row
+  const uint32_t *crow[kGvRows], *mrow[kGvRows];
+#pragma unroll
+  for (int r = 0; r < kGvRows; ++r) {
+    const int64_t row = row0 + (two ? r : 0);
+    crow[r] = reinterpret_cast<const uint32_t *>(codes + row * ldc);
+    mrow[r] = reinterpret_cast<const uint32_t *>(meta + row * ldm);
+  }
   int acc[kGvRows][T];
 #pragma unroll
   for (int r = 0; r < kGvRows; ++r)
 #pragma unroll
     for (int t = 0; t < T; ++t) acc[r][t] = 0;
-  for (int c0 = 0; c0 < nchunks; c0 += 32 * CPL) {  // one pass unless in > 2048 * CPL
-    if constexpr (!kCompact) {
-      uint4 cw[kGvRows][CPL];
+  for (int w0 = 0; w0 < nwords; w0 += 32 * SPL) {  // one pass for rows up to 32 * SPL words
+    uint32_t cw[kGvRows][SPL], mw[kGvRows][SPL];
 #pragma unroll
-      for (int r = 0; r < kGvRows; ++r) {
-        const uint4 *crow = reinterpret_cast<const uint4 *>(codes + (row0 + (two ? r : 0)) * ldc);
+    for (int r = 0; r < kGvRows; ++r)
 #pragma unroll
-        for (int i = 0; i < CPL; ++i)
-          cw[r][i] = c0 + lane + 32 * i < nchunks ? __ldg(crow + c0 + lane + 32 * i)
-                                                  : make_uint4(0, 0, 0, 0);
+      for (int i = 0; i < SPL; ++i) {
+        const int wi = w0 + 32 * i + lane;
+        cw[r][i] = wi < nwords ? __ldg(crow[r] + wi) : 0u;
+        if constexpr (kCompact) mw[r][i] = wi < nwords ? __ldg(mrow[r] + wi) : 0u;
       }
 #pragma unroll
-      for (int i = 0; i < CPL; ++i) {
-        const int ch = c0 + lane + 32 * i;
-        if (ch >= nchunks) continue;
+    for (int i = 0; i < SPL; ++i) {
+      const int wi = w0 + 32 * i + lane;
+      if (wi >= nwords) continue;
 #pragma unroll
-        for (int t = 0; t < T; ++t) {
-          const uint4 *xs = reinterpret_cast<const uint4 *>(Xq + t * in + (int64_t)ch * 64);
+      for (int t = 0; t < T; ++t) {
+        if constexpr (!kCompact) {
+          const uint4 x4 = __ldg(reinterpret_cast<const uint4 *>(Xq + t * in + (int64_t)wi * 16));
+          const uint32_t xw[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 x4 = __ldg(xs + q);
-            const uint32_t xw[4] = {x4.x, x4.y, x4.z, x4.w};
+          for (int r = 0; r < kGvRows; ++r)
 #pragma unroll
-            for (int r = 0; r < kGvRows; ++r) {
-              const uint32_t w4[4] = {cw[r][i].x, cw[r][i].y, cw[r][i].z, cw[r][i].w};
+            for (int j = 0; j < 4; ++j)  // weights 4j..4j+3 sit in bits 7-2j..6-2j of the bytes
+              acc[r][t] = __dp4a((int)((cw[r][i] << (2 * j)) & 0xC0C0C0C0u), (int)xw[j], acc[r][t]);
+        } else {
+          const uint4 *xs = reinterpret_cast<const uint4 *>(Xq + t * in + (int64_t)wi * 32);
+          const uint4 xa = __ldg(xs), xb = __ldg(xs + 1);
+          const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
 #pragma unroll
-              for (int j = 0; j < 4; ++j)
-                acc[r][t] = __dp4a((int)((w4[q] << (2 * j)) & 0xC0C0C0C0u), (int)xw[j], acc[r][t]);
-            }
-          }
-        }
-      }
-    } else {
-      uint2 cw[kGvRows][CPL], mw[kGvRows][CPL];
+          for (int r = 0; r < kGvRows; ++r) {
+            // selectors of groups (0,1), (2,3) | (4,5), (6,7); the same for every token
+            const uint32_t s01 = pair_selectors(mw[r][i]), s23 = pair_selectors(mw[r][i] >> 16);
+            const uint32_t sel[4] = {s01, s01 >> 16, s23, s23 >> 16};
 #pragma unroll
-      for (int r = 0; r < kGvRows; ++r) {
-        const int64_t row = row0 + (two ? r : 0);
-        const uint2 *crow = reinterpret_cast<const uint2 *>(codes + row * ldc);
-        const uint2 *mrow = reinterpret_cast<const uint2 *>(meta + row * ldm);
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-          const bool ok = c0 + lane + 32 * i < nchunks;
-          cw[r][i] = ok ? __ldg(crow + c0 + lane + 32 * i) : make_uint2(0, 0);
-          mw[r][i] = ok ? __ldg(mrow + c0 + lane + 32 * i) : make_uint2(0, 0);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < CPL; ++i) {
-        const int ch = c0 + lane + 32 * i;
-        if (ch >= nchunks) continue;
-#pragma unroll
-        for (int t = 0; t < T; ++t) {
-          const uint4 *xs = reinterpret_cast<const uint4 *>(Xq + t * in + (int64_t)ch * 64);
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {  // 32 stored codes = 8 groups = 32 positions
-            const uint4 xa = __ldg(xs + 2 * q), xb = __ldg(xs + 2 * q + 1);
-            const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-#pragma unroll
-            for (int r = 0; r < kGvRows; ++r) {
-              const uint32_t w2 = q ? cw[r][i].y : cw[r][i].x, m2 = q ? mw[r][i].y : mw[r][i].x;
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const uint32_t sel = pair_selector((m2 >> (8 * j)) & 0xffu);
-                const uint32_t xk = __byte_perm(xw[2 * j], xw[2 * j + 1], sel);
-                acc[r][t] = __dp4a((int)((w2 << (2 * j)) & 0xC0C0C0C0u), (int)xk, acc[r][t]);
-              }
+            for (int j = 0; j < 4; ++j) {  // groups 2j, 2j+1: stored codes 4j..4j+3
+              const uint32_t xk = __byte_perm(xw[2 * j], xw[2 * j + 1], sel[j]);
+              acc[r][t] = __dp4a((int)((cw[r][i] << (2 * j)) & 0xC0C0C0C0u), (int)xk, acc[r][t]);
             }
           }
         }
@@ -144,14 +132,14 @@ __global__ void __launch_bounds__(kGvThreads)
   }
 }
 
-template <int T, int CPL>
+template <int T, int SPL>
 static sbn_status gemv_tc(const int8_t *Xq, const float *absmax, const uint8_t *codes,
                           const uint8_t *meta, const float *gamma_eff, int64_t out, int64_t in,
                           bool compact, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
                           int32_t *acc_dbg, cudaStream_t st) {
   const int64_t rows_per_cta = kGvRows * (kGvThreads / 32);
   const int64_t grid = (out + rows_per_cta - 1) / rows_per_cta;
-  auto kern = compact ? k_gemv<T, CPL, true> : k_gemv<T, CPL, false>;
+  auto kern = compact ? k_gemv<T, SPL, true> : k_gemv<T, SPL, false>;
   kern<<<(unsigned)grid, kGvThreads, 0, st>>>(Xq, absmax, codes, meta, gamma_eff, out, in, ldc,
                                               ldm, Y, y_is_bf16, acc_dbg);
   SBN_LAUNCH_CHECK();
@@ -163,15 +151,16 @@ static sbn_status gemv_t(const int8_t *Xq, const float *absmax, const uint8_t *c
                          const uint8_t *meta, const float *gamma_eff, int64_t out, int64_t in,
                          bool compact, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
                          int32_t *acc_dbg, cudaStream_t st) {
-  const int64_t cpl = (in / 64 + 31) / 32;
-  if (cpl <= 1)
-    return gemv_tc<T, 1>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
-                         y_is_bf16, acc_dbg, st);
-  if (cpl <= 2)
+  const int64_t words = in / (compact ? 32 : 16);  // code words per row
+  const int64_t spl = (words + 31) / 32;
+  if (spl <= 2)
     return gemv_tc<T, 2>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
                          y_is_bf16, acc_dbg, st);
-  if (cpl <= 4)
+  if (spl <= 4)
     return gemv_tc<T, 4>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
+                         y_is_bf16, acc_dbg, st);
+  if (spl <= 6 || T > 2)
+    return gemv_tc<T, 6>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
                          y_is_bf16, acc_dbg, st);
   return gemv_tc<T, 8>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
                        y_is_bf16, acc_dbg, st);

@@ -48,18 +48,15 @@ struct FastPackArgs {
   uint8_t *meta;
   int64_t ldm, meta_row_bytes;
   int8_t *dense_dbg;
-  int nparts;       // partial sums left by the first pass
+  int nparts;       // partial sums left by k_abs_sum
   int64_t n;        // weights in the tensor
   float eps;
   float *gamma_eff;  // written by CTA 0
 };
 
-// 6:8 (compact false) and 2:4 (compact true) in two launches: pass 1 writes the metadata
-// plane and fast_pack_parts(a) exact partial sums (a.nparts must equal that), pass 2
-// finishes the scale and writes the codes plane.
-int64_t fast_pack_parts(const FastPackArgs &a);
-sbn_status launch_fast_pack(const FastPackArgs &a, bool compact, int32_t *err_flag,
-                            cudaStream_t st);
+// 6:8 (compact false) and 2:4 (compact true): the keep masks, metadata and codes in one
+// launch after k_abs_sum left a.nparts partial sums in a.ws.
+sbn_status launch_fast_pack(const FastPackArgs &a, bool compact, cudaStream_t st);
 
 sbn_status launch_pack(const void *W, int64_t out, int64_t in, int n, int m, float eps,
                        uint8_t *codes, int64_t ldc, int64_t crow, uint8_t *meta, int64_t ldm,

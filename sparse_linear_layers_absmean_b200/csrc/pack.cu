@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "kernels.cuh"
 #include "pack_common.cuh"
+#include "ptx.cuh"
 
 namespace sbn {
 
@@ -22,33 +23,37 @@ namespace sbn {
 // S1: per-tensor absmean scale.
 // ---------------------------------------------------------------------------------------
 
-__global__ void __launch_bounds__(256) k_abs_sum(const uint4 *__restrict__ W, int64_t nvec,
-                                                 PackWorkspace *ws, int32_t *err_flag) {
-  unsigned long long acc = 0;
+// One pass over W at the full HBM bandwidth: four CTAs of 256 threads per SM, four 16-byte
+// loads in flight per thread, one fp64 add per weight (pack_common.cuh) and a packed
+// 16-bit max for the range check.  One partial sum per CTA goes to the workspace.
+constexpr int kAsThreads = 256;
+constexpr int kAsLoads = 4;
+
+__global__ void __launch_bounds__(kAsThreads, 4) k_abs_sum(const uint4 *__restrict__ W, int64_t nvec,
+                                                         PackWorkspace *ws, int32_t *err_flag) {
+  // the quant/mask/pack kernel may start launching; it waits for this one's results
+  ptx::grid_dep_launch();
+  double acc0 = kAccBias, acc1 = kAccBias;
   uint32_t mx = 0;  // largest magnitude bits seen, per 16-bit half
-  auto consume = [&](const uint4 &v) {
-    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint32_t a = w4[q] & 0x7fff7fffu;  // |W| of both halves
-      asm("max.u16x2 %0, %0, %1;" : "+r"(mx) : "r"(a));
-      // |W| * 2^24 is exact in fp32; the conversion truncates toward zero.
-      const float lo = __fmul_rn(__uint_as_float(a << 16), 16777216.0f);
-      const float hi = __fmul_rn(__uint_as_float(a & 0xffff0000u), 16777216.0f);
-      acc += (unsigned long long)__float2uint_rz(lo) + __float2uint_rz(hi);
-    }
-  };
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  int64_t i = i0;
-  for (; i < nvec; i += 8 * stride) {  // up to eight 16-byte loads in flight per round
-    uint4 v[8];
+  for (int64_t i = i0; i < nvec; i += kAsLoads * stride) {
+    uint4 v[kAsLoads];
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
+    for (int u = 0; u < kAsLoads; ++u)
       v[u] = i + u * stride < nvec ? __ldg(W + i + u * stride) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) consume(v[u]);  // zero words add nothing
+    for (int u = 0; u < kAsLoads; ++u) {  // zero words add nothing
+      const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        asm("max.u16x2 %0, %0, %1;" : "+r"(mx) : "r"(w4[q] & 0x7fff7fffu));
+        acc0 = __dadd_rz(acc0, mag_lo_x2p128(w4[q]));
+        acc1 = __dadd_rz(acc1, mag_hi_x2p128(w4[q]));
+      }
+    }
   }
+  unsigned long long acc = acc_value(acc0) + acc_value(acc1);
   // Rare path: some |W| >= 256 (or NaN/Inf).  Re-read this thread's weights to tell the
   // two error kinds apart.
   uint32_t mx_all = 0, mx_fin = 0;
@@ -64,8 +69,8 @@ __global__ void __launch_bounds__(256) k_abs_sum(const uint4 *__restrict__ W, in
         }
     }
   }
-  __shared__ unsigned long long s_sum[8];
-  __shared__ uint32_t s_all[8], s_fin[8];
+  __shared__ unsigned long long s_sum[kAsThreads / 32];
+  __shared__ uint32_t s_all[kAsThreads / 32], s_fin[kAsThreads / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   acc = warp_sum_u64(acc);
   uint32_t ma = warp_max_u32(mx_all);
@@ -79,7 +84,7 @@ __global__ void __launch_bounds__(256) k_abs_sum(const uint4 *__restrict__ W, in
   if (threadIdx.x == 0) {
     unsigned long long sum = 0;
     uint32_t a = 0, f = 0;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+    for (int w = 0; w < kAsThreads / 32; ++w) {
       sum += s_sum[w];
       a = max(a, s_all[w]);
       f = max(f, s_fin[w]);
@@ -336,23 +341,23 @@ sbn_status launch_pack(const void *W, int64_t out, int64_t in, int n, int m, flo
   const int64_t nel = out * in;
   const uint4 *W4 = reinterpret_cast<const uint4 *>(W);
   const int64_t nblocks = nel / 64, bpr = in / 64;
-  if ((n == 6 && m == 8) || (n == 2 && m == 4)) {
-    FastPackArgs fa{W4,  nblocks, (uint32_t)bpr, make_fast_div((uint32_t)bpr),
-                    ws,  codes,   ldc,           crow,
-                    meta, ldm,    mrow,          dense_dbg,
-                    0,   nel,     eps,           gamma_eff};
-    fa.nparts = (int)fast_pack_parts(fa);
-    return launch_fast_pack(fa, n == 2, err_flag, st);
-  }
+  // S1 for every pattern: one exact partial sum per CTA
   const int64_t nvec = nel / 8;
-  int64_t grid = (nvec + 256 * 8 - 1) / (256 * 8);
-  const int64_t cap = (int64_t)num_sms() * 4;  // 32 resident warps per SM, 8 loads each
+  int64_t grid = (nvec + kAsThreads * kAsLoads - 1) / (kAsThreads * kAsLoads);
+  const int64_t cap = (int64_t)num_sms() * 4;  // one wave of 4 CTAs per SM
   if (grid > cap) grid = cap;
   if (grid > kPackMaxParts) grid = kPackMaxParts;
   if (grid < 1) grid = 1;
   const int nparts = (int)grid;
-  k_abs_sum<<<(unsigned)grid, 256, 0, st>>>(W4, nvec, ws, err_flag);
+  k_abs_sum<<<(unsigned)grid, kAsThreads, 0, st>>>(W4, nvec, ws, err_flag);
   SBN_LAUNCH_CHECK();
+  if ((n == 6 && m == 8) || (n == 2 && m == 4)) {
+    FastPackArgs fa{W4,  nblocks, (uint32_t)bpr, make_fast_div((uint32_t)bpr),
+                    ws,  codes,   ldc,           crow,
+                    meta, ldm,    mrow,          dense_dbg,
+                    nparts, nel,  eps,           gamma_eff};
+    return launch_fast_pack(fa, n == 2, st);
+  }
 #define SBN_QMP(NN, MM)                                                                    \
   case (NN * 16 + MM):                                                                     \
     launch_qmp<NN, MM>(W4, nblocks, bpr, ws, codes, ldc, crow, meta, ldm, mrow, dense_dbg, \

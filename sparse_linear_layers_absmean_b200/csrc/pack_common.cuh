@@ -1,12 +1,36 @@
-// Finishing the absmean scale, shared by the quant/mask/pack kernels (pack.cu,
-// pack_fast.cu).  k_abs_sum leaves one exact partial sum per CTA in the workspace; every
-// CTA of the next kernel turns them into gamma, g = gamma + eps and the code threshold.
+// The absmean scale, shared by the quant/mask/pack kernels (pack.cu, pack_fast.cu): the
+// exact fp64 accumulation k_abs_sum uses, and the prologue with which every CTA of the
+// next kernel turns k_abs_sum's per-CTA partial sums into gamma, g = gamma + eps and the
+// code threshold.
 #pragma once
 
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace sbn {
+
+// ---------------------------------------------------------------------------------------
+// Exact absmean sum S = sum trunc(|W| * 2^24) with one fp64 add per weight.
+// ((h << 13) & 0x0fffe000) | 0x40000000, for the 15 magnitude bits h of a bf16 value, is
+// the high word of the fp64 number |W| * 2^128 (bf16 exponent e -> fp64 exponent field
+// e + 1024, the seven mantissa bits after it; zero and subnormals give values below 4).
+// The accumulator starts at 2^156, where the fp64 spacing is 2^104, and every add rounds
+// toward zero: with acc on that grid and 0 <= v, floor(acc + v) = acc + floor(v), so each
+// add contributes exactly floor(|W| * 2^128 / 2^104) = trunc(|W| * 2^24).  The low 52 bits
+// of the final accumulator are the sum (below 2^52 for any one thread's share).  Exact for
+// |W| < 256, the supported range.
+// ---------------------------------------------------------------------------------------
+constexpr double kAccBias = 9.1343852333181432e46;  // 2^156
+
+__device__ __forceinline__ double mag_lo_x2p128(uint32_t w) {
+  return __hiloint2double((int)(((w << 13) & 0x0fffe000u) | 0x40000000u), 0);
+}
+__device__ __forceinline__ double mag_hi_x2p128(uint32_t w) {
+  return __hiloint2double((int)(((w >> 3) & 0x0fffe000u) | 0x40000000u), 0);
+}
+__device__ __forceinline__ unsigned long long acc_value(double acc) {
+  return (unsigned long long)__double_as_longlong(acc) & ((1ull << 52) - 1);
+}
 
 // Smallest bf16 magnitude (as bits) whose ternary code is non-zero for this g.
 // round_half_even(x / g) != 0  <=>  fl(x / g) > 0.5, and fl(x / g) is non-decreasing in x,

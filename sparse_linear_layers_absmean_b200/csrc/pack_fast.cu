@@ -1,12 +1,10 @@
 // Quant/mask/pack for the two patterns the pages use most, 6:8 and 2:4, with far fewer
 // instructions per weight than the generic kernel (pack.cu).  Same results, bit for bit.
 //
-// Two passes over W.  The N:M selection does not depend on the scale, so it runs in the
-// pass that must read all of W anyway for the absmean sum: k_mask_sum streams W from HBM,
-// writes the metadata plane and the per-CTA partial sums, and its selection arithmetic
-// overlaps the loads.  k_codes finishes the scale and then needs only a compare per
-// weight: it re-reads W (from L2 where W fits there) with the metadata and writes the
-// codes plane.
+// The absmean sum needs all of W before any code is known, so W is read twice: k_abs_sum
+// (pack.cu) streams it once at the full HBM bandwidth with little arithmetic per weight,
+// then k_qmp here re-reads it (from L2 where W fits there), finishes the scale and does
+// the heavy per-weight work - N:M selection, metadata and codes - in one pass.
 //
 // Each lane owns 16 consecutive weights (two 16-byte loads).  The arithmetic runs on the
 // bf16 words as they are loaded (two weights per 32-bit register):
@@ -144,34 +142,10 @@ __device__ uint32_t pair_entry(uint32_t keep8) {
   return meta | (sel << 8);
 }
 
-// ---------------------------------------------------------------------------------------
-// Exact absmean sum S = sum trunc(|W| * 2^24) with one fp64 add per weight.
-// ((h << 13) & 0x0fffe000) | 0x40000000, for the 15 magnitude bits h of a bf16 value, is
-// the high word of the fp64 number |W| * 2^128 (bf16 exponent e -> fp64 exponent field
-// e + 1024, the seven mantissa bits after it; zero and subnormals give values below 4).
-// The accumulator starts at 2^156, where the fp64 spacing is 2^104, and every add rounds
-// toward zero: with acc on that grid and 0 <= v, floor(acc + v) = acc + floor(v), so each
-// add contributes exactly floor(|W| * 2^128 / 2^104) = trunc(|W| * 2^24).  The low 52 bits
-// of the final accumulator are the sum (below 2^52 for any one thread's share).  Exact for
-// |W| < 256, the supported range.
-// ---------------------------------------------------------------------------------------
-constexpr double kAccBias = 9.1343852333181432e46;  // 2^156
-
-__device__ __forceinline__ double mag_lo_x2p128(uint32_t w) {
-  return __hiloint2double((int)(((w << 13) & 0x0fffe000u) | 0x40000000u), 0);
-}
-__device__ __forceinline__ double mag_hi_x2p128(uint32_t w) {
-  return __hiloint2double((int)(((w >> 3) & 0x0fffe000u) | 0x40000000u), 0);
-}
-__device__ __forceinline__ unsigned long long acc_value(double acc) {
-  return (unsigned long long)__double_as_longlong(acc) & ((1ull << 52) - 1);
-}
-
-// Work split of both passes: warp-iteration q covers 64-weight blocks 8q .. 8q+7 (1 KB of
-// W); lane l owns weights 16 (l & 3) .. +15 of block 8q + (l >> 2), loaded as two 16-byte
-// words.  Warps stride over q; four 256-thread CTAs per SM keep about 64 KB of loads in
-// flight per SM (the next iteration's words are requested before the current ones are
-// used), enough for the full HBM bandwidth.
+// Work split: warp-iteration q covers 64-weight blocks 8q .. 8q+7 (1 KB of W); lane l
+// owns weights 16 (l & 3) .. +15 of block 8q + (l >> 2), loaded as two 16-byte words.
+// Warps stride over q two iterations at a time (four 16-byte loads in flight per lane);
+// four 256-thread CTAs per SM.
 constexpr int kPkThreads = 256;
 constexpr int kPkCtasPerSm = 4;
 
@@ -186,135 +160,29 @@ __device__ __forceinline__ void pk_load(const uint4 *W, uint32_t nb, uint32_t b,
   }
 }
 
-// ---------------------------------------------------------------------------------------
-// Pass 1: keep masks and the exact absmean sum, in one read of W.  The metadata plane is
-// written here (6:8: the keep bits of each group of 8; 2:4: i0 | i1 << 2 per group of 4);
-// each CTA leaves its partial sum in the workspace and raises the weight error flags.
-// ---------------------------------------------------------------------------------------
+// One lane's 16 weights: keep masks, metadata, codes.
 template <bool kCompact>
-__device__ __forceinline__ void mask_sum_unit(const FastPackArgs &a, const uint32_t *s_meta,
-                                              uint4 v0, uint4 v1, uint32_t b, int s, double &acc0,
-                                              double &acc1, uint32_t &mx) {
-  if (b >= (uint32_t)a.nblocks) return;
-  const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    mx = vmax16(mx, w[k] & kMag);
-    acc0 = __dadd_rz(acc0, mag_lo_x2p128(w[k]));
-    acc1 = __dadd_rz(acc1, mag_hi_x2p128(w[k]));
-  }
-  uint32_t meta16;
-  if constexpr (kCompact) {
-    const uint32_t KA = keep_2of4(w[0], w[1]), KB = keep_2of4(w[2], w[3]);
-    const uint32_t KC = keep_2of4(w[4], w[5]), KD = keep_2of4(w[6], w[7]);
-    meta16 = s_meta[top_bits_to_byte(KA, KB)] | (s_meta[top_bits_to_byte(KC, KD)] << 8);
-  } else {
-    uint32_t KGA, KGB, KHA, KHB;
-    keep_6of8(w, KGA, KGB);
-    keep_6of8(w + 4, KHA, KHB);
-    meta16 = top_bits_to_byte(KGA, KGB) | (top_bits_to_byte(KHA, KHB) << 8);
-  }
-  const uint32_t row = fast_div(b, a.div_bpr);
-  const uint32_t col = b - row * a.bpr;
-  uint8_t *mrow = a.meta + (int64_t)row * a.ldm;
-  reinterpret_cast<uint16_t *>(mrow + col * 8)[s] = (uint16_t)meta16;
-  if (s == 0 && col == a.bpr - 1 && a.ldm > a.meta_row_bytes)
-    *reinterpret_cast<uint2 *>(mrow + a.meta_row_bytes) = make_uint2(0u, 0u);
-}
-
-template <bool kCompact>
-__global__ void __launch_bounds__(kPkThreads, kPkCtasPerSm)
-    k_mask_sum(const FastPackArgs a, int32_t *err_flag) {
-  __shared__ uint32_t s_meta[256];  // 2:4: keep byte of two groups -> their meta byte
-  __shared__ unsigned long long s_sum[kPkThreads / 32];
-  __shared__ uint32_t s_all[kPkThreads / 32], s_fin[kPkThreads / 32];
-  // the codes pass may start launching; its CTAs find room only as these ones leave
-  ptx::grid_dep_launch();
-  if (kCompact) s_meta[threadIdx.x] = pair_entry(threadIdx.x) & 0xffu;
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int s = lane & 3;
-  const uint32_t nb = (uint32_t)a.nblocks;
-  const uint32_t bstep = 8 * gridDim.x * (kPkThreads / 32);
-  const uint32_t first = 8 * (blockIdx.x * (kPkThreads / 32) + warp);  // warp-uniform
-  const uint32_t sub = lane >> 2;
-  double acc0 = kAccBias, acc1 = kAccBias;
-  uint32_t mx = 0;  // largest magnitude bits seen, per 16-bit half
-  // two warp-iterations per loop trip: four 16-byte loads in flight per lane
-  for (uint32_t base = first; base < nb; base += 2 * bstep) {
-    uint4 p0, p1, q0, q1;
-    pk_load(a.W, nb, base + sub, s, p0, p1);
-    pk_load(a.W, nb, base + bstep + sub, s, q0, q1);
-    mask_sum_unit<kCompact>(a, s_meta, p0, p1, base + sub, s, acc0, acc1, mx);
-    mask_sum_unit<kCompact>(a, s_meta, q0, q1, base + bstep + sub, s, acc0, acc1, mx);
-  }
-  unsigned long long sum = acc_value(acc0) + acc_value(acc1);
-  // Rare path: some |W| >= 256 (or NaN/Inf).  Re-read this lane's weights to tell the two
-  // error kinds apart.
-  uint32_t mx_all = 0, mx_fin = 0;
-  if (max(mx & 0xffffu, mx >> 16) >= kBf16Mag256Bits) {
-    for (uint32_t bb = first + sub; bb < nb; bb += bstep) {
-      uint4 v0, v1;
-      pk_load(a.W, nb, bb, s, v0, v1);
-      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      for (int k = 0; k < 16; ++k) {
-        const uint32_t m = (w[k >> 1] >> (16 * (k & 1))) & 0x7fffu;
-        mx_all = max(mx_all, m);
-        if (m < kBf16InfBits) mx_fin = max(mx_fin, m);
-      }
-    }
-  }
-  sum = warp_sum_u64(sum);
-  const uint32_t ma = warp_max_u32(mx_all), mf = warp_max_u32(mx_fin);
-  if (lane == 0) {
-    s_sum[warp] = sum;
-    s_all[warp] = ma;
-    s_fin[warp] = mf;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    unsigned long long tot = 0;
-    uint32_t am = 0, fm = 0;
-    for (int i = 0; i < kPkThreads / 32; ++i) {
-      tot += s_sum[i];
-      am = max(am, s_all[i]);
-      fm = max(fm, s_fin[i]);
-    }
-    const_cast<PackWorkspace *>(a.ws)->part[blockIdx.x] = tot;
-    int flags = 0;
-    if (am >= kBf16InfBits) flags |= SBN_FLAG_W_NONFINITE;
-    if (fm >= kBf16Mag256Bits) flags |= SBN_FLAG_W_RANGE;
-    if (flags && err_flag) atomicOr(err_flag, flags);
-  }
-}
-
-// prmt selector that compacts the kept weights of two 2:4 groups: meta byte
-// (i0A | i1A << 2 | i0B << 4 | i1B << 6) -> byte selectors i0A, i1A, 4 + i0B, 4 + i1B.
-__device__ __forceinline__ uint32_t compact_selector(uint32_t mb) {
-  return (mb & 3u) | (((mb >> 2) & 3u) << 4) | ((((mb >> 4) & 3u) + 4u) << 8) |
-         ((((mb >> 6) & 3u) + 4u) << 12);
-}
-
-// Meta bits of this lane for block b (pass 1's output), 0 past the end.
-__device__ __forceinline__ uint32_t meta_of(const FastPackArgs &a, uint32_t nb, uint32_t b, int s) {
-  if (b >= nb) return 0u;
-  const uint32_t row = fast_div(b, a.div_bpr);
-  const uint32_t col = b - row * a.bpr;
-  return reinterpret_cast<const uint16_t *>(a.meta + (int64_t)row * a.ldm + col * 8)[s];
-}
-
-// ---------------------------------------------------------------------------------------
-// Pass 2: codes.  Each lane requests its first W words at once (W does not depend on
-// pass 1; after pass 1 they are mostly L2 hits), then the CTA waits for pass 1 to
-// complete, finishes the scale (pack_prologue) and stores the 2-bit codes of the kept
-// weights.
-// ---------------------------------------------------------------------------------------
-template <bool kCompact>
-__device__ __forceinline__ void codes_unit(const FastPackArgs &a, const uint32_t *s_sel, uint4 v0,
-                                           uint4 v1, uint32_t m16, uint32_t b, int s,
-                                           uint32_t thr2) {
+__device__ __forceinline__ void qmp_unit(const FastPackArgs &a, const uint32_t *s_pair, uint4 v0,
+                                         uint4 v1, uint32_t b, int s, uint32_t thr2) {
   const bool valid = b < (uint32_t)a.nblocks;  // both lanes of a shuffle pair share the block
   const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  // keep flags of weights 0-3, 4-7, 8-11, 12-15 (byte-top) and the metadata bits
+  uint32_t K0, K1, K2, K3, meta16, selAB = 0, selCD = 0;
+  if constexpr (kCompact) {
+    K0 = keep_2of4(w[0], w[1]);
+    K1 = keep_2of4(w[2], w[3]);
+    K2 = keep_2of4(w[4], w[5]);
+    K3 = keep_2of4(w[6], w[7]);
+    const uint32_t eAB = s_pair[top_bits_to_byte(K0, K1)];
+    const uint32_t eCD = s_pair[top_bits_to_byte(K2, K3)];
+    meta16 = (eAB & 0xffu) | ((eCD & 0xffu) << 8);
+    selAB = eAB >> 8;
+    selCD = eCD >> 8;
+  } else {
+    keep_6of8(w, K0, K1);
+    keep_6of8(w + 4, K2, K3);
+    meta16 = top_bits_to_byte(K0, K1) | (top_bits_to_byte(K2, K3) << 8);
+  }
   const uint32_t N0 = __byte_perm(nonzero_flags(w[0], thr2), nonzero_flags(w[1], thr2), 0x7531);
   const uint32_t N1 = __byte_perm(nonzero_flags(w[2], thr2), nonzero_flags(w[3], thr2), 0x7531);
   const uint32_t N2 = __byte_perm(nonzero_flags(w[4], thr2), nonzero_flags(w[5], thr2), 0x7531);
@@ -326,7 +194,6 @@ __device__ __forceinline__ void codes_unit(const FastPackArgs &a, const uint32_t
     // kept weights in order: stored elements 8s..8s+7 = (A.first, A.second, B.first,
     // B.second | C.first, ..., D.second): j = 2*(s&1) (+1 for C, D), byte k = position
     const int js = 4 * (s & 1);
-    const uint32_t selAB = s_sel[m16 & 0xffu], selCD = s_sel[(m16 >> 8) & 0xffu];
     const uint32_t LAB = __byte_perm(N0, N1, selAB) & kTop;
     const uint32_t HAB = LAB & __byte_perm(S0, S1, selAB);
     const uint32_t LCD = __byte_perm(N2, N3, selCD) & kTop;
@@ -334,8 +201,7 @@ __device__ __forceinline__ void codes_unit(const FastPackArgs &a, const uint32_t
     word = (HAB >> js) | (LAB >> (1 + js)) | (HCD >> (2 + js)) | (LCD >> (3 + js));
     word |= __shfl_xor_sync(0xffffffffu, word, 1);
   } else {
-    const uint32_t L0 = N0 & nibble_to_top_bits(m16), L1 = N1 & nibble_to_top_bits(m16 >> 4);
-    const uint32_t L2 = N2 & nibble_to_top_bits(m16 >> 8), L3 = N3 & nibble_to_top_bits(m16 >> 12);
+    const uint32_t L0 = N0 & K0, L1 = N1 & K1, L2 = N2 & K2, L3 = N3 & K3;
     const uint32_t H0 = L0 & S0, H1 = L1 & S1, H2 = L2 & S2, H3 = L3 & S3;
     // weights e = 0..15 of this lane are elements 16s+e of the block: word s, byte e%4,
     // bits (7,6) - 2*(e/4) for (negative, non-zero)
@@ -345,29 +211,20 @@ __device__ __forceinline__ void codes_unit(const FastPackArgs &a, const uint32_t
   const uint32_t row = fast_div(b, a.div_bpr);
   const uint32_t col = b - row * a.bpr;
   uint8_t *crow = a.codes + (int64_t)row * a.ldc;
+  uint8_t *mrow = a.meta + (int64_t)row * a.ldm;
   if constexpr (kCompact) {
     if ((s & 1) == 0) reinterpret_cast<uint32_t *>(crow + col * 8)[s >> 1] = word;
   } else {
     reinterpret_cast<uint32_t *>(crow + col * 16)[s] = word;
   }
-  if (col == a.bpr - 1 && s == 0 && a.ldc > a.codes_row_bytes)
-    *reinterpret_cast<uint2 *>(crow + a.codes_row_bytes) = make_uint2(0u, 0u);
+  reinterpret_cast<uint16_t *>(mrow + col * 8)[s] = (uint16_t)meta16;
+  if (col == a.bpr - 1 && s == 0) {  // zero the row padding
+    if (a.ldc > a.codes_row_bytes)
+      *reinterpret_cast<uint2 *>(crow + a.codes_row_bytes) = make_uint2(0u, 0u);
+    if (a.ldm > a.meta_row_bytes)
+      *reinterpret_cast<uint2 *>(mrow + a.meta_row_bytes) = make_uint2(0u, 0u);
+  }
   if (a.dense_dbg) {
-    uint32_t K0, K1, K2, K3;
-    if constexpr (kCompact) {
-      auto keep_of = [](uint32_t nib) {
-        return (0x80u << (8 * (nib & 3u))) | (0x80u << (8 * ((nib >> 2) & 3u)));
-      };
-      K0 = keep_of(m16);
-      K1 = keep_of(m16 >> 4);
-      K2 = keep_of(m16 >> 8);
-      K3 = keep_of(m16 >> 12);
-    } else {
-      K0 = nibble_to_top_bits(m16);
-      K1 = nibble_to_top_bits(m16 >> 4);
-      K2 = nibble_to_top_bits(m16 >> 8);
-      K3 = nibble_to_top_bits(m16 >> 12);
-    }
     const uint32_t l0 = N0 & K0, l1 = N1 & K1, l2 = N2 & K2, l3 = N3 & K3;
     *reinterpret_cast<uint4 *>(a.dense_dbg + (uint64_t)b * 64 + 16 * s) =
         make_uint4(flags_to_i8(l0, l0 & S0), flags_to_i8(l1, l1 & S1), flags_to_i8(l2, l2 & S2),
@@ -375,10 +232,15 @@ __device__ __forceinline__ void codes_unit(const FastPackArgs &a, const uint32_t
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Keep masks, metadata and codes in one pass over W, after k_abs_sum (launched as its
+// programmatic dependent: each lane requests its first W words before waiting for the
+// partial sums, then the CTA finishes the scale in pack_prologue).
+// ---------------------------------------------------------------------------------------
 template <bool kCompact>
-__global__ void __launch_bounds__(kPkThreads, kPkCtasPerSm) k_codes(const FastPackArgs a) {
-  __shared__ uint32_t s_sel[256];  // 2:4: meta byte -> compaction selector
-  if (kCompact) s_sel[threadIdx.x] = compact_selector(threadIdx.x);
+__global__ void __launch_bounds__(kPkThreads, kPkCtasPerSm) k_qmp(const FastPackArgs a) {
+  __shared__ uint32_t s_pair[256];  // 2:4: keep byte -> meta byte | compaction selector << 8
+  if (kCompact) s_pair[threadIdx.x] = pair_entry(threadIdx.x);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int s = lane & 3;
   const uint32_t nb = (uint32_t)a.nblocks;
@@ -388,14 +250,12 @@ __global__ void __launch_bounds__(kPkThreads, kPkCtasPerSm) k_codes(const FastPa
   uint4 p0, p1, q0, q1;
   pk_load(a.W, nb, first + sub, s, p0, p1);
   pk_load(a.W, nb, first + bstep + sub, s, q0, q1);
-  ptx::grid_dep_wait();  // pass 1 complete: partial sums and metadata visible
+  ptx::grid_dep_wait();  // k_abs_sum complete: partial sums visible
   const uint32_t thr = pack_prologue(a.ws, a.nparts, a.n, a.eps, a.gamma_eff);  // syncs
   const uint32_t thr2 = thr | (thr << 16);
-  // two warp-iterations per loop trip: four 16-byte loads in flight per lane
   for (uint32_t base = first;;) {
-    const uint32_t mp = meta_of(a, nb, base + sub, s), mq = meta_of(a, nb, base + bstep + sub, s);
-    codes_unit<kCompact>(a, s_sel, p0, p1, mp, base + sub, s, thr2);
-    codes_unit<kCompact>(a, s_sel, q0, q1, mq, base + bstep + sub, s, thr2);
+    qmp_unit<kCompact>(a, s_pair, p0, p1, base + sub, s, thr2);
+    qmp_unit<kCompact>(a, s_pair, q0, q1, base + bstep + sub, s, thr2);
     base += 2 * bstep;
     if (base >= nb) break;
     pk_load(a.W, nb, base + sub, s, p0, p1);
@@ -403,13 +263,15 @@ __global__ void __launch_bounds__(kPkThreads, kPkCtasPerSm) k_codes(const FastPa
   }
 }
 
-template <bool kCompact>
-static sbn_status launch_two_pass(const FastPackArgs &a, int64_t grid, int32_t *err_flag,
-                                  cudaStream_t st) {
-  k_mask_sum<kCompact><<<(unsigned)grid, kPkThreads, 0, st>>>(a, err_flag);
-  SBN_LAUNCH_CHECK();
-  // pass 2 may launch while pass 1 drains (programmatic dependent launch); it waits for
-  // pass 1's completion before reading anything pass 1 wrote
+sbn_status launch_fast_pack(const FastPackArgs &a, bool compact, cudaStream_t st) {
+  // one wave: enough CTAs for one warp-iteration per warp, at most kPkCtasPerSm per SM
+  const int64_t warp_iters = (a.nblocks + 7) / 8;
+  int64_t grid = (warp_iters + kPkThreads / 32 - 1) / (kPkThreads / 32);
+  const int64_t cap = (int64_t)num_sms() * kPkCtasPerSm;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  // launched as a programmatic dependent of k_abs_sum: it may start while k_abs_sum
+  // drains and waits for its completion before reading the partial sums
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(kPkThreads);
@@ -420,30 +282,13 @@ static sbn_status launch_two_pass(const FastPackArgs &a, int64_t grid, int32_t *
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, k_codes<kCompact>, a) != cudaSuccess) {
+  const cudaError_t e = compact ? cudaLaunchKernelEx(&cfg, k_qmp<true>, a)
+                                : cudaLaunchKernelEx(&cfg, k_qmp<false>, a);
+  if (e != cudaSuccess) {
     (void)cudaGetLastError();
     return SBN_ERR_CUDA;
   }
   return SBN_OK;
-}
-
-// Grid of both passes: one wave of kPkCtasPerSm CTAs per SM (fewer for small tensors:
-// one warp-iteration per warp at least).
-int64_t fast_pack_parts(const FastPackArgs &a) {
-  const int64_t warp_iters = (a.nblocks + 7) / 8;
-  int64_t g = (warp_iters + kPkThreads / 32 - 1) / (kPkThreads / 32);
-  const int64_t cap = (int64_t)num_sms() * kPkCtasPerSm;
-  if (g > cap) g = cap;
-  if (g > kPackMaxParts) g = kPackMaxParts;
-  return g < 1 ? 1 : g;
-}
-
-sbn_status launch_fast_pack(const FastPackArgs &a, bool compact, int32_t *err_flag,
-                            cudaStream_t st) {
-  const int64_t g = fast_pack_parts(a);
-  if (a.nparts != g) return SBN_ERR_ARG;
-  return compact ? launch_two_pass<true>(a, g, err_flag, st)
-                 : launch_two_pass<false>(a, g, err_flag, st);
 }
 
 }  // namespace sbn
