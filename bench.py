@@ -326,7 +326,7 @@ def run_cuda(args, cfg):
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm"], "traffic": traffic,
                 "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs; of measured)"}
-    roof["kernel"] = {"pack": "quant_mask_pack (k_mask_sum + k_codes)", "act": "act_quant",
+    roof["kernel"] = {"pack": "quant_mask_pack (k_abs_sum + k_qmp)", "act": "act_quant",
                       "linear": "contraction"}[dom]
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
