@@ -440,6 +440,38 @@ def run_reference(args, cfg):
     }))
 
 
+def run_only(args, cfg):
+    """Profiling aid: one C-ABI call of the step (pack, act or linear) on the workload's
+    first seeded input set, `warmup + steps` times on the current stream, nothing timed.
+    Used to capture a single kernel under ncu; prints one JSON line saying what ran."""
+    import sparse_linear_layers_absmean_b200 as sbn
+
+    dev = torch.device("cuda", 0)
+    O, K, T, n, m = cfg["O"], cfg["K"], cfg["T"], cfg["n"], cfg["m"]
+    W = workloads.torch_bf16(workloads.masters(O, K, seed=0, config=1, tensor=0), dev)
+    X = workloads.torch_bf16(workloads.activations(T, K, seed=0, config=1, tensor=1), dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    w = sbn.pack_weights(W, n, m, err_flag=err)
+    Xq, s = sbn.quantize_acts(X, err_flag=err)
+    Y = torch.empty((T, O), dtype=torch.float32, device=dev)
+    ws = sbn.new_workspace(O, K, n, m, dev)
+    calls = args.warmup + args.steps
+    for _ in range(calls):
+        if args.only == "pack":
+            sbn.sbn_quantize_mask_pack_weights(W, n, m, 1e-5, w.codes, w.meta, w.gamma_eff, ws,
+                                               None, err)
+        elif args.only == "act":
+            sbn.sbn_quantize_acts(X, Xq, s, err)
+        else:
+            sbn.sbn_linear(Xq, s, w.codes, w.meta, w.gamma_eff, O, K, n, m, Y, None, err)
+    torch.cuda.synchronize()
+    flag = int(err.item())
+    print(json.dumps({"only": args.only, "workload": cfg["name"], "calls": calls,
+                      "err_flag": flag}))
+    if flag:
+        sys.exit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -449,10 +481,15 @@ def main():
     ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["pack", "act", "linear"],
+                    help="profiling aid: run one C-ABI call of the step, untimed")
     args = ap.parse_args()
+    cfg = WORKLOADS[args.workload]
+    if args.only:
+        run_only(args, cfg)
+        return
     if args.warmup < 3:
         args.warmup = 3
-    cfg = WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, cfg)
     else:
