@@ -42,13 +42,14 @@ template <int T, int SPL, bool kCompact>
 __global__ void __launch_bounds__(kGvThreads)
     k_gemv(const int8_t *__restrict__ Xq, const float *__restrict__ absmax,
            const uint8_t *__restrict__ codes, const uint8_t *__restrict__ meta,
-           const float *__restrict__ gamma_eff, int64_t out, int64_t in, int64_t ldc,
+           const float *__restrict__ gamma_eff, int nt, int64_t out, int64_t in, int64_t ldc,
            int64_t ldm, void *__restrict__ Y, int y_is_bf16, int32_t *__restrict__ acc_dbg) {
+  // T: tokens the kernel is built for; nt <= T: tokens present (rows nt.. of Xq do not exist)
   const int lane = threadIdx.x & 31;
   const int64_t row0 = kGvRows * (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   if (row0 >= out) return;  // whole warps leave together
   const bool two = row0 + 1 < out;
-  const float c = lane < T ? rescale_factor(__ldg(gamma_eff), __ldg(absmax + lane)) : 0.0f;
+  const float c = lane < nt ? rescale_factor(__ldg(gamma_eff), __ldg(absmax + lane)) : 0.0f;
   const int nwords = (int)(in / (kCompact ? 32 : 16));  // code words per row
   const uint32_t *crow[kGvRows], *mrow[kGvRows];
 #pragma unroll
@@ -78,6 +79,7 @@ __global__ void __launch_bounds__(kGvThreads)
       if (wi >= nwords) continue;
 #pragma unroll
       for (int t = 0; t < T; ++t) {
+        if (t >= nt) break;
         if constexpr (!kCompact) {
           const uint4 x4 = __ldg(reinterpret_cast<const uint4 *>(Xq + t * in + (int64_t)wi * 16));
           const uint32_t xw[4] = {x4.x, x4.y, x4.z, x4.w};
@@ -112,7 +114,7 @@ __global__ void __launch_bounds__(kGvThreads)
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) acc[r][t] += __shfl_xor_sync(0xffffffffu, acc[r][t], o);
     }
-  if (lane < T) {
+  if (lane < nt) {
 #pragma unroll
     for (int r = 0; r < kGvRows; ++r) {
       if (r == 1 && !two) break;
@@ -134,35 +136,37 @@ __global__ void __launch_bounds__(kGvThreads)
 
 template <int T, int SPL>
 static sbn_status gemv_tc(const int8_t *Xq, const float *absmax, const uint8_t *codes,
-                          const uint8_t *meta, const float *gamma_eff, int64_t out, int64_t in,
+                          const uint8_t *meta, const float *gamma_eff, int nt, int64_t out,
+                          int64_t in,
                           bool compact, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
                           int32_t *acc_dbg, cudaStream_t st) {
   const int64_t rows_per_cta = kGvRows * (kGvThreads / 32);
   const int64_t grid = (out + rows_per_cta - 1) / rows_per_cta;
   auto kern = compact ? k_gemv<T, SPL, true> : k_gemv<T, SPL, false>;
-  kern<<<(unsigned)grid, kGvThreads, 0, st>>>(Xq, absmax, codes, meta, gamma_eff, out, in, ldc,
-                                              ldm, Y, y_is_bf16, acc_dbg);
+  kern<<<(unsigned)grid, kGvThreads, 0, st>>>(Xq, absmax, codes, meta, gamma_eff, nt, out, in,
+                                              ldc, ldm, Y, y_is_bf16, acc_dbg);
   SBN_LAUNCH_CHECK();
   return SBN_OK;
 }
 
 template <int T>
 static sbn_status gemv_t(const int8_t *Xq, const float *absmax, const uint8_t *codes,
-                         const uint8_t *meta, const float *gamma_eff, int64_t out, int64_t in,
+                         const uint8_t *meta, const float *gamma_eff, int nt, int64_t out,
+                         int64_t in,
                          bool compact, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
                          int32_t *acc_dbg, cudaStream_t st) {
   const int64_t words = in / (compact ? 32 : 16);  // code words per row
   const int64_t spl = (words + 31) / 32;
   if (spl <= 2)
-    return gemv_tc<T, 2>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
+    return gemv_tc<T, 2>(Xq, absmax, codes, meta, gamma_eff, nt, out, in, compact, ldc, ldm, Y,
                          y_is_bf16, acc_dbg, st);
   if (spl <= 4)
-    return gemv_tc<T, 4>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
+    return gemv_tc<T, 4>(Xq, absmax, codes, meta, gamma_eff, nt, out, in, compact, ldc, ldm, Y,
                          y_is_bf16, acc_dbg, st);
   if (spl <= 6 || T > 2)
-    return gemv_tc<T, 6>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
+    return gemv_tc<T, 6>(Xq, absmax, codes, meta, gamma_eff, nt, out, in, compact, ldc, ldm, Y,
                          y_is_bf16, acc_dbg, st);
-  return gemv_tc<T, 8>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
+  return gemv_tc<T, 8>(Xq, absmax, codes, meta, gamma_eff, nt, out, in, compact, ldc, ldm, Y,
                        y_is_bf16, acc_dbg, st);
 }
 
@@ -171,22 +175,16 @@ sbn_status launch_gemv(const int8_t *Xq, const float *absmax, const uint8_t *cod
                        int64_t out, int64_t in, int n, int m, int64_t ldc, int64_t ldm,
                        void *Y, int y_is_bf16, int32_t *acc_dbg, cudaStream_t st) {
   const bool compact = (n == 2 && m == 4);
-  switch (tokens) {
-    case 1:
-      return gemv_t<1>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
-                       y_is_bf16, acc_dbg, st);
-    case 2:
-      return gemv_t<2>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
-                       y_is_bf16, acc_dbg, st);
-    case 3:
-      return gemv_t<3>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
-                       y_is_bf16, acc_dbg, st);
-    case 4:
-      return gemv_t<4>(Xq, absmax, codes, meta, gamma_eff, out, in, compact, ldc, ldm, Y,
-                       y_is_bf16, acc_dbg, st);
-    default:
-      return SBN_ERR_SHAPE;
-  }
+  const int nt = (int)tokens;
+#define SBN_GEMV(TT)                                                                         \
+  return gemv_t<TT>(Xq, absmax, codes, meta, gamma_eff, nt, out, in, compact, ldc, ldm, Y, \
+                    y_is_bf16, acc_dbg, st)
+  if (tokens == 1) SBN_GEMV(1);
+  if (tokens == 2) SBN_GEMV(2);
+  if (tokens == 3) SBN_GEMV(3);
+  if (tokens == 4) SBN_GEMV(4);
+#undef SBN_GEMV
+  return SBN_ERR_SHAPE;
 }
 
 }  // namespace sbn

@@ -136,7 +136,7 @@ def check_linear(T, O, K, n, m, seed, out_dtype=torch.float32, eps=1e-5):
 
 @pytest.mark.parametrize("n,m", [(2, 4), (6, 8), (4, 4), (1, 8)])
 @pytest.mark.parametrize("T", [1, 2, 3, 4])
-@pytest.mark.parametrize("O,K", [(37, 192), (300, 640)])
+@pytest.mark.parametrize("O,K", [(37, 192), (300, 640), (129, 11008)])
 def test_linear_cuda_cores(T, O, K, n, m):
     check_linear(T, O, K, n, m, seed=T + O + K + n)
 
@@ -154,6 +154,14 @@ def test_linear_many_tiles_per_cta(T, O, K):
     so both TMEM accumulators and the stage ring wrap across tiles (ragged rows, tokens
     and K in each case)."""
     check_linear(T, O, K, 2, 4, seed=T + O + K)
+
+
+@pytest.mark.parametrize("T,O,K", [(5, 4100, 4096), (16, 1000, 11008), (17, 300, 2048),
+                                   (32, 130, 8192), (24, 4096, 576)])
+def test_linear_few_tokens_long_k(T, O, K):
+    """5-32 tokens on the 2:4 tensor-core kernel with long rows (up to 86 K blocks, so the
+    stage ring wraps many times), ragged rows and a K that ends in half a block."""
+    check_linear(T, O, K, 2, 4, seed=T * 3 + O + K)
 
 
 @pytest.mark.parametrize("T", [1, 3, 9, 300])

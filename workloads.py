@@ -30,12 +30,17 @@ TRAIN_LAYER_SHAPES = [("qkv", 9600, 3200), ("o", 3200, 3200), ("gate", 8640, 320
 TRAIN_LAYERS = 26
 TRAIN_STEPS = 10
 
+TRAIN_STEP = dict(name="train-step-26x3200-6of8+2of4", kind="train")
+
 # Full 32-layer block stack, hidden 4096, FFN 11008.
 STACK_LAYER_SHAPES = [("qkv", 12288, 4096), ("o", 4096, 4096), ("gate", 11008, 4096),
                       ("up", 11008, 4096), ("down", 4096, 11008)]
 STACK_LAYERS = 32
 STACK_DECODE_T = 16
 STACK_PREFILL_T = 4096
+STACK_DECODE = dict(name="stack-decode-32x4096-t16-2of4", kind="stack", T=STACK_DECODE_T)
+STACK_PREFILL = dict(name="stack-prefill-32x4096-t4096-2of4", kind="stack",
+                     T=STACK_PREFILL_T)
 
 
 def rng(seed: int = 0, config: int = 0, tensor: int = 0, step: int = 0):
@@ -57,6 +62,15 @@ def bf16_bits_to_f32(b) -> np.ndarray:
 def masters(O: int, K: int, *, seed=0, config=0, tensor=0, step=0, std=0.02) -> np.ndarray:
     r = rng(seed, config, tensor, step)
     return to_bf16_bits(r.standard_normal((O, K), dtype=np.float32) * np.float32(std))
+
+
+def masters_device(O: int, K: int, *, device, seed=0, config=0, tensor=0, std=0.02):
+    """bf16 masters N(0, std^2) drawn on the GPU from a seeded torch generator: for the
+    multi-GB benchmark workloads (whole decoder stacks), where host generation would take
+    minutes.  Not used by the parity tests, whose inputs come from `masters`."""
+    g = torch.Generator(device=device)
+    g.manual_seed(((seed * 1000003 + config) * 1000003 + tensor) & ((1 << 62) - 1))
+    return (torch.randn((O, K), device=device, generator=g) * std).to(torch.bfloat16)
 
 
 def activations(T: int, K: int, *, seed=0, config=0, tensor=1, step=0, outliers=True,
