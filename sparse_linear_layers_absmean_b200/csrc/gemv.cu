@@ -8,6 +8,7 @@
 // Work split: two output rows per warp; see k_gemv.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace sbn {
 
@@ -47,6 +48,8 @@ __global__ void __launch_bounds__(kGvThreads)
   // T: tokens the kernel is built for; nt <= T: tokens present (rows nt.. of Xq do not exist)
   const int lane = threadIdx.x & 31;
   const int64_t row0 = kGvRows * (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  // launched as a programmatic dependent: everything read below comes from earlier kernels
+  ptx::grid_dep_wait();
   if (row0 >= out) return;  // whole warps leave together
   const bool two = row0 + 1 < out;
   const float c = lane < nt ? rescale_factor(__ldg(gamma_eff), __ldg(absmax + lane)) : 0.0f;
@@ -143,9 +146,23 @@ static sbn_status gemv_tc(const int8_t *Xq, const float *absmax, const uint8_t *
   const int64_t rows_per_cta = kGvRows * (kGvThreads / 32);
   const int64_t grid = (out + rows_per_cta - 1) / rows_per_cta;
   auto kern = compact ? k_gemv<T, SPL, true> : k_gemv<T, SPL, false>;
-  kern<<<(unsigned)grid, kGvThreads, 0, st>>>(Xq, absmax, codes, meta, gamma_eff, nt, out, in,
-                                              ldc, ldm, Y, y_is_bf16, acc_dbg);
-  SBN_LAUNCH_CHECK();
+  // programmatic dependent launch: the GEMV's CTAs may be scheduled while the kernel before
+  // it on the stream (the pack) drains; griddepcontrol.wait in the kernel keeps the order
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kGvThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, Xq, absmax, codes, meta, gamma_eff, nt, out, in, ldc, ldm, Y,
+                         y_is_bf16, acc_dbg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
   return SBN_OK;
 }
 

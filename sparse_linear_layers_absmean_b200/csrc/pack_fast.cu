@@ -240,6 +240,9 @@ __device__ __forceinline__ void qmp_unit(const FastPackArgs &a, const uint32_t *
 template <bool kCompact>
 __global__ void __launch_bounds__(kPkThreads, kPkCtasPerSm) k_qmp(const FastPackArgs a) {
   __shared__ uint32_t s_pair[256];  // 2:4: keep byte -> meta byte | compaction selector << 8
+  // a programmatic dependent (the contraction) may start launching; it waits for this
+  // kernel's completion before reading the planes
+  ptx::grid_dep_launch();
   if (kCompact) s_pair[threadIdx.x] = pair_entry(threadIdx.x);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int s = lane & 3;
