@@ -1120,8 +1120,16 @@ static sbn_status gemm_sp24_pair_t(const int8_t *Xq, const float *absmax, const 
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  // as many pairs as can be resident at once (the kernel strides over the tiles)
-  static int max_pairs = 0;
+  // as many pairs as can be resident at once (the kernel strides over the tiles); cached
+  // per device
+  constexpr int kMaxDevices = 64;
+  static int pairs_cache[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    dev = 0;
+  }
+  int max_pairs = (dev >= 0 && dev < kMaxDevices) ? pairs_cache[dev] : 0;
   if (max_pairs == 0) {
     cfg.gridDim = dim3((unsigned)num_sms());
     int n = 0;
@@ -1130,6 +1138,7 @@ static sbn_status gemm_sp24_pair_t(const int8_t *Xq, const float *absmax, const 
       n = num_sms() / 2;
     }
     max_pairs = n;
+    if (dev >= 0 && dev < kMaxDevices) pairs_cache[dev] = n;
   }
   const int64_t ntiles = ((O + 2 * kBM - 1) / (2 * kBM)) * ((T + BN - 1) / BN);
   const int64_t npairs = ntiles < max_pairs ? ntiles : max_pairs;

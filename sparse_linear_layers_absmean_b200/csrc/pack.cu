@@ -292,14 +292,24 @@ __global__ void __launch_bounds__(256) k_quant_mask_pack(const QmpArgs<N, M> a) 
 // Host launchers
 // ---------------------------------------------------------------------------------------
 
+// SM count of the current device (cached per device; a concurrent first query stores the
+// same value).
 int num_sms() {
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      sms = 148;
+  constexpr int kMaxDevices = 64;
+  static int cache[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    (void)cudaGetLastError();
+    return 148;
   }
+  if (dev < kMaxDevices && cache[dev] > 0) return cache[dev];
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      sms < 1) {
+    (void)cudaGetLastError();
+    sms = 148;
+  }
+  if (dev < kMaxDevices) cache[dev] = sms;
   return sms;
 }
 
