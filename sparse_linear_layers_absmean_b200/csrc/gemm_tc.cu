@@ -8,7 +8,11 @@
 // is not available).
 //
 // One CTA computes a 128 (outputs) x BN (tokens) tile with a multi-stage shared-memory
-// pipeline over K in blocks of 128:
+// pipeline over K in blocks of 128 (a stage holds one to four consecutive blocks: each
+// hand-off between the roles has a fixed cost, so the narrow tiles move several blocks per
+// hand-off).  Up to 32 tokens, k_gemm_sp24 may split a tile's K blocks over a cluster of
+// CTAs when there are too few tiles to occupy the SMs; CTA 0 of the cluster receives the
+// others' partial accumulators through distributed shared memory and stores the tile.
 //   warp 4     TMA producer: per K block, the int8 activation tile (128-byte swizzle,
 //              K-major) and the packed weight tile (codes, plus the 2:4 metadata) of the
 //              CTA's 128 rows.
@@ -52,15 +56,28 @@ __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity) {
   }
 }
 
+// Partial accumulators of a K-split tile, as CTA 0 of the cluster receives them: slot q
+// holds [128 rows][BN] int32, the 16-byte chunks of row r XOR-swizzled by r so that a
+// warp's chunk reads spread over the banks.
+template <int BN>
+__device__ __forceinline__ int red_word(int r, int col) {
+  constexpr int kSwz = (BN / 4 < 8 ? BN / 4 : 8) - 1;
+  return r * BN + ((((col >> 2) ^ (r & kSwz))) << 2) + (col & 3);
+}
+
 // Epilogue of the tensor-core kernels: warp w (0..3) owns accumulator lanes 32w..32w+31
 // (output rows o), TMEM column j is token t0 + j and holds 64 * acc.  s_scale[j] holds
 // c_t = fp32(fp32(g * s_t) / 127).  y = fp32(acc * c_t): acc is converted exactly (the
 // magic-number addition is exact for |acc| < 2^22, a plain conversion is used otherwise)
-// and multiplied once, the same rounding as acc * c_t.
+// and multiplied once, the same rounding as acc * c_t.  With nred > 0 the nred partial
+// accumulators in `red` (tile row r) are added first; integer sums, so the order of the
+// parts does not change the result.
 template <int BN>
 __device__ __forceinline__ void store_tile(uint32_t trow, const float *s_scale, int64_t o,
                                            int64_t O, int64_t t0, int64_t T, bool small_acc,
-                                           void *Y, int y_is_bf16, int32_t *acc_dbg) {
+                                           void *Y, int y_is_bf16, int32_t *acc_dbg,
+                                           const uint32_t *red = nullptr, int nred = 0,
+                                           int r = 0) {
   constexpr int kCols = BN < 32 ? BN : 32;
   const bool row_ok = o < O;
 #pragma unroll 1
@@ -92,6 +109,21 @@ __device__ __forceinline__ void store_tile(uint32_t trow, const float *s_scale, 
       for (int i = 0; i < 16; ++i) va[i] = v16[i];
     }
     ptx::tmem_ld_wait();
+    for (int q = 0; q < nred; ++q) {
+      const uint32_t *slot = red + q * (kBM * BN);
+#pragma unroll
+      for (int i = 0; i < kCols; i += 4) {
+        if (cb + i < BN) {
+          const uint4 p = *reinterpret_cast<const uint4 *>(slot + red_word<BN>(r, cb + i));
+          va[i] += p.x, va[i + 1] += p.y, va[i + 2] += p.z, va[i + 3] += p.w;
+        }
+        if (cb + kCols + i < BN) {
+          const uint4 p =
+              *reinterpret_cast<const uint4 *>(slot + red_word<BN>(r, cb + kCols + i));
+          vb[i] += p.x, vb[i + 1] += p.y, vb[i + 2] += p.z, vb[i + 3] += p.w;
+        }
+      }
+    }
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const int c0 = cb + half * kCols;
@@ -325,20 +357,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 template <int BN>
 struct SpCfg {
-  static constexpr int kKL = 128;                 // logical K per stage
+  static constexpr int kKL = 128;                 // logical K of one block
   static constexpr int kABytes = kBM * kKL / 2;   // compressed int8: 64 bytes per row
   static constexpr int kBBytes = BN * kKL;        // activations: 128 bytes per token
   static constexpr int kPBytes = kBM * 16 * 2;    // packed codes + metadata, 16 B each per row
-  static constexpr int kStageBytes = kABytes + kBBytes + kPBytes;
+  static constexpr int kBlockBytes = kABytes + kBBytes + kPBytes;
   static constexpr int kBudget = 225 * 1024 - BN * 4 - 512;
-  static constexpr int kStages = (kBudget / kStageBytes) > 8 ? 8 : (kBudget / kStageBytes);
+  // kG consecutive K blocks share one set of pipeline barriers (a stage): every hand-off
+  // between the roles has a fixed cost, so few tokens per tile move several blocks per
+  // hand-off.  kSub block buffers in all, kStages = kSub / kG stages.
+  static constexpr int kG = BN <= 32 ? 4 : BN <= 128 ? 2 : 1;
+  static constexpr int kMaxSub = BN <= 32 ? 16 : 8;
+  static constexpr int kFit = kBudget / kBlockBytes;
+  static constexpr int kSub = ((kFit > kMaxSub ? kMaxSub : kFit) / kG) * kG;
+  static constexpr int kStages = kSub / kG;
+  static_assert(kStages >= 2, "at least two pipeline stages");
   static constexpr int kMetaCol = BN < 32 ? 32 : BN;  // first TMEM column of the metadata
-  static constexpr int kNeedCols = kMetaCol + 4 * kStages;
+  static constexpr int kNeedCols = kMetaCol + 4 * kSub;
   static constexpr int kTmemCols = kNeedCols <= 32 ? 32 : kNeedCols <= 64 ? 64
                                    : kNeedCols <= 128 ? 128 : kNeedCols <= 256 ? 256 : 512;
-  static constexpr uint32_t kTxBytes = kBBytes + kPBytes;
-  static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes +
+  static constexpr uint32_t kTxBytes = kBBytes + kPBytes;  // TMA bytes of one block
+  static constexpr size_t kSmem = 1024 + (size_t)kSub * kBlockBytes +
                                   (size_t)(3 * kStages + 1) * 8 + 16 + (size_t)BN * 4;
+  // K split over a cluster (BN <= 32): CTA 0 receives the other CTAs' partial tiles in its
+  // block buffers
+  static constexpr int kMaxSplit = BN <= 32 ? 8 : 1;
+  static_assert((kMaxSplit - 1) * kBM * BN * 4 <= kSub * kBlockBytes,
+                "the partial tiles of a split must fit in the stage memory");
 };
 
 template <int BN>
@@ -349,14 +394,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 void *__restrict__ Y, int y_is_bf16, int32_t *__restrict__ acc_dbg,
                 int32_t *err_flag) {
   using Cfg = SpCfg<BN>;
-  constexpr int S = Cfg::kStages;
+  constexpr int S = Cfg::kStages, G = Cfg::kG, U = Cfg::kSub;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *sB = smem;                        // 1024-aligned stages (128-byte swizzle)
-  uint8_t *sA = sB + S * Cfg::kBBytes;       // 512-aligned stages (64-byte swizzle)
-  uint8_t *sP = sA + S * Cfg::kABytes;       // packed codes [128][16] then metadata [128][16]
-  uint64_t *full_a = reinterpret_cast<uint64_t *>(sP + S * Cfg::kPBytes);
+  // block buffer u = G * stage + g holds K block g of the stage
+  uint8_t *sB = smem;                        // 1024-aligned blocks (128-byte swizzle)
+  uint8_t *sA = sB + U * Cfg::kBBytes;       // 512-aligned blocks (64-byte swizzle)
+  uint8_t *sP = sA + U * Cfg::kABytes;       // packed codes [128][16] then metadata [128][16]
+  uint64_t *full_a = reinterpret_cast<uint64_t *>(sP + U * Cfg::kPBytes);
   uint64_t *full_t = full_a + S;
   uint64_t *empty = full_t + S;
   uint64_t *done = empty + S;
@@ -364,9 +410,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   float *s_scale = reinterpret_cast<float *>(tmem_slot + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t o0 = (int64_t)blockIdx.x * kBM;
+  // A launch with clusters of C CTAs along x splits each tile's K blocks into C contiguous
+  // ranges, one per CTA; CTA 0 of the cluster sums the partial accumulators and stores.
+  const uint32_t csplit = ptx::cluster_nctarank();
+  const uint32_t crank = csplit > 1 ? ptx::cluster_ctarank() : 0u;
+  const int64_t o0 = (int64_t)(blockIdx.x / csplit) * kBM;
   const int64_t t0 = (int64_t)blockIdx.y * BN;
-  const int nkb = (int)((K + Cfg::kKL - 1) / Cfg::kKL);
+  const int nkb_all = (int)((K + Cfg::kKL - 1) / Cfg::kKL);
+  const int kb0 = (int)((int64_t)nkb_all * crank / csplit);
+  const int nkb = (int)((int64_t)nkb_all * (crank + 1) / csplit) - kb0;
+  const int nst = (nkb + G - 1) / G;  // stages of this CTA; the last may hold fewer blocks
   bool timed_out = false;
 
   if (threadIdx.x == 0) {
@@ -394,31 +447,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp < 4) {
     // ---------------- compressed-weight expanders ----------------
     const int r = threadIdx.x;
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % S;
-      const uint32_t ph = (uint32_t)(kb / S) & 1u;
-      if ((kb >= S && !wait_phase(&empty[s], ph ^ 1u)) || !wait_phase(&full_t[s], ph)) {
+    for (int j = 0; j < nst; ++j) {
+      const int s = j % S;
+      const uint32_t ph = (uint32_t)(j / S) & 1u;
+      if ((j >= S && !wait_phase(&empty[s], ph ^ 1u)) || !wait_phase(&full_t[s], ph)) {
         timed_out = true;
         break;
       }
-      const uint4 cw = *reinterpret_cast<const uint4 *>(sP + s * Cfg::kPBytes + r * 16);
-      const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
-      // Groups past the matrix (rows >= O, or the second half of the last block when
-      // K % 128 == 64) were zero-filled by the TMA; give them the valid index pair (0, 1)
-      // so the MMA never sees a malformed metadata nibble (their codes are zero anyway).
-      if (o0 + r >= O) {
-        *reinterpret_cast<uint4 *>(sP + s * Cfg::kPBytes + kBM * 16 + r * 16) =
-            make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
-      } else if ((int64_t)kb * Cfg::kKL + 64 >= K) {
-        *reinterpret_cast<uint2 *>(sP + s * Cfg::kPBytes + kBM * 16 + r * 16 + 8) =
-            make_uint2(0x44444444u, 0x44444444u);
-      }
-      uint8_t *dst = sA + s * Cfg::kABytes + r * 64;
+      const int nb = min(G, nkb - j * G);
 #pragma unroll
-      for (int c = 0; c < 4; ++c)  // 16 kept codes -> 16 int8 lanes, in order
-        *reinterpret_cast<uint4 *>(dst + ((c ^ ((r >> 1) & 3)) << 4)) =
-            make_uint4(w[c] & 0xC0C0C0C0u, (w[c] << 2) & 0xC0C0C0C0u,
-                       (w[c] << 4) & 0xC0C0C0C0u, (w[c] << 6) & 0xC0C0C0C0u);
+      for (int g = 0; g < G; ++g) {
+        if (g >= nb) break;
+        const int u = s * G + g;
+        const int kb = kb0 + j * G + g;
+        const uint4 cw = *reinterpret_cast<const uint4 *>(sP + u * Cfg::kPBytes + r * 16);
+        const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+        // Groups past the matrix (rows >= O, or the second half of the last block when
+        // K % 128 == 64) were zero-filled by the TMA; give them the valid index pair (0, 1)
+        // so the MMA never sees a malformed metadata nibble (their codes are zero anyway).
+        if (o0 + r >= O) {
+          *reinterpret_cast<uint4 *>(sP + u * Cfg::kPBytes + kBM * 16 + r * 16) =
+              make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+        } else if ((int64_t)kb * Cfg::kKL + 64 >= K) {
+          *reinterpret_cast<uint2 *>(sP + u * Cfg::kPBytes + kBM * 16 + r * 16 + 8) =
+              make_uint2(0x44444444u, 0x44444444u);
+        }
+        uint8_t *dst = sA + u * Cfg::kABytes + r * 64;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)  // 16 kept codes -> 16 int8 lanes, in order
+          *reinterpret_cast<uint4 *>(dst + ((c ^ ((r >> 1) & 3)) << 4)) =
+              make_uint4(w[c] & 0xC0C0C0C0u, (w[c] << 2) & 0xC0C0C0C0u,
+                         (w[c] << 4) & 0xC0C0C0C0u, (w[c] << 6) & 0xC0C0C0C0u);
+      }
       ptx::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&full_a[s]);
@@ -430,61 +490,102 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ptx::prefetch_tmap(&tmap_c);
       ptx::prefetch_tmap(&tmap_m);
       int issued = 0;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = (uint32_t)(kb / S) & 1u;
-        if (kb >= S && !wait_phase(&empty[s], ph ^ 1u)) {
+      for (int j = 0; j < nst; ++j) {
+        const int s = j % S;
+        const uint32_t ph = (uint32_t)(j / S) & 1u;
+        if (j >= S && !wait_phase(&empty[s], ph ^ 1u)) {
           timed_out = true;
           break;
         }
-        ptx::mbar_arrive_expect_tx(&full_t[s], Cfg::kTxBytes);
-        ptx::tma_load_2d(sB + s * Cfg::kBBytes, &tmap_x, &full_t[s], kb * Cfg::kKL, (int32_t)t0);
-        uint8_t *p = sP + s * Cfg::kPBytes;
-        ptx::tma_load_2d(p, &tmap_c, &full_t[s], kb * 16, (int32_t)o0);
-        ptx::tma_load_2d(p + kBM * 16, &tmap_m, &full_t[s], kb * 16, (int32_t)o0);
-        issued = kb + 1;
+        const int nb = min(G, nkb - j * G);
+        ptx::mbar_arrive_expect_tx(&full_t[s], (uint32_t)nb * Cfg::kTxBytes);
+        for (int g = 0; g < nb; ++g) {
+          const int u = s * G + g;
+          const int kb = kb0 + j * G + g;
+          ptx::tma_load_2d(sB + u * Cfg::kBBytes, &tmap_x, &full_t[s], kb * Cfg::kKL,
+                           (int32_t)t0);
+          uint8_t *p = sP + u * Cfg::kPBytes;
+          ptx::tma_load_2d(p, &tmap_c, &full_t[s], kb * 16, (int32_t)o0);
+          ptx::tma_load_2d(p + kBM * 16, &tmap_m, &full_t[s], kb * 16, (int32_t)o0);
+        }
+        issued = j + 1;
       }
-      for (int kb = issued - S < 0 ? 0 : issued - S; kb < issued; ++kb)
-        if (!wait_phase(&full_t[kb % S], (uint32_t)(kb / S) & 1u)) timed_out = true;
+      for (int j = issued - S < 0 ? 0 : issued - S; j < issued; ++j)
+        if (!wait_phase(&full_t[j % S], (uint32_t)(j / S) & 1u)) timed_out = true;
     }
   } else {
     // ---------------- metadata copy + sparse MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc = ptx::idesc_i8_sparse(kBM, BN);
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = (uint32_t)(kb / S) & 1u;
+      for (int j = 0; j < nst; ++j) {
+        const int s = j % S;
+        const uint32_t ph = (uint32_t)(j / S) & 1u;
         if (!wait_phase(&full_a[s], ph) || !wait_phase(&full_t[s], ph)) {
           timed_out = true;
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t e_col = tmem + Cfg::kMetaCol + 4 * s;
-        ptx::tmem_cp_128x128b(e_col, ptx::smem_desc_rows16(ptx::smem_u32(sP + s * Cfg::kPBytes +
-                                                                        kBM * 16)));
-        const uint32_t a_addr = ptx::smem_u32(sA + s * Cfg::kABytes);
-        const uint32_t b_addr = ptx::smem_u32(sB + s * Cfg::kBBytes);
+        const int nb = min(G, nkb - j * G);
+        for (int g = 0; g < nb; ++g) {
+          const int u = s * G + g;
+          const uint32_t e_col = tmem + Cfg::kMetaCol + 4 * u;
+          ptx::tmem_cp_128x128b(
+              e_col, ptx::smem_desc_rows16(ptx::smem_u32(sP + u * Cfg::kPBytes + kBM * 16)));
+          const uint32_t a_addr = ptx::smem_u32(sA + u * Cfg::kABytes);
+          const uint32_t b_addr = ptx::smem_u32(sB + u * Cfg::kBBytes);
 #pragma unroll
-        for (int k = 0; k < 2; ++k)  // logical K 64 per MMA: 32 bytes of A, 64 of B
-          ptx::mma_sp_i8(tmem, ptx::smem_desc_sw64(a_addr + 32 * k),
-                         ptx::smem_desc_sw128(b_addr + 64 * k), e_col + 2 * k, idesc,
-                         (kb | k) != 0);
+          for (int k = 0; k < 2; ++k)  // logical K 64 per MMA: 32 bytes of A, 64 of B
+            ptx::mma_sp_i8(tmem, ptx::smem_desc_sw64(a_addr + 32 * k),
+                           ptx::smem_desc_sw128(b_addr + 64 * k), e_col + 2 * k, idesc,
+                           (j | g | k) != 0);
+        }
         ptx::mma_commit(&empty[s]);
       }
       ptx::mma_commit(done);
     }
   }
 
+  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
   if (warp < 4) {
-    // ---------------- epilogue ----------------
     __syncwarp();
     if (!timed_out && !wait_phase(done, 0)) timed_out = true;
     ptx::tc_fence_after();
+  }
+  if (csplit > 1) {
+    // ---------------- K-split reduction into CTA 0 ----------------
+    // After the first cluster barrier every CTA's MMAs have completed, so CTA 0's stage
+    // memory is free; CTAs 1.. store their partial tiles there; after the second, CTA 0
+    // reads them.  A CTA that timed out sends what it has (the flag marks the output).
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+    ptx::cluster_sync();
+    if (warp < 4 && crank != 0) {
+      const int r = threadIdx.x;
+      const uint32_t slot = ptx::mapa_shared(ptx::smem_u32(smem), 0) +
+                            (crank - 1) * (uint32_t)(kBM * BN * 4);
+#pragma unroll
+      for (int cb = 0; cb < BN; cb += 16) {
+        uint32_t v[16];
+        ptx::tmem_ld_16(trow + cb, v);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) {
+          const uint4 p = nkb > 0 ? make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3])
+                                  : make_uint4(0u, 0u, 0u, 0u);
+          ptx::st_cluster_v4(slot + 4u * (uint32_t)red_word<BN>(r, cb + i), p);
+        }
+      }
+    }
+    __syncwarp();
+    ptx::cluster_sync();
+  }
+  if (warp < 4 && crank == 0) {
+    // ---------------- epilogue ----------------
     const int64_t o = o0 + warp * 32 + lane;
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
     // |acc| <= 127 * K < 2^22 for K <= 32768
     if (!timed_out)
-      store_tile<BN>(trow, s_scale, o, O, t0, T, K <= 32768, Y, y_is_bf16, acc_dbg);
+      store_tile<BN>(trow, s_scale, o, O, t0, T, K <= 32768, Y, y_is_bf16, acc_dbg,
+                     reinterpret_cast<const uint32_t *>(smem), (int)csplit - 1, threadIdx.x);
   }
   if (timed_out && err_flag) atomicOr(err_flag, SBN_FLAG_TIMEOUT);
   ptx::tc_fence_before();
@@ -772,22 +873,27 @@ struct PairCfg {
   static constexpr int kABytes = kBM * kKL / 2;
   static constexpr int kBBytes = kBHalf * kKL;
   static constexpr int kPBytes = kBM * 16 * 2;
-  static constexpr int kStageBytes = kABytes + kBBytes + kPBytes;
+  static constexpr int kBlockBytes = kABytes + kBBytes + kPBytes;
   static constexpr int kBudget = 225 * 1024 - BN * 4 - 1024;
-  static constexpr int kStages = (kBudget / kStageBytes) > 12 ? 12 : (kBudget / kStageBytes);
+  // kG consecutive K blocks per pipeline stage (one set of barriers); kSub block buffers
+  static constexpr int kG = 2;
+  static constexpr int kFit = (kBudget / kBlockBytes) > 12 ? 12 : (kBudget / kBlockBytes);
+  static constexpr int kSub = (kFit / kG) * kG;
+  static constexpr int kStages = kSub / kG;
+  static_assert(kStages >= 2, "at least two pipeline stages");
   static constexpr int kAccStride = 256;
   static constexpr int kGap = (256 - BN) / 4;
   static_assert(BN <= 256 && BN % 32 == 0, "pair tile width");
-  static_assert(kBBytes % 1024 == 0, "B stages must keep the 1024-byte swizzle alignment");
-  static_assert(2 * kGap >= kStages, "two accumulators and the metadata must fit in TMEM");
+  static_assert(kBBytes % 1024 == 0, "B blocks must keep the 1024-byte swizzle alignment");
+  static_assert(2 * kGap >= kSub, "two accumulators and the metadata must fit in TMEM");
   static constexpr int kTmemCols = 512;
   __device__ static constexpr uint32_t meta_col(int s) {
     return s < kGap ? (uint32_t)(BN + 4 * s) : (uint32_t)(kAccStride + BN + 4 * (s - kGap));
   }
-  static constexpr uint32_t kTxBytes = kBBytes + kPBytes;  // per CTA, on its own barrier
+  static constexpr uint32_t kTxBytes = kBBytes + kPBytes;  // per block and CTA
   // barriers: full_a[S], full_t[S], empty[S], acc_full[2], acc_empty[2], mma_done; then the
   // TMEM address, the abort flag (32 bytes) and the per-token scales
-  static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes +
+  static constexpr size_t kSmem = 1024 + (size_t)kSub * kBlockBytes +
                                   (size_t)(3 * kStages + 5) * 8 + 32 + (size_t)BN * 4;
 };
 
@@ -800,15 +906,16 @@ __global__ void __launch_bounds__(kPsThreads, 1)
                      int64_t T, int64_t O, int64_t K, void *__restrict__ Y, int y_is_bf16,
                      int32_t *__restrict__ acc_dbg, int32_t *err_flag) {
   using Cfg = PairCfg<BN>;
-  constexpr int S = Cfg::kStages;
+  constexpr int S = Cfg::kStages, G = Cfg::kG, U = Cfg::kSub;
   constexpr int kTileM = 2 * kBM;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // block buffer u = G * stage + g holds K block g of the stage
   uint8_t *sB = smem;
-  uint8_t *sA = sB + S * Cfg::kBBytes;
-  uint8_t *sP = sA + S * Cfg::kABytes;
-  uint64_t *full_a = reinterpret_cast<uint64_t *>(sP + S * Cfg::kPBytes);  // CTA 0: both CTAs
+  uint8_t *sA = sB + U * Cfg::kBBytes;
+  uint8_t *sP = sA + U * Cfg::kABytes;
+  uint64_t *full_a = reinterpret_cast<uint64_t *>(sP + U * Cfg::kPBytes);  // CTA 0: both CTAs
   uint64_t *full_t = full_a + S;                                          // own TMA loads
   uint64_t *empty = full_t + S;                                           // own stage free
   uint64_t *acc_full = empty + S;                                         // [2], own
@@ -822,6 +929,7 @@ __global__ void __launch_bounds__(kPsThreads, 1)
   const uint32_t rank = ptx::cluster_ctarank();  // 0: issues the pair's MMAs
   const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int nkb = (int)((K + Cfg::kKL - 1) / Cfg::kKL);
+  const int nst = (nkb + G - 1) / G;  // stages per tile; the last may hold fewer blocks
   const int64_t n_o = (O + kTileM - 1) / kTileM, n_t = (T + BN - 1) / BN;
   const int64_t ntiles = n_o * n_t;
 
@@ -860,27 +968,34 @@ __global__ void __launch_bounds__(kPsThreads, 1)
     for (int64_t tile = pair;
          tile < ntiles && !__any_sync(0xffffffffu, *s_abort != 0); tile += npairs) {
       const int64_t o0 = (tile % n_o) * kTileM + (int64_t)rank * kBM;
-      for (int kb = 0; kb < nkb; ++kb, ++kg) {
+      for (int j = 0; j < nst; ++j, ++kg) {
         const int s = (int)(kg % S);
         const uint32_t ph = (uint32_t)(kg / S) & 1u;
         const bool ok = (kg < S || wait_or_abort(&empty[s], ph ^ 1u, s_abort)) &&
                         wait_or_abort(&full_t[s], ph, s_abort);
         if (!__all_sync(0xffffffffu, ok)) break;  // the whole warp leaves together
-        const uint4 cw = *reinterpret_cast<const uint4 *>(sP + s * Cfg::kPBytes + r * 16);
-        const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
-        if (o0 + r >= O) {
-          *reinterpret_cast<uint4 *>(sP + s * Cfg::kPBytes + kBM * 16 + r * 16) =
-              make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
-        } else if ((int64_t)kb * Cfg::kKL + 64 >= K) {
-          *reinterpret_cast<uint2 *>(sP + s * Cfg::kPBytes + kBM * 16 + r * 16 + 8) =
-              make_uint2(0x44444444u, 0x44444444u);
-        }
-        uint8_t *dst = sA + s * Cfg::kABytes + r * 64;
+        const int nb = min(G, nkb - j * G);
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4 *>(dst + ((c ^ ((r >> 1) & 3)) << 4)) =
-              make_uint4(w[c] & 0xC0C0C0C0u, (w[c] << 2) & 0xC0C0C0C0u,
-                         (w[c] << 4) & 0xC0C0C0C0u, (w[c] << 6) & 0xC0C0C0C0u);
+        for (int g = 0; g < G; ++g) {
+          if (g >= nb) break;
+          const int u = s * G + g;
+          const int kb = j * G + g;
+          const uint4 cw = *reinterpret_cast<const uint4 *>(sP + u * Cfg::kPBytes + r * 16);
+          const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+          if (o0 + r >= O) {
+            *reinterpret_cast<uint4 *>(sP + u * Cfg::kPBytes + kBM * 16 + r * 16) =
+                make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+          } else if ((int64_t)kb * Cfg::kKL + 64 >= K) {
+            *reinterpret_cast<uint2 *>(sP + u * Cfg::kPBytes + kBM * 16 + r * 16 + 8) =
+                make_uint2(0x44444444u, 0x44444444u);
+          }
+          uint8_t *dst = sA + u * Cfg::kABytes + r * 64;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4 *>(dst + ((c ^ ((r >> 1) & 3)) << 4)) =
+                make_uint4(w[c] & 0xC0C0C0C0u, (w[c] << 2) & 0xC0C0C0C0u,
+                           (w[c] << 4) & 0xC0C0C0C0u, (w[c] << 6) & 0xC0C0C0C0u);
+        }
         ptx::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive_cluster(full_a0 + 8u * (uint32_t)s);
@@ -896,16 +1011,21 @@ __global__ void __launch_bounds__(kPsThreads, 1)
       for (int64_t tile = pair; tile < ntiles && !*s_abort; tile += npairs) {
         const int64_t o0 = (tile % n_o) * kTileM + (int64_t)rank * kBM;
         const int64_t t0 = (tile / n_o) * BN + (int64_t)rank * Cfg::kBHalf;
-        for (int kb = 0; kb < nkb; ++kb, ++kg) {
+        for (int j = 0; j < nst; ++j, ++kg) {
           const int s = (int)(kg % S);
           const uint32_t ph = (uint32_t)(kg / S) & 1u;
           if (kg >= S && !wait_or_abort(&empty[s], ph ^ 1u, s_abort)) break;
-          ptx::mbar_arrive_expect_tx(&full_t[s], Cfg::kTxBytes);
-          ptx::tma_load_2d(sB + s * Cfg::kBBytes, &tmap_x, &full_t[s], kb * Cfg::kKL,
-                           (int32_t)t0);
-          uint8_t *p = sP + s * Cfg::kPBytes;
-          ptx::tma_load_2d(p, &tmap_c, &full_t[s], kb * 16, (int32_t)o0);
-          ptx::tma_load_2d(p + kBM * 16, &tmap_m, &full_t[s], kb * 16, (int32_t)o0);
+          const int nb = min(G, nkb - j * G);
+          ptx::mbar_arrive_expect_tx(&full_t[s], (uint32_t)nb * Cfg::kTxBytes);
+          for (int g = 0; g < nb; ++g) {
+            const int u = s * G + g;
+            const int kb = j * G + g;
+            ptx::tma_load_2d(sB + u * Cfg::kBBytes, &tmap_x, &full_t[s], kb * Cfg::kKL,
+                             (int32_t)t0);
+            uint8_t *p = sP + u * Cfg::kPBytes;
+            ptx::tma_load_2d(p, &tmap_c, &full_t[s], kb * 16, (int32_t)o0);
+            ptx::tma_load_2d(p + kBM * 16, &tmap_m, &full_t[s], kb * 16, (int32_t)o0);
+          }
           issued = kg + 1;
         }
       }
@@ -925,7 +1045,7 @@ __global__ void __launch_bounds__(kPsThreads, 1)
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(buf * Cfg::kAccStride);
         bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb, ++kg) {
+        for (int j = 0; j < nst; ++j, ++kg) {
           const int s = (int)(kg % S);
           const uint32_t ph = (uint32_t)(kg / S) & 1u;
           if (!wait_or_abort(&full_a[s], ph, s_abort)) {  // both CTAs expanded (and loaded)
@@ -933,16 +1053,20 @@ __global__ void __launch_bounds__(kPsThreads, 1)
             break;
           }
           ptx::tc_fence_after();
-          const uint32_t e_col = tmem + Cfg::meta_col(s);
-          ptx::tmem_cp_128x128b_pair(
-              e_col, ptx::smem_desc_rows16(ptx::smem_u32(sP + s * Cfg::kPBytes + kBM * 16)));
-          const uint32_t a_addr = ptx::smem_u32(sA + s * Cfg::kABytes);
-          const uint32_t b_addr = ptx::smem_u32(sB + s * Cfg::kBBytes);
+          const int nb = min(G, nkb - j * G);
+          for (int g = 0; g < nb; ++g) {
+            const int u = s * G + g;
+            const uint32_t e_col = tmem + Cfg::meta_col(u);
+            ptx::tmem_cp_128x128b_pair(
+                e_col, ptx::smem_desc_rows16(ptx::smem_u32(sP + u * Cfg::kPBytes + kBM * 16)));
+            const uint32_t a_addr = ptx::smem_u32(sA + u * Cfg::kABytes);
+            const uint32_t b_addr = ptx::smem_u32(sB + u * Cfg::kBBytes);
 #pragma unroll
-          for (int k = 0; k < 2; ++k)
-            ptx::mma_sp_i8_pair(d_tmem, ptx::smem_desc_sw64(a_addr + 32 * k),
-                                ptx::smem_desc_sw128(b_addr + 64 * k), e_col + 2 * k, idesc,
-                                (kb | k) != 0);
+            for (int k = 0; k < 2; ++k)
+              ptx::mma_sp_i8_pair(d_tmem, ptx::smem_desc_sw64(a_addr + 32 * k),
+                                  ptx::smem_desc_sw128(b_addr + 64 * k), e_col + 2 * k, idesc,
+                                  (j | g | k) != 0);
+          }
           ptx::mma_commit_pair(&empty[s], 0x3);
         }
         if (!ok) break;
@@ -1023,6 +1147,69 @@ static bool encode_u8(CUtensorMap *map, const void *base, int64_t cols, int64_t 
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// CTAs per tile along K for k_gemm_sp24<BN> (1 = no split).  The kernel holds one CTA per
+// SM; a split trades longer-running tiles for more CTAs.  Estimated time in units of one
+// K block's pipeline time (measured on B200 at 16 and 32 tokens: about 0.22 us per block,
+// 4 us of fixed cost per CTA wave, 2.5 us for the cluster reduction):
+// waves x (19 + K blocks per CTA) + 11 for a split.  The number of clusters that fit at
+// once comes from the occupancy API (clusters stay inside a GPC) and is cached per device
+// and split.
+template <int BN, typename Kern>
+static int sp24_split(Kern kern, int64_t tiles, int nkb) {
+  using Cfg = SpCfg<BN>;
+  if (Cfg::kMaxSplit <= 1 || nkb < 2) return 1;
+  constexpr int kMaxDevices = 64;
+  static int slots_cache[kMaxDevices][Cfg::kMaxSplit + 1] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    (void)cudaGetLastError();
+    return 1;
+  }
+  int best = 1;
+  double best_cost = 0.0;
+  for (int c = 1; c <= Cfg::kMaxSplit && c <= nkb; ++c) {
+    int &slots = slots_cache[dev][c];  // CTAs resident at once with clusters of c
+    if (slots == 0) {
+      if (c == 1) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kTcThreads,
+                                                          Cfg::kSmem) != cudaSuccess ||
+            per_sm < 1) {
+          (void)cudaGetLastError();
+          per_sm = 1;
+        }
+        slots = per_sm * num_sms();
+      } else {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)c;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3((unsigned)(c * (num_sms() / c)));
+        cfg.blockDim = dim3(kTcThreads);
+        cfg.dynamicSmemBytes = Cfg::kSmem;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+          (void)cudaGetLastError();
+          n = -1;  // not launchable with this cluster size
+        }
+        slots = n > 0 ? n * c : -1;
+      }
+    }
+    if (slots <= 0) continue;
+    const int64_t waves = (tiles * c + slots - 1) / slots;
+    const double cost = (double)waves * (19.0 + (nkb + c - 1) / c) + (c > 1 ? 11.0 : 0.0);
+    if (c == 1 || cost < best_cost) {
+      best = c;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
 template <int BN, bool kCompact>
 static sbn_status gemm_tc_t(const int8_t *Xq, const float *absmax, const uint8_t *codes,
                             const uint8_t *meta, const float *gamma_eff, int64_t T, int64_t O,
@@ -1061,7 +1248,28 @@ static sbn_status gemm_sp24_t(const int8_t *Xq, const float *absmax, const uint8
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::kSmem) !=
       cudaSuccess)
     return SBN_ERR_CUDA;
-  dim3 grid((unsigned)((O + kBM - 1) / kBM), (unsigned)((T + BN - 1) / BN));
+  const int64_t row_tiles = (O + kBM - 1) / kBM, tok_tiles = (T + BN - 1) / BN;
+  const int nkb = (int)((K + Cfg::kKL - 1) / Cfg::kKL);
+  const int csplit = sp24_split<BN>(kern, row_tiles * tok_tiles, nkb);
+  if (csplit > 1) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)csplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(row_tiles * csplit), (unsigned)tok_tiles);
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = Cfg::kSmem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tx, tc, tm, absmax, gamma_eff, T, O, K, Y, y_is_bf16,
+                           acc_dbg, err_flag) == cudaSuccess)
+      return SBN_OK;
+    (void)cudaGetLastError();  // the device rejected the cluster launch: one CTA per tile
+  }
+  dim3 grid((unsigned)row_tiles, (unsigned)tok_tiles);
   kern<<<grid, kTcThreads, Cfg::kSmem, st>>>(tx, tc, tm, absmax, gamma_eff, T, O, K, Y, y_is_bf16,
                                              acc_dbg, err_flag);
   SBN_LAUNCH_CHECK();

@@ -164,6 +164,17 @@ def test_linear_few_tokens_long_k(T, O, K):
     check_linear(T, O, K, 2, 4, seed=T * 3 + O + K)
 
 
+@pytest.mark.parametrize("T,O,K,out", [(16, 4096, 4096, "f32"), (16, 12288, 4096, "f32"),
+                                       (9, 260, 2048, "bf16"), (32, 1100, 11008, "f32"),
+                                       (20, 4000, 4160, "bf16"), (7, 640, 704, "f32")])
+def test_linear_split_k(T, O, K, out):
+    """Up to 32 tokens with few row tiles and long rows: the 2:4 kernel splits each tile's
+    K blocks over a cluster of 2-8 CTAs and CTA 0 adds the partial tiles (the decode
+    shapes of a 4096-hidden layer, a K that ends in half a block, bf16 output)."""
+    check_linear(T, O, K, 2, 4, seed=T + O + K,
+                 out_dtype=torch.bfloat16 if out == "bf16" else torch.float32)
+
+
 @pytest.mark.parametrize("T", [1, 3, 9, 300])
 def test_linear_bf16_output(T):
     check_linear(T, 260, 256, 2, 4, seed=11, out_dtype=torch.bfloat16)
