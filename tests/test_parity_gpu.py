@@ -82,8 +82,28 @@ def test_pack_workspace_is_reusable():
         got = gpu_path.pack(W, 2, 4, workspace=ws)
         ref = oracle.quantize_mask_pack(W, 2, 4)
         assert got["g"] == ref["g"] and np.array_equal(got["codes"], ref["codes"])
-    # the reserved word after the 1024 partial sums is never written
-    assert ws[8192:8196].cpu().numpy().view(np.uint32)[0] == 0
+    # the reserved words after the 1024 partial sums are never written
+    assert not ws[8192:8200].cpu().numpy().any()
+
+
+def test_pack_workspace_many_sizes():
+    """One workspace through calls of many sizes and both fast patterns (the reduction's
+    grid size changes from call to call): every result exact, the reserved words after the
+    partial sums untouched."""
+    import sparse_linear_layers_absmean_b200 as sbn
+    ws = sbn.new_workspace(8, 64, 2, 4)
+    shapes = [(1, 64), (4096, 4096), (3, 192), (700, 2560), (1, 64), (6912, 2560), (130, 320)]
+    for i, (O, K) in enumerate(shapes * 2):
+        n, m = ((2, 4), (6, 8))[i % 2]
+        W = workloads.masters(O, K, seed=100 + i)
+        got = gpu_path.pack(W, n, m, workspace=ws)
+        torch.cuda.synchronize()
+        assert got["err"] == 0
+        assert not ws[8192:8200].cpu().numpy().any()
+        if O * K <= 1 << 22:
+            ref = oracle.quantize_mask_pack(W, n, m)
+            assert got["g"] == ref["g"] and np.array_equal(got["codes"], ref["codes"])
+            assert np.array_equal(got["meta"], ref["meta"])
 
 
 @pytest.mark.parametrize("bad,flag", [(np.nan, 1), (np.inf, 1), (-np.inf, 1), (300.0, 2),
