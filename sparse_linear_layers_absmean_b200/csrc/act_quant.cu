@@ -4,9 +4,12 @@
 //   s = max(max_k |x_k|, 1e-5),  q_k = clamp(rint((127 * x_k) / s), -127, 127).
 // Few tokens: one CTA per token; rows of up to 16384 inputs stay in registers between the
 // max pass and the quantise pass (one HBM read), longer rows are read twice.  Many tokens
-// with rows of up to 4096 inputs: one warp per token (k_act_quant_warp).
+// with rows of up to 4096 inputs: one warp per token (k_act_quant_warp).  Every kernel is
+// launched as a programmatic dependent of the previous kernel on the stream and waits for
+// it before reading X.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace sbn {
 
@@ -53,6 +56,8 @@ template <int R>
 __global__ void __launch_bounds__(kAqThreads)
     k_act_quant_reg(const uint4 *__restrict__ X, int64_t nv, int8_t *__restrict__ Xq,
                     float *__restrict__ absmax, int32_t *err_flag) {
+  ptx::grid_dep_launch();
+  ptx::grid_dep_wait();
   const int64_t t = blockIdx.x;
   const uint4 *row = X + t * nv;
   uint4 v[R];
@@ -76,6 +81,8 @@ __global__ void __launch_bounds__(kAqThreads)
 __global__ void __launch_bounds__(kAqThreads)
     k_act_quant_loop(const uint4 *__restrict__ X, int64_t nv, int8_t *__restrict__ Xq,
                      float *__restrict__ absmax, int32_t *err_flag) {
+  ptx::grid_dep_launch();
+  ptx::grid_dep_wait();
   const int64_t t = blockIdx.x;
   const uint4 *row = X + t * nv;
   uint32_t mx = 0;
@@ -93,6 +100,8 @@ template <int R>
 __global__ void __launch_bounds__(kAqThreads)
     k_act_quant_warp(const uint4 *__restrict__ X, int64_t tokens, int64_t nv,
                      int8_t *__restrict__ Xq, float *__restrict__ absmax, int32_t *err_flag) {
+  ptx::grid_dep_launch();
+  ptx::grid_dep_wait();
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * (kAqThreads / 32) + (threadIdx.x >> 5);
   if (t >= tokens) return;  // whole warps leave together
@@ -122,27 +131,25 @@ sbn_status launch_act_quant(const void *X, int64_t tokens, int64_t in, int8_t *X
                             float *absmax, int32_t *err_flag, cudaStream_t st) {
   const int64_t nv = in / 8;
   const uint4 *X4 = reinterpret_cast<const uint4 *>(X);
-  const unsigned grid = (unsigned)tokens;
+  const dim3 block(kAqThreads);
   if (tokens > 16 && nv <= 32 * 16) {
     // many tokens: one warp each (a CTA-wide reduction per token costs more than the row)
-    const unsigned wgrid = (unsigned)((tokens + kAqThreads / 32 - 1) / (kAqThreads / 32));
+    const dim3 wgrid((unsigned)((tokens + kAqThreads / 32 - 1) / (kAqThreads / 32)));
     if (nv <= 32 * 4)
-      k_act_quant_warp<4><<<wgrid, kAqThreads, 0, st>>>(X4, tokens, nv, Xq, absmax, err_flag);
-    else if (nv <= 32 * 8)
-      k_act_quant_warp<8><<<wgrid, kAqThreads, 0, st>>>(X4, tokens, nv, Xq, absmax, err_flag);
-    else
-      k_act_quant_warp<16><<<wgrid, kAqThreads, 0, st>>>(X4, tokens, nv, Xq, absmax, err_flag);
-    SBN_LAUNCH_CHECK();
-    return SBN_OK;
+      return launch_pdl(k_act_quant_warp<4>, wgrid, block, 0, st, X4, tokens, nv, Xq, absmax,
+                        err_flag);
+    if (nv <= 32 * 8)
+      return launch_pdl(k_act_quant_warp<8>, wgrid, block, 0, st, X4, tokens, nv, Xq, absmax,
+                        err_flag);
+    return launch_pdl(k_act_quant_warp<16>, wgrid, block, 0, st, X4, tokens, nv, Xq, absmax,
+                      err_flag);
   }
+  const dim3 grid((unsigned)tokens);
   if (nv <= 2 * kAqThreads)
-    k_act_quant_reg<2><<<grid, kAqThreads, 0, st>>>(X4, nv, Xq, absmax, err_flag);
-  else if (nv <= 8 * kAqThreads)
-    k_act_quant_reg<8><<<grid, kAqThreads, 0, st>>>(X4, nv, Xq, absmax, err_flag);
-  else
-    k_act_quant_loop<<<grid, kAqThreads, 0, st>>>(X4, nv, Xq, absmax, err_flag);
-  SBN_LAUNCH_CHECK();
-  return SBN_OK;
+    return launch_pdl(k_act_quant_reg<2>, grid, block, 0, st, X4, nv, Xq, absmax, err_flag);
+  if (nv <= 8 * kAqThreads)
+    return launch_pdl(k_act_quant_reg<8>, grid, block, 0, st, X4, nv, Xq, absmax, err_flag);
+  return launch_pdl(k_act_quant_loop, grid, block, 0, st, X4, nv, Xq, absmax, err_flag);
 }
 
 }  // namespace sbn

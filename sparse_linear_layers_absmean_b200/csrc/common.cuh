@@ -48,6 +48,30 @@ __device__ __forceinline__ float rescale_factor(float g, float s) {
 }  // namespace sbn
 
 // Host-side launch check shared by the entry points.
+// Launch as a programmatic dependent of the previous kernel on the stream (programmatic
+// stream serialisation): the launch and the kernel's prologue may overlap that kernel's
+// tail; the kernel executes griddepcontrol.wait before it touches global memory, which
+// returns once the previous kernel has completed and its writes are visible.
+template <typename... KArgs, typename... Args>
+inline sbn_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SBN_ERR_CUDA;
+  }
+  return SBN_OK;
+}
+
 #define SBN_LAUNCH_CHECK()                                         \
   do {                                                             \
     if (cudaPeekAtLastError() != cudaSuccess) {                    \

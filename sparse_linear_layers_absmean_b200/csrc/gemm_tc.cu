@@ -199,6 +199,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
   float *s_scale = reinterpret_cast<float *>(tmem_slot + 4);
 
+  // the next kernel on the stream may start its prologue; it waits for this one
+  ptx::grid_dep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t o0 = (int64_t)blockIdx.x * kBM;
   const int64_t t0 = (int64_t)blockIdx.y * BN;
@@ -218,6 +220,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     ptx::tmem_alloc(tmem_slot, Cfg::kTmemCols);
     ptx::tmem_relinquish();
   }
+  ptx::grid_dep_wait();  // the previous kernel's outputs (activations, scales) are visible
   for (int i = threadIdx.x; i < BN; i += kTcThreads) {
     const int64_t t = t0 + i;
     s_scale[i] = t < T ? rescale_factor(__ldg(gamma_eff), __ldg(absmax + t)) : 0.0f;
@@ -409,6 +412,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
   float *s_scale = reinterpret_cast<float *>(tmem_slot + 4);
 
+  // the next kernel on the stream may start its prologue; it waits for this one
+  ptx::grid_dep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // A launch with clusters of C CTAs along x splits each tile's K blocks into C contiguous
   // ranges, one per CTA; CTA 0 of the cluster sums the partial accumulators and stores.
@@ -435,6 +440,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     ptx::tmem_alloc(tmem_slot, Cfg::kTmemCols);
     ptx::tmem_relinquish();
   }
+  ptx::grid_dep_wait();  // the previous kernel's outputs (activations, scales) are visible
   for (int i = threadIdx.x; i < BN; i += kTcThreads) {
     const int64_t t = t0 + i;
     s_scale[i] = t < T ? rescale_factor(__ldg(gamma_eff), __ldg(absmax + t)) : 0.0f;
@@ -688,6 +694,8 @@ __global__ void __launch_bounds__(kPsThreads, 1)
   volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_slot + 2);
   float *s_scale = reinterpret_cast<float *>(tmem_slot + 8);
 
+  // the next kernel on the stream may start its prologue; it waits for this one
+  ptx::grid_dep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nkb = (int)((K + Cfg::kKL - 1) / Cfg::kKL);
   const int64_t n_o = (O + kBM - 1) / kBM, n_t = (T + BN - 1) / BN;
@@ -711,6 +719,7 @@ __global__ void __launch_bounds__(kPsThreads, 1)
     ptx::tmem_alloc(tmem_slot, Cfg::kTmemCols);
     ptx::tmem_relinquish();
   }
+  ptx::grid_dep_wait();  // the previous kernel's outputs (activations, scales) are visible
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -925,6 +934,8 @@ __global__ void __launch_bounds__(kPsThreads, 1)
   volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_slot + 2);
   float *s_scale = reinterpret_cast<float *>(tmem_slot + 8);
 
+  // the next kernel on the stream may start its prologue; it waits for this one
+  ptx::grid_dep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = ptx::cluster_ctarank();  // 0: issues the pair's MMAs
   const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
@@ -953,6 +964,7 @@ __global__ void __launch_bounds__(kPsThreads, 1)
     ptx::tmem_alloc_pair(tmem_slot, Cfg::kTmemCols);
     ptx::tmem_relinquish_pair();
   }
+  ptx::grid_dep_wait();  // the previous kernel's outputs (activations, scales) are visible
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -1226,11 +1238,9 @@ static sbn_status gemm_tc_t(const int8_t *Xq, const float *absmax, const uint8_t
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::kSmem) !=
       cudaSuccess)
     return SBN_ERR_CUDA;
-  dim3 grid((unsigned)((O + kBM - 1) / kBM), (unsigned)((T + BN - 1) / BN));
-  kern<<<grid, kTcThreads, Cfg::kSmem, st>>>(tx, tc, tm, absmax, gamma_eff, T, O, K, Y, y_is_bf16,
-                                             acc_dbg, err_flag);
-  SBN_LAUNCH_CHECK();
-  return SBN_OK;
+  const dim3 grid((unsigned)((O + kBM - 1) / kBM), (unsigned)((T + BN - 1) / BN));
+  return launch_pdl(kern, grid, dim3(kTcThreads), Cfg::kSmem, st, tx, tc, tm, absmax, gamma_eff,
+                    T, O, K, Y, y_is_bf16, acc_dbg, err_flag);
 }
 
 template <int BN>
@@ -1253,27 +1263,27 @@ static sbn_status gemm_sp24_t(const int8_t *Xq, const float *absmax, const uint8
   const int csplit = sp24_split<BN>(kern, row_tiles * tok_tiles, nkb);
   if (csplit > 1) {
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)csplit;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3((unsigned)(row_tiles * csplit), (unsigned)tok_tiles);
     cfg.blockDim = dim3(kTcThreads);
     cfg.dynamicSmemBytes = Cfg::kSmem;
     cfg.stream = st;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, kern, tx, tc, tm, absmax, gamma_eff, T, O, K, Y, y_is_bf16,
                            acc_dbg, err_flag) == cudaSuccess)
       return SBN_OK;
     (void)cudaGetLastError();  // the device rejected the cluster launch: one CTA per tile
   }
-  dim3 grid((unsigned)row_tiles, (unsigned)tok_tiles);
-  kern<<<grid, kTcThreads, Cfg::kSmem, st>>>(tx, tc, tm, absmax, gamma_eff, T, O, K, Y, y_is_bf16,
-                                             acc_dbg, err_flag);
-  SBN_LAUNCH_CHECK();
-  return SBN_OK;
+  return launch_pdl(kern, dim3((unsigned)row_tiles, (unsigned)tok_tiles), dim3(kTcThreads),
+                    Cfg::kSmem, st, tx, tc, tm, absmax, gamma_eff, T, O, K, Y, y_is_bf16, acc_dbg,
+                    err_flag);
 }
 
 template <int BN>
@@ -1295,10 +1305,8 @@ static sbn_status gemm_sp24_persist_t(const int8_t *Xq, const float *absmax, con
   const int64_t ntiles = ((O + kBM - 1) / kBM) * ((T + BN - 1) / BN);
   int64_t grid = num_sms();
   if (grid > ntiles) grid = ntiles;
-  kern<<<(unsigned)grid, kPsThreads, Cfg::kSmem, st>>>(tx, tc, tm, absmax, gamma_eff, T, O, K, Y,
-                                                       y_is_bf16, acc_dbg, err_flag);
-  SBN_LAUNCH_CHECK();
-  return SBN_OK;
+  return launch_pdl(kern, dim3((unsigned)grid), dim3(kPsThreads), Cfg::kSmem, st, tx, tc, tm,
+                    absmax, gamma_eff, T, O, K, Y, y_is_bf16, acc_dbg, err_flag);
 }
 
 template <int BN>
@@ -1318,16 +1326,18 @@ static sbn_status gemm_sp24_pair_t(const int8_t *Xq, const float *absmax, const 
       cudaSuccess)
     return SBN_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(kPsThreads);
   cfg.dynamicSmemBytes = Cfg::kSmem;
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1;  // the occupancy query takes the cluster shape only
   // as many pairs as can be resident at once (the kernel strides over the tiles); cached
   // per device
   constexpr int kMaxDevices = 64;
@@ -1351,6 +1361,7 @@ static sbn_status gemm_sp24_pair_t(const int8_t *Xq, const float *absmax, const 
   const int64_t ntiles = ((O + 2 * kBM - 1) / (2 * kBM)) * ((T + BN - 1) / BN);
   const int64_t npairs = ntiles < max_pairs ? ntiles : max_pairs;
   cfg.gridDim = dim3((unsigned)(2 * npairs));
+  cfg.numAttrs = 2;  // and a programmatic dependent of the previous kernel
   if (cudaLaunchKernelEx(&cfg, kern, tx, tc, tm, absmax, gamma_eff, T, O, K, Y, y_is_bf16,
                          acc_dbg, err_flag) != cudaSuccess) {
     (void)cudaGetLastError();

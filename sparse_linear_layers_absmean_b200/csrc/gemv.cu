@@ -48,7 +48,9 @@ __global__ void __launch_bounds__(kGvThreads)
   // T: tokens the kernel is built for; nt <= T: tokens present (rows nt.. of Xq do not exist)
   const int lane = threadIdx.x & 31;
   const int64_t row0 = kGvRows * (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
-  // launched as a programmatic dependent: everything read below comes from earlier kernels
+  // launched as a programmatic dependent: everything read below comes from earlier kernels;
+  // the next kernel on the stream may start its prologue (it waits for this one)
+  ptx::grid_dep_launch();
   ptx::grid_dep_wait();
   if (row0 >= out) return;  // whole warps leave together
   const bool two = row0 + 1 < out;

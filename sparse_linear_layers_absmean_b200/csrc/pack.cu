@@ -31,7 +31,10 @@ constexpr int kAsLoads = 4;
 
 __global__ void __launch_bounds__(kAsThreads, 4) k_abs_sum(const uint4 *__restrict__ W, int64_t nvec,
                                                          PackWorkspace *ws, int32_t *err_flag) {
-  // the quant/mask/pack kernel may start launching; it waits for this one's results
+  // A programmatic dependent of the previous kernel on the stream (which may write W): wait
+  // for it first, then let the quant/mask/pack kernel launch.  That kernel requests W
+  // before its own wait, so W must be final by the time it can start.
+  ptx::grid_dep_wait();
   ptx::grid_dep_launch();
   double acc0 = kAccBias, acc1 = kAccBias;
   uint32_t mx = 0;  // largest magnitude bits seen, per 16-bit half
@@ -359,8 +362,9 @@ sbn_status launch_pack(const void *W, int64_t out, int64_t in, int n, int m, flo
   if (grid > kPackMaxParts) grid = kPackMaxParts;
   if (grid < 1) grid = 1;
   const int nparts = (int)grid;
-  k_abs_sum<<<(unsigned)grid, kAsThreads, 0, st>>>(W4, nvec, ws, err_flag);
-  SBN_LAUNCH_CHECK();
+  const sbn_status ls = launch_pdl(k_abs_sum, dim3((unsigned)grid), dim3(kAsThreads), 0, st, W4,
+                                   nvec, ws, err_flag);
+  if (ls != SBN_OK) return ls;
   if ((n == 6 && m == 8) || (n == 2 && m == 4)) {
     FastPackArgs fa{W4,  nblocks, (uint32_t)bpr, make_fast_div((uint32_t)bpr),
                     ws,  codes,   ldc,           crow,
