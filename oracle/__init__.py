@@ -43,6 +43,10 @@ def load_library(path):
     lib.oracle_contract.restype = ctypes.c_int
     lib.oracle_rescale.argtypes = [p, p, ctypes.c_float, i64, i64, p]
     lib.oracle_rescale.restype = None
+    lib.oracle_count_zero_codes.argtypes = [p, i64]
+    lib.oracle_count_zero_codes.restype = i64
+    lib.oracle_count_mask_flips.argtypes = [p, p, i64]
+    lib.oracle_count_mask_flips.restype = i64
     if not lib.oracle_rounding_is_nearest():
         raise RuntimeError("oracle needs round-to-nearest-even on the host FPU")
     return lib
@@ -179,3 +183,16 @@ def linear(X_bits, W_bits, n: int, m: int, eps: float = 1e-5):
     w.update(Xq=Xq, s=s, xerr=xerr, acc=acc, y=y)
     return w
 
+
+def count_zero_codes(t):
+    """Natural zeros: positions whose ternary code (before the mask) is 0."""
+    t = np.ascontiguousarray(t, np.int8)
+    return int(_lib().oracle_count_zero_codes(_ptr(t), t.size))
+
+
+def count_mask_flips(keep_a, keep_b):
+    """Positions kept by one of two masks of the same tensor and pruned by the other."""
+    a = np.ascontiguousarray(keep_a, np.uint8)
+    b = np.ascontiguousarray(keep_b, np.uint8)
+    assert a.shape == b.shape
+    return int(_lib().oracle_count_mask_flips(_ptr(a), _ptr(b), a.size))

@@ -282,3 +282,30 @@ void oracle_rescale(const int32_t *acc, const float *s, float g, int64_t T, int6
     for (int64_t o = 0; o < O; ++o)
       y[t * O + o] = (double)acc[t * O + o] * (double)g * (double)s[t] / 127.0;
 }
+
+/*
+ * Mask statistics, by-products of S2-S3 that follow how the masks evolve in training.
+ *
+ * Natural zeros [SBN-es §3 "Contribuciones Clave" item 1 (the "quantisation valley": a
+ * large share of the ternary weights is 0); SBN-ar §1, the hypothesis bullet]: the number
+ * of positions whose ternary code t (S2, before the mask) is 0.
+ */
+int64_t oracle_count_zero_codes(const int8_t *t, int64_t n) {
+  int64_t c = 0;
+  for (int64_t i = 0; i < n; ++i)
+    if (t[i] == 0) ++c;
+  return c;
+}
+
+/*
+ * Mask flips [SBN-es §2 "Recomputación Dinámica de Máscaras"; SBN-ar §2 dynamic
+ * recomputation: the mask is rebuilt every step from the current masters, so the
+ * topology moves]: the number of positions kept by one of two masks of the same tensor
+ * and pruned by the other.
+ */
+int64_t oracle_count_mask_flips(const uint8_t *keep_a, const uint8_t *keep_b, int64_t n) {
+  int64_t c = 0;
+  for (int64_t i = 0; i < n; ++i)
+    if ((keep_a[i] != 0) != (keep_b[i] != 0)) ++c;
+  return c;
+}

@@ -17,6 +17,9 @@ What pins what:
   invariants          code range, no 0b10 pattern, N bits per group, zero padding
   scale_invariance    W -> 2W leaves the mask and codes unchanged and doubles gamma
   rescale_closed_form S7, against acc * g * s / 127 recomputed with Fraction
+  mask_stats          natural-zero and mask-flip counts: hand-worked values (golden file),
+                      a closed form, and the invariances of the mask (sign, power-of-two
+                      scale, dense pattern)
 """
 import itertools
 import math
@@ -306,6 +309,33 @@ def rescale_closed_form(o):
             assert abs(Fraction(float(y[t, j])) - want) <= abs(want) * Fraction(1, 2 ** 50)
 
 
+def mask_stats(o):
+    g = _read_golden("hand_example_2of4.txt")
+    n, m = int(g["n"][0]), int(g["m"][0])
+    W = workloads.to_bf16_bits(np.array([[float(v) for v in g["W"]]], np.float32))
+    W2 = workloads.to_bf16_bits(np.array([[float(v) for v in g["W2"]]], np.float32))
+    r1 = o.quantize_mask_pack(W, n, m, eps=float(g["eps"][0]))
+    r2 = o.quantize_mask_pack(W2, n, m, eps=float(g["eps"][0]))
+    assert o.count_zero_codes(r1["t"]) == int(g["zeros"][0])
+    assert o.count_mask_flips(r1["keep"], r2["keep"]) == int(g["flips"][0])
+    assert o.count_mask_flips(r2["keep"], r1["keep"]) == int(g["flips"][0])
+    # closed form: three exact zeros and five weights of magnitude 1 give mean |W| = 5/8,
+    # 1 / (5/8) = 1.6 -> code +-1, so exactly the three zeros are natural zeros
+    Wc = workloads.to_bf16_bits(np.array([[0, 1, -1, 0, 1, 1, 0, -1]], np.float32))
+    assert o.count_zero_codes(o.quantize_mask_pack(Wc, 2, 4, eps=0.0)["t"]) == 3
+    # the mask depends on the master magnitudes only, and W -> 2W keeps their order: no
+    # flips; with n == m every position is kept whatever the weights
+    Wt = _tie_heavy_masters(6, 64, seed=11)
+    W2x = workloads.to_bf16_bits(workloads.bf16_bits_to_f32(Wt) * np.float32(2.0))
+    for (nn, mm) in [(2, 4), (6, 8), (3, 8), (1, 4)]:
+        k = o.quantize_mask_pack(Wt, nn, mm)["keep"]
+        assert o.count_mask_flips(k, o.quantize_mask_pack(Wt ^ np.uint16(0x8000), nn, mm)["keep"]) == 0
+        assert o.count_mask_flips(k, o.quantize_mask_pack(W2x, nn, mm)["keep"]) == 0
+    Wr = workloads.masters(6, 64, seed=12)
+    assert o.count_mask_flips(o.quantize_mask_pack(Wt, 8, 8)["keep"],
+                              o.quantize_mask_pack(Wr, 8, 8)["keep"]) == 0
+
+
 ALL = [hand_example, mask_bruteforce, gamma_closed_form, rounding_ties, dense_pattern,
        constant_magnitude, act_absmax, contract_bruteforce, unpack_roundtrip, invariants,
-       scale_invariance, rescale_closed_form]
+       scale_invariance, rescale_closed_form, mask_stats]

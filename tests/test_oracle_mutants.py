@@ -38,6 +38,9 @@ MUTANTS = [
     ("rescale_qb_128", "(double)s[t] / 127.0", "(double)s[t] / 128.0"),
     ("rescale_drops_g", "(double)acc[t * O + o] * (double)g * (double)s[t]",
      "(double)acc[t * O + o] * (double)s[t]"),
+    ("zero_count_counts_nonzeros", "if (t[i] == 0) ++c;", "if (t[i] != 0) ++c;"),
+    ("flips_one_direction", "if ((keep_a[i] != 0) != (keep_b[i] != 0)) ++c;",
+     "if (keep_a[i] && !keep_b[i]) ++c;"),
 ]
 
 
