@@ -488,6 +488,7 @@ def run_model(args, cfg):
     peaks = load_peaks()
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.Stream(device=dev)
+    extra = {}
     if cfg["kind"] == "stack":
         T, n, m = cfg["T"], 2, 4
         lin = []
@@ -567,6 +568,7 @@ def run_model(args, cfg):
         metric_value, unit = moved * world / per_step / 1e9, "GB/s"
         detail = {"tensors": len(lin), "weights": weights, "bytes_per_step": moved,
                   "patterns": ["6:8", "2:4"]}
+        extra["mask_stats"] = mask_stats(sbn, lin, ws, err, stream, dev, peaks)
     flag = int(err.item())
     if rank == 0:
         print(json.dumps({
@@ -577,9 +579,54 @@ def run_model(args, cfg):
             "on the GPU N(0,0.02); Student-t(4) activations)",
             "config": {"workload": cfg["name"], **detail,
                        "l2": "working set of GBs > 126 MB L2"},
-            "roofline": roof, "err_flag": flag, "clocks": clocks}))
+            "roofline": roof, "err_flag": flag, "clocks": clocks, **extra}))
     if flag:
         sys.exit(1)
+
+
+def mask_stats(sbn, lin, ws, err, stream, dev, peaks):
+    """The training-step mask statistics, after the timed steps: natural zeros of every
+    tensor (one read of W each) and mask flips of both patterns against the next step's
+    masters (W plus N(0, 1e-3^2) noise, packed here), timed with CUDA events around the
+    counting calls only.  Algorithmic bytes: 2 B per weight for the zero count, two meta
+    planes per flip count."""
+    zeros = torch.zeros(1, dtype=torch.int64, device=dev)
+    flips = {(6, 8): torch.zeros(1, dtype=torch.int64, device=dev),
+             (2, 4): torch.zeros(1, dtype=torch.int64, device=dev)}
+    nxt = []
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4)
+    with torch.cuda.stream(stream):
+        for O, K, W, outs in lin:
+            W2 = (W.float() + 1e-3 * torch.randn(W.shape, generator=gen, device=dev)).bfloat16()
+            packs = {}
+            for (n, m) in outs:
+                d = sbn.sbn_linear_ref_dims(O, K, n, m)
+                c = torch.empty((O, d.codes_ld), dtype=torch.uint8, device=dev)
+                mt = torch.empty((O, d.meta_ld), dtype=torch.uint8, device=dev)
+                gm = torch.empty(1, dtype=torch.float32, device=dev)
+                sbn.sbn_quantize_mask_pack_weights(W2, n, m, 1e-5, c, mt, gm, ws, None, err)
+                packs[(n, m)] = mt
+            del W2
+            nxt.append(packs)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for (O, K, W, outs), packs in zip(lin, nxt):
+            sbn.sbn_count_zero_codes(W, outs[(6, 8)][2], zeros)
+            for (n, m), (c, mt, gm) in outs.items():
+                sbn.sbn_count_mask_flips(mt, packs[(n, m)], O, K, n, m, flips[(n, m)])
+        e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    weights = sum(O * K for O, K, _, _ in lin)
+    moved = weights * 2 + 2 * 2 * (weights // 8)  # W once; two meta planes per pattern
+    gbs = moved / (ms * 1e-3) / 1e9
+    return {"natural_zero_frac": int(zeros.item()) / weights,
+            "flip_frac_6of8": int(flips[(6, 8)].item()) / weights,
+            "flip_frac_2of4": int(flips[(2, 4)].item()) / weights,
+            "ms": ms, "GB/s": gbs, "frac_of_hbm": gbs / peaks["hbm"],
+            "kernels": "k_count_zero_codes, k_count_mask_flips (130 tensors each)",
+            "next_step": "masters + N(0, 1e-3^2) noise"}
 
 
 def run_only(args, cfg):

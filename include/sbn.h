@@ -174,6 +174,28 @@ SBN_API sbn_status sbn_linear(const int8_t *Xq, const float *absmax, const uint8
                       int64_t out, int64_t in, int n, int m, void *Y, int y_is_bf16,
                       int32_t *acc_dbg, int32_t *err_flag, void *stream);
 
+/*
+ * Mask statistics: by-products of steps 2-3 that follow how the masks evolve over training
+ * steps (Sparse-BitNet summaries: section 3 "Contribuciones Clave" item 1, the large share
+ * of ternary zeros; section 2, the mask recomputed every step from the current masters).
+ * Both calls ADD their count into *count, one uint64 in device memory (8-byte aligned)
+ * that the caller zeroes before the first call; several calls may accumulate into it.
+ *
+ * sbn_count_zero_codes: the number of weights of W (bf16 [out, in]) whose ternary code
+ *   (step 2, before the mask) is 0, for g = *gamma_eff as written by
+ *   sbn_quantize_mask_pack_weights for the same W.  Weights that are NaN, or a g that is
+ *   not a finite positive number or zero, give an unspecified count.
+ * sbn_count_mask_flips: the number of positions whose keep bit differs between two meta
+ *   planes written by sbn_quantize_mask_pack_weights for the same (out, in, n, m) (for
+ *   instance the masks of two training steps).
+ * Shape, pattern and alignment rules are those of sbn_quantize_mask_pack_weights.
+ */
+SBN_API sbn_status sbn_count_zero_codes(const void *W, const float *gamma_eff, int64_t out,
+                                        int64_t in, unsigned long long *count, void *stream);
+SBN_API sbn_status sbn_count_mask_flips(const uint8_t *meta_a, const uint8_t *meta_b,
+                                        int64_t out, int64_t in, int n, int m,
+                                        unsigned long long *count, void *stream);
+
 /* A static, human-readable name for a status code. */
 SBN_API const char *sbn_status_string(sbn_status s);
 

@@ -67,6 +67,10 @@ def lib():
         L.sbn_quantize_acts.restype = i32
         L.sbn_linear.argtypes = [p, p, p, p, p, i64, i64, i64, i32, i32, p, i32, p, p, p]
         L.sbn_linear.restype = i32
+        L.sbn_count_zero_codes.argtypes = [p, p, i64, i64, p, p]
+        L.sbn_count_zero_codes.restype = i32
+        L.sbn_count_mask_flips.argtypes = [p, p, i64, i64, i32, i32, p, p]
+        L.sbn_count_mask_flips.restype = i32
         L.sbn_status_string.argtypes = [i32]
         L.sbn_status_string.restype = ctypes.c_char_p
         _LIB = L
@@ -151,6 +155,20 @@ class PackedWeights(NamedTuple):
     m: int
 
 
+def sbn_count_zero_codes(W, gamma_eff, count, stream=None):
+    """Adds to count (int64 [1], caller-zeroed) the weights of W whose ternary code is 0."""
+    out, in_ = W.shape
+    _check(lib().sbn_count_zero_codes(_ptr(W), _ptr(gamma_eff), out, in_, _ptr(count),
+                                      _stream(stream)), "sbn_count_zero_codes")
+
+
+def sbn_count_mask_flips(meta_a, meta_b, out, in_, n, m, count, stream=None):
+    """Adds to count (int64 [1], caller-zeroed) the positions whose keep bit differs between
+    two meta planes of the same (out, in, n, m)."""
+    _check(lib().sbn_count_mask_flips(_ptr(meta_a), _ptr(meta_b), out, in_, n, m, _ptr(count),
+                                      _stream(stream)), "sbn_count_mask_flips")
+
+
 def new_workspace(out: int, in_: int, n: int, m: int, device="cuda") -> torch.Tensor:
     """Pack workspace (reusable by later calls on the same stream)."""
     d = sbn_linear_ref_dims(out, in_, n, m)
@@ -189,6 +207,24 @@ def linear(Xq: torch.Tensor, s: torch.Tensor, w: PackedWeights, out_dtype=torch.
 
 
 _SIDE_STREAMS = {}
+
+
+def count_zero_codes(W: torch.Tensor, w: "PackedWeights", stream=None) -> torch.Tensor:
+    """Natural zeros of W (codes that are 0 before the mask) for the scale of its pack w;
+    an int64 [1] device tensor."""
+    count = torch.zeros(1, dtype=torch.int64, device=W.device)
+    sbn_count_zero_codes(W, w.gamma_eff, count, stream)
+    return count
+
+
+def count_mask_flips(a: "PackedWeights", b: "PackedWeights", stream=None) -> torch.Tensor:
+    """Positions kept by one of two packs of the same shape and pattern and pruned by the
+    other; an int64 [1] device tensor."""
+    if (a.out, a.in_, a.n, a.m) != (b.out, b.in_, b.n, b.m):
+        raise ValueError("mask flips need two packs of the same shape and pattern")
+    count = torch.zeros(1, dtype=torch.int64, device=a.meta.device)
+    sbn_count_mask_flips(a.meta, b.meta, a.out, a.in_, a.n, a.m, count, stream)
+    return count
 
 
 def _side_stream(device: torch.device):

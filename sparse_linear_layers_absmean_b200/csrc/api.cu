@@ -118,4 +118,30 @@ sbn_status sbn_linear(const int8_t *Xq, const float *absmax, const uint8_t *code
                              d.codes_ld, d.meta_ld, Y, y_is_bf16, acc_dbg, err_flag, s);
 }
 
+sbn_status sbn_count_zero_codes(const void *W, const float *gamma_eff, int64_t out, int64_t in,
+                                unsigned long long *count, void *stream) {
+  sbn_dims d;
+  sbn_status st = sbn_linear_ref_dims(out, in, 2, 4, &d);  // the shape rules of the pack
+  if (st != SBN_OK) return st;
+  if (!W || !gamma_eff || !count) return SBN_ERR_NULL;
+  if (!aligned16(W) || (reinterpret_cast<uintptr_t>(gamma_eff) & 3u) ||
+      (reinterpret_cast<uintptr_t>(count) & 7u))
+    return SBN_ERR_ALIGN;
+  return sbn::launch_count_zero_codes(W, out * in, gamma_eff, count,
+                                      static_cast<cudaStream_t>(stream));
+}
+
+sbn_status sbn_count_mask_flips(const uint8_t *meta_a, const uint8_t *meta_b, int64_t out,
+                                int64_t in, int n, int m, unsigned long long *count,
+                                void *stream) {
+  sbn_dims d;
+  sbn_status st = sbn_linear_ref_dims(out, in, n, m, &d);
+  if (st != SBN_OK) return st;
+  if (!meta_a || !meta_b || !count) return SBN_ERR_NULL;
+  if (!aligned16(meta_a) || !aligned16(meta_b) || (reinterpret_cast<uintptr_t>(count) & 7u))
+    return SBN_ERR_ALIGN;
+  return sbn::launch_count_mask_flips(meta_a, meta_b, d.meta_bytes, n == 2 && m == 4, count,
+                                      static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

@@ -79,6 +79,14 @@ sbn_status launch_gemm_tc(const int8_t *Xq, const float *absmax, const uint8_t *
                           void *Y, int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag,
                           cudaStream_t st);
 
+// Mask statistics (stats.cu): natural zeros of W for the scale *gamma_eff (n weights),
+// and keep-bit differences between two meta planes of nbytes bytes each (index-pair
+// nibbles for 2:4, keep masks otherwise).  Both add into *count.
+sbn_status launch_count_zero_codes(const void *W, int64_t n, const float *gamma_eff,
+                                   unsigned long long *count, cudaStream_t st);
+sbn_status launch_count_mask_flips(const uint8_t *meta_a, const uint8_t *meta_b, int64_t nbytes,
+                                   bool index_pairs, unsigned long long *count, cudaStream_t st);
+
 // Largest token count routed to the CUDA-core kernel; larger calls use the tensor cores.
 constexpr int64_t kGemvMaxTokens = 4;
 

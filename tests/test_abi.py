@@ -93,6 +93,25 @@ def test_entry_points_validate_before_launching(L):
     assert ln(A, A, A, A, A, 0, 8, 64, 2, 4, A, 0, None, None, None) == 0
 
 
+def test_statistics_entry_points_validate(L):
+    A = _p(0x10000)
+    U = _p(0x10004)   # 4-byte aligned only
+    z = L.sbn_count_zero_codes
+    assert z(None, A, 8, 64, A, None) == 1
+    assert z(A, A, 8, 64, None, None) == 1
+    assert z(A, A, 8, 96, A, None) == 2
+    assert z(A, A, 0, 64, A, None) == 2
+    assert z(U, A, 8, 64, A, None) == 4
+    assert z(A, A, 8, 64, U, None) == 4   # the uint64 count must be 8-byte aligned
+    f = L.sbn_count_mask_flips
+    assert f(None, A, 8, 64, 2, 4, A, None) == 1
+    assert f(A, A, 8, 64, 2, 4, None, None) == 1
+    assert f(A, A, 8, 96, 2, 4, A, None) == 2
+    assert f(A, A, 8, 64, 5, 4, A, None) == 3
+    assert f(A, U, 8, 64, 2, 4, A, None) == 4
+    assert f(A, A, 8, 64, 6, 8, U, None) == 4
+
+
 def test_status_strings(L):
     for s in range(7):
         assert L.sbn_status_string(s)

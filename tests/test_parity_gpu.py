@@ -235,3 +235,40 @@ def test_forward_public_api(T, n, m):
         del W, X  # freed while the side stream may still read X: record_stream keeps it
         y = Y.cpu().numpy()
     gpu_path.assert_y_close(y, ref["y"])
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (6, 8), (1, 4), (3, 8), (8, 8)])
+@pytest.mark.parametrize("O,K", [(1, 64), (37, 192), (300, 2560), (1000, 4096)])
+def test_mask_stats(O, K, n, m):
+    """Natural zeros and mask flips between two training steps (the masters plus small
+    noise, and a copy with tie-heavy rows) against the oracle's counts."""
+    import sparse_linear_layers_absmean_b200 as sbn
+    W1 = workloads.masters(O, K, seed=O + K + n)
+    rng = np.random.default_rng(O * K + m)
+    W2f = workloads.bf16_bits_to_f32(W1) + rng.normal(0.0, 1e-3, size=(O, K)).astype(np.float32)
+    W2 = workloads.to_bf16_bits(W2f.astype(np.float32))
+    W2[::3] = workloads.to_bf16_bits(np.round(workloads.bf16_bits_to_f32(W1[::3]) * 64) / 64)
+    r1 = oracle.quantize_mask_pack(W1, n, m)
+    r2 = oracle.quantize_mask_pack(W2, n, m)
+    Wd1, Wd2 = workloads.torch_bf16(W1, "cuda"), workloads.torch_bf16(W2, "cuda")
+    p1, p2 = sbn.pack_weights(Wd1, n, m), sbn.pack_weights(Wd2, n, m)
+    z1 = int(sbn.count_zero_codes(Wd1, p1).item())
+    z2 = int(sbn.count_zero_codes(Wd2, p2).item())
+    flips = int(sbn.count_mask_flips(p1, p2).item())
+    assert z1 == oracle.count_zero_codes(r1["t"])
+    assert z2 == oracle.count_zero_codes(r2["t"])
+    assert flips == oracle.count_mask_flips(r1["keep"], r2["keep"])
+    assert int(sbn.count_mask_flips(p1, p1).item()) == 0
+    # the counts accumulate into a caller-zeroed counter
+    c = torch.zeros(1, dtype=torch.int64, device="cuda")
+    sbn.sbn_count_zero_codes(Wd1, p1.gamma_eff, c)
+    sbn.sbn_count_zero_codes(Wd2, p2.gamma_eff, c)
+    assert int(c.item()) == z1 + z2
+
+
+def test_mask_stats_all_zero_tensor():
+    """g = 0 (all-zero masters, eps = 0): every code is 0."""
+    import sparse_linear_layers_absmean_b200 as sbn
+    W = torch.zeros((16, 128), dtype=torch.bfloat16, device="cuda")
+    w = sbn.pack_weights(W, 2, 4, eps=0.0)
+    assert int(sbn.count_zero_codes(W, w).item()) == 16 * 128
