@@ -64,22 +64,25 @@ __global__ void __launch_bounds__(kStThreads)
   add_cta_count(c, count);
 }
 
-// Eight 2:4 metadata nibbles (i0 | i1 << 2) -> eight keep nibbles (bits i0 and i1).  A zero
-// padding nibble maps to the same keep nibble in both planes.
-__device__ __forceinline__ uint32_t keep_of_index_pairs(uint32_t w) {
-  uint32_t k = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint32_t nib = (w >> (4 * j)) & 15u;
-    k |= ((1u << (nib & 3u)) | (1u << (nib >> 2))) << (4 * j);
-  }
-  return k;
+// A 2:4 metadata byte (two nibbles i0 | i1 << 2) -> its keep byte (bits i0 and i1 of each
+// nibble).  A zero padding byte maps to the same keep byte in both planes.
+__device__ __forceinline__ uint32_t keep_byte_of_index_pairs(uint32_t b) {
+  const uint32_t n0 = b & 15u, n1 = (b >> 4) & 15u;
+  return ((1u << (n0 & 3u)) | (1u << (n0 >> 2))) | (((1u << (n1 & 3u)) | (1u << (n1 >> 2))) << 4);
+}
+
+__device__ __forceinline__ uint32_t keep_word(const uint8_t *s_keep, uint32_t w) {
+  return (uint32_t)s_keep[w & 255u] | ((uint32_t)s_keep[(w >> 8) & 255u] << 8) |
+         ((uint32_t)s_keep[(w >> 16) & 255u] << 16) | ((uint32_t)s_keep[w >> 24] << 24);
 }
 
 __global__ void __launch_bounds__(kStThreads)
     k_count_mask_flips(const uint4 *__restrict__ a, const uint4 *__restrict__ b, int64_t nvec,
                        int index_pairs, unsigned long long *count) {
+  __shared__ uint8_t s_keep[256];  // 2:4: metadata byte -> keep byte
   ptx::grid_dep_launch();
+  s_keep[threadIdx.x] = (uint8_t)keep_byte_of_index_pairs(threadIdx.x);
+  __syncthreads();
   ptx::grid_dep_wait();  // the previous kernel on the stream (the pack) wrote the planes
   uint32_t c = 0;
   const int64_t stride = (int64_t)gridDim.x * kStThreads;
@@ -97,7 +100,7 @@ __global__ void __launch_bounds__(kStThreads)
       const uint32_t wb[4] = {vb[u].x, vb[u].y, vb[u].z, vb[u].w};
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        c += index_pairs ? __popc(keep_of_index_pairs(wa[q]) ^ keep_of_index_pairs(wb[q]))
+        c += index_pairs ? __popc(keep_word(s_keep, wa[q]) ^ keep_word(s_keep, wb[q]))
                          : __popc(wa[q] ^ wb[q]);
     }
   }
