@@ -47,6 +47,8 @@ def load_library(path):
     lib.oracle_count_zero_codes.restype = i64
     lib.oracle_count_mask_flips.argtypes = [p, p, i64]
     lib.oracle_count_mask_flips.restype = i64
+    lib.oracle_backward.argtypes = [p, p, p, p, ctypes.c_float, i64, i64, i64, p, p]
+    lib.oracle_backward.restype = None
     if not lib.oracle_rounding_is_nearest():
         raise RuntimeError("oracle needs round-to-nearest-even on the host FPU")
     return lib
@@ -196,3 +198,20 @@ def count_mask_flips(keep_a, keep_b):
     b = np.ascontiguousarray(keep_b, np.uint8)
     assert a.shape == b.shape
     return int(_lib().oracle_count_mask_flips(_ptr(a), _ptr(b), a.size))
+
+
+def backward(dY, Xq, s, Ws, g):
+    """Dual-STE backward: (dX [T, K], dW [O, K]) in fp64 for the forward's effective
+    operands W_eff = g * Ws and X_eff = s / 127 * Xq; dW reaches every master weight."""
+    dY = np.ascontiguousarray(dY, np.float32)
+    Xq = np.ascontiguousarray(Xq, np.int8)
+    s = np.ascontiguousarray(s, np.float32)
+    Ws = np.ascontiguousarray(Ws, np.int8)
+    T, O = dY.shape
+    O2, K = Ws.shape
+    assert O == O2 and Xq.shape == (T, K) and s.shape == (T,)
+    dX = np.empty((T, K), np.float64)
+    dW = np.empty((O, K), np.float64)
+    _lib().oracle_backward(_ptr(dY), _ptr(Xq), _ptr(s), _ptr(Ws), ctypes.c_float(float(g)), T, O,
+                           K, _ptr(dX), _ptr(dW))
+    return dX, dW

@@ -309,3 +309,36 @@ int64_t oracle_count_mask_flips(const uint8_t *keep_a, const uint8_t *keep_b, in
     if ((keep_a[i] != 0) != (keep_b[i] != 0)) ++c;
   return c;
 }
+
+/*
+ * Backward of the layer under the dual straight-through estimator [SBN-es §2 "Estrategia
+ * de Entrenamiento", "Estimador de Paso Directo Dual": quantisation and mask selection
+ * are not differentiable, so both pass gradients as the identity, and the gradient reaches
+ * every master weight, the pruned ones included].  The forward's effective operands are
+ *   W_eff[o, k] = g * Ws[o, k]            (the dequantised masked codes)
+ *   X_eff[t, k] = s[t] / 127 * Xq[t, k]   (the dequantised activations)
+ * and, in fp64,
+ *   dX[t, k] = sum_o dY[t, o] * W_eff[o, k]
+ *   dW[o, k] = sum_t dY[t, o] * X_eff[t, k]   (dense: neither the mask nor the ternary
+ *                                              quantiser stops it)
+ * dY is [T, O] fp32; dX is [T, K] and dW is [O, K] fp64.
+ */
+void oracle_backward(const float *dY, const int8_t *Xq, const float *s, const int8_t *Ws,
+                     float g, int64_t T, int64_t O, int64_t K, double *dX, double *dW) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t)
+    for (int64_t k = 0; k < K; ++k) {
+      double acc = 0.0;
+      for (int64_t o = 0; o < O; ++o)
+        acc += (double)dY[t * O + o] * ((double)g * (double)Ws[o * K + k]);
+      dX[t * K + k] = acc;
+    }
+#pragma omp parallel for schedule(static)
+  for (int64_t o = 0; o < O; ++o)
+    for (int64_t k = 0; k < K; ++k) {
+      double acc = 0.0;
+      for (int64_t t = 0; t < T; ++t)
+        acc += (double)dY[t * O + o] * (((double)s[t]) / 127.0 * (double)Xq[t * K + k]);
+      dW[o * K + k] = acc;
+    }
+}

@@ -20,6 +20,10 @@ What pins what:
   mask_stats          natural-zero and mask-flip counts: hand-worked values (golden file),
                       a closed form, and the invariances of the mask (sign, power-of-two
                       scale, dense pattern)
+  backward_hand       dual-STE backward on the hand-worked example (golden file): the
+                      pruned position still receives its weight gradient
+  backward_adjoint    <dY, y> = <dX, X_eff> = <dW, W_eff> against the forward's y, and dW
+                      independent of the mask
 """
 import itertools
 import math
@@ -336,6 +340,42 @@ def mask_stats(o):
                               o.quantize_mask_pack(Wr, 8, 8)["keep"]) == 0
 
 
+def backward_hand(o):
+    g = _read_golden("hand_example_2of4.txt")
+    n, m = int(g["n"][0]), int(g["m"][0])
+    W = workloads.to_bf16_bits(np.array([[float(v) for v in g["W"]]], np.float32))
+    X = workloads.to_bf16_bits(np.array([[float(v) for v in g["x"]]], np.float32))
+    r = o.linear(X, W, n, m, eps=float(g["eps"][0]))
+    dY = np.array([[float(g["dY"][0])]], np.float32)
+    dX, dW = o.backward(dY, r["Xq"], r["s"], r["ws"], r["g"])
+    gamma = Fraction(g["gamma"][0])
+    for k, v in enumerate(g["dX_over_gamma"]):
+        assert Fraction(float(dX[0, k])) == gamma * int(v), (k, dX[0, k])
+    den = int(g["dW_den"][0])
+    for k, v in enumerate(g["dW_num"]):
+        assert abs(Fraction(float(dW[0, k])) - Fraction(int(v), den)) <= Fraction(1, 2 ** 48)
+
+
+def backward_adjoint(o):
+    rng = np.random.default_rng(21)
+    T, O, K = 3, 5, 64
+    W = _tie_heavy_masters(O, K, seed=22)
+    X = workloads.activations(T, K, seed=23)
+    r = o.linear(X, W, 2, 4)
+    dY = rng.standard_normal((T, O)).astype(np.float32)
+    dX, dW = o.backward(dY, r["Xq"], r["s"], r["ws"], r["g"])
+    X_eff = r["Xq"].astype(np.float64) * (r["s"].astype(np.float64) / 127.0)[:, None]
+    W_eff = r["ws"].astype(np.float64) * float(r["g"])
+    lhs = float(np.sum(dY.astype(np.float64) * r["y"]))
+    for rhs in (float(np.sum(dX * X_eff)), float(np.sum(dW * W_eff))):
+        assert abs(lhs - rhs) <= 1e-9 * max(1.0, abs(lhs)), (lhs, rhs)
+    # the weight gradient does not depend on the mask (dense n == m gives the same dW)
+    rd = o.linear(X, W, 4, 4)
+    _, dWd = o.backward(dY, rd["Xq"], rd["s"], rd["ws"], rd["g"])
+    assert np.array_equal(dW, dWd)
+    assert np.any(dW[r["keep"] == 0] != 0)
+
+
 ALL = [hand_example, mask_bruteforce, gamma_closed_form, rounding_ties, dense_pattern,
        constant_magnitude, act_absmax, contract_bruteforce, unpack_roundtrip, invariants,
-       scale_invariance, rescale_closed_form, mask_stats]
+       scale_invariance, rescale_closed_form, mask_stats, backward_hand, backward_adjoint]

@@ -41,6 +41,14 @@ MUTANTS = [
     ("zero_count_counts_nonzeros", "if (t[i] == 0) ++c;", "if (t[i] != 0) ++c;"),
     ("flips_one_direction", "if ((keep_a[i] != 0) != (keep_b[i] != 0)) ++c;",
      "if (keep_a[i] && !keep_b[i]) ++c;"),
+    ("backward_dw_masked",
+     "acc += (double)dY[t * O + o] * (((double)s[t]) / 127.0 * (double)Xq[t * K + k]);",
+     "acc += (double)dY[t * O + o] * (((double)s[t]) / 127.0 * (double)Xq[t * K + k]) *"
+     " (Ws[o * K + k] != 0);"),
+    ("backward_dx_drops_g", "acc += (double)dY[t * O + o] * ((double)g * (double)Ws[o * K + k]);",
+     "acc += (double)dY[t * O + o] * ((double)Ws[o * K + k]);"),
+    ("backward_dw_unscaled_acts", "(((double)s[t]) / 127.0 * (double)Xq[t * K + k])",
+     "((double)Xq[t * K + k])"),
 ]
 
 
