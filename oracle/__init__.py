@@ -47,7 +47,7 @@ def load_library(path):
     lib.oracle_count_zero_codes.restype = i64
     lib.oracle_count_mask_flips.argtypes = [p, p, i64]
     lib.oracle_count_mask_flips.restype = i64
-    lib.oracle_backward.argtypes = [p, p, p, p, ctypes.c_float, i64, i64, i64, p, p]
+    lib.oracle_backward.argtypes = [p, p, p, p, p, ctypes.c_float, i64, i64, i64, p, p]
     lib.oracle_backward.restype = None
     if not lib.oracle_rounding_is_nearest():
         raise RuntimeError("oracle needs round-to-nearest-even on the host FPU")
@@ -200,18 +200,20 @@ def count_mask_flips(keep_a, keep_b):
     return int(_lib().oracle_count_mask_flips(_ptr(a), _ptr(b), a.size))
 
 
-def backward(dY, Xq, s, Ws, g):
+def backward(dY, Xq, s, Ws, W_bits, g):
     """Dual-STE backward: (dX [T, K], dW [O, K]) in fp64 for the forward's effective
-    operands W_eff = g * Ws and X_eff = s / 127 * Xq; dW reaches every master weight."""
+    operands W_eff = g * Ws and X_eff = s / 127 * Xq.  dW reaches every master weight the
+    mask pruned, and is zero where the quantiser clips (fl32(|W| / g) > 1)."""
     dY = np.ascontiguousarray(dY, np.float32)
     Xq = np.ascontiguousarray(Xq, np.int8)
     s = np.ascontiguousarray(s, np.float32)
     Ws = np.ascontiguousarray(Ws, np.int8)
+    W_bits = np.ascontiguousarray(W_bits, np.uint16)
     T, O = dY.shape
     O2, K = Ws.shape
-    assert O == O2 and Xq.shape == (T, K) and s.shape == (T,)
+    assert O == O2 and Xq.shape == (T, K) and s.shape == (T,) and W_bits.shape == (O, K)
     dX = np.empty((T, K), np.float64)
     dW = np.empty((O, K), np.float64)
-    _lib().oracle_backward(_ptr(dY), _ptr(Xq), _ptr(s), _ptr(Ws), ctypes.c_float(float(g)), T, O,
-                           K, _ptr(dX), _ptr(dW))
+    _lib().oracle_backward(_ptr(dY), _ptr(Xq), _ptr(s), _ptr(Ws), _ptr(W_bits),
+                           ctypes.c_float(float(g)), T, O, K, _ptr(dX), _ptr(dW))
     return dX, dW

@@ -313,18 +313,26 @@ int64_t oracle_count_mask_flips(const uint8_t *keep_a, const uint8_t *keep_b, in
 /*
  * Backward of the layer under the dual straight-through estimator [SBN-es §2 "Estrategia
  * de Entrenamiento", "Estimador de Paso Directo Dual": quantisation and mask selection
- * are not differentiable, so both pass gradients as the identity, and the gradient reaches
- * every master weight, the pruned ones included].  The forward's effective operands are
+ * are not differentiable, so both are passed by straight-through estimators, and the
+ * gradient reaches every master weight, the pruned ones included; SBN-ar §2, Sparse-BitLinear
+ * item 3: the quantisation STE is the identity inside the clipping range, the mask STE
+ * sends a dense gradient to all masters].  The forward's effective operands are
  *   W_eff[o, k] = g * Ws[o, k]            (the dequantised masked codes)
  *   X_eff[t, k] = s[t] / 127 * Xq[t, k]   (the dequantised activations)
  * and, in fp64,
  *   dX[t, k] = sum_o dY[t, o] * W_eff[o, k]
- *   dW[o, k] = sum_t dY[t, o] * X_eff[t, k]   (dense: neither the mask nor the ternary
- *                                              quantiser stops it)
- * dY is [T, O] fp32; dX is [T, K] and dW is [O, K] fp64.
+ *   dW[o, k] = pass[o, k] * sum_t dY[t, o] * X_eff[t, k]
+ * where pass[o, k] is the quantisation STE: with round() taken as the identity the
+ * quantiser is clip(W / g, -1, 1), whose derivative is 1 for |W / g| <= 1 and 0 outside
+ * (the boundary included, as a clamp's gradient is).  The quotient is the fp32 one the
+ * codes are decided from: pass = (fl32(|W| / g) <= 1).  The mask does not enter dW.
+ * dY is [T, O] fp32; W holds the bf16 masters [O, K]; dX is [T, K] and dW is [O, K] fp64.
  */
+int oracle_ste_pass(float w, float g) { return fabsf(w) / g <= 1.0f; }
+
 void oracle_backward(const float *dY, const int8_t *Xq, const float *s, const int8_t *Ws,
-                     float g, int64_t T, int64_t O, int64_t K, double *dX, double *dW) {
+                     const uint16_t *W, float g, int64_t T, int64_t O, int64_t K, double *dX,
+                     double *dW) {
 #pragma omp parallel for schedule(static)
   for (int64_t t = 0; t < T; ++t)
     for (int64_t k = 0; k < K; ++k) {
@@ -339,6 +347,6 @@ void oracle_backward(const float *dY, const int8_t *Xq, const float *s, const in
       double acc = 0.0;
       for (int64_t t = 0; t < T; ++t)
         acc += (double)dY[t * O + o] * (((double)s[t]) / 127.0 * (double)Xq[t * K + k]);
-      dW[o * K + k] = acc;
+      dW[o * K + k] = oracle_ste_pass(bf16_bits_to_float(W[o * K + k]), g) ? acc : 0.0;
     }
 }

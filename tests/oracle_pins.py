@@ -20,10 +20,12 @@ What pins what:
   mask_stats          natural-zero and mask-flip counts: hand-worked values (golden file),
                       a closed form, and the invariances of the mask (sign, power-of-two
                       scale, dense pattern)
-  backward_hand       dual-STE backward on the hand-worked example (golden file): the
-                      pruned position still receives its weight gradient
-  backward_adjoint    <dY, y> = <dX, X_eff> = <dW, W_eff> against the forward's y, and dW
-                      independent of the mask
+  backward_hand       dual-STE backward on the hand-worked example (golden file): pruned
+                      positions still receive their weight gradient, clipped ones none
+  backward_adjoint    <dY, y> = <dX, X_eff> against the forward's y; <dW, V> = <dY,
+                      X_eff (V * pass)^T> for a random V (the weight gradient is the adjoint
+                      of the gated product); dW independent of the mask; the clip gate on
+                      weights placed exactly at |W| = g and next to it
 """
 import itertools
 import math
@@ -347,13 +349,15 @@ def backward_hand(o):
     X = workloads.to_bf16_bits(np.array([[float(v) for v in g["x"]]], np.float32))
     r = o.linear(X, W, n, m, eps=float(g["eps"][0]))
     dY = np.array([[float(g["dY"][0])]], np.float32)
-    dX, dW = o.backward(dY, r["Xq"], r["s"], r["ws"], r["g"])
+    dX, dW = o.backward(dY, r["Xq"], r["s"], r["ws"], W, r["g"])
     gamma = Fraction(g["gamma"][0])
     for k, v in enumerate(g["dX_over_gamma"]):
         assert Fraction(float(dX[0, k])) == gamma * int(v), (k, dX[0, k])
     den = int(g["dW_den"][0])
-    for k, v in enumerate(g["dW_num"]):
+    for k, (v, p) in enumerate(zip(g["dW_num"], g["ste_pass"])):
         assert abs(Fraction(float(dW[0, k])) - Fraction(int(v), den)) <= Fraction(1, 2 ** 48)
+        if p == "0":
+            assert dW[0, k] == 0.0, (k, dW[0, k])
 
 
 def backward_adjoint(o):
@@ -363,17 +367,43 @@ def backward_adjoint(o):
     X = workloads.activations(T, K, seed=23)
     r = o.linear(X, W, 2, 4)
     dY = rng.standard_normal((T, O)).astype(np.float32)
-    dX, dW = o.backward(dY, r["Xq"], r["s"], r["ws"], r["g"])
+    dX, dW = o.backward(dY, r["Xq"], r["s"], r["ws"], W, r["g"])
     X_eff = r["Xq"].astype(np.float64) * (r["s"].astype(np.float64) / 127.0)[:, None]
     W_eff = r["ws"].astype(np.float64) * float(r["g"])
     lhs = float(np.sum(dY.astype(np.float64) * r["y"]))
-    for rhs in (float(np.sum(dX * X_eff)), float(np.sum(dW * W_eff))):
-        assert abs(lhs - rhs) <= 1e-9 * max(1.0, abs(lhs)), (lhs, rhs)
+    rhs = float(np.sum(dX * X_eff))
+    assert abs(lhs - rhs) <= 1e-9 * max(1.0, abs(lhs)), (lhs, rhs)
+    # dW is the adjoint of V -> X_eff (V * pass)^T, pass = the clip range of W / g; the
+    # magnitudes of these masters straddle g, so both sides of the gate occur
+    ratio = np.abs(workloads.bf16_bits_to_f32(W)) / np.float32(r["g"])
+    gate = (ratio <= np.float32(1.0)).astype(np.float64)
+    assert 0 < gate.sum() < gate.size
+    for trial in range(3):
+        V = rng.standard_normal((O, K))
+        lhs = float(np.sum(dW * V))
+        rhs = float(np.sum(dY.astype(np.float64) * (X_eff @ (V * gate).T)))
+        assert abs(lhs - rhs) <= 1e-9 * max(1.0, abs(lhs)), (trial, lhs, rhs)
+    assert np.all(dW[gate == 0] == 0)
     # the weight gradient does not depend on the mask (dense n == m gives the same dW)
     rd = o.linear(X, W, 4, 4)
-    _, dWd = o.backward(dY, rd["Xq"], rd["s"], rd["ws"], rd["g"])
+    _, dWd = o.backward(dY, rd["Xq"], rd["s"], rd["ws"], W, rd["g"])
     assert np.array_equal(dW, dWd)
     assert np.any(dW[r["keep"] == 0] != 0)
+    # the gate's boundary: one row of masters that are all +-m (so g = m + eps with eps = 0
+    # gives |W| / g == 1 exactly: passes), and one with a single larger magnitude (that one
+    # is clipped, the rest pass since the mean is above their magnitude)
+    Wb = workloads.to_bf16_bits(np.array([[0.25, -0.25, 0.25, -0.25] * 16,
+                                          [0.25, -0.25, 0.25, -0.25] * 15 + [4.0, 0.25, 0.25, 0.25]],
+                                         np.float32))
+    for row in range(2):
+        rb = o.linear(X, Wb[row:row + 1], 2, 4, eps=0.0)
+        dYb = np.ones((T, 1), np.float32)
+        _, dWb = o.backward(dYb, rb["Xq"], rb["s"], rb["ws"], Wb[row:row + 1], rb["g"])
+        full = X_eff.sum(axis=0)
+        if row == 0:
+            assert np.all(dWb[0] == full)
+        else:
+            assert dWb[0, 60] == 0.0 and np.all(np.delete(dWb[0], 60) == np.delete(full, 60))
 
 
 ALL = [hand_example, mask_bruteforce, gamma_closed_form, rounding_ties, dense_pattern,

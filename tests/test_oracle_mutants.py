@@ -49,6 +49,14 @@ MUTANTS = [
      "acc += (double)dY[t * O + o] * ((double)Ws[o * K + k]);"),
     ("backward_dw_unscaled_acts", "(((double)s[t]) / 127.0 * (double)Xq[t * K + k])",
      "((double)Xq[t * K + k])"),
+    ("backward_dw_ungated",
+     "dW[o * K + k] = oracle_ste_pass(bf16_bits_to_float(W[o * K + k]), g) ? acc : 0.0;",
+     "dW[o * K + k] = acc;"),
+    ("backward_gate_round_range", "return fabsf(w) / g <= 1.0f;", "return fabsf(w) / g < 1.5f;"),
+    ("backward_gate_strict", "return fabsf(w) / g <= 1.0f;", "return fabsf(w) / g < 1.0f;"),
+    ("backward_gate_by_mask",
+     "dW[o * K + k] = oracle_ste_pass(bf16_bits_to_float(W[o * K + k]), g) ? acc : 0.0;",
+     "dW[o * K + k] = Ws[o * K + k] != 0 ? acc : 0.0;"),
 ]
 
 
