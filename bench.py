@@ -1,18 +1,31 @@
 """Benchmark of the Sparse-BitLinear forward hot path on B200.
 
-One step = the whole forward for one synthetic batch: pack the bf16 master weights
-(absmean gamma, ternary codes, N:M mask, 2-bit pack), quantise the activations to int8,
-contract and rescale.  Default workload: decode GEMV, W [6912 x 2560] 6:8, one token.
+Default workload: the largest single-GPU configuration, a 32-layer decoder stack of
+pre-packed 2:4 Sparse-BitLinear layers (hidden 4096, FFN 11008: QKV 4096->12288, O
+4096->4096, gate and up 4096->11008, down 11008->4096; 160 layers, 6.48 G weights).
+One step is the decode step of the whole stack at 16 tokens: the activation quantiser
+(step 5) and the contraction with rescale (steps 6-7) of all 160 layers, each as one
+grouped launch through the C ABI (sbn_quantize_acts_group, sbn_linear_group).  The
+weights are packed once before timing, as a server does when it loads a model.
 
-Timing: the K timed steps are captured in one CUDA graph (after W warm-up steps) and
+The same JSON line carries sub-records: the stack's 4096-token prefill (per-layer tensor-
+core contraction, TOPS), and the single-tensor configurations -- decode GEMV (W 6912x2560
+6:8, pack + act quant + GEMV per step), prefill GEMM (W 11008x4096 2:4, 2048 tokens) and
+the training-step weight path (re-pack all 130 linears of a 26-layer decoder in 6:8 and
+2:4).  Each has its own roofline and its own oracle leg.
+
+Timing: W untimed warm-up steps, then exactly K steps captured in one CUDA graph and
 replayed between a barrier + synchronize on both sides; the device time is the max over
-ranks.  Inputs rotate over R sets whose total exceeds the 126 MB L2, so every step reads
-its weights from HBM.  CUDA events recorded inside the graph bracket every C-ABI call and
-give the per-call durations used for the roofline.  nvidia-smi clocks are sampled during
-the timed region.
+ranks.  The stack's packed weights (1.62 GB) and the rotating input sets of the single-
+tensor configurations exceed the 126 MB L2, so every step reads its weights from HBM.
+Per-call durations come from a second graph of the same steps with CUDA events recorded
+around every C-ABI call on the streams the calls run on.  nvidia-smi clocks are sampled
+during the timed region.
 
 `--impl reference` times the CPU oracle (test infrastructure) on a bounded sample of the
-same workload instead.
+same workload instead.  `--gpus N` without torchrun relaunches itself under torchrun with
+N local ranks; each rank runs its own replica of the workload on its own seeded inputs
+(weak scaling, no collective in the data path).
 """
 import argparse
 import json
@@ -30,44 +43,14 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import workloads  # noqa: E402
+from sparse_linear_layers_absmean_b200 import dist  # noqa: E402
 
 METRIC = "Sparse-BitLinear TOPS & packed-weight GB/s vs roofline; quant+mask GB/s"
 L2_BYTES = 126 * 1024 * 1024
-
-WORKLOADS = {
-    "decode": workloads.DECODE_GEMV,
-    "prefill": workloads.PREFILL_GEMM,
-    "tiny": workloads.TINY,
-    # whole-model configurations: a 32-layer stack of pre-packed 2:4 linears (the step is the
-    # activation quantisation and contraction of all 160 linears), and the training-step
-    # weight path (the step re-packs all 130 linears of a 26-layer decoder, 6:8 and 2:4)
-    "stack-decode": workloads.STACK_DECODE,
-    "stack-prefill": workloads.STACK_PREFILL,
-    "train-step": workloads.TRAIN_STEP,
-}
+WORKLOADS = ("stack", "decode", "prefill", "train-step", "stack-prefill")
 
 
-# ---- algorithmic bytes / ops (per step) --------------------------------------------------
-
-def packed_bytes(O, K, n, m):
-    """Bytes of the packed planes without row padding: codes + metadata."""
-    stored = K // 2 if (n, m) == (2, 4) else K
-    return O * (stored // 4), O * (K // 8)
-
-
-def step_accounting(cfg):
-    O, K, T, n, m = cfg["O"], cfg["K"], cfg["T"], cfg["n"], cfg["m"]
-    codes_b, meta_b = packed_bytes(O, K, n, m)
-    # the contraction reads the codes, and the metadata only for 2:4
-    linear_w = codes_b + (meta_b if (n, m) == (2, 4) else 0)
-    pack = 2 * O * K + codes_b + meta_b
-    act = 2 * T * K + T * K + 4 * T
-    linear = linear_w + T * K + 4 * T + 4 * T * O
-    return dict(pack=pack, act=act, linear=linear, linear_weight=linear_w,
-                ops=2 * T * O * K * n // m, total=pack + act + linear)
-
-
-# ---- helpers -----------------------------------------------------------------------------
+# ---- peaks, clocks -------------------------------------------------------------------------
 
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -77,6 +60,23 @@ def load_peaks():
         return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"],
                     bf16_sustained=d.get("bf16_tflops_sustained"), source="measured")
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def hbm_roof(achieved, peaks, kernel, traffic=None, unit_note=""):
+    return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm"], "traffic": traffic, "kernel": kernel,
+            "peak_source": f"hbm_gbs of MEASURED_PEAKS.json ({peaks['source']}: of measured)"
+                           + unit_note}
+
+
+def tensor_roof(achieved, peaks, kernel, traffic=None):
+    # int8 dense tensor peak = 2 x the measured bf16 burst peak (the nominal int8/bf16 ratio
+    # is 2); the burst figure because each contraction is timed per call, ~0.1 ms long
+    peak = 2.0 * peaks["bf16"]
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": traffic, "kernel": kernel,
+            "peak_source": f"2 x bf16_tflops (burst) of MEASURED_PEAKS.json ({peaks['source']}: "
+                           "of measured); kept int8 ops"}
 
 
 class ClockSampler:
@@ -136,56 +136,261 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def dist_setup():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    return world, rank, local
+def load_traffic(workload, call):
+    """DRAM bytes per launch of a call from the committed ncu summary, if any."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    return d.get(workload, {}).get(call)
 
 
-def barrier(world):
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
+# ---- timing harness -----------------------------------------------------------------------
+
+class Timer:
+    """Captures `steps` steps in one CUDA graph and times its replay (barrier + synchronize
+    on both sides, max over ranks), and a second graph of the same steps with external
+    events around every call for the per-call durations."""
+
+    def __init__(self, dev, local):
+        self.dev, self.local = dev, local
+        self.stream = torch.cuda.Stream(device=dev)
+
+    def run(self, step, steps, warmup, calls=(), sample_clocks=True):
+        """step(i, ev) runs step i; ev is None or a dict call -> (start, end) events to record
+        around each call on the stream it runs on.  Returns (ms per step, per-call ms, clocks)."""
+        with torch.cuda.stream(self.stream):
+            for i in range(warmup):
+                step(i, None)
+        torch.cuda.synchronize(self.dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            for i in range(steps):
+                step(i, None)
+        evs = [{c: (torch.cuda.Event(enable_timing=True, external=True),
+                    torch.cuda.Event(enable_timing=True, external=True)) for c in calls}
+               for _ in range(steps)]
+        g_ev = None
+        if calls:
+            g_ev = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_ev, stream=self.stream):
+                for i in range(steps):
+                    step(i, evs[i])
+        with torch.cuda.stream(self.stream):
+            g.replay()  # graph warm-up
+        torch.cuda.synchronize(self.dev)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        clk = ClockSampler(self.local) if sample_clocks else None
+        if clk:
+            clk.__enter__()
+        try:
+            dist.barrier(self.dev)
+            with torch.cuda.stream(self.stream):
+                t0.record()
+                g.replay()
+                t1.record()
+            torch.cuda.synchronize(self.dev)
+            dist.barrier(self.dev)
+            ms = t0.elapsed_time(t1)
+            if clk and ms < 300:  # keep the clocks sampled for at least ~0.3 s of load
+                with torch.cuda.stream(self.stream):
+                    for _ in range(max(1, int(300 / max(ms, 1e-3)))):
+                        g.replay()
+                torch.cuda.synchronize(self.dev)
+        finally:
+            if clk:
+                clk.__exit__()
+        per = {}
+        if g_ev is not None:
+            with torch.cuda.stream(self.stream):
+                g_ev.replay()
+            torch.cuda.synchronize(self.dev)
+            for c in calls:
+                per[c] = sum(e[c][0].elapsed_time(e[c][1]) for e in evs) / steps
+        del g, g_ev
+        ms = dist.max_over_ranks(ms, self.dev)
+        return ms / steps, per, (clk.summary() if clk else None)
 
 
-def max_over_ranks(x, world):
-    if world == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
+# ---- the stack (configuration 5) ----------------------------------------------------------
+
+def stack_layers(rank=0):
+    """(index, name, O, K, tensor id) of the 160 layers of one replica of the stack; rank r
+    draws its replica's weights and activations from tensor ids offset by 1000 r."""
+    out = []
+    for layer in range(workloads.STACK_LAYERS):
+        for i, (name, O, K) in enumerate(workloads.STACK_LAYER_SHAPES):
+            out.append((5 * layer + i, name, O, K, 5 * layer + i + 1000 * rank))
+    return out
 
 
-# ---- the CUDA arm ------------------------------------------------------------------------
+def build_stack(sbn, dev, rank, err):
+    """Packs the 160 layers of the stack (2:4) on the GPU from seeded masters."""
+    packed = []
+    for idx, name, O, K, tid in stack_layers(rank):
+        W = workloads.masters_device(O, K, device=dev, config=5, tensor=tid)
+        packed.append(sbn.pack_weights(W, 2, 4, err_flag=err))
+        del W
+    return packed
 
-def run_cuda(args, cfg):
-    import sparse_linear_layers_absmean_b200 as sbn
 
-    world, rank, local = dist_setup()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
+def bench_stack_decode(args, sbn, dev, local, rank, world, peaks, timer, packed, err):
+    T = workloads.STACK_DECODE_T
+    lay = stack_layers(rank)
+    # per-layer Student-t(4) activations, drawn on the host (seeded), one buffer each
+    Xh = [workloads.torch_bf16(workloads.student_t(T, K, config=5, tensor=10000 + tid))
+          for _, _, O, K, tid in lay]
+    layers = []
+    for (idx, name, O, K, tid), w, x in zip(lay, packed, Xh):
+        layers.append(dict(X=x.to(dev), Xq=torch.empty((T, K), dtype=torch.int8, device=dev),
+                           s=torch.empty((T,), dtype=torch.float32, device=dev), w=w,
+                           Y=torch.empty((T, O), dtype=torch.float32, device=dev)))
+    plan = sbn.GroupPlan(layers, device=dev)
+    st = timer.stream
+
+    def step(i, ev):
+        if ev is not None:
+            ev["act"][0].record(st)
+        plan.quantize_acts(err, st)
+        if ev is not None:
+            ev["act"][1].record(st)
+            ev["linear"][0].record(st)
+        plan.linear(err, st)
+        if ev is not None:
+            ev["linear"][1].record(st)
+
+    ms, per, clocks = timer.run(step, args.steps, args.warmup, calls=("act", "linear"))
+    weights = sum(O * K for _, _, O, K, _ in lay)
+    packed_b = weights // 4  # 2:4: K/8 code bytes + K/8 metadata bytes per row
+    act_b = sum(2 * T * K + T * K + 4 * T for _, _, _, K, _ in lay)   # read X, write Xq, s
+    lin_b = packed_b + sum(T * K + 4 * T + 4 * T * O for _, _, O, K, _ in lay)  # + read Xq, write Y
+    total = act_b + lin_b
+    roof = hbm_roof(packed_b / (per["linear"] * 1e-3) / 1e9, peaks,
+                    "k_gemm_group (grouped 2:4 contraction, 160 layers, one launch)",
+                    traffic=load_traffic("stack-decode", "linear"),
+                    unit_note="; achieved on packed-weight bytes (0.25 B per weight)")
+    rec = {
+        "value": total * world / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+        "roofline": roof,
+        "kernels": {
+            "act_quant_group": {"ms": per["act"], "GB/s": act_b / (per["act"] * 1e-3) / 1e9,
+                                "launches": 1},
+            "linear_group": {"ms": per["linear"],
+                             "packed_weight_GB/s": packed_b / (per["linear"] * 1e-3) / 1e9,
+                             "all_bytes_GB/s": lin_b / (per["linear"] * 1e-3) / 1e9,
+                             "TOPS": weights * T / (per["linear"] * 1e-3) / 1e12,
+                             "launches": 1, "units": plan.nunits, "ctas": plan.ncta,
+                             "split": plan.split}},
+        "gpu_launches": 2 * args.steps, "clocks": clocks,
+        "bytes_per_step": {"packed_weights": packed_b, "act_quant": act_b, "contraction": lin_b},
+    }
+    # e2e through the public API (GroupPlan) with pinned host buffers: every step copies its
+    # 160 activation blocks in and its 160 outputs out, and waits for them on the host
+    hostX = [x.pin_memory() for x in Xh]
+    hostY = [torch.empty(L["Y"].shape, dtype=torch.float32).pin_memory() for L in layers]
+    ke = min(args.steps, 20)
+
+    def e2e_step():
+        for L, hx in zip(layers, hostX):
+            L["X"].copy_(hx, non_blocking=True)
+        plan.quantize_acts(err, st)
+        plan.linear(err, st)
+        for L, hy in zip(layers, hostY):
+            hy.copy_(L["Y"], non_blocking=True)
+        st.synchronize()
+
+    with torch.cuda.stream(st):
+        for _ in range(3):
+            e2e_step()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(ke):
+            e2e_step()
+        b.record(st)
+    torch.cuda.synchronize(dev)
+    e2e_ms = dist.max_over_ranks(a.elapsed_time(b) / ke, dev)
+    h2d = sum(x.numel() * 2 for x in Xh)
+    d2h = sum(L["Y"].numel() * 4 for L in layers)
+    rec["e2e"] = {"value": total * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                  "api": "GroupPlan.quantize_acts + GroupPlan.linear (sbn_quantize_acts_group, "
+                         "sbn_linear_group); weights resident, X in / Y out over PCIe"}
+    rec["config"] = {"workload": "stack-decode-32x4096-t16-2of4", "layers": len(lay),
+                     "weights": weights, "packed_bytes": packed_b, "tokens": T,
+                     "pattern": "2:4",
+                     "step": "grouped act quant (S5) + grouped contraction/rescale (S6-S7) of "
+                             "all 160 pre-packed layers",
+                     "l2": "1.62 GB of packed weights per step > 126 MB L2",
+                     "parallelism": f"replicas x{world} (one stack per GPU, own inputs)"}
+    return rec, Xh, layers
+
+
+def bench_stack_prefill(args, sbn, dev, local, rank, world, peaks, timer, packed, err):
+    T = workloads.STACK_PREFILL_T
+    lay = stack_layers(rank)
+    Ks = sorted({K for _, _, _, K, _ in lay})
+    Os = sorted({O for _, _, O, _, _ in lay})
+    # Student-t(4) activations (seeded, host), one input per distinct K shared by its layers
+    X = {K: workloads.torch_bf16(workloads.student_t(T, K, config=5, tensor=30000 + K + 1000 * rank),
+                                 dev) for K in Ks}
+    Xq = {K: torch.empty((T, K), dtype=torch.int8, device=dev) for K in Ks}
+    sc = {K: torch.empty((T,), dtype=torch.float32, device=dev) for K in Ks}
+    Y = {O: torch.empty((T, O), dtype=torch.float32, device=dev) for O in Os}
+    st = timer.stream
+    steps = min(args.steps, 10)
+
+    def step(i, ev):
+        for j, ((_, _, O, K, _), w) in enumerate(zip(lay, packed)):
+            sbn.sbn_quantize_acts(X[K], Xq[K], sc[K], err, st)
+            if ev is not None and j == 0:
+                ev["linear"][0].record(st)
+            sbn.sbn_linear(Xq[K], sc[K], w.codes, w.meta, w.gamma_eff, O, K, 2, 4, Y[O], None,
+                           err, st)
+            if ev is not None and j == 0:
+                ev["linear"][1].record(st)
+
+    ms, per, clocks = timer.run(step, steps, min(args.warmup, 3), calls=("linear",))
+    weights = sum(O * K for _, _, O, K, _ in lay)
+    ops = T * weights  # 2 x kept MACs = 2 T O K / 2
+    qkv_ops = T * lay[0][2] * lay[0][3]
+    return {"value": ops * world / (ms * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": ms,
+            "steps": steps,
+            "roofline": tensor_roof(qkv_ops / (per["linear"] * 1e-3) / 1e12, peaks,
+                                    "k_gemm_sp24_pair<224> (QKV 12288x4096, 4096 tokens, per call)"),
+            "whole_step_frac_of_int8_peak": ops / (ms * 1e-3) / 1e12 / (2.0 * peaks["bf16"]),
+            "gpu_launches": 2 * len(lay) * steps, "clocks": clocks,
+            "config": {"workload": "stack-prefill-32x4096-t4096-2of4", "tokens": T,
+                       "kept_ops": ops, "step": "per layer: act quant + tensor-core contraction"}}
+
+
+# ---- single-tensor configurations (2, 3) -------------------------------------------------
+
+def step_accounting(cfg):
+    O, K, T, n, m = cfg["O"], cfg["K"], cfg["T"], cfg["n"], cfg["m"]
+    stored = K // 2 if (n, m) == (2, 4) else K
+    codes_b, meta_b = O * (stored // 4), O * (K // 8)
+    linear_w = codes_b + (meta_b if (n, m) == (2, 4) else 0)
+    pack = 2 * O * K + codes_b + meta_b
+    act = 2 * T * K + T * K + 4 * T
+    linear = linear_w + T * K + 4 * T + 4 * T * O
+    return dict(pack=pack, act=act, linear=linear, linear_weight=linear_w,
+                ops=2 * T * O * K * n // m, total=pack + act + linear)
+
+
+def bench_single(args, sbn, dev, local, rank, world, peaks, timer, cfg, err):
     O, K, T, n, m = cfg["O"], cfg["K"], cfg["T"], cfg["n"], cfg["m"]
     acct = step_accounting(cfg)
     set_bytes = 2 * O * K + 2 * T * K
-    R = max(2, -(-2 * L2_BYTES // set_bytes)) if set_bytes < 2 * L2_BYTES else 1
-    R = min(R, 64)
-
-    # R rotating input sets generated on the host (seeded, same recipe as the tests);
-    # a rank draws its own sets (tensor id offset by the rank).
+    R = min(64, max(2, -(-2 * L2_BYTES // set_bytes))) if set_bytes < 2 * L2_BYTES else 1
     sets = []
+    d = sbn.sbn_linear_ref_dims(O, K, n, m)
     for r in range(R):
         Wb = workloads.masters(O, K, seed=0, config=1, tensor=2 * (r + R * rank))
         Xb = workloads.activations(T, K, seed=0, config=1, tensor=2 * (r + R * rank) + 1)
-        W = workloads.torch_bf16(Wb, dev)
-        X = workloads.torch_bf16(Xb, dev)
-        d = sbn.sbn_linear_ref_dims(O, K, n, m)
         sets.append(dict(
-            W=W, X=X,
+            W=workloads.torch_bf16(Wb, dev), X=workloads.torch_bf16(Xb, dev),
             codes=torch.empty((O, d.codes_ld), dtype=torch.uint8, device=dev),
             meta=torch.empty((O, d.meta_ld), dtype=torch.uint8, device=dev),
             g=torch.empty(1, dtype=torch.float32, device=dev),
@@ -193,501 +398,416 @@ def run_cuda(args, cfg):
             s=torch.empty((T,), dtype=torch.float32, device=dev),
             Y=torch.empty((T, O), dtype=torch.float32, device=dev)))
     ws = sbn.new_workspace(O, K, n, m, dev)
-    err = torch.zeros(1, dtype=torch.int32, device=dev)
-
+    main = timer.stream
     side = torch.cuda.Stream(device=dev)
 
-    def step(st, ev=None):
-        # the activation quantiser does not depend on the weights: it runs on a side stream
-        # while the pack runs on the main stream; the contraction waits for both
-        main = torch.cuda.current_stream()
+    def step(i, ev):
+        # the activation quantiser does not depend on the weights: side stream, overlapped
+        # with the pack on the main stream; the contraction waits for both
+        s = sets[i % R]
         if ev is not None:
-            ev[0].record(main)
+            ev["pack"][0].record(main)
         side.wait_stream(main)
-        with torch.cuda.stream(side):
-            sbn.sbn_quantize_acts(st["X"], st["Xq"], st["s"], err, side)
-            if ev is not None:
-                ev[1].record(side)
-        sbn.sbn_quantize_mask_pack_weights(st["W"], n, m, 1e-5, st["codes"], st["meta"], st["g"],
-                                           ws, None, err, main)
         if ev is not None:
-            ev[2].record(main)
+            ev["act"][0].record(side)
+        sbn.sbn_quantize_acts(s["X"], s["Xq"], s["s"], err, side)
+        if ev is not None:
+            ev["act"][1].record(side)
+        sbn.sbn_quantize_mask_pack_weights(s["W"], n, m, 1e-5, s["codes"], s["meta"], s["g"], ws,
+                                           None, err, main)
+        if ev is not None:
+            ev["pack"][1].record(main)
         main.wait_stream(side)
         if ev is not None:
-            ev[3].record(main)
-        sbn.sbn_linear(st["Xq"], st["s"], st["codes"], st["meta"], st["g"], O, K, n, m, st["Y"],
-                       None, err, main)
+            ev["linear"][0].record(main)
+        sbn.sbn_linear(s["Xq"], s["s"], s["codes"], s["meta"], s["g"], O, K, n, m, s["Y"], None,
+                       err, main)
         if ev is not None:
-            ev[4].record(main)
+            ev["linear"][1].record(main)
 
-    kernels_per_step = 4  # pack pass 1 + pass 2, act quant, contraction
-    stream = torch.cuda.Stream(device=dev)
-    # warm-up (also loads the module and sets kernel attributes outside capture)
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            step(sets[i % R])
-    torch.cuda.synchronize()
-
-    # the timed graph: K steps and nothing else
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        for i in range(args.steps):
-            step(sets[i % R])
-    # a second graph of the same K steps with external events around every call (recorded
-    # by the replay itself, readable afterwards): the per-call durations for the roofline
-    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)]
-           for _ in range(args.steps)]
-    g_ev = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_ev, stream=stream):
-        for i in range(args.steps):
-            step(sets[i % R], evs[i])
-    wg = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(wg, stream=stream):
-        for i in range(max(args.warmup, 3)):
-            step(sets[i % R])
-    wg.replay()
-    torch.cuda.synchronize()
-
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    with ClockSampler(local) as clk:
-        with torch.cuda.stream(stream):
-            t0.record()
-            g.replay()
-            t1.record()
-        torch.cuda.synchronize()
-        # per-call durations (not part of the timed region), then keep sampling briefly if
-        # the timed region was shorter than the sampling period
-        with torch.cuda.stream(stream):
-            g_ev.replay()
-        torch.cuda.synchronize()
-        if t0.elapsed_time(t1) < 300:
-            with torch.cuda.stream(stream):
-                for _ in range(max(1, int(300 / max(t0.elapsed_time(t1), 1e-3)))):
-                    g.replay()
-            torch.cuda.synchronize()
-    barrier(world)
-    ms = max_over_ranks(t0.elapsed_time(t1), world)
-    flag = int(err.item())
-
-    per = {"pack": [], "act": [], "linear": []}
-    for e in evs:
-        per["pack"].append(e[0].elapsed_time(e[2]))
-        per["act"].append(e[0].elapsed_time(e[1]))
-        per["linear"].append(e[3].elapsed_time(e[4]))
-    avg = {k: sum(v) / len(v) for k, v in per.items()}
-
-    # e2e through the public API with host buffers (pinned), copies in the timed region
-    e2e = None
-    if True:
-        hostW = [sets[r]["W"].cpu().pin_memory() for r in range(R)]
-        hostX = [sets[r]["X"].cpu().pin_memory() for r in range(R)]
-        hostY = torch.empty((T, O), dtype=torch.float32).pin_memory()
-        Wd = torch.empty_like(sets[0]["W"])
-        Xd = torch.empty_like(sets[0]["X"])
-        ke = min(args.steps, 20)
-        with torch.cuda.stream(stream):
-            for i in range(3):
-                Wd.copy_(hostW[i % R], non_blocking=True)
-                Xd.copy_(hostX[i % R], non_blocking=True)
-                Y = sbn.forward(Xd, Wd, n, m, workspace=ws)
-                hostY.copy_(Y, non_blocking=True)
-            torch.cuda.synchronize()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record()
-            for i in range(ke):
-                Wd.copy_(hostW[i % R], non_blocking=True)
-                Xd.copy_(hostX[i % R], non_blocking=True)
-                Y = sbn.forward(Xd, Wd, n, m, workspace=ws)
-                hostY.copy_(Y, non_blocking=True)
-                torch.cuda.current_stream().synchronize()  # the step's result is on the host
-            b.record()
-        torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(a.elapsed_time(b) / ke, world)
-        e2e = {"value": acct["total"] * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
-               "h2d_bytes_per_step": 2 * O * K + 2 * T * K, "d2h_bytes_per_step": 4 * T * O,
-               "ms_per_step": e2e_ms}
-
-    peaks = load_peaks()
-    total_s = ms * 1e-3
-    value = acct["total"] * args.steps * world / total_s / 1e9
-    # dominant C-ABI call by time share
-    dom = max(avg, key=avg.get)
-    traffic = load_traffic(cfg["name"], dom)
-    tensor_bound = dom == "linear" and T > 4  # the tensor-core contraction
-    if tensor_bound:
-        # kept-MAC ops against the int8 dense peak (measured bf16 burst x 2, the nominal
-        # int8/bf16 ratio); the timed kernel runs inside a long step
-        achieved = acct["ops"] / (avg[dom] * 1e-3) / 1e12
-        peak = 2.0 * (peaks["bf16_sustained"] or peaks["bf16"])
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic,
-                "peak_source": peaks["source"] + " (MEASURED_PEAKS.json bf16_tflops_sustained"
-                               " x 2 = int8 dense; of measured)"}
+    steps = args.steps
+    ms, per, clocks = timer.run(step, steps, args.warmup, calls=("pack", "act", "linear"))
+    dom = max(per, key=per.get)
+    if dom == "linear" and T > 4:
+        roof = tensor_roof(acct["ops"] / (per["linear"] * 1e-3) / 1e12, peaks,
+                           "tensor-core contraction", load_traffic(cfg["name"], "linear"))
     else:
-        dom_bytes = {"pack": acct["pack"], "act": acct["act"], "linear": acct["linear"]}[dom]
-        achieved = dom_bytes / (avg[dom] * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm"], "traffic": traffic,
-                "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs; of measured)"}
-    roof["kernel"] = {"pack": "quant_mask_pack (k_abs_sum + k_qmp)", "act": "act_quant",
-                      "linear": "contraction"}[dom]
-    result = {
-        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8xternary->int32, fp32 out",
-        "data": "synthetic (seeded N(0,0.02) bf16 masters; N(0,1) activations, 0.5% x20 outliers)",
-        "config": {"workload": cfg["name"], "O": O, "K": K, "tokens": T, "pattern": f"{n}:{m}",
-                   "step": "pack(S1-S4) on the main stream, act quant(S5) on a side stream, then contract/rescale(S6-S7)",
-                   "l2": f"{R} rotating input sets ({R * set_bytes / 1e6:.0f} MB > 126 MB L2)",
-                   "parallelism": f"replicas x{world} (independent problems)"},
-        "kernels": {
-            "pack": {"ms": avg["pack"], "GB/s": acct["pack"] / (avg["pack"] * 1e-3) / 1e9,
-                     "launches": 2},
-            "act_quant": {"ms": avg["act"], "GB/s": acct["act"] / (avg["act"] * 1e-3) / 1e9},
-            "linear": {"ms": avg["linear"],
-                       "packed_weight_GB/s": acct["linear_weight"] / (avg["linear"] * 1e-3) / 1e9,
-                       "TOPS": acct["ops"] / (avg["linear"] * 1e-3) / 1e12},
-        },
-        "roofline": roof,
-        "gpu_launches": kernels_per_step * args.steps,
-        "err_flag": flag,
-        "e2e": e2e,
-    }
-    if rank == 0:
-        result["clocks"] = clk.summary()
-        if world == 1 and not args.no_cpu_baseline:
-            result["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_seconds)
-        print(json.dumps(result))
-    if world > 1:
-        del g, wg
-        torch.distributed.destroy_process_group()
+        b = {"pack": acct["pack"], "act": acct["act"], "linear": acct["linear"]}[dom]
+        roof = hbm_roof(b / (per[dom] * 1e-3) / 1e9, peaks,
+                        {"pack": "quant_mask_pack (k_abs_sum + k_qmp)", "act": "act_quant",
+                         "linear": "GEMV"}[dom], load_traffic(cfg["name"], dom))
+    return {"value": acct["total"] * world / (ms * 1e-3) / 1e9, "unit": "GB/s",
+            "ms_per_step": ms, "steps": steps, "roofline": roof,
+            "kernels": {"pack": {"ms": per["pack"], "GB/s": acct["pack"] / (per["pack"] * 1e-3) / 1e9},
+                        "act_quant": {"ms": per["act"],
+                                      "GB/s": acct["act"] / (per["act"] * 1e-3) / 1e9},
+                        "linear": {"ms": per["linear"],
+                                   "packed_weight_GB/s": acct["linear_weight"] / (per["linear"] * 1e-3) / 1e9,
+                                   "TOPS": acct["ops"] / (per["linear"] * 1e-3) / 1e12}},
+            "gpu_launches": 4 * steps, "clocks": clocks,
+            "config": {"workload": cfg["name"], "O": O, "K": K, "tokens": T,
+                       "pattern": f"{n}:{m}",
+                       "step": "pack (S1-S4) | act quant (S5) on a side stream, then contract "
+                               "(S6-S7)",
+                       "l2": f"{R} rotating input sets ({R * set_bytes / 1e6:.0f} MB > 126 MB L2)"}}
 
 
-def load_traffic(workload, dom):
-    """DRAM bytes per launch of the dominant call from the committed ncu summary, if any."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(p):
-        return None
-    with open(p) as f:
-        d = json.load(f)
-    return d.get(workload, {}).get(dom)
+# ---- training-step weight path (configuration 4) -----------------------------------------
+
+def bench_train(args, sbn, dev, local, rank, world, peaks, timer, err):
+    lin = []
+    for layer in range(workloads.TRAIN_LAYERS):
+        for i, (name, O, K) in enumerate(workloads.TRAIN_LAYER_SHAPES):
+            W = workloads.masters_device(O, K, device=dev, config=4,
+                                         tensor=5 * layer + i + 1000 * rank)
+            outs = {}
+            for (n, m) in ((6, 8), (2, 4)):
+                d = sbn.sbn_linear_ref_dims(O, K, n, m)
+                outs[(n, m)] = (torch.empty((O, d.codes_ld), dtype=torch.uint8, device=dev),
+                                torch.empty((O, d.meta_ld), dtype=torch.uint8, device=dev),
+                                torch.empty(1, dtype=torch.float32, device=dev))
+            lin.append((O, K, W, outs))
+    ws = sbn.new_workspace(8, 64, 2, 4, dev)
+    st = timer.stream
+
+    def step(i, ev):
+        for O, K, W, outs in lin:
+            for (n, m), (c, mt, gm) in outs.items():
+                sbn.sbn_quantize_mask_pack_weights(W, n, m, 1e-5, c, mt, gm, ws, None, err, st)
+
+    steps = min(args.steps, 10)
+    ms, _, clocks = timer.run(step, steps, min(args.warmup, 3))
+    weights = sum(O * K for O, K, _, _ in lin)
+    moved = weights * 2 * 2 + weights * 3 // 8 + weights // 4  # per pattern: read W + planes
+    gbs = moved / (ms * 1e-3) / 1e9
+    return {"value": gbs * world, "unit": "GB/s", "ms_per_step": ms, "steps": steps,
+            "roofline": hbm_roof(gbs, peaks, "quant_mask_pack, 130 tensors x (6:8, 2:4)"),
+            "gpu_launches": 2 * 2 * len(lin) * steps, "clocks": clocks,
+            "config": {"workload": "train-step-26x3200-6of8+2of4", "tensors": len(lin),
+                       "weights": weights, "bytes_per_step": moved}}
 
 
-# ---- the oracle (CPU baseline / reference arm) -------------------------------------------
+# ---- the oracle (CPU baseline legs and the reference arm) ---------------------------------
 
-def oracle_step(cfg, Wb, Xb):
+_ORACLE_PREP = {}
+
+
+def oracle_stack_decode(budget_s, steps=None):
+    """The oracle on layer 0 of the stack at 16 tokens (weights packed by the oracle outside
+    the timing, as the GPU step has them pre-packed): per layer quant_acts + contract +
+    rescale.  Extrapolated x32 to the whole stack."""
     import oracle
-    w = oracle.quantize_mask_pack(Wb, cfg["n"], cfg["m"], 1e-5)
-    Xq, s, _ = oracle.quant_acts(Xb)
-    acc = oracle.contract(Xq, w["ws"])
-    return oracle.rescale(acc, s, w["g"])
+    T = workloads.STACK_DECODE_T
+    lay = stack_layers(0)[:5]
+    if "stack_decode" not in _ORACLE_PREP:
+        packs, xs = [], []
+        for idx, name, O, K, tid in lay:
+            Wb = workloads.masters(O, K, config=5, tensor=tid)
+            packs.append(oracle.quantize_mask_pack(Wb, 2, 4, 1e-5))
+            xs.append(workloads.student_t(T, K, config=5, tensor=10000 + tid))
+        _ORACLE_PREP["stack_decode"] = (packs, xs)
+    packs, xs = _ORACLE_PREP["stack_decode"]
 
+    def one():
+        for w, xb in zip(packs, xs):
+            Xq, s, _ = oracle.quant_acts(xb)
+            oracle.rescale(oracle.contract(Xq, w["ws"]), s, w["g"])
 
-def cpu_baseline(cfg, budget_s=10.0, steps=None):
-    """Times the oracle as it stands on this host's cores on whole steps of the workload
-    (bounded: stops after `budget_s` seconds or `steps` steps)."""
-    import oracle
-    acct = step_accounting(cfg)
-    Wb = workloads.masters(cfg["O"], cfg["K"], seed=0, config=1, tensor=0)
-    Xb = workloads.activations(cfg["T"], cfg["K"], seed=0, config=1, tensor=1)
-    oracle_step(cfg, Wb, Xb)  # load / build outside the timing
+    one()
     done, t0 = 0, time.perf_counter()
     while True:
-        oracle_step(cfg, Wb, Xb)
+        one()
         done += 1
         el = time.perf_counter() - t0
         if (steps is not None and done >= steps) or (steps is None and el >= budget_s):
             break
-    return {"value": acct["total"] * done / el / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
-            "kind": "oracle", "sample": f"{done} whole steps of {cfg['name']} ({el:.1f} s)",
-            "ms_per_step": el / done * 1e3}
+    per_layer = el / done
+    per_step = per_layer * workloads.STACK_LAYERS
+    Ttok = T
+    packed_b = sum(O * K for _, _, O, K, _ in lay) // 4
+    act_b = sum(3 * Ttok * K + 4 * Ttok for _, _, _, K, _ in lay)
+    lin_b = packed_b + sum(Ttok * K + 4 * Ttok + 4 * Ttok * O for _, _, O, K, _ in lay)
+    total = (act_b + lin_b) * workloads.STACK_LAYERS
+    return {"value": total / per_step / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "ms_per_step": per_step * 1e3,
+            "sample": f"layer 0 of 32 (5 layers, 16 tokens, quant_acts + contract + rescale), "
+                      f"{done} runs in {el:.1f} s; step time extrapolated x32"}
 
 
-def run_reference(args, cfg):
-    """The oracle as the reference arm: W warm-up steps, then K timed steps on the host cores.
-    Each step is the whole forward on a bounded sample of the workload (a slice of output
-    rows, all tokens) sized so that the whole run stays within about two minutes."""
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
+def oracle_single(cfg, budget_s):
+    import oracle
+    acct = step_accounting(cfg)
+    Wb = workloads.masters(cfg["O"], cfg["K"], seed=0, config=1, tensor=0)
+    Xb = workloads.activations(cfg["T"], cfg["K"], seed=0, config=1, tensor=1)
+
+    def one():
+        w = oracle.quantize_mask_pack(Wb, cfg["n"], cfg["m"], 1e-5)
+        Xq, s, _ = oracle.quant_acts(Xb)
+        oracle.rescale(oracle.contract(Xq, w["ws"]), s, w["g"])
+
+    one()
+    done, t0 = 0, time.perf_counter()
+    while True:
+        one()
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": acct["total"] * done / el / 1e9, "unit": "GB/s",
+            "cores": oracle.num_threads(), "kind": "oracle", "ms_per_step": el / done * 1e3,
+            "sample": f"{done} whole steps of {cfg['name']} ({el:.1f} s)"}
+
+
+def oracle_train(budget_s):
+    """The oracle packs the 5 tensors of one layer in both patterns per sample, extrapolated
+    x26 to the training step."""
+    import oracle
+    Ws = [workloads.masters(O, K, config=4, tensor=i)
+          for i, (_, O, K) in enumerate(workloads.TRAIN_LAYER_SHAPES)]
+
+    def one():
+        for W in Ws:
+            for (n, m) in ((6, 8), (2, 4)):
+                oracle.quantize_mask_pack(W, n, m, 1e-5)
+
+    done, t0 = 0, time.perf_counter()
+    while True:
+        one()
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    weights = sum(O * K for _, O, K in workloads.TRAIN_LAYER_SHAPES)
+    moved = weights * 4 + weights * 3 // 8 + weights // 4
+    return {"value": moved * done / el / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "ms_per_step": el / done * 1e3 * workloads.TRAIN_LAYERS,
+            "sample": f"one layer (5 tensors x 6:8 and 2:4), {done} runs in {el:.1f} s; "
+                      "step time extrapolated x26"}
+
+
+def oracle_stack_prefill(budget_s):
+    """The oracle on 128 of the 4096 tokens of layer 0 (per layer quant_acts + contract +
+    rescale), in kept TOPS."""
+    import oracle
+    T = 128
+    lay = stack_layers(0)[:5]
+    packs, xs = [], []
+    for idx, name, O, K, tid in lay:
+        packs.append(oracle.quantize_mask_pack(workloads.masters(O, K, config=5, tensor=tid),
+                                               2, 4, 1e-5))
+        xs.append(workloads.student_t(T, K, config=5, tensor=20000 + tid))
+    done, t0 = 0, time.perf_counter()
+    while True:
+        for w, xb in zip(packs, xs):
+            Xq, s, _ = oracle.quant_acts(xb)
+            oracle.rescale(oracle.contract(Xq, w["ws"]), s, w["g"])
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    ops = T * sum(O * K for _, _, O, K, _ in lay) * done
+    return {"value": ops / el / 1e12, "unit": "TOPS", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"128 of 4096 tokens of layer 0 (5 layers), {done} runs in {el:.1f} s"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm, on the default workload's metric and unit: each step
+    is layer 0 of the stack (5 layers, 16 tokens) -- a bounded sample of the stack's decode
+    step -- timed on the host cores.  Under torchrun only rank 0 runs."""
+    world, rank, _ = dist.env_world()
     if rank != 0:
         return
     import oracle
-    O = cfg["O"]
-    Wb = workloads.masters(O, cfg["K"], seed=0, config=1, tensor=0)
-    Xb = workloads.activations(cfg["T"], cfg["K"], seed=0, config=1, tensor=1)
-    t0 = time.perf_counter()
-    oracle_step(cfg, Wb, Xb)
-    full = time.perf_counter() - t0
-    frac = min(1.0, 100.0 / max(full * (args.steps + args.warmup), 1e-9))
-    rows = max(8, int(O * frac) // 8 * 8)
-    sub = dict(cfg, O=rows)
-    Ws = np.ascontiguousarray(Wb[:rows])
     for _ in range(args.warmup):
-        oracle_step(sub, Ws, Xb)
+        oracle_stack_decode(0.0, steps=1)
     t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_step(sub, Ws, Xb)
+    rec = oracle_stack_decode(0.0, steps=args.steps)
     el = time.perf_counter() - t0
-    value = step_accounting(sub)["total"] * args.steps / el / 1e9
-    sample = f"{args.steps} steps, each {rows} of {O} output rows x all tokens of {cfg['name']}"
+    sample = (f"{args.steps} steps, each layer 0 of the 32-layer stack (5 layers, 16 tokens); "
+              "the value counts the whole stack's bytes with the step time extrapolated x32")
     print(json.dumps({
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int8xternary->int64, fp64 out", "data": "synthetic",
-        "config": {"workload": cfg["name"], "O": O, "K": cfg["K"], "tokens": cfg["T"],
-                   "pattern": f"{cfg['n']}:{cfg['m']}"},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(),
+        "impl": "reference", "metric": METRIC, "value": rec["value"], "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": rec["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8xternary->int64, fp64 out", "data": "synthetic",
+        "config": {"workload": "stack-decode-32x4096-t16-2of4", "tokens": 16, "pattern": "2:4"},
+        "cpu_baseline": {"value": rec["value"], "unit": "GB/s", "cores": oracle.num_threads(),
                          "kind": "oracle", "sample": sample},
-        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }))
+        "e2e": {"value": rec["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "wall_s": el}))
 
 
-def timed_graph(step, steps, warmup, stream, world, local):
-    """Warm-up, then `steps` steps captured in one graph and replayed between barrier +
-    synchronize; returns (max-over-ranks ms, clock summary)."""
-    with torch.cuda.stream(stream):
-        for _ in range(warmup):
-            step()
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        for _ in range(steps):
-            step()
-    g.replay()
-    torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    with ClockSampler(local) as clk:
-        with torch.cuda.stream(stream):
-            t0.record()
-            g.replay()
-            t1.record()
-        torch.cuda.synchronize()
-        if t0.elapsed_time(t1) < 300:
-            with torch.cuda.stream(stream):
-                for _ in range(max(1, int(300 / max(t0.elapsed_time(t1), 1e-3)))):
-                    g.replay()
-            torch.cuda.synchronize()
-    barrier(world)
-    return max_over_ranks(t0.elapsed_time(t1), world), clk.summary()
+# ---- main ----------------------------------------------------------------------------------
 
-
-def run_model(args, cfg):
-    """The whole-model workloads (configurations 4 and 5).  Weights are drawn on the GPU
-    from seeded generators (workloads.masters_device); activations on the host."""
+def run_cuda(args):
     import sparse_linear_layers_absmean_b200 as sbn
 
-    world, rank, local = dist_setup()
+    world, rank, local = dist.init("nccl")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     peaks = load_peaks()
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    stream = torch.cuda.Stream(device=dev)
-    extra = {}
-    if cfg["kind"] == "stack":
-        T, n, m = cfg["T"], 2, 4
-        lin = []
-        for layer in range(workloads.STACK_LAYERS):
-            for i, (name, O, K) in enumerate(workloads.STACK_LAYER_SHAPES):
-                W = workloads.masters_device(O, K, device=dev, config=4,
-                                             tensor=5 * layer + i + 1000 * rank)
-                lin.append((O, K, sbn.pack_weights(W, n, m, err_flag=err)))
-                del W
-        Ks = sorted({K for _, K, _ in lin})
-        X = {K: workloads.torch_bf16(workloads.student_t(T, K, config=4, tensor=100 + K), dev)
-             for K in Ks}
-        Xq = {K: torch.empty((T, K), dtype=torch.int8, device=dev) for K in Ks}
-        sc = {K: torch.empty((T,), dtype=torch.float32, device=dev) for K in Ks}
-        Y = {O: torch.empty((T, O), dtype=torch.float32, device=dev) for O, _, _ in lin}
-
-        def step():
-            for O, K, w in lin:
-                sbn.sbn_quantize_acts(X[K], Xq[K], sc[K], err)
-                sbn.sbn_linear(Xq[K], sc[K], w.codes, w.meta, w.gamma_eff, O, K, n, m, Y[O],
-                               None, err)
-
-        ms, clocks = timed_graph(step, args.steps, args.warmup, stream, world, local)
-        weights = sum(O * K for O, K, _ in lin)
-        packed = weights // 4  # 2:4: K/8 code bytes + K/8 metadata bytes per row
-        ops = 2 * T * weights // 2
-        act = sum(3 * T * K + 4 * T for _, K, _ in lin)
-        out_b = sum(4 * T * O for O, _, _ in lin)
-        per_step = ms * 1e-3 / args.steps
-        if T <= 16:
-            achieved = packed / per_step / 1e9
-            roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
-                    "frac": achieved / peaks["hbm"], "traffic": None,
-                    "peak_source": peaks["source"] + " (hbm_gbs; of measured)",
-                    "kernel": "whole step on packed-weight bytes (act quant + contraction)"}
-            metric_value, unit = (packed + act + out_b) * world / per_step / 1e9, "GB/s"
+    timer = Timer(dev, local)
+    result = None
+    if args.workload in ("stack", "stack-prefill"):
+        packed = build_stack(sbn, dev, rank, err)
+        head, _, _ = bench_stack_decode(args, sbn, dev, local, rank, world, peaks, timer,
+                                        packed, err)
+        if args.workload == "stack-prefill":
+            head = bench_stack_prefill(args, sbn, dev, local, rank, world, peaks, timer, packed,
+                                       err)
+            subs = {}
         else:
-            achieved = ops / per_step / 1e12
-            peak = 2.0 * (peaks["bf16_sustained"] or peaks["bf16"])
-            roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": None,
-                    "peak_source": peaks["source"] + " (2 x bf16_tflops_sustained; of measured)",
-                    "kernel": "whole step on kept ops (act quant + contraction)"}
-            metric_value, unit = ops * world / per_step / 1e12, "TOPS"
-        detail = {"linears": len(lin), "weights": weights, "packed_bytes": packed,
-                  "kept_ops": ops, "tokens": T}
+            subs = {}
+            if world == 1 and not args.no_sub:
+                subs["stack_prefill"] = bench_stack_prefill(args, sbn, dev, local, rank, world,
+                                                            peaks, timer, packed, err)
+        del packed
+        torch.cuda.empty_cache()
+        if world == 1 and not args.no_sub and args.workload == "stack":
+            subs["decode_gemv"] = bench_single(args, sbn, dev, local, rank, world, peaks, timer,
+                                               workloads.DECODE_GEMV, err)
+            subs["prefill_gemm"] = bench_single(args, sbn, dev, local, rank, world, peaks, timer,
+                                                workloads.PREFILL_GEMM, err)
+            subs["train_step"] = bench_train(args, sbn, dev, local, rank, world, peaks, timer,
+                                             err)
+    elif args.workload == "decode":
+        head, subs = bench_single(args, sbn, dev, local, rank, world, peaks, timer,
+                                  workloads.DECODE_GEMV, err), {}
+    elif args.workload == "prefill":
+        head, subs = bench_single(args, sbn, dev, local, rank, world, peaks, timer,
+                                  workloads.PREFILL_GEMM, err), {}
     else:
-        lin = []
-        for layer in range(workloads.TRAIN_LAYERS):
-            for i, (name, O, K) in enumerate(workloads.TRAIN_LAYER_SHAPES):
-                W = workloads.masters_device(O, K, device=dev, config=3,
-                                             tensor=5 * layer + i + 1000 * rank)
-                outs = {}
-                for (n, m) in ((6, 8), (2, 4)):
-                    d = sbn.sbn_linear_ref_dims(O, K, n, m)
-                    outs[(n, m)] = (torch.empty((O, d.codes_ld), dtype=torch.uint8, device=dev),
-                                    torch.empty((O, d.meta_ld), dtype=torch.uint8, device=dev),
-                                    torch.empty(1, dtype=torch.float32, device=dev))
-                lin.append((O, K, W, outs))
-        ws = sbn.new_workspace(8, 64, 2, 4, dev)
-
-        def step():
-            for O, K, W, outs in lin:
-                for (n, m), (c, mt, gm) in outs.items():
-                    sbn.sbn_quantize_mask_pack_weights(W, n, m, 1e-5, c, mt, gm, ws, None, err)
-
-        ms, clocks = timed_graph(step, args.steps, args.warmup, stream, world, local)
-        weights = sum(O * K for O, K, _, _ in lin)
-        # per pattern: read W (2 B/w) + write the planes (6:8: 0.375 B/w, 2:4: 0.25 B/w)
-        moved = weights * 2 * 2 + weights * 3 // 8 + weights // 4
-        per_step = ms * 1e-3 / args.steps
-        achieved = moved / per_step / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm"], "traffic": None,
-                "peak_source": peaks["source"] + " (hbm_gbs; of measured)",
-                "kernel": "quant_mask_pack, 130 tensors x (6:8, 2:4)"}
-        metric_value, unit = moved * world / per_step / 1e9, "GB/s"
-        detail = {"tensors": len(lin), "weights": weights, "bytes_per_step": moved,
-                  "patterns": ["6:8", "2:4"]}
-        extra["mask_stats"] = mask_stats(sbn, lin, ws, err, stream, dev, peaks)
+        head, subs = bench_train(args, sbn, dev, local, rank, world, peaks, timer, err), {}
     flag = int(err.item())
     if rank == 0:
-        print(json.dumps({
-            "metric": METRIC, "value": metric_value, "unit": unit, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "int8xternary->int32, fp32 out", "data": "synthetic (seeded; weights drawn "
-            "on the GPU N(0,0.02); Student-t(4) activations)",
-            "config": {"workload": cfg["name"], **detail,
-                       "l2": "working set of GBs > 126 MB L2"},
-            "roofline": roof, "err_flag": flag, "clocks": clocks, **extra}))
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            b = args.cpu_seconds
+            if args.workload == "stack":
+                cpu = oracle_stack_decode(b)
+                if "stack_prefill" in subs:
+                    subs["stack_prefill"]["cpu_baseline"] = oracle_stack_prefill(b / 2)
+                for key, cfg in (("decode_gemv", workloads.DECODE_GEMV),
+                                 ("prefill_gemm", workloads.PREFILL_GEMM)):
+                    if key in subs:
+                        subs[key]["cpu_baseline"] = oracle_single(cfg, b / 2)
+                if "train_step" in subs:
+                    subs["train_step"]["cpu_baseline"] = oracle_train(b / 2)
+            elif args.workload == "stack-prefill":
+                cpu = oracle_stack_prefill(b)
+            elif args.workload == "decode":
+                cpu = oracle_single(workloads.DECODE_GEMV, b)
+            elif args.workload == "prefill":
+                cpu = oracle_single(workloads.PREFILL_GEMM, b)
+            else:
+                cpu = oracle_train(b)
+        line = {
+            "metric": METRIC, "value": head["value"], "unit": head["unit"], "n_gpus": world,
+            "steps": head.get("steps", args.steps), "warmup": args.warmup,
+            "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8 x ternary -> int32, fp32 out",
+            "data": "synthetic (seeded: N(0,0.02) bf16 masters drawn on the GPU, packed once; "
+                    "Student-t(4) bf16 activations)",
+            "config": head["config"], "roofline": head["roofline"],
+            "cpu_baseline": cpu, "e2e": head.get("e2e"), "gpu_launches": head["gpu_launches"],
+            "clocks": head["clocks"], "kernels": head.get("kernels"), "err_flag": flag,
+            "bytes_per_step": head.get("bytes_per_step"), "sub": subs,
+            "peaks": {k: peaks[k] for k in ("hbm", "bf16", "bf16_sustained", "source")},
+        }
+        print(json.dumps(line))
+    dist.barrier(dev)
+    dist.shutdown()
     if flag:
         sys.exit(1)
 
 
-def mask_stats(sbn, lin, ws, err, stream, dev, peaks):
-    """The training-step mask statistics, after the timed steps: natural zeros of every
-    tensor (one read of W each) and mask flips of both patterns against the next step's
-    masters (W plus N(0, 1e-3^2) noise, packed here), timed with CUDA events around the
-    counting calls only.  Algorithmic bytes: 2 B per weight for the zero count, two meta
-    planes per flip count."""
-    zeros = torch.zeros(1, dtype=torch.int64, device=dev)
-    flips = {(6, 8): torch.zeros(1, dtype=torch.int64, device=dev),
-             (2, 4): torch.zeros(1, dtype=torch.int64, device=dev)}
-    nxt = []
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(4)
-    with torch.cuda.stream(stream):
-        for O, K, W, outs in lin:
-            W2 = (W.float() + 1e-3 * torch.randn(W.shape, generator=gen, device=dev)).bfloat16()
-            packs = {}
-            for (n, m) in outs:
-                d = sbn.sbn_linear_ref_dims(O, K, n, m)
-                c = torch.empty((O, d.codes_ld), dtype=torch.uint8, device=dev)
-                mt = torch.empty((O, d.meta_ld), dtype=torch.uint8, device=dev)
-                gm = torch.empty(1, dtype=torch.float32, device=dev)
-                sbn.sbn_quantize_mask_pack_weights(W2, n, m, 1e-5, c, mt, gm, ws, None, err)
-                packs[(n, m)] = mt
-            del W2
-            nxt.append(packs)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for (O, K, W, outs), packs in zip(lin, nxt):
-            sbn.sbn_count_zero_codes(W, outs[(6, 8)][2], zeros)
-            for (n, m), (c, mt, gm) in outs.items():
-                sbn.sbn_count_mask_flips(mt, packs[(n, m)], O, K, n, m, flips[(n, m)])
-        e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    weights = sum(O * K for O, K, _, _ in lin)
-    moved = weights * 2 + 2 * 2 * (weights // 8)  # W once; two meta planes per pattern
-    gbs = moved / (ms * 1e-3) / 1e9
-    return {"natural_zero_frac": int(zeros.item()) / weights,
-            "flip_frac_6of8": int(flips[(6, 8)].item()) / weights,
-            "flip_frac_2of4": int(flips[(2, 4)].item()) / weights,
-            "ms": ms, "GB/s": gbs, "frac_of_hbm": gbs / peaks["hbm"],
-            "kernels": "k_count_zero_codes, k_count_mask_flips (130 tensors each)",
-            "next_step": "masters + N(0, 1e-3^2) noise"}
-
-
-def run_only(args, cfg):
-    """Profiling aid: one C-ABI call of the step (pack, act or linear) on the workload's
-    first seeded input set, `warmup + steps` times on the current stream, nothing timed.
-    Used to capture a single kernel under ncu; prints one JSON line saying what ran."""
+def run_only(args):
+    """Profiling aid: one kind of C-ABI call on the workload's first inputs, `warmup + steps`
+    times on one stream, nothing timed (for single-kernel ncu captures).  Prints one JSON
+    line saying what ran."""
     import sparse_linear_layers_absmean_b200 as sbn
 
     dev = torch.device("cuda", 0)
-    O, K, T, n, m = cfg["O"], cfg["K"], cfg["T"], cfg["n"], cfg["m"]
-    W = workloads.torch_bf16(workloads.masters(O, K, seed=0, config=1, tensor=0), dev)
-    X = workloads.torch_bf16(workloads.activations(T, K, seed=0, config=1, tensor=1), dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    w = sbn.pack_weights(W, n, m, err_flag=err)
-    Xq, s = sbn.quantize_acts(X, err_flag=err)
-    Y = torch.empty((T, O), dtype=torch.float32, device=dev)
-    ws = sbn.new_workspace(O, K, n, m, dev)
     calls = args.warmup + args.steps
-    for _ in range(calls):
-        if args.only == "pack":
-            sbn.sbn_quantize_mask_pack_weights(W, n, m, 1e-5, w.codes, w.meta, w.gamma_eff, ws,
-                                               None, err)
-        elif args.only == "act":
-            sbn.sbn_quantize_acts(X, Xq, s, err)
-        else:
-            sbn.sbn_linear(Xq, s, w.codes, w.meta, w.gamma_eff, O, K, n, m, Y, None, err)
+    if args.workload == "stack":
+        packed = build_stack(sbn, dev, 0, err)
+        T = workloads.STACK_DECODE_T
+        layers = []
+        for (idx, name, O, K, tid), w in zip(stack_layers(0), packed):
+            X = workloads.torch_bf16(workloads.student_t(T, K, config=5, tensor=10000 + tid), dev)
+            layers.append(dict(X=X, Xq=torch.empty((T, K), dtype=torch.int8, device=dev),
+                               s=torch.empty((T,), dtype=torch.float32, device=dev), w=w,
+                               Y=torch.empty((T, O), dtype=torch.float32, device=dev)))
+        plan = sbn.GroupPlan(layers, device=dev)
+        plan.quantize_acts(err)
+        for _ in range(calls):
+            if args.only == "act":
+                plan.quantize_acts(err)
+            else:
+                plan.linear(err)
+    else:
+        cfg = {"decode": workloads.DECODE_GEMV, "prefill": workloads.PREFILL_GEMM}[args.workload]
+        O, K, T, n, m = cfg["O"], cfg["K"], cfg["T"], cfg["n"], cfg["m"]
+        W = workloads.torch_bf16(workloads.masters(O, K, seed=0, config=1, tensor=0), dev)
+        X = workloads.torch_bf16(workloads.activations(T, K, seed=0, config=1, tensor=1), dev)
+        w = sbn.pack_weights(W, n, m, err_flag=err)
+        Xq, s = sbn.quantize_acts(X, err_flag=err)
+        Y = torch.empty((T, O), dtype=torch.float32, device=dev)
+        ws = sbn.new_workspace(O, K, n, m, dev)
+        for _ in range(calls):
+            if args.only == "pack":
+                sbn.sbn_quantize_mask_pack_weights(W, n, m, 1e-5, w.codes, w.meta, w.gamma_eff,
+                                                   ws, None, err)
+            elif args.only == "act":
+                sbn.sbn_quantize_acts(X, Xq, s, err)
+            else:
+                sbn.sbn_linear(Xq, s, w.codes, w.meta, w.gamma_eff, O, K, n, m, Y, None, err)
     torch.cuda.synchronize()
     flag = int(err.item())
-    print(json.dumps({"only": args.only, "workload": cfg["name"], "calls": calls,
+    print(json.dumps({"only": args.only, "workload": args.workload, "calls": calls,
                       "err_flag": flag}))
     if flag:
         sys.exit(1)
 
 
+def relaunch(args):
+    """`--gpus N` outside torchrun: start N local ranks under torchrun and return its status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1",
+           f"--master-port={29500 + os.getpid() % 1000}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="stack", choices=WORKLOADS)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sub", action="store_true", help="headline only, no sub-records")
     ap.add_argument("--only", choices=["pack", "act", "linear"],
-                    help="profiling aid: run one C-ABI call of the step, untimed")
+                    help="profiling aid: one kind of C-ABI call, untimed (decode, prefill, stack)")
     args = ap.parse_args()
-    cfg = WORKLOADS[args.workload]
-    if args.only:
-        run_only(args, cfg)
-        return
-    if cfg.get("kind") in ("stack", "train"):
-        if args.warmup < 3:
-            args.warmup = 3
-        run_model(args, cfg)
-        return
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
-        run_reference(args, cfg)
+    world = int(os.environ.get("WORLD_SIZE", "0"))
+    if args.gpus > 1 and world == 0:
+        sys.exit(relaunch(args))
+    if world and world != args.gpus:
+        sys.exit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.only:
+        run_only(args)
+    elif args.impl == "reference":
+        run_reference(args)
     else:
-        run_cuda(args, cfg)
+        run_cuda(args)
 
 
 if __name__ == "__main__":

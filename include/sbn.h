@@ -123,16 +123,16 @@ SBN_API sbn_status sbn_quantize_mask_pack_weights(const void *W, int64_t out, in
  * path because those calls can synchronise the device and fragment its memory.  (The
  * pages have no counterpart: this is an interface convenience, not part of the method.)
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.  The pack's
- *     scratch (absmean partial sums and an arrival counter) is a fixed 8448-byte array in
- *     the library's own device memory; every GPU that loads the library holds it until
- *     the process exits.
+ *     scratch (the absmean partial sums) is a fixed 8448-byte array in the library's own
+ *     device memory; every GPU that loads the library holds it until the process exits.
  *   - Sizes: the same limits as sbn_quantize_mask_pack_weights (out * in < 2^31,
  *     in <= 131072); anything larger is refused with SBN_ERR_SHAPE.
- *   - The first call on a device looks up the array's device address (with that device
- *     current) and caches it; make that first call before any stream capture.
- *   - Each call clears the arrival counter on `stream` before its kernels run.  All calls
- *     in the process share the one array per device: calls that overlap on the GPU (for
- *     instance on two streams) race and give wrong results.
+ *   - Each call looks up the array's address in the current device's context.  The
+ *     first call on a device loads the library's device code there; make it before any
+ *     stream capture.
+ *   - Each call rewrites every part of the array it later reads, so nothing needs
+ *     clearing.  All calls in the process share the one array per device: calls that
+ *     overlap on the GPU (for instance on two streams) race and give wrong results.
  * Arguments and outputs are those of sbn_quantize_mask_pack_weights without `workspace`.
  */
 SBN_API sbn_status sbn_quantize_mask_pack_weights_noalloc(const void *W, int64_t out,
@@ -173,6 +173,109 @@ SBN_API sbn_status sbn_linear(const int8_t *Xq, const float *absmax, const uint8
                       const uint8_t *meta, const float *gamma_eff, int64_t tokens,
                       int64_t out, int64_t in, int n, int m, void *Y, int y_is_bf16,
                       int32_t *acc_dbg, int32_t *err_flag, void *stream);
+
+/*
+ * Tensor-core operand (2:4): the packed planes expanded once into the form the sparse
+ * tensor cores read, for contractions with many tokens (prefill).  The codes of each row
+ * become int8 values t in {-1, 0, 1} (0.5 byte per weight) so that the contraction only
+ * stages tiles with TMA and issues MMAs; the expansion costs one pass over the planes and
+ * is done when the weights change (after sbn_quantize_mask_pack_weights), not per call.
+ *
+ * Layout (opaque to callers; described for completeness): with O_pad = out rounded up to
+ * 256 and K_pad = in rounded up to 128, an int8 [O_pad][K_pad / 2] plane of the kept values
+ * in K order (zero in the padding), then a uint8 [O_pad][K_pad / 8] copy of the metadata
+ * plane (the index pair (0, 1) in the padding).
+ */
+
+/* Host only: *bytes = size of the operand of an (out, in) layer.  SBN_ERR_PATTERN unless
+ * n:m is 2:4; the shape rules of sbn_linear_ref_dims. */
+SBN_API sbn_status sbn_operand_bytes(int64_t out, int64_t in, int n, int m, int64_t *bytes);
+
+/* Writes the operand (device memory of sbn_operand_bytes, 16-byte aligned) from the codes
+ * and meta planes of sbn_quantize_mask_pack_weights (2:4).  One launch on `stream`. */
+SBN_API sbn_status sbn_expand_operand(const uint8_t *codes, const uint8_t *meta, int64_t out,
+                                      int64_t in, int n, int m, void *operand, void *stream);
+
+/* Steps 6-7 from the operand: y[t, o] = (sum_k Xq[t,k] * Ws[o,k]) * c_t, exactly the result of
+ * sbn_linear (every bit), with the other arguments as there.  Made for many tokens (tiles of
+ * 224 tokens on CTA pairs); any tokens >= 0 is accepted. */
+SBN_API sbn_status sbn_linear_operand(const int8_t *Xq, const float *absmax, const void *operand,
+                                      const float *gamma_eff, int64_t tokens, int64_t out,
+                                      int64_t in, int n, int m, void *Y, int y_is_bf16,
+                                      int32_t *acc_dbg, int32_t *err_flag, void *stream);
+
+/*
+ * Grouped calls: steps 5-7 for many independent 2:4 layers of at most 32 tokens each (the
+ * decode phase of a whole decoder stack) in one launch per step, instead of one launch
+ * per layer.  Each layer is described by one sbn_group_linear; the arithmetic and every
+ * output bit are those of sbn_quantize_acts and sbn_linear for that layer alone.
+ *
+ * Use: sbn_group_plan_sizes -> allocate a HOST plan buffer (128-byte aligned) and a device
+ * buffer of the same size, plus the device workspace -> sbn_group_plan fills the host plan
+ * -> copy it to the device buffer -> then, as often as wanted (for instance every decode
+ * step, with new activations in the same X buffers):
+ * sbn_quantize_acts_group and sbn_linear_group on a stream.  The plan records the device
+ * pointers of every layer, so the buffers must stay allocated and in place while it is in
+ * use; rebuild it when a pointer or a shape changes.
+ */
+typedef struct sbn_group_linear {
+  const void *X;             /* bf16 [tokens, in] input of the grouped quantiser; may be
+                                NULL if only sbn_linear_group is called (Xq given) */
+  int8_t *Xq;                /* int8 [tokens, in] quantised activations */
+  float *absmax;             /* fp32 [tokens] per-token scales s */
+  const uint8_t *codes;      /* packed planes from sbn_quantize_mask_pack_weights (2:4) */
+  const uint8_t *meta;
+  const float *gamma_eff;    /* one fp32 on the device */
+  void *Y;                   /* fp32 or bf16 [tokens, out], written */
+  int32_t *acc_dbg;          /* optional int32 [tokens, out] exact sums (NULL to skip) */
+  int64_t tokens;            /* 0..32; a layer with 0 tokens is skipped */
+  int64_t out, in;           /* shape rules of sbn_linear */
+  int32_t n, m;              /* must be 2 and 4 */
+  int32_t y_is_bf16;
+  int32_t reserved;          /* set to 0 */
+} sbn_group_linear;
+
+/*
+ * Host only.  Validates the layers (SBN_ERR_PATTERN unless every n:m is 2:4; SBN_ERR_SHAPE
+ * for tokens outside 0..32 or a bad shape; SBN_ERR_NULL / SBN_ERR_ALIGN for the pointers
+ * of layers with tokens > 0, device pointers 16-byte aligned, absmax and gamma_eff 4-byte)
+ * and returns the plan size and the device workspace size (0 when the schedule splits no
+ * row tile over several work units).
+ */
+SBN_API sbn_status sbn_group_plan_sizes(const sbn_group_linear *lins, int32_t count,
+                                        int64_t *plan_bytes, int64_t *workspace_bytes);
+
+/*
+ * Host only (queries the current device's SM count; no allocation, no synchronisation).
+ * Writes the plan into the HOST buffer `plan` (128-byte aligned, plan_bytes from
+ * sbn_group_plan_sizes): the TMA descriptors of every layer, the work units of the
+ * contraction (128 weight rows x a range of K, spread over one CTA per SM) and the rows
+ * of the activation quantiser.
+ */
+SBN_API sbn_status sbn_group_plan(const sbn_group_linear *lins, int32_t count, void *plan,
+                                  int64_t plan_bytes);
+
+/*
+ * Step 5 for every layer of the plan (s and Xq of each layer's X), one launch.
+ *   plan      the host plan; plan_dev the same bytes in device memory (128-byte aligned).
+ *   err_flag  optional: SBN_FLAG_X_NONFINITE.
+ * SBN_ERR_NULL if a layer of the plan has no X.
+ */
+SBN_API sbn_status sbn_quantize_acts_group(const void *plan, const void *plan_dev,
+                                           int32_t *err_flag, void *stream);
+
+/*
+ * Steps 6-7 for every layer of the plan, one launch: Y = (Xq . Ws^T) * c_t exactly as
+ * sbn_linear computes it.
+ *   workspace  device memory of workspace_bytes (NULL allowed when that is 0), ZEROED by
+ *              the caller before its first use; every call leaves it zeroed again, so it
+ *              needs no clearing between calls.  After a call that raised
+ *              SBN_FLAG_TIMEOUT it must be zeroed again.  Calls that share a workspace
+ *              must not overlap on the GPU.
+ *   err_flag   optional: SBN_FLAG_TIMEOUT if the tensor-core pipeline stalled.
+ */
+SBN_API sbn_status sbn_linear_group(const void *plan, const void *plan_dev, void *workspace,
+                                    int32_t *err_flag, void *stream);
 
 /*
  * Mask statistics: by-products of steps 2-3 that follow how the masks evolve over training

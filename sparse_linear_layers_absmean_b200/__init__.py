@@ -9,6 +9,7 @@ torch and call them.
 There is no CPU fallback: if libsbn.so cannot be loaded, or a tensor is not on a CUDA
 device, the call raises.
 """
+import contextlib
 import ctypes
 import os
 from typing import NamedTuple, Optional
@@ -27,7 +28,10 @@ FLAG_X_NONFINITE = 4
 FLAG_TIMEOUT = 8
 
 EXPORTED = ("sbn_linear_ref_dims", "sbn_quantize_mask_pack_weights", "sbn_quantize_acts",
-            "sbn_linear", "sbn_status_string", "sbn_quantize_mask_pack_weights_noalloc")
+            "sbn_linear", "sbn_status_string", "sbn_quantize_mask_pack_weights_noalloc",
+            "sbn_count_zero_codes", "sbn_count_mask_flips", "sbn_group_plan_sizes",
+            "sbn_group_plan", "sbn_quantize_acts_group", "sbn_linear_group",
+            "sbn_operand_bytes", "sbn_expand_operand", "sbn_linear_operand")
 
 
 class SbnError(RuntimeError):
@@ -41,6 +45,17 @@ class SbnDims(ctypes.Structure):
                 ("codes_row_bytes", ctypes.c_int64), ("meta_row_bytes", ctypes.c_int64),
                 ("codes_bytes", ctypes.c_int64), ("meta_bytes", ctypes.c_int64),
                 ("pack_workspace_bytes", ctypes.c_int64)]
+
+
+class SbnGroupLinear(ctypes.Structure):
+    """One layer of a grouped call (sbn_group_linear in sbn.h)."""
+    _fields_ = [("X", ctypes.c_void_p), ("Xq", ctypes.c_void_p), ("absmax", ctypes.c_void_p),
+                ("codes", ctypes.c_void_p), ("meta", ctypes.c_void_p),
+                ("gamma_eff", ctypes.c_void_p), ("Y", ctypes.c_void_p),
+                ("acc_dbg", ctypes.c_void_p), ("tokens", ctypes.c_int64),
+                ("out", ctypes.c_int64), ("in_", ctypes.c_int64), ("n", ctypes.c_int32),
+                ("m", ctypes.c_int32), ("y_is_bf16", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 _LIB = None
@@ -71,6 +86,20 @@ def lib():
         L.sbn_count_zero_codes.restype = i32
         L.sbn_count_mask_flips.argtypes = [p, p, i64, i64, i32, i32, p, p]
         L.sbn_count_mask_flips.restype = i32
+        L.sbn_group_plan_sizes.argtypes = [p, i32, p, p]
+        L.sbn_group_plan_sizes.restype = i32
+        L.sbn_group_plan.argtypes = [p, i32, p, i64]
+        L.sbn_group_plan.restype = i32
+        L.sbn_quantize_acts_group.argtypes = [p, p, p, p]
+        L.sbn_quantize_acts_group.restype = i32
+        L.sbn_linear_group.argtypes = [p, p, p, p, p]
+        L.sbn_linear_group.restype = i32
+        L.sbn_operand_bytes.argtypes = [i64, i64, i32, i32, p]
+        L.sbn_operand_bytes.restype = i32
+        L.sbn_expand_operand.argtypes = [p, p, i64, i64, i32, i32, p, p]
+        L.sbn_expand_operand.restype = i32
+        L.sbn_linear_operand.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, p, i32, p, p, p]
+        L.sbn_linear_operand.restype = i32
         L.sbn_status_string.argtypes = [i32]
         L.sbn_status_string.restype = ctypes.c_char_p
         _LIB = L
@@ -169,6 +198,15 @@ def sbn_count_mask_flips(meta_a, meta_b, out, in_, n, m, count, stream=None):
                                       _stream(stream)), "sbn_count_mask_flips")
 
 
+def _alloc_stream(stream):
+    """Context in which output tensors are allocated: the stream the kernel will run on,
+    so that the caching allocator ties the memory to that stream (a tensor allocated on
+    another stream could be handed out again while the kernel still writes it)."""
+    if stream is None or not isinstance(stream, torch.cuda.Stream):
+        return contextlib.nullcontext()
+    return torch.cuda.stream(stream)
+
+
 def new_workspace(out: int, in_: int, n: int, m: int, device="cuda") -> torch.Tensor:
     """Pack workspace (reusable by later calls on the same stream)."""
     d = sbn_linear_ref_dims(out, in_, n, m)
@@ -180,11 +218,12 @@ def pack_weights(W: torch.Tensor, n: int, m: int, eps: float = 1e-5,
                  err_flag: Optional[torch.Tensor] = None, stream=None) -> PackedWeights:
     out, in_ = W.shape
     d = sbn_linear_ref_dims(out, in_, n, m)
-    codes = torch.empty((out, d.codes_ld), dtype=torch.uint8, device=W.device)
-    meta = torch.empty((out, d.meta_ld), dtype=torch.uint8, device=W.device)
-    gamma = torch.empty(1, dtype=torch.float32, device=W.device)
-    if workspace is None:
-        workspace = new_workspace(out, in_, n, m, W.device)
+    with _alloc_stream(stream):
+        codes = torch.empty((out, d.codes_ld), dtype=torch.uint8, device=W.device)
+        meta = torch.empty((out, d.meta_ld), dtype=torch.uint8, device=W.device)
+        gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+        if workspace is None:
+            workspace = new_workspace(out, in_, n, m, W.device)
     sbn_quantize_mask_pack_weights(W, n, m, eps, codes, meta, gamma, workspace, dense_dbg,
                                    err_flag, stream)
     return PackedWeights(codes, meta, gamma, out, in_, n, m)
@@ -192,15 +231,17 @@ def pack_weights(W: torch.Tensor, n: int, m: int, eps: float = 1e-5,
 
 def quantize_acts(X: torch.Tensor, err_flag=None, stream=None):
     tokens, in_ = X.shape
-    Xq = torch.empty((tokens, in_), dtype=torch.int8, device=X.device)
-    s = torch.empty((tokens,), dtype=torch.float32, device=X.device)
+    with _alloc_stream(stream):
+        Xq = torch.empty((tokens, in_), dtype=torch.int8, device=X.device)
+        s = torch.empty((tokens,), dtype=torch.float32, device=X.device)
     sbn_quantize_acts(X, Xq, s, err_flag, stream)
     return Xq, s
 
 
 def linear(Xq: torch.Tensor, s: torch.Tensor, w: PackedWeights, out_dtype=torch.float32,
            acc_dbg=None, err_flag=None, stream=None) -> torch.Tensor:
-    Y = torch.empty((Xq.shape[0], w.out), dtype=out_dtype, device=Xq.device)
+    with _alloc_stream(stream):
+        Y = torch.empty((Xq.shape[0], w.out), dtype=out_dtype, device=Xq.device)
     sbn_linear(Xq, s, w.codes, w.meta, w.gamma_eff, w.out, w.in_, w.n, w.m, Y, acc_dbg, err_flag,
                stream)
     return Y
@@ -253,3 +294,114 @@ def forward(X: torch.Tensor, W: torch.Tensor, n: int, m: int, eps: float = 1e-5,
     Xq.record_stream(main)
     s.record_stream(main)
     return linear(Xq, s, w, out_dtype, stream=main)
+
+
+# ---- grouped calls ---------------------------------------------------------------------------
+
+def sbn_group_plan_sizes(lins):
+    """(plan_bytes, workspace_bytes) for a ctypes array of SbnGroupLinear."""
+    pb, wb = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().sbn_group_plan_sizes(ctypes.cast(lins, ctypes.c_void_p), len(lins),
+                                      ctypes.byref(pb), ctypes.byref(wb)), "sbn_group_plan_sizes")
+    return pb.value, wb.value
+
+
+def sbn_group_plan(lins, plan_host):
+    """Fill plan_host (a 128-byte aligned uint8 CPU tensor) with the plan of `lins`."""
+    _check(lib().sbn_group_plan(ctypes.cast(lins, ctypes.c_void_p), len(lins),
+                                ctypes.c_void_p(plan_host.data_ptr()), plan_host.numel()),
+           "sbn_group_plan")
+
+
+def sbn_quantize_acts_group(plan_host, plan_dev, err_flag=None, stream=None):
+    _check(lib().sbn_quantize_acts_group(ctypes.c_void_p(plan_host.data_ptr()), _ptr(plan_dev),
+                                         _ptr(err_flag), _stream(stream)), "sbn_quantize_acts_group")
+
+
+def sbn_linear_group(plan_host, plan_dev, workspace, err_flag=None, stream=None):
+    _check(lib().sbn_linear_group(ctypes.c_void_p(plan_host.data_ptr()), _ptr(plan_dev),
+                                  _ptr(workspace), _ptr(err_flag), _stream(stream)),
+           "sbn_linear_group")
+
+
+class GroupPlan:
+    """A grouped call over many 2:4 layers of at most 32 tokens each: the plan (host and
+    device copies) and the zeroed workspace.  `layers` is a list of dicts with the torch
+    tensors X (bf16 [T, K], may be None), Xq (int8 [T, K]), s (fp32 [T]), w (PackedWeights),
+    Y (fp32 or bf16 [T, O]) and optionally acc_dbg (int32 [T, O]).  The tensors must stay
+    alive and in place while the plan is used."""
+
+    def __init__(self, layers, device=None):
+        self.layers = layers
+        arr = (SbnGroupLinear * len(layers))()
+        for i, L in enumerate(layers):
+            w = L["w"]
+            Y = L["Y"]
+            arr[i] = SbnGroupLinear(
+                X=_ptr(L.get("X")), Xq=_ptr(L["Xq"]), absmax=_ptr(L["s"]), codes=_ptr(w.codes),
+                meta=_ptr(w.meta), gamma_eff=_ptr(w.gamma_eff), Y=_ptr(Y),
+                acc_dbg=_ptr(L.get("acc_dbg")), tokens=L["Xq"].shape[0], out=w.out, in_=w.in_,
+                n=w.n, m=w.m, y_is_bf16=1 if Y.dtype == torch.bfloat16 else 0, reserved=0)
+        self._arr = arr
+        pb, wb = sbn_group_plan_sizes(arr)
+        # 128-byte aligned host buffer
+        raw = torch.empty(pb + 128, dtype=torch.uint8)
+        off = (-raw.data_ptr()) % 128
+        self.plan_host = raw[off:off + pb]
+        self._raw = raw
+        sbn_group_plan(arr, self.plan_host)
+        device = device if device is not None else layers[0]["Xq"].device
+        self.plan_dev = self.plan_host.to(device)
+        self.workspace = torch.zeros(max(wb, 256), dtype=torch.uint8, device=device)
+        self.workspace_bytes = wb
+        hdr = self.plan_host[:48].numpy().view("int32")
+        self.nunits, self.ncta, self.bn, self.nrows, self.split = (int(hdr[3]), int(hdr[4]),
+                                                                   int(hdr[5]), int(hdr[6]),
+                                                                   int(hdr[9]))
+
+    def quantize_acts(self, err_flag=None, stream=None):
+        sbn_quantize_acts_group(self.plan_host, self.plan_dev, err_flag, stream)
+
+    def linear(self, err_flag=None, stream=None):
+        sbn_linear_group(self.plan_host, self.plan_dev, self.workspace, err_flag, stream)
+
+
+# ---- tensor-core operand (2:4, many tokens) ----------------------------------------------
+
+def sbn_operand_bytes(out, in_, n, m):
+    b = ctypes.c_int64()
+    _check(lib().sbn_operand_bytes(out, in_, n, m, ctypes.byref(b)), "sbn_operand_bytes")
+    return b.value
+
+
+def sbn_expand_operand(codes, meta, out, in_, n, m, operand, stream=None):
+    _check(lib().sbn_expand_operand(_ptr(codes), _ptr(meta), out, in_, n, m, _ptr(operand),
+                                    _stream(stream)), "sbn_expand_operand")
+
+
+def sbn_linear_operand(Xq, absmax, operand, gamma_eff, out, in_, n, m, Y, acc_dbg=None,
+                       err_flag=None, stream=None):
+    if Y.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("Y must be float32 or bfloat16")
+    _check(lib().sbn_linear_operand(_ptr(Xq), _ptr(absmax), _ptr(operand), _ptr(gamma_eff),
+                                    Xq.shape[0], out, in_, n, m, _ptr(Y),
+                                    1 if Y.dtype == torch.bfloat16 else 0, _ptr(acc_dbg),
+                                    _ptr(err_flag), _stream(stream)), "sbn_linear_operand")
+
+
+def expand_operand(w: PackedWeights, stream=None) -> torch.Tensor:
+    """The tensor-core operand of a 2:4 pack (uint8 device tensor)."""
+    with _alloc_stream(stream):
+        op = torch.empty(sbn_operand_bytes(w.out, w.in_, w.n, w.m), dtype=torch.uint8,
+                         device=w.codes.device)
+    sbn_expand_operand(w.codes, w.meta, w.out, w.in_, w.n, w.m, op, stream)
+    return op
+
+
+def linear_operand(Xq, s, w: PackedWeights, operand, out_dtype=torch.float32, acc_dbg=None,
+                   err_flag=None, stream=None) -> torch.Tensor:
+    with _alloc_stream(stream):
+        Y = torch.empty((Xq.shape[0], w.out), dtype=out_dtype, device=Xq.device)
+    sbn_linear_operand(Xq, s, operand, w.gamma_eff, w.out, w.in_, w.n, w.m, Y, acc_dbg, err_flag,
+                       stream)
+    return Y

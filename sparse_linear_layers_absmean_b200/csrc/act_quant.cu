@@ -8,6 +8,7 @@
 // launched as a programmatic dependent of the previous kernel on the stream and waits for
 // it before reading X.
 #include "common.cuh"
+#include "group.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -125,6 +126,57 @@ __global__ void __launch_bounds__(kAqThreads)
     const int64_t i = lane + 32 * r;
     if (i < nv) qrow[i] = quant_vec8(v[r], s);
   }
+}
+
+// Grouped form: one CTA per (layer, token) row of a group plan.  R > 0 keeps the row in
+// registers (rows of up to 8 * 256 * R inputs); R == 0 reads it twice.
+template <int R>
+__global__ void __launch_bounds__(kAqThreads)
+    k_act_quant_group(const uint8_t *__restrict__ plan, int32_t *err_flag) {
+  ptx::grid_dep_launch();
+  ptx::grid_dep_wait();
+  const GroupHeader &hd = *reinterpret_cast<const GroupHeader *>(plan);
+  const GroupRow rw = reinterpret_cast<const GroupRow *>(plan + hd.off_rows)[blockIdx.x];
+  const GroupProb &p = reinterpret_cast<const GroupProb *>(plan + hd.off_probs)[rw.prob];
+  const int64_t nv = p.K / 8;
+  const uint4 *row = reinterpret_cast<const uint4 *>(p.X) + (int64_t)rw.token * nv;
+  uint2 *qrow = reinterpret_cast<uint2 *>(p.Xq + (int64_t)rw.token * p.K);
+  if constexpr (R > 0) {
+    uint4 v[R];
+    uint32_t mx = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t i = threadIdx.x + (int64_t)r * kAqThreads;
+      v[r] = i < nv ? __ldg(row + i) : make_uint4(0u, 0u, 0u, 0u);
+      mx = vec8_absmax_bits(v[r], mx);
+    }
+    const float s = block_scale(mx, err_flag);
+    if (threadIdx.x == 0) p.absmax[rw.token] = s;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t i = threadIdx.x + (int64_t)r * kAqThreads;
+      if (i < nv) qrow[i] = quant_vec8(v[r], s);
+    }
+  } else {
+    uint32_t mx = 0;
+    for (int64_t i = threadIdx.x; i < nv; i += kAqThreads) mx = vec8_absmax_bits(__ldg(row + i), mx);
+    const float s = block_scale(mx, err_flag);
+    if (threadIdx.x == 0) p.absmax[rw.token] = s;
+    for (int64_t i = threadIdx.x; i < nv; i += kAqThreads) qrow[i] = quant_vec8(__ldg(row + i), s);
+  }
+}
+
+sbn_status launch_act_quant_group(const void *plan_host, const void *plan_dev, int32_t *err_flag,
+                                  cudaStream_t st) {
+  const GroupHeader *hd = static_cast<const GroupHeader *>(plan_host);
+  if (hd->nrows == 0) return SBN_OK;
+  const uint8_t *P = static_cast<const uint8_t *>(plan_dev);
+  const dim3 grid((unsigned)hd->nrows), block(kAqThreads);
+  if (hd->max_nv <= 2 * kAqThreads)
+    return launch_pdl(k_act_quant_group<2>, grid, block, 0, st, P, err_flag);
+  if (hd->max_nv <= 8 * kAqThreads)
+    return launch_pdl(k_act_quant_group<8>, grid, block, 0, st, P, err_flag);
+  return launch_pdl(k_act_quant_group<0>, grid, block, 0, st, P, err_flag);
 }
 
 sbn_status launch_act_quant(const void *X, int64_t tokens, int64_t in, int8_t *Xq,

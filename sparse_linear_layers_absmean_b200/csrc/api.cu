@@ -2,7 +2,10 @@
 // Nothing here allocates device memory or synchronises.
 #include <cmath>
 
+#include <cstring>
+
 #include "common.cuh"
+#include "group.cuh"
 #include "kernels.cuh"
 
 namespace {
@@ -33,6 +36,36 @@ void fill_dims(int64_t out, int64_t in, int n, int m, sbn_dims *d) {
   d->codes_bytes = out * d->codes_ld;
   d->meta_bytes = out * d->meta_ld;
   d->pack_workspace_bytes = (int64_t)((sizeof(sbn::PackWorkspace) + 255) / 256 * 256);
+}
+
+sbn_status check_group(const sbn_group_linear *lins, int32_t count) {
+  if (count < 0 || count > (1 << 20)) return SBN_ERR_SHAPE;
+  if (count > 0 && !lins) return SBN_ERR_NULL;
+  for (int32_t p = 0; p < count; ++p) {
+    const sbn_group_linear &l = lins[p];
+    if (l.n != 2 || l.m != 4) return SBN_ERR_PATTERN;
+    sbn_dims d;
+    sbn_status st = sbn_linear_ref_dims(l.out, l.in, l.n, l.m, &d);
+    if (st != SBN_OK) return st;
+    if (l.tokens < 0 || l.tokens > sbn::kGroupMaxTokens) return SBN_ERR_SHAPE;
+    if (l.tokens == 0) continue;
+    if (!l.Xq || !l.absmax || !l.codes || !l.meta || !l.gamma_eff || !l.Y) return SBN_ERR_NULL;
+    if (!aligned16(l.Xq) || !aligned16(l.codes) || !aligned16(l.meta) || !aligned16(l.Y) ||
+        (l.X && !aligned16(l.X)) || (l.acc_dbg && !aligned16(l.acc_dbg)) ||
+        (reinterpret_cast<uintptr_t>(l.absmax) & 3u) ||
+        (reinterpret_cast<uintptr_t>(l.gamma_eff) & 3u))
+      return SBN_ERR_ALIGN;
+  }
+  return SBN_OK;
+}
+
+sbn_status check_plan(const void *plan, const void *plan_dev) {
+  if (!plan || !plan_dev) return SBN_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(plan) & 127u) || (reinterpret_cast<uintptr_t>(plan_dev) & 127u))
+    return SBN_ERR_ALIGN;
+  const sbn::GroupHeader *hd = static_cast<const sbn::GroupHeader *>(plan);
+  if (hd->magic != sbn::kGroupMagic || hd->version != sbn::kGroupVersion) return SBN_ERR_ARG;
+  return SBN_OK;
 }
 
 }  // namespace
@@ -116,6 +149,85 @@ sbn_status sbn_linear(const int8_t *Xq, const float *absmax, const uint8_t *code
                             d.meta_ld, Y, y_is_bf16, acc_dbg, s);
   return sbn::launch_gemm_tc(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, n, m,
                              d.codes_ld, d.meta_ld, Y, y_is_bf16, acc_dbg, err_flag, s);
+}
+
+sbn_status sbn_operand_bytes(int64_t out, int64_t in, int n, int m, int64_t *bytes) {
+  if (!bytes) return SBN_ERR_NULL;
+  sbn_dims d;
+  sbn_status st = sbn_linear_ref_dims(out, in, n, m, &d);
+  if (st != SBN_OK) return st;
+  if (n != 2 || m != 4) return SBN_ERR_PATTERN;
+  *bytes = sbn::operand_bytes(out, in);
+  return SBN_OK;
+}
+
+sbn_status sbn_expand_operand(const uint8_t *codes, const uint8_t *meta, int64_t out, int64_t in,
+                              int n, int m, void *operand, void *stream) {
+  int64_t bytes = 0;
+  sbn_status st = sbn_operand_bytes(out, in, n, m, &bytes);
+  if (st != SBN_OK) return st;
+  if (!codes || !meta || !operand) return SBN_ERR_NULL;
+  if (!aligned16(codes) || !aligned16(meta) || !aligned16(operand)) return SBN_ERR_ALIGN;
+  sbn_dims d;
+  sbn_linear_ref_dims(out, in, n, m, &d);
+  return sbn::launch_expand_operand(codes, meta, out, in, d.codes_ld, d.meta_ld, operand,
+                                    static_cast<cudaStream_t>(stream));
+}
+
+sbn_status sbn_linear_operand(const int8_t *Xq, const float *absmax, const void *operand,
+                              const float *gamma_eff, int64_t tokens, int64_t out, int64_t in,
+                              int n, int m, void *Y, int y_is_bf16, int32_t *acc_dbg,
+                              int32_t *err_flag, void *stream) {
+  int64_t bytes = 0;
+  sbn_status st = sbn_operand_bytes(out, in, n, m, &bytes);
+  if (st != SBN_OK) return st;
+  if (tokens < 0 || tokens > (1ll << 31) - 1) return SBN_ERR_SHAPE;
+  if (tokens == 0) return SBN_OK;
+  if (!Xq || !absmax || !operand || !gamma_eff || !Y) return SBN_ERR_NULL;
+  if (!aligned16(Xq) || !aligned16(operand) || !aligned16(Y) ||
+      (acc_dbg && !aligned16(acc_dbg)) || (reinterpret_cast<uintptr_t>(absmax) & 3u) ||
+      (reinterpret_cast<uintptr_t>(gamma_eff) & 3u) || (reinterpret_cast<uintptr_t>(err_flag) & 3u))
+    return SBN_ERR_ALIGN;
+  return sbn::launch_gemm_operand(Xq, absmax, operand, gamma_eff, tokens, out, in, Y, y_is_bf16,
+                                  acc_dbg, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+sbn_status sbn_group_plan_sizes(const sbn_group_linear *lins, int32_t count, int64_t *plan_bytes,
+                                int64_t *workspace_bytes) {
+  if (!plan_bytes || !workspace_bytes) return SBN_ERR_NULL;
+  sbn_status st = check_group(lins, count);
+  if (st != SBN_OK) return st;
+  return sbn::group_plan_sizes(lins, count, plan_bytes, workspace_bytes);
+}
+
+sbn_status sbn_group_plan(const sbn_group_linear *lins, int32_t count, void *plan,
+                          int64_t plan_bytes) {
+  if (!plan) return SBN_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(plan) & 127u) return SBN_ERR_ALIGN;
+  sbn_status st = check_group(lins, count);
+  if (st != SBN_OK) return st;
+  return sbn::group_plan(lins, count, plan, plan_bytes);
+}
+
+sbn_status sbn_quantize_acts_group(const void *plan, const void *plan_dev, int32_t *err_flag,
+                                   void *stream) {
+  sbn_status st = check_plan(plan, plan_dev);
+  if (st != SBN_OK) return st;
+  if (reinterpret_cast<uintptr_t>(err_flag) & 3u) return SBN_ERR_ALIGN;
+  if (!static_cast<const sbn::GroupHeader *>(plan)->has_x) return SBN_ERR_NULL;
+  return sbn::launch_act_quant_group(plan, plan_dev, err_flag, static_cast<cudaStream_t>(stream));
+}
+
+sbn_status sbn_linear_group(const void *plan, const void *plan_dev, void *workspace,
+                            int32_t *err_flag, void *stream) {
+  sbn_status st = check_plan(plan, plan_dev);
+  if (st != SBN_OK) return st;
+  if (reinterpret_cast<uintptr_t>(err_flag) & 3u) return SBN_ERR_ALIGN;
+  const sbn::GroupHeader *hd = static_cast<const sbn::GroupHeader *>(plan);
+  if (hd->ws_bytes > 0 && !workspace) return SBN_ERR_NULL;
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SBN_ERR_ALIGN;
+  return sbn::launch_linear_group(plan, plan_dev, workspace, err_flag,
+                                  static_cast<cudaStream_t>(stream));
 }
 
 sbn_status sbn_count_zero_codes(const void *W, const float *gamma_eff, int64_t out, int64_t in,

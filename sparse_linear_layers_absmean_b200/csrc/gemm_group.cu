@@ -1,0 +1,679 @@
+// Grouped small-batch contraction: Y_p = (Xq_p . Ws_p^T) * c_t for many independent 2:4
+// Sparse-BitLinear layers p of at most 32 tokens each, in ONE persistent launch on the
+// sparse tensor cores (tcgen05.mma.sp kind::i8, int32 accumulators in TMEM).
+//
+// At a few tokens per layer the contraction streams the packed weights (0.25 bytes per
+// weight) from HBM and does little arithmetic per byte, so what matters is that every SM
+// keeps enough weight bytes in flight and that no launch, pipeline fill or drain repeats
+// per layer.  The host plan (sbn_group_plan) cuts every layer into work units of 128 weight
+// rows x a range of 128-deep K blocks and gives each CTA (one per SM) a contiguous run of
+// units with about the same number of K blocks; the CTA walks its run as one pipeline in
+// super-blocks of four 128-deep K blocks (every hand-off between the roles has a fixed cost,
+// so each one moves four blocks):
+//   warp 4     TMA producer, ring 1 (the HBM stream, 4-6 slots): per super-block the packed
+//              codes and the metadata of the unit's 128 rows as two boxes of 64 bytes x 128
+//              rows (64-byte swizzle), and the four activation tiles (bn tokens x 128 inputs,
+//              128-byte swizzle; L2 hits, all row tiles of a layer share them).
+//   warps 0-3  expanders, ring 2 (2 slots): thread r turns row r's kept codes into 64 int8
+//              lanes of 64 * t per block (the compressed A tile, 64-byte swizzle) and copies
+//              the metadata into the 16-byte-row layout tcgen05.cp reads (groups outside the
+//              matrix get the valid index pair (0, 1)); one proxy fence and one arrival per
+//              super-block.
+//   warp 5     TMEM allocation and the MMA thread: per block the metadata goes to TMEM
+//              (tcgen05.cp) and two sparse MMAs (M 128, N bn, logical K 64 each) accumulate
+//              into one of 2-4 accumulator chains (block b into chain b mod chains, so that
+//              consecutive blocks' MMAs do not wait on one another); one commit frees both
+//              rings' slots per super-block; a unit's last block commits its accumulators to
+//              the epilogue and the next unit starts in the other set.
+//   warps 6-9  epilogue: drain and add the chains (tcgen05.ld), release them, rescale by
+//              c_t = fp32(fp32(g * s_t) / 127) and store fp32 or bf16.  A row tile whose K
+//              blocks were split over several units writes its int32 partial to the
+//              workspace; the unit that arrives last on the tile's counter adds the others
+//              (integer sums: the split changes no result bit), stores the tile and resets
+//              the counter to zero for the next call.
+// Every mbarrier wait gives up after about a second and raises SBN_FLAG_TIMEOUT; a shared
+// abort flag then ends every role's loop, in-flight copies and MMAs are waited for
+// (bounded) and TMEM is freed.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <vector>
+
+#include "common.cuh"
+#include "group.cuh"
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace sbn {
+
+namespace {
+
+constexpr int kGrpThreads = 320;
+constexpr long long kGrpWaitCycles = 1ll << 31;  // about 1 s at 1.9 GHz
+constexpr int kSuper = 4;  // K blocks per weight super-block (one 64-byte box per row)
+
+template <int BN>
+struct GrpCfg {
+  // ring 1 in shared memory (the HBM stream), one slot per super-block of four 128-deep K
+  // blocks: the packed codes and the metadata of 128 rows (64 bytes per row each, 64-byte
+  // swizzle) and the four activation tiles (bn tokens x 128 inputs each, 128-byte swizzle)
+  static constexpr int kPlane = kGroupRows * 16 * kSuper;  // 8 KB
+  static constexpr int kBBytes = BN * kGroupKB;
+  static constexpr int kSlot1 = 2 * kPlane + kSuper * kBBytes;
+  static constexpr int kD1 = BN <= 16 ? 9 : 6;
+  // ring 2 in TMEM, one slot per super-block: per block the compressed A tile (lane r = row r,
+  // 16 columns of four int8 values) and the metadata (4 columns)
+  static constexpr int kD2 = 4;
+  // independent accumulator chains per unit: consecutive K blocks go to different TMEM
+  // accumulators so that their MMAs do not wait on one another; the epilogue adds them
+  static constexpr int kChains = BN <= 16 ? 4 : 2;
+  static constexpr int kAccCols = kChains * BN;         // one unit's accumulators
+  static constexpr int kACol = 2 * kAccCols;            // A ring after the two units' accumulators
+  static constexpr int kAColsPerSlot = kSuper * 16;
+  static constexpr int kMetaCol = kACol + kD2 * kAColsPerSlot;
+  static constexpr int kMColsPerSlot = kSuper * 4;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kBars = 2 * kD1 + 2 * kD2 + 5;
+  static constexpr size_t kSmem = 1024 + (size_t)kD1 * kSlot1 + (size_t)kBars * 8 + 64;
+  static_assert(kSlot1 % 1024 == 0 && kBBytes % 1024 == 0, "tile alignment");
+  static_assert(kMetaCol + kD2 * kMColsPerSlot <= kTmemCols, "TMEM columns");
+  static_assert(kSmem <= 227 * 1024, "shared memory budget");
+};
+
+__device__ __forceinline__ bool grp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    for (int i = 0; i < 64; ++i)
+      if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > kGrpWaitCycles) {
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// Bounded wait that ignores the abort flag: used to let in-flight copies and MMAs finish
+// before the CTA exits.
+__device__ __forceinline__ bool grp_drain(uint64_t *bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!ptx::mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kGrpWaitCycles) return false;
+  return true;
+}
+
+__device__ __forceinline__ bool grp_bar_any(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, 1, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void grp_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int BN>
+__global__ void __launch_bounds__(kGrpThreads, 1)
+    k_gemm_group(const uint8_t *__restrict__ plan, uint8_t *__restrict__ ws,
+                 int32_t *err_flag) {
+  using Cfg = GrpCfg<BN>;
+  constexpr int D1 = Cfg::kD1, D2 = Cfg::kD2, C = Cfg::kChains;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *ring1 = smem;  // [D1][codes | meta | 4 x B]
+  uint64_t *full1 = reinterpret_cast<uint64_t *>(ring1 + D1 * Cfg::kSlot1);
+  uint64_t *empty1 = full1 + D1;
+  uint64_t *full2 = empty1 + D1;
+  uint64_t *empty2 = full2 + D2;
+  uint64_t *acc_full = empty2 + D2;   // [2]
+  uint64_t *acc_empty = acc_full + 2;  // [2]
+  uint64_t *mma_done = acc_empty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+  volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_slot + 2);
+  volatile int *s_last = reinterpret_cast<volatile int *>(tmem_slot + 4);
+
+  ptx::grid_dep_launch();
+  const GroupHeader &hd = *reinterpret_cast<const GroupHeader *>(plan);
+  const GroupProb *probs = reinterpret_cast<const GroupProb *>(plan + hd.off_probs);
+  const GroupUnit *units = reinterpret_cast<const GroupUnit *>(plan + hd.off_units);
+  const int32_t *cta_begin = reinterpret_cast<const int32_t *>(plan + hd.off_cta);
+  const int u0 = cta_begin[blockIdx.x], u1 = cta_begin[blockIdx.x + 1];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < D1; ++s) {
+      ptx::mbar_init(&full1[s], 1);
+      ptx::mbar_init(&empty1[s], 1);
+    }
+    for (int s = 0; s < D2; ++s) {
+      ptx::mbar_init(&full2[s], 4);
+      ptx::mbar_init(&empty2[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&acc_full[b], 1);
+      ptx::mbar_init(&acc_empty[b], 4);
+    }
+    ptx::mbar_init(mma_done, 1);
+    *s_abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 5) {
+    ptx::tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::grid_dep_wait();  // the activation quantiser's Xq and scales are visible
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < 4) {
+    // ---------------- expanders: one super-block per hand-off ----------------
+    const int r = threadIdx.x;  // tile row
+    const int swz = (r >> 1) & 3;  // 64-byte swizzle of row r's 16-byte chunks
+    int64_t js = 0;  // super-block counter over this CTA's units
+    bool stop = false;
+    for (int u = u0; u < u1 && !stop; ++u) {
+      const GroupUnit un = units[u];
+      const GroupProb &p = probs[un.prob];
+      const bool row_ok = (int64_t)un.row_tile * kGroupRows + r < p.O;
+      const int64_t K = p.K;
+      for (int b0 = 0; b0 < un.nkb; b0 += kSuper, ++js) {
+        const int s1 = (int)(js % D1), s2 = (int)(js % D2);
+        const uint32_t ph1 = (uint32_t)(js / D1) & 1u, ph2 = (uint32_t)(js / D2) & 1u;
+        const bool ok = grp_wait(&full1[s1], ph1, s_abort) &&
+                        (js < D2 || grp_wait(&empty2[s2], ph2 ^ 1u, s_abort));
+        if (!__all_sync(0xffffffffu, ok)) {
+          stop = true;
+          break;
+        }
+        const int nb = min(kSuper, un.nkb - b0);
+        const uint8_t *slot1 = ring1 + s1 * Cfg::kSlot1;
+        const uint32_t lrow = ((uint32_t)(warp * 32)) << 16;  // this warp's TMEM lanes
+#pragma unroll
+        for (int g = 0; g < kSuper; ++g) {
+          if (g >= nb) break;
+          const int off = r * 64 + ((g ^ swz) << 4);
+          const uint4 cw = *reinterpret_cast<const uint4 *>(slot1 + off);
+          uint4 m4 = *reinterpret_cast<const uint4 *>(slot1 + Cfg::kPlane + off);
+          // metadata groups outside the matrix (rows >= O, or the second half of a last
+          // block with K % 128 == 64) were zero-filled by the TMA: give them the valid index
+          // pair (0, 1); their codes are zero
+          if (!row_ok) {
+            m4 = make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+          } else if ((int64_t)(un.kb0 + b0 + g) * kGroupKB + 64 >= K) {
+            m4.z = 0x44444444u;
+            m4.w = 0x44444444u;
+          }
+          ptx::tmem_st_4(tmem + lrow + (uint32_t)(Cfg::kMetaCol + s2 * Cfg::kMColsPerSlot + 4 * g),
+                         m4);
+          // 16 kept codes per word -> 16 int8 lanes of 64 * t, in K order: column 4c + q holds
+          // the four values (w[c] << 2q) & 0xC0C0C0C0
+          const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+          uint32_t a[16];
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) a[4 * c + q] = (w[c] << (2 * q)) & 0xC0C0C0C0u;
+          ptx::tmem_st_16(tmem + lrow + (uint32_t)(Cfg::kACol + s2 * Cfg::kAColsPerSlot + 16 * g),
+                          a);
+        }
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&full2[s2]);
+      }
+    }
+  } else if (warp == 4) {
+    // ---------------- TMA producer (ring 1: packed weights + activation tiles) ----------------
+    if (lane == 0) {
+      int64_t js = 0, issued = 0;
+      int last_prob = -1;
+      for (int u = u0; u < u1 && !*s_abort; ++u) {
+        const GroupUnit un = units[u];
+        const GroupProb &p = probs[un.prob];
+        if (un.prob != last_prob) {
+          ptx::prefetch_tmap(&p.tc);
+          ptx::prefetch_tmap(&p.tm);
+          ptx::prefetch_tmap(&p.tx);
+          last_prob = un.prob;
+        }
+        const int32_t row0 = un.row_tile * kGroupRows;
+        bool ok = true;
+        for (int b0 = 0; b0 < un.nkb; b0 += kSuper, ++js) {
+          const int s1 = (int)(js % D1);
+          const uint32_t ph1 = (uint32_t)(js / D1) & 1u;
+          if (js >= D1 && !grp_wait(&empty1[s1], ph1 ^ 1u, s_abort)) {
+            ok = false;
+            break;
+          }
+          const int nb = min(kSuper, un.nkb - b0);
+          const int32_t kb = un.kb0 + b0;
+          uint8_t *slot = ring1 + s1 * Cfg::kSlot1;
+          ptx::mbar_arrive_expect_tx(&full1[s1], (uint32_t)(2 * Cfg::kPlane + nb * Cfg::kBBytes));
+          ptx::tma_load_2d(slot, &p.tc, &full1[s1], kb * 16, row0);
+          ptx::tma_load_2d(slot + Cfg::kPlane, &p.tm, &full1[s1], kb * 16, row0);
+          for (int g = 0; g < nb; ++g)
+            ptx::tma_load_2d(slot + 2 * Cfg::kPlane + g * Cfg::kBBytes, &p.tx, &full1[s1],
+                             (kb + g) * kGroupKB, 0);
+          issued = js + 1;
+        }
+        if (!ok) break;
+      }
+      // every issued copy lands before the CTA can exit (bounded, also after an abort)
+      for (int64_t q = issued - D1 < 0 ? 0 : issued - D1; q < issued; ++q)
+        if (!grp_drain(&full1[q % D1], (uint32_t)(q / D1) & 1u)) *s_abort = 1;
+    }
+  } else if (warp == 5) {
+    // ---------------- metadata copy + sparse MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = ptx::idesc_i8_sparse(kGroupRows, BN);
+      int64_t js = 0;
+      int i = 0;
+      for (int u = u0; u < u1 && !*s_abort; ++u, ++i) {
+        const int nkb = units[u].nkb;
+        const int buf = i & 1;
+        if (i >= 2 && !grp_wait(&acc_empty[buf], ((uint32_t)(i >> 1) & 1u) ^ 1u, s_abort))
+          break;
+        ptx::tc_fence_after();
+        const uint32_t acc0 = tmem + (uint32_t)(buf * Cfg::kAccCols);
+        bool ok = true;
+        for (int b0 = 0; b0 < nkb; b0 += kSuper, ++js) {
+          const int s1 = (int)(js % D1), s2 = (int)(js % D2);
+          const uint32_t ph1 = (uint32_t)(js / D1) & 1u, ph2 = (uint32_t)(js / D2) & 1u;
+          if (!grp_wait(&full2[s2], ph2, s_abort) || !grp_wait(&full1[s1], ph1, s_abort)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint8_t *slot1 = ring1 + s1 * Cfg::kSlot1;
+          const int nb = min(kSuper, nkb - b0);
+          for (int g = 0; g < nb; ++g) {
+            const int b = b0 + g;
+            const uint32_t e_col = tmem + (uint32_t)(Cfg::kMetaCol + s2 * Cfg::kMColsPerSlot + 4 * g);
+            const uint32_t a_col = tmem + (uint32_t)(Cfg::kACol + s2 * Cfg::kAColsPerSlot + 16 * g);
+            const uint32_t b_addr = ptx::smem_u32(slot1 + 2 * Cfg::kPlane + g * Cfg::kBBytes);
+            const uint32_t d = acc0 + (uint32_t)((b % C) * BN);
+#pragma unroll
+            for (int k = 0; k < 2; ++k)  // logical K 64 per MMA: 8 columns of A, 64 bytes of B
+              ptx::mma_sp_i8_tmem_a(d, a_col + 8 * k, ptx::smem_desc_sw128(b_addr + 64 * k),
+                                    e_col + 2 * k, idesc, (b >= C || k != 0) ? 1u : 0u);
+          }
+          ptx::mma_commit(&empty2[s2]);
+          ptx::mma_commit(&empty1[s1]);
+        }
+        if (!ok) break;
+        ptx::mma_commit(&acc_full[buf]);
+      }
+      // every MMA issued has completed before TMEM can be released (also after an abort)
+      ptx::mma_commit(mma_done);
+      if (!grp_drain(mma_done, 0)) *s_abort = 1;
+    }
+  } else {
+    // ---------------- epilogue (warps 6-9) ----------------
+    const int q = warp & 3;  // the TMEM lane quarter this warp may read
+    const int et = q * 32 + lane;  // tile row
+    const uint64_t part_off = (uint64_t)hd.ws_part_off;
+    bool failed = false;
+    int i = 0;
+    for (int u = u0; u < u1; ++u, ++i) {
+      const int buf = i & 1;
+      // all four warps stop together if any wait of the previous unit gave up
+      if (grp_bar_any(failed)) break;
+      const GroupUnit un = units[u];
+      const GroupProb &p = probs[un.prob];
+      failed = !__all_sync(0xffffffffu, !*s_abort && grp_wait(&acc_full[buf],
+                                                              (uint32_t)(i >> 1) & 1u, s_abort));
+      ptx::tc_fence_after();
+      int32_t a[BN];
+#pragma unroll
+      for (int x = 0; x < BN; ++x) a[x] = 0;
+      if (!failed) {
+        const int nch = un.nkb < C ? un.nkb : C;  // chains this unit wrote
+        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * Cfg::kAccCols);
+#pragma unroll
+        for (int ch = 0; ch < C; ++ch) {
+          if (ch >= nch) break;
+#pragma unroll
+          for (int c = 0; c < BN; c += 16) {
+            uint32_t v[16];
+            ptx::tmem_ld_16(taddr + ch * BN + c, v);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 16; ++x) a[c + x] += (int32_t)v[x];
+          }
+        }
+#pragma unroll
+        for (int x = 0; x < BN; ++x) a[x] >>= 6;  // exact: the sums hold 64 * acc
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
+      if (grp_bar_any(failed)) {
+        failed = true;
+        break;
+      }
+      if (p.nparts > 1) {
+        // K split: publish this part, and let the last part to arrive finish the tile
+        int32_t *parts = reinterpret_cast<int32_t *>(ws + part_off) +
+                         (p.part_base + (int64_t)un.row_tile * p.nparts) * (kGroupRows * BN);
+        unsigned int *ticket = reinterpret_cast<unsigned int *>(ws) + p.ticket_base + un.row_tile;
+        int4 *mine = reinterpret_cast<int4 *>(parts + (int64_t)un.part * (kGroupRows * BN) +
+                                              (int64_t)et * BN);
+#pragma unroll
+        for (int c = 0; c < BN; c += 4) __stcg(mine + c / 4, make_int4(a[c], a[c + 1], a[c + 2], a[c + 3]));
+        __threadfence();
+        grp_bar_sync();
+        if (et == 0) *s_last = (atomicAdd(ticket, 1u) == (unsigned)(p.nparts - 1)) ? 1 : 0;
+        grp_bar_sync();
+        const bool last = *s_last != 0;
+        if (!last) continue;
+        __threadfence();
+        for (int pt = 0; pt < p.nparts; ++pt) {
+          if (pt == un.part) continue;
+          const int4 *other = reinterpret_cast<const int4 *>(parts + (int64_t)pt * (kGroupRows * BN) +
+                                                             (int64_t)et * BN);
+#pragma unroll
+          for (int c = 0; c < BN; c += 4) {
+            const int4 o4 = __ldcg(other + c / 4);
+            a[c] += o4.x, a[c + 1] += o4.y, a[c + 2] += o4.z, a[c + 3] += o4.w;
+          }
+        }
+        if (et == 0) *ticket = 0u;  // ready for the next call
+      }
+      // rescale and store: lane t holds c_t for token t
+      const int64_t T = p.T, O = p.O;
+      const float g = __ldg(p.gamma_eff);
+      const float c_lane = lane < T ? rescale_factor(g, __ldg(p.absmax + lane)) : 0.0f;
+      const int64_t o = (int64_t)un.row_tile * kGroupRows + et;
+      float *yf = reinterpret_cast<float *>(p.Y) + o;
+      __nv_bfloat16 *yb = reinterpret_cast<__nv_bfloat16 *>(p.Y) + o;
+#pragma unroll
+      for (int t = 0; t < BN; ++t) {
+        const float c = __shfl_sync(0xffffffffu, c_lane, t);
+        if (t < T && o < O) {
+          const float y = __fmul_rn(__int2float_rn(a[t]), c);
+          if (p.y_is_bf16)
+            yb[(int64_t)t * O] = __float2bfloat16_rn(y);
+          else
+            yf[(int64_t)t * O] = y;
+          if (p.acc_dbg) p.acc_dbg[(int64_t)t * O + o] = a[t];
+        }
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *s_abort && err_flag) atomicOr(err_flag, SBN_FLAG_TIMEOUT);
+  if (warp == 5) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+struct PlanShape {
+  int bn = 16;
+  int split = 1;
+  int64_t nunits = 0, nrows = 0, ntickets = 0, nparts_tiles = 0;
+  int ncta = 0;
+  int32_t max_nv = 0;
+  bool has_x = true;
+};
+
+// Linear partition of the units (in order) over at most `ncta` CTAs so that every CTA gets
+// about the same number of K blocks; returns the largest per-CTA cost (blocks + a fixed
+// cost per unit) and fills `begin` (ncta + 1 entries, may end with empty CTAs trimmed).
+int64_t partition_units(const std::vector<int32_t> &nkb, int ncta, int64_t unit_cost,
+                        std::vector<int32_t> *begin) {
+  int64_t total = 0;
+  for (int32_t b : nkb) total += b + unit_cost;
+  const int64_t n = (int64_t)nkb.size();
+  if (ncta > n) ncta = (int)n;
+  if (begin) begin->assign(1, 0);
+  int64_t worst = 0, cum = 0, cur = 0;
+  int c = 0;
+  for (int64_t u = 0; u < n; ++u) {
+    const int64_t w = nkb[u] + unit_cost;
+    // start a new CTA when this unit's midpoint lies past the current CTA's share
+    if (cur > 0 && c + 1 < ncta && 2 * (cum + w / 2) >= 2 * total * (c + 1) / ncta) {
+      worst = cur > worst ? cur : worst;
+      if (begin) begin->push_back((int32_t)u);
+      ++c;
+      cur = 0;
+    }
+    cur += w;
+    cum += w;
+  }
+  worst = cur > worst ? cur : worst;
+  if (begin) begin->push_back((int32_t)n);
+  return worst;
+}
+
+void build_units(const sbn_group_linear *lins, int count, int split,
+                 std::vector<GroupUnit> *units) {
+  units->clear();
+  for (int p = 0; p < count; ++p) {
+    const sbn_group_linear &l = lins[p];
+    if (l.tokens == 0) continue;
+    const int nkb = (int)((l.in + kGroupKB - 1) / kGroupKB);
+    const int parts = split < nkb ? split : nkb;
+    const int tiles = (int)((l.out + kGroupRows - 1) / kGroupRows);
+    for (int t = 0; t < tiles; ++t)
+      for (int q = 0; q < parts; ++q) {
+        GroupUnit u = {};
+        u.prob = p;
+        u.row_tile = t;
+        u.kb0 = (int)((int64_t)nkb * q / parts);
+        u.nkb = (int)((int64_t)nkb * (q + 1) / parts) - u.kb0;
+        u.part = q;
+        units->push_back(u);
+      }
+  }
+}
+
+// Cost model of the schedule in units of one K block's pipeline time: a unit adds a fixed
+// cost (accumulator hand-off, epilogue), a split adds the partial write and read-back.
+constexpr int64_t kUnitCost = 2;
+constexpr int64_t kSplitCost = 6;
+
+sbn_status plan_shape(const sbn_group_linear *lins, int count, PlanShape *ps,
+                      std::vector<GroupUnit> *units, std::vector<int32_t> *begin) {
+  int64_t maxT = 0;
+  ps->max_nv = 0;
+  ps->has_x = true;
+  ps->nrows = 0;
+  for (int p = 0; p < count; ++p) {
+    const sbn_group_linear &l = lins[p];
+    maxT = l.tokens > maxT ? l.tokens : maxT;
+    if (l.tokens > 0) {
+      ps->nrows += l.tokens;
+      if ((int32_t)(l.in / 8) > ps->max_nv) ps->max_nv = (int32_t)(l.in / 8);
+      if (!l.X) ps->has_x = false;
+    }
+  }
+  ps->bn = maxT <= 16 ? 16 : 32;
+  const int sms = num_sms();
+  // the split factor (the same for every layer) with the smallest estimated makespan
+  int best = 1;
+  int64_t best_cost = -1;
+  std::vector<GroupUnit> tmp;
+  std::vector<int32_t> nkb;
+  for (int split = 1; split <= 8; ++split) {
+    build_units(lins, count, split, &tmp);
+    if (tmp.empty()) break;
+    nkb.resize(tmp.size());
+    for (size_t u = 0; u < tmp.size(); ++u) nkb[u] = tmp[u].nkb;
+    const int64_t cost =
+        partition_units(nkb, sms, kUnitCost, nullptr) + (split > 1 ? kSplitCost : 0);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = split;
+    }
+  }
+  ps->split = best;
+  build_units(lins, count, best, units);
+  ps->nunits = (int64_t)units->size();
+  nkb.resize(units->size());
+  for (size_t u = 0; u < units->size(); ++u) nkb[u] = (*units)[u].nkb;
+  if (!units->empty()) {
+    partition_units(nkb, sms, kUnitCost, begin);
+    ps->ncta = (int)begin->size() - 1;
+  } else {
+    begin->assign(1, 0);
+    ps->ncta = 0;
+  }
+  // split layers: one counter per row tile, nparts partial tiles per row tile
+  ps->ntickets = 0;
+  ps->nparts_tiles = 0;
+  for (int p = 0; p < count; ++p) {
+    const sbn_group_linear &l = lins[p];
+    if (l.tokens == 0) continue;
+    const int nkbp = (int)((l.in + kGroupKB - 1) / kGroupKB);
+    const int parts = best < nkbp ? best : nkbp;
+    if (parts <= 1) continue;
+    const int64_t tiles = (l.out + kGroupRows - 1) / kGroupRows;
+    ps->ntickets += tiles;
+    ps->nparts_tiles += tiles * parts;
+  }
+  return SBN_OK;
+}
+
+struct PlanLayout {
+  int64_t off_probs, off_units, off_cta, off_rows, bytes;
+  int64_t ws_part_off, ws_bytes;
+};
+
+PlanLayout plan_layout(int count, const PlanShape &ps) {
+  PlanLayout L;
+  L.off_probs = 128;
+  L.off_units = L.off_probs + (int64_t)count * (int64_t)sizeof(GroupProb);
+  L.off_cta = align_up(L.off_units + ps.nunits * (int64_t)sizeof(GroupUnit), 128);
+  L.off_rows = align_up(L.off_cta + (int64_t)(ps.ncta + 1) * 4, 128);
+  L.bytes = align_up(L.off_rows + ps.nrows * (int64_t)sizeof(GroupRow), 128);
+  if (ps.ntickets > 0) {
+    L.ws_part_off = align_up(ps.ntickets * 4, 256);
+    L.ws_bytes = L.ws_part_off + ps.nparts_tiles * (int64_t)(kGroupRows * ps.bn * 4);
+  } else {
+    L.ws_part_off = 0;
+    L.ws_bytes = 0;
+  }
+  return L;
+}
+
+}  // namespace
+
+sbn_status group_plan_sizes(const sbn_group_linear *lins, int count, int64_t *plan_bytes,
+                            int64_t *workspace_bytes) {
+  PlanShape ps;
+  std::vector<GroupUnit> units;
+  std::vector<int32_t> begin;
+  sbn_status st = plan_shape(lins, count, &ps, &units, &begin);
+  if (st != SBN_OK) return st;
+  const PlanLayout L = plan_layout(count, ps);
+  *plan_bytes = L.bytes;
+  *workspace_bytes = L.ws_bytes;
+  return SBN_OK;
+}
+
+sbn_status group_plan(const sbn_group_linear *lins, int count, void *plan, int64_t plan_bytes) {
+  PlanShape ps;
+  std::vector<GroupUnit> units;
+  std::vector<int32_t> begin;
+  sbn_status st = plan_shape(lins, count, &ps, &units, &begin);
+  if (st != SBN_OK) return st;
+  const PlanLayout L = plan_layout(count, ps);
+  if (plan_bytes < L.bytes) return SBN_ERR_SHAPE;
+  uint8_t *P = static_cast<uint8_t *>(plan);
+  memset(P, 0, (size_t)L.bytes);
+  GroupHeader *hd = reinterpret_cast<GroupHeader *>(P);
+  hd->magic = kGroupMagic;
+  hd->version = kGroupVersion;
+  hd->count = count;
+  hd->nunits = (int32_t)ps.nunits;
+  hd->ncta = ps.ncta;
+  hd->bn = ps.bn;
+  hd->nrows = (int32_t)ps.nrows;
+  hd->max_nv = ps.max_nv;
+  hd->has_x = ps.has_x ? 1 : 0;
+  hd->split = ps.split;
+  hd->off_probs = L.off_probs;
+  hd->off_units = L.off_units;
+  hd->off_cta = L.off_cta;
+  hd->off_rows = L.off_rows;
+  hd->bytes = L.bytes;
+  hd->ws_bytes = L.ws_bytes;
+  hd->ntickets = ps.ntickets;
+  hd->ws_part_off = L.ws_part_off;
+  GroupProb *probs = reinterpret_cast<GroupProb *>(P + L.off_probs);
+  GroupRow *rows = reinterpret_cast<GroupRow *>(P + L.off_rows);
+  int64_t ticket = 0, part = 0, row = 0;
+  for (int p = 0; p < count; ++p) {
+    const sbn_group_linear &l = lins[p];
+    GroupProb &g = probs[p];
+    g.X = l.X;
+    g.Xq = l.Xq;
+    g.absmax = l.absmax;
+    g.gamma_eff = l.gamma_eff;
+    g.Y = l.Y;
+    g.acc_dbg = l.acc_dbg;
+    g.T = l.tokens;
+    g.O = l.out;
+    g.K = l.in;
+    g.y_is_bf16 = l.y_is_bf16 ? 1 : 0;
+    if (l.tokens == 0) continue;
+    const int64_t ldc = (l.in / 8 + 15) / 16 * 16, ldm = ldc;  // 2:4: K/8 bytes per plane row
+    if (!encode_u8(&g.tx, l.Xq, l.in, l.tokens, l.in, kGroupKB, (uint32_t)ps.bn,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_u8(&g.tc, l.codes, l.in / 8, l.out, ldc, 16 * kSuper, kGroupRows,
+                   CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode_u8(&g.tm, l.meta, l.in / 8, l.out, ldm, 16 * kSuper, kGroupRows,
+                   CU_TENSOR_MAP_SWIZZLE_64B))
+      return SBN_ERR_CUDA;
+    const int nkb = (int)((l.in + kGroupKB - 1) / kGroupKB);
+    g.nparts = ps.split < nkb ? ps.split : nkb;
+    if (g.nparts > 1) {
+      const int64_t tiles = (l.out + kGroupRows - 1) / kGroupRows;
+      g.ticket_base = ticket;
+      g.part_base = part;
+      ticket += tiles;
+      part += tiles * g.nparts;
+    }
+    for (int64_t t = 0; t < l.tokens; ++t) rows[row++] = GroupRow{p, (int32_t)t};
+  }
+  memcpy(P + L.off_units, units.data(), units.size() * sizeof(GroupUnit));
+  memcpy(P + L.off_cta, begin.data(), begin.size() * sizeof(int32_t));
+  return SBN_OK;
+}
+
+sbn_status launch_linear_group(const void *plan_host, const void *plan_dev, void *workspace,
+                               int32_t *err_flag, cudaStream_t st) {
+  const GroupHeader *hd = static_cast<const GroupHeader *>(plan_host);
+  if (hd->ncta == 0) return SBN_OK;
+  const uint8_t *P = static_cast<const uint8_t *>(plan_dev);
+  uint8_t *W = static_cast<uint8_t *>(workspace);
+  if (hd->bn == 16) {
+    auto kern = k_gemm_group<16>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)GrpCfg<16>::kSmem) != cudaSuccess)
+      return SBN_ERR_CUDA;
+    return launch_pdl(kern, dim3((unsigned)hd->ncta), dim3(kGrpThreads), GrpCfg<16>::kSmem, st,
+                      P, W, err_flag);
+  }
+  auto kern = k_gemm_group<32>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)GrpCfg<32>::kSmem) != cudaSuccess)
+    return SBN_ERR_CUDA;
+  return launch_pdl(kern, dim3((unsigned)hd->ncta), dim3(kGrpThreads), GrpCfg<32>::kSmem, st, P,
+                    W, err_flag);
+}
+
+}  // namespace sbn

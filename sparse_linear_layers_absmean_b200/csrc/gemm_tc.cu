@@ -1146,7 +1146,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 }
 
 // 2-D tensor map over a row-major uint8 matrix [rows, cols] with row stride `ld` bytes.
-static bool encode_u8(CUtensorMap *map, const void *base, int64_t cols, int64_t rows, int64_t ld,
+bool encode_u8(CUtensorMap *map, const void *base, int64_t cols, int64_t rows, int64_t ld,
                       uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
   auto encode = get_encode_fn();
   if (!encode) return false;

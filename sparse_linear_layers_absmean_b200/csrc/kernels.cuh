@@ -2,6 +2,7 @@
 // validated by the entry point and enqueues work on `st` without synchronising.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -86,6 +87,31 @@ sbn_status launch_count_zero_codes(const void *W, int64_t n, const float *gamma_
                                    unsigned long long *count, cudaStream_t st);
 sbn_status launch_count_mask_flips(const uint8_t *meta_a, const uint8_t *meta_b, int64_t nbytes,
                                    bool index_pairs, unsigned long long *count, cudaStream_t st);
+
+// 2-D tensor map over a row-major uint8 matrix [rows, cols] with row stride `ld` bytes and
+// a box of box_cols x box_rows bytes (zero fill outside the matrix); false on failure.
+bool encode_u8(CUtensorMap *map, const void *base, int64_t cols, int64_t rows, int64_t ld,
+               uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
+
+// Grouped calls (gemm_group.cu, act_quant.cu): host-side plan and the two launches.
+sbn_status group_plan_sizes(const sbn_group_linear *lins, int count, int64_t *plan_bytes,
+                            int64_t *workspace_bytes);
+sbn_status group_plan(const sbn_group_linear *lins, int count, void *plan, int64_t plan_bytes);
+sbn_status launch_act_quant_group(const void *plan_host, const void *plan_dev, int32_t *err_flag,
+                                  cudaStream_t st);
+sbn_status launch_linear_group(const void *plan_host, const void *plan_dev, void *workspace,
+                               int32_t *err_flag, cudaStream_t st);
+
+// Pre-expanded tensor-core operand of a 2:4 pack (gemm_operand.cu): size, expansion and the
+// contraction that reads it (rows padded to 256, K to 128; see k_expand_operand).
+int64_t operand_bytes(int64_t out, int64_t in);
+sbn_status launch_expand_operand(const uint8_t *codes, const uint8_t *meta, int64_t out,
+                                 int64_t in, int64_t ldc, int64_t ldm, void *operand,
+                                 cudaStream_t st);
+sbn_status launch_gemm_operand(const int8_t *Xq, const float *absmax, const void *operand,
+                               const float *gamma_eff, int64_t T, int64_t O, int64_t K, void *Y,
+                               int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag,
+                               cudaStream_t st);
 
 // Largest token count routed to the CUDA-core kernel; larger calls use the tensor cores.
 constexpr int64_t kGemvMaxTokens = 4;

@@ -6,36 +6,29 @@
 // whole device and fragment its memory.  For them the pack's only scratch -- the per-CTA
 // partial sums of the absmean reduction and the arrival counter -- lives in a fixed
 // array in this library's own device memory instead of a caller workspace.
-#include <mutex>
-
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace {
 
-// The scratch: one pack workspace (kPackMaxParts partial sums + counter + published
-// values).  8448 bytes on every GPU that loads the library, held until the process exits.
+// The scratch: one pack workspace (kPackMaxParts partial sums + reserved words).  8448
+// bytes on every GPU that loads the library, held until the process exits.
 constexpr size_t kNoallocScratchBytes = 8448;
 static_assert(sizeof(sbn::PackWorkspace) <= kNoallocScratchBytes, "scratch too small");
 static __device__ __align__(256) unsigned char g_pack_scratch[kNoallocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mutex;
-void *g_scratch_addr[kMaxDevices] = {};
-
-// Device address of g_pack_scratch on the current device.  In host code the symbol
-// itself is only a host-side stand-in, so the address is looked up once per device
-// (with that device current) and cached.
+// Device address of g_pack_scratch in the current context.  In host code the symbol is
+// only a host-side stand-in, so the address is looked up with the target device current.
+// It is looked up on every call (no allocation, a host-side table lookup once the module
+// is loaded) rather than cached: a cached address would go stale if the caller's context
+// were destroyed and recreated (cudaDeviceReset) or a different context made current.
 sbn_status scratch_for_current_device(void **out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SBN_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_mutex);
-  if (!g_scratch_addr[dev]) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_pack_scratch) != cudaSuccess || !p) return SBN_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_pack_scratch) != cudaSuccess || !p) {
+    (void)cudaGetLastError();
+    return SBN_ERR_CUDA;
   }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return SBN_OK;
 }
 
@@ -59,11 +52,9 @@ extern "C" SBN_API sbn_status sbn_quantize_mask_pack_weights_noalloc(
     return SBN_ERR_ALIGN;
   void *scratch = nullptr;
   if ((st = scratch_for_current_device(&scratch)) != SBN_OK) return st;
-  // The array keeps whatever the previous call left; the arrival counter must start at 0.
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(static_cast<unsigned char *>(scratch) + offsetof(sbn::PackWorkspace, ticket),
-                      0, sizeof(unsigned int), s) != cudaSuccess)
-    return SBN_ERR_CUDA;
+  // Nothing in the array needs clearing: the reduction kernel rewrites every partial sum
+  // the quant/mask/pack kernel reads (one per CTA it launches), and the second kernel
+  // waits for the first on the stream before reading them.
   return sbn_quantize_mask_pack_weights(W, out, in, n, m, eps, codes, meta, gamma_eff, scratch,
                                         dense_dbg, err_flag, stream);
 }

@@ -115,3 +115,55 @@ def test_statistics_entry_points_validate(L):
 def test_status_strings(L):
     for s in range(7):
         assert L.sbn_status_string(s)
+
+
+def _group(specs, A=0x10000):
+    """ctypes array of layers with placeholder (aligned, never dereferenced) pointers."""
+    arr = (sbn.SbnGroupLinear * len(specs))()
+    for i, (O, K, T, n, m) in enumerate(specs):
+        arr[i] = sbn.SbnGroupLinear(X=A, Xq=A, absmax=A, codes=A, meta=A, gamma_eff=A, Y=A,
+                                    acc_dbg=None, tokens=T, out=O, in_=K, n=n, m=m,
+                                    y_is_bf16=0, reserved=0)
+    return arr
+
+
+def _sizes(L, arr):
+    pb, wb = ctypes.c_int64(), ctypes.c_int64()
+    st = L.sbn_group_plan_sizes(ctypes.cast(arr, ctypes.c_void_p), len(arr), ctypes.byref(pb),
+                                ctypes.byref(wb))
+    return st, pb.value, wb.value
+
+
+def test_group_plan_sizes_validate(L):
+    assert _sizes(L, _group([(128, 256, 16, 6, 8)]))[0] == 3      # 2:4 only
+    assert _sizes(L, _group([(128, 256, 33, 2, 4)]))[0] == 2      # at most 32 tokens
+    assert _sizes(L, _group([(128, 96, 16, 2, 4)]))[0] == 2       # in % 64
+    assert _sizes(L, _group([(128, 256, 16, 2, 4)], A=0x10004))[0] == 4
+    arr = _group([(128, 256, 16, 2, 4)])
+    arr[0].Y = None
+    assert _sizes(L, arr)[0] == 1
+    arr = _group([(128, 256, 0, 2, 4)])
+    arr[0].Y = None                                               # 0 tokens: not checked
+    assert _sizes(L, arr)[0] == 0
+    assert L.sbn_group_plan_sizes(None, 1, ctypes.byref(ctypes.c_int64()),
+                                  ctypes.byref(ctypes.c_int64())) == 1
+    A = _p(0x10000)
+    assert L.sbn_group_plan(ctypes.cast(arr, ctypes.c_void_p), 1, _p(0x10040), 4096) == 4
+    assert L.sbn_linear_group(None, A, A, None, None) == 1
+    assert L.sbn_linear_group(A, _p(0x10040), A, None, None) == 4
+    assert L.sbn_quantize_acts_group(A, None, None, None) == 1
+
+
+def test_group_schedule_sizes(L):
+    """Host-side schedule (SM count 148 without a device): the whole 4096-hidden stack at 16
+    tokens has enough row tiles for every SM, so no split and no workspace; one small layer
+    alone is split over several units and needs a workspace for its partials."""
+    import workloads
+    stack = [(O, K, 16, 2, 4) for _ in range(workloads.STACK_LAYERS)
+             for _, O, K in workloads.STACK_LAYER_SHAPES]
+    st, pb, wb = _sizes(L, _group(stack))
+    assert st == 0 and wb == 0
+    tiles = workloads.STACK_LAYERS * sum((O + 127) // 128 for _, O, _ in workloads.STACK_LAYER_SHAPES)
+    assert pb >= 128 + 512 * len(stack) + 32 * tiles
+    st, pb, wb = _sizes(L, _group([(256, 4096, 16, 2, 4)]))
+    assert st == 0 and wb > 0

@@ -20,4 +20,4 @@ def test_reference_arm_json_line():
     assert d["value"] > 0 and d["steps"] == 1 and d["warmup"] == 3
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
-    assert d["config"]["workload"].startswith("decode")
+    assert d["config"]["workload"].startswith("stack-decode")
