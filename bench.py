@@ -216,11 +216,14 @@ class Timer:
 
 # ---- the stack (configuration 5) ----------------------------------------------------------
 
+STACK_LAYERS = workloads.STACK_LAYERS  # --stack-layers (profiling captures of a smaller stack)
+
+
 def stack_layers(rank=0):
     """(index, name, O, K, tensor id) of the 160 layers of one replica of the stack; rank r
     draws its replica's weights and activations from tensor ids offset by 1000 r."""
     out = []
-    for layer in range(workloads.STACK_LAYERS):
+    for layer in range(STACK_LAYERS):
         for i, (name, O, K) in enumerate(workloads.STACK_LAYER_SHAPES):
             out.append((5 * layer + i, name, O, K, 5 * layer + i + 1000 * rank))
     return out
@@ -794,7 +797,13 @@ def main():
     ap.add_argument("--no-sub", action="store_true", help="headline only, no sub-records")
     ap.add_argument("--only", choices=["pack", "act", "linear"],
                     help="profiling aid: one kind of C-ABI call, untimed (decode, prefill, stack)")
+    ap.add_argument("--stack-layers", type=int, default=workloads.STACK_LAYERS,
+                    help="profiling aid with --only: decoder layers of the stack (default 32)")
     args = ap.parse_args()
+    if args.stack_layers != workloads.STACK_LAYERS and not args.only:
+        sys.exit("--stack-layers is a profiling aid for --only runs")
+    global STACK_LAYERS
+    STACK_LAYERS = args.stack_layers
     if args.warmup < 3:
         args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "0"))

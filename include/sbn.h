@@ -278,6 +278,36 @@ SBN_API sbn_status sbn_linear_group(const void *plan, const void *plan_dev, void
                                     int32_t *err_flag, void *stream);
 
 /*
+ * Backward of the layer under the dual straight-through estimator (Sparse-BitNet summaries,
+ * section 2 "Estimador de Paso Directo Dual" / Sparse-BitLinear item 3: the quantiser passes
+ * the gradient as the identity inside its clip range; the mask passes it to every master
+ * weight, the pruned ones included):
+ *   dX[t, k] = g * sum_o dY[t, o] * Ws[o, k]
+ *   dW[o, k] = pass[o, k] * sum_t dY[t, o] * (s[t] / 127) * Xq[t, k],
+ *   pass[o, k] = (fl32(|W[o, k]| / g) <= 1)   (clip(W / g, -1, 1) has slope 1 there)
+ * with Ws the masked ternary matrix of (codes, meta), g = *gamma_eff, s and Xq from the
+ * forward's sbn_quantize_acts.  Computed on the tensor cores in bf16 x bf16 -> fp32 with
+ * exact products (dY * Ws is exact; s / 127 is folded into dY and carried as two bf16
+ * terms): the results differ from the exact sums only by fp32 accumulation and a relative
+ * 2^-17 on the scaled dY.
+ *   dY         bf16 [tokens, out], the upstream gradient.
+ *   W          bf16 [out, in] masters (read for the clip gate; may be NULL if dW is NULL).
+ *   dX         fp32 [tokens, in], written (NULL to skip).
+ *   dW         fp32 [out, in], written (NULL to skip).
+ *   workspace  device memory of sbn_backward_workspace_bytes (contents need no
+ *              initialisation; calls sharing it must not overlap).
+ *   err_flag   optional: SBN_FLAG_TIMEOUT.
+ * Shapes: those of sbn_linear, and out % 8 == 0.  tokens == 0 is a no-op.
+ */
+SBN_API sbn_status sbn_backward_workspace_bytes(int64_t tokens, int64_t out, int64_t in,
+                                                int64_t *bytes);
+SBN_API sbn_status sbn_backward(const void *dY, const int8_t *Xq, const float *absmax,
+                                const uint8_t *codes, const uint8_t *meta, const void *W,
+                                const float *gamma_eff, int64_t tokens, int64_t out, int64_t in,
+                                int n, int m, float *dX, float *dW, void *workspace,
+                                int32_t *err_flag, void *stream);
+
+/*
  * Mask statistics: by-products of steps 2-3 that follow how the masks evolve over training
  * steps (Sparse-BitNet summaries: section 3 "Contribuciones Clave" item 1, the large share
  * of ternary zeros; section 2, the mask recomputed every step from the current masters).

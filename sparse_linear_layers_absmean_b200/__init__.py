@@ -31,7 +31,8 @@ EXPORTED = ("sbn_linear_ref_dims", "sbn_quantize_mask_pack_weights", "sbn_quanti
             "sbn_linear", "sbn_status_string", "sbn_quantize_mask_pack_weights_noalloc",
             "sbn_count_zero_codes", "sbn_count_mask_flips", "sbn_group_plan_sizes",
             "sbn_group_plan", "sbn_quantize_acts_group", "sbn_linear_group",
-            "sbn_operand_bytes", "sbn_expand_operand", "sbn_linear_operand")
+            "sbn_operand_bytes", "sbn_expand_operand", "sbn_linear_operand",
+            "sbn_backward_workspace_bytes", "sbn_backward")
 
 
 class SbnError(RuntimeError):
@@ -100,6 +101,10 @@ def lib():
         L.sbn_expand_operand.restype = i32
         L.sbn_linear_operand.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, p, i32, p, p, p]
         L.sbn_linear_operand.restype = i32
+        L.sbn_backward_workspace_bytes.argtypes = [i64, i64, i64, p]
+        L.sbn_backward_workspace_bytes.restype = i32
+        L.sbn_backward.argtypes = [p, p, p, p, p, p, p, i64, i64, i64, i32, i32, p, p, p, p, p]
+        L.sbn_backward.restype = i32
         L.sbn_status_string.argtypes = [i32]
         L.sbn_status_string.restype = ctypes.c_char_p
         _LIB = L
@@ -405,3 +410,34 @@ def linear_operand(Xq, s, w: PackedWeights, operand, out_dtype=torch.float32, ac
     sbn_linear_operand(Xq, s, operand, w.gamma_eff, w.out, w.in_, w.n, w.m, Y, acc_dbg, err_flag,
                        stream)
     return Y
+
+
+# ---- dual-STE backward ---------------------------------------------------------------------
+
+def sbn_backward_workspace_bytes(tokens, out, in_):
+    b = ctypes.c_int64()
+    _check(lib().sbn_backward_workspace_bytes(tokens, out, in_, ctypes.byref(b)),
+           "sbn_backward_workspace_bytes")
+    return b.value
+
+
+def sbn_backward(dY, Xq, absmax, codes, meta, W, gamma_eff, out, in_, n, m, dX, dW, workspace,
+                 err_flag=None, stream=None):
+    _check(lib().sbn_backward(_ptr(dY), _ptr(Xq), _ptr(absmax), _ptr(codes), _ptr(meta), _ptr(W),
+                              _ptr(gamma_eff), dY.shape[0], out, in_, n, m, _ptr(dX), _ptr(dW),
+                              _ptr(workspace), _ptr(err_flag), _stream(stream)), "sbn_backward")
+
+
+def backward(dY: torch.Tensor, Xq: torch.Tensor, s: torch.Tensor, w: PackedWeights,
+             W: torch.Tensor, need_dX=True, need_dW=True, err_flag=None, stream=None):
+    """(dX fp32 [T, in] or None, dW fp32 [out, in] or None) for the upstream gradient dY
+    (bf16 [T, out]) of the forward that used Xq, s and the pack w of the masters W."""
+    T = dY.shape[0]
+    with _alloc_stream(stream):
+        dX = torch.empty((T, w.in_), dtype=torch.float32, device=dY.device) if need_dX else None
+        dW = torch.empty((w.out, w.in_), dtype=torch.float32, device=dY.device) if need_dW else None
+        ws = torch.empty(max(256, sbn_backward_workspace_bytes(T, w.out, w.in_)), dtype=torch.uint8,
+                         device=dY.device)
+    sbn_backward(dY, Xq, s, w.codes, w.meta, W, w.gamma_eff, w.out, w.in_, w.n, w.m, dX, dW, ws,
+                 err_flag, stream)
+    return dX, dW

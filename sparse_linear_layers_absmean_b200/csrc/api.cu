@@ -192,6 +192,38 @@ sbn_status sbn_linear_operand(const int8_t *Xq, const float *absmax, const void 
                                   acc_dbg, err_flag, static_cast<cudaStream_t>(stream));
 }
 
+sbn_status sbn_backward_workspace_bytes(int64_t tokens, int64_t out, int64_t in, int64_t *bytes) {
+  if (!bytes) return SBN_ERR_NULL;
+  sbn_dims d;
+  sbn_status st = sbn_linear_ref_dims(out, in, 2, 4, &d);
+  if (st != SBN_OK) return st;
+  if (out % 8 != 0 || tokens < 0 || tokens > (1ll << 24)) return SBN_ERR_SHAPE;
+  *bytes = sbn::backward_workspace_bytes(tokens, out, in);
+  return SBN_OK;
+}
+
+sbn_status sbn_backward(const void *dY, const int8_t *Xq, const float *absmax, const uint8_t *codes,
+                        const uint8_t *meta, const void *W, const float *gamma_eff, int64_t tokens,
+                        int64_t out, int64_t in, int n, int m, float *dX, float *dW,
+                        void *workspace, int32_t *err_flag, void *stream) {
+  sbn_dims d;
+  sbn_status st = sbn_linear_ref_dims(out, in, n, m, &d);
+  if (st != SBN_OK) return st;
+  if (out % 8 != 0 || tokens < 0 || tokens > (1ll << 24)) return SBN_ERR_SHAPE;
+  if (tokens == 0 || (!dX && !dW)) return SBN_OK;
+  if (!dY || !gamma_eff || !workspace) return SBN_ERR_NULL;
+  if (dX && (!codes || !meta)) return SBN_ERR_NULL;
+  if (dW && (!Xq || !absmax || !W)) return SBN_ERR_NULL;
+  if (!aligned16(dY) || !aligned16(workspace) || (dX && (!aligned16(dX) || !aligned16(codes) ||
+                                                         !aligned16(meta))) ||
+      (dW && (!aligned16(dW) || !aligned16(W))) || (absmax && (reinterpret_cast<uintptr_t>(absmax) & 3u)) ||
+      (reinterpret_cast<uintptr_t>(gamma_eff) & 3u) || (reinterpret_cast<uintptr_t>(err_flag) & 3u))
+    return SBN_ERR_ALIGN;
+  return sbn::launch_backward(dY, Xq, absmax, codes, meta, W, gamma_eff, tokens, out, in, n, m,
+                              d.codes_ld, d.meta_ld, dX, dW, workspace, err_flag,
+                              static_cast<cudaStream_t>(stream));
+}
+
 sbn_status sbn_group_plan_sizes(const sbn_group_linear *lins, int32_t count, int64_t *plan_bytes,
                                 int64_t *workspace_bytes) {
   if (!plan_bytes || !workspace_bytes) return SBN_ERR_NULL;

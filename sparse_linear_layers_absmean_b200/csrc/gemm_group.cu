@@ -10,21 +10,23 @@
 // units with about the same number of K blocks; the CTA walks its run as one pipeline in
 // super-blocks of four 128-deep K blocks (every hand-off between the roles has a fixed cost,
 // so each one moves four blocks):
-//   warp 4     TMA producer, ring 1 (the HBM stream, 4-6 slots): per super-block the packed
+//   warp 4     TMA producer, ring 1 (the HBM stream, 6-9 slots): per super-block the packed
 //              codes and the metadata of the unit's 128 rows as two boxes of 64 bytes x 128
 //              rows (64-byte swizzle), and the four activation tiles (bn tokens x 128 inputs,
 //              128-byte swizzle; L2 hits, all row tiles of a layer share them).
-//   warps 0-3  expanders, ring 2 (2 slots): thread r turns row r's kept codes into 64 int8
-//              lanes of 64 * t per block (the compressed A tile, 64-byte swizzle) and copies
-//              the metadata into the 16-byte-row layout tcgen05.cp reads (groups outside the
-//              matrix get the valid index pair (0, 1)); one proxy fence and one arrival per
-//              super-block.
-//   warp 5     TMEM allocation and the MMA thread: per block the metadata goes to TMEM
-//              (tcgen05.cp) and two sparse MMAs (M 128, N bn, logical K 64 each) accumulate
-//              into one of 2-4 accumulator chains (block b into chain b mod chains, so that
-//              consecutive blocks' MMAs do not wait on one another); one commit frees both
-//              rings' slots per super-block; a unit's last block commits its accumulators to
-//              the epilogue and the next unit starts in the other set.
+//   warps 0-3, 10-13  two groups of expanders taking alternate super-blocks, ring 2 in TMEM
+//              (4 slots): thread r turns row r's kept codes into 64 int8 lanes of 64 * t per
+//              block (the compressed A tile) and writes them with the block's metadata
+//              (groups outside the matrix get the valid index pair (0, 1)) into TMEM lane r
+//              with tcgen05.st; one wait and one arrival per super-block.  A never passes
+//              through shared memory, and no tcgen05.cp is needed.
+//   warps 5, 14  two MMA threads taking alternate super-blocks (the issue of a tcgen05.mma
+//              of this small shape, not the tensor pipe, sets the pace of one thread): per
+//              block two sparse MMAs (M 128, N bn, logical K 64 each; A and the metadata read
+//              from TMEM, B from shared memory) into one of the thread's two accumulator
+//              chains; one commit frees both rings' slots per super-block; at a unit's end
+//              both commit its accumulators to the epilogue and the next unit starts in the
+//              other set (warp 5 also allocates TMEM).
 //   warps 6-9  epilogue: drain and add the chains (tcgen05.ld), release them, rescale by
 //              c_t = fp32(fp32(g * s_t) / 127) and store fp32 or bf16.  A row tile whose K
 //              blocks were split over several units writes its int32 partial to the
@@ -48,7 +50,7 @@ namespace sbn {
 
 namespace {
 
-constexpr int kGrpThreads = 320;
+constexpr int kGrpThreads = 480;  // 15 warps (two expander groups, two MMA threads)
 constexpr long long kGrpWaitCycles = 1ll << 31;  // about 1 s at 1.9 GHz
 constexpr int kSuper = 4;  // K blocks per weight super-block (one 64-byte box per row)
 
@@ -63,10 +65,12 @@ struct GrpCfg {
   static constexpr int kD1 = BN <= 16 ? 9 : 6;
   // ring 2 in TMEM, one slot per super-block: per block the compressed A tile (lane r = row r,
   // 16 columns of four int8 values) and the metadata (4 columns)
-  static constexpr int kD2 = 4;
-  // independent accumulator chains per unit: consecutive K blocks go to different TMEM
-  // accumulators so that their MMAs do not wait on one another; the epilogue adds them
-  static constexpr int kChains = BN <= 16 ? 4 : 2;
+  static constexpr int kD2 = BN <= 16 ? 4 : 2;
+  // accumulator chains per unit: two MMA threads take alternate super-blocks, each into its
+  // own kChains / 2 chains (block b of its super-blocks into chain b mod (kChains / 2)); the
+  // epilogue adds the chains
+  static constexpr int kChains = 4;
+  static constexpr int kCpt = kChains / 2;  // chains per MMA thread
   static constexpr int kAccCols = kChains * BN;         // one unit's accumulators
   static constexpr int kACol = 2 * kAccCols;            // A ring after the two units' accumulators
   static constexpr int kAColsPerSlot = kSuper * 16;
@@ -157,10 +161,10 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
       ptx::mbar_init(&empty2[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(&acc_full[b], 1);
+      ptx::mbar_init(&acc_full[b], 2);  // both MMA threads commit
       ptx::mbar_init(&acc_empty[b], 4);
     }
-    ptx::mbar_init(mma_done, 1);
+    ptx::mbar_init(mma_done, 2);
     *s_abort = 0;
     ptx::fence_mbar_init();
   }
@@ -174,9 +178,12 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < 4) {
-    // ---------------- expanders: one super-block per hand-off ----------------
-    const int r = threadIdx.x;  // tile row
+  if (warp < 4 || (warp >= 10 && warp < 14)) {
+    // ---------------- expanders: two groups of four warps take alternate super-blocks;
+    // warp w writes TMEM lanes 32 (w mod 4) .. + 31, i.e. tile rows of that quarter ----------
+    const int grp = warp < 4 ? 0 : 1;
+    const int qw = warp & 3;
+    const int r = qw * 32 + lane;  // tile row
     const int swz = (r >> 1) & 3;  // 64-byte swizzle of row r's 16-byte chunks
     int64_t js = 0;  // super-block counter over this CTA's units
     bool stop = false;
@@ -186,6 +193,7 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
       const bool row_ok = (int64_t)un.row_tile * kGroupRows + r < p.O;
       const int64_t K = p.K;
       for (int b0 = 0; b0 < un.nkb; b0 += kSuper, ++js) {
+        if ((int)(js & 1) != grp) continue;
         const int s1 = (int)(js % D1), s2 = (int)(js % D2);
         const uint32_t ph1 = (uint32_t)(js / D1) & 1u, ph2 = (uint32_t)(js / D2) & 1u;
         const bool ok = grp_wait(&full1[s1], ph1, s_abort) &&
@@ -196,7 +204,7 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
         }
         const int nb = min(kSuper, un.nkb - b0);
         const uint8_t *slot1 = ring1 + s1 * Cfg::kSlot1;
-        const uint32_t lrow = ((uint32_t)(warp * 32)) << 16;  // this warp's TMEM lanes
+        const uint32_t lrow = ((uint32_t)(qw * 32)) << 16;  // this warp's TMEM lanes
 #pragma unroll
         for (int g = 0; g < kSuper; ++g) {
           if (g >= nb) break;
@@ -271,9 +279,10 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
       for (int64_t q = issued - D1 < 0 ? 0 : issued - D1; q < issued; ++q)
         if (!grp_drain(&full1[q % D1], (uint32_t)(q / D1) & 1u)) *s_abort = 1;
     }
-  } else if (warp == 5) {
-    // ---------------- metadata copy + sparse MMA issuer ----------------
+  } else if (warp == 5 || warp == 14) {
+    // ---------------- two sparse-MMA threads: alternate super-blocks ----------------
     if (lane == 0) {
+      const int mt = warp == 5 ? 0 : 1;  // takes the unit's super-blocks j with j % 2 == mt
       constexpr uint32_t idesc = ptx::idesc_i8_sparse(kGroupRows, BN);
       int64_t js = 0;
       int i = 0;
@@ -286,6 +295,7 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
         const uint32_t acc0 = tmem + (uint32_t)(buf * Cfg::kAccCols);
         bool ok = true;
         for (int b0 = 0; b0 < nkb; b0 += kSuper, ++js) {
+          if (((b0 / kSuper) & 1) != mt) continue;  // by the unit's own super-block index
           const int s1 = (int)(js % D1), s2 = (int)(js % D2);
           const uint32_t ph1 = (uint32_t)(js / D1) & 1u, ph2 = (uint32_t)(js / D2) & 1u;
           if (!grp_wait(&full2[s2], ph2, s_abort) || !grp_wait(&full1[s1], ph1, s_abort)) {
@@ -300,11 +310,13 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
             const uint32_t e_col = tmem + (uint32_t)(Cfg::kMetaCol + s2 * Cfg::kMColsPerSlot + 4 * g);
             const uint32_t a_col = tmem + (uint32_t)(Cfg::kACol + s2 * Cfg::kAColsPerSlot + 16 * g);
             const uint32_t b_addr = ptx::smem_u32(slot1 + 2 * Cfg::kPlane + g * Cfg::kBBytes);
-            const uint32_t d = acc0 + (uint32_t)((b % C) * BN);
+            const uint32_t d = acc0 + (uint32_t)((mt * Cfg::kCpt + g % Cfg::kCpt) * BN);
+            // the first blocks of this thread's first super-block of the unit start its chains
+            const bool first = b0 / kSuper == mt && g < Cfg::kCpt;
 #pragma unroll
             for (int k = 0; k < 2; ++k)  // logical K 64 per MMA: 8 columns of A, 64 bytes of B
               ptx::mma_sp_i8_tmem_a(d, a_col + 8 * k, ptx::smem_desc_sw128(b_addr + 64 * k),
-                                    e_col + 2 * k, idesc, (b >= C || k != 0) ? 1u : 0u);
+                                    e_col + 2 * k, idesc, (!first || k != 0) ? 1u : 0u);
           }
           ptx::mma_commit(&empty2[s2]);
           ptx::mma_commit(&empty1[s1]);
@@ -336,11 +348,11 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
 #pragma unroll
       for (int x = 0; x < BN; ++x) a[x] = 0;
       if (!failed) {
-        const int nch = un.nkb < C ? un.nkb : C;  // chains this unit wrote
         const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * Cfg::kAccCols);
 #pragma unroll
         for (int ch = 0; ch < C; ++ch) {
-          if (ch >= nch) break;
+          // chain ch starts at block 4 t + r of the unit (t = ch / kCpt, r = ch % kCpt)
+          if (kSuper * (ch / Cfg::kCpt) + ch % Cfg::kCpt >= un.nkb) continue;
 #pragma unroll
           for (int c = 0; c < BN; c += 16) {
             uint32_t v[16];

@@ -4,8 +4,7 @@
 // Three kernels share the pipeline below: k_gemm_tc (dense codes, any N:M pattern; one
 // tile per CTA), k_gemm_sp24 (2:4 on the sparse MMA; one tile per CTA, up to 128 tokens)
 // and, for more tokens, k_gemm_sp24_pair (2:4, CTA pairs, persistent, double-buffered
-// accumulators; k_gemm_sp24_persist is its single-CTA form, used where a cluster launch
-// is not available).
+// accumulators).
 //
 // One CTA computes a 128 (outputs) x BN (tokens) tile with a multi-stage shared-memory
 // pipeline over K in blocks of 128 (a stage holds one to four consecutive blocks: each
@@ -42,7 +41,14 @@ constexpr int kBK = 128;
 // Waits give up after 2^31 SM cycles (about 1 s at the 1965 MHz boost clock, 2 s at 1 GHz).
 // The bound is kept with the SM's cycle counter: reading the global nanosecond timer costs
 // about a tenth of a microsecond, which would sit on the critical path of every hand-off.
+#ifdef SBN_TIMEOUT_TEST
+// Test build only (tests/test_timeout_gpu.py): waits give up after 2^20 cycles (about half
+// a millisecond), and in k_gemm_sp24 the first expander warp withholds its arrival for the
+// second pipeline stage, so the MMA thread's wait on that stage runs out.
+constexpr long long kWaitCycles = 1ll << 20;
+#else
 constexpr long long kWaitCycles = 1ll << 31;
+#endif
 
 // Bounded wait on an mbarrier phase; false on timeout.  (mbarrier.try_wait itself suspends
 // the thread for a while when the phase is not yet complete.)
@@ -324,6 +330,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ptx::mma_commit(&empty[s]);
       }
       ptx::mma_commit(done);
+      // every MMA issued has completed before TMEM can be released, also after a timeout
+      // (the epilogue skips its wait then)
+      if (!wait_phase(done, 0)) timed_out = true;
     }
   }
 
@@ -487,7 +496,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       ptx::fence_proxy_async_smem();
       __syncwarp();
+#ifdef SBN_TIMEOUT_TEST
+      if (lane == 0 && !(warp == 0 && j == 1)) ptx::mbar_arrive(&full_a[s]);
+#else
       if (lane == 0) ptx::mbar_arrive(&full_a[s]);
+#endif
     }
   } else if (warp == 4) {
     // ---------------- TMA producer ----------------
@@ -548,6 +561,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ptx::mma_commit(&empty[s]);
       }
       ptx::mma_commit(done);
+      // every MMA issued has completed before TMEM can be released, also after a timeout
+      // (the epilogue skips its wait then)
+      if (!wait_phase(done, 0)) timed_out = true;
     }
   }
 
@@ -603,41 +619,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------------
-// Persistent 2:4 kernel for large token counts.  Each CTA loops over output tiles
-// (128 weight rows x BN tokens); the TMEM holds two accumulators so that four dedicated
-// epilogue warps drain tile i while the MMA already accumulates tile i+1.
-//   warps 0-3  expanders (compressed A tiles), warp 4 TMA, warp 5 TMEM + MMA issue,
-//   warps 6-9  epilogue (warp w reads accumulator lanes 32*(w%4) .. +31).
-// Every wait is bounded; a timeout anywhere raises a shared abort flag that ends all loops.
+// Helpers of the persistent CTA-pair kernel below: every wait is bounded; a timeout anywhere
+// raises a shared abort flag that ends all loops.
 // ---------------------------------------------------------------------------------------
 
 constexpr int kPsThreads = 320;
-
-template <int BN>
-struct PsCfg {
-  static constexpr int kKL = 128;
-  static constexpr int kABytes = kBM * kKL / 2;
-  static constexpr int kBBytes = BN * kKL;
-  static constexpr int kPBytes = kBM * 16 * 2;
-  static constexpr int kStageBytes = kABytes + kBBytes + kPBytes;
-  static constexpr int kBudget = 225 * 1024 - BN * 4 - 1024;
-  static constexpr int kStages = (kBudget / kStageBytes) > 8 ? 8 : (kBudget / kStageBytes);
-  // accumulator b at TMEM columns 256 * b .. 256 * b + BN - 1; each stage's 4 metadata
-  // columns sit in the gaps after the accumulators
-  static constexpr int kAccStride = 256;
-  static constexpr int kGap = (256 - BN) / 4;  // metadata slots after one accumulator
-  static_assert(BN <= 256 && BN % 16 == 0, "tile width");
-  static_assert(2 * kGap >= kStages, "two accumulators and the metadata must fit in TMEM");
-  static constexpr int kTmemCols = 512;
-  __device__ static constexpr uint32_t meta_col(int s) {
-    return s < kGap ? (uint32_t)(BN + 4 * s) : (uint32_t)(kAccStride + BN + 4 * (s - kGap));
-  }
-  static constexpr uint32_t kTxBytes = kBBytes + kPBytes;
-  // barriers: full_a[S], full_t[S], empty[S], acc_full[2], acc_empty[2], mma_done; then the
-  // TMEM address, the abort flag (32 bytes) and the per-token scales
-  static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes +
-                                  (size_t)(3 * kStages + 5) * 8 + 32 + (size_t)BN * 4;
-};
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
@@ -668,203 +654,6 @@ __device__ __forceinline__ bool bar_any(int id, int n, bool pred) {
   return r != 0;
 }
 
-template <int BN>
-__global__ void __launch_bounds__(kPsThreads, 1)
-    k_gemm_sp24_persist(const __grid_constant__ CUtensorMap tmap_x,
-                        const __grid_constant__ CUtensorMap tmap_c,
-                        const __grid_constant__ CUtensorMap tmap_m,
-                        const float *__restrict__ absmax, const float *__restrict__ gamma_eff,
-                        int64_t T, int64_t O, int64_t K, void *__restrict__ Y, int y_is_bf16,
-                        int32_t *__restrict__ acc_dbg, int32_t *err_flag) {
-  using Cfg = PsCfg<BN>;
-  constexpr int S = Cfg::kStages;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *sB = smem;
-  uint8_t *sA = sB + S * Cfg::kBBytes;
-  uint8_t *sP = sA + S * Cfg::kABytes;
-  uint64_t *full_a = reinterpret_cast<uint64_t *>(sP + S * Cfg::kPBytes);
-  uint64_t *full_t = full_a + S;
-  uint64_t *empty = full_t + S;
-  uint64_t *acc_full = empty + S;   // [2]
-  uint64_t *acc_empty = acc_full + 2;  // [2]
-  uint64_t *mma_done = acc_empty + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
-  volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_slot + 2);
-  float *s_scale = reinterpret_cast<float *>(tmem_slot + 8);
-
-  // the next kernel on the stream may start its prologue; it waits for this one
-  ptx::grid_dep_launch();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nkb = (int)((K + Cfg::kKL - 1) / Cfg::kKL);
-  const int64_t n_o = (O + kBM - 1) / kBM, n_t = (T + BN - 1) / BN;
-  const int64_t ntiles = n_o * n_t;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      ptx::mbar_init(&full_a[s], 4);
-      ptx::mbar_init(&full_t[s], 1);
-      ptx::mbar_init(&empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(&acc_full[b], 1);
-      ptx::mbar_init(&acc_empty[b], 4);
-    }
-    ptx::mbar_init(mma_done, 1);
-    *s_abort = 0;
-    ptx::fence_mbar_init();
-  }
-  if (warp == 5) {
-    ptx::tmem_alloc(tmem_slot, Cfg::kTmemCols);
-    ptx::tmem_relinquish();
-  }
-  ptx::grid_dep_wait();  // the previous kernel's outputs (activations, scales) are visible
-  ptx::tc_fence_before();
-  __syncthreads();
-  ptx::tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp < 4) {
-    // ---------------- compressed-weight expanders ----------------
-    const int r = threadIdx.x;
-    int64_t kg = 0;
-    for (int64_t tile = blockIdx.x;
-         tile < ntiles && !__any_sync(0xffffffffu, *s_abort != 0); tile += gridDim.x) {
-      const int64_t o0 = (tile % n_o) * kBM;
-      for (int kb = 0; kb < nkb; ++kb, ++kg) {
-        const int s = (int)(kg % S);
-        const uint32_t ph = (uint32_t)(kg / S) & 1u;
-        const bool ok = (kg < S || wait_or_abort(&empty[s], ph ^ 1u, s_abort)) &&
-                        wait_or_abort(&full_t[s], ph, s_abort);
-        if (!__all_sync(0xffffffffu, ok)) break;  // the whole warp leaves together
-        const uint4 cw = *reinterpret_cast<const uint4 *>(sP + s * Cfg::kPBytes + r * 16);
-        const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
-        if (o0 + r >= O) {
-          *reinterpret_cast<uint4 *>(sP + s * Cfg::kPBytes + kBM * 16 + r * 16) =
-              make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
-        } else if ((int64_t)kb * Cfg::kKL + 64 >= K) {
-          *reinterpret_cast<uint2 *>(sP + s * Cfg::kPBytes + kBM * 16 + r * 16 + 8) =
-              make_uint2(0x44444444u, 0x44444444u);
-        }
-        uint8_t *dst = sA + s * Cfg::kABytes + r * 64;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4 *>(dst + ((c ^ ((r >> 1) & 3)) << 4)) =
-              make_uint4(w[c] & 0xC0C0C0C0u, (w[c] << 2) & 0xC0C0C0C0u,
-                         (w[c] << 4) & 0xC0C0C0C0u, (w[c] << 6) & 0xC0C0C0C0u);
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&full_a[s]);
-      }
-    }
-  } else if (warp == 4) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
-      ptx::prefetch_tmap(&tmap_x);
-      ptx::prefetch_tmap(&tmap_c);
-      ptx::prefetch_tmap(&tmap_m);
-      int64_t kg = 0, issued = 0;
-      for (int64_t tile = blockIdx.x; tile < ntiles && !*s_abort; tile += gridDim.x) {
-        const int64_t o0 = (tile % n_o) * kBM, t0 = (tile / n_o) * BN;
-        for (int kb = 0; kb < nkb; ++kb, ++kg) {
-          const int s = (int)(kg % S);
-          const uint32_t ph = (uint32_t)(kg / S) & 1u;
-          if (kg >= S && !wait_or_abort(&empty[s], ph ^ 1u, s_abort)) break;
-          ptx::mbar_arrive_expect_tx(&full_t[s], Cfg::kTxBytes);
-          ptx::tma_load_2d(sB + s * Cfg::kBBytes, &tmap_x, &full_t[s], kb * Cfg::kKL,
-                           (int32_t)t0);
-          uint8_t *p = sP + s * Cfg::kPBytes;
-          ptx::tma_load_2d(p, &tmap_c, &full_t[s], kb * 16, (int32_t)o0);
-          ptx::tma_load_2d(p + kBM * 16, &tmap_m, &full_t[s], kb * 16, (int32_t)o0);
-          issued = kg + 1;
-        }
-      }
-      // every issued copy lands before the CTA can exit (bounded, even after an abort)
-      for (int64_t q = issued - S < 0 ? 0 : issued - S; q < issued; ++q)
-        if (!wait_phase(&full_t[q % S], (uint32_t)(q / S) & 1u)) *s_abort = 1;
-    }
-  } else if (warp == 5) {
-    // ---------------- metadata copy + sparse MMA issuer ----------------
-    if (lane == 0) {
-      constexpr uint32_t idesc = ptx::idesc_i8_sparse(kBM, BN);
-      int64_t kg = 0;
-      int i = 0;
-      for (int64_t tile = blockIdx.x; tile < ntiles && !*s_abort; tile += gridDim.x, ++i) {
-        const int buf = i & 1;
-        if (i >= 2 && !wait_or_abort(&acc_empty[buf], ((uint32_t)(i >> 1) & 1u) ^ 1u, s_abort))
-          break;
-        ptx::tc_fence_after();
-        const uint32_t d_tmem = tmem + (uint32_t)(buf * Cfg::kAccStride);
-        bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb, ++kg) {
-          const int s = (int)(kg % S);
-          const uint32_t ph = (uint32_t)(kg / S) & 1u;
-          if (!wait_or_abort(&full_a[s], ph, s_abort) || !wait_or_abort(&full_t[s], ph, s_abort)) {
-            ok = false;
-            break;
-          }
-          ptx::tc_fence_after();
-          const uint32_t e_col = tmem + Cfg::meta_col(s);
-          ptx::tmem_cp_128x128b(
-              e_col, ptx::smem_desc_rows16(ptx::smem_u32(sP + s * Cfg::kPBytes + kBM * 16)));
-          const uint32_t a_addr = ptx::smem_u32(sA + s * Cfg::kABytes);
-          const uint32_t b_addr = ptx::smem_u32(sB + s * Cfg::kBBytes);
-#pragma unroll
-          for (int k = 0; k < 2; ++k)
-            ptx::mma_sp_i8(d_tmem, ptx::smem_desc_sw64(a_addr + 32 * k),
-                           ptx::smem_desc_sw128(b_addr + 64 * k), e_col + 2 * k, idesc,
-                           (kb | k) != 0);
-          ptx::mma_commit(&empty[s]);
-        }
-        if (!ok) break;
-        ptx::mma_commit(&acc_full[buf]);
-      }
-      // every MMA issued has completed before TMEM can be released (also after an abort)
-      ptx::mma_commit(mma_done);
-      if (!wait_phase(mma_done, 0)) *s_abort = 1;
-    }
-  } else {
-    // ---------------- epilogue (warps 6-9) ----------------
-    const int q = warp & 3;  // TMEM lane quadrant this warp may read
-    const int et = threadIdx.x - 6 * 32;  // 0..127
-    const float g = __ldg(gamma_eff);
-    bool failed = false;
-    int i = 0;
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
-      const int buf = i & 1;
-      const int64_t o0 = (tile % n_o) * kBM, t0 = (tile / n_o) * BN;
-      // all four warps are done with the previous tile's scales, and all of them stop
-      // together if any wait of the previous tile gave up
-      if (bar_any(1, 128, failed)) break;
-      for (int c = et; c < BN; c += 128) {
-        const int64_t t = t0 + c;
-        s_scale[c] = t < T ? rescale_factor(g, __ldg(absmax + t)) : 0.0f;
-      }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      failed = !__all_sync(0xffffffffu, !*s_abort && wait_or_abort(&acc_full[buf],
-                                                                   (uint32_t)(i >> 1) & 1u,
-                                                                   s_abort));
-      ptx::tc_fence_after();
-      if (!failed) {
-        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * Cfg::kAccStride);
-        store_tile<BN>(trow, s_scale, o0 + q * 32 + lane, O, t0, T, K <= 32768, Y, y_is_bf16,
-                       acc_dbg);
-      }
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&acc_empty[buf]);
-    }
-  }
-  ptx::tc_fence_before();
-  __syncthreads();
-  if (threadIdx.x == 0 && *s_abort && err_flag) atomicOr(err_flag, SBN_FLAG_TIMEOUT);
-  if (warp == 5) {
-    ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
-  }
-}
-
 // ---------------------------------------------------------------------------------------
 // CTA-pair 2:4 kernel for large token counts.  A cluster of two CTAs computes 256 weight
 // rows x BN tokens per tile with the pair form of the sparse MMA: each CTA stages, expands
@@ -873,7 +662,8 @@ __global__ void __launch_bounds__(kPsThreads, 1)
 // work and fits more stages.  CTA 0 of the pair issues the metadata copies, the MMAs and
 // the commits for both (commits reach the same barrier in both CTAs); the expanders and
 // the epilogue warps of both CTAs report to CTA 0's barriers.  Persistent over tiles with
-// two TMEM accumulators (columns 0 and 256) per CTA, as in k_gemm_sp24_persist.
+// two TMEM accumulators (columns 0 and 256) per CTA: the epilogue warps drain tile i while
+// the MMA already accumulates tile i+1.
 // ---------------------------------------------------------------------------------------
 template <int BN>
 struct PairCfg {
@@ -1276,37 +1066,19 @@ static sbn_status gemm_sp24_t(const int8_t *Xq, const float *absmax, const uint8
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, kern, tx, tc, tm, absmax, gamma_eff, T, O, K, Y, y_is_bf16,
-                           acc_dbg, err_flag) == cudaSuccess)
-      return SBN_OK;
-    (void)cudaGetLastError();  // the device rejected the cluster launch: one CTA per tile
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tx, tc, tm, absmax, gamma_eff, T, O, K,
+                                             Y, y_is_bf16, acc_dbg, err_flag);
+    if (e == cudaSuccess) return SBN_OK;
+    (void)cudaGetLastError();
+    // only a cluster the device cannot place falls back to one CTA per tile (same results);
+    // any other launch error is reported
+    if (e != cudaErrorInvalidClusterSize && e != cudaErrorLaunchOutOfResources &&
+        e != cudaErrorNotSupported)
+      return SBN_ERR_CUDA;
   }
   return launch_pdl(kern, dim3((unsigned)row_tiles, (unsigned)tok_tiles), dim3(kTcThreads),
                     Cfg::kSmem, st, tx, tc, tm, absmax, gamma_eff, T, O, K, Y, y_is_bf16, acc_dbg,
                     err_flag);
-}
-
-template <int BN>
-static sbn_status gemm_sp24_persist_t(const int8_t *Xq, const float *absmax, const uint8_t *codes,
-                                      const uint8_t *meta, const float *gamma_eff, int64_t T,
-                                      int64_t O, int64_t K, int64_t ldc, int64_t ldm, void *Y,
-                                      int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag,
-                                      cudaStream_t st) {
-  using Cfg = PsCfg<BN>;
-  CUtensorMap tx, tc, tm;
-  if (!encode_u8(&tx, Xq, K, T, K, Cfg::kKL, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_u8(&tc, codes, K / 8, O, ldc, 16, kBM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !encode_u8(&tm, meta, K / 8, O, ldm, 16, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return SBN_ERR_CUDA;
-  auto kern = k_gemm_sp24_persist<BN>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::kSmem) !=
-      cudaSuccess)
-    return SBN_ERR_CUDA;
-  const int64_t ntiles = ((O + kBM - 1) / kBM) * ((T + BN - 1) / BN);
-  int64_t grid = num_sms();
-  if (grid > ntiles) grid = ntiles;
-  return launch_pdl(kern, dim3((unsigned)grid), dim3(kPsThreads), Cfg::kSmem, st, tx, tc, tm,
-                    absmax, gamma_eff, T, O, K, Y, y_is_bf16, acc_dbg, err_flag);
 }
 
 template <int BN>
@@ -1388,14 +1160,9 @@ sbn_status launch_gemm_tc(const int8_t *Xq, const float *absmax, const uint8_t *
                           void *Y, int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag,
                           cudaStream_t st) {
   const bool compact = (n == 2 && m == 4);
-  if (compact && tokens > 128) {
-    // CTA pairs; the single-CTA persistent kernel if this device rejects the cluster launch
-    if (gemm_sp24_pair_t<224>(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc, ldm, Y,
-                              y_is_bf16, acc_dbg, err_flag, st) == SBN_OK)
-      return SBN_OK;
-    return gemm_sp24_persist_t<240>(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc, ldm,
-                                    Y, y_is_bf16, acc_dbg, err_flag, st);
-  }
+  if (compact && tokens > 128)  // CTA pairs (every sm_100 device runs 2-CTA clusters)
+    return gemm_sp24_pair_t<224>(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc, ldm, Y,
+                                 y_is_bf16, acc_dbg, err_flag, st);
   if (tokens > 128)
     return gemm_tc_bn<256>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc,
                            ldm, Y, y_is_bf16, acc_dbg, err_flag, st);

@@ -113,6 +113,14 @@ sbn_status launch_gemm_operand(const int8_t *Xq, const float *absmax, const void
                                int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag,
                                cudaStream_t st);
 
+// Dual-STE backward (backward.cu).
+int64_t backward_workspace_bytes(int64_t tokens, int64_t out, int64_t in);
+sbn_status launch_backward(const void *dY, const int8_t *Xq, const float *absmax,
+                           const uint8_t *codes, const uint8_t *meta, const void *W,
+                           const float *gamma_eff, int64_t T, int64_t O, int64_t K, int n, int m,
+                           int64_t ldc, int64_t ldm, float *dX, float *dW, void *workspace,
+                           int32_t *err_flag, cudaStream_t st);
+
 // Largest token count routed to the CUDA-core kernel; larger calls use the tensor cores.
 constexpr int64_t kGemvMaxTokens = 4;
 
