@@ -308,6 +308,20 @@ SBN_API sbn_status sbn_backward(const void *dY, const int8_t *Xq, const float *a
                                 int32_t *err_flag, void *stream);
 
 /*
+ * Steps 5-7 in one call: exactly sbn_quantize_acts followed by sbn_linear (every output bit,
+ * Xq and absmax included).  For tokens <= 4 and in <= 16384 (decode) it is ONE launch: each
+ * CTA of the GEMV quantises the few token rows into shared memory in its prologue (the
+ * activation quantiser's launch and its round trip through global memory leave the
+ * critical path); CTA 0 also writes Xq and absmax.  Otherwise the two launches of the
+ * separate calls.  Arguments as in those two calls; Xq and absmax are required outputs.
+ */
+SBN_API sbn_status sbn_quantize_linear(const void *X, const uint8_t *codes, const uint8_t *meta,
+                                       const float *gamma_eff, int64_t tokens, int64_t out,
+                                       int64_t in, int n, int m, int8_t *Xq, float *absmax,
+                                       void *Y, int y_is_bf16, int32_t *acc_dbg,
+                                       int32_t *err_flag, void *stream);
+
+/*
  * Mask statistics: by-products of steps 2-3 that follow how the masks evolve over training
  * steps (Sparse-BitNet summaries: section 3 "Contribuciones Clave" item 1, the large share
  * of ternary zeros; section 2, the mask recomputed every step from the current masters).

@@ -32,7 +32,7 @@ EXPORTED = ("sbn_linear_ref_dims", "sbn_quantize_mask_pack_weights", "sbn_quanti
             "sbn_count_zero_codes", "sbn_count_mask_flips", "sbn_group_plan_sizes",
             "sbn_group_plan", "sbn_quantize_acts_group", "sbn_linear_group",
             "sbn_operand_bytes", "sbn_expand_operand", "sbn_linear_operand",
-            "sbn_backward_workspace_bytes", "sbn_backward")
+            "sbn_backward_workspace_bytes", "sbn_backward", "sbn_quantize_linear")
 
 
 class SbnError(RuntimeError):
@@ -105,6 +105,9 @@ def lib():
         L.sbn_backward_workspace_bytes.restype = i32
         L.sbn_backward.argtypes = [p, p, p, p, p, p, p, i64, i64, i64, i32, i32, p, p, p, p, p]
         L.sbn_backward.restype = i32
+        L.sbn_quantize_linear.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, p, p, p, i32, p, p,
+                                          p]
+        L.sbn_quantize_linear.restype = i32
         L.sbn_status_string.argtypes = [i32]
         L.sbn_status_string.restype = ctypes.c_char_p
         _LIB = L
@@ -441,3 +444,28 @@ def backward(dY: torch.Tensor, Xq: torch.Tensor, s: torch.Tensor, w: PackedWeigh
     sbn_backward(dY, Xq, s, w.codes, w.meta, W, w.gamma_eff, w.out, w.in_, w.n, w.m, dX, dW, ws,
                  err_flag, stream)
     return dX, dW
+
+
+# ---- steps 5-7 in one call -------------------------------------------------------------------
+
+def sbn_quantize_linear(X, codes, meta, gamma_eff, out, in_, n, m, Xq, absmax, Y, acc_dbg=None,
+                        err_flag=None, stream=None):
+    if Y.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("Y must be float32 or bfloat16")
+    _check(lib().sbn_quantize_linear(_ptr(X), _ptr(codes), _ptr(meta), _ptr(gamma_eff),
+                                     X.shape[0], out, in_, n, m, _ptr(Xq), _ptr(absmax), _ptr(Y),
+                                     1 if Y.dtype == torch.bfloat16 else 0, _ptr(acc_dbg),
+                                     _ptr(err_flag), _stream(stream)), "sbn_quantize_linear")
+
+
+def quantize_linear(X: torch.Tensor, w: PackedWeights, out_dtype=torch.float32, acc_dbg=None,
+                    err_flag=None, stream=None):
+    """Steps 5-7 (activation quantiser + contraction) in one call; (Y, Xq, s)."""
+    T, K = X.shape
+    with _alloc_stream(stream):
+        Xq = torch.empty((T, K), dtype=torch.int8, device=X.device)
+        s = torch.empty((T,), dtype=torch.float32, device=X.device)
+        Y = torch.empty((T, w.out), dtype=out_dtype, device=X.device)
+    sbn_quantize_linear(X, w.codes, w.meta, w.gamma_eff, w.out, w.in_, w.n, w.m, Xq, s, Y, acc_dbg,
+                        err_flag, stream)
+    return Y, Xq, s

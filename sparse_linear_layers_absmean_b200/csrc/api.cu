@@ -262,6 +262,29 @@ sbn_status sbn_linear_group(const void *plan, const void *plan_dev, void *worksp
                                   static_cast<cudaStream_t>(stream));
 }
 
+sbn_status sbn_quantize_linear(const void *X, const uint8_t *codes, const uint8_t *meta,
+                               const float *gamma_eff, int64_t tokens, int64_t out, int64_t in,
+                               int n, int m, int8_t *Xq, float *absmax, void *Y, int y_is_bf16,
+                               int32_t *acc_dbg, int32_t *err_flag, void *stream) {
+  sbn_dims d;
+  sbn_status st = sbn_linear_ref_dims(out, in, n, m, &d);
+  if (st != SBN_OK) return st;
+  if (tokens < 0 || tokens > (1ll << 31) - 1) return SBN_ERR_SHAPE;
+  if (tokens == 0) return SBN_OK;
+  if (!X || !codes || !meta || !gamma_eff || !Xq || !absmax || !Y) return SBN_ERR_NULL;
+  if (!aligned16(X) || !aligned16(Xq) || !aligned16(codes) || !aligned16(meta) || !aligned16(Y) ||
+      (acc_dbg && !aligned16(acc_dbg)) || (reinterpret_cast<uintptr_t>(absmax) & 3u) ||
+      (reinterpret_cast<uintptr_t>(gamma_eff) & 3u) || (reinterpret_cast<uintptr_t>(err_flag) & 3u))
+    return SBN_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (tokens <= sbn::kGemvMaxTokens && in <= 16384)
+    return sbn::launch_gemv_fused(X, codes, meta, gamma_eff, tokens, out, in, n, m, d.codes_ld,
+                                  d.meta_ld, Y, y_is_bf16, Xq, absmax, acc_dbg, err_flag, s);
+  if ((st = sbn::launch_act_quant(X, tokens, in, Xq, absmax, err_flag, s)) != SBN_OK) return st;
+  return sbn_linear(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, n, m, Y, y_is_bf16,
+                    acc_dbg, err_flag, stream);
+}
+
 sbn_status sbn_count_zero_codes(const void *W, const float *gamma_eff, int64_t out, int64_t in,
                                 unsigned long long *count, void *stream) {
   sbn_dims d;

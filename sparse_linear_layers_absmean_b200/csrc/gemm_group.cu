@@ -10,7 +10,10 @@
 // units with about the same number of K blocks; the CTA walks its run as one pipeline in
 // super-blocks of four 128-deep K blocks (every hand-off between the roles has a fixed cost,
 // so each one moves four blocks):
-//   warp 4     TMA producer, ring 1 (the HBM stream, 6-9 slots): per super-block the packed
+//   warps 4, 15  two TMA producers on alternate super-blocks, each into its own half of ring 1
+//              (the HBM stream, 6-8 slots; the issue of a TMA copy, not the copy engine,
+//              limits one thread): per
+//              super-block the packed
 //              codes and the metadata of the unit's 128 rows as two boxes of 64 bytes x 128
 //              rows (64-byte swizzle), and the four activation tiles (bn tokens x 128 inputs,
 //              128-byte swizzle; L2 hits, all row tiles of a layer share them).
@@ -50,7 +53,7 @@ namespace sbn {
 
 namespace {
 
-constexpr int kGrpThreads = 480;  // 15 warps (two expander groups, two MMA threads)
+constexpr int kGrpThreads = 512;  // 16 warps (two expander groups, two TMA and two MMA threads)
 constexpr long long kGrpWaitCycles = 1ll << 31;  // about 1 s at 1.9 GHz
 constexpr int kSuper = 4;  // K blocks per weight super-block (one 64-byte box per row)
 
@@ -62,7 +65,7 @@ struct GrpCfg {
   static constexpr int kPlane = kGroupRows * 16 * kSuper;  // 8 KB
   static constexpr int kBBytes = BN * kGroupKB;
   static constexpr int kSlot1 = 2 * kPlane + kSuper * kBBytes;
-  static constexpr int kD1 = BN <= 16 ? 9 : 6;
+  static constexpr int kD1 = BN <= 16 ? 8 : 6;  // even: half the slots per producer
   // ring 2 in TMEM, one slot per super-block: per block the compressed A tile (lane r = row r,
   // 16 columns of four int8 values) and the metadata (4 columns)
   static constexpr int kD2 = BN <= 16 ? 4 : 2;
@@ -78,7 +81,11 @@ struct GrpCfg {
   static constexpr int kMColsPerSlot = kSuper * 4;
   static constexpr int kTmemCols = 512;
   static constexpr int kBars = 2 * kD1 + 2 * kD2 + 5;
-  static constexpr size_t kSmem = 1024 + (size_t)kD1 * kSlot1 + (size_t)kBars * 8 + 64;
+  // this CTA's unit records, staged in shared memory at the start (units past the first
+  // kUnitCache are read from global memory)
+  static constexpr int kUnitCache = 256;
+  static constexpr size_t kSmem = 1024 + (size_t)kD1 * kSlot1 + (size_t)kBars * 8 + 64 +
+                                  (size_t)kUnitCache * sizeof(GroupUnit);
   static_assert(kSlot1 % 1024 == 0 && kBBytes % 1024 == 0, "tile alignment");
   static_assert(kMetaCol + kD2 * kMColsPerSlot <= kTmemCols, "TMEM columns");
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
@@ -122,6 +129,18 @@ __device__ __forceinline__ bool grp_bar_any(bool pred) {
 
 __device__ __forceinline__ void grp_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// Ring 1 is filled by two producers, super-block js by producer js % 2 into its own half of
+// the slots (even / odd): no slot is ever shared between them, so each producer's copies and
+// phases stay its own.  H = D1 / 2 slots per producer.
+template <int D1>
+__device__ __forceinline__ int ring1_slot(int64_t js) {
+  return 2 * (int)((js >> 1) % (D1 / 2)) + (int)(js & 1);
+}
+template <int D1>
+__device__ __forceinline__ uint32_t ring1_phase(int64_t js) {
+  return (uint32_t)((js >> 1) / (D1 / 2)) & 1u;
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kGrpThreads, 1)
     k_gemm_group(const uint8_t *__restrict__ plan, uint8_t *__restrict__ ws,
@@ -142,6 +161,7 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
   volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_slot + 2);
   volatile int *s_last = reinterpret_cast<volatile int *>(tmem_slot + 4);
+  GroupUnit *s_units = reinterpret_cast<GroupUnit *>(tmem_slot + 16);  // 64 bytes past the slot
 
   ptx::grid_dep_launch();
   const GroupHeader &hd = *reinterpret_cast<const GroupHeader *>(plan);
@@ -150,6 +170,13 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
   const int32_t *cta_begin = reinterpret_cast<const int32_t *>(plan + hd.off_cta);
   const int u0 = cta_begin[blockIdx.x], u1 = cta_begin[blockIdx.x + 1];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the plan is written before the launch (not by the previous kernel): read it early
+  const int ncache = min(u1 - u0, Cfg::kUnitCache);
+  for (int i = threadIdx.x; i < ncache * 8; i += blockDim.x)
+    reinterpret_cast<int32_t *>(s_units)[i] = reinterpret_cast<const int32_t *>(units + u0)[i];
+  auto unit = [&](int u) -> GroupUnit {
+    return u - u0 < Cfg::kUnitCache ? s_units[u - u0] : units[u];
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < D1; ++s) {
@@ -188,14 +215,13 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
     int64_t js = 0;  // super-block counter over this CTA's units
     bool stop = false;
     for (int u = u0; u < u1 && !stop; ++u) {
-      const GroupUnit un = units[u];
-      const GroupProb &p = probs[un.prob];
-      const bool row_ok = (int64_t)un.row_tile * kGroupRows + r < p.O;
-      const int64_t K = p.K;
+      const GroupUnit un = unit(u);
+      const bool row_ok = un.row_tile * kGroupRows + r < un.O;
+      const int64_t K = un.K;
       for (int b0 = 0; b0 < un.nkb; b0 += kSuper, ++js) {
         if ((int)(js & 1) != grp) continue;
-        const int s1 = (int)(js % D1), s2 = (int)(js % D2);
-        const uint32_t ph1 = (uint32_t)(js / D1) & 1u, ph2 = (uint32_t)(js / D2) & 1u;
+        const int s1 = ring1_slot<D1>(js), s2 = (int)(js % D2);
+        const uint32_t ph1 = ring1_phase<D1>(js), ph2 = (uint32_t)(js / D2) & 1u;
         const bool ok = grp_wait(&full1[s1], ph1, s_abort) &&
                         (js < D2 || grp_wait(&empty2[s2], ph2 ^ 1u, s_abort));
         if (!__all_sync(0xffffffffu, ok)) {
@@ -239,14 +265,17 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
         if (lane == 0) ptx::mbar_arrive(&full2[s2]);
       }
     }
-  } else if (warp == 4) {
-    // ---------------- TMA producer (ring 1: packed weights + activation tiles) ----------------
+  } else if (warp == 4 || warp == 15) {
+    // ---------------- two TMA producers (ring 1: packed weights + activation tiles), taking
+    // alternate super-blocks: the issue of a TMA copy, not the copy engine, sets the pace of
+    // one thread ----------------
     if (lane == 0) {
-      int64_t js = 0, issued = 0;
+      const int pt = warp == 4 ? 0 : 1;  // super-blocks js with js % 2 == pt
+      int64_t js = 0, issued = -1;
       int last_prob = -1;
       for (int u = u0; u < u1 && !*s_abort; ++u) {
-        const GroupUnit un = units[u];
-        const GroupProb &p = probs[un.prob];
+        const GroupUnit un = unit(u);
+        const GroupProb &p = probs[un.prob];  // address only: the tensor maps stay in global memory
         if (un.prob != last_prob) {
           ptx::prefetch_tmap(&p.tc);
           ptx::prefetch_tmap(&p.tm);
@@ -256,8 +285,9 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
         const int32_t row0 = un.row_tile * kGroupRows;
         bool ok = true;
         for (int b0 = 0; b0 < un.nkb; b0 += kSuper, ++js) {
-          const int s1 = (int)(js % D1);
-          const uint32_t ph1 = (uint32_t)(js / D1) & 1u;
+          if ((int)(js & 1) != pt) continue;
+          const int s1 = ring1_slot<D1>(js);
+          const uint32_t ph1 = ring1_phase<D1>(js);
           if (js >= D1 && !grp_wait(&empty1[s1], ph1 ^ 1u, s_abort)) {
             ok = false;
             break;
@@ -271,13 +301,14 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
           for (int g = 0; g < nb; ++g)
             ptx::tma_load_2d(slot + 2 * Cfg::kPlane + g * Cfg::kBBytes, &p.tx, &full1[s1],
                              (kb + g) * kGroupKB, 0);
-          issued = js + 1;
+          issued = js;  // the last super-block this thread issued
         }
         if (!ok) break;
       }
-      // every issued copy lands before the CTA can exit (bounded, also after an abort)
-      for (int64_t q = issued - D1 < 0 ? 0 : issued - D1; q < issued; ++q)
-        if (!grp_drain(&full1[q % D1], (uint32_t)(q / D1) & 1u)) *s_abort = 1;
+      // every copy this thread issued lands before the CTA can exit (bounded, also after an
+      // abort): the last D1 / 2 super-blocks it issued, one per slot of its half
+      for (int64_t q = issued, i = 0; q >= 0 && i < D1 / 2; q -= 2, ++i)
+        if (!grp_drain(&full1[ring1_slot<D1>(q)], ring1_phase<D1>(q))) *s_abort = 1;
     }
   } else if (warp == 5 || warp == 14) {
     // ---------------- two sparse-MMA threads: alternate super-blocks ----------------
@@ -287,7 +318,7 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
       int64_t js = 0;
       int i = 0;
       for (int u = u0; u < u1 && !*s_abort; ++u, ++i) {
-        const int nkb = units[u].nkb;
+        const int nkb = unit(u).nkb;
         const int buf = i & 1;
         if (i >= 2 && !grp_wait(&acc_empty[buf], ((uint32_t)(i >> 1) & 1u) ^ 1u, s_abort))
           break;
@@ -296,8 +327,8 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
         bool ok = true;
         for (int b0 = 0; b0 < nkb; b0 += kSuper, ++js) {
           if (((b0 / kSuper) & 1) != mt) continue;  // by the unit's own super-block index
-          const int s1 = (int)(js % D1), s2 = (int)(js % D2);
-          const uint32_t ph1 = (uint32_t)(js / D1) & 1u, ph2 = (uint32_t)(js / D2) & 1u;
+          const int s1 = ring1_slot<D1>(js), s2 = (int)(js % D2);
+          const uint32_t ph1 = ring1_phase<D1>(js), ph2 = (uint32_t)(js / D2) & 1u;
           if (!grp_wait(&full2[s2], ph2, s_abort) || !grp_wait(&full1[s1], ph1, s_abort)) {
             ok = false;
             break;
@@ -339,7 +370,7 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
       const int buf = i & 1;
       // all four warps stop together if any wait of the previous unit gave up
       if (grp_bar_any(failed)) break;
-      const GroupUnit un = units[u];
+      const GroupUnit un = unit(u);
       const GroupProb &p = probs[un.prob];
       failed = !__all_sync(0xffffffffu, !*s_abort && grp_wait(&acc_full[buf],
                                                               (uint32_t)(i >> 1) & 1u, s_abort));
@@ -487,6 +518,8 @@ void build_units(const sbn_group_linear *lins, int count, int split,
         u.kb0 = (int)((int64_t)nkb * q / parts);
         u.nkb = (int)((int64_t)nkb * (q + 1) / parts) - u.kb0;
         u.part = q;
+        u.O = (int32_t)l.out;
+        u.K = (int32_t)l.in;
         units->push_back(u);
       }
   }

@@ -54,7 +54,9 @@ struct alignas(128) GroupProb {
 static_assert(sizeof(GroupProb) == 512, "plan layer record is 512 bytes");
 
 struct GroupUnit {
-  int32_t prob, row_tile, kb0, nkb, part, pad[3];
+  int32_t prob, row_tile, kb0, nkb, part;
+  int32_t O, K;  // the layer's shape (so a unit's pipeline needs no other record)
+  int32_t pad;
 };
 static_assert(sizeof(GroupUnit) == 32, "plan unit record is 32 bytes");
 

@@ -73,6 +73,13 @@ sbn_status launch_gemv(const int8_t *Xq, const float *absmax, const uint8_t *cod
                        int64_t out, int64_t in, int n, int m, int64_t ldc, int64_t ldm,
                        void *Y, int y_is_bf16, int32_t *acc_dbg, cudaStream_t st);
 
+// Steps 5-7 in one launch for at most kGemvMaxTokens tokens and in <= 16384 (gemv.cu).
+sbn_status launch_gemv_fused(const void *X, const uint8_t *codes, const uint8_t *meta,
+                             const float *gamma_eff, int64_t tokens, int64_t out, int64_t in,
+                             int n, int m, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
+                             int8_t *Xq, float *absmax, int32_t *acc_dbg, int32_t *err_flag,
+                             cudaStream_t st);
+
 // Tensor-core (tcgen05, int8) contraction.
 sbn_status launch_gemm_tc(const int8_t *Xq, const float *absmax, const uint8_t *codes,
                           const uint8_t *meta, const float *gamma_eff, int64_t tokens,
