@@ -623,8 +623,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // raises a shared abort flag that ends all loops.
 // ---------------------------------------------------------------------------------------
 
-constexpr int kPsThreads = 320;
-
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
@@ -696,8 +694,10 @@ struct PairCfg {
                                   (size_t)(3 * kStages + 5) * 8 + 32 + (size_t)BN * 4;
 };
 
+constexpr int kPairThreads = 352;  // 11 warps: expanders 0-3, producers 4 and 10, MMA 5, epilogue 6-9
+
 template <int BN>
-__global__ void __launch_bounds__(kPsThreads, 1)
+__global__ void __launch_bounds__(kPairThreads, 1)
     k_gemm_sp24_pair(const __grid_constant__ CUtensorMap tmap_x,
                      const __grid_constant__ CUtensorMap tmap_c,
                      const __grid_constant__ CUtensorMap tmap_m,
@@ -706,6 +706,7 @@ __global__ void __launch_bounds__(kPsThreads, 1)
                      int32_t *__restrict__ acc_dbg, int32_t *err_flag) {
   using Cfg = PairCfg<BN>;
   constexpr int S = Cfg::kStages, G = Cfg::kG, U = Cfg::kSub;
+  static_assert(S % 2 == 0, "two producers fill disjoint halves of the stages");
   constexpr int kTileM = 2 * kBM;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -784,13 +785,16 @@ __global__ void __launch_bounds__(kPsThreads, 1)
           const int kb = j * G + g;
           const uint4 cw = *reinterpret_cast<const uint4 *>(sP + u * Cfg::kPBytes + r * 16);
           const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+          // this row's metadata goes straight to its TMEM lane (the sparse MMA reads it
+          // there); groups outside the matrix get the valid index pair (0, 1)
+          uint4 m4 = *reinterpret_cast<const uint4 *>(sP + u * Cfg::kPBytes + kBM * 16 + r * 16);
           if (o0 + r >= O) {
-            *reinterpret_cast<uint4 *>(sP + u * Cfg::kPBytes + kBM * 16 + r * 16) =
-                make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+            m4 = make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
           } else if ((int64_t)kb * Cfg::kKL + 64 >= K) {
-            *reinterpret_cast<uint2 *>(sP + u * Cfg::kPBytes + kBM * 16 + r * 16 + 8) =
-                make_uint2(0x44444444u, 0x44444444u);
+            m4.z = 0x44444444u;
+            m4.w = 0x44444444u;
           }
+          ptx::tmem_st_4(tmem + ((uint32_t)(warp * 32) << 16) + Cfg::meta_col(u), m4);
           uint8_t *dst = sA + u * Cfg::kABytes + r * 64;
 #pragma unroll
           for (int c = 0; c < 4; ++c)
@@ -798,22 +802,27 @@ __global__ void __launch_bounds__(kPsThreads, 1)
                 make_uint4(w[c] & 0xC0C0C0C0u, (w[c] << 2) & 0xC0C0C0C0u,
                            (w[c] << 4) & 0xC0C0C0C0u, (w[c] << 6) & 0xC0C0C0C0u);
         }
+        ptx::tmem_st_wait();
         ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive_cluster(full_a0 + 8u * (uint32_t)s);
       }
     }
-  } else if (warp == 4) {
-    // ---------------- TMA producer (this CTA's rows and half of the tokens) ----------------
+  } else if (warp == 4 || warp == 10) {
+    // ---------------- two TMA producers (this CTA's rows and half of the tokens): stage kg
+    // by producer kg % 2; S is even, so each one fills its own half of the stages ----------
     if (lane == 0) {
+      const int pt = warp == 4 ? 0 : 1;
       ptx::prefetch_tmap(&tmap_x);
       ptx::prefetch_tmap(&tmap_c);
       ptx::prefetch_tmap(&tmap_m);
-      int64_t kg = 0, issued = 0;
+      int64_t kg = 0, issued = -1;
       for (int64_t tile = pair; tile < ntiles && !*s_abort; tile += npairs) {
         const int64_t o0 = (tile % n_o) * kTileM + (int64_t)rank * kBM;
         const int64_t t0 = (tile / n_o) * BN + (int64_t)rank * Cfg::kBHalf;
         for (int j = 0; j < nst; ++j, ++kg) {
+          if ((int)(kg & 1) != pt) continue;
           const int s = (int)(kg % S);
           const uint32_t ph = (uint32_t)(kg / S) & 1u;
           if (kg >= S && !wait_or_abort(&empty[s], ph ^ 1u, s_abort)) break;
@@ -828,10 +837,11 @@ __global__ void __launch_bounds__(kPsThreads, 1)
             ptx::tma_load_2d(p, &tmap_c, &full_t[s], kb * 16, (int32_t)o0);
             ptx::tma_load_2d(p + kBM * 16, &tmap_m, &full_t[s], kb * 16, (int32_t)o0);
           }
-          issued = kg + 1;
+          issued = kg;  // the last stage this thread issued
         }
       }
-      for (int64_t q = issued - S < 0 ? 0 : issued - S; q < issued; ++q)
+      // its last S / 2 stages, one per slot of its half, land before the CTA can exit
+      for (int64_t q = issued, i = 0; q >= 0 && i < S / 2; q -= 2, ++i)
         if (!wait_phase(&full_t[q % S], (uint32_t)(q / S) & 1u)) *s_abort = 1;
     }
   } else if (warp == 5) {
@@ -859,8 +869,7 @@ __global__ void __launch_bounds__(kPsThreads, 1)
           for (int g = 0; g < nb; ++g) {
             const int u = s * G + g;
             const uint32_t e_col = tmem + Cfg::meta_col(u);
-            ptx::tmem_cp_128x128b_pair(
-                e_col, ptx::smem_desc_rows16(ptx::smem_u32(sP + u * Cfg::kPBytes + kBM * 16)));
+            // (the metadata is already in both CTAs' TMEM, written by the expanders)
             const uint32_t a_addr = ptx::smem_u32(sA + u * Cfg::kABytes);
             const uint32_t b_addr = ptx::smem_u32(sB + u * Cfg::kBBytes);
 #pragma unroll
@@ -1105,7 +1114,7 @@ static sbn_status gemm_sp24_pair_t(const int8_t *Xq, const float *absmax, const 
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.blockDim = dim3(kPsThreads);
+  cfg.blockDim = dim3(kPairThreads);
   cfg.dynamicSmemBytes = Cfg::kSmem;
   cfg.stream = st;
   cfg.attrs = attr;

@@ -48,6 +48,13 @@ def _worker(rank, world, port, q):
         gamma_sharded = np.float32(float(t.item()) / (float(n) * 16777216.0))
         out["S"] = (int(t.item()), S_full)
         out["gamma"] = (float(gamma_sharded), float(gamma_full))
+        # the benchmark's per-rank workload: each rank runs one replica of the 32-layer stack
+        # on its own seeded tensors; the reductions of its timing go through dist
+        import bench
+        out["stack"] = bench.stack_layers(rank)
+        out["sum"] = sbn_dist.sum_over_ranks(float(rank + 1))
+        w, r, l = sbn_dist.init("gloo")  # already joined: returns the environment's view
+        out["init"] = (w, r, l)
         sbn_dist.barrier()
         q.put((rank, out))
     finally:
@@ -87,6 +94,17 @@ def test_row_sharded_gamma_is_exact(results):
         assert S_red == S_full
         g_sh, g_full = results[r]["gamma"]
         assert g_sh == g_full
+
+
+def test_bench_rank_replicas(results):
+    """Both ranks run the same 160 layer shapes (weak scaling: one stack replica per GPU) on
+    disjoint seeded tensors."""
+    a, b = results[0]["stack"], results[1]["stack"]
+    assert len(a) == len(b) == 160
+    assert [x[:4] for x in a] == [x[:4] for x in b]
+    assert not set(x[4] for x in a) & set(x[4] for x in b)
+    assert results[0]["sum"] == results[1]["sum"] == 3.0
+    assert results[0]["init"] == (2, 0, 0) and results[1]["init"] == (2, 1, 1)
 
 
 @pytest.mark.parametrize("n,world", [(0, 1), (1, 3), (7, 2), (130, 8), (5, 5)])
