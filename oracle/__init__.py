@@ -49,6 +49,15 @@ def load_library(path):
     lib.oracle_count_mask_flips.restype = i64
     lib.oracle_backward.argtypes = [p, p, p, p, p, ctypes.c_float, i64, i64, i64, p, p]
     lib.oracle_backward.restype = None
+    lib.oracle_group_gamma.argtypes = [p, i64, i64, ctypes.c_int, ctypes.c_float, p, p, p]
+    lib.oracle_group_gamma.restype = ctypes.c_int
+    lib.oracle_group_ternary_mask.argtypes = [p, i64, i64, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int, p, p, p, p]
+    lib.oracle_group_ternary_mask.restype = None
+    lib.oracle_group_quant_acts.argtypes = [p, i64, i64, ctypes.c_int, p, p]
+    lib.oracle_group_quant_acts.restype = ctypes.c_int
+    lib.oracle_group_contract_rescale.argtypes = [p, p, p, p, i64, i64, i64, ctypes.c_int, p, p]
+    lib.oracle_group_contract_rescale.restype = ctypes.c_int
     if not lib.oracle_rounding_is_nearest():
         raise RuntimeError("oracle needs round-to-nearest-even on the host FPU")
     return lib
@@ -217,3 +226,33 @@ def backward(dY, Xq, s, Ws, W_bits, g):
     _lib().oracle_backward(_ptr(dY), _ptr(Xq), _ptr(s), _ptr(Ws), _ptr(W_bits),
                            ctypes.c_float(float(g)), T, O, K, _ptr(dX), _ptr(dW))
     return dX, dW
+
+
+def group_linear(X_bits, W_bits, n: int, m: int, G: int, eps: float = 1e-5):
+    """Group-quantised forward (G blocks along K, each with its own weight scale g_j and
+    per-token activation scale s_tj); a dict with every intermediate and y (fp64)."""
+    W = np.ascontiguousarray(W_bits, np.uint16)
+    X = np.ascontiguousarray(X_bits, np.uint16)
+    O, K = W.shape
+    T = X.shape[0]
+    assert K % G == 0 and X.shape[1] == K
+    S = np.empty(G, np.uint64)
+    gamma = np.empty(G, np.float32)
+    g = np.empty(G, np.float32)
+    err = _lib().oracle_group_gamma(_ptr(W), O, K, G, ctypes.c_float(eps), _ptr(S), _ptr(gamma),
+                                    _ptr(g))
+    t = np.empty((O, K), np.int8)
+    keep = np.empty((O, K), np.uint8)
+    ws = np.empty((O, K), np.int8)
+    _lib().oracle_group_ternary_mask(_ptr(W), O, K, n, m, G, _ptr(g), _ptr(t), _ptr(keep), _ptr(ws))
+    codes, meta = pack(t, keep, n, m)
+    Xq = np.empty((T, K), np.int8)
+    s = np.empty((T, G), np.float32)
+    xerr = _lib().oracle_group_quant_acts(_ptr(X), T, K, G, _ptr(Xq), _ptr(s))
+    acc = np.empty((G, T, O), np.int32)
+    y = np.empty((T, O), np.float64)
+    if _lib().oracle_group_contract_rescale(_ptr(Xq), _ptr(ws), _ptr(s), _ptr(g), T, O, K, G,
+                                            _ptr(acc), _ptr(y)):
+        raise OverflowError("int32 accumulator overflow")
+    return dict(S=S, gamma=gamma, g=g, err=int(err), t=t, keep=keep, ws=ws, codes=codes,
+                meta=meta, Xq=Xq, s=s, xerr=int(xerr), acc=acc, y=y)

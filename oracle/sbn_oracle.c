@@ -350,3 +350,126 @@ void oracle_backward(const float *dY, const int8_t *Xq, const float *s, const in
       dW[o * K + k] = oracle_ste_pass(bf16_bits_to_float(W[o * K + k]), g) ? acc : 0.0;
     }
 }
+
+/*
+ * Group quantisation [bitnet.cpp article, "Cuantización y normalización de grupos": instead
+ * of one set of parameters for the whole weight matrix, weights and activations are split
+ * into G groups, each with its own parameters, so that groups need no communication].
+ * Reading: G equal blocks along the input dimension K (block j = inputs j*K/G ..
+ * (j+1)*K/G - 1, K/G a multiple of 64), for the weights and for every token's activations;
+ * each block is a Sparse-BitLinear of its own and the layer's output is their sum:
+ *   S_j   = sum over the block's weights of trunc(|W| * 2^24)    (exact, all rows)
+ *   g_j   = fp32( fp32( fp64(S_j) / (fp64(O * K / G) * 2^24) ) + eps )
+ *   t     = clamp(round(W / g_j), -1, 1) for W in block j      (fp32 divide, half-even)
+ *   mask  = the N:M rule on the master magnitudes (independent of the scales)
+ *   s_tj  = max(max over the block of |x_t|, 1e-5)
+ *   q     = clamp(round((127 x) / s_tj), -127, 127)
+ *   acc_j = sum over the block of q * ws                       (exact)
+ *   y     = sum_j acc_j * g_j * s_tj / 127                     (fp64, j ascending)
+ * With G == 1 this is the per-tensor layer above.  The functions below implement each
+ * step for all groups at once.
+ */
+int oracle_group_gamma(const uint16_t *W, int64_t O, int64_t K, int G, float eps,
+                       uint64_t *S_out, float *gamma_out, float *g_out) {
+  const int64_t kg = K / G;
+  int err = 0;
+  for (int j = 0; j < G; ++j) {
+    uint64_t S = 0;
+    for (int64_t r = 0; r < O; ++r)
+      for (int64_t k = j * kg; k < (j + 1) * kg; ++k) {
+        float a = fabsf(bf16_bits_to_float(W[r * K + k]));
+        if (!isfinite(a)) {
+          err |= ORACLE_ERR_W_NONFINITE;
+          continue;
+        }
+        if (a >= 256.0f) {
+          err |= ORACLE_ERR_W_RANGE;
+          continue;
+        }
+        S += (uint64_t)((double)a * 16777216.0); /* exact product, truncating conversion */
+      }
+    const float gamma = (float)((double)S / ((double)O * (double)kg * 16777216.0));
+    S_out[j] = S;
+    gamma_out[j] = gamma;
+    g_out[j] = gamma + eps;
+  }
+  return err;
+}
+
+/* Codes with the scale of each input's block, the N:M mask, and the masked codes. */
+void oracle_group_ternary_mask(const uint16_t *W, int64_t O, int64_t K, int N, int M, int G,
+                               const float *g, int8_t *t_out, uint8_t *keep_out,
+                               int8_t *ws_out) {
+  const int64_t kg = K / G;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < O; ++r) {
+    for (int64_t base = 0; base < K; base += M) {
+      for (int i = 0; i < M; ++i) {
+        const int64_t idx = r * K + base + i;
+        const float wi = bf16_bits_to_float(W[idx]);
+        int ahead = 0; /* group members ranked before position i */
+        for (int j = 0; j < M; ++j) {
+          const float mj = fabsf(bf16_bits_to_float(W[r * K + base + j]));
+          if (mj > fabsf(wi) || (mj == fabsf(wi) && j < i)) ++ahead;
+        }
+        const float q = wi / g[(base + i) / kg];
+        const float rq = rintf(q);
+        const int8_t t = rq >= 1.0f ? 1 : (rq <= -1.0f ? -1 : 0);
+        const uint8_t keep = (uint8_t)(ahead < N);
+        t_out[idx] = t;
+        keep_out[idx] = keep;
+        ws_out[idx] = (int8_t)(keep ? t : 0);
+      }
+    }
+  }
+}
+
+/* s[t * G + j] and Xq for every token and block.  Returns error bits. */
+int oracle_group_quant_acts(const uint16_t *X, int64_t T, int64_t K, int G, int8_t *Xq,
+                            float *s_out) {
+  const int64_t kg = K / G;
+  int err = 0;
+  for (int64_t t = 0; t < T; ++t)
+    for (int j = 0; j < G; ++j) {
+      float a = 0.0f;
+      for (int64_t k = j * kg; k < (j + 1) * kg; ++k) {
+        float v = fabsf(bf16_bits_to_float(X[t * K + k]));
+        if (!isfinite(v)) {
+          err |= ORACLE_ERR_X_NONFINITE;
+          continue;
+        }
+        a = v > a ? v : a;
+      }
+      const float s = a < 1e-5f ? 1e-5f : a;
+      s_out[t * G + j] = s;
+      for (int64_t k = j * kg; k < (j + 1) * kg; ++k) {
+        float r = rintf((127.0f * bf16_bits_to_float(X[t * K + k])) / s);
+        r = r > 127.0f ? 127.0f : (r < -127.0f ? -127.0f : r);
+        Xq[t * K + k] = (int8_t)(r != r ? 0.0f : r);
+      }
+    }
+  return err;
+}
+
+/* acc[(j * T + t) * O + o] = the block-j sum; y[t * O + o] = sum_j acc * g_j * s_tj / 127. */
+int oracle_group_contract_rescale(const int8_t *Xq, const int8_t *Ws, const float *s,
+                                  const float *g, int64_t T, int64_t O, int64_t K, int G,
+                                  int32_t *acc, double *y) {
+  const int64_t kg = K / G;
+  int err = 0;
+#pragma omp parallel for reduction(| : err) schedule(static)
+  for (int64_t o = 0; o < O; ++o)
+    for (int64_t t = 0; t < T; ++t) {
+      double yo = 0.0;
+      for (int j = 0; j < G; ++j) {
+        int64_t sum = 0;
+        for (int64_t k = j * kg; k < (j + 1) * kg; ++k)
+          sum += (int64_t)Xq[t * K + k] * (int64_t)Ws[o * K + k];
+        if (sum > INT32_MAX || sum < INT32_MIN) err |= ORACLE_ERR_ACC_OVERFLOW;
+        acc[(j * T + t) * O + o] = (int32_t)sum;
+        yo += (double)sum * (double)g[j] * (double)s[t * G + j] / 127.0;
+      }
+      y[t * O + o] = yo;
+    }
+  return err;
+}

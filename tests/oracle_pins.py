@@ -20,6 +20,10 @@ What pins what:
   mask_stats          natural-zero and mask-flip counts: hand-worked values (golden file),
                       a closed form, and the invariances of the mask (sign, power-of-two
                       scale, dense pattern)
+  group_one           group quantisation with G = 1 is the per-tensor layer (every output)
+  group_slices        G blocks: every block is the per-tensor layer on its K-slice (scales,
+                      codes, mask, activations, sums) and y is the sum of the blocks' outputs
+  group_hand          G = 2 on a hand-worked row (golden file)
   backward_hand       dual-STE backward on the hand-worked example (golden file): pruned
                       positions still receive their weight gradient, clipped ones none
   backward_adjoint    <dY, y> = <dX, X_eff> against the forward's y; <dW, V> = <dY,
@@ -406,6 +410,67 @@ def backward_adjoint(o):
             assert dWb[0, 60] == 0.0 and np.all(np.delete(dWb[0], 60) == np.delete(full, 60))
 
 
+def group_one(o):
+    W = _tie_heavy_masters(12, 192, seed=31)
+    X = workloads.activations(5, 192, seed=32)
+    for (n, m) in [(2, 4), (6, 8), (3, 8)]:
+        r1, r = o.group_linear(X, W, n, m, 1), o.linear(X, W, n, m)
+        assert float(r1["g"][0]) == float(r["g"]) and int(r1["S"][0]) == int(r["S"])
+        for k in ("t", "keep", "ws", "codes", "meta", "Xq"):
+            assert np.array_equal(r1[k], r[k]), k
+        assert np.array_equal(r1["s"][:, 0], r["s"])
+        assert np.array_equal(r1["acc"][0], r["acc"]) and np.array_equal(r1["y"], r["y"])
+
+
+def group_slices(o):
+    rng = np.random.default_rng(33)
+    O, K, T = 9, 256, 4
+    W = workloads.masters(O, K, seed=34)
+    X = workloads.activations(T, K, seed=35)
+    # make the blocks' scales differ a lot: scale block 2 of W and block 1 of X by 4
+    Wf = workloads.bf16_bits_to_f32(W)
+    Wf[:, 128:192] *= 4.0
+    W = workloads.to_bf16_bits(Wf)
+    Xf = workloads.bf16_bits_to_f32(X)
+    Xf[:, 64:128] *= 4.0
+    X = workloads.to_bf16_bits(Xf)
+    for (n, m, G) in [(2, 4, 4), (6, 8, 2), (1, 4, 4)]:
+        r = o.group_linear(X, W, n, m, G)
+        kg = K // G
+        y = np.zeros((T, O))
+        for j in range(G):
+            sl = slice(j * kg, (j + 1) * kg)
+            rj = o.linear(np.ascontiguousarray(X[:, sl]), np.ascontiguousarray(W[:, sl]), n, m)
+            assert float(r["g"][j]) == float(rj["g"]) and int(r["S"][j]) == int(rj["S"])
+            for k in ("t", "keep", "ws", "Xq"):
+                assert np.array_equal(r[k][:, sl], rj[k]), (G, j, k)
+            assert np.array_equal(r["s"][:, j], rj["s"])
+            assert np.array_equal(r["acc"][j], rj["acc"])
+            y = y + rj["y"]
+        assert np.array_equal(r["y"], y)
+    assert rng is not None
+
+
+def group_hand(o):
+    g = _read_golden("group_example_g2.txt")
+    G, n, m = int(g["G"][0]), int(g["n"][0]), int(g["m"][0])
+    W0 = np.array([float(v) for v in g["W0"]] * 8, np.float32)
+    x0 = np.array([float(v) for v in g["x0"]] * 8, np.float32)
+    W = workloads.to_bf16_bits(np.concatenate([W0, 2 * W0])[None, :])
+    X = workloads.to_bf16_bits(np.concatenate([x0, x0 / 2])[None, :])
+    r = o.group_linear(X, W, n, m, G, eps=float(g["eps"][0]))
+    assert [float(v) for v in r["gamma"]] == [float(v) for v in g["gamma"]]
+    ws = np.array([int(v) for v in g["ws"]] * 16, np.int8)
+    assert np.array_equal(r["ws"][0], ws)
+    assert [float(v) for v in r["s"][0]] == [float(v) for v in g["s"]]
+    assert [int(v) for v in r["acc"][:, 0, 0]] == [int(v) for v in g["acc"]]
+    y_ref = Fraction(g["y_num"][0]) / int(g["y_den"][0])
+    assert abs(Fraction(float(r["y"][0, 0])) - y_ref) <= abs(y_ref) * Fraction(1, 2 ** 50)
+    r1 = o.group_linear(X, W, n, m, 1, eps=float(g["eps"][0]))
+    assert float(r1["gamma"][0]) == float(g["gamma_g1"][0]) and r1["t"][0, 1] == 0
+
+
 ALL = [hand_example, mask_bruteforce, gamma_closed_form, rounding_ties, dense_pattern,
        constant_magnitude, act_absmax, contract_bruteforce, unpack_roundtrip, invariants,
-       scale_invariance, rescale_closed_form, mask_stats, backward_hand, backward_adjoint]
+       scale_invariance, rescale_closed_form, mask_stats, group_one, group_slices, group_hand,
+       backward_hand, backward_adjoint]

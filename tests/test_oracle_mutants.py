@@ -54,6 +54,13 @@ MUTANTS = [
      "dW[o * K + k] = acc;"),
     ("backward_gate_round_range", "return fabsf(w) / g <= 1.0f;", "return fabsf(w) / g < 1.5f;"),
     ("backward_gate_strict", "return fabsf(w) / g <= 1.0f;", "return fabsf(w) / g < 1.0f;"),
+    ("group_codes_one_scale", "const float q = wi / g[(base + i) / kg];", "const float q = wi / g[0];"),
+    ("group_gamma_whole_row_count", "((double)O * (double)kg * 16777216.0)",
+     "((double)O * (double)K * 16777216.0)"),
+    ("group_rescale_first_scale", "(double)g[j] * (double)s[t * G + j] / 127.0",
+     "(double)g[j] * (double)s[t * G] / 127.0"),
+    ("group_acts_row_absmax", "for (int64_t k = j * kg; k < (j + 1) * kg; ++k) {\n        float v = fabsf",
+     "for (int64_t k = 0; k < K; ++k) {\n        float v = fabsf"),
     ("backward_gate_by_mask",
      "dW[o * K + k] = oracle_ste_pass(bf16_bits_to_float(W[o * K + k]), g) ? acc : 0.0;",
      "dW[o * K + k] = Ws[o * K + k] != 0 ? acc : 0.0;"),
