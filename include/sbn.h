@@ -322,6 +322,46 @@ SBN_API sbn_status sbn_quantize_linear(const void *X, const uint8_t *codes, cons
                                        int32_t *err_flag, void *stream);
 
 /*
+ * Group quantisation ("Marco de inferencia de Microsoft lleva modelos de lenguaje grande de
+ * 1 bit a dispositivos locales", unite.ai, "Cuantización y normalización de grupos": weights
+ * and activations split into G groups with parameters of their own, so that the groups need
+ * no communication).  Here: G equal blocks along the input dimension; block j (inputs
+ * j*in/G .. (j+1)*in/G - 1) is a Sparse-BitLinear of its own and the layer's output is the sum
+ * of the blocks' outputs:
+ *   g_j   = fp32(fp32(fp64(S_j) / (fp64(out * in / G) * 2^24)) + eps), S_j the exact sum of
+ *           trunc(|W| * 2^24) over the block's weights (all rows)
+ *   codes = clamp(round(W / g_j)) in block j; the N:M mask as in the per-tensor calls
+ *   s_tj  = max(max |x_t| over block j, 1e-5); Xq by s_tj
+ *   y[t,o]= sum_j fp32(acc_j[t,o] * c_tj), c_tj = fp32(fp32(g_j * s_tj) / 127), added in fp32
+ *           in ascending j (acc_j the exact int32 sum over block j)
+ * groups = 1 gives the per-tensor layer.  Shapes: 1 <= groups <= 64, in % groups == 0 and
+ * (in / groups) % 128 == 0; the other rules and the packed planes are those of the per-tensor
+ * calls (sbn_linear_ref_dims).  Scales: gamma_eff holds groups floats; absmax holds
+ * groups * tokens floats, group-major (absmax[j * tokens + t]).
+ */
+/* Host only: *workspace_bytes = the contraction's scratch (groups * tokens * out fp32). */
+SBN_API sbn_status sbn_gq_workspace_bytes(int64_t tokens, int64_t out, int64_t in, int groups,
+                                          int64_t *workspace_bytes);
+/* Steps 1-4 with per-group scales; workspace as for sbn_quantize_mask_pack_weights. */
+SBN_API sbn_status sbn_quantize_mask_pack_weights_gq(const void *W, int64_t out, int64_t in,
+                                                     int n, int m, int groups, float eps,
+                                                     uint8_t *codes, uint8_t *meta,
+                                                     float *gamma_eff, void *workspace,
+                                                     int8_t *dense_dbg, int32_t *err_flag,
+                                                     void *stream);
+/* Step 5 with per-(token, group) scales. */
+SBN_API sbn_status sbn_quantize_acts_gq(const void *X, int64_t tokens, int64_t in, int groups,
+                                        int8_t *Xq, float *absmax, int32_t *err_flag,
+                                        void *stream);
+/* Steps 6-7: each block on the contraction kernels of sbn_linear, then the ordered sum.
+ * acc_dbg (optional) is int32 [groups][tokens][out]: the blocks' exact sums. */
+SBN_API sbn_status sbn_linear_gq(const int8_t *Xq, const float *absmax, const uint8_t *codes,
+                                 const uint8_t *meta, const float *gamma_eff, int64_t tokens,
+                                 int64_t out, int64_t in, int n, int m, int groups, void *Y,
+                                 int y_is_bf16, void *workspace, int32_t *acc_dbg,
+                                 int32_t *err_flag, void *stream);
+
+/*
  * Mask statistics: by-products of steps 2-3 that follow how the masks evolve over training
  * steps (Sparse-BitNet summaries: section 3 "Contribuciones Clave" item 1, the large share
  * of ternary zeros; section 2, the mask recomputed every step from the current masters).

@@ -32,7 +32,9 @@ EXPORTED = ("sbn_linear_ref_dims", "sbn_quantize_mask_pack_weights", "sbn_quanti
             "sbn_count_zero_codes", "sbn_count_mask_flips", "sbn_group_plan_sizes",
             "sbn_group_plan", "sbn_quantize_acts_group", "sbn_linear_group",
             "sbn_operand_bytes", "sbn_expand_operand", "sbn_linear_operand",
-            "sbn_backward_workspace_bytes", "sbn_backward", "sbn_quantize_linear")
+            "sbn_backward_workspace_bytes", "sbn_backward", "sbn_quantize_linear",
+            "sbn_gq_workspace_bytes", "sbn_quantize_mask_pack_weights_gq", "sbn_quantize_acts_gq",
+            "sbn_linear_gq")
 
 
 class SbnError(RuntimeError):
@@ -108,6 +110,15 @@ def lib():
         L.sbn_quantize_linear.argtypes = [p, p, p, p, i64, i64, i64, i32, i32, p, p, p, i32, p, p,
                                           p]
         L.sbn_quantize_linear.restype = i32
+        L.sbn_gq_workspace_bytes.argtypes = [i64, i64, i64, i32, p]
+        L.sbn_gq_workspace_bytes.restype = i32
+        L.sbn_quantize_mask_pack_weights_gq.argtypes = [p, i64, i64, i32, i32, i32, ctypes.c_float,
+                                                        p, p, p, p, p, p, p]
+        L.sbn_quantize_mask_pack_weights_gq.restype = i32
+        L.sbn_quantize_acts_gq.argtypes = [p, i64, i64, i32, p, p, p, p]
+        L.sbn_quantize_acts_gq.restype = i32
+        L.sbn_linear_gq.argtypes = [p, p, p, p, p, i64, i64, i64, i32, i32, i32, p, i32, p, p, p, p]
+        L.sbn_linear_gq.restype = i32
         L.sbn_status_string.argtypes = [i32]
         L.sbn_status_string.restype = ctypes.c_char_p
         _LIB = L
@@ -469,3 +480,58 @@ def quantize_linear(X: torch.Tensor, w: PackedWeights, out_dtype=torch.float32, 
     sbn_quantize_linear(X, w.codes, w.meta, w.gamma_eff, w.out, w.in_, w.n, w.m, Xq, s, Y, acc_dbg,
                         err_flag, stream)
     return Y, Xq, s
+
+
+# ---- group quantisation (G blocks along K) ---------------------------------------------------
+
+class GqPackedWeights(NamedTuple):
+    codes: torch.Tensor      # uint8 [out, codes_ld]
+    meta: torch.Tensor       # uint8 [out, meta_ld]
+    gamma_eff: torch.Tensor  # fp32 [groups]
+    out: int
+    in_: int
+    n: int
+    m: int
+    groups: int
+
+
+def pack_weights_gq(W, n, m, groups, eps=1e-5, dense_dbg=None, err_flag=None, stream=None):
+    out, in_ = W.shape
+    d = sbn_linear_ref_dims(out, in_, n, m)
+    with _alloc_stream(stream):
+        codes = torch.empty((out, d.codes_ld), dtype=torch.uint8, device=W.device)
+        meta = torch.empty((out, d.meta_ld), dtype=torch.uint8, device=W.device)
+        gamma = torch.empty(groups, dtype=torch.float32, device=W.device)
+        ws = new_workspace(out, in_, n, m, W.device)
+    _check(lib().sbn_quantize_mask_pack_weights_gq(
+        _ptr(W), out, in_, n, m, groups, ctypes.c_float(eps), _ptr(codes), _ptr(meta), _ptr(gamma),
+        _ptr(ws), _ptr(dense_dbg), _ptr(err_flag), _stream(stream)),
+        "sbn_quantize_mask_pack_weights_gq")
+    return GqPackedWeights(codes, meta, gamma, out, in_, n, m, groups)
+
+
+def quantize_acts_gq(X, groups, err_flag=None, stream=None):
+    """(Xq int8 [T, K], s fp32 [groups, T])."""
+    T, K = X.shape
+    with _alloc_stream(stream):
+        Xq = torch.empty((T, K), dtype=torch.int8, device=X.device)
+        s = torch.empty((groups, T), dtype=torch.float32, device=X.device)
+    _check(lib().sbn_quantize_acts_gq(_ptr(X), T, K, groups, _ptr(Xq), _ptr(s), _ptr(err_flag),
+                                      _stream(stream)), "sbn_quantize_acts_gq")
+    return Xq, s
+
+
+def linear_gq(Xq, s, w: GqPackedWeights, out_dtype=torch.float32, acc_dbg=None, err_flag=None,
+              stream=None):
+    T = Xq.shape[0]
+    b = ctypes.c_int64()
+    _check(lib().sbn_gq_workspace_bytes(T, w.out, w.in_, w.groups, ctypes.byref(b)),
+           "sbn_gq_workspace_bytes")
+    with _alloc_stream(stream):
+        Y = torch.empty((T, w.out), dtype=out_dtype, device=Xq.device)
+        ws = torch.empty(max(b.value, 16), dtype=torch.uint8, device=Xq.device)
+    _check(lib().sbn_linear_gq(_ptr(Xq), _ptr(s), _ptr(w.codes), _ptr(w.meta), _ptr(w.gamma_eff), T,
+                               w.out, w.in_, w.n, w.m, w.groups, _ptr(Y),
+                               1 if out_dtype == torch.bfloat16 else 0, _ptr(ws), _ptr(acc_dbg),
+                               _ptr(err_flag), _stream(stream)), "sbn_linear_gq")
+    return Y

@@ -9,7 +9,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsbn.so")
 SOURCES = ["api.cu", "pack.cu", "pack_fast.cu", "pack_noalloc.cu", "act_quant.cu", "gemv.cu", "gemm_tc.cu",
-           "gemm_group.cu", "gemm_operand.cu", "backward.cu", "stats.cu"]
+           "gemm_group.cu", "gemm_operand.cu", "backward.cu", "group_quant.cu", "stats.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

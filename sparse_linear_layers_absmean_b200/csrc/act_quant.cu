@@ -128,6 +128,55 @@ __global__ void __launch_bounds__(kAqThreads)
   }
 }
 
+// Group quantisation: one CTA per (token t, group j) of G blocks along K; s is stored
+// group-major, s[j * tokens + t], so that each group's scales are contiguous.  R > 0 keeps the
+// block in registers (blocks of up to 8 * 256 * R inputs); R == 0 reads it twice.
+template <int R>
+__global__ void __launch_bounds__(kAqThreads)
+    k_act_quant_gq(const uint4 *__restrict__ X, int64_t tokens, int64_t K, int G,
+                   int8_t *__restrict__ Xq, float *__restrict__ absmax, int32_t *err_flag) {
+  ptx::grid_dep_launch();
+  ptx::grid_dep_wait();
+  const int64_t t = blockIdx.x, j = blockIdx.y, kg = K / G, nv = kg / 8;
+  const uint4 *row = X + (t * K + j * kg) / 8;
+  uint2 *qrow = reinterpret_cast<uint2 *>(Xq + t * K + j * kg);
+  if constexpr (R > 0) {
+    uint4 v[R];
+    uint32_t mx = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t i = threadIdx.x + (int64_t)r * kAqThreads;
+      v[r] = i < nv ? __ldg(row + i) : make_uint4(0u, 0u, 0u, 0u);
+      mx = vec8_absmax_bits(v[r], mx);
+    }
+    const float s = block_scale(mx, err_flag);
+    if (threadIdx.x == 0) absmax[j * tokens + t] = s;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int64_t i = threadIdx.x + (int64_t)r * kAqThreads;
+      if (i < nv) qrow[i] = quant_vec8(v[r], s);
+    }
+  } else {
+    uint32_t mx = 0;
+    for (int64_t i = threadIdx.x; i < nv; i += kAqThreads) mx = vec8_absmax_bits(__ldg(row + i), mx);
+    const float s = block_scale(mx, err_flag);
+    if (threadIdx.x == 0) absmax[j * tokens + t] = s;
+    for (int64_t i = threadIdx.x; i < nv; i += kAqThreads) qrow[i] = quant_vec8(__ldg(row + i), s);
+  }
+}
+
+sbn_status launch_act_quant_gq(const void *X, int64_t tokens, int64_t in, int G, int8_t *Xq,
+                               float *absmax, int32_t *err_flag, cudaStream_t st) {
+  const int64_t nv = in / G / 8;
+  const uint4 *X4 = reinterpret_cast<const uint4 *>(X);
+  const dim3 grid((unsigned)tokens, (unsigned)G), block(kAqThreads);
+  if (nv <= 2 * kAqThreads)
+    return launch_pdl(k_act_quant_gq<2>, grid, block, 0, st, X4, tokens, in, G, Xq, absmax, err_flag);
+  if (nv <= 8 * kAqThreads)
+    return launch_pdl(k_act_quant_gq<8>, grid, block, 0, st, X4, tokens, in, G, Xq, absmax, err_flag);
+  return launch_pdl(k_act_quant_gq<0>, grid, block, 0, st, X4, tokens, in, G, Xq, absmax, err_flag);
+}
+
 // Grouped form: one CTA per (layer, token) row of a group plan.  R > 0 keeps the row in
 // registers (rows of up to 8 * 256 * R inputs); R == 0 reads it twice.
 template <int R>

@@ -59,6 +59,12 @@ sbn_status check_group(const sbn_group_linear *lins, int32_t count) {
   return SBN_OK;
 }
 
+sbn_status check_groups(int64_t in, int groups) {
+  if (groups < 1 || groups > 64 || in % groups != 0 || (in / groups) % 128 != 0)
+    return SBN_ERR_SHAPE;
+  return SBN_OK;
+}
+
 sbn_status check_plan(const void *plan, const void *plan_dev) {
   if (!plan || !plan_dev) return SBN_ERR_NULL;
   if ((reinterpret_cast<uintptr_t>(plan) & 127u) || (reinterpret_cast<uintptr_t>(plan_dev) & 127u))
@@ -145,9 +151,9 @@ sbn_status sbn_linear(const int8_t *Xq, const float *absmax, const uint8_t *code
     return SBN_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (tokens <= sbn::kGemvMaxTokens)
-    return sbn::launch_gemv(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, n, m, d.codes_ld,
+    return sbn::launch_gemv(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, in, n, m, d.codes_ld,
                             d.meta_ld, Y, y_is_bf16, acc_dbg, s);
-  return sbn::launch_gemm_tc(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, n, m,
+  return sbn::launch_gemm_tc(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, in, n, m,
                              d.codes_ld, d.meta_ld, Y, y_is_bf16, acc_dbg, err_flag, s);
 }
 
@@ -283,6 +289,75 @@ sbn_status sbn_quantize_linear(const void *X, const uint8_t *codes, const uint8_
   if ((st = sbn::launch_act_quant(X, tokens, in, Xq, absmax, err_flag, s)) != SBN_OK) return st;
   return sbn_linear(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, n, m, Y, y_is_bf16,
                     acc_dbg, err_flag, stream);
+}
+
+sbn_status sbn_gq_workspace_bytes(int64_t tokens, int64_t out, int64_t in, int groups,
+                                  int64_t *workspace_bytes) {
+  if (!workspace_bytes) return SBN_ERR_NULL;
+  sbn_dims d;
+  sbn_status st = sbn_linear_ref_dims(out, in, 2, 4, &d);
+  if (st != SBN_OK) return st;
+  if ((st = check_groups(in, groups)) != SBN_OK) return st;
+  if (tokens < 0 || tokens > (1ll << 31) - 1) return SBN_ERR_SHAPE;
+  *workspace_bytes = (int64_t)groups * tokens * out * 4;
+  return SBN_OK;
+}
+
+sbn_status sbn_quantize_mask_pack_weights_gq(const void *W, int64_t out, int64_t in, int n, int m,
+                                             int groups, float eps, uint8_t *codes, uint8_t *meta,
+                                             float *gamma_eff, void *workspace, int8_t *dense_dbg,
+                                             int32_t *err_flag, void *stream) {
+  sbn_dims d;
+  sbn_status st = sbn_linear_ref_dims(out, in, n, m, &d);
+  if (st != SBN_OK) return st;
+  if ((st = check_groups(in, groups)) != SBN_OK) return st;
+  if (!W || !codes || !meta || !gamma_eff || !workspace) return SBN_ERR_NULL;
+  if (!std::isfinite(eps) || eps < 0.0f) return SBN_ERR_ARG;
+  if (!aligned16(W) || !aligned16(codes) || !aligned16(meta) || !aligned16(workspace) ||
+      (dense_dbg && !aligned16(dense_dbg)) || (reinterpret_cast<uintptr_t>(gamma_eff) & 3u) ||
+      (reinterpret_cast<uintptr_t>(err_flag) & 3u))
+    return SBN_ERR_ALIGN;
+  return sbn::launch_pack_gq(W, out, in, n, m, groups, eps, codes, d.codes_ld, d.codes_row_bytes,
+                             meta, d.meta_ld, d.meta_row_bytes, gamma_eff,
+                             static_cast<sbn::PackWorkspace *>(workspace), dense_dbg, err_flag,
+                             static_cast<cudaStream_t>(stream));
+}
+
+sbn_status sbn_quantize_acts_gq(const void *X, int64_t tokens, int64_t in, int groups, int8_t *Xq,
+                                float *absmax, int32_t *err_flag, void *stream) {
+  sbn_status st = check_in(in);
+  if (st != SBN_OK) return st;
+  if ((st = check_groups(in, groups)) != SBN_OK) return st;
+  if (tokens < 0 || tokens > (1ll << 31) - 1) return SBN_ERR_SHAPE;
+  if (tokens == 0) return SBN_OK;
+  if (!X || !Xq || !absmax) return SBN_ERR_NULL;
+  if (!aligned16(X) || !aligned16(Xq) || (reinterpret_cast<uintptr_t>(absmax) & 3u) ||
+      (reinterpret_cast<uintptr_t>(err_flag) & 3u))
+    return SBN_ERR_ALIGN;
+  return sbn::launch_act_quant_gq(X, tokens, in, groups, Xq, absmax, err_flag,
+                                  static_cast<cudaStream_t>(stream));
+}
+
+sbn_status sbn_linear_gq(const int8_t *Xq, const float *absmax, const uint8_t *codes,
+                         const uint8_t *meta, const float *gamma_eff, int64_t tokens, int64_t out,
+                         int64_t in, int n, int m, int groups, void *Y, int y_is_bf16,
+                         void *workspace, int32_t *acc_dbg, int32_t *err_flag, void *stream) {
+  sbn_dims d;
+  sbn_status st = sbn_linear_ref_dims(out, in, n, m, &d);
+  if (st != SBN_OK) return st;
+  if ((st = check_groups(in, groups)) != SBN_OK) return st;
+  if (tokens < 0 || tokens > (1ll << 31) - 1) return SBN_ERR_SHAPE;
+  if (tokens == 0) return SBN_OK;
+  if (!Xq || !absmax || !codes || !meta || !gamma_eff || !Y || !workspace) return SBN_ERR_NULL;
+  if (!aligned16(Xq) || !aligned16(codes) || !aligned16(meta) || !aligned16(Y) ||
+      !aligned16(workspace) || (acc_dbg && !aligned16(acc_dbg)) ||
+      (reinterpret_cast<uintptr_t>(absmax) & 3u) || (reinterpret_cast<uintptr_t>(gamma_eff) & 3u) ||
+      (reinterpret_cast<uintptr_t>(err_flag) & 3u))
+    return SBN_ERR_ALIGN;
+  return sbn::launch_linear_gq(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, n, m, groups,
+                               d.codes_ld, d.meta_ld, Y, y_is_bf16,
+                               static_cast<float *>(workspace), acc_dbg, err_flag,
+                               static_cast<cudaStream_t>(stream));
 }
 
 sbn_status sbn_count_zero_codes(const void *W, const float *gamma_eff, int64_t out, int64_t in,

@@ -1024,12 +1024,12 @@ static int sp24_split(Kern kern, int64_t tiles, int nkb) {
 template <int BN, bool kCompact>
 static sbn_status gemm_tc_t(const int8_t *Xq, const float *absmax, const uint8_t *codes,
                             const uint8_t *meta, const float *gamma_eff, int64_t T, int64_t O,
-                            int64_t K, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
+                            int64_t K, int64_t ldx, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
                             int32_t *acc_dbg, int32_t *err_flag, cudaStream_t st) {
   using Cfg = TcCfg<BN, kCompact>;
   CUtensorMap tx, tc, tm;
   const int64_t crow = kCompact ? K / 8 : K / 4;  // data bytes of a codes row
-  if (!encode_u8(&tx, Xq, K, T, K, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  if (!encode_u8(&tx, Xq, K, T, ldx, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_u8(&tc, codes, crow, O, ldc, Cfg::kPackRow, kBM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !encode_u8(&tm, meta, K / 8, O, ldm, 16, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
     return SBN_ERR_CUDA;
@@ -1045,11 +1045,11 @@ static sbn_status gemm_tc_t(const int8_t *Xq, const float *absmax, const uint8_t
 template <int BN>
 static sbn_status gemm_sp24_t(const int8_t *Xq, const float *absmax, const uint8_t *codes,
                               const uint8_t *meta, const float *gamma_eff, int64_t T, int64_t O,
-                              int64_t K, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
+                              int64_t K, int64_t ldx, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
                               int32_t *acc_dbg, int32_t *err_flag, cudaStream_t st) {
   using Cfg = SpCfg<BN>;
   CUtensorMap tx, tc, tm;
-  if (!encode_u8(&tx, Xq, K, T, K, Cfg::kKL, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  if (!encode_u8(&tx, Xq, K, T, ldx, Cfg::kKL, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_u8(&tc, codes, K / 8, O, ldc, 16, kBM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !encode_u8(&tm, meta, K / 8, O, ldm, 16, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
     return SBN_ERR_CUDA;
@@ -1093,12 +1093,12 @@ static sbn_status gemm_sp24_t(const int8_t *Xq, const float *absmax, const uint8
 template <int BN>
 static sbn_status gemm_sp24_pair_t(const int8_t *Xq, const float *absmax, const uint8_t *codes,
                                    const uint8_t *meta, const float *gamma_eff, int64_t T,
-                                   int64_t O, int64_t K, int64_t ldc, int64_t ldm, void *Y,
+                                   int64_t O, int64_t K, int64_t ldx, int64_t ldc, int64_t ldm, void *Y,
                                    int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag,
                                    cudaStream_t st) {
   using Cfg = PairCfg<BN>;
   CUtensorMap tx, tc, tm;
-  if (!encode_u8(&tx, Xq, K, T, K, Cfg::kKL, Cfg::kBHalf, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  if (!encode_u8(&tx, Xq, K, T, ldx, Cfg::kKL, Cfg::kBHalf, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_u8(&tc, codes, K / 8, O, ldc, 16, kBM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !encode_u8(&tm, meta, K / 8, O, ldm, 16, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
     return SBN_ERR_CUDA;
@@ -1154,37 +1154,37 @@ static sbn_status gemm_sp24_pair_t(const int8_t *Xq, const float *absmax, const 
 template <int BN>
 static sbn_status gemm_tc_bn(bool compact, const int8_t *Xq, const float *absmax,
                              const uint8_t *codes, const uint8_t *meta, const float *gamma_eff,
-                             int64_t T, int64_t O, int64_t K, int64_t ldc, int64_t ldm, void *Y,
+                             int64_t T, int64_t O, int64_t K, int64_t ldx, int64_t ldc, int64_t ldm, void *Y,
                              int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag, cudaStream_t st) {
   if (compact)
-    return gemm_sp24_t<BN>(Xq, absmax, codes, meta, gamma_eff, T, O, K, ldc, ldm, Y, y_is_bf16,
+    return gemm_sp24_t<BN>(Xq, absmax, codes, meta, gamma_eff, T, O, K, ldx, ldc, ldm, Y, y_is_bf16,
                            acc_dbg, err_flag, st);
-  return gemm_tc_t<BN, false>(Xq, absmax, codes, meta, gamma_eff, T, O, K, ldc, ldm, Y,
+  return gemm_tc_t<BN, false>(Xq, absmax, codes, meta, gamma_eff, T, O, K, ldx, ldc, ldm, Y,
                               y_is_bf16, acc_dbg, err_flag, st);
 }
 
 sbn_status launch_gemm_tc(const int8_t *Xq, const float *absmax, const uint8_t *codes,
                           const uint8_t *meta, const float *gamma_eff, int64_t tokens,
-                          int64_t out, int64_t in, int n, int m, int64_t ldc, int64_t ldm,
+                          int64_t out, int64_t in, int64_t ldx, int n, int m, int64_t ldc, int64_t ldm,
                           void *Y, int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag,
                           cudaStream_t st) {
   const bool compact = (n == 2 && m == 4);
   if (compact && tokens > 128)  // CTA pairs (every sm_100 device runs 2-CTA clusters)
-    return gemm_sp24_pair_t<224>(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc, ldm, Y,
+    return gemm_sp24_pair_t<224>(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldx, ldc, ldm, Y,
                                  y_is_bf16, acc_dbg, err_flag, st);
   if (tokens > 128)
-    return gemm_tc_bn<256>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc,
+    return gemm_tc_bn<256>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldx, ldc,
                            ldm, Y, y_is_bf16, acc_dbg, err_flag, st);
   if (tokens > 64)
-    return gemm_tc_bn<128>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc,
+    return gemm_tc_bn<128>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldx, ldc,
                            ldm, Y, y_is_bf16, acc_dbg, err_flag, st);
   if (tokens > 32)
-    return gemm_tc_bn<64>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc,
+    return gemm_tc_bn<64>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldx, ldc,
                           ldm, Y, y_is_bf16, acc_dbg, err_flag, st);
   if (tokens > 16)
-    return gemm_tc_bn<32>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc,
+    return gemm_tc_bn<32>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldx, ldc,
                           ldm, Y, y_is_bf16, acc_dbg, err_flag, st);
-  return gemm_tc_bn<16>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldc, ldm,
+  return gemm_tc_bn<16>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldx, ldc, ldm,
                         Y, y_is_bf16, acc_dbg, err_flag, st);
 }
 

@@ -43,9 +43,11 @@ template <int T, int SPL, bool kCompact>
 __global__ void __launch_bounds__(kGvThreads)
     k_gemv(const int8_t *__restrict__ Xq, const float *__restrict__ absmax,
            const uint8_t *__restrict__ codes, const uint8_t *__restrict__ meta,
-           const float *__restrict__ gamma_eff, int nt, int64_t out, int64_t in, int64_t ldc,
-           int64_t ldm, void *__restrict__ Y, int y_is_bf16, int32_t *__restrict__ acc_dbg) {
-  // T: tokens the kernel is built for; nt <= T: tokens present (rows nt.. of Xq do not exist)
+           const float *__restrict__ gamma_eff, int nt, int64_t out, int64_t in, int64_t ldx,
+           int64_t ldc, int64_t ldm, void *__restrict__ Y, int y_is_bf16,
+           int32_t *__restrict__ acc_dbg) {
+  // T: tokens the kernel is built for; nt <= T: tokens present (rows nt.. of Xq do not exist);
+  // ldx: elements between Xq rows (in, or more for a slice of wider rows)
   const int lane = threadIdx.x & 31;
   const int64_t row0 = kGvRows * (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   // launched as a programmatic dependent: everything read below comes from earlier kernels;
@@ -86,7 +88,7 @@ __global__ void __launch_bounds__(kGvThreads)
       for (int t = 0; t < T; ++t) {
         if (t >= nt) break;
         if constexpr (!kCompact) {
-          const uint4 x4 = __ldg(reinterpret_cast<const uint4 *>(Xq + t * in + (int64_t)wi * 16));
+          const uint4 x4 = __ldg(reinterpret_cast<const uint4 *>(Xq + t * ldx + (int64_t)wi * 16));
           const uint32_t xw[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
           for (int r = 0; r < kGvRows; ++r)
@@ -94,7 +96,7 @@ __global__ void __launch_bounds__(kGvThreads)
             for (int j = 0; j < 4; ++j)  // weights 4j..4j+3 sit in bits 7-2j..6-2j of the bytes
               acc[r][t] = __dp4a((int)((cw[r][i] << (2 * j)) & 0xC0C0C0C0u), (int)xw[j], acc[r][t]);
         } else {
-          const uint4 *xs = reinterpret_cast<const uint4 *>(Xq + t * in + (int64_t)wi * 32);
+          const uint4 *xs = reinterpret_cast<const uint4 *>(Xq + t * ldx + (int64_t)wi * 32);
           const uint4 xa = __ldg(xs), xb = __ldg(xs + 1);
           const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
 #pragma unroll
@@ -358,7 +360,7 @@ sbn_status launch_gemv_fused(const void *X, const uint8_t *codes, const uint8_t 
 template <int T, int SPL>
 static sbn_status gemv_tc(const int8_t *Xq, const float *absmax, const uint8_t *codes,
                           const uint8_t *meta, const float *gamma_eff, int nt, int64_t out,
-                          int64_t in,
+                          int64_t in, int64_t ldx,
                           bool compact, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
                           int32_t *acc_dbg, cudaStream_t st) {
   const int64_t rows_per_cta = kGvRows * (kGvThreads / 32);
@@ -376,8 +378,8 @@ static sbn_status gemv_tc(const int8_t *Xq, const float *absmax, const uint8_t *
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, Xq, absmax, codes, meta, gamma_eff, nt, out, in, ldc, ldm, Y,
-                         y_is_bf16, acc_dbg) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, kern, Xq, absmax, codes, meta, gamma_eff, nt, out, in, ldx, ldc,
+                         ldm, Y, y_is_bf16, acc_dbg) != cudaSuccess) {
     (void)cudaGetLastError();
     return SBN_ERR_CUDA;
   }
@@ -387,32 +389,32 @@ static sbn_status gemv_tc(const int8_t *Xq, const float *absmax, const uint8_t *
 template <int T>
 static sbn_status gemv_t(const int8_t *Xq, const float *absmax, const uint8_t *codes,
                          const uint8_t *meta, const float *gamma_eff, int nt, int64_t out,
-                         int64_t in,
+                         int64_t in, int64_t ldx,
                          bool compact, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
                          int32_t *acc_dbg, cudaStream_t st) {
   const int64_t words = in / (compact ? 32 : 16);  // code words per row
   const int64_t spl = (words + 31) / 32;
   if (spl <= 2)
-    return gemv_tc<T, 2>(Xq, absmax, codes, meta, gamma_eff, nt, out, in, compact, ldc, ldm, Y,
+    return gemv_tc<T, 2>(Xq, absmax, codes, meta, gamma_eff, nt, out, in, ldx, compact, ldc, ldm, Y,
                          y_is_bf16, acc_dbg, st);
   if (spl <= 4)
-    return gemv_tc<T, 4>(Xq, absmax, codes, meta, gamma_eff, nt, out, in, compact, ldc, ldm, Y,
+    return gemv_tc<T, 4>(Xq, absmax, codes, meta, gamma_eff, nt, out, in, ldx, compact, ldc, ldm, Y,
                          y_is_bf16, acc_dbg, st);
   if (spl <= 6 || T > 2)
-    return gemv_tc<T, 6>(Xq, absmax, codes, meta, gamma_eff, nt, out, in, compact, ldc, ldm, Y,
+    return gemv_tc<T, 6>(Xq, absmax, codes, meta, gamma_eff, nt, out, in, ldx, compact, ldc, ldm, Y,
                          y_is_bf16, acc_dbg, st);
-  return gemv_tc<T, 8>(Xq, absmax, codes, meta, gamma_eff, nt, out, in, compact, ldc, ldm, Y,
+  return gemv_tc<T, 8>(Xq, absmax, codes, meta, gamma_eff, nt, out, in, ldx, compact, ldc, ldm, Y,
                        y_is_bf16, acc_dbg, st);
 }
 
 sbn_status launch_gemv(const int8_t *Xq, const float *absmax, const uint8_t *codes,
                        const uint8_t *meta, const float *gamma_eff, int64_t tokens,
-                       int64_t out, int64_t in, int n, int m, int64_t ldc, int64_t ldm,
+                       int64_t out, int64_t in, int64_t ldx, int n, int m, int64_t ldc, int64_t ldm,
                        void *Y, int y_is_bf16, int32_t *acc_dbg, cudaStream_t st) {
   const bool compact = (n == 2 && m == 4);
   const int nt = (int)tokens;
 #define SBN_GEMV(TT)                                                                         \
-  return gemv_t<TT>(Xq, absmax, codes, meta, gamma_eff, nt, out, in, compact, ldc, ldm, Y, \
+  return gemv_t<TT>(Xq, absmax, codes, meta, gamma_eff, nt, out, in, ldx, compact, ldc, ldm, Y, \
                     y_is_bf16, acc_dbg, st)
   if (tokens == 1) SBN_GEMV(1);
   if (tokens == 2) SBN_GEMV(2);

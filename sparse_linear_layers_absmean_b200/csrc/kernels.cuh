@@ -70,7 +70,7 @@ sbn_status launch_act_quant(const void *X, int64_t tokens, int64_t in, int8_t *X
 // CUDA-core contraction for few tokens.
 sbn_status launch_gemv(const int8_t *Xq, const float *absmax, const uint8_t *codes,
                        const uint8_t *meta, const float *gamma_eff, int64_t tokens,
-                       int64_t out, int64_t in, int n, int m, int64_t ldc, int64_t ldm,
+                       int64_t out, int64_t in, int64_t ldx, int n, int m, int64_t ldc, int64_t ldm,
                        void *Y, int y_is_bf16, int32_t *acc_dbg, cudaStream_t st);
 
 // Steps 5-7 in one launch for at most kGemvMaxTokens tokens and in <= 16384 (gemv.cu).
@@ -83,7 +83,7 @@ sbn_status launch_gemv_fused(const void *X, const uint8_t *codes, const uint8_t 
 // Tensor-core (tcgen05, int8) contraction.
 sbn_status launch_gemm_tc(const int8_t *Xq, const float *absmax, const uint8_t *codes,
                           const uint8_t *meta, const float *gamma_eff, int64_t tokens,
-                          int64_t out, int64_t in, int n, int m, int64_t ldc, int64_t ldm,
+                          int64_t out, int64_t in, int64_t ldx, int n, int m, int64_t ldc, int64_t ldm,
                           void *Y, int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag,
                           cudaStream_t st);
 
@@ -127,6 +127,19 @@ sbn_status launch_backward(const void *dY, const int8_t *Xq, const float *absmax
                            const float *gamma_eff, int64_t T, int64_t O, int64_t K, int n, int m,
                            int64_t ldc, int64_t ldm, float *dX, float *dW, void *workspace,
                            int32_t *err_flag, cudaStream_t st);
+
+// Group quantisation (pack.cu, act_quant.cu, group_quant.cu): G blocks along K.
+sbn_status launch_pack_gq(const void *W, int64_t out, int64_t in, int n, int m, int G, float eps,
+                          uint8_t *codes, int64_t ldc, int64_t crow, uint8_t *meta, int64_t ldm,
+                          int64_t mrow, float *gamma_eff, PackWorkspace *ws, int8_t *dense_dbg,
+                          int32_t *err_flag, cudaStream_t st);
+sbn_status launch_act_quant_gq(const void *X, int64_t tokens, int64_t in, int G, int8_t *Xq,
+                               float *absmax, int32_t *err_flag, cudaStream_t st);
+sbn_status launch_linear_gq(const int8_t *Xq, const float *absmax, const uint8_t *codes,
+                            const uint8_t *meta, const float *gamma_eff, int64_t T, int64_t O,
+                            int64_t K, int n, int m, int G, int64_t ldc, int64_t ldm, void *Y,
+                            int y_is_bf16, float *part, int32_t *acc_dbg, int32_t *err_flag,
+                            cudaStream_t st);
 
 // Largest token count routed to the CUDA-core kernel; larger calls use the tensor cores.
 constexpr int64_t kGemvMaxTokens = 4;

@@ -292,6 +292,116 @@ __global__ void __launch_bounds__(256) k_quant_mask_pack(const QmpArgs<N, M> a) 
 }
 
 // ---------------------------------------------------------------------------------------
+// Group quantisation: G blocks along the input dimension K, each with its own absmean scale
+// g_j.  k_gq_abs_sum leaves P exact partial sums per group (CTA (p, j) of the grid takes
+// every P-th 64-weight block of group j); k_gq_quant_mask_pack turns them into the G
+// scales and code thresholds in its prologue and packs as k_quant_mask_pack does, each
+// 64-weight block with its group's threshold (K / G is a multiple of 64, so no block
+// straddles two groups).
+// ---------------------------------------------------------------------------------------
+constexpr int kGqMaxGroups = 64;
+
+__global__ void __launch_bounds__(kAsThreads)
+    k_gq_abs_sum(const uint4 *__restrict__ W, int64_t O, int64_t K, int G,
+                 PackWorkspace *ws, int32_t *err_flag) {
+  ptx::grid_dep_wait();
+  ptx::grid_dep_launch();
+  const int j = blockIdx.y, P = gridDim.x;
+  const int64_t bpg = K / G / 64;  // 64-weight blocks per row of a group
+  const int64_t nb = O * bpg;
+  double acc0 = kAccBias, acc1 = kAccBias;
+  uint32_t mx = 0, mx_fin = 0, mx_all = 0;
+  for (int64_t i = (int64_t)blockIdx.x * (blockDim.x / 8) + (threadIdx.x >> 3); i < nb;
+       i += (int64_t)P * (blockDim.x / 8)) {
+    const int64_t r = i / bpg, b = i - r * bpg;
+    // 8 threads per block, one 16-byte word each
+    const uint4 v = __ldg(W + (r * K + (int64_t)j * (K / G) + b * 64) / 8 + (threadIdx.x & 7));
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      asm("max.u16x2 %0, %0, %1;" : "+r"(mx) : "r"(w4[q] & 0x7fff7fffu));
+      acc0 = __dadd_rz(acc0, mag_lo_x2p128(w4[q]));
+      acc1 = __dadd_rz(acc1, mag_hi_x2p128(w4[q]));
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t m = (w4[q] >> (16 * h)) & 0x7fffu;
+        mx_all = max(mx_all, m);
+        if (m < kBf16InfBits) mx_fin = max(mx_fin, m);
+      }
+    }
+  }
+  unsigned long long acc = warp_sum_u64(acc_value(acc0) + acc_value(acc1));
+  const uint32_t ma = warp_max_u32(mx_all), mf = warp_max_u32(mx_fin);
+  __shared__ unsigned long long s_sum[kAsThreads / 32];
+  __shared__ uint32_t s_all[kAsThreads / 32], s_fin[kAsThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) {
+    s_sum[warp] = acc;
+    s_all[warp] = ma;
+    s_fin[warp] = mf;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long sum = 0;
+    uint32_t a = 0, f = 0;
+    for (int w = 0; w < kAsThreads / 32; ++w) {
+      sum += s_sum[w];
+      a = max(a, s_all[w]);
+      f = max(f, s_fin[w]);
+    }
+    ws->part[j * P + blockIdx.x] = sum;
+    int flags = 0;
+    if (a >= kBf16InfBits) flags |= SBN_FLAG_W_NONFINITE;
+    if (f >= kBf16Mag256Bits) flags |= SBN_FLAG_W_RANGE;
+    if (flags && err_flag) atomicOr(err_flag, flags);
+  }
+  (void)mx;
+}
+
+template <int N, int M>
+__global__ void __launch_bounds__(256)
+    k_gq_quant_mask_pack(const QmpArgs<N, M> a, int G, int P, uint32_t bpg, FastDiv div_bpg) {
+  __shared__ uint32_t s_thr[kGqMaxGroups];
+  ptx::grid_dep_launch();
+  ptx::grid_dep_wait();
+  // prologue: warp w finishes groups w, w + 8, ...: exact sum of the group's P partials,
+  // g_j = fp32(fp32(fp64(S_j) / (fp64(n / G) * 2^24)) + eps), code threshold of g_j
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int j = warp; j < G; j += blockDim.x >> 5) {
+    unsigned long long S = 0;
+    for (int i = lane; i < P; i += 32) S += a.ws->part[j * P + i];
+    S = warp_sum_u64(S);
+    const double mean = __ddiv_rn(__ull2double_rn(S), (double)(a.n / G) * 16777216.0);
+    const float g = __fadd_rn(__double2float_rn(mean), a.eps);
+    const uint32_t thr = code_threshold_warp(g, lane);
+    if (lane == 0) {
+      s_thr[j] = thr;
+      if (blockIdx.x == 0) a.gamma_eff[j] = g;
+    }
+  }
+  __syncthreads();
+  const int sub = lane & 7;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t nquads = (a.nblocks + 3) >> 2;
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+  auto thr_of = [&](int64_t b) -> uint32_t {
+    if (b >= a.nblocks) return s_thr[0];
+    const uint32_t row = fast_div((uint32_t)b, a.div_bpr);
+    const uint32_t col = (uint32_t)b - row * a.bpr;
+    return s_thr[fast_div(col, div_bpg)];
+  };
+  for (int64_t q = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; q < nquads;
+       q += 2 * nwarps) {
+    const int64_t b0 = 4 * q + (lane >> 3);
+    const int64_t b1 = b0 + 4 * nwarps;
+    const uint4 v0 = b0 < a.nblocks ? __ldg(a.W + b0 * 8 + sub) : zero;
+    const uint4 v1 = b1 < a.nblocks ? __ldg(a.W + b1 * 8 + sub) : zero;
+    qmp_block<N, M>(a, v0, b0, sub, thr_of(b0));
+    if (q + nwarps < nquads) qmp_block<N, M>(a, v1, b1, sub, thr_of(b1));
+  }
+  (void)bpg;
+}
+
+// ---------------------------------------------------------------------------------------
 // Host launchers
 // ---------------------------------------------------------------------------------------
 
@@ -396,6 +506,64 @@ sbn_status launch_pack(const void *W, int64_t out, int64_t in, int n, int m, flo
 #undef SBN_QMP
   SBN_LAUNCH_CHECK();
   return SBN_OK;
+}
+
+template <int N, int M>
+static sbn_status launch_gq_qmp(const uint4 *W, int64_t nblocks, int64_t bpr, int64_t bpg, int G,
+                                int P, const PackWorkspace *ws, uint8_t *codes, int64_t ldc,
+                                int64_t crow, uint8_t *meta, int64_t ldm, int64_t mrow,
+                                int8_t *dense_dbg, int64_t n, float eps, float *gamma_eff,
+                                cudaStream_t st) {
+  const int64_t nquads = (nblocks + 3) / 4;
+  int64_t grid = (nquads + 15) / 16;
+  const int64_t cap = (int64_t)num_sms() * 8;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  QmpArgs<N, M> a{W,    nblocks,   (uint32_t)bpr, make_fast_div((uint32_t)bpr), ws, codes, ldc,
+                  crow, meta,      ldm,           mrow,          dense_dbg,    P,  n,
+                  eps,  gamma_eff};
+  return launch_pdl(k_gq_quant_mask_pack<N, M>, dim3((unsigned)grid), dim3(256), 0, st, a, G, P,
+                    (uint32_t)bpg, make_fast_div((uint32_t)bpg));
+}
+
+sbn_status launch_pack_gq(const void *W, int64_t out, int64_t in, int n, int m, int G, float eps,
+                          uint8_t *codes, int64_t ldc, int64_t crow, uint8_t *meta, int64_t ldm,
+                          int64_t mrow, float *gamma_eff, PackWorkspace *ws, int8_t *dense_dbg,
+                          int32_t *err_flag, cudaStream_t st) {
+  if (G < 1 || G > kGqMaxGroups) return SBN_ERR_SHAPE;
+  const uint4 *W4 = reinterpret_cast<const uint4 *>(W);
+  const int64_t nblocks = out * in / 64, bpr = in / 64, bpg = bpr / G;
+  // P CTAs per group, at most kPackMaxParts partial sums in all
+  int64_t P = ((int64_t)num_sms() * 4 + G - 1) / G;
+  const int64_t per_group = (out * bpg + (kAsThreads / 8) - 1) / (kAsThreads / 8);
+  if (P > per_group) P = per_group;
+  if (P > kPackMaxParts / G) P = kPackMaxParts / G;
+  if (P < 1) P = 1;
+  sbn_status s = launch_pdl(k_gq_abs_sum, dim3((unsigned)P, (unsigned)G), dim3(kAsThreads), 0, st,
+                            W4, out, in, G, ws, err_flag);
+  if (s != SBN_OK) return s;
+  const int64_t nel = out * in;
+#define SBN_GQMP(NN, MM)                                                                       \
+  case (NN * 16 + MM):                                                                         \
+    return launch_gq_qmp<NN, MM>(W4, nblocks, bpr, bpg, G, (int)P, ws, codes, ldc, crow, meta, \
+                                 ldm, mrow, dense_dbg, nel, eps, gamma_eff, st);
+  switch (n * 16 + m) {
+    SBN_GQMP(1, 4)
+    SBN_GQMP(2, 4)
+    SBN_GQMP(3, 4)
+    SBN_GQMP(4, 4)
+    SBN_GQMP(1, 8)
+    SBN_GQMP(2, 8)
+    SBN_GQMP(3, 8)
+    SBN_GQMP(4, 8)
+    SBN_GQMP(5, 8)
+    SBN_GQMP(6, 8)
+    SBN_GQMP(7, 8)
+    SBN_GQMP(8, 8)
+    default:
+      return SBN_ERR_PATTERN;
+  }
+#undef SBN_GQMP
 }
 
 }  // namespace sbn
