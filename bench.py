@@ -470,13 +470,20 @@ def bench_train(args, sbn, dev, local, rank, world, peaks, timer, err):
                                 torch.empty((O, d.meta_ld), dtype=torch.uint8, device=dev),
                                 torch.empty(1, dtype=torch.float32, device=dev))
             lin.append((O, K, W, outs))
-    ws = sbn.new_workspace(8, 64, 2, 4, dev)
+    # the 6:8 and 2:4 packs of a tensor are independent: one stream each (own workspace), so
+    # their launches overlap and the second read of W can come from L2
+    ws = {(6, 8): sbn.new_workspace(8, 64, 2, 4, dev), (2, 4): sbn.new_workspace(8, 64, 2, 4, dev)}
     st = timer.stream
+    side = torch.cuda.Stream(device=dev)
 
     def step(i, ev):
+        side.wait_stream(st)
         for O, K, W, outs in lin:
             for (n, m), (c, mt, gm) in outs.items():
-                sbn.sbn_quantize_mask_pack_weights(W, n, m, 1e-5, c, mt, gm, ws, None, err, st)
+                s_ = st if (n, m) == (6, 8) else side
+                sbn.sbn_quantize_mask_pack_weights(W, n, m, 1e-5, c, mt, gm, ws[(n, m)], None, err,
+                                                   s_)
+        st.wait_stream(side)
 
     steps = min(args.steps, 10)
     ms, _, clocks = timer.run(step, steps, min(args.warmup, 3))
@@ -487,7 +494,139 @@ def bench_train(args, sbn, dev, local, rank, world, peaks, timer, err):
             "roofline": hbm_roof(gbs, peaks, "quant_mask_pack, 130 tensors x (6:8, 2:4)"),
             "gpu_launches": 2 * 2 * len(lin) * steps, "clocks": clocks,
             "config": {"workload": "train-step-26x3200-6of8+2of4", "tensors": len(lin),
-                       "weights": weights, "bytes_per_step": moved}}
+                       "weights": weights, "bytes_per_step": moved,
+                       "step": "every tensor packed in 6:8 (main stream) and 2:4 (side stream)"}}
+
+
+# ---- next rows: backward, group quantisation, one-launch decode ----------------------------
+
+def bench_backward(args, sbn, dev, local, rank, world, peaks, timer, err):
+    """The dual-STE backward on the prefill configuration's shape (W 11008 x 4096 2:4, 2048
+    tokens): dX and the clip-gated dW, both tensor-core GEMMs.  Algorithmic flops: 2 T O K
+    for each (dW's second bf16 term is an implementation cost, not counted)."""
+    cfg = workloads.PREFILL_GEMM
+    O, K, T = cfg["O"], cfg["K"], cfg["T"]
+    W = workloads.masters_device(O, K, device=dev, config=6, tensor=0)
+    X = workloads.torch_bf16(workloads.activations(T, K, seed=0, config=6, tensor=1), dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(6)
+    dY = torch.randn((T, O), device=dev, generator=g).bfloat16()
+    w = sbn.pack_weights(W, 2, 4, err_flag=err)
+    Xq, s = sbn.quantize_acts(X, err_flag=err)
+    dX = torch.empty((T, K), dtype=torch.float32, device=dev)
+    dW = torch.empty((O, K), dtype=torch.float32, device=dev)
+    ws = torch.empty(sbn.sbn_backward_workspace_bytes(T, O, K), dtype=torch.uint8, device=dev)
+    st = timer.stream
+
+    def step(i, ev):
+        if ev is not None:
+            ev["dX"][0].record(st)
+        sbn.sbn_backward(dY, Xq, s, w.codes, w.meta, W, w.gamma_eff, O, K, 2, 4, dX, None, ws, err,
+                         st)
+        if ev is not None:
+            ev["dX"][1].record(st)
+            ev["dW"][0].record(st)
+        sbn.sbn_backward(dY, Xq, s, w.codes, w.meta, W, w.gamma_eff, O, K, 2, 4, None, dW, ws, err,
+                         st)
+        if ev is not None:
+            ev["dW"][1].record(st)
+
+    steps = min(args.steps, 10)
+    ms, per, clocks = timer.run(step, steps, min(args.warmup, 3), calls=("dX", "dW"))
+    flops = 2 * T * O * K
+    peak = peaks["bf16"]
+    return {"value": 2 * flops * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
+            "steps": steps,
+            "roofline": {"bound": "tensor", "achieved": flops / (per["dX"] * 1e-3) / 1e12,
+                         "peak": peak, "unit": "TFLOP/s",
+                         "frac": flops / (per["dX"] * 1e-3) / 1e12 / peak, "traffic": None,
+                         "kernel": "k_gemm_bf16<0> (dX = g dY Ws, bf16 x bf16 -> fp32)",
+                         "peak_source": f"bf16_tflops (burst) of MEASURED_PEAKS.json "
+                                        f"({peaks['source']}: of measured)"},
+            "kernels": {"dX": {"ms": per["dX"], "TFLOP/s": flops / (per["dX"] * 1e-3) / 1e12},
+                        "dW": {"ms": per["dW"], "TFLOP/s": flops / (per["dW"] * 1e-3) / 1e12,
+                               "note": "two bf16 terms of the scaled dY: 2x the MMA work"}},
+            "gpu_launches": 6 * steps, "clocks": clocks,
+            "config": {"workload": "backward-11008x4096-t2048-2of4", "flops_per_gemm": flops}}
+
+
+def bench_group_quant(args, sbn, dev, local, rank, world, peaks, timer, err):
+    """Group quantisation (G = 4 blocks along K) on the stack's QKV shape (12288 x 4096 2:4)
+    at 16 tokens: per step the group activation quantiser and the contraction (4 block
+    contractions + the ordered sum), weights packed once with per-group scales."""
+    O, K, T, G = 12288, 4096, workloads.STACK_DECODE_T, 4
+    R = 8  # rotating weight sets: 8 x 12.6 MB of packed weights > L2
+    ws_ = []
+    for r in range(R):
+        W = workloads.masters_device(O, K, device=dev, config=7, tensor=r)
+        ws_.append(sbn.pack_weights_gq(W, 2, 4, G, err_flag=err))
+        del W
+    X = workloads.torch_bf16(workloads.student_t(T, K, config=7, tensor=100), dev)
+    Xq = torch.empty((T, K), dtype=torch.int8, device=dev)
+    s = torch.empty((G, T), dtype=torch.float32, device=dev)
+    Y = torch.empty((T, O), dtype=torch.float32, device=dev)
+    part = torch.empty(G * T * O * 4, dtype=torch.uint8, device=dev)
+    st = timer.stream
+
+    def step(i, ev):
+        w = ws_[i % R]
+        sbn.sbn_quantize_acts_gq(X, G, Xq, s, err, st)
+        if ev is not None:
+            ev["linear"][0].record(st)
+        sbn.sbn_linear_gq(Xq, s, w.codes, w.meta, w.gamma_eff, O, K, 2, 4, G, Y, part, None, err, st)
+        if ev is not None:
+            ev["linear"][1].record(st)
+
+    steps = args.steps
+    ms, per, clocks = timer.run(step, steps, args.warmup, calls=("linear",))
+    packed = O * K // 4
+    gbs = packed / (per["linear"] * 1e-3) / 1e9
+    return {"value": packed * world / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+            "steps": steps,
+            "roofline": hbm_roof(gbs, peaks, "per-block contraction (k_gemm_sp24<16> on 4 slices) "
+                                 "+ ordered sum", unit_note="; on packed-weight bytes"),
+            "gpu_launches": 6 * steps, "clocks": clocks,
+            "config": {"workload": "group-quant-12288x4096-t16-2of4-G4", "groups": G,
+                       "l2": f"{R} rotating packed weight sets"}}
+
+
+def bench_fused_decode(args, sbn, dev, local, rank, world, peaks, timer, err):
+    """One-launch decode (sbn_quantize_linear: activation quantiser in the GEMV prologue) on
+    the decode configuration's pre-packed weights (W 6912 x 2560 6:8, 1 token), against the
+    two separate launches; 8 rotating weight sets beyond L2."""
+    cfg = workloads.DECODE_GEMV
+    O, K, T, n, m = cfg["O"], cfg["K"], cfg["T"], cfg["n"], cfg["m"]
+    R = 16
+    packs = []
+    for r in range(R):
+        W = workloads.masters_device(O, K, device=dev, config=2, tensor=r)
+        packs.append(sbn.pack_weights(W, n, m, err_flag=err))
+        del W
+    X = workloads.torch_bf16(workloads.activations(T, K, seed=0, config=2, tensor=1), dev)
+    Xq = torch.empty((T, K), dtype=torch.int8, device=dev)
+    s = torch.empty((T,), dtype=torch.float32, device=dev)
+    Y = torch.empty((T, O), dtype=torch.float32, device=dev)
+    st = timer.stream
+
+    def fused(i, ev):
+        w = packs[i % R]
+        sbn.sbn_quantize_linear(X, w.codes, w.meta, w.gamma_eff, O, K, n, m, Xq, s, Y, None, err, st)
+
+    def separate(i, ev):
+        w = packs[i % R]
+        sbn.sbn_quantize_acts(X, Xq, s, err, st)
+        sbn.sbn_linear(Xq, s, w.codes, w.meta, w.gamma_eff, O, K, n, m, Y, None, err, st)
+
+    ms_f, _, clocks = timer.run(fused, args.steps, args.warmup)
+    ms_s, _, _ = timer.run(separate, args.steps, args.warmup, sample_clocks=False)
+    codes_b = O * K // 4
+    return {"value": codes_b * world / (ms_f * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms_f,
+            "separate_ms_per_step": ms_s,
+            "roofline": hbm_roof(codes_b / (ms_f * 1e-3) / 1e9, peaks,
+                                 "k_gemv_fused (act quant in the GEMV prologue)",
+                                 unit_note="; on the 0.25 B/w codes the GEMV reads"),
+            "gpu_launches": args.steps, "clocks": clocks,
+            "config": {"workload": "fused-decode-6912x2560-t1-6of8", "rotating_sets": R}}
 
 
 # ---- the oracle (CPU baseline legs and the reference arm) ---------------------------------
@@ -676,6 +815,11 @@ def run_cuda(args):
                                                 workloads.PREFILL_GEMM, err)
             subs["train_step"] = bench_train(args, sbn, dev, local, rank, world, peaks, timer,
                                              err)
+            subs["backward"] = bench_backward(args, sbn, dev, local, rank, world, peaks, timer, err)
+            subs["group_quant"] = bench_group_quant(args, sbn, dev, local, rank, world, peaks,
+                                                    timer, err)
+            subs["fused_decode"] = bench_fused_decode(args, sbn, dev, local, rank, world, peaks,
+                                                      timer, err)
     elif args.workload == "decode":
         head, subs = bench_single(args, sbn, dev, local, rank, world, peaks, timer,
                                   workloads.DECODE_GEMV, err), {}

@@ -510,28 +510,46 @@ def pack_weights_gq(W, n, m, groups, eps=1e-5, dense_dbg=None, err_flag=None, st
     return GqPackedWeights(codes, meta, gamma, out, in_, n, m, groups)
 
 
+def sbn_quantize_acts_gq(X, groups, Xq, absmax, err_flag=None, stream=None):
+    T, K = X.shape
+    _check(lib().sbn_quantize_acts_gq(_ptr(X), T, K, groups, _ptr(Xq), _ptr(absmax), _ptr(err_flag),
+                                      _stream(stream)), "sbn_quantize_acts_gq")
+
+
+def sbn_gq_workspace_bytes(tokens, out, in_, groups):
+    b = ctypes.c_int64()
+    _check(lib().sbn_gq_workspace_bytes(tokens, out, in_, groups, ctypes.byref(b)),
+           "sbn_gq_workspace_bytes")
+    return b.value
+
+
+def sbn_linear_gq(Xq, absmax, codes, meta, gamma_eff, out, in_, n, m, groups, Y, workspace,
+                  acc_dbg=None, err_flag=None, stream=None):
+    if Y.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("Y must be float32 or bfloat16")
+    _check(lib().sbn_linear_gq(_ptr(Xq), _ptr(absmax), _ptr(codes), _ptr(meta), _ptr(gamma_eff),
+                               Xq.shape[0], out, in_, n, m, groups, _ptr(Y),
+                               1 if Y.dtype == torch.bfloat16 else 0, _ptr(workspace),
+                               _ptr(acc_dbg), _ptr(err_flag), _stream(stream)), "sbn_linear_gq")
+
+
 def quantize_acts_gq(X, groups, err_flag=None, stream=None):
     """(Xq int8 [T, K], s fp32 [groups, T])."""
     T, K = X.shape
     with _alloc_stream(stream):
         Xq = torch.empty((T, K), dtype=torch.int8, device=X.device)
         s = torch.empty((groups, T), dtype=torch.float32, device=X.device)
-    _check(lib().sbn_quantize_acts_gq(_ptr(X), T, K, groups, _ptr(Xq), _ptr(s), _ptr(err_flag),
-                                      _stream(stream)), "sbn_quantize_acts_gq")
+    sbn_quantize_acts_gq(X, groups, Xq, s, err_flag, stream)
     return Xq, s
 
 
 def linear_gq(Xq, s, w: GqPackedWeights, out_dtype=torch.float32, acc_dbg=None, err_flag=None,
               stream=None):
     T = Xq.shape[0]
-    b = ctypes.c_int64()
-    _check(lib().sbn_gq_workspace_bytes(T, w.out, w.in_, w.groups, ctypes.byref(b)),
-           "sbn_gq_workspace_bytes")
     with _alloc_stream(stream):
         Y = torch.empty((T, w.out), dtype=out_dtype, device=Xq.device)
-        ws = torch.empty(max(b.value, 16), dtype=torch.uint8, device=Xq.device)
-    _check(lib().sbn_linear_gq(_ptr(Xq), _ptr(s), _ptr(w.codes), _ptr(w.meta), _ptr(w.gamma_eff), T,
-                               w.out, w.in_, w.n, w.m, w.groups, _ptr(Y),
-                               1 if out_dtype == torch.bfloat16 else 0, _ptr(ws), _ptr(acc_dbg),
-                               _ptr(err_flag), _stream(stream)), "sbn_linear_gq")
+        ws = torch.empty(max(sbn_gq_workspace_bytes(T, w.out, w.in_, w.groups), 16),
+                         dtype=torch.uint8, device=Xq.device)
+    sbn_linear_gq(Xq, s, w.codes, w.meta, w.gamma_eff, w.out, w.in_, w.n, w.m, w.groups, Y, ws,
+                  acc_dbg, err_flag, stream)
     return Y
