@@ -144,9 +144,13 @@ __global__ void __launch_bounds__(kGvThreads)
 // Steps 5-7 in one launch for a few tokens: every CTA quantises the (small) token rows
 // itself -- the per-token absmax by a block reduction over X (bf16, read from L2), then
 // q = clamp(rint((127 x) / s), -127, 127) with the IEEE divide into shared memory -- and
-// runs the GEMV above on them (two rows per warp, activations from shared memory).  CTA 0
-// also writes Xq and s to global memory.  Shared memory: T * in bytes (in <= 16384).
+// runs the GEMV above on them (two rows per warp, 8 warps per CTA, activations from shared
+// memory).  CTA 0 also writes Xq and s to global memory.  Shared memory: T * in bytes
+// (in <= 16384).
 constexpr int64_t kFusedMaxIn = 16384;
+// 8 warps (16 rows) per CTA: the row quantisation every CTA repeats is spread over 256
+// threads and over 2x fewer CTAs than the GEMV's 8-row CTAs
+constexpr int kGfThreads = 256;
 
 __device__ __forceinline__ uint32_t fused_q2(uint32_t w, float s) {
   const float xl = bf16_lo_to_float(w), xh = bf16_hi_to_float(w);
@@ -158,14 +162,14 @@ __device__ __forceinline__ uint32_t fused_q2(uint32_t w, float s) {
 }
 
 template <int T, int SPL, bool kCompact>
-__global__ void __launch_bounds__(kGvThreads)
+__global__ void __launch_bounds__(kGfThreads)
     k_gemv_fused(const uint16_t *__restrict__ X, const uint8_t *__restrict__ codes,
                  const uint8_t *__restrict__ meta, const float *__restrict__ gamma_eff, int nt,
                  int64_t out, int64_t in, int64_t ldc, int64_t ldm, void *__restrict__ Y,
                  int y_is_bf16, int8_t *__restrict__ Xq_out, float *__restrict__ absmax_out,
                  int32_t *__restrict__ acc_dbg, int32_t *err_flag) {
   extern __shared__ __align__(16) uint8_t s_xq[];  // [T][in] int8
-  __shared__ uint32_t s_red[T][kGvThreads / 32];
+  __shared__ uint32_t s_red[T][kGfThreads / 32];
   __shared__ float s_scale[T];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   ptx::grid_dep_launch();
@@ -176,7 +180,7 @@ __global__ void __launch_bounds__(kGvThreads)
     if (t >= nt) break;
     const uint4 *row = reinterpret_cast<const uint4 *>(X + t * in);
     uint32_t mx = 0;
-    for (int64_t i = threadIdx.x; i < nv; i += kGvThreads) {
+    for (int64_t i = threadIdx.x; i < nv; i += kGfThreads) {
       const uint4 v = __ldg(row + i);
       mx = __vmaxu2(mx, v.x & 0x7fff7fffu);
       mx = __vmaxu2(mx, v.y & 0x7fff7fffu);
@@ -190,7 +194,7 @@ __global__ void __launch_bounds__(kGvThreads)
   if (threadIdx.x < nt) {
     uint32_t m = 0;
 #pragma unroll
-    for (int w = 0; w < kGvThreads / 32; ++w) m = max(m, s_red[threadIdx.x][w]);
+    for (int w = 0; w < kGfThreads / 32; ++w) m = max(m, s_red[threadIdx.x][w]);
     if (m >= kBf16InfBits && blockIdx.x == 0 && err_flag) atomicOr(err_flag, SBN_FLAG_X_NONFINITE);
     const float sc = fmaxf(__uint_as_float(m << 16), 1e-5f);
     s_scale[threadIdx.x] = sc;
@@ -203,7 +207,7 @@ __global__ void __launch_bounds__(kGvThreads)
     const uint4 *row = reinterpret_cast<const uint4 *>(X + t * in);
     uint2 *q = reinterpret_cast<uint2 *>(s_xq + t * in);
     uint2 *qg = Xq_out ? reinterpret_cast<uint2 *>(Xq_out + t * in) : nullptr;
-    for (int64_t i = threadIdx.x; i < nv; i += kGvThreads) {
+    for (int64_t i = threadIdx.x; i < nv; i += kGfThreads) {
       const uint4 v = __ldg(row + i);
       const uint2 o = make_uint2(fused_q2(v.x, sc) | (fused_q2(v.y, sc) << 16),
                                  fused_q2(v.z, sc) | (fused_q2(v.w, sc) << 16));
@@ -306,14 +310,14 @@ static sbn_status gemv_fused_t(const void *X, const uint8_t *codes, const uint8_
                                bool compact, int64_t ldc, int64_t ldm, void *Y, int y_is_bf16,
                                int8_t *Xq, float *absmax, int32_t *acc_dbg, int32_t *err_flag,
                                cudaStream_t st) {
-  const int64_t rows_per_cta = kGvRows * (kGvThreads / 32);
+  const int64_t rows_per_cta = kGvRows * (kGfThreads / 32);
   const int64_t grid = (out + rows_per_cta - 1) / rows_per_cta;
   auto kern = compact ? k_gemv_fused<T, SPL, true> : k_gemv_fused<T, SPL, false>;
   const size_t smem = (size_t)T * (size_t)in;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)(T * kFusedMaxIn)) != cudaSuccess)
     return SBN_ERR_CUDA;
-  return launch_pdl(kern, dim3((unsigned)grid), dim3(kGvThreads), smem, st,
+  return launch_pdl(kern, dim3((unsigned)grid), dim3(kGfThreads), smem, st,
                     static_cast<const uint16_t *>(X), codes, meta, gamma_eff, nt, out, in, ldc,
                     ldm, Y, y_is_bf16, Xq, absmax, acc_dbg, err_flag);
 }
