@@ -62,11 +62,19 @@ def load_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
+def peak_source(peaks, key, value, what=""):
+    """Where a roofline denominator came from: the measured file, or (when it is
+    absent) the earlier measurement on the same B200 pool that stands in for it."""
+    if peaks["source"] == "measured":
+        return f"{what}{key} of MEASURED_PEAKS.json: of measured"
+    return (f"{what}{key} = {value} (MEASURED_PEAKS.json absent; earlier measurement on "
+            "this B200 pool): of fallback")
+
+
 def hbm_roof(achieved, peaks, kernel, traffic=None, unit_note=""):
     return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
             "frac": achieved / peaks["hbm"], "traffic": traffic, "kernel": kernel,
-            "peak_source": f"hbm_gbs of MEASURED_PEAKS.json ({peaks['source']}: of measured)"
-                           + unit_note}
+            "peak_source": peak_source(peaks, "hbm_gbs", peaks["hbm"]) + unit_note}
 
 
 def tensor_roof(achieved, peaks, kernel, traffic=None):
@@ -75,8 +83,8 @@ def tensor_roof(achieved, peaks, kernel, traffic=None):
     peak = 2.0 * peaks["bf16"]
     return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": traffic, "kernel": kernel,
-            "peak_source": f"2 x bf16_tflops (burst) of MEASURED_PEAKS.json ({peaks['source']}: "
-                           "of measured); kept int8 ops"}
+            "peak_source": peak_source(peaks, "bf16_tflops", peaks["bf16"], "2 x burst ")
+                           + "; kept int8 ops"}
 
 
 class ClockSampler:
@@ -541,8 +549,7 @@ def bench_backward(args, sbn, dev, local, rank, world, peaks, timer, err):
                          "peak": peak, "unit": "TFLOP/s",
                          "frac": flops / (per["dX"] * 1e-3) / 1e12 / peak, "traffic": None,
                          "kernel": "k_gemm_bf16<0> (dX = g dY Ws, bf16 x bf16 -> fp32)",
-                         "peak_source": f"bf16_tflops (burst) of MEASURED_PEAKS.json "
-                                        f"({peaks['source']}: of measured)"},
+                         "peak_source": peak_source(peaks, "bf16_tflops", peaks["bf16"], "burst ")},
             "kernels": {"dX": {"ms": per["dX"], "TFLOP/s": flops / (per["dX"] * 1e-3) / 1e12},
                         "dW": {"ms": per["dW"], "TFLOP/s": flops / (per["dW"] * 1e-3) / 1e12,
                                "note": "two bf16 terms of the scaled dY: 2x the MMA work"}},

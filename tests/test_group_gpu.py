@@ -5,8 +5,8 @@ Bit-exact: int8 activations, per-token scales (fp32 bits), int32 accumulators of
 layer.  Float: fp32 y within 1e-5 relative of the oracle's fp64 y; bf16 within 8e-3.
 Shapes cover ragged row tiles (O % 128 != 0), K % 128 == 64, 1..32 tokens, layers with 0
 tokens, a schedule that splits row tiles over several work units (called twice: the
-split's arrival counters must be back at zero), and the 4096-hidden stack layer at 16
-tokens."""
+split's arrival counters must be back at zero), the 4096-hidden stack layer at 16 tokens
+compared in full, and the whole 160-linear stack in one plan on sampled linears and rows."""
 import numpy as np
 import pytest
 import torch
@@ -130,3 +130,61 @@ def test_group_stack_layer_full_size():
     plan = sbn.GroupPlan(layers)
     run(plan)
     check(layers, host)
+
+
+# sampled linears of the full stack: first, middle and last layers, every projection kind,
+# the last linear of the plan included (the end of the unit schedule)
+STACK_SAMPLE = [0, 1, 2, 3, 4, 77, 83, 155, 159]
+
+
+def test_group_full_stack_sampled():
+    """All 160 linears of the 32-layer stack (hidden 4096, FFN 11008) at 16 tokens, 2:4, in
+    one plan: the launch the benchmark times, with its seeded weights and activations.  The
+    oracle checks every output of sampled linears on sampled rows (row tiles' first and last
+    rows, the ragged end, random rows): codes and meta of those rows, Xq and s of the
+    linear, int32 sums and y.  Every other output must be finite."""
+    T = workloads.STACK_DECODE_T
+    rng = np.random.default_rng(5)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    layers, sampled = [], {}
+    for layer in range(workloads.STACK_LAYERS):
+        for i, (_, O, K) in enumerate(workloads.STACK_LAYER_SHAPES):
+            idx = 5 * layer + i
+            W = workloads.masters_device(O, K, device="cuda", config=5, tensor=idx)
+            w = sbn.pack_weights(W, 2, 4, 1e-5, err_flag=err)
+            X_bits = workloads.student_t(T, K, config=5, tensor=10000 + idx)
+            L = dict(X=workloads.torch_bf16(X_bits, "cuda"),
+                     Xq=torch.empty((T, K), dtype=torch.int8, device="cuda"),
+                     s=torch.empty((T,), dtype=torch.float32, device="cuda"), w=w,
+                     Y=torch.empty((T, O), dtype=torch.float32, device="cuda"))
+            if idx in STACK_SAMPLE:
+                L["acc_dbg"] = torch.empty((T, O), dtype=torch.int32, device="cuda")
+                W_bits = W.view(torch.int16).cpu().numpy().view(np.uint16)
+                rows = np.unique(np.concatenate([[0, 127, 128, O - 1],
+                                                 rng.choice(O, size=12, replace=False)]))
+                sampled[idx] = (W_bits, X_bits, rows)
+            layers.append(L)
+            del W
+    plan = sbn.GroupPlan(layers)
+    run(plan)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    for idx, (W_bits, X_bits, rows) in sampled.items():
+        L = layers[idx]
+        ri = torch.as_tensor(rows, device="cuda")
+        _, _, g, werr = oracle.weight_gamma(W_bits, 1e-5)
+        assert werr == 0
+        assert L["w"].gamma_eff.cpu().numpy().view(np.uint32)[0] == np.float32(g).view(np.uint32)
+        t, keep, ws = oracle.ternary_mask(W_bits[rows], 2, 4, g)
+        codes, meta = oracle.pack(t, keep, 2, 4)
+        assert np.array_equal(L["w"].codes[ri].cpu().numpy(), codes)
+        assert np.array_equal(L["w"].meta[ri].cpu().numpy(), meta)
+        Xq, s, xerr = oracle.quant_acts(X_bits)
+        assert xerr == 0
+        assert np.array_equal(L["Xq"].cpu().numpy(), Xq)
+        assert np.array_equal(L["s"].cpu().numpy().view(np.uint32), s.view(np.uint32))
+        acc = oracle.contract(Xq, ws)
+        assert np.array_equal(L["acc_dbg"][:, ri].cpu().numpy(), acc)
+        gpu_path.assert_y_close(L["Y"][:, ri].cpu().numpy(), oracle.rescale(acc, s, g))
+    for L in layers:
+        assert torch.isfinite(L["Y"]).all()
