@@ -466,44 +466,87 @@ def bench_single(args, sbn, dev, local, rank, world, peaks, timer, cfg, err):
 # ---- training-step weight path (configuration 4) -----------------------------------------
 
 def bench_train(args, sbn, dev, local, rank, world, peaks, timer, err):
-    lin = []
+    """Every linear of the 26-layer decoder re-packed from its masters in 6:8 and 2:4: one
+    grouped pack (two launches for all 130 tensors, W read once for the absmean sums and
+    once for both patterns' planes).  The per-tensor calls (two launches per tensor and
+    pattern, the patterns on two streams) are timed beside it for comparison."""
+    Ws = []
     for layer in range(workloads.TRAIN_LAYERS):
         for i, (name, O, K) in enumerate(workloads.TRAIN_LAYER_SHAPES):
-            W = workloads.masters_device(O, K, device=dev, config=4,
-                                         tensor=5 * layer + i + 1000 * rank)
-            outs = {}
-            for (n, m) in ((6, 8), (2, 4)):
-                d = sbn.sbn_linear_ref_dims(O, K, n, m)
-                outs[(n, m)] = (torch.empty((O, d.codes_ld), dtype=torch.uint8, device=dev),
-                                torch.empty((O, d.meta_ld), dtype=torch.uint8, device=dev),
-                                torch.empty(1, dtype=torch.float32, device=dev))
-            lin.append((O, K, W, outs))
-    # the 6:8 and 2:4 packs of a tensor are independent: one stream each (own workspace), so
-    # their launches overlap and the second read of W can come from L2
-    ws = {(6, 8): sbn.new_workspace(8, 64, 2, 4, dev), (2, 4): sbn.new_workspace(8, 64, 2, 4, dev)}
+            Ws.append(workloads.masters_device(O, K, device=dev, config=4,
+                                               tensor=5 * layer + i + 1000 * rank))
+    pg = sbn.PackGroup(Ws, ((6, 8), (2, 4)), device=dev)
     st = timer.stream
-    side = torch.cuda.Stream(device=dev)
 
     def step(i, ev):
-        side.wait_stream(st)
-        for O, K, W, outs in lin:
-            for (n, m), (c, mt, gm) in outs.items():
-                s_ = st if (n, m) == (6, 8) else side
-                sbn.sbn_quantize_mask_pack_weights(W, n, m, 1e-5, c, mt, gm, ws[(n, m)], None, err,
-                                                   s_)
-        st.wait_stream(side)
+        pg.run(err, st)
 
     steps = min(args.steps, 10)
     ms, _, clocks = timer.run(step, steps, min(args.warmup, 3))
-    weights = sum(O * K for O, K, _, _ in lin)
+
+    # the per-tensor calls, into the same planes
+    ws = {(6, 8): sbn.new_workspace(8, 64, 2, 4, dev), (2, 4): sbn.new_workspace(8, 64, 2, 4, dev)}
+    side = torch.cuda.Stream(device=dev)
+
+    def step_single(i, ev):
+        side.wait_stream(st)
+        for W, pw in zip(Ws, pg.packed):
+            for w in pw:
+                s_ = st if (w.n, w.m) == (6, 8) else side
+                sbn.sbn_quantize_mask_pack_weights(W, w.n, w.m, 1e-5, w.codes, w.meta,
+                                                   w.gamma_eff, ws[(w.n, w.m)], None, err, s_)
+        st.wait_stream(side)
+
+    ms_single, _, _ = timer.run(step_single, steps, min(args.warmup, 3))
+
+    # mask statistics of the step: natural zeros of every tensor, and keep-bit flips of both
+    # patterns against the previous step's masks (the masters before one update of
+    # N(0, 1e-3^2) noise, packed once here)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4000 + rank)
+    Wp = [(W.float() + torch.randn(W.shape, device=dev, generator=gen) * 1e-3).to(torch.bfloat16)
+          for W in Ws]
+    pg_prev = sbn.PackGroup(Wp, ((6, 8), (2, 4)), device=dev)
+    pg_prev.run(err, st)
+    torch.cuda.synchronize(dev)
+    pg_prev.Ws = []
+    del Wp
+    cnt = torch.zeros((len(Ws), 3), dtype=torch.int64, device=dev)
+
+    def step_stats(i, ev):
+        cnt.zero_()
+        for k, (W, pw, pp) in enumerate(zip(Ws, pg.packed, pg_prev.packed)):
+            sbn.sbn_count_zero_codes(W, pw[0].gamma_eff, cnt[k, 0:1], st)
+            for j in range(2):
+                sbn.sbn_count_mask_flips(pp[j].meta, pw[j].meta, pw[j].out, pw[j].in_, pw[j].n,
+                                         pw[j].m, cnt[k, 1 + j:2 + j], st)
+
+    ms_stats, _, _ = timer.run(step_stats, steps, min(args.warmup, 3))
+    tot = cnt.sum(dim=0).tolist()
+    weights = sum(W.numel() for W in Ws)
+    stats_bytes = weights * 2 + 2 * (weights // 8) + 2 * (weights // 8)
+    stats = {"ms_per_step": ms_stats, "GB/s": stats_bytes / (ms_stats * 1e-3) / 1e9,
+             "frac": stats_bytes / (ms_stats * 1e-3) / 1e9 / peaks["hbm"],
+             "natural_zeros": tot[0] / weights, "flips_6of8": tot[1] / weights,
+             "flips_2of4": tot[2] / weights, "launches_per_step": 3 * len(Ws),
+             "bytes_per_step": stats_bytes,
+             "what": "k_count_zero_codes on W (2 B/w) + k_count_mask_flips on both patterns' "
+                     "meta planes of two steps (2 x 0.125 B/w each)"}
     moved = weights * 2 * 2 + weights * 3 // 8 + weights // 4  # per pattern: read W + planes
     gbs = moved / (ms * 1e-3) / 1e9
     return {"value": gbs * world, "unit": "GB/s", "ms_per_step": ms, "steps": steps,
-            "roofline": hbm_roof(gbs, peaks, "quant_mask_pack, 130 tensors x (6:8, 2:4)"),
-            "gpu_launches": 2 * 2 * len(lin) * steps, "clocks": clocks,
-            "config": {"workload": "train-step-26x3200-6of8+2of4", "tensors": len(lin),
+            "roofline": hbm_roof(gbs, peaks, "k_abs_sum_group + k_qmp_group, 130 tensors x "
+                                 "(6:8, 2:4)",
+                                 unit_note="; algorithmic bytes count W once per pattern"),
+            "per_tensor_calls": {"ms_per_step": ms_single,
+                                 "GB/s": moved / (ms_single * 1e-3) / 1e9,
+                                 "launches_per_step": 2 * 2 * len(Ws)},
+            "mask_stats": stats,
+            "gpu_launches": 2 * steps, "clocks": clocks,
+            "config": {"workload": "train-step-26x3200-6of8+2of4", "tensors": len(Ws),
                        "weights": weights, "bytes_per_step": moved,
-                       "step": "every tensor packed in 6:8 (main stream) and 2:4 (side stream)"}}
+                       "step": "grouped pack of every tensor into 6:8 and 2:4 (sbn_quantize_"
+                               "mask_pack_weights_group)"}}
 
 
 # ---- next rows: backward, group quantisation, one-launch decode ----------------------------

@@ -117,6 +117,63 @@ SBN_API sbn_status sbn_quantize_mask_pack_weights(const void *W, int64_t out, in
                                           void *stream);
 
 /*
+ * Grouped pack: steps 1-4 for many master tensors in two launches, each tensor into one
+ * pattern or into both of 6:8 and 2:4 (the training-step re-mask of Sparse-BitNet section 2,
+ * "Recomputacion Dinamica": every step re-quantises and re-masks every linear from its
+ * masters).  Every output bit is that of sbn_quantize_mask_pack_weights for the tensor and
+ * pattern alone.  A tensor packed into two patterns is read twice in all (once for the
+ * absmean sum, once for both patterns' codes and metadata), not twice per pattern.
+ *
+ * Use: sbn_pack_group_sizes -> allocate a HOST plan buffer (16-byte aligned) and a device
+ * buffer of the same size, plus the device workspace, ZEROED once -> sbn_pack_group_plan
+ * fills the host plan -> copy it to the device -> sbn_quantize_mask_pack_weights_group as
+ * often as wanted (for instance after every optimizer step, masters updated in place).  The
+ * plan records device pointers: the buffers must stay allocated and in place while it is
+ * in use.
+ */
+typedef struct sbn_pack_group_tensor {
+  const void *W;          /* bf16 [out, in] masters, read only */
+  uint8_t *codes;         /* planes of the first pattern (n:m), sizes from sbn_linear_ref_dims */
+  uint8_t *meta;
+  uint8_t *codes2;        /* planes of the second pattern (n2:m2); NULL when m2 == 0 */
+  uint8_t *meta2;
+  float *gamma_eff;       /* one fp32, written: g, the same for both patterns */
+  int8_t *dense_dbg;      /* optional int8 [out, in] masked ternary matrix, first pattern */
+  int8_t *dense_dbg2;     /* optional, second pattern */
+  int64_t out, in;        /* shape rules of sbn_quantize_mask_pack_weights */
+  int32_t n, m;           /* 6:8 or 2:4 */
+  int32_t n2, m2;         /* the other of 6:8 / 2:4, or 0, 0 for one pattern */
+  float eps;              /* finite, >= 0 */
+  int32_t reserved;       /* set to 0 */
+} sbn_pack_group_tensor;
+
+/*
+ * Host only.  Validates the tensors (SBN_ERR_PATTERN for a pattern other than 6:8 / 2:4 or
+ * two equal patterns; SBN_ERR_SHAPE / NULL / ALIGN / ARG as sbn_quantize_mask_pack_weights;
+ * SBN_ERR_SHAPE for more than 65536 tensors) and returns the plan size and the device
+ * workspace size (16 bytes per tensor).
+ */
+SBN_API sbn_status sbn_pack_group_sizes(const sbn_pack_group_tensor *tensors, int32_t count,
+                                        int64_t *plan_bytes, int64_t *workspace_bytes);
+
+/* Host only.  Writes the plan into the HOST buffer `plan` (16-byte aligned, plan_bytes). */
+SBN_API sbn_status sbn_pack_group_plan(const sbn_pack_group_tensor *tensors, int32_t count,
+                                       void *plan, int64_t plan_bytes);
+
+/*
+ * Steps 1-4 for every tensor of the plan.
+ *   plan       the host plan; plan_dev the same bytes in device memory (16-byte aligned).
+ *   workspace  workspace_bytes of device memory, ZEROED by the caller before its first use;
+ *              every call leaves its counters at zero again, so it needs no clearing
+ *              between calls.  Calls that share a workspace must not overlap on the GPU.
+ *   err_flag   optional: SBN_FLAG_W_NONFINITE / SBN_FLAG_W_RANGE.
+ * SBN_ERR_ARG if `plan` is not a plan from sbn_pack_group_plan.
+ */
+SBN_API sbn_status sbn_quantize_mask_pack_weights_group(const void *plan, const void *plan_dev,
+                                                        void *workspace, int32_t *err_flag,
+                                                        void *stream);
+
+/*
  * The same computation as sbn_quantize_mask_pack_weights, for callers that cannot give
  * this library any device memory: plugin hosts that own every allocation and hand an
  * operator no workspace, or serving loops that forbid cudaMalloc/cudaFree on their hot

@@ -34,7 +34,8 @@ EXPORTED = ("sbn_linear_ref_dims", "sbn_quantize_mask_pack_weights", "sbn_quanti
             "sbn_operand_bytes", "sbn_expand_operand", "sbn_linear_operand",
             "sbn_backward_workspace_bytes", "sbn_backward", "sbn_quantize_linear",
             "sbn_gq_workspace_bytes", "sbn_quantize_mask_pack_weights_gq", "sbn_quantize_acts_gq",
-            "sbn_linear_gq")
+            "sbn_linear_gq", "sbn_pack_group_sizes", "sbn_pack_group_plan",
+            "sbn_quantize_mask_pack_weights_group")
 
 
 class SbnError(RuntimeError):
@@ -59,6 +60,16 @@ class SbnGroupLinear(ctypes.Structure):
                 ("out", ctypes.c_int64), ("in_", ctypes.c_int64), ("n", ctypes.c_int32),
                 ("m", ctypes.c_int32), ("y_is_bf16", ctypes.c_int32),
                 ("reserved", ctypes.c_int32)]
+
+
+class SbnPackGroupTensor(ctypes.Structure):
+    """One tensor of a grouped pack (sbn_pack_group_tensor in sbn.h)."""
+    _fields_ = [("W", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("meta", ctypes.c_void_p),
+                ("codes2", ctypes.c_void_p), ("meta2", ctypes.c_void_p),
+                ("gamma_eff", ctypes.c_void_p), ("dense_dbg", ctypes.c_void_p),
+                ("dense_dbg2", ctypes.c_void_p), ("out", ctypes.c_int64), ("in_", ctypes.c_int64),
+                ("n", ctypes.c_int32), ("m", ctypes.c_int32), ("n2", ctypes.c_int32),
+                ("m2", ctypes.c_int32), ("eps", ctypes.c_float), ("reserved", ctypes.c_int32)]
 
 
 _LIB = None
@@ -89,6 +100,12 @@ def lib():
         L.sbn_count_zero_codes.restype = i32
         L.sbn_count_mask_flips.argtypes = [p, p, i64, i64, i32, i32, p, p]
         L.sbn_count_mask_flips.restype = i32
+        L.sbn_pack_group_sizes.argtypes = [p, i32, p, p]
+        L.sbn_pack_group_sizes.restype = i32
+        L.sbn_pack_group_plan.argtypes = [p, i32, p, i64]
+        L.sbn_pack_group_plan.restype = i32
+        L.sbn_quantize_mask_pack_weights_group.argtypes = [p, p, p, p, p]
+        L.sbn_quantize_mask_pack_weights_group.restype = i32
         L.sbn_group_plan_sizes.argtypes = [p, i32, p, p]
         L.sbn_group_plan_sizes.restype = i32
         L.sbn_group_plan.argtypes = [p, i32, p, i64]
@@ -383,6 +400,83 @@ class GroupPlan:
 
     def linear(self, err_flag=None, stream=None):
         sbn_linear_group(self.plan_host, self.plan_dev, self.workspace, err_flag, stream)
+
+
+# ---- grouped pack (many tensors, 6:8 and/or 2:4) -----------------------------------------
+
+def sbn_pack_group_sizes(tensors):
+    """(plan_bytes, workspace_bytes) for a ctypes array of SbnPackGroupTensor."""
+    pb, wb = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().sbn_pack_group_sizes(ctypes.cast(tensors, ctypes.c_void_p), len(tensors),
+                                      ctypes.byref(pb), ctypes.byref(wb)), "sbn_pack_group_sizes")
+    return pb.value, wb.value
+
+
+def sbn_pack_group_plan(tensors, plan_host):
+    """Fill plan_host (a 16-byte aligned uint8 CPU tensor) with the plan of `tensors`."""
+    _check(lib().sbn_pack_group_plan(ctypes.cast(tensors, ctypes.c_void_p), len(tensors),
+                                     ctypes.c_void_p(plan_host.data_ptr()), plan_host.numel()),
+           "sbn_pack_group_plan")
+
+
+def sbn_quantize_mask_pack_weights_group(plan_host, plan_dev, workspace, err_flag=None,
+                                         stream=None):
+    _check(lib().sbn_quantize_mask_pack_weights_group(
+        ctypes.c_void_p(plan_host.data_ptr()), _ptr(plan_dev), _ptr(workspace), _ptr(err_flag),
+        _stream(stream)), "sbn_quantize_mask_pack_weights_group")
+
+
+class PackGroup:
+    """A grouped pack: every master tensor of `Ws` (bf16 [O, K] CUDA tensors) into each
+    pattern of `patterns` (one or two of (6, 8) and (2, 4)), in two launches per call.
+    Allocates the outputs: ``packed[i][j]`` is tensor i's PackedWeights for patterns[j]
+    (both patterns share one gamma_eff).  ``dense_dbg`` optionally gives, per tensor, a
+    list of int8 [O, K] tensors (or None) per pattern.  The masters may change between
+    calls (in place); the plan keeps their pointers."""
+
+    def __init__(self, Ws, patterns=((6, 8), (2, 4)), eps=1e-5, dense_dbg=None, device=None):
+        if len(patterns) not in (1, 2):
+            raise ValueError("one or two patterns")
+        device = device if device is not None else Ws[0].device
+        self.Ws, self.patterns, self.packed = list(Ws), tuple(patterns), []
+        arr = (SbnPackGroupTensor * len(self.Ws))()
+        for i, W in enumerate(self.Ws):
+            out, in_ = W.shape
+            gamma = torch.empty(1, dtype=torch.float32, device=device)
+            pw = []
+            for (n, m) in self.patterns:
+                d = sbn_linear_ref_dims(out, in_, n, m)
+                pw.append(PackedWeights(
+                    torch.empty((out, d.codes_ld), dtype=torch.uint8, device=device),
+                    torch.empty((out, d.meta_ld), dtype=torch.uint8, device=device),
+                    gamma, out, in_, n, m))
+            self.packed.append(pw)
+            dd = (dense_dbg[i] if dense_dbg is not None else None) or [None, None]
+            two = len(pw) == 2
+            arr[i] = SbnPackGroupTensor(
+                W=_ptr(W), codes=_ptr(pw[0].codes), meta=_ptr(pw[0].meta),
+                codes2=_ptr(pw[1].codes) if two else None, meta2=_ptr(pw[1].meta) if two else None,
+                gamma_eff=_ptr(gamma), dense_dbg=_ptr(dd[0]),
+                dense_dbg2=_ptr(dd[1]) if two and len(dd) > 1 else None, out=out, in_=in_,
+                n=self.patterns[0][0], m=self.patterns[0][1],
+                n2=self.patterns[1][0] if two else 0, m2=self.patterns[1][1] if two else 0,
+                eps=eps, reserved=0)
+        self._arr = arr
+        pb, wb = sbn_pack_group_sizes(arr)
+        raw = torch.empty(pb + 16, dtype=torch.uint8)
+        off = (-raw.data_ptr()) % 16
+        self.plan_host = raw[off:off + pb]
+        self._raw = raw
+        sbn_pack_group_plan(arr, self.plan_host)
+        self.plan_dev = self.plan_host.to(device)
+        self.workspace = torch.zeros(max(wb, 16), dtype=torch.uint8, device=device)
+        hdr = self.plan_host[:20].numpy().view("int32")
+        self.total_chunks, self.total_q = int(hdr[2]) & 0xffffffff, int(hdr[3]) & 0xffffffff
+        self.mode = int(hdr[4])  # 0 / 1 / 2: the fixed-pattern kernel; -1: the general one
+
+    def run(self, err_flag=None, stream=None):
+        sbn_quantize_mask_pack_weights_group(self.plan_host, self.plan_dev, self.workspace,
+                                             err_flag, stream)
 
 
 # ---- tensor-core operand (2:4, many tokens) ----------------------------------------------

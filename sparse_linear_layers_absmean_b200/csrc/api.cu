@@ -74,6 +74,47 @@ sbn_status check_plan(const void *plan, const void *plan_dev) {
   return SBN_OK;
 }
 
+bool fast_pattern(int n, int m) { return (n == 6 && m == 8) || (n == 2 && m == 4); }
+
+sbn_status check_pack_group(const sbn_pack_group_tensor *ts, int32_t count) {
+  if (count < 0 || count > sbn::kPackGroupMaxTensors) return SBN_ERR_SHAPE;
+  if (count > 0 && !ts) return SBN_ERR_NULL;
+  uint64_t total_q = 0;
+  for (int32_t i = 0; i < count; ++i) {
+    const sbn_pack_group_tensor &t = ts[i];
+    sbn_dims d;
+    sbn_status st = sbn_linear_ref_dims(t.out, t.in, t.n, t.m, &d);
+    if (st != SBN_OK) return st;
+    if (!fast_pattern(t.n, t.m)) return SBN_ERR_PATTERN;
+    const bool two = t.m2 != 0 || t.n2 != 0;
+    if (two && (!fast_pattern(t.n2, t.m2) || (t.n2 == t.n && t.m2 == t.m))) return SBN_ERR_PATTERN;
+    if (!std::isfinite(t.eps) || t.eps < 0.0f) return SBN_ERR_ARG;
+    if (!t.W || !t.codes || !t.meta || !t.gamma_eff) return SBN_ERR_NULL;
+    if (two && (!t.codes2 || !t.meta2)) return SBN_ERR_NULL;
+    if (!aligned16(t.W) || !aligned16(t.codes) || !aligned16(t.meta) ||
+        (t.dense_dbg && !aligned16(t.dense_dbg)) ||
+        (two && (!aligned16(t.codes2) || !aligned16(t.meta2) ||
+                 (t.dense_dbg2 && !aligned16(t.dense_dbg2)))) ||
+        (reinterpret_cast<uintptr_t>(t.gamma_eff) & 3u))
+      return SBN_ERR_ALIGN;
+    total_q += (uint64_t)((t.out * t.in / 64 + 7) / 8);
+  }
+  if (total_q >= (1ull << 32)) return SBN_ERR_SHAPE;
+  return SBN_OK;
+}
+
+// One pattern's arguments for the shared per-lane pack routine.
+sbn::FastPackArgs pack_args(const void *W, int64_t out, int64_t in, int n, int m, float eps,
+                            uint8_t *codes, uint8_t *meta, int8_t *dense_dbg, float *gamma_eff) {
+  sbn_dims d;
+  fill_dims(out, in, n, m, &d);
+  const uint32_t bpr = (uint32_t)(in / 64);
+  return sbn::FastPackArgs{reinterpret_cast<const uint4 *>(W), out * in / 64, bpr,
+                           sbn::make_fast_div(bpr), nullptr, codes, d.codes_ld,
+                           d.codes_row_bytes, meta, d.meta_ld, d.meta_row_bytes, dense_dbg,
+                           0, out * in, eps, gamma_eff};
+}
+
 }  // namespace
 
 extern "C" {
@@ -358,6 +399,83 @@ sbn_status sbn_linear_gq(const int8_t *Xq, const float *absmax, const uint8_t *c
                                d.codes_ld, d.meta_ld, Y, y_is_bf16,
                                static_cast<float *>(workspace), acc_dbg, err_flag,
                                static_cast<cudaStream_t>(stream));
+}
+
+sbn_status sbn_pack_group_sizes(const sbn_pack_group_tensor *tensors, int32_t count,
+                               int64_t *plan_bytes, int64_t *workspace_bytes) {
+  if (!plan_bytes || !workspace_bytes) return SBN_ERR_NULL;
+  sbn_status st = check_pack_group(tensors, count);
+  if (st != SBN_OK) return st;
+  *plan_bytes = sbn::pack_group_plan_bytes(count);
+  *workspace_bytes = (int64_t)count * (int64_t)sizeof(sbn::PackGroupSlot);
+  return SBN_OK;
+}
+
+sbn_status sbn_pack_group_plan(const sbn_pack_group_tensor *tensors, int32_t count, void *plan,
+                               int64_t plan_bytes) {
+  if (!plan) return SBN_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(plan) & 15u) return SBN_ERR_ALIGN;
+  sbn_status st = check_pack_group(tensors, count);
+  if (st != SBN_OK) return st;
+  if (plan_bytes < sbn::pack_group_plan_bytes(count)) return SBN_ERR_ARG;
+  auto *hd = static_cast<sbn::PackGroupHeader *>(plan);
+  auto *T = reinterpret_cast<sbn::PackGroupTensor *>(hd + 1);
+  std::memset(hd, 0, sizeof(*hd));
+  uint32_t chunk = 0, q = 0;
+  int mode = -2;  // not yet known
+  for (int32_t i = 0; i < count; ++i) {
+    const sbn_pack_group_tensor &t = tensors[i];
+    sbn::PackGroupTensor e;
+    std::memset(&e, 0, sizeof(e));
+    if (t.m2 != 0) {  // both patterns: 6:8 into pa, 2:4 into pb, whichever order was asked
+      const bool first68 = t.m == 8;
+      e.pa = first68 ? pack_args(t.W, t.out, t.in, 6, 8, t.eps, t.codes, t.meta, t.dense_dbg,
+                                 t.gamma_eff)
+                     : pack_args(t.W, t.out, t.in, 6, 8, t.eps, t.codes2, t.meta2, t.dense_dbg2,
+                                 t.gamma_eff);
+      e.pb = first68 ? pack_args(t.W, t.out, t.in, 2, 4, t.eps, t.codes2, t.meta2, t.dense_dbg2,
+                                 t.gamma_eff)
+                     : pack_args(t.W, t.out, t.in, 2, 4, t.eps, t.codes, t.meta, t.dense_dbg,
+                                 t.gamma_eff);
+      e.pa_compact = 0;
+      e.pb_compact = 1;
+    } else {
+      e.pa = pack_args(t.W, t.out, t.in, t.n, t.m, t.eps, t.codes, t.meta, t.dense_dbg,
+                       t.gamma_eff);
+      e.pa_compact = t.n == 2;
+    }
+    const int tmode = (t.dense_dbg || t.dense_dbg2) ? -1 : (t.m2 != 0 ? 2 : (t.n == 2 ? 1 : 0));
+    mode = mode == -2 ? tmode : (mode == tmode ? mode : -1);
+    e.nvec = t.out * t.in / 8;
+    e.chunk_begin = chunk;
+    e.nchunks = (uint32_t)((e.nvec + sbn::kPackGroupChunkVecs - 1) / sbn::kPackGroupChunkVecs);
+    e.q_begin = q;
+    e.nq = (uint32_t)((e.pa.nblocks + 7) / 8);
+    chunk += e.nchunks;
+    q += e.nq;
+    std::memcpy(&T[i], &e, sizeof(e));
+  }
+  hd->magic = sbn::kPackGroupMagic;
+  hd->count = count;
+  hd->total_chunks = chunk;
+  hd->total_q = q;
+  hd->mode = mode < 0 ? -1 : mode;
+  return SBN_OK;
+}
+
+sbn_status sbn_quantize_mask_pack_weights_group(const void *plan, const void *plan_dev,
+                                                void *workspace, int32_t *err_flag,
+                                                void *stream) {
+  if (!plan || !plan_dev) return SBN_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(plan) & 15u) || (reinterpret_cast<uintptr_t>(plan_dev) & 15u) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 15u) || (reinterpret_cast<uintptr_t>(err_flag) & 3u))
+    return SBN_ERR_ALIGN;
+  const auto *hd = static_cast<const sbn::PackGroupHeader *>(plan);
+  if (hd->magic != sbn::kPackGroupMagic) return SBN_ERR_ARG;
+  if (hd->count == 0) return SBN_OK;
+  if (!workspace) return SBN_ERR_NULL;
+  return sbn::launch_pack_group(hd, plan_dev, static_cast<sbn::PackGroupSlot *>(workspace),
+                                err_flag, static_cast<cudaStream_t>(stream));
 }
 
 sbn_status sbn_count_zero_codes(const void *W, const float *gamma_eff, int64_t out, int64_t in,

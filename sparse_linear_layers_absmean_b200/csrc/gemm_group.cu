@@ -337,7 +337,6 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
           const uint8_t *slot1 = ring1 + s1 * Cfg::kSlot1;
           const int nb = min(kSuper, nkb - b0);
           for (int g = 0; g < nb; ++g) {
-            const int b = b0 + g;
             const uint32_t e_col = tmem + (uint32_t)(Cfg::kMetaCol + s2 * Cfg::kMColsPerSlot + 4 * g);
             const uint32_t a_col = tmem + (uint32_t)(Cfg::kACol + s2 * Cfg::kAColsPerSlot + 16 * g);
             const uint32_t b_addr = ptx::smem_u32(slot1 + 2 * Cfg::kPlane + g * Cfg::kBBytes);

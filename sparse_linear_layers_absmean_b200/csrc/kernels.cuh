@@ -59,6 +59,41 @@ struct FastPackArgs {
 // launch after k_abs_sum left a.nparts partial sums in a.ws.
 sbn_status launch_fast_pack(const FastPackArgs &a, bool compact, cudaStream_t st);
 
+// Grouped pack: many tensors, one or two of the fast patterns each, in two launches.
+// Plan in device memory: a PackGroupHeader, then one PackGroupTensor per tensor.  The
+// workspace holds one PackGroupSlot per tensor, zeroed before first use and left zeroed.
+constexpr int kPackGroupMaxTensors = 1 << 16;
+constexpr int64_t kPackGroupChunkVecs = 16384;  // 16-byte vectors per k_abs_sum_group chunk
+constexpr uint32_t kPackGroupMagic = 0x31475053u;  // "SPG1"
+struct PackGroupHeader {
+  uint32_t magic;
+  int32_t count;
+  uint32_t total_chunks;  // k_abs_sum_group chunks over all tensors
+  uint32_t total_q;       // k_qmp_group warp-iterations (8 blocks of 64 weights each)
+  int32_t mode;           // every tensor 6:8 only (0), 2:4 only (1), both (2); mixed: -1
+  uint32_t reserved[11];
+};
+static_assert(sizeof(PackGroupHeader) == 64, "plan header layout");
+struct PackGroupTensor {
+  FastPackArgs pa;      // first pattern (pa.W, pa.n, pa.eps, pa.gamma_eff used by both);
+                        // 6:8 when the tensor packs both patterns
+  FastPackArgs pb;      // second pattern (2:4); pb.codes == nullptr when the tensor has one
+  int64_t nvec;         // 16-byte vectors of W
+  uint32_t chunk_begin, nchunks;
+  uint32_t q_begin, nq;
+  int32_t pa_compact, pb_compact;  // 1: 2:4, 0: 6:8
+};
+static_assert(sizeof(PackGroupTensor) % 16 == 0, "plan entries stay 16-byte aligned");
+struct PackGroupSlot {
+  unsigned long long S;  // exact sum, accumulated by the chunks
+  unsigned int done;     // chunks finished
+  unsigned int thr;      // code threshold, written by the last chunk
+};
+
+int64_t pack_group_plan_bytes(int count);
+sbn_status launch_pack_group(const PackGroupHeader *hdr_host, const void *plan_dev,
+                             PackGroupSlot *slots, int32_t *err_flag, cudaStream_t st);
+
 sbn_status launch_pack(const void *W, int64_t out, int64_t in, int n, int m, float eps,
                        uint8_t *codes, int64_t ldc, int64_t crow, uint8_t *meta, int64_t ldm,
                        int64_t mrow, float *gamma_eff, PackWorkspace *ws, int8_t *dense_dbg,

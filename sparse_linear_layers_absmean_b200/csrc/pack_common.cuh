@@ -55,6 +55,16 @@ __device__ __forceinline__ uint32_t code_threshold_warp(float g, int lane) {
   return hi;
 }
 
+// g = fp32(gamma + eps) with gamma = fp32(fp64(S) / (fp64(n) * 2^24)), S the exact sum of
+// trunc(|W| * 2^24) over the n weights, and the code threshold for that g.  Called by all
+// 32 lanes of one warp; every lane returns both.
+__device__ __forceinline__ uint32_t scale_from_sum(unsigned long long S, int64_t n, float eps,
+                                                   int lane, float &g) {
+  const double mean = __ddiv_rn(__ull2double_rn(S), (double)n * 16777216.0);
+  g = __fadd_rn(__double2float_rn(mean), eps);
+  return code_threshold_warp(g, lane);
+}
+
 // Run by every thread of a CTA at the start of a quant/mask/pack kernel.  Returns the code
 // threshold; CTA 0 also publishes g = fp32(gamma + eps) to *gamma_eff, where
 // gamma = fp32(fp64(S) / (fp64(n) * 2^24)) and S is the exact sum of the partials.  All
@@ -73,9 +83,8 @@ __device__ __forceinline__ uint32_t pack_prologue(const PackWorkspace *ws, int n
     const int lane = threadIdx.x;
     S = lane < (int)(blockDim.x >> 5) ? s_part[lane] : 0ull;
     S = warp_sum_u64(S);
-    const double mean = __ddiv_rn(__ull2double_rn(S), (double)n * 16777216.0);
-    const float g = __fadd_rn(__double2float_rn(mean), eps);
-    const uint32_t thr = code_threshold_warp(g, lane);
+    float g;
+    const uint32_t thr = scale_from_sum(S, n, eps, lane, g);
     if (lane == 0) {
       s_thr = thr;
       if (blockIdx.x == 0) *gamma_eff = g;

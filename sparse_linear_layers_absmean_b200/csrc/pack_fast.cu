@@ -160,76 +160,126 @@ __device__ __forceinline__ void pk_load(const uint4 *W, uint32_t nb, uint32_t b,
   }
 }
 
+// The flags every pattern uses, from one lane's 16 weights (w[i] = weights 2i, 2i+1): N
+// "code non-zero" and S "negative", byte-top, for weights 4i..4i+3 in N[i] / S[i].
+struct LaneFlags {
+  uint32_t N[4], S[4];
+};
+__device__ __forceinline__ LaneFlags lane_flags(const uint32_t *w, uint32_t thr2) {
+  LaneFlags f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f.N[i] = __byte_perm(nonzero_flags(w[2 * i], thr2), nonzero_flags(w[2 * i + 1], thr2), 0x7531);
+    f.S[i] = __byte_perm(w[2 * i], w[2 * i + 1], 0x7531);
+  }
+  return f;
+}
+
+// One pattern's result for a lane: keep flags (byte-top, weights 4i..4i+3 in K[i]), the
+// lane's code word and its 16 metadata bits.
+struct LanePack {
+  uint32_t K[4], word, meta16;
+};
+
+// 2:4: the lane's 16 weights are two 8-weight halves of one 32-bit code word (kept elements
+// 8s..8s+7 of the block); lanes s and s^1 exchange halves, so both hold the whole word.
+__device__ __forceinline__ LanePack pack_lane_2of4(const uint32_t *w, const LaneFlags &f,
+                                                   const uint32_t *s_pair, int s) {
+  LanePack r;
+  r.K[0] = keep_2of4(w[0], w[1]);
+  r.K[1] = keep_2of4(w[2], w[3]);
+  r.K[2] = keep_2of4(w[4], w[5]);
+  r.K[3] = keep_2of4(w[6], w[7]);
+  const uint32_t eAB = s_pair[top_bits_to_byte(r.K[0], r.K[1])];
+  const uint32_t eCD = s_pair[top_bits_to_byte(r.K[2], r.K[3])];
+  r.meta16 = (eAB & 0xffu) | ((eCD & 0xffu) << 8);
+  const uint32_t selAB = eAB >> 8, selCD = eCD >> 8;
+  // kept weights in order: stored elements 8s..8s+7 = (A.first, A.second, B.first,
+  // B.second | C.first, ..., D.second): j = 2*(s&1) (+1 for C, D), byte k = position
+  const int js = 4 * (s & 1);
+  const uint32_t LAB = __byte_perm(f.N[0], f.N[1], selAB) & kTop;
+  const uint32_t HAB = LAB & __byte_perm(f.S[0], f.S[1], selAB);
+  const uint32_t LCD = __byte_perm(f.N[2], f.N[3], selCD) & kTop;
+  const uint32_t HCD = LCD & __byte_perm(f.S[2], f.S[3], selCD);
+  uint32_t word = (HAB >> js) | (LAB >> (1 + js)) | (HCD >> (2 + js)) | (LCD >> (3 + js));
+  r.word = word | __shfl_xor_sync(0xffffffffu, word, 1);
+  return r;
+}
+
+// 6:8: the lane's 16 weights are the 16 elements of one code word (word s of the block).
+__device__ __forceinline__ LanePack pack_lane_6of8(const uint32_t *w, const LaneFlags &f) {
+  LanePack r;
+  keep_6of8(w, r.K[0], r.K[1]);
+  keep_6of8(w + 4, r.K[2], r.K[3]);
+  r.meta16 = top_bits_to_byte(r.K[0], r.K[1]) | (top_bits_to_byte(r.K[2], r.K[3]) << 8);
+  const uint32_t L0 = f.N[0] & r.K[0], L1 = f.N[1] & r.K[1], L2 = f.N[2] & r.K[2],
+                 L3 = f.N[3] & r.K[3];
+  const uint32_t H0 = L0 & f.S[0], H1 = L1 & f.S[1], H2 = L2 & f.S[2], H3 = L3 & f.S[3];
+  // weights e = 0..15 of this lane are elements 16s+e of the block: word s, byte e%4,
+  // bits (7,6) - 2*(e/4) for (negative, non-zero)
+  r.word = H0 | (L0 >> 1) | (H1 >> 2) | (L1 >> 3) | (H2 >> 4) | (L2 >> 5) | (H3 >> 6) | (L3 >> 7);
+  return r;
+}
+
+// Where one pattern's planes go: the plane pointers and row strides (multiples of 16).
+// Every row's data is a multiple of 8 bytes, so a row either fills its stride or ends 8
+// bytes short of it; bit 0 of ldc / ldm marks the second case (those 8 bytes are zeroed).
+struct PlaneOut {
+  uint8_t *codes, *meta;
+  uint32_t ldc, ldm;
+};
+__device__ __forceinline__ PlaneOut plane_out(const FastPackArgs &a) {
+  return PlaneOut{a.codes, a.meta, (uint32_t)a.ldc | (a.codes_row_bytes != a.ldc ? 1u : 0u),
+                  (uint32_t)a.ldm | (a.meta_row_bytes != a.ldm ? 1u : 0u)};
+}
+
+// Stores a lane's part of block (row, col) of one pattern: code word, metadata bits and
+// the row padding (by the row's last block).
+template <bool kCompact>
+__device__ __forceinline__ void store_lane(const PlaneOut &o, const LanePack &r, uint32_t row,
+                                           uint32_t col, bool row_end, int s) {
+  const uint32_t ldc = o.ldc & ~1u, ldm = o.ldm & ~1u;
+  uint8_t *crow = o.codes + (uint64_t)row * ldc;
+  uint8_t *mrow = o.meta + (uint64_t)row * ldm;
+  if constexpr (kCompact) {
+    if ((s & 1) == 0) reinterpret_cast<uint32_t *>(crow + col * 8)[s >> 1] = r.word;
+  } else {
+    reinterpret_cast<uint32_t *>(crow + col * 16)[s] = r.word;
+  }
+  reinterpret_cast<uint16_t *>(mrow + col * 8)[s] = (uint16_t)r.meta16;
+  if (row_end && s == 0) {
+    if (o.ldc & 1u) *reinterpret_cast<uint2 *>(crow + ldc - 8) = make_uint2(0u, 0u);
+    if (o.ldm & 1u) *reinterpret_cast<uint2 *>(mrow + ldm - 8) = make_uint2(0u, 0u);
+  }
+}
+
+// The optional masked ternary matrix: the lane's 16 int8 values of block b.
+__device__ __forceinline__ void store_dense(int8_t *dense, const LaneFlags &f, const LanePack &r,
+                                            uint32_t b, int s) {
+  const uint32_t l0 = f.N[0] & r.K[0], l1 = f.N[1] & r.K[1], l2 = f.N[2] & r.K[2],
+                 l3 = f.N[3] & r.K[3];
+  *reinterpret_cast<uint4 *>(dense + (uint64_t)b * 64 + 16 * s) =
+      make_uint4(flags_to_i8(l0, l0 & f.S[0]), flags_to_i8(l1, l1 & f.S[1]),
+                 flags_to_i8(l2, l2 & f.S[2]), flags_to_i8(l3, l3 & f.S[3]));
+}
+
 // One lane's 16 weights: keep masks, metadata, codes.
 template <bool kCompact>
 __device__ __forceinline__ void qmp_unit(const FastPackArgs &a, const uint32_t *s_pair, uint4 v0,
                                          uint4 v1, uint32_t b, int s, uint32_t thr2) {
   const bool valid = b < (uint32_t)a.nblocks;  // both lanes of a shuffle pair share the block
   const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-  // keep flags of weights 0-3, 4-7, 8-11, 12-15 (byte-top) and the metadata bits
-  uint32_t K0, K1, K2, K3, meta16, selAB = 0, selCD = 0;
-  if constexpr (kCompact) {
-    K0 = keep_2of4(w[0], w[1]);
-    K1 = keep_2of4(w[2], w[3]);
-    K2 = keep_2of4(w[4], w[5]);
-    K3 = keep_2of4(w[6], w[7]);
-    const uint32_t eAB = s_pair[top_bits_to_byte(K0, K1)];
-    const uint32_t eCD = s_pair[top_bits_to_byte(K2, K3)];
-    meta16 = (eAB & 0xffu) | ((eCD & 0xffu) << 8);
-    selAB = eAB >> 8;
-    selCD = eCD >> 8;
-  } else {
-    keep_6of8(w, K0, K1);
-    keep_6of8(w + 4, K2, K3);
-    meta16 = top_bits_to_byte(K0, K1) | (top_bits_to_byte(K2, K3) << 8);
-  }
-  const uint32_t N0 = __byte_perm(nonzero_flags(w[0], thr2), nonzero_flags(w[1], thr2), 0x7531);
-  const uint32_t N1 = __byte_perm(nonzero_flags(w[2], thr2), nonzero_flags(w[3], thr2), 0x7531);
-  const uint32_t N2 = __byte_perm(nonzero_flags(w[4], thr2), nonzero_flags(w[5], thr2), 0x7531);
-  const uint32_t N3 = __byte_perm(nonzero_flags(w[6], thr2), nonzero_flags(w[7], thr2), 0x7531);
-  const uint32_t S0 = __byte_perm(w[0], w[1], 0x7531), S1 = __byte_perm(w[2], w[3], 0x7531);
-  const uint32_t S2 = __byte_perm(w[4], w[5], 0x7531), S3 = __byte_perm(w[6], w[7], 0x7531);
-  uint32_t word;
-  if constexpr (kCompact) {
-    // kept weights in order: stored elements 8s..8s+7 = (A.first, A.second, B.first,
-    // B.second | C.first, ..., D.second): j = 2*(s&1) (+1 for C, D), byte k = position
-    const int js = 4 * (s & 1);
-    const uint32_t LAB = __byte_perm(N0, N1, selAB) & kTop;
-    const uint32_t HAB = LAB & __byte_perm(S0, S1, selAB);
-    const uint32_t LCD = __byte_perm(N2, N3, selCD) & kTop;
-    const uint32_t HCD = LCD & __byte_perm(S2, S3, selCD);
-    word = (HAB >> js) | (LAB >> (1 + js)) | (HCD >> (2 + js)) | (LCD >> (3 + js));
-    word |= __shfl_xor_sync(0xffffffffu, word, 1);
-  } else {
-    const uint32_t L0 = N0 & K0, L1 = N1 & K1, L2 = N2 & K2, L3 = N3 & K3;
-    const uint32_t H0 = L0 & S0, H1 = L1 & S1, H2 = L2 & S2, H3 = L3 & S3;
-    // weights e = 0..15 of this lane are elements 16s+e of the block: word s, byte e%4,
-    // bits (7,6) - 2*(e/4) for (negative, non-zero)
-    word = H0 | (L0 >> 1) | (H1 >> 2) | (L1 >> 3) | (H2 >> 4) | (L2 >> 5) | (H3 >> 6) | (L3 >> 7);
-  }
+  const LaneFlags f = lane_flags(w, thr2);
+  LanePack r;
+  if constexpr (kCompact)
+    r = pack_lane_2of4(w, f, s_pair, s);
+  else
+    r = pack_lane_6of8(w, f);
   if (!valid) return;
   const uint32_t row = fast_div(b, a.div_bpr);
   const uint32_t col = b - row * a.bpr;
-  uint8_t *crow = a.codes + (int64_t)row * a.ldc;
-  uint8_t *mrow = a.meta + (int64_t)row * a.ldm;
-  if constexpr (kCompact) {
-    if ((s & 1) == 0) reinterpret_cast<uint32_t *>(crow + col * 8)[s >> 1] = word;
-  } else {
-    reinterpret_cast<uint32_t *>(crow + col * 16)[s] = word;
-  }
-  reinterpret_cast<uint16_t *>(mrow + col * 8)[s] = (uint16_t)meta16;
-  if (col == a.bpr - 1 && s == 0) {  // zero the row padding
-    if (a.ldc > a.codes_row_bytes)
-      *reinterpret_cast<uint2 *>(crow + a.codes_row_bytes) = make_uint2(0u, 0u);
-    if (a.ldm > a.meta_row_bytes)
-      *reinterpret_cast<uint2 *>(mrow + a.meta_row_bytes) = make_uint2(0u, 0u);
-  }
-  if (a.dense_dbg) {
-    const uint32_t l0 = N0 & K0, l1 = N1 & K1, l2 = N2 & K2, l3 = N3 & K3;
-    *reinterpret_cast<uint4 *>(a.dense_dbg + (uint64_t)b * 64 + 16 * s) =
-        make_uint4(flags_to_i8(l0, l0 & S0), flags_to_i8(l1, l1 & S1), flags_to_i8(l2, l2 & S2),
-                   flags_to_i8(l3, l3 & S3));
-  }
+  store_lane<kCompact>(plane_out(a), r, row, col, col == a.bpr - 1, s);
+  if (a.dense_dbg) store_dense(a.dense_dbg, f, r, b, s);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -292,6 +342,297 @@ sbn_status launch_fast_pack(const FastPackArgs &a, bool compact, cudaStream_t st
     return SBN_ERR_CUDA;
   }
   return SBN_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// Grouped pack (many tensors, each packed into one or two of the patterns above).
+//
+// k_abs_sum_group streams every tensor's W in chunks of kPackGroupChunkVecs 16-byte
+// vectors (256 KB), CTAs striding over the chunks of all tensors.  Each chunk's exact
+// partial sum goes into its tensor's slot with one 64-bit atomic add (integer: the order
+// of the adds cannot change S); the CTA that finishes a tensor's last chunk turns S into g
+// and the code threshold, publishes them, and clears the slot for the next call.
+// k_qmp_group then re-reads W once and writes both patterns' planes from the same words:
+// a tensor asked for 6:8 and 2:4 is read twice in all, not four times.
+// ---------------------------------------------------------------------------------------
+constexpr int kAgThreads = 256;
+constexpr int kAgLoads = 4;
+static_assert(kPackGroupChunkVecs % (kAgThreads * kAgLoads) == 0, "whole iterations per chunk");
+
+__global__ void __launch_bounds__(kAgThreads, 4)
+    k_abs_sum_group(const PackGroupHeader *__restrict__ hdr, const PackGroupTensor *__restrict__ T,
+                    PackGroupSlot *slots, int32_t *err_flag) {
+  ptx::grid_dep_wait();  // the previous kernel on the stream may have written W
+  ptx::grid_dep_launch();
+  __shared__ unsigned long long s_sum[kAgThreads / 32];
+  __shared__ uint32_t s_all[kAgThreads / 32], s_fin[kAgThreads / 32];
+  __shared__ int s_last;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t total = hdr->total_chunks;
+  int t = 0;  // chunks ascend per CTA, so the tensor index only moves forward
+  for (uint32_t c = blockIdx.x; c < total; c += gridDim.x) {
+    while (c >= T[t].chunk_begin + T[t].nchunks) ++t;
+    const uint4 *W = T[t].pa.W;
+    const int64_t v0 = (int64_t)(c - T[t].chunk_begin) * kPackGroupChunkVecs;
+    const int64_t v1 = min(v0 + kPackGroupChunkVecs, T[t].nvec);
+    double acc0 = kAccBias, acc1 = kAccBias;
+    uint32_t mx = 0;
+    for (int64_t i = v0 + threadIdx.x; i < v1; i += kAgLoads * kAgThreads) {
+      uint4 v[kAgLoads];
+#pragma unroll
+      for (int u = 0; u < kAgLoads; ++u)
+        v[u] = i + u * kAgThreads < v1 ? __ldg(W + i + u * kAgThreads) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int u = 0; u < kAgLoads; ++u) {
+        const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          asm("max.u16x2 %0, %0, %1;" : "+r"(mx) : "r"(w4[q] & 0x7fff7fffu));
+          acc0 = __dadd_rz(acc0, mag_lo_x2p128(w4[q]));
+          acc1 = __dadd_rz(acc1, mag_hi_x2p128(w4[q]));
+        }
+      }
+    }
+    unsigned long long acc = acc_value(acc0) + acc_value(acc1);
+    uint32_t mx_all = 0, mx_fin = 0;
+    if (max(mx & 0xffffu, mx >> 16) >= kBf16Mag256Bits) {  // rare: tell NaN/Inf from range
+      for (int64_t j = v0 + threadIdx.x; j < v1; j += kAgThreads) {
+        const uint4 v = __ldg(W + j);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        for (int q = 0; q < 4; ++q)
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t m = (w4[q] >> (16 * h)) & 0x7fffu;
+            mx_all = max(mx_all, m);
+            if (m < kBf16InfBits) mx_fin = max(mx_fin, m);
+          }
+      }
+    }
+    acc = warp_sum_u64(acc);
+    mx_all = warp_max_u32(mx_all);
+    mx_fin = warp_max_u32(mx_fin);
+    if (lane == 0) {
+      s_sum[warp] = acc;
+      s_all[warp] = mx_all;
+      s_fin[warp] = mx_fin;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      unsigned long long sum = 0;
+      uint32_t a = 0, f = 0;
+      for (int w = 0; w < kAgThreads / 32; ++w) {
+        sum += s_sum[w];
+        a = max(a, s_all[w]);
+        f = max(f, s_fin[w]);
+      }
+      int flags = 0;
+      if (a >= kBf16InfBits) flags |= SBN_FLAG_W_NONFINITE;
+      if (f >= kBf16Mag256Bits) flags |= SBN_FLAG_W_RANGE;
+      if (flags && err_flag) atomicOr(err_flag, flags);
+      atomicAdd(&slots[t].S, sum);
+      __threadfence();  // the add is visible before the chunk counts as done
+      const unsigned int prev = atomicAdd(&slots[t].done, 1u);
+      s_last = prev == T[t].nchunks - 1;
+    }
+    __syncthreads();
+    if (s_last && warp == 0) {  // every chunk of tensor t is in S
+      __threadfence();
+      unsigned long long S = 0;
+      if (lane == 0) S = atomicExch(&slots[t].S, 0ull);  // read and clear
+      S = __shfl_sync(0xffffffffu, S, 0);
+      float g;
+      const uint32_t thr = scale_from_sum(S, T[t].pa.n, T[t].pa.eps, lane, g);
+      if (lane == 0) {
+        *T[t].pa.gamma_eff = g;
+        slots[t].thr = thr;
+        slots[t].done = 0u;
+      }
+    }
+    __syncthreads();  // s_sum and s_last are reused by the next chunk
+  }
+}
+
+__device__ __forceinline__ void qg_advance(const PackGroupTensor *__restrict__ T, int &t,
+                                           uint32_t q) {
+  while (q >= T[t].q_begin + T[t].nq) ++t;
+}
+
+__global__ void __launch_bounds__(kPkThreads, kPkCtasPerSm)
+    k_qmp_group(const PackGroupHeader *__restrict__ hdr, const PackGroupTensor *__restrict__ T,
+                const PackGroupSlot *__restrict__ slots) {
+  __shared__ uint32_t s_pair[256];
+  ptx::grid_dep_launch();
+  s_pair[threadIdx.x] = pair_entry(threadIdx.x);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int s = lane & 3;
+  const uint32_t sub = lane >> 2;
+  const uint32_t nq = hdr->total_q;
+  const uint32_t qstep = gridDim.x * (kPkThreads / 32);
+  uint32_t q = blockIdx.x * (kPkThreads / 32) + warp;  // warp-uniform
+  int t = 0;
+  uint4 p0 = make_uint4(0u, 0u, 0u, 0u), p1 = p0;
+  uint32_t b = 0;
+  if (q < nq) {  // request the first words before waiting (W is final: k_abs_sum_group
+                 // waited for its predecessor before it let this kernel launch)
+    qg_advance(T, t, q);
+    b = (q - T[t].q_begin) * 8 + sub;
+    pk_load(T[t].pa.W, (uint32_t)T[t].pa.nblocks, b, s, p0, p1);
+  }
+  ptx::grid_dep_wait();  // k_abs_sum_group complete: thresholds and g published
+  __syncthreads();       // s_pair
+  while (q < nq) {
+    const uint32_t qn = q + qstep;
+    int tn = t;
+    uint4 n0 = make_uint4(0u, 0u, 0u, 0u), n1 = n0;
+    uint32_t bn = 0;
+    if (qn < nq) {
+      qg_advance(T, tn, qn);
+      bn = (qn - T[tn].q_begin) * 8 + sub;
+      pk_load(T[tn].pa.W, (uint32_t)T[tn].pa.nblocks, bn, s, n0, n1);
+    }
+    const PackGroupTensor &e = T[t];
+    const uint32_t thr = slots[t].thr;
+    const uint32_t thr2 = thr | (thr << 16);
+    if (e.pa_compact)
+      qmp_unit<true>(e.pa, s_pair, p0, p1, b, s, thr2);
+    else
+      qmp_unit<false>(e.pa, s_pair, p0, p1, b, s, thr2);
+    if (e.pb.codes) {
+      if (e.pb_compact)
+        qmp_unit<true>(e.pb, s_pair, p0, p1, b, s, thr2);
+      else
+        qmp_unit<false>(e.pb, s_pair, p0, p1, b, s, thr2);
+    }
+    q = qn;
+    t = tn;
+    b = bn;
+    p0 = n0;
+    p1 = n1;
+  }
+}
+
+// Fixed-pattern form of k_qmp_group, for plans whose tensors all pack the same patterns
+// (kMode 0: 6:8, 1: 2:4, 2: 6:8 into pa and 2:4 into pb) and ask for no dense matrix.  A warp keeps its current
+// tensor's geometry and output pointers in registers while its iterations stay in that
+// tensor: the plan entry is read once per tensor, not once per iteration, and the flags,
+// row and column of a block serve both patterns.  The words of the next iteration are
+// requested before the current ones are packed.
+constexpr int kQgCtasPerSm = 3;
+
+template <int kMode>
+__global__ void __launch_bounds__(kPkThreads, kQgCtasPerSm)
+    k_qmp_group_fixed(const PackGroupHeader *__restrict__ hdr,
+                      const PackGroupTensor *__restrict__ T,
+                      const PackGroupSlot *__restrict__ slots) {
+  __shared__ uint32_t s_pair[256];
+  ptx::grid_dep_launch();
+  if (kMode != 0) s_pair[threadIdx.x] = pair_entry(threadIdx.x);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int s = lane & 3;
+  const uint32_t sub = lane >> 2;
+  const uint32_t nq = hdr->total_q;
+  const uint32_t qstep = gridDim.x * (kPkThreads / 32);
+  uint32_t q = blockIdx.x * (kPkThreads / 32) + warp;  // warp-uniform
+  // the load stream: tensor tl holds iterations [qbl, qel)
+  int tl = -1;
+  const uint4 *Wl = nullptr;
+  uint32_t qbl = 0, qel = 0, nbl = 0;
+  uint4 p0 = make_uint4(0u, 0u, 0u, 0u), p1 = p0;
+  int tcur = -1;  // tensor of p0, p1
+  if (q < nq) {
+    do ++tl; while (q >= T[tl].q_begin + T[tl].nq);
+    Wl = T[tl].pa.W;
+    qbl = T[tl].q_begin;
+    qel = qbl + T[tl].nq;
+    nbl = (uint32_t)T[tl].pa.nblocks;
+    tcur = tl;
+    pk_load(Wl, nbl, (q - qbl) * 8 + sub, s, p0, p1);
+  }
+  ptx::grid_dep_wait();  // k_abs_sum_group complete: thresholds and g published
+  __syncthreads();       // s_pair
+  // the pack state of tensor tp
+  int tp = -1;
+  uint32_t qbp = 0, nbp = 0, bpr = 1, thr2 = 0;
+  FastDiv div{};
+  PlaneOut oa{}, ob{};
+  while (q < nq) {
+    const uint32_t qn = q + qstep;
+    uint4 n0 = make_uint4(0u, 0u, 0u, 0u), n1 = n0;
+    int tn = tcur;
+    if (qn < nq) {
+      if (qn >= qel) {
+        do ++tl; while (qn >= T[tl].q_begin + T[tl].nq);
+        Wl = T[tl].pa.W;
+        qbl = T[tl].q_begin;
+        qel = qbl + T[tl].nq;
+        nbl = (uint32_t)T[tl].pa.nblocks;
+      }
+      tn = tl;
+      pk_load(Wl, nbl, (qn - qbl) * 8 + sub, s, n0, n1);
+    }
+    if (tcur != tp) {
+      tp = tcur;
+      const PackGroupTensor &e = T[tp];
+      qbp = e.q_begin;
+      nbp = (uint32_t)e.pa.nblocks;
+      bpr = e.pa.bpr;
+      div = e.pa.div_bpr;
+      oa = plane_out(e.pa);
+      if (kMode == 2) ob = plane_out(e.pb);
+      const uint32_t thr = slots[tp].thr;
+      thr2 = thr | (thr << 16);
+    }
+    const uint32_t b = (q - qbp) * 8 + sub;
+    const bool valid = b < nbp;
+    const uint32_t row = fast_div(b, div);
+    const uint32_t col = b - row * bpr;
+    const bool row_end = col == bpr - 1;
+    const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    const LaneFlags f = lane_flags(w, thr2);
+    if constexpr (kMode == 0 || kMode == 2) {
+      const LanePack r = pack_lane_6of8(w, f);
+      if (valid) store_lane<false>(oa, r, row, col, row_end, s);
+    }
+    if constexpr (kMode == 1) {
+      const LanePack r = pack_lane_2of4(w, f, s_pair, s);
+      if (valid) store_lane<true>(oa, r, row, col, row_end, s);
+    }
+    if constexpr (kMode == 2) {
+      const LanePack r = pack_lane_2of4(w, f, s_pair, s);
+      if (valid) store_lane<true>(ob, r, row, col, row_end, s);
+    }
+    q = qn;
+    tcur = tn;
+    p0 = n0;
+    p1 = n1;
+  }
+}
+
+int64_t pack_group_plan_bytes(int count) {
+  return (int64_t)sizeof(PackGroupHeader) + (int64_t)count * (int64_t)sizeof(PackGroupTensor);
+}
+
+sbn_status launch_pack_group(const PackGroupHeader *hdr_host, const void *plan_dev,
+                             PackGroupSlot *slots, int32_t *err_flag, cudaStream_t st) {
+  if (hdr_host->count == 0 || hdr_host->total_chunks == 0) return SBN_OK;
+  const PackGroupHeader *hdr = static_cast<const PackGroupHeader *>(plan_dev);
+  const PackGroupTensor *T = reinterpret_cast<const PackGroupTensor *>(hdr + 1);
+  const int64_t cap = (int64_t)num_sms() * 4;
+  int64_t g1 = hdr_host->total_chunks;
+  if (g1 > cap) g1 = cap;
+  sbn_status ls = launch_pdl(k_abs_sum_group, dim3((unsigned)g1), dim3(kAgThreads), 0, st, hdr, T,
+                             slots, err_flag);
+  if (ls != SBN_OK) return ls;
+  const int per_sm = hdr_host->mode >= 0 ? kQgCtasPerSm : kPkCtasPerSm;
+  int64_t g2 = ((int64_t)hdr_host->total_q + kPkThreads / 32 - 1) / (kPkThreads / 32);
+  if (g2 > (int64_t)num_sms() * per_sm) g2 = (int64_t)num_sms() * per_sm;
+  if (g2 < 1) g2 = 1;
+  const dim3 grid2((unsigned)g2), block2(kPkThreads);
+  switch (hdr_host->mode) {
+    case 0: return launch_pdl(k_qmp_group_fixed<0>, grid2, block2, 0, st, hdr, T, slots);
+    case 1: return launch_pdl(k_qmp_group_fixed<1>, grid2, block2, 0, st, hdr, T, slots);
+    case 2: return launch_pdl(k_qmp_group_fixed<2>, grid2, block2, 0, st, hdr, T, slots);
+    default: return launch_pdl(k_qmp_group, grid2, block2, 0, st, hdr, T, slots);
+  }
 }
 
 }  // namespace sbn

@@ -167,3 +167,103 @@ def test_group_schedule_sizes(L):
     assert pb >= 128 + 512 * len(stack) + 32 * tiles
     st, pb, wb = _sizes(L, _group([(256, 4096, 16, 2, 4)]))
     assert st == 0 and wb > 0
+
+
+def _pack_group(specs, A=0x10000):
+    """ctypes array of grouped-pack tensors with placeholder pointers; specs are
+    (O, K, n, m, n2, m2)."""
+    arr = (sbn.SbnPackGroupTensor * len(specs))()
+    for i, (O, K, n, m, n2, m2) in enumerate(specs):
+        two = m2 != 0
+        arr[i] = sbn.SbnPackGroupTensor(W=A, codes=A, meta=A, codes2=A if two else None,
+                                        meta2=A if two else None, gamma_eff=A, dense_dbg=None,
+                                        dense_dbg2=None, out=O, in_=K, n=n, m=m, n2=n2, m2=m2,
+                                        eps=1e-5, reserved=0)
+    return arr
+
+
+def _pack_sizes(L, arr):
+    pb, wb = ctypes.c_int64(), ctypes.c_int64()
+    st = L.sbn_pack_group_sizes(ctypes.cast(arr, ctypes.c_void_p), len(arr), ctypes.byref(pb),
+                                ctypes.byref(wb))
+    return st, pb.value, wb.value
+
+
+def test_pack_group_sizes_validate(L):
+    assert _pack_sizes(L, _pack_group([(128, 256, 6, 8, 2, 4)]))[0] == 0
+    assert _pack_sizes(L, _pack_group([(128, 256, 2, 4, 0, 0)]))[0] == 0
+    assert _pack_sizes(L, _pack_group([(128, 256, 1, 4, 0, 0)]))[0] == 3   # fast patterns only
+    assert _pack_sizes(L, _pack_group([(128, 256, 6, 8, 6, 8)]))[0] == 3   # two equal patterns
+    assert _pack_sizes(L, _pack_group([(128, 256, 6, 8, 3, 8)]))[0] == 3
+    assert _pack_sizes(L, _pack_group([(128, 96, 6, 8, 2, 4)]))[0] == 2    # in % 64
+    assert _pack_sizes(L, _pack_group([(1 << 16, 1 << 15, 2, 4, 0, 0)]))[0] == 2  # 2^31 weights
+    assert _pack_sizes(L, _pack_group([(128, 256, 6, 8, 2, 4)], A=0x10008))[0] == 4
+    arr = _pack_group([(128, 256, 6, 8, 2, 4)])
+    arr[0].codes2 = None
+    assert _pack_sizes(L, arr)[0] == 1
+    arr = _pack_group([(128, 256, 6, 8, 2, 4)])
+    arr[0].eps = float("nan")
+    assert _pack_sizes(L, arr)[0] == 6
+    assert L.sbn_pack_group_sizes(None, 1, ctypes.byref(ctypes.c_int64()),
+                                  ctypes.byref(ctypes.c_int64())) == 1
+    A = _p(0x10000)
+    # a plan buffer that is not a plan: refused before any launch
+    junk = (ctypes.c_uint8 * 64)()
+    assert L.sbn_quantize_mask_pack_weights_group(ctypes.cast(junk, ctypes.c_void_p), A, A,
+                                                  None, None) == 6
+    assert L.sbn_quantize_mask_pack_weights_group(None, A, A, None, None) == 1
+    assert L.sbn_quantize_mask_pack_weights_group(A, _p(0x10008), A, None, None) == 4
+
+
+def test_pack_group_plan_layout(L):
+    """The plan's chunk and warp-iteration bookkeeping for the training-step tensors plus
+    ragged ones: 256 KB chunks of W per tensor, 8 blocks of 64 weights per iteration, both
+    counted from each tensor's start."""
+    import numpy as np
+    import workloads
+    specs = [(O, K, 6, 8, 2, 4) for _, O, K in workloads.TRAIN_LAYER_SHAPES]
+    specs += [(1, 64, 2, 4, 6, 8), (37, 192, 6, 8, 0, 0), (130, 4160, 2, 4, 0, 0)]
+    arr = _pack_group(specs)
+    st, pb, wb = _pack_sizes(L, arr)
+    assert st == 0 and wb == 16 * len(specs)
+    entry = (pb - 64) // len(specs)
+    assert pb == 64 + entry * len(specs) and entry % 16 == 0
+    buf = (ctypes.c_uint8 * (pb + 16))()
+    base = (ctypes.addressof(buf) + 15) // 16 * 16
+    assert L.sbn_pack_group_plan(ctypes.cast(arr, ctypes.c_void_p), len(arr), _p(base), pb) == 0
+    raw = np.frombuffer(buf, dtype=np.uint8)[base - ctypes.addressof(buf):][:pb]
+    hdr = raw[:20].view(np.uint32)
+    chunks = [-(-(O * K // 8) // 16384) for O, K, *_ in specs]
+    iters = [-(-(O * K // 64) // 8) for O, K, *_ in specs]
+    assert hdr[0] == 0x31475053 and hdr[1] == len(specs)
+    assert hdr[2] == sum(chunks) and hdr[3] == sum(iters)
+    assert hdr[4].view(np.int32) == -1  # mixed patterns: the general kernel
+    for i, (O, K, n, m, n2, m2) in enumerate(specs):
+        e = raw[64 + i * entry:64 + (i + 1) * entry]
+        nvec = int(e[256:264].view(np.int64)[0])
+        cb, nc, qb, nq, ca, cb2 = e[264:288].view(np.int32)
+        assert nvec == O * K // 8
+        assert (cb, nc) == (sum(chunks[:i]), chunks[i]) and (qb, nq) == (sum(iters[:i]), iters[i])
+        # two patterns are stored 6:8 first, 2:4 second, whichever order was asked
+        assert (ca, cb2) == (0, 1) if m2 else ca == (n == 2)
+
+
+@pytest.mark.parametrize("specs,mode", [([(96, 256, 6, 8, 2, 4), (8, 64, 2, 4, 6, 8)], 2),
+                                        ([(96, 256, 6, 8, 0, 0)] * 2, 0),
+                                        ([(96, 256, 2, 4, 0, 0)] * 3, 1),
+                                        ([(96, 256, 2, 4, 0, 0), (96, 256, 6, 8, 0, 0)], -1)])
+def test_pack_group_plan_mode(L, specs, mode):
+    """Plans whose tensors share their patterns (and ask for no dense matrix) name the
+    fixed-pattern kernel; any other plan the general one."""
+    import numpy as np
+    for dense in (False, True):
+        arr = _pack_group(specs)
+        if dense:
+            arr[0].dense_dbg = 0x10000
+        st, pb, _ = _pack_sizes(L, arr)
+        buf = (ctypes.c_uint8 * (pb + 16))()
+        base = (ctypes.addressof(buf) + 15) // 16 * 16
+        assert L.sbn_pack_group_plan(ctypes.cast(arr, ctypes.c_void_p), len(arr), _p(base),
+                                     pb) == 0
+        raw = np.frombuffer(buf, dtype=np.uint8)[base - ctypes.addressof(buf):][:pb]
+        assert raw[16:20].view(np.int32)[0] == (-1 if dense else mode)
