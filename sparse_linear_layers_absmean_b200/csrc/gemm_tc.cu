@@ -4,7 +4,7 @@
 // Three kernels share the pipeline below: k_gemm_tc (dense codes, any N:M pattern; one
 // tile per CTA), k_gemm_sp24 (2:4 on the sparse MMA; one tile per CTA, up to 128 tokens)
 // and, for more tokens, k_gemm_sp24_pair (2:4, CTA pairs, persistent, double-buffered
-// accumulators).
+// accumulators, the expanded weights and their metadata in TMEM).
 //
 // One CTA computes a 128 (outputs) x BN (tokens) tile with a multi-stage shared-memory
 // pipeline over K in blocks of 128 (a stage holds one to four consecutive blocks: each
@@ -69,6 +69,34 @@ template <int BN>
 __device__ __forceinline__ int red_word(int r, int col) {
   constexpr int kSwz = (BN / 4 < 8 ? BN / 4 : 8) - 1;
   return r * BN + ((((col >> 2) ^ (r & kSwz))) << 2) + (col & 3);
+}
+
+// One thread's chunk of an output row: y_i = fp32(acc_i * c_i) for the first nt of kCols
+// accumulator columns (acc_i = v[i] / 64, exact), stored with stride O.  A full chunk has
+// no per-column bound check; the pointer advances by O per column.
+__device__ __forceinline__ void store_y(float *p, float y) { *p = y; }
+__device__ __forceinline__ void store_y(__nv_bfloat16 *p, float y) { *p = __float2bfloat16_rn(y); }
+template <int kCols, typename Out>
+__device__ __forceinline__ void store_chunk(const uint32_t *v, const float *sc, int nt, Out *p,
+                                            int64_t O, bool small_acc) {
+  auto conv = [small_acc](uint32_t x) {
+    const int a = ((int)x) >> 6;
+    return small_acc ? __fsub_rn(__int_as_float(a + 0x4B400000), 12582912.0f) : __int2float_rn(a);
+  };
+  if (nt >= kCols) {
+#pragma unroll
+    for (int i = 0; i < kCols; ++i) {
+      store_y(p, __fmul_rn(conv(v[i]), sc[i]));
+      p += O;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kCols; ++i) {
+      if (i >= nt) break;
+      store_y(p, __fmul_rn(conv(v[i]), sc[i]));
+      p += O;
+    }
+  }
 }
 
 // Epilogue of the tensor-core kernels: warp w (0..3) owns accumulator lanes 32w..32w+31
@@ -136,21 +164,20 @@ __device__ __forceinline__ void store_tile(uint32_t trow, const float *s_scale, 
       if (c0 >= BN || !row_ok) continue;
       const uint32_t *v = half ? vb : va;
       // columns of this chunk that are real tokens of this tile
-      const int64_t nt = min(T - (t0 + c0), (int64_t)(BN - c0));
-      float *yf = reinterpret_cast<float *>(Y) + (t0 + c0) * O + o;
-      __nv_bfloat16 *yb = reinterpret_cast<__nv_bfloat16 *>(Y) + (t0 + c0) * O + o;
+      const int nt = (int)min(T - (t0 + c0), (int64_t)(BN - c0));
+      const int64_t off = (t0 + c0) * O + o;
+      if (y_is_bf16)
+        store_chunk<kCols>(v, s_scale + c0, nt, reinterpret_cast<__nv_bfloat16 *>(Y) + off, O,
+                           small_acc);
+      else
+        store_chunk<kCols>(v, s_scale + c0, nt, reinterpret_cast<float *>(Y) + off, O,
+                           small_acc);
+      if (acc_dbg) {
 #pragma unroll
-      for (int i = 0; i < kCols; ++i) {
-        if (i >= nt) break;
-        const int a = ((int)v[i]) >> 6;
-        const float fa = small_acc ? __fsub_rn(__int_as_float(a + 0x4B400000), 12582912.0f)
-                                   : __int2float_rn(a);
-        const float y = __fmul_rn(fa, s_scale[c0 + i]);
-        if (y_is_bf16)
-          yb[(int64_t)i * O] = __float2bfloat16_rn(y);
-        else
-          yf[(int64_t)i * O] = y;
-        if (acc_dbg) acc_dbg[(t0 + c0 + i) * O + o] = a;
+        for (int i = 0; i < kCols; ++i) {
+          if (i >= nt) break;
+          acc_dbg[off + (int64_t)i * O] = ((int)v[i]) >> 6;
+        }
       }
     }
   }
@@ -654,164 +681,182 @@ __device__ __forceinline__ bool bar_any(int id, int n, bool pred) {
 
 // ---------------------------------------------------------------------------------------
 // CTA-pair 2:4 kernel for large token counts.  A cluster of two CTAs computes 256 weight
-// rows x BN tokens per tile with the pair form of the sparse MMA: each CTA stages, expands
-// and stores its own 128 rows and loads half of the activation tile (BN / 2 tokens), so
-// every SM streams half the activation bytes of the single-CTA kernel per unit of MMA
-// work and fits more stages.  CTA 0 of the pair issues the metadata copies, the MMAs and
-// the commits for both (commits reach the same barrier in both CTAs); the expanders and
-// the epilogue warps of both CTAs report to CTA 0's barriers.  Persistent over tiles with
-// two TMEM accumulators (columns 0 and 256) per CTA: the epilogue warps drain tile i while
-// the MMA already accumulates tile i+1.
+// rows x BN tokens per tile with the pair form of the sparse MMA: each CTA stages and
+// expands its own 128 rows and loads half of the activation tile (BN / 2 tokens), so every
+// SM streams half the activation bytes of a single-CTA tile per unit of MMA work.  CTA 0 of
+// the pair issues the MMAs and the commits for both (commits reach the same barrier in
+// both CTAs); the expanders and the epilogue warps of both CTAs report to CTA 0's
+// barriers.  Persistent over tiles with two TMEM accumulators (columns 0 and 256) per CTA:
+// the epilogue warps drain tile i while the MMA already accumulates tile i+1.
+//
+// A and its metadata live in TMEM: the expanders write each row's expanded codes (16
+// columns per K block) and its metadata (4 columns) into their CTA's TMEM (tcgen05.st,
+// lane = row), and the pair MMA reads A from there.  Shared memory then holds only B and
+// the packed planes (17 KB per K block at 208 tokens), so the TMA ring is six stages of two
+// blocks deep; the A ring lives in the TMEM columns the two accumulators leave free (two
+// stages at 208 tokens).  Ring 1 (shared memory) is filled by the producers and freed by
+// the MMA's commit of the stage; ring 2 (TMEM) is filled by the expanders, which wait for
+// stage kg - S2's commit before they write stage kg's ring-2 slot.  The tile width 208 puts
+// a 2048-token batch in 10 token tiles (six rounds of tiles on 74 pairs for 11008 rows).
 // ---------------------------------------------------------------------------------------
+constexpr int kPairThreads = 352;  // 11 warps: expanders 0-3, producers 4 and 10, MMA 5, epilogue 6-9
+
 template <int BN>
 struct PairCfg {
   static constexpr int kKL = 128;
-  static constexpr int kBHalf = BN / 2;                 // tokens per CTA
-  static constexpr int kABytes = kBM * kKL / 2;
+  static constexpr int kBHalf = BN / 2;  // tokens per CTA
   static constexpr int kBBytes = kBHalf * kKL;
-  static constexpr int kPBytes = kBM * 16 * 2;
-  static constexpr int kBlockBytes = kABytes + kBBytes + kPBytes;
+  static constexpr int kPBytes = kBM * 16;  // one plane (codes or meta) of a block
+  static constexpr int kG = 2;              // K blocks per stage
+  static constexpr int kSlot1 = kG * (kBBytes + 2 * kPBytes);
   static constexpr int kBudget = 225 * 1024 - BN * 4 - 1024;
-  // kG consecutive K blocks per pipeline stage (one set of barriers); kSub block buffers
-  static constexpr int kG = 2;
-  static constexpr int kFit = (kBudget / kBlockBytes) > 12 ? 12 : (kBudget / kBlockBytes);
-  static constexpr int kSub = (kFit / kG) * kG;
-  static constexpr int kStages = kSub / kG;
-  static_assert(kStages >= 2, "at least two pipeline stages");
+  static constexpr int kS1 = (kBudget / kSlot1) / 2 * 2;  // even: two producers
+  static_assert(kS1 >= 2, "at least two shared-memory stages");
+  static_assert(kBBytes % 1024 == 0, "B blocks keep the 1024-byte swizzle alignment");
+  // TMEM: accumulators at columns 0 and 256; each gap [BN, 256) holds kPerGap blocks of A
+  // (16 columns each, from the gap's start) and their metadata (4 columns each, after them)
   static constexpr int kAccStride = 256;
-  static constexpr int kGap = (256 - BN) / 4;
-  static_assert(BN <= 256 && BN % 32 == 0, "pair tile width");
-  static_assert(kBBytes % 1024 == 0, "B blocks must keep the 1024-byte swizzle alignment");
-  static_assert(2 * kGap >= kSub, "two accumulators and the metadata must fit in TMEM");
-  static constexpr int kTmemCols = 512;
-  __device__ static constexpr uint32_t meta_col(int s) {
-    return s < kGap ? (uint32_t)(BN + 4 * s) : (uint32_t)(kAccStride + BN + 4 * (s - kGap));
+  static constexpr int kPerGap = (256 - BN) / 20;
+  static constexpr int kS2 = (2 * kPerGap) / kG;  // TMEM stages
+  static_assert(kS2 >= 2, "at least two TMEM stages");
+  static_assert(BN % 16 == 0 && BN <= 224, "pair tile width");
+  static_assert(kBHalf % 8 == 0, "B tiles of whole 8-row swizzle atoms");
+  __device__ static constexpr uint32_t a_col(int b) {  // b: block slot of ring 2
+    return (uint32_t)((b / kPerGap) * kAccStride + BN + 16 * (b % kPerGap));
   }
-  static constexpr uint32_t kTxBytes = kBBytes + kPBytes;  // per block and CTA
-  // barriers: full_a[S], full_t[S], empty[S], acc_full[2], acc_empty[2], mma_done; then the
-  // TMEM address, the abort flag (32 bytes) and the per-token scales
-  static constexpr size_t kSmem = 1024 + (size_t)kSub * kBlockBytes +
-                                  (size_t)(3 * kStages + 5) * 8 + 32 + (size_t)BN * 4;
+  __device__ static constexpr uint32_t e_col(int b) {
+    return (uint32_t)((b / kPerGap) * kAccStride + BN + 16 * kPerGap + 4 * (b % kPerGap));
+  }
+  static constexpr int kTmemCols = 512;
+  static constexpr uint32_t kTxBytes = kBBytes + 2 * kPBytes;  // per block and CTA
+  // barriers: full_t[S1], empty1[S1], full_a[S2], acc_full[2], acc_empty[2], mma_done;
+  // then the TMEM address, the abort flag (32 bytes) and the per-token scales
+  static constexpr size_t kSmem = 1024 + (size_t)kS1 * kSlot1 +
+                                  (size_t)(2 * kS1 + kS2 + 5) * 8 + 32 + (size_t)BN * 4;
+  static_assert(kS2 < kS1, "a stage's ring-2 slot is freed by the completion of stage kg - S2");
 };
-
-constexpr int kPairThreads = 352;  // 11 warps: expanders 0-3, producers 4 and 10, MMA 5, epilogue 6-9
 
 template <int BN>
 __global__ void __launch_bounds__(kPairThreads, 1)
     k_gemm_sp24_pair(const __grid_constant__ CUtensorMap tmap_x,
-                     const __grid_constant__ CUtensorMap tmap_c,
-                     const __grid_constant__ CUtensorMap tmap_m,
-                     const float *__restrict__ absmax, const float *__restrict__ gamma_eff,
-                     int64_t T, int64_t O, int64_t K, void *__restrict__ Y, int y_is_bf16,
-                     int32_t *__restrict__ acc_dbg, int32_t *err_flag) {
+                      const __grid_constant__ CUtensorMap tmap_c,
+                      const __grid_constant__ CUtensorMap tmap_m,
+                      const float *__restrict__ absmax, const float *__restrict__ gamma_eff,
+                      int64_t T, int64_t O, int64_t K, void *__restrict__ Y, int y_is_bf16,
+                      int32_t *__restrict__ acc_dbg, int32_t *err_flag) {
   using Cfg = PairCfg<BN>;
-  constexpr int S = Cfg::kStages, G = Cfg::kG, U = Cfg::kSub;
-  static_assert(S % 2 == 0, "two producers fill disjoint halves of the stages");
+  constexpr int S1 = Cfg::kS1, S2 = Cfg::kS2, G = Cfg::kG;
   constexpr int kTileM = 2 * kBM;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  // block buffer u = G * stage + g holds K block g of the stage
-  uint8_t *sB = smem;
-  uint8_t *sA = sB + U * Cfg::kBBytes;
-  uint8_t *sP = sA + U * Cfg::kABytes;
-  uint64_t *full_a = reinterpret_cast<uint64_t *>(sP + U * Cfg::kPBytes);  // CTA 0: both CTAs
-  uint64_t *full_t = full_a + S;                                          // own TMA loads
-  uint64_t *empty = full_t + S;                                           // own stage free
-  uint64_t *acc_full = empty + S;                                         // [2], own
-  uint64_t *acc_empty = acc_full + 2;                                     // [2], CTA 0: both
-  uint64_t *mma_done = acc_empty + 2;                                     // CTA 0: drain
+  // ring-1 slot s: B of its G blocks, then their codes planes, then their meta planes
+  uint8_t *ring1 = smem;
+  uint64_t *full_t = reinterpret_cast<uint64_t *>(ring1 + (size_t)S1 * Cfg::kSlot1);  // own TMA
+  // own stage done (the pair's commit of its MMAs): frees the ring-1 slot of stage kg, and
+  // (S2 stages later) the ring-2 slot of stage kg
+  uint64_t *empty1 = full_t + S1;
+  uint64_t *full_a = empty1 + S1;     // CTA 0: both CTAs' expanders
+  uint64_t *acc_full = full_a + S2;   // [2], own
+  uint64_t *acc_empty = acc_full + 2;  // [2], CTA 0: both
+  uint64_t *mma_done = acc_empty + 2;  // CTA 0: drain
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
   volatile int *s_abort = reinterpret_cast<volatile int *>(tmem_slot + 2);
   float *s_scale = reinterpret_cast<float *>(tmem_slot + 8);
 
-  // the next kernel on the stream may start its prologue; it waits for this one
   ptx::grid_dep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = ptx::cluster_ctarank();  // 0: issues the pair's MMAs
+  const uint32_t rank = ptx::cluster_ctarank();
   const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int nkb = (int)((K + Cfg::kKL - 1) / Cfg::kKL);
-  const int nst = (nkb + G - 1) / G;  // stages per tile; the last may hold fewer blocks
+  const int nst = (nkb + G - 1) / G;
   const int64_t n_o = (O + kTileM - 1) / kTileM, n_t = (T + BN - 1) / BN;
   const int64_t ntiles = n_o * n_t;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      ptx::mbar_init(&full_a[s], 8);  // the expander warps of both CTAs (used in CTA 0)
+    for (int s = 0; s < S1; ++s) {
       ptx::mbar_init(&full_t[s], 1);
-      ptx::mbar_init(&empty[s], 1);
+      ptx::mbar_init(&empty1[s], 1);
     }
+    for (int s = 0; s < S2; ++s)
+      ptx::mbar_init(&full_a[s], 8);  // the expander warps of both CTAs (used in CTA 0)
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&acc_full[b], 1);
-      ptx::mbar_init(&acc_empty[b], 8);  // the epilogue warps of both CTAs (used in CTA 0)
+      ptx::mbar_init(&acc_empty[b], 8);
     }
     ptx::mbar_init(mma_done, 1);
     *s_abort = 0;
     ptx::fence_mbar_init();
   }
-  // both CTAs' barriers exist before anyone arrives on a remote one
   ptx::cluster_sync();
   if (warp == 5) {
     ptx::tmem_alloc_pair(tmem_slot, Cfg::kTmemCols);
     ptx::tmem_relinquish_pair();
   }
-  ptx::grid_dep_wait();  // the previous kernel's outputs (activations, scales) are visible
+  ptx::grid_dep_wait();
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // CTA 0's barriers as seen from this CTA
   const uint32_t full_a0 = ptx::mapa_shared(ptx::smem_u32(full_a), 0);
   const uint32_t acc_empty0 = ptx::mapa_shared(ptx::smem_u32(acc_empty), 0);
 
   if (warp < 4) {
-    // ---------------- compressed-weight expanders (this CTA's 128 rows) ----------------
+    // ---------------- expanders: this CTA's 128 rows into its TMEM ----------------
     const int r = threadIdx.x;
-    int64_t kg = 0;
+    const uint32_t lrow = (uint32_t)(warp * 32) << 16;
+    // stage kg's slots and phases; (f1, fph) the ring-1 slot of stage kg - S2, whose
+    // completion frees ring-2 slot s2
+    int kg = 0, s1 = 0, s2 = 0, f1 = S1 - S2;
+    uint32_t ph1 = 0, fph = 1;
     for (int64_t tile = pair;
          tile < ntiles && !__any_sync(0xffffffffu, *s_abort != 0); tile += npairs) {
       const int64_t o0 = (tile % n_o) * kTileM + (int64_t)rank * kBM;
-      for (int j = 0; j < nst; ++j, ++kg) {
-        const int s = (int)(kg % S);
-        const uint32_t ph = (uint32_t)(kg / S) & 1u;
-        const bool ok = (kg < S || wait_or_abort(&empty[s], ph ^ 1u, s_abort)) &&
-                        wait_or_abort(&full_t[s], ph, s_abort);
-        if (!__all_sync(0xffffffffu, ok)) break;  // the whole warp leaves together
+      const bool row_ok = o0 + r < O;
+      for (int j = 0; j < nst; ++j) {
+        const bool ok = (kg < S2 || wait_or_abort(&empty1[f1], fph, s_abort)) &&
+                        wait_or_abort(&full_t[s1], ph1, s_abort);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        ptx::tc_fence_after();
+        const uint8_t *slot = ring1 + (size_t)s1 * Cfg::kSlot1 + G * Cfg::kBBytes;
         const int nb = min(G, nkb - j * G);
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           if (g >= nb) break;
-          const int u = s * G + g;
           const int kb = j * G + g;
-          const uint4 cw = *reinterpret_cast<const uint4 *>(sP + u * Cfg::kPBytes + r * 16);
-          const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
-          // this row's metadata goes straight to its TMEM lane (the sparse MMA reads it
-          // there); groups outside the matrix get the valid index pair (0, 1)
-          uint4 m4 = *reinterpret_cast<const uint4 *>(sP + u * Cfg::kPBytes + kBM * 16 + r * 16);
-          if (o0 + r >= O) {
+          const int b2 = s2 * G + g;
+          const uint4 cw = *reinterpret_cast<const uint4 *>(slot + g * Cfg::kPBytes + r * 16);
+          uint4 m4 = *reinterpret_cast<const uint4 *>(slot + (G + g) * Cfg::kPBytes + r * 16);
+          // groups outside the matrix get the valid index pair (0, 1); their codes are zero
+          if (!row_ok) {
             m4 = make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
           } else if ((int64_t)kb * Cfg::kKL + 64 >= K) {
             m4.z = 0x44444444u;
             m4.w = 0x44444444u;
           }
-          ptx::tmem_st_4(tmem + ((uint32_t)(warp * 32) << 16) + Cfg::meta_col(u), m4);
-          uint8_t *dst = sA + u * Cfg::kABytes + r * 64;
+          ptx::tmem_st_4(tmem + lrow + Cfg::e_col(b2), m4);
+          // 16 kept codes per word -> 16 int8 lanes of 64 * t, in K order: column 4c + q
+          // holds the four values (w[c] << 2q) & 0xC0C0C0C0
+          const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+          uint32_t a[16];
 #pragma unroll
           for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4 *>(dst + ((c ^ ((r >> 1) & 3)) << 4)) =
-                make_uint4(w[c] & 0xC0C0C0C0u, (w[c] << 2) & 0xC0C0C0C0u,
-                           (w[c] << 4) & 0xC0C0C0C0u, (w[c] << 6) & 0xC0C0C0C0u);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) a[4 * c + q] = (w[c] << (2 * q)) & 0xC0C0C0C0u;
+          ptx::tmem_st_16(tmem + lrow + Cfg::a_col(b2), a);
         }
         ptx::tmem_st_wait();
-        ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive_cluster(full_a0 + 8u * (uint32_t)s);
+        if (lane == 0) ptx::mbar_arrive_cluster(full_a0 + 8u * (uint32_t)s2);
+        ++kg;
+        if (++s1 == S1) s1 = 0, ph1 ^= 1u;
+        if (++s2 == S2) s2 = 0;
+        if (++f1 == S1) f1 = 0, fph ^= 1u;
       }
     }
   } else if (warp == 4 || warp == 10) {
-    // ---------------- two TMA producers (this CTA's rows and half of the tokens): stage kg
-    // by producer kg % 2; S is even, so each one fills its own half of the stages ----------
+    // ---------------- two TMA producers: stage kg by producer kg % 2 (S1 is even) --------
     if (lane == 0) {
       const int pt = warp == 4 ? 0 : 1;
       ptx::prefetch_tmap(&tmap_x);
@@ -823,32 +868,36 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const int64_t t0 = (tile / n_o) * BN + (int64_t)rank * Cfg::kBHalf;
         for (int j = 0; j < nst; ++j, ++kg) {
           if ((int)(kg & 1) != pt) continue;
-          const int s = (int)(kg % S);
-          const uint32_t ph = (uint32_t)(kg / S) & 1u;
-          if (kg >= S && !wait_or_abort(&empty[s], ph ^ 1u, s_abort)) break;
+          const int s = (int)(kg % S1);
+          const uint32_t ph = (uint32_t)(kg / S1) & 1u;
+          if (kg >= S1 && !wait_or_abort(&empty1[s], ph ^ 1u, s_abort)) break;
           const int nb = min(G, nkb - j * G);
           ptx::mbar_arrive_expect_tx(&full_t[s], (uint32_t)nb * Cfg::kTxBytes);
+          uint8_t *slot = ring1 + (size_t)s * Cfg::kSlot1;
           for (int g = 0; g < nb; ++g) {
-            const int u = s * G + g;
             const int kb = j * G + g;
-            ptx::tma_load_2d(sB + u * Cfg::kBBytes, &tmap_x, &full_t[s], kb * Cfg::kKL,
+            ptx::tma_load_2d(slot + g * Cfg::kBBytes, &tmap_x, &full_t[s], kb * Cfg::kKL,
                              (int32_t)t0);
-            uint8_t *p = sP + u * Cfg::kPBytes;
-            ptx::tma_load_2d(p, &tmap_c, &full_t[s], kb * 16, (int32_t)o0);
-            ptx::tma_load_2d(p + kBM * 16, &tmap_m, &full_t[s], kb * 16, (int32_t)o0);
+            ptx::tma_load_2d(slot + G * Cfg::kBBytes + g * Cfg::kPBytes, &tmap_c, &full_t[s],
+                             kb * 16, (int32_t)o0);
+            ptx::tma_load_2d(slot + G * Cfg::kBBytes + (G + g) * Cfg::kPBytes, &tmap_m,
+                             &full_t[s], kb * 16, (int32_t)o0);
           }
-          issued = kg;  // the last stage this thread issued
+          issued = kg;
         }
       }
-      // its last S / 2 stages, one per slot of its half, land before the CTA can exit
-      for (int64_t q = issued, i = 0; q >= 0 && i < S / 2; q -= 2, ++i)
-        if (!wait_phase(&full_t[q % S], (uint32_t)(q / S) & 1u)) *s_abort = 1;
+      // its last S1 / 2 stages, one per slot of its half, land before the CTA can exit
+      for (int64_t q = issued, i = 0; q >= 0 && i < S1 / 2; q -= 2, ++i)
+        if (!wait_phase(&full_t[q % S1], (uint32_t)(q / S1) & 1u)) *s_abort = 1;
     }
   } else if (warp == 5) {
-    // ---------------- CTA 0: metadata copies + pair MMAs ----------------
+    // ---------------- CTA 0: the pair's MMAs ----------------
     if (rank == 0 && lane == 0) {
       constexpr uint32_t idesc = ptx::idesc_i8_sparse(kTileM, BN);
-      int64_t kg = 0;
+      // B descriptor of ring 1's first byte; a slot, block and K half add (offset >> 4)
+      const uint64_t b_desc0 = ptx::smem_desc_sw128(ptx::smem_u32(ring1));
+      int s1 = 0, s2 = 0;
+      uint32_t ph2 = 0;
       int i = 0;
       for (int64_t tile = pair; tile < ntiles && !*s_abort; tile += npairs, ++i) {
         const int buf = i & 1;
@@ -857,33 +906,30 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(buf * Cfg::kAccStride);
         bool ok = true;
-        for (int j = 0; j < nst; ++j, ++kg) {
-          const int s = (int)(kg % S);
-          const uint32_t ph = (uint32_t)(kg / S) & 1u;
-          if (!wait_or_abort(&full_a[s], ph, s_abort)) {  // both CTAs expanded (and loaded)
+        for (int j = 0; j < nst; ++j) {
+          // both CTAs expanded this stage, after their own B and planes had landed
+          if (!wait_or_abort(&full_a[s2], ph2, s_abort)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
           const int nb = min(G, nkb - j * G);
+          const uint64_t b_desc = b_desc0 + (uint64_t)((s1 * Cfg::kSlot1) >> 4);
           for (int g = 0; g < nb; ++g) {
-            const int u = s * G + g;
-            const uint32_t e_col = tmem + Cfg::meta_col(u);
-            // (the metadata is already in both CTAs' TMEM, written by the expanders)
-            const uint32_t a_addr = ptx::smem_u32(sA + u * Cfg::kABytes);
-            const uint32_t b_addr = ptx::smem_u32(sB + u * Cfg::kBBytes);
+            const int b2 = s2 * G + g;
 #pragma unroll
             for (int k = 0; k < 2; ++k)
-              ptx::mma_sp_i8_pair(d_tmem, ptx::smem_desc_sw64(a_addr + 32 * k),
-                                  ptx::smem_desc_sw128(b_addr + 64 * k), e_col + 2 * k, idesc,
-                                  (j | g | k) != 0);
+              ptx::mma_sp_i8_pair_tmem_a(d_tmem, tmem + Cfg::a_col(b2) + 8 * k,
+                                         b_desc + (uint64_t)((g * Cfg::kBBytes + 64 * k) >> 4),
+                                         tmem + Cfg::e_col(b2) + 2 * k, idesc, (j | g | k) != 0);
           }
-          ptx::mma_commit_pair(&empty[s], 0x3);
+          ptx::mma_commit_pair(&empty1[s1], 0x3);
+          if (++s1 == S1) s1 = 0;
+          if (++s2 == S2) s2 = 0, ph2 ^= 1u;
         }
         if (!ok) break;
         ptx::mma_commit_pair(&acc_full[buf], 0x3);
       }
-      // every MMA issued has completed before TMEM can be released (also after an abort)
       ptx::mma_commit_pair(mma_done, 0x1);
       if (!wait_phase(mma_done, 0)) *s_abort = 1;
     }
@@ -921,7 +967,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   ptx::tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && *s_abort && err_flag) atomicOr(err_flag, SBN_FLAG_TIMEOUT);
-  // neither CTA frees its TMEM or leaves while the pair's MMAs may still use it
   ptx::cluster_sync();
   if (warp == 5) {
     ptx::tc_fence_after();
@@ -1170,7 +1215,7 @@ sbn_status launch_gemm_tc(const int8_t *Xq, const float *absmax, const uint8_t *
                           cudaStream_t st) {
   const bool compact = (n == 2 && m == 4);
   if (compact && tokens > 128)  // CTA pairs (every sm_100 device runs 2-CTA clusters)
-    return gemm_sp24_pair_t<224>(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldx, ldc, ldm, Y,
+    return gemm_sp24_pair_t<208>(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldx, ldc, ldm, Y,
                                  y_is_bf16, acc_dbg, err_flag, st);
   if (tokens > 128)
     return gemm_tc_bn<256>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldx, ldc,

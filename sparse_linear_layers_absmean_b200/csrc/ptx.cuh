@@ -278,6 +278,19 @@ __device__ __forceinline__ void mma_sp_i8_tmem_a(uint32_t d_tmem, uint32_t a_tme
       : "memory");
 }
 
+// The CTA-pair form: each CTA's TMEM holds its 128 rows of A (and of the metadata) at the
+// same column address; B is split over the two CTAs' shared memory as in mma_sp_i8_pair.
+__device__ __forceinline__ void mma_sp_i8_pair_tmem_a(uint32_t d_tmem, uint32_t a_tmem,
+                                                      uint64_t b_desc, uint32_t e_tmem,
+                                                      uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::2.kind::i8 [%0], [%1], %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
