@@ -369,7 +369,7 @@ def bench_stack_prefill(args, sbn, dev, local, rank, world, peaks, timer, packed
     return {"value": ops * world / (ms * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": ms,
             "steps": steps,
             "roofline": tensor_roof(qkv_ops / (per["linear"] * 1e-3) / 1e12, peaks,
-                                    "k_gemm_sp24_pair<224> (QKV 12288x4096, 4096 tokens, per call)"),
+                                    "k_gemm_sp24_pair<208> (QKV 12288x4096, 4096 tokens, per call)"),
             "whole_step_frac_of_int8_peak": ops / (ms * 1e-3) / 1e12 / (2.0 * peaks["bf16"]),
             "gpu_launches": 2 * len(lay) * steps, "clocks": clocks,
             "config": {"workload": "stack-prefill-32x4096-t4096-2of4", "tokens": T,
@@ -946,6 +946,15 @@ def run_only(args):
                 plan.quantize_acts(err)
             else:
                 plan.linear(err)
+    elif args.workload == "train-step":
+        if args.only != "pack":
+            sys.exit("train-step --only takes pack (the grouped 6:8 + 2:4 pack)")
+        Ws = [workloads.masters_device(O, K, device=dev, config=4, tensor=5 * layer + i)
+              for layer in range(args.train_layers)
+              for i, (name, O, K) in enumerate(workloads.TRAIN_LAYER_SHAPES)]
+        pg = sbn.PackGroup(Ws, ((6, 8), (2, 4)), device=dev)
+        for _ in range(calls):
+            pg.run(err)
     else:
         cfg = {"decode": workloads.DECODE_GEMV, "prefill": workloads.PREFILL_GEMM}[args.workload]
         O, K, T, n, m = cfg["O"], cfg["K"], cfg["T"], cfg["n"], cfg["m"]
@@ -990,12 +999,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub", action="store_true", help="headline only, no sub-records")
     ap.add_argument("--only", choices=["pack", "act", "linear"],
-                    help="profiling aid: one kind of C-ABI call, untimed (decode, prefill, stack)")
+                    help="profiling aid: one kind of C-ABI call, untimed (decode, prefill, stack; "
+                         "train-step: pack)")
+    ap.add_argument("--train-layers", type=int, default=workloads.TRAIN_LAYERS,
+                    help="profiling aid with --only: decoder layers of the training step "
+                         "(default 26)")
     ap.add_argument("--stack-layers", type=int, default=workloads.STACK_LAYERS,
                     help="profiling aid with --only: decoder layers of the stack (default 32)")
     args = ap.parse_args()
-    if args.stack_layers != workloads.STACK_LAYERS and not args.only:
-        sys.exit("--stack-layers is a profiling aid for --only runs")
+    if (args.stack_layers != workloads.STACK_LAYERS or
+            args.train_layers != workloads.TRAIN_LAYERS) and not args.only:
+        sys.exit("--stack-layers / --train-layers are profiling aids for --only runs")
     global STACK_LAYERS
     STACK_LAYERS = args.stack_layers
     if args.warmup < 3:
