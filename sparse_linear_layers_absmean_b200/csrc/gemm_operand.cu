@@ -153,6 +153,31 @@ __device__ __forceinline__ bool op_bar_any(bool pred) {
   return r != 0;
 }
 
+// 32 columns of one output row: y_i = fp32(acc_i * c_i) for the first nt, stride O (a full
+// chunk without per-column checks; the pointer advances by O per column).
+__device__ __forceinline__ void op_store_y(float *p, float y) { *p = y; }
+__device__ __forceinline__ void op_store_y(__nv_bfloat16 *p, float y) {
+  *p = __float2bfloat16_rn(y);
+}
+template <typename Out>
+__device__ __forceinline__ void op_store_chunk(const uint32_t *v, const float *sc, int nt, Out *p,
+                                               int64_t O) {
+  if (nt >= 32) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      op_store_y(p, __fmul_rn(__int2float_rn((int32_t)v[i]), sc[i]));
+      p += O;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if (i >= nt) break;
+      op_store_y(p, __fmul_rn(__int2float_rn((int32_t)v[i]), sc[i]));
+      p += O;
+    }
+  }
+}
+
 // Epilogue of one accumulator: warp quarter q holds rows 32q..32q+31 (TMEM lanes), column j
 // is token t0 + j and holds the exact int32 sum; y = fp32(acc * c_t).
 template <int BN>
@@ -166,19 +191,18 @@ __device__ __forceinline__ void op_store(uint32_t trow, const float *s_scale, in
     ptx::tmem_ld_32(trow + cb, v);
     ptx::tmem_ld_wait();
     if (!row_ok) continue;
-    const int64_t nt = min(T - (t0 + cb), (int64_t)32);
-    float *yf = reinterpret_cast<float *>(Y) + (t0 + cb) * O + o;
-    __nv_bfloat16 *yb = reinterpret_cast<__nv_bfloat16 *>(Y) + (t0 + cb) * O + o;
+    const int nt = (int)min(T - (t0 + cb), (int64_t)32);
+    const int64_t off = (t0 + cb) * O + o;
+    if (y_is_bf16)
+      op_store_chunk(v, s_scale + cb, nt, reinterpret_cast<__nv_bfloat16 *>(Y) + off, O);
+    else
+      op_store_chunk(v, s_scale + cb, nt, reinterpret_cast<float *>(Y) + off, O);
+    if (acc_dbg) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      if (i >= nt) break;
-      const int32_t a = (int32_t)v[i];
-      const float y = __fmul_rn(__int2float_rn(a), s_scale[cb + i]);
-      if (y_is_bf16)
-        yb[(int64_t)i * O] = __float2bfloat16_rn(y);
-      else
-        yf[(int64_t)i * O] = y;
-      if (acc_dbg) acc_dbg[(t0 + cb + i) * O + o] = a;
+      for (int i = 0; i < 32; ++i) {
+        if (i >= nt) break;
+        acc_dbg[off + (int64_t)i * O] = (int32_t)v[i];
+      }
     }
   }
 }
