@@ -601,43 +601,73 @@ def bench_backward(args, sbn, dev, local, rank, world, peaks, timer, err):
 
 
 def bench_group_quant(args, sbn, dev, local, rank, world, peaks, timer, err):
-    """Group quantisation (G = 4 blocks along K) on the stack's QKV shape (12288 x 4096 2:4)
-    at 16 tokens: per step the group activation quantiser and the contraction (4 block
-    contractions + the ordered sum), weights packed once with per-group scales."""
-    O, K, T, G = 12288, 4096, workloads.STACK_DECODE_T, 4
-    R = 8  # rotating weight sets: 8 x 12.6 MB of packed weights > L2
-    ws_ = []
-    for r in range(R):
-        W = workloads.masters_device(O, K, device=dev, config=7, tensor=r)
-        ws_.append(sbn.pack_weights_gq(W, 2, 4, G, err_flag=err))
+    """Group quantisation (G = 2 blocks along K: the largest G that cuts every layer of the
+    stack, K = 4096 or 11008 = 86 x 128, into whole 128-deep blocks): the 32-layer stack's
+    decode step at 16 tokens with every layer packed with per-group scales, on the grouped
+    calls (the grouped quantiser with per-(token, group) scales, the grouped contraction of
+    every block of every layer, the ordered sum: 3 launches).  Beside it, one layer (QKV
+    12288 x 4096) through the one-layer calls (a contraction per block + the sum)."""
+    G, T = 2, workloads.STACK_DECODE_T
+    layers = []
+    for idx, name, O, K, tid in stack_layers(rank):
+        W = workloads.masters_device(O, K, device=dev, config=7, tensor=tid)
+        w = sbn.pack_weights_gq(W, 2, 4, G, err_flag=err)
         del W
-    X = workloads.torch_bf16(workloads.student_t(T, K, config=7, tensor=100), dev)
-    Xq = torch.empty((T, K), dtype=torch.int8, device=dev)
-    s = torch.empty((G, T), dtype=torch.float32, device=dev)
-    Y = torch.empty((T, O), dtype=torch.float32, device=dev)
-    part = torch.empty(G * T * O * 4, dtype=torch.uint8, device=dev)
+        X = workloads.torch_bf16(workloads.student_t(T, K, config=7, tensor=10000 + tid), dev)
+        layers.append(dict(X=X, w=w))
+    plan = sbn.GqGroupPlan(layers, device=dev)
     st = timer.stream
 
     def step(i, ev):
-        w = ws_[i % R]
-        sbn.sbn_quantize_acts_gq(X, G, Xq, s, err, st)
         if ev is not None:
+            ev["act"][0].record(st)
+        plan.quantize_acts(err, st)
+        if ev is not None:
+            ev["act"][1].record(st)
             ev["linear"][0].record(st)
-        sbn.sbn_linear_gq(Xq, s, w.codes, w.meta, w.gamma_eff, O, K, 2, 4, G, Y, part, None, err, st)
+        plan.linear(err, st)
         if ev is not None:
             ev["linear"][1].record(st)
 
     steps = args.steps
-    ms, per, clocks = timer.run(step, steps, args.warmup, calls=("linear",))
-    packed = O * K // 4
+    ms, per, clocks = timer.run(step, steps, args.warmup, calls=("act", "linear"))
+    packed = sum(L["w"].out * L["w"].in_ // 4 for L in layers)
+    xbytes = sum(L["X"].numel() * 3 + 4 * G * L["X"].shape[0] for L in layers)  # X in, Xq, s
+    ybytes = plan.n * 4 * (G + G + 1)  # partials written and read, Y written
     gbs = packed / (per["linear"] * 1e-3) / 1e9
-    return {"value": packed * world / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
-            "steps": steps,
-            "roofline": hbm_roof(gbs, peaks, "per-block contraction (k_gemm_sp24<16> on 4 slices) "
-                                 "+ ordered sum", unit_note="; on packed-weight bytes"),
-            "gpu_launches": 6 * steps, "clocks": clocks,
-            "config": {"workload": "group-quant-12288x4096-t16-2of4-G4", "groups": G,
-                       "l2": f"{R} rotating packed weight sets"}}
+
+    # one layer through the one-layer calls (QKV), 8 rotating weight sets beyond L2
+    O, K = 12288, 4096
+    R = 8
+    ws_ = [layers[5 * r]["w"] for r in range(R)]
+    X = layers[0]["X"]
+    Xq = torch.empty((T, K), dtype=torch.int8, device=dev)
+    s1 = torch.empty((G, T), dtype=torch.float32, device=dev)
+    Y1 = torch.empty((T, O), dtype=torch.float32, device=dev)
+    part = torch.empty(G * T * O * 4, dtype=torch.uint8, device=dev)
+
+    def step1(i, ev):
+        w = ws_[i % R]
+        sbn.sbn_quantize_acts_gq(X, G, Xq, s1, err, st)
+        sbn.sbn_linear_gq(Xq, s1, w.codes, w.meta, w.gamma_eff, O, K, 2, 4, G, Y1, part, None,
+                          err, st)
+
+    ms1, _, _ = timer.run(step1, steps, args.warmup, sample_clocks=False)
+    return {"value": (packed + xbytes + ybytes) * world / (ms * 1e-3) / 1e9, "unit": "GB/s",
+            "ms_per_step": ms, "steps": steps,
+            "roofline": hbm_roof(gbs, peaks, f"k_gemm_group over {G * len(layers)} layer blocks "
+                                 "+ k_gq_sum",
+                                 unit_note="; on packed-weight bytes"),
+            "kernels": {"act_quant_group": {"ms": per["act"]},
+                        "linear_group_and_sum": {"ms": per["linear"],
+                                                 "packed_weight_GB/s": gbs}},
+            "one_layer_calls": {"workload": f"12288x4096-t16-G{G}", "ms_per_step": ms1,
+                                "packed_weight_GB/s": O * K / 4 / (ms1 * 1e-3) / 1e9,
+                                "launches_per_step": 2 + G + 1},
+            "gpu_launches": 3 * steps, "clocks": clocks,
+            "config": {"workload": f"group-quant-stack-32x4096-t16-2of4-G{G}", "groups": G,
+                       "layers": len(layers), "packed_bytes": packed,
+                       "l2": f"{packed / 1e9:.2f} GB of packed weights per step > 126 MB L2"}}
 
 
 def bench_fused_decode(args, sbn, dev, local, rank, world, peaks, timer, err):
@@ -847,6 +877,8 @@ def run_cuda(args):
         packed = build_stack(sbn, dev, rank, err)
         head, _, _ = bench_stack_decode(args, sbn, dev, local, rank, world, peaks, timer,
                                         packed, err)
+        head_flag = int(err.item())  # the head line's own flag; the sub-records keep theirs
+        err.zero_()
         if args.workload == "stack-prefill":
             head = bench_stack_prefill(args, sbn, dev, local, rank, world, peaks, timer, packed,
                                        err)
@@ -856,20 +888,38 @@ def run_cuda(args):
             if world == 1 and not args.no_sub:
                 subs["stack_prefill"] = bench_stack_prefill(args, sbn, dev, local, rank, world,
                                                             peaks, timer, packed, err)
+                subs["stack_prefill"]["err_flag"] = int(err.item())
+                err.zero_()
         del packed
         torch.cuda.empty_cache()
         if world == 1 and not args.no_sub and args.workload == "stack":
             subs["decode_gemv"] = bench_single(args, sbn, dev, local, rank, world, peaks, timer,
                                                workloads.DECODE_GEMV, err)
+            subs["decode_gemv"]["err_flag"] = int(err.item())
+            err.zero_()
             subs["prefill_gemm"] = bench_single(args, sbn, dev, local, rank, world, peaks, timer,
                                                 workloads.PREFILL_GEMM, err)
+            subs["prefill_gemm"]["err_flag"] = int(err.item())
+            err.zero_()
             subs["train_step"] = bench_train(args, sbn, dev, local, rank, world, peaks, timer,
                                              err)
+            subs["train_step"]["err_flag"] = int(err.item())
+            err.zero_()
             subs["backward"] = bench_backward(args, sbn, dev, local, rank, world, peaks, timer, err)
+            subs["backward"]["err_flag"] = int(err.item())
+            err.zero_()
             subs["group_quant"] = bench_group_quant(args, sbn, dev, local, rank, world, peaks,
                                                     timer, err)
+            subs["group_quant"]["err_flag"] = int(err.item())
+            err.zero_()
             subs["fused_decode"] = bench_fused_decode(args, sbn, dev, local, rank, world, peaks,
                                                       timer, err)
+            subs["fused_decode"]["err_flag"] = int(err.item())
+            err.zero_()
+        # the line's flag: every flag raised anywhere in the run
+        for rec in subs.values():
+            head_flag |= rec.get("err_flag", 0)
+        err.fill_(head_flag)
     elif args.workload == "decode":
         head, subs = bench_single(args, sbn, dev, local, rank, world, peaks, timer,
                                   workloads.DECODE_GEMV, err), {}

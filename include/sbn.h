@@ -290,6 +290,14 @@ typedef struct sbn_group_linear {
   int32_t n, m;              /* must be 2 and 4 */
   int32_t y_is_bf16;
   int32_t reserved;          /* set to 0 */
+  /* Row strides, 0 for the defaults.  A layer may be a K slice of a wider one (a block of
+   * a group-quantised layer): X, Xq point at the slice's first column, `in` is the slice
+   * width, and the strides are the wide layer's.
+   *   ldx  elements between token rows of X and Xq (default in; a multiple of 16, >= in)
+   *   ldc  bytes between rows of the codes plane (default that of sbn_linear_ref_dims for
+   *        (out, in, 2, 4); a multiple of 16, >= in / 8)
+   *   ldm  bytes between rows of the meta plane (likewise) */
+  int64_t ldx, ldc, ldm;
 } sbn_group_linear;
 
 /*
@@ -333,6 +341,17 @@ SBN_API sbn_status sbn_quantize_acts_group(const void *plan, const void *plan_de
  */
 SBN_API sbn_status sbn_linear_group(const void *plan, const void *plan_dev, void *workspace,
                                     int32_t *err_flag, void *stream);
+
+/*
+ * The ordered sum of group quantisation: Y[i] = fp32 sum over j = 0..G-1 of part[j * n + i],
+ * added in j order, stored fp32 or bf16 (RNE).  With the G blocks of group-quantised
+ * layers as slices of a grouped call (each block's output y_j = fp32(acc_j * c_tj) written
+ * into part), this completes their forward: the same bits as sbn_linear_gq.  Layers of
+ * one G may share one call when their partial outputs and their Y are laid out back to
+ * back (part as [G][n], Y as [n]).  n >= 0, 1 <= G <= 64; part and Y 16-byte aligned.
+ */
+SBN_API sbn_status sbn_gq_sum(const float *part, int64_t n, int32_t G, void *Y, int32_t y_is_bf16,
+                              void *stream);
 
 /*
  * Backward of the layer under the dual straight-through estimator (Sparse-BitNet summaries,

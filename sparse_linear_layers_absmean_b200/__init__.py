@@ -35,7 +35,7 @@ EXPORTED = ("sbn_linear_ref_dims", "sbn_quantize_mask_pack_weights", "sbn_quanti
             "sbn_backward_workspace_bytes", "sbn_backward", "sbn_quantize_linear",
             "sbn_gq_workspace_bytes", "sbn_quantize_mask_pack_weights_gq", "sbn_quantize_acts_gq",
             "sbn_linear_gq", "sbn_pack_group_sizes", "sbn_pack_group_plan",
-            "sbn_quantize_mask_pack_weights_group")
+            "sbn_quantize_mask_pack_weights_group", "sbn_gq_sum")
 
 
 class SbnError(RuntimeError):
@@ -59,7 +59,8 @@ class SbnGroupLinear(ctypes.Structure):
                 ("acc_dbg", ctypes.c_void_p), ("tokens", ctypes.c_int64),
                 ("out", ctypes.c_int64), ("in_", ctypes.c_int64), ("n", ctypes.c_int32),
                 ("m", ctypes.c_int32), ("y_is_bf16", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("reserved", ctypes.c_int32), ("ldx", ctypes.c_int64), ("ldc", ctypes.c_int64),
+                ("ldm", ctypes.c_int64)]
 
 
 class SbnPackGroupTensor(ctypes.Structure):
@@ -100,6 +101,8 @@ def lib():
         L.sbn_count_zero_codes.restype = i32
         L.sbn_count_mask_flips.argtypes = [p, p, i64, i64, i32, i32, p, p]
         L.sbn_count_mask_flips.restype = i32
+        L.sbn_gq_sum.argtypes = [p, i64, i32, p, i32, p]
+        L.sbn_gq_sum.restype = i32
         L.sbn_pack_group_sizes.argtypes = [p, i32, p, p]
         L.sbn_pack_group_sizes.restype = i32
         L.sbn_pack_group_plan.argtypes = [p, i32, p, i64]
@@ -367,18 +370,22 @@ class GroupPlan:
     Y (fp32 or bf16 [T, O]) and optionally acc_dbg (int32 [T, O]).  The tensors must stay
     alive and in place while the plan is used."""
 
-    def __init__(self, layers, device=None):
+    def __init__(self, layers, device=None, _arr=None):
         self.layers = layers
-        arr = (SbnGroupLinear * len(layers))()
-        for i, L in enumerate(layers):
-            w = L["w"]
-            Y = L["Y"]
-            arr[i] = SbnGroupLinear(
-                X=_ptr(L.get("X")), Xq=_ptr(L["Xq"]), absmax=_ptr(L["s"]), codes=_ptr(w.codes),
-                meta=_ptr(w.meta), gamma_eff=_ptr(w.gamma_eff), Y=_ptr(Y),
-                acc_dbg=_ptr(L.get("acc_dbg")), tokens=L["Xq"].shape[0], out=w.out, in_=w.in_,
-                n=w.n, m=w.m, y_is_bf16=1 if Y.dtype == torch.bfloat16 else 0, reserved=0)
-        self._arr = arr
+        if _arr is None:
+            arr = (SbnGroupLinear * len(layers))()
+            for i, L in enumerate(layers):
+                w = L["w"]
+                Y = L["Y"]
+                arr[i] = SbnGroupLinear(
+                    X=_ptr(L.get("X")), Xq=_ptr(L["Xq"]), absmax=_ptr(L["s"]),
+                    codes=_ptr(w.codes), meta=_ptr(w.meta), gamma_eff=_ptr(w.gamma_eff),
+                    Y=_ptr(Y), acc_dbg=_ptr(L.get("acc_dbg")), tokens=L["Xq"].shape[0],
+                    out=w.out, in_=w.in_, n=w.n, m=w.m,
+                    y_is_bf16=1 if Y.dtype == torch.bfloat16 else 0, reserved=0, ldx=0, ldc=0,
+                    ldm=0)
+            _arr = arr
+        arr = self._arr = _arr
         pb, wb = sbn_group_plan_sizes(arr)
         # 128-byte aligned host buffer
         raw = torch.empty(pb + 128, dtype=torch.uint8)
@@ -400,6 +407,67 @@ class GroupPlan:
 
     def linear(self, err_flag=None, stream=None):
         sbn_linear_group(self.plan_host, self.plan_dev, self.workspace, err_flag, stream)
+
+
+def sbn_gq_sum(part, n, G, Y, stream=None):
+    """Y[i] = sum over j of part[j * n + i] in j order (fp32 adds), fp32 or bf16 Y."""
+    _check(lib().sbn_gq_sum(_ptr(part), n, G, _ptr(Y), 1 if Y.dtype == torch.bfloat16 else 0,
+                            _stream(stream)), "sbn_gq_sum")
+
+
+class GqGroupPlan:
+    """The decode step of many group-quantised 2:4 layers (each packed by pack_weights_gq
+    with its own G) in three launches: the grouped quantiser (per-(token, group) scales,
+    each block of a layer being a K slice of a grouped call), the grouped contraction (each
+    block's y_j = fp32(acc_j * c_tj) into a partial buffer) and the ordered sum over the
+    blocks.  All layers share one G.  `layers`: dicts with X (bf16 [T, K], T <= 32) and w
+    (GqPackedWeights).  Allocates Xq, s ([G, T] per layer), the partials and Y (fp32 or
+    bf16; layer i's output is ``self.Y[i]``)."""
+
+    def __init__(self, layers, out_dtype=torch.float32, device=None):
+        G = layers[0]["w"].groups
+        if any(L["w"].groups != G for L in layers):
+            raise ValueError("the layers of a GqGroupPlan share one G")
+        device = device if device is not None else layers[0]["X"].device
+        self.G = G
+        # each layer's outputs start on a 16-byte boundary (the grouped call's rule for Y)
+        ns = [-(-L["X"].shape[0] * L["w"].out // 8) * 8 for L in layers]
+        self.n = sum(ns)
+        self.part = torch.zeros((G, max(self.n, 8)), dtype=torch.float32, device=device)
+        self.Yflat = torch.zeros(max(self.n, 8), dtype=out_dtype, device=device)
+        self.Xq, self.s, self.Y, slices = [], [], [], []
+        arr = (SbnGroupLinear * (G * len(layers)))()
+        off = 0
+        for i, L in enumerate(layers):
+            X, w = L["X"], L["w"]
+            T, K = X.shape
+            if not X.is_cuda or not X.is_contiguous():
+                raise ValueError("X: a contiguous CUDA tensor")
+            kg = K // G
+            Xq = torch.empty((T, K), dtype=torch.int8, device=device)
+            s = torch.empty((G, T), dtype=torch.float32, device=device)
+            self.Xq.append(Xq)
+            self.s.append(s)
+            self.Y.append(self.Yflat[off:off + T * w.out].view(T, w.out))
+            for j in range(G):
+                arr[i * G + j] = SbnGroupLinear(
+                    X=X.data_ptr() + 2 * j * kg, Xq=Xq.data_ptr() + j * kg,
+                    absmax=s.data_ptr() + 4 * j * T, codes=w.codes.data_ptr() + j * (kg // 8),
+                    meta=w.meta.data_ptr() + j * (kg // 8), gamma_eff=w.gamma_eff.data_ptr() + 4 * j,
+                    Y=self.part.data_ptr() + 4 * (j * self.part.shape[1] + off), acc_dbg=None,
+                    tokens=T, out=w.out, in_=kg, n=w.n, m=w.m, y_is_bf16=0, reserved=0, ldx=K,
+                    ldc=w.codes.shape[1], ldm=w.meta.shape[1])
+            off += ns[i]
+        self.layers = layers
+        self.plan = GroupPlan([], device=device, _arr=arr) if len(layers) else None
+
+    def quantize_acts(self, err_flag=None, stream=None):
+        self.plan.quantize_acts(err_flag, stream)
+
+    def linear(self, err_flag=None, stream=None):
+        self.plan.linear(err_flag, stream)
+        if self.n:
+            sbn_gq_sum(self.part, self.part.shape[1], self.G, self.Yflat, stream)
 
 
 # ---- grouped pack (many tensors, 6:8 and/or 2:4) -----------------------------------------

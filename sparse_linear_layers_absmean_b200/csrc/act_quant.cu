@@ -188,8 +188,9 @@ __global__ void __launch_bounds__(kAqThreads)
   const GroupRow rw = reinterpret_cast<const GroupRow *>(plan + hd.off_rows)[blockIdx.x];
   const GroupProb &p = reinterpret_cast<const GroupProb *>(plan + hd.off_probs)[rw.prob];
   const int64_t nv = p.K / 8;
-  const uint4 *row = reinterpret_cast<const uint4 *>(p.X) + (int64_t)rw.token * nv;
-  uint2 *qrow = reinterpret_cast<uint2 *>(p.Xq + (int64_t)rw.token * p.K);
+  // rows ldx elements apart (a multiple of 16): K, or more for a K slice of a wider row
+  const uint4 *row = reinterpret_cast<const uint4 *>(p.X) + (int64_t)rw.token * (p.ldx / 8);
+  uint2 *qrow = reinterpret_cast<uint2 *>(p.Xq + (int64_t)rw.token * p.ldx);
   if constexpr (R > 0) {
     uint4 v[R];
     uint32_t mx = 0;

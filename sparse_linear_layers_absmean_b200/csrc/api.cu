@@ -48,6 +48,10 @@ sbn_status check_group(const sbn_group_linear *lins, int32_t count) {
     sbn_status st = sbn_linear_ref_dims(l.out, l.in, l.n, l.m, &d);
     if (st != SBN_OK) return st;
     if (l.tokens < 0 || l.tokens > sbn::kGroupMaxTokens) return SBN_ERR_SHAPE;
+    if (l.ldx < 0 || l.ldc < 0 || l.ldm < 0) return SBN_ERR_SHAPE;
+    if ((l.ldx && (l.ldx < l.in || l.ldx % 16)) || (l.ldc && (l.ldc < d.codes_row_bytes || l.ldc % 16)) ||
+        (l.ldm && (l.ldm < d.meta_row_bytes || l.ldm % 16)))
+      return SBN_ERR_SHAPE;
     if (l.tokens == 0) continue;
     if (!l.Xq || !l.absmax || !l.codes || !l.meta || !l.gamma_eff || !l.Y) return SBN_ERR_NULL;
     if (!aligned16(l.Xq) || !aligned16(l.codes) || !aligned16(l.meta) || !aligned16(l.Y) ||
@@ -476,6 +480,15 @@ sbn_status sbn_quantize_mask_pack_weights_group(const void *plan, const void *pl
   if (!workspace) return SBN_ERR_NULL;
   return sbn::launch_pack_group(hd, plan_dev, static_cast<sbn::PackGroupSlot *>(workspace),
                                 err_flag, static_cast<cudaStream_t>(stream));
+}
+
+sbn_status sbn_gq_sum(const float *part, int64_t n, int32_t G, void *Y, int32_t y_is_bf16,
+                      void *stream) {
+  if (n < 0 || G < 1 || G > 64) return SBN_ERR_SHAPE;
+  if (n == 0) return SBN_OK;
+  if (!part || !Y) return SBN_ERR_NULL;
+  if (!aligned16(part) || !aligned16(Y)) return SBN_ERR_ALIGN;
+  return sbn::launch_gq_sum(part, n, G, Y, y_is_bf16, static_cast<cudaStream_t>(stream));
 }
 
 sbn_status sbn_count_zero_codes(const void *W, const float *gamma_eff, int64_t out, int64_t in,

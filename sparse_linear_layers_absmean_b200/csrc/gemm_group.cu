@@ -312,13 +312,18 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
     }
   } else if (warp == 5 || warp == 14) {
     // ---------------- two sparse-MMA threads: alternate super-blocks ----------------
+    // Thread mt takes the super-blocks js with js % 2 == mt, as the producers and the
+    // expander groups do, so every ring slot has one consumer and its uses stay in order.
+    // Within a unit its first super-block is then js0 or js0 + 1 (js0: the unit's first),
+    // whichever has its parity; that one starts the thread's accumulator chains.
     if (lane == 0) {
-      const int mt = warp == 5 ? 0 : 1;  // takes the unit's super-blocks j with j % 2 == mt
+      const int mt = warp == 5 ? 0 : 1;
       constexpr uint32_t idesc = ptx::idesc_i8_sparse(kGroupRows, BN);
       int64_t js = 0;
       int i = 0;
       for (int u = u0; u < u1 && !*s_abort; ++u, ++i) {
         const int nkb = unit(u).nkb;
+        const int64_t js0 = js;
         const int buf = i & 1;
         if (i >= 2 && !grp_wait(&acc_empty[buf], ((uint32_t)(i >> 1) & 1u) ^ 1u, s_abort))
           break;
@@ -326,7 +331,7 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
         const uint32_t acc0 = tmem + (uint32_t)(buf * Cfg::kAccCols);
         bool ok = true;
         for (int b0 = 0; b0 < nkb; b0 += kSuper, ++js) {
-          if (((b0 / kSuper) & 1) != mt) continue;  // by the unit's own super-block index
+          if ((int)(js & 1) != mt) continue;
           const int s1 = ring1_slot<D1>(js), s2 = (int)(js % D2);
           const uint32_t ph1 = ring1_phase<D1>(js), ph2 = (uint32_t)(js / D2) & 1u;
           if (!grp_wait(&full2[s2], ph2, s_abort) || !grp_wait(&full1[s1], ph1, s_abort)) {
@@ -342,7 +347,7 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
             const uint32_t b_addr = ptx::smem_u32(slot1 + 2 * Cfg::kPlane + g * Cfg::kBBytes);
             const uint32_t d = acc0 + (uint32_t)((mt * Cfg::kCpt + g % Cfg::kCpt) * BN);
             // the first blocks of this thread's first super-block of the unit start its chains
-            const bool first = b0 / kSuper == mt && g < Cfg::kCpt;
+            const bool first = js - js0 < 2 && g < Cfg::kCpt;
 #pragma unroll
             for (int k = 0; k < 2; ++k)  // logical K 64 per MMA: 8 columns of A, 64 bytes of B
               ptx::mma_sp_i8_tmem_a(d, a_col + 8 * k, ptx::smem_desc_sw128(b_addr + 64 * k),
@@ -365,12 +370,15 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
     const uint64_t part_off = (uint64_t)hd.ws_part_off;
     bool failed = false;
     int i = 0;
+    int64_t js = 0;  // the super-block counter of the MMA threads
     for (int u = u0; u < u1; ++u, ++i) {
       const int buf = i & 1;
       // all four warps stop together if any wait of the previous unit gave up
       if (grp_bar_any(failed)) break;
       const GroupUnit un = unit(u);
       const GroupProb &p = probs[un.prob];
+      const int js0p = (int)(js & 1);  // parity of the unit's first super-block
+      js += (un.nkb + kSuper - 1) / kSuper;
       failed = !__all_sync(0xffffffffu, !*s_abort && grp_wait(&acc_full[buf],
                                                               (uint32_t)(i >> 1) & 1u, s_abort));
       ptx::tc_fence_after();
@@ -381,8 +389,10 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
         const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * Cfg::kAccCols);
 #pragma unroll
         for (int ch = 0; ch < C; ++ch) {
-          // chain ch starts at block 4 t + r of the unit (t = ch / kCpt, r = ch % kCpt)
-          if (kSuper * (ch / Cfg::kCpt) + ch % Cfg::kCpt >= un.nkb) continue;
+          // chain ch belongs to MMA thread t = ch / kCpt, whose first super-block of the unit
+          // is the unit's local super-block (t + js0) % 2, and starts at its block r = ch % kCpt
+          const int jt = ((ch / Cfg::kCpt) + js0p) & 1;
+          if (kSuper * jt + ch % Cfg::kCpt >= un.nkb) continue;
 #pragma unroll
           for (int c = 0; c < BN; c += 16) {
             uint32_t v[16];
@@ -673,9 +683,13 @@ sbn_status group_plan(const sbn_group_linear *lins, int count, void *plan, int64
     g.O = l.out;
     g.K = l.in;
     g.y_is_bf16 = l.y_is_bf16 ? 1 : 0;
+    g.ldx = l.ldx ? l.ldx : l.in;
     if (l.tokens == 0) continue;
-    const int64_t ldc = (l.in / 8 + 15) / 16 * 16, ldm = ldc;  // 2:4: K/8 bytes per plane row
-    if (!encode_u8(&g.tx, l.Xq, l.in, l.tokens, l.in, kGroupKB, (uint32_t)ps.bn,
+    // 2:4 planes: K/8 bytes per row, strides rounded up to 16 bytes (or the caller's, for a
+    // K slice of a wider tensor's planes)
+    const int64_t ldc = l.ldc ? l.ldc : (l.in / 8 + 15) / 16 * 16;
+    const int64_t ldm = l.ldm ? l.ldm : (l.in / 8 + 15) / 16 * 16;
+    if (!encode_u8(&g.tx, l.Xq, l.in, l.tokens, g.ldx, kGroupKB, (uint32_t)ps.bn,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_u8(&g.tc, l.codes, l.in / 8, l.out, ldc, 16 * kSuper, kGroupRows,
                    CU_TENSOR_MAP_SWIZZLE_64B) ||

@@ -50,6 +50,7 @@ struct alignas(128) GroupProb {
   int64_t part_base;    // first partial tile (int32 units from ws_part_off) (split only)
   int32_t y_is_bf16;
   int32_t nparts;       // K parts per row tile
+  int64_t ldx;          // row stride (elements) of X and Xq: K, or more for a K slice
 };
 static_assert(sizeof(GroupProb) == 512, "plan layer record is 512 bytes");
 

@@ -55,12 +55,15 @@ sbn_status launch_linear_gq(const int8_t *Xq, const float *absmax, const uint8_t
                              ldm, yj, 0, aj, err_flag, st);
     if (s != SBN_OK) return s;
   }
-  const int64_t total = T * O;
-  int64_t grid = (total + 255) / 256;
+  return launch_gq_sum(part, T * O, G, Y, y_is_bf16, st);
+}
+
+sbn_status launch_gq_sum(const float *part, int64_t n, int G, void *Y, int y_is_bf16,
+                         cudaStream_t st) {
+  int64_t grid = (n + 255) / 256;
   const int64_t cap = (int64_t)num_sms() * 8;
   if (grid > cap) grid = cap;
-  return launch_pdl(k_gq_sum, dim3((unsigned)grid), dim3(256), 0, st, (const float *)part, total,
-                    G, Y, y_is_bf16);
+  return launch_pdl(k_gq_sum, dim3((unsigned)grid), dim3(256), 0, st, part, n, G, Y, y_is_bf16);
 }
 
 }  // namespace sbn

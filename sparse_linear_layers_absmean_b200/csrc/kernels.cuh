@@ -170,6 +170,10 @@ sbn_status launch_pack_gq(const void *W, int64_t out, int64_t in, int n, int m, 
                           int32_t *err_flag, cudaStream_t st);
 sbn_status launch_act_quant_gq(const void *X, int64_t tokens, int64_t in, int G, int8_t *Xq,
                                float *absmax, int32_t *err_flag, cudaStream_t st);
+// y[i] = fp32 sum over j of part[j * n + i] in j order (group quantisation).
+sbn_status launch_gq_sum(const float *part, int64_t n, int G, void *Y, int y_is_bf16,
+                         cudaStream_t st);
+
 sbn_status launch_linear_gq(const int8_t *Xq, const float *absmax, const uint8_t *codes,
                             const uint8_t *meta, const float *gamma_eff, int64_t T, int64_t O,
                             int64_t K, int n, int m, int G, int64_t ldc, int64_t ldm, void *Y,

@@ -123,7 +123,7 @@ def _group(specs, A=0x10000):
     for i, (O, K, T, n, m) in enumerate(specs):
         arr[i] = sbn.SbnGroupLinear(X=A, Xq=A, absmax=A, codes=A, meta=A, gamma_eff=A, Y=A,
                                     acc_dbg=None, tokens=T, out=O, in_=K, n=n, m=m,
-                                    y_is_bf16=0, reserved=0)
+                                    y_is_bf16=0, reserved=0, ldx=0, ldc=0, ldm=0)
     return arr
 
 
@@ -267,3 +267,22 @@ def test_pack_group_plan_mode(L, specs, mode):
                                      pb) == 0
         raw = np.frombuffer(buf, dtype=np.uint8)[base - ctypes.addressof(buf):][:pb]
         assert raw[16:20].view(np.int32)[0] == (-1 if dense else mode)
+
+
+def test_group_strides_validate(L):
+    """A layer may be a K slice of a wider one: strides at least the slice's row, multiples
+    of 16; the ordered sum of group quantisation checks its arguments on the host."""
+    arr = _group([(128, 256, 16, 2, 4)])
+    arr[0].ldx, arr[0].ldc, arr[0].ldm = 1024, 128, 128
+    assert _sizes(L, arr)[0] == 0
+    for field, bad in (("ldx", 128), ("ldx", 1040 + 8), ("ldc", 16), ("ldc", 40), ("ldm", 24),
+                       ("ldx", -16)):
+        arr = _group([(128, 256, 16, 2, 4)])
+        setattr(arr[0], field, bad)
+        assert _sizes(L, arr)[0] == 2, (field, bad)
+    A = _p(0x10000)
+    assert L.sbn_gq_sum(A, 0, 4, A, 0, None) == 0            # nothing to add
+    assert L.sbn_gq_sum(A, 16, 0, A, 0, None) == 2           # G in 1..64
+    assert L.sbn_gq_sum(A, 16, 65, A, 0, None) == 2
+    assert L.sbn_gq_sum(None, 16, 4, A, 0, None) == 1
+    assert L.sbn_gq_sum(_p(0x10004), 16, 4, A, 0, None) == 4

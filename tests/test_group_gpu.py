@@ -188,3 +188,32 @@ def test_group_full_stack_sampled():
         gpu_path.assert_y_close(L["Y"][:, ri].cpu().numpy(), oracle.rescale(acc, s, g))
     for L in layers:
         assert torch.isfinite(L["Y"]).all()
+
+
+def test_group_odd_super_blocks_repeated():
+    """Units with odd and even numbers of super-blocks (K = 384, 1152, 640, 5504: 1, 3, 2
+    and 11 super-blocks of four 128-deep K blocks) follow one another on every CTA, and the
+    plan runs 40 times back to back: which MMA thread consumes a ring slot must not depend
+    on the units' lengths (no timeout flag; every call gives the single-layer results)."""
+    Ks = [384, 1152, 640, 5504]
+    T = 16
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    layers = []
+    for i in range(64):
+        O, K = 2048, Ks[i % 4]
+        W = workloads.masters_device(O, K, device="cuda", config=5, tensor=i)
+        w = sbn.pack_weights(W, 2, 4, 1e-5, err_flag=err)
+        X = workloads.torch_bf16(workloads.student_t(T, K, config=5, tensor=1000 + i), "cuda")
+        layers.append(dict(X=X, Xq=torch.empty((T, K), dtype=torch.int8, device="cuda"),
+                           s=torch.empty((T,), dtype=torch.float32, device="cuda"), w=w,
+                           Y=torch.empty((T, O), dtype=torch.float32, device="cuda")))
+    plan = sbn.GroupPlan(layers)
+    plan.quantize_acts(err_flag=err)
+    torch.cuda.synchronize()
+    refs = [sbn.linear(L["Xq"], L["s"], L["w"]) for L in layers]
+    for _ in range(40):
+        plan.linear(err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    for L, Y in zip(layers, refs):
+        assert torch.equal(L["Y"], Y)
