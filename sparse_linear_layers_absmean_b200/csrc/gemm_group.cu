@@ -23,13 +23,15 @@
 //              (groups outside the matrix get the valid index pair (0, 1)) into TMEM lane r
 //              with tcgen05.st; one wait and one arrival per super-block.  A never passes
 //              through shared memory, and no tcgen05.cp is needed.
-//   warps 5, 14  two MMA threads taking alternate super-blocks (the issue of a tcgen05.mma
-//              of this small shape, not the tensor pipe, sets the pace of one thread): per
-//              block two sparse MMAs (M 128, N bn, logical K 64 each; A and the metadata read
-//              from TMEM, B from shared memory) into one of the thread's two accumulator
-//              chains; one commit frees both rings' slots per super-block; at a unit's end
-//              both commit its accumulators to the epilogue and the next unit starts in the
-//              other set (warp 5 also allocates TMEM).
+//   warps 5, 14, 16, 17  MMA threads (four at bn 16, two at bn 32) taking every fourth
+//              (second) super-block (the issue of a tcgen05.mma of this small shape, not the
+//              tensor pipe, sets the pace of one thread): per block two sparse MMAs (M 128,
+//              N bn, logical K 64 each; A and the metadata read from TMEM, B from shared
+//              memory) into the thread's accumulator chain(s); one commit frees both rings'
+//              slots per super-block; at a unit's end all commit its accumulators to the
+//              epilogue and the next unit starts in the other set (warp 5 also allocates
+//              TMEM).  Every role picks super-blocks by the CTA's running counter, so each
+//              ring slot has one producer and one consumer.
 //   warps 6-9  epilogue: drain and add the chains (tcgen05.ld), release them, rescale by
 //              c_t = fp32(fp32(g * s_t) / 127) and store fp32 or bf16.  A row tile whose K
 //              blocks were split over several units writes its int32 partial to the
@@ -53,7 +55,8 @@ namespace sbn {
 
 namespace {
 
-constexpr int kGrpThreads = 512;  // 16 warps (two expander groups, two TMA and two MMA threads)
+// 18 warps: two expander groups, two TMA producers, up to four MMA threads, the epilogue
+constexpr int kGrpThreads = 576;
 constexpr long long kGrpWaitCycles = 1ll << 31;  // about 1 s at 1.9 GHz
 constexpr int kSuper = 4;  // K blocks per weight super-block (one 64-byte box per row)
 
@@ -69,11 +72,17 @@ struct GrpCfg {
   // ring 2 in TMEM, one slot per super-block: per block the compressed A tile (lane r = row r,
   // 16 columns of four int8 values) and the metadata (4 columns)
   static constexpr int kD2 = BN <= 16 ? 4 : 2;
-  // accumulator chains per unit: two MMA threads take alternate super-blocks, each into its
-  // own kChains / 2 chains (block b of its super-blocks into chain b mod (kChains / 2)); the
-  // epilogue adds the chains
+  static_assert(kD1 % (BN <= 16 ? 4 : 2) == 0 && kD2 % (BN <= 16 ? 4 : 2) == 0,
+                "one consumer per ring slot: ring depths are multiples of the MMA threads");
+  // kMma MMA threads take every kMma-th super-block (by the running counter, as the
+  // producers and expanders do): each ring slot keeps one consumer because both rings'
+  // depths are multiples of kMma.  Four threads at 16 tokens (each MMA of N 16 is short and
+  // one thread issues one per ~100 cycles), two at 32 (the TMEM ring has two slots there).
+  static constexpr int kMma = BN <= 16 ? 4 : 2;
+  // accumulator chains per unit: each MMA thread owns kChains / kMma of them (block b of its
+  // super-blocks into chain b mod kCpt); the epilogue adds the chains
   static constexpr int kChains = 4;
-  static constexpr int kCpt = kChains / 2;  // chains per MMA thread
+  static constexpr int kCpt = kChains / kMma;  // chains per MMA thread
   static constexpr int kAccCols = kChains * BN;         // one unit's accumulators
   static constexpr int kACol = 2 * kAccCols;            // A ring after the two units' accumulators
   static constexpr int kAColsPerSlot = kSuper * 16;
@@ -188,10 +197,10 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
       ptx::mbar_init(&empty2[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(&acc_full[b], 2);  // both MMA threads commit
+      ptx::mbar_init(&acc_full[b], Cfg::kMma);  // every MMA thread commits
       ptx::mbar_init(&acc_empty[b], 4);
     }
-    ptx::mbar_init(mma_done, 2);
+    ptx::mbar_init(mma_done, Cfg::kMma);
     *s_abort = 0;
     ptx::fence_mbar_init();
   }
@@ -310,14 +319,13 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
       for (int64_t q = issued, i = 0; q >= 0 && i < D1 / 2; q -= 2, ++i)
         if (!grp_drain(&full1[ring1_slot<D1>(q)], ring1_phase<D1>(q))) *s_abort = 1;
     }
-  } else if (warp == 5 || warp == 14) {
-    // ---------------- two sparse-MMA threads: alternate super-blocks ----------------
-    // Thread mt takes the super-blocks js with js % 2 == mt, as the producers and the
-    // expander groups do, so every ring slot has one consumer and its uses stay in order.
-    // Within a unit its first super-block is then js0 or js0 + 1 (js0: the unit's first),
-    // whichever has its parity; that one starts the thread's accumulator chains.
-    if (lane == 0) {
-      const int mt = warp == 5 ? 0 : 1;
+  } else if (warp == 5 || warp == 14 || warp >= 16) {
+    // ---------------- kMma sparse-MMA threads (warps 5, 14, 16, 17) ----------------
+    // Thread mt takes the super-blocks js with js % kMma == mt, so every ring slot has one
+    // consumer and its uses stay in order.  Within a unit its first super-block is then one
+    // of js0 .. js0 + kMma - 1 (js0: the unit's first); that one starts its chains.
+    const int mt = warp == 5 ? 0 : warp == 14 ? 1 : warp - 14;
+    if (lane == 0 && mt < Cfg::kMma) {
       constexpr uint32_t idesc = ptx::idesc_i8_sparse(kGroupRows, BN);
       int64_t js = 0;
       int i = 0;
@@ -331,7 +339,7 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
         const uint32_t acc0 = tmem + (uint32_t)(buf * Cfg::kAccCols);
         bool ok = true;
         for (int b0 = 0; b0 < nkb; b0 += kSuper, ++js) {
-          if ((int)(js & 1) != mt) continue;
+          if ((int)(js % Cfg::kMma) != mt) continue;
           const int s1 = ring1_slot<D1>(js), s2 = (int)(js % D2);
           const uint32_t ph1 = ring1_phase<D1>(js), ph2 = (uint32_t)(js / D2) & 1u;
           if (!grp_wait(&full2[s2], ph2, s_abort) || !grp_wait(&full1[s1], ph1, s_abort)) {
@@ -347,7 +355,7 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
             const uint32_t b_addr = ptx::smem_u32(slot1 + 2 * Cfg::kPlane + g * Cfg::kBBytes);
             const uint32_t d = acc0 + (uint32_t)((mt * Cfg::kCpt + g % Cfg::kCpt) * BN);
             // the first blocks of this thread's first super-block of the unit start its chains
-            const bool first = js - js0 < 2 && g < Cfg::kCpt;
+            const bool first = js - js0 < Cfg::kMma && g < Cfg::kCpt;
 #pragma unroll
             for (int k = 0; k < 2; ++k)  // logical K 64 per MMA: 8 columns of A, 64 bytes of B
               ptx::mma_sp_i8_tmem_a(d, a_col + 8 * k, ptx::smem_desc_sw128(b_addr + 64 * k),
@@ -377,7 +385,7 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
       if (grp_bar_any(failed)) break;
       const GroupUnit un = unit(u);
       const GroupProb &p = probs[un.prob];
-      const int js0p = (int)(js & 1);  // parity of the unit's first super-block
+      const int js0m = (int)(js % Cfg::kMma);  // the unit's first super-block, mod kMma
       js += (un.nkb + kSuper - 1) / kSuper;
       failed = !__all_sync(0xffffffffu, !*s_abort && grp_wait(&acc_full[buf],
                                                               (uint32_t)(i >> 1) & 1u, s_abort));
@@ -390,8 +398,9 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
 #pragma unroll
         for (int ch = 0; ch < C; ++ch) {
           // chain ch belongs to MMA thread t = ch / kCpt, whose first super-block of the unit
-          // is the unit's local super-block (t + js0) % 2, and starts at its block r = ch % kCpt
-          const int jt = ((ch / Cfg::kCpt) + js0p) & 1;
+          // is the unit's local super-block (t - js0) mod kMma, and starts at its block
+          // r = ch % kCpt
+          const int jt = ((ch / Cfg::kCpt) - js0m + Cfg::kMma) % Cfg::kMma;
           if (kSuper * jt + ch % Cfg::kCpt >= un.nkb) continue;
 #pragma unroll
           for (int c = 0; c < BN; c += 16) {
