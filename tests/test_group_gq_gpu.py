@@ -87,3 +87,20 @@ def test_gq_grouped_twice():
         L["X"].copy_(workloads.torch_bf16(X2, "cuda"))
         host2.append((W_bits, X2))
     check(plan, layers, host2, 2)
+
+
+@pytest.mark.parametrize("G,n", [(1, 100), (2, 1 << 16), (5, 4096 + 3), (64, 257)])
+def test_gq_sum(G, n):
+    """sbn_gq_sum: y[i] = part[0, i] + part[1, i] + ... in that order, in fp32."""
+    rng = np.random.default_rng(G + n)
+    part = (rng.standard_normal((G, n)) * 10.0 ** rng.integers(-3, 4, (G, n))).astype(np.float32)
+    ref = part[0].copy()
+    for j in range(1, G):
+        ref = (ref + part[j]).astype(np.float32)
+    pt = torch.from_numpy(part).cuda()
+    for dt in (torch.float32, torch.bfloat16):
+        Y = torch.empty(n, dtype=dt, device="cuda")
+        sbn.sbn_gq_sum(pt, n, G, Y)
+        torch.cuda.synchronize()
+        want = torch.from_numpy(ref).to(dt)
+        assert torch.equal(Y.cpu(), want)
