@@ -683,11 +683,12 @@ __device__ __forceinline__ bool bar_any(int id, int n, bool pred) {
 // CTA-pair 2:4 kernel for large token counts.  A cluster of two CTAs computes 256 weight
 // rows x BN tokens per tile with the pair form of the sparse MMA: each CTA stages and
 // expands its own 128 rows and loads half of the activation tile (BN / 2 tokens), so every
-// SM streams half the activation bytes of a single-CTA tile per unit of MMA work.  CTA 0 of
-// the pair issues the MMAs and the commits for both (commits reach the same barrier in
-// both CTAs); the expanders and the epilogue warps of both CTAs report to CTA 0's
-// barriers.  Persistent over tiles with two TMEM accumulators (columns 0 and 256) per CTA:
-// the epilogue warps drain tile i while the MMA already accumulates tile i+1.
+// SM streams half the activation bytes of a single-CTA tile per unit of MMA work.  Two
+// threads of CTA 0 issue the MMAs and the commits for both CTAs (commits reach the same
+// barrier in both), alternate stages each; the expanders and the epilogue warps of both
+// CTAs report to CTA 0's barriers.  Persistent over tiles with two TMEM accumulators
+// (columns 0 and 256) per CTA: the epilogue warps drain tile i (and zero its accumulator)
+// while the MMAs already accumulate tile i+1.
 //
 // A and its metadata live in TMEM: the expanders write each row's expanded codes (16
 // columns per K block) and its metadata (4 columns) into their CTA's TMEM (tcgen05.st,
@@ -699,7 +700,8 @@ __device__ __forceinline__ bool bar_any(int id, int n, bool pred) {
 // stage kg - S2's commit before they write stage kg's ring-2 slot.  The tile width 208 puts
 // a 2048-token batch in 10 token tiles (six rounds of tiles on 74 pairs for 11008 rows).
 // ---------------------------------------------------------------------------------------
-constexpr int kPairThreads = 352;  // 11 warps: expanders 0-3, producers 4 and 10, MMA 5, epilogue 6-9
+// 12 warps: expanders 0-3, producers 4 and 10, MMA threads in warps 5 and 11, epilogue 6-9
+constexpr int kPairThreads = 384;
 
 template <int BN>
 struct PairCfg {
@@ -781,10 +783,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     for (int s = 0; s < S2; ++s)
       ptx::mbar_init(&full_a[s], 8);  // the expander warps of both CTAs (used in CTA 0)
     for (int b = 0; b < 2; ++b) {
-      ptx::mbar_init(&acc_full[b], 1);
-      ptx::mbar_init(&acc_empty[b], 8);
+      ptx::mbar_init(&acc_full[b], 2);   // a commit of each MMA thread
+      ptx::mbar_init(&acc_empty[b], 8);  // the epilogue warps of both CTAs
     }
-    ptx::mbar_init(mma_done, 1);
+    ptx::mbar_init(mma_done, 2);
     *s_abort = 0;
     ptx::fence_mbar_init();
   }
@@ -890,23 +892,29 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       for (int64_t q = issued, i = 0; q >= 0 && i < S1 / 2; q -= 2, ++i)
         if (!wait_phase(&full_t[q % S1], (uint32_t)(q / S1) & 1u)) *s_abort = 1;
     }
-  } else if (warp == 5) {
-    // ---------------- CTA 0: the pair's MMAs ----------------
+  } else if (warp == 5 || warp == 11) {
+    // ---------------- CTA 0: the pair's MMAs, stage kg by MMA thread kg % 2 ----------------
+    // Every MMA accumulates: the epilogue zeroes an accumulator before its tile (integer
+    // sums, so the order in which the two threads' MMAs reach it does not matter).  A thread's
+    // commit covers its own MMAs: stage kg's slots are freed by the thread that issued kg.
     if (rank == 0 && lane == 0) {
+      const int mt = warp == 5 ? 0 : 1;
       constexpr uint32_t idesc = ptx::idesc_i8_sparse(kTileM, BN);
       // B descriptor of ring 1's first byte; a slot, block and K half add (offset >> 4)
       const uint64_t b_desc0 = ptx::smem_desc_sw128(ptx::smem_u32(ring1));
-      int s1 = 0, s2 = 0;
+      // this thread's next stage kg = mt, mt + 2, ...: its ring slots (S1 and S2 are even)
+      int s1 = mt, s2 = mt;
       uint32_t ph2 = 0;
+      int64_t kg = 0;
       int i = 0;
       for (int64_t tile = pair; tile < ntiles && !*s_abort; tile += npairs, ++i) {
         const int buf = i & 1;
-        if (i >= 2 && !wait_or_abort(&acc_empty[buf], ((uint32_t)(i >> 1) & 1u) ^ 1u, s_abort))
-          break;
+        if (!wait_or_abort(&acc_empty[buf], (uint32_t)(i >> 1) & 1u, s_abort)) break;
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(buf * Cfg::kAccStride);
         bool ok = true;
-        for (int j = 0; j < nst; ++j) {
+        for (int j = 0; j < nst; ++j, ++kg) {
+          if ((int)(kg & 1) != mt) continue;
           // both CTAs expanded this stage, after their own B and planes had landed
           if (!wait_or_abort(&full_a[s2], ph2, s_abort)) {
             ok = false;
@@ -921,11 +929,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             for (int k = 0; k < 2; ++k)
               ptx::mma_sp_i8_pair_tmem_a(d_tmem, tmem + Cfg::a_col(b2) + 8 * k,
                                          b_desc + (uint64_t)((g * Cfg::kBBytes + 64 * k) >> 4),
-                                         tmem + Cfg::e_col(b2) + 2 * k, idesc, (j | g | k) != 0);
+                                         tmem + Cfg::e_col(b2) + 2 * k, idesc, 1u);
           }
           ptx::mma_commit_pair(&empty1[s1], 0x3);
-          if (++s1 == S1) s1 = 0;
-          if (++s2 == S2) s2 = 0, ph2 ^= 1u;
+          if ((s1 += 2) >= S1) s1 -= S1;
+          if ((s2 += 2) >= S2) s2 -= S2, ph2 ^= 1u;
         }
         if (!ok) break;
         ptx::mma_commit_pair(&acc_full[buf], 0x3);
@@ -938,6 +946,19 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const int q = warp & 3;
     const int et = threadIdx.x - 6 * 32;
     const float g = __ldg(gamma_eff);
+    const uint32_t zero[16] = {};
+    const uint32_t tlane = tmem + ((uint32_t)(q * 32) << 16);
+    // both accumulators start at zero; each is zeroed again after its tile is read
+#pragma unroll 1
+    for (int b = 0; b < 2; ++b)
+      for (int c = 0; c < BN; c += 16) ptx::tmem_st_16(tlane + b * Cfg::kAccStride + c, zero);
+    ptx::tmem_st_wait();
+    ptx::tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+      ptx::mbar_arrive_cluster(acc_empty0);
+      ptx::mbar_arrive_cluster(acc_empty0 + 8u);
+    }
     bool failed = false;
     int i = 0;
     for (int64_t tile = pair; tile < ntiles; tile += npairs, ++i) {
@@ -955,9 +976,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                                                                    s_abort));
       ptx::tc_fence_after();
       if (!failed) {
-        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * Cfg::kAccStride);
+        const uint32_t trow = tlane + (uint32_t)(buf * Cfg::kAccStride);
         store_tile<BN>(trow, s_scale, o0 + q * 32 + lane, O, t0, T, K <= 32768, Y, y_is_bf16,
                        acc_dbg);
+        for (int c = 0; c < BN; c += 16) ptx::tmem_st_16(trow + c, zero);
+        ptx::tmem_st_wait();
       }
       ptx::tc_fence_before();
       __syncwarp();
