@@ -1,7 +1,9 @@
 // Per-token absmax int8 activation quantisation ("Marco de inferencia de Microsoft lleva
 // modelos de lenguaje grande de 1 bit a dispositivos locales", unite.ai, "Fundamento
 // matemático" item 2; Qb = 127):
-//   s = max(max_k |x_k|, 1e-5),  q_k = clamp(rint((127 * x_k) / s), -127, 127).
+//   s = max(max_k |x_k|, 1e-5),  q_k = clamp(rint((127 * x_k) / s), -127, 127),
+// the quotient rounded as the IEEE divide rounds it (act_codes8: products with the token's
+// reciprocal, and the divide itself where a product lies near a half-integer).
 // Few tokens: one CTA per token; rows of up to 16384 inputs stay in registers between the
 // max pass and the quantise pass (one HBM read), longer rows are read twice.  Many tokens
 // with rows of up to 4096 inputs: one warp per token (k_act_quant_warp).  Every kernel is
@@ -16,20 +18,9 @@ namespace sbn {
 
 constexpr int kAqThreads = 256;
 
-__device__ __forceinline__ uint32_t quant_pair(uint32_t w, float s) {
-  // two bf16 values -> two int8 codes in the low 16 bits
-  float xl = bf16_lo_to_float(w), xh = bf16_hi_to_float(w);
-  int ql = __float2int_rn(__fdiv_rn(__fmul_rn(127.0f, xl), s));
-  int qh = __float2int_rn(__fdiv_rn(__fmul_rn(127.0f, xh), s));
-  ql = min(127, max(-127, ql));
-  qh = min(127, max(-127, qh));
-  return ((uint32_t)ql & 0xffu) | (((uint32_t)qh & 0xffu) << 8);
-}
-
-__device__ __forceinline__ uint2 quant_vec8(uint4 v, float s) {
-  uint32_t a = quant_pair(v.x, s) | (quant_pair(v.y, s) << 16);
-  uint32_t b = quant_pair(v.z, s) | (quant_pair(v.w, s) << 16);
-  return make_uint2(a, b);
+// eight bf16 values -> eight int8 codes; inv = fl(1 / s)
+__device__ __forceinline__ uint2 quant_vec8(uint4 v, float s, float inv) {
+  return act_codes_vec8(v, s, inv);
 }
 
 __device__ __forceinline__ uint32_t vec8_absmax_bits(uint4 v, uint32_t mx) {
@@ -70,12 +61,13 @@ __global__ void __launch_bounds__(kAqThreads)
     mx = vec8_absmax_bits(v[r], mx);
   }
   const float s = block_scale(mx, err_flag);
+  const float inv = __frcp_rn(s);
   if (threadIdx.x == 0) absmax[t] = s;
   uint2 *qrow = reinterpret_cast<uint2 *>(Xq + t * nv * 8);
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     int64_t i = threadIdx.x + (int64_t)r * kAqThreads;
-    if (i < nv) qrow[i] = quant_vec8(v[r], s);
+    if (i < nv) qrow[i] = quant_vec8(v[r], s, inv);
   }
 }
 
@@ -89,9 +81,10 @@ __global__ void __launch_bounds__(kAqThreads)
   uint32_t mx = 0;
   for (int64_t i = threadIdx.x; i < nv; i += kAqThreads) mx = vec8_absmax_bits(__ldg(row + i), mx);
   const float s = block_scale(mx, err_flag);
+  const float inv = __frcp_rn(s);
   if (threadIdx.x == 0) absmax[t] = s;
   uint2 *qrow = reinterpret_cast<uint2 *>(Xq + t * nv * 8);
-  for (int64_t i = threadIdx.x; i < nv; i += kAqThreads) qrow[i] = quant_vec8(__ldg(row + i), s);
+  for (int64_t i = threadIdx.x; i < nv; i += kAqThreads) qrow[i] = quant_vec8(__ldg(row + i), s, inv);
 }
 
 // One warp per token for rows of up to 32 * 8 * R inputs: the whole row stays in the
@@ -119,12 +112,13 @@ __global__ void __launch_bounds__(kAqThreads)
   const uint32_t m = warp_max_u32(max(mx & 0xffffu, mx >> 16));
   if (m >= kBf16InfBits && lane == 0 && err_flag) atomicOr(err_flag, SBN_FLAG_X_NONFINITE);
   const float s = fmaxf(__uint_as_float(m << 16), 1e-5f);
+  const float inv = __frcp_rn(s);
   if (lane == 0) absmax[t] = s;
   uint2 *qrow = reinterpret_cast<uint2 *>(Xq + t * nv * 8);
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     const int64_t i = lane + 32 * r;
-    if (i < nv) qrow[i] = quant_vec8(v[r], s);
+    if (i < nv) qrow[i] = quant_vec8(v[r], s, inv);
   }
 }
 
@@ -150,18 +144,20 @@ __global__ void __launch_bounds__(kAqThreads)
       mx = vec8_absmax_bits(v[r], mx);
     }
     const float s = block_scale(mx, err_flag);
+    const float inv = __frcp_rn(s);
     if (threadIdx.x == 0) absmax[j * tokens + t] = s;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int64_t i = threadIdx.x + (int64_t)r * kAqThreads;
-      if (i < nv) qrow[i] = quant_vec8(v[r], s);
+      if (i < nv) qrow[i] = quant_vec8(v[r], s, inv);
     }
   } else {
     uint32_t mx = 0;
     for (int64_t i = threadIdx.x; i < nv; i += kAqThreads) mx = vec8_absmax_bits(__ldg(row + i), mx);
     const float s = block_scale(mx, err_flag);
+    const float inv = __frcp_rn(s);
     if (threadIdx.x == 0) absmax[j * tokens + t] = s;
-    for (int64_t i = threadIdx.x; i < nv; i += kAqThreads) qrow[i] = quant_vec8(__ldg(row + i), s);
+    for (int64_t i = threadIdx.x; i < nv; i += kAqThreads) qrow[i] = quant_vec8(__ldg(row + i), s, inv);
   }
 }
 
@@ -201,18 +197,20 @@ __global__ void __launch_bounds__(kAqThreads)
       mx = vec8_absmax_bits(v[r], mx);
     }
     const float s = block_scale(mx, err_flag);
+    const float inv = __frcp_rn(s);
     if (threadIdx.x == 0) p.absmax[rw.token] = s;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int64_t i = threadIdx.x + (int64_t)r * kAqThreads;
-      if (i < nv) qrow[i] = quant_vec8(v[r], s);
+      if (i < nv) qrow[i] = quant_vec8(v[r], s, inv);
     }
   } else {
     uint32_t mx = 0;
     for (int64_t i = threadIdx.x; i < nv; i += kAqThreads) mx = vec8_absmax_bits(__ldg(row + i), mx);
     const float s = block_scale(mx, err_flag);
+    const float inv = __frcp_rn(s);
     if (threadIdx.x == 0) p.absmax[rw.token] = s;
-    for (int64_t i = threadIdx.x; i < nv; i += kAqThreads) qrow[i] = quant_vec8(__ldg(row + i), s);
+    for (int64_t i = threadIdx.x; i < nv; i += kAqThreads) qrow[i] = quant_vec8(__ldg(row + i), s, inv);
   }
 }
 
@@ -222,10 +220,13 @@ sbn_status launch_act_quant_group(const void *plan_host, const void *plan_dev, i
   if (hd->nrows == 0) return SBN_OK;
   const uint8_t *P = static_cast<const uint8_t *>(plan_dev);
   const dim3 grid((unsigned)hd->nrows), block(kAqThreads);
+  // When no row has more than 4096 inputs, rows stay in registers.  Otherwise every row is
+  // read twice (the second read from L2): holding 8 words per thread keeps 4 CTAs per SM
+  // resident, the two-pass form about twice as many, and with one short row per CTA the
+  // number of rows in flight decides the time (the 160-layer, 16-token stack: 14.7 us with
+  // 8 words per thread, 13.5 us in two passes).
   if (hd->max_nv <= 2 * kAqThreads)
     return launch_pdl(k_act_quant_group<2>, grid, block, 0, st, P, err_flag);
-  if (hd->max_nv <= 8 * kAqThreads)
-    return launch_pdl(k_act_quant_group<8>, grid, block, 0, st, P, err_flag);
   return launch_pdl(k_act_quant_group<0>, grid, block, 0, st, P, err_flag);
 }
 

@@ -39,6 +39,52 @@ __device__ __forceinline__ uint32_t warp_or_u32(uint32_t v) {
   return __reduce_or_sync(0xffffffffu, v);
 }
 
+// Activation codes q = clamp(rint(fl(r / s)), -127, 127) of eight values r = fl(127 x) of one
+// token, with the quotient rounded as the IEEE divide rounds it, from the products
+// p = fl(r * inv), inv = fl(1 / s) (correctly rounded, once per token).  inv and the product
+// each carry a relative error of at most 2^-24 and the rounded quotient another 2^-24, so
+// for |r / s| < 128 the product is within 3 * 128 * 2^-24 < 2^-15 of the rounded quotient.
+// rint changes value only at half-integers: a product farther than 2^-15 from every k + 1/2
+// rounds to the same integer as the rounded quotient.  When one of the eight lies nearer
+// (exact ties among them), all eight take the divide, on a branch of their own.  Past
+// +-127.5 both sides clamp to the same code; NaN and infinity propagate through the product
+// as through the divide.
+__device__ __forceinline__ void act_codes8(const float (&r)[8], float s, float inv,
+                                           int (&q)[8]) {
+  float p[8];
+  bool near = false;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    p[i] = __fmul_rn(r[i], inv);
+    // distance to the nearest integer (exact); at least 1/2 - 2^-15 <=> within 2^-15 of a
+    // half-integer.  NaN and infinity give NaN here and stay on the product.
+    near |= fabsf(__fsub_rn(p[i], rintf(p[i]))) >= 0.5f - 0x1p-15f;
+  }
+  if (near) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) p[i] = __fdiv_rn(r[i], s);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) q[i] = min(127, max(-127, __float2int_rn(p[i])));
+}
+
+// Eight bf16 activations (one 16-byte word) -> eight int8 codes, in order.
+__device__ __forceinline__ uint2 act_codes_vec8(uint4 v, float s, float inv) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float r[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    r[2 * i] = __fmul_rn(127.0f, bf16_lo_to_float(w[i]));
+    r[2 * i + 1] = __fmul_rn(127.0f, bf16_hi_to_float(w[i]));
+  }
+  int q[8];
+  act_codes8(r, s, inv, q);
+  uint32_t o[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i >> 2] |= ((uint32_t)q[i] & 0xffu) << (8 * (i & 3));
+  return make_uint2(o[0], o[1]);
+}
+
 // Per-token activation scale and weight scale combined as the rescale factor
 // c = fp32(fp32(g * s) / 127), then y = fp32(acc * c); no FMA contraction anywhere.
 __device__ __forceinline__ float rescale_factor(float g, float s) {

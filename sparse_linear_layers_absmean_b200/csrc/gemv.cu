@@ -143,7 +143,8 @@ __global__ void __launch_bounds__(kGvThreads)
 
 // Steps 5-7 in one launch for a few tokens: every CTA quantises the (small) token rows
 // itself -- the per-token absmax by a block reduction over X (bf16, read from L2), then
-// q = clamp(rint((127 x) / s), -127, 127) with the IEEE divide into shared memory -- and
+// q = clamp(rint((127 x) / s), -127, 127) (rounded as the IEEE divide rounds the quotient)
+// into shared memory -- and
 // runs the GEMV above on them (two rows per warp, 8 warps per CTA, activations from shared
 // memory).  CTA 0 also writes Xq and s to global memory.  Shared memory: T * in bytes
 // (in <= 16384).
@@ -151,15 +152,6 @@ constexpr int64_t kFusedMaxIn = 16384;
 // 8 warps (16 rows) per CTA: the row quantisation every CTA repeats is spread over 256
 // threads and over 2x fewer CTAs than the GEMV's 8-row CTAs
 constexpr int kGfThreads = 256;
-
-__device__ __forceinline__ uint32_t fused_q2(uint32_t w, float s) {
-  const float xl = bf16_lo_to_float(w), xh = bf16_hi_to_float(w);
-  int ql = __float2int_rn(__fdiv_rn(__fmul_rn(127.0f, xl), s));
-  int qh = __float2int_rn(__fdiv_rn(__fmul_rn(127.0f, xh), s));
-  ql = min(127, max(-127, ql));
-  qh = min(127, max(-127, qh));
-  return ((uint32_t)ql & 0xffu) | (((uint32_t)qh & 0xffu) << 8);
-}
 
 template <int T, int SPL, bool kCompact>
 __global__ void __launch_bounds__(kGfThreads)
@@ -204,13 +196,13 @@ __global__ void __launch_bounds__(kGfThreads)
   for (int t = 0; t < T; ++t) {
     if (t >= nt) break;
     const float sc = s_scale[t];
+    const float inv = __frcp_rn(sc);
     const uint4 *row = reinterpret_cast<const uint4 *>(X + t * in);
     uint2 *q = reinterpret_cast<uint2 *>(s_xq + t * in);
     uint2 *qg = Xq_out ? reinterpret_cast<uint2 *>(Xq_out + t * in) : nullptr;
     for (int64_t i = threadIdx.x; i < nv; i += kGfThreads) {
       const uint4 v = __ldg(row + i);
-      const uint2 o = make_uint2(fused_q2(v.x, sc) | (fused_q2(v.y, sc) << 16),
-                                 fused_q2(v.z, sc) | (fused_q2(v.w, sc) << 16));
+      const uint2 o = act_codes_vec8(v, sc, inv);
       q[i] = o;
       if (blockIdx.x == 0 && qg) qg[i] = o;
     }

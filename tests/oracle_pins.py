@@ -160,6 +160,22 @@ def rounding_ties(o):
     assert s[0] == 127 and Xq[0].tolist() == [0, 127, 62, -62, 62, 0, 2, 2], Xq
 
 
+def act_quotient_ties(o):
+    # every exact tie of 127 x / s in three row scales; ties go to the even integer
+    # (np.rint rounds half to even).  s = 127: the quotient is x; s = 254: x / 2 for odd x;
+    # s = 127/64: 64 x for x = (2k + 1) / 128
+    half = np.arange(-127, 127) + 0.5
+    odd = np.arange(-253, 254, 2).astype(np.float64)
+    for s, x, quot in [(127.0, half, half), (254.0, odd, odd / 2),
+                       (127.0 / 64, (2 * np.arange(-127, 127) + 1) / 128.0, half)]:
+        row = np.concatenate([[s], x, [-s / 2]]).astype(np.float32)[None, :]
+        Xq, sc, err = o.quant_acts(workloads.to_bf16_bits(row))
+        assert err == 0 and sc[0] == np.float32(s)
+        want = np.rint(quot).astype(np.int64)
+        assert np.array_equal(Xq[0, 1:1 + len(x)].astype(np.int64), want), (s, Xq[0, :8])
+        assert Xq[0, 0] == 127
+
+
 def dense_pattern(o):
     W = workloads.masters(5, 128, seed=5)
     for m in (4, 8):
@@ -470,7 +486,8 @@ def group_hand(o):
     assert float(r1["gamma"][0]) == float(g["gamma_g1"][0]) and r1["t"][0, 1] == 0
 
 
-ALL = [hand_example, mask_bruteforce, gamma_closed_form, rounding_ties, dense_pattern,
+ALL = [hand_example, mask_bruteforce, gamma_closed_form, rounding_ties, act_quotient_ties,
+       dense_pattern,
        constant_magnitude, act_absmax, contract_bruteforce, unpack_roundtrip, invariants,
        scale_invariance, rescale_closed_form, mask_stats, group_one, group_slices, group_hand,
        backward_hand, backward_adjoint]
