@@ -4,9 +4,9 @@
 //   s = max(max_k |x_k|, 1e-5),  q_k = clamp(rint((127 * x_k) / s), -127, 127),
 // the quotient rounded as the IEEE divide rounds it (act_codes8: products with the token's
 // reciprocal, and the divide itself where a product lies near a half-integer).
-// Few tokens: one CTA per token; rows of up to 16384 inputs stay in registers between the
-// max pass and the quantise pass (one HBM read), longer rows are read twice.  Many tokens
-// with rows of up to 4096 inputs: one warp per token (k_act_quant_warp).  Every kernel is
+// One CTA per token; rows of up to 16384 inputs stay in registers between the max pass and
+// the quantise pass (one HBM read), longer rows are read twice.  Many tokens with rows of up
+// to 1024 inputs: one warp per token (k_act_quant_warp).  Every kernel is
 // launched as a programmatic dependent of the previous kernel on the stream and waits for
 // it before reading X.
 #include "common.cuh"
@@ -235,16 +235,13 @@ sbn_status launch_act_quant(const void *X, int64_t tokens, int64_t in, int8_t *X
   const int64_t nv = in / 8;
   const uint4 *X4 = reinterpret_cast<const uint4 *>(X);
   const dim3 block(kAqThreads);
-  if (tokens > 16 && nv <= 32 * 16) {
-    // many tokens: one warp each (a CTA-wide reduction per token costs more than the row)
+  if (tokens > 16 && nv <= 32 * 4) {
+    // many tokens with rows of up to 1024 inputs: one warp each (a CTA-wide reduction per
+    // token costs more than such a row).  Longer rows take a CTA per token: one warp per
+    // token leaves each warp a long serial run of codes and the SMs mostly idle (2048 x 4096:
+    // 11.4 us with a warp per token, 6.8 us with a CTA per token).
     const dim3 wgrid((unsigned)((tokens + kAqThreads / 32 - 1) / (kAqThreads / 32)));
-    if (nv <= 32 * 4)
-      return launch_pdl(k_act_quant_warp<4>, wgrid, block, 0, st, X4, tokens, nv, Xq, absmax,
-                        err_flag);
-    if (nv <= 32 * 8)
-      return launch_pdl(k_act_quant_warp<8>, wgrid, block, 0, st, X4, tokens, nv, Xq, absmax,
-                        err_flag);
-    return launch_pdl(k_act_quant_warp<16>, wgrid, block, 0, st, X4, tokens, nv, Xq, absmax,
+    return launch_pdl(k_act_quant_warp<4>, wgrid, block, 0, st, X4, tokens, nv, Xq, absmax,
                       err_flag);
   }
   const dim3 grid((unsigned)tokens);

@@ -119,8 +119,9 @@ def test_pack_flags_bad_weights(bad, flag):
                                  (2, 20480), (17, 64), (300, 1024), (101, 2048), (40, 4160),
                                  (1000, 3200)])
 def test_act_quant(T, K):
-    """Few tokens take the one-CTA-per-token kernel, many tokens with rows up to 4096 the
-    one-warp-per-token kernel (ragged last CTA in each case)."""
+    """Rows of more than 1024 inputs, and few tokens, take the one-CTA-per-token kernels
+    (rows in registers, or read twice past 16384); many tokens with rows of up to 1024 the
+    one-warp-per-token kernel (ragged last CTA)."""
     X = workloads.activations(T, K, seed=T * K)
     X[0, :7] = workloads.to_bf16_bits(np.array([0.5, -0.5, 1.5, 2.5, -2.5, 0, -0.0], np.float32))
     if T > 2:
