@@ -169,11 +169,14 @@ def test_linear_tensor_cores(T, O, K, n, m):
     check_linear(T, O, K, n, m, seed=T * 7 + O + K + n)
 
 
-@pytest.mark.parametrize("T,O,K", [(1500, 6000, 320), (1000, 8000, 128), (500, 12000, 64)])
+@pytest.mark.parametrize("T,O,K", [(1500, 6000, 320), (1000, 8000, 128), (500, 12000, 64),
+                                   (1200, 5000, 1152), (700, 9000, 1664)])
 def test_linear_many_tiles_per_cta(T, O, K):
-    """Enough 128 x 240 output tiles that the persistent 2:4 kernel gives each CTA several,
-    so both TMEM accumulators and the stage ring wrap across tiles (ragged rows, tokens
-    and K in each case)."""
+    """Enough 256 x 208 output tiles that the persistent CTA-pair 2:4 kernel gives each pair
+    several, so both TMEM accumulators and the stage rings wrap across tiles (ragged rows,
+    tokens and K in each case).  Odd stage counts per tile (K = 128, 64, 1152, 1664: 1, 1, 5
+    and 7 stages of two K blocks) move the two MMA-issuing threads' share of stages from
+    one tile to the next."""
     check_linear(T, O, K, 2, 4, seed=T + O + K)
 
 
