@@ -202,6 +202,12 @@ class Timer:
             torch.cuda.synchronize(self.dev)
             dist.barrier(self.dev)
             ms = t0.elapsed_time(t1)
+            # the per-call durations right after the timed steps, in the same thermal and
+            # clock state (and inside the clock sampling)
+            if g_ev is not None:
+                with torch.cuda.stream(self.stream):
+                    g_ev.replay()
+                torch.cuda.synchronize(self.dev)
             if clk and ms < 300:  # keep the clocks sampled for at least ~0.3 s of load
                 with torch.cuda.stream(self.stream):
                     for _ in range(max(1, int(300 / max(ms, 1e-3)))):
@@ -212,9 +218,6 @@ class Timer:
                 clk.__exit__()
         per = {}
         if g_ev is not None:
-            with torch.cuda.stream(self.stream):
-                g_ev.replay()
-            torch.cuda.synchronize(self.dev)
             for c in calls:
                 per[c] = sum(e[c][0].elapsed_time(e[c][1]) for e in evs) / steps
         del g, g_ev

@@ -33,7 +33,9 @@
 //              TMEM).  Every role picks super-blocks by the CTA's running counter, so each
 //              ring slot has one producer and one consumer.
 //   warps 6-9  epilogue: drain and add the chains (tcgen05.ld), release them, rescale by
-//              c_t = fp32(fp32(g * s_t) / 127) and store fp32 or bf16.  A row tile whose K
+//              c_t = fp32(fp32(g * s_t) / 127) and store fp32 or bf16.  The unit's layer
+//              record and scales are fetched ahead (software-pipelined over the units), so
+//              short units (K slices) do not wait on those loads after each drain.  A row tile whose K
 //              blocks were split over several units writes its int32 partial to the
 //              workspace; the unit that arrives last on the tile's counter adds the others
 //              (integer sums: the split changes no result bit), stores the tile and resets
@@ -379,14 +381,72 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
     bool failed = false;
     int i = 0;
     int64_t js = 0;  // the super-block counter of the MMA threads
+    // A unit's output description and scales are two pointer chases through the plan (the
+    // layer record, then g and s_t), two L2 round trips that would otherwise sit between the
+    // drain of one unit and the next.  At 16 tokens the record of unit u + 2 is loaded while
+    // unit u is handled, and the scales of unit u + 1; at 32 tokens (no registers to spare
+    // for that) both are loaded before the wait for the unit's accumulators.
+    struct EpiRec {
+      const float *absmax = nullptr, *gamma = nullptr;
+      void *Y = nullptr;
+      int32_t *acc_dbg = nullptr;
+      int32_t T = 0, O = 0;  // at most 32 tokens; rows < 2^31 (checked by the plan)
+      int32_t y_is_bf16 = 0, nparts = 1;
+    };
+    auto load_rec = [&](int u) {
+      EpiRec r;
+      if (u < u1) {
+        const GroupProb &pp = probs[unit(u).prob];
+        r.absmax = pp.absmax;
+        r.gamma = pp.gamma_eff;
+        r.Y = pp.Y;
+        r.acc_dbg = pp.acc_dbg;
+        r.T = (int32_t)pp.T;
+        r.O = (int32_t)pp.O;
+        r.y_is_bf16 = pp.y_is_bf16;
+        r.nparts = pp.nparts;
+      }
+      return r;
+    };
+    auto load_scales = [&](const EpiRec &r, float &g, float &sa) {
+      g = r.gamma ? __ldg(r.gamma) : 0.0f;
+      sa = r.gamma && lane < r.T ? __ldg(r.absmax + lane) : 0.0f;
+    };
+    constexpr bool kAhead = BN <= 16;
+    EpiRec rn, rnn;
+    float gn = 0.0f, sn = 0.0f;
+    if constexpr (kAhead) {
+      rn = load_rec(u0);
+      rnn = load_rec(u0 + 1);
+      load_scales(rn, gn, sn);
+    }
     for (int u = u0; u < u1; ++u, ++i) {
       const int buf = i & 1;
+      // this unit's record and scales (and the loads for the next two units')
+      EpiRec rc;
+      float g, sa;
+      if constexpr (kAhead) {
+        rc = rn;
+        g = gn;
+        sa = sn;
+        rn = rnn;
+        rnn = load_rec(u + 2);
+        load_scales(rn, gn, sn);
+      } else {
+        rc = load_rec(u);
+        load_scales(rc, g, sa);
+      }
       // all four warps stop together if any wait of the previous unit gave up
       if (grp_bar_any(failed)) break;
       const GroupUnit un = unit(u);
       const GroupProb &p = probs[un.prob];
       const int js0m = (int)(js % Cfg::kMma);  // the unit's first super-block, mod kMma
       js += (un.nkb + kSuper - 1) / kSuper;
+      const int64_t T = rc.T, O = rc.O;
+      const int y_is_bf16 = rc.y_is_bf16;
+      void *const Yp = rc.Y;
+      int32_t *const acc_dbg = rc.acc_dbg;
+      const float c_lane = lane < T ? rescale_factor(g, sa) : 0.0f;
       failed = !__all_sync(0xffffffffu, !*s_abort && grp_wait(&acc_full[buf],
                                                               (uint32_t)(i >> 1) & 1u, s_abort));
       ptx::tc_fence_after();
@@ -421,7 +481,7 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
         failed = true;
         break;
       }
-      if (p.nparts > 1) {
+      if (rc.nparts > 1) {
         // K split: publish this part, and let the last part to arrive finish the tile
         int32_t *parts = reinterpret_cast<int32_t *>(ws + part_off) +
                          (p.part_base + (int64_t)un.row_tile * p.nparts) * (kGroupRows * BN);
@@ -450,22 +510,19 @@ __global__ void __launch_bounds__(kGrpThreads, 1)
         if (et == 0) *ticket = 0u;  // ready for the next call
       }
       // rescale and store: lane t holds c_t for token t
-      const int64_t T = p.T, O = p.O;
-      const float g = __ldg(p.gamma_eff);
-      const float c_lane = lane < T ? rescale_factor(g, __ldg(p.absmax + lane)) : 0.0f;
       const int64_t o = (int64_t)un.row_tile * kGroupRows + et;
-      float *yf = reinterpret_cast<float *>(p.Y) + o;
-      __nv_bfloat16 *yb = reinterpret_cast<__nv_bfloat16 *>(p.Y) + o;
+      float *yf = reinterpret_cast<float *>(Yp) + o;
+      __nv_bfloat16 *yb = reinterpret_cast<__nv_bfloat16 *>(Yp) + o;
 #pragma unroll
       for (int t = 0; t < BN; ++t) {
         const float c = __shfl_sync(0xffffffffu, c_lane, t);
         if (t < T && o < O) {
           const float y = __fmul_rn(__int2float_rn(a[t]), c);
-          if (p.y_is_bf16)
+          if (y_is_bf16)
             yb[(int64_t)t * O] = __float2bfloat16_rn(y);
           else
             yf[(int64_t)t * O] = y;
-          if (p.acc_dbg) p.acc_dbg[(int64_t)t * O + o] = a[t];
+          if (acc_dbg) acc_dbg[(int64_t)t * O + o] = a[t];
         }
       }
     }
