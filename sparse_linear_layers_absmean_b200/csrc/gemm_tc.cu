@@ -21,6 +21,8 @@
 //              permute) and stores them in the swizzled K-major layout the MMA reads;
 //              then the epilogue.
 //   warp 5     TMEM allocation and the single MMA-issuing thread.
+// (k_gemm_sp24_pair has its own roles, described at its definition: two MMA-issuing
+// threads, expanders writing TMEM, two producers.)
 // The accumulator carries 64 * acc; the epilogue divides by 64 exactly, multiplies by
 // c_t = fp32(fp32(g * s_t) / 127) and stores fp32 or bf16.
 // Every mbarrier wait gives up after about a second (2^31 SM cycles) and raises
