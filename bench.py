@@ -356,10 +356,13 @@ def bench_stack_decode(args, sbn, dev, local, rank, world, peaks, timer, packed,
         b.record(s_out)
     torch.cuda.synchronize(dev)
     e2e_ms = dist.max_over_ranks(a.elapsed_time(b) / ke, dev)
+    # the outputs that crossed PCIe are the device's outputs, bit for bit
+    e2e_same = bool(torch.equal(hostY, Yall.cpu()))
     h2d = sum(x.numel() * 2 for x in Xh)
     d2h = sum(L["Y"].numel() * 4 for L in layers)
     rec["e2e"] = {"value": total * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                  "outputs_match_device": e2e_same,
                   "api": "GroupPlan.quantize_acts + GroupPlan.linear (sbn_quantize_acts_group, "
                          "sbn_linear_group) as 4 plans of 40 layers; weights resident, X in / Y "
                          "out over PCIe, one copy each way per plan, overlapped with the other "
