@@ -63,12 +63,12 @@ def load_peaks():
 
 
 def peak_source(peaks, key, value, what=""):
-    """Where a roofline denominator came from: the measured file, or (when it is
-    absent) the earlier measurement on the same B200 pool that stands in for it."""
+    """Where a roofline denominator came from: the measured-peaks file beside this script,
+    or (when it is absent) an earlier measurement on B200s of the same kind."""
     if peaks["source"] == "measured":
         return f"{what}{key} of MEASURED_PEAKS.json: of measured"
-    return (f"{what}{key} = {value} (MEASURED_PEAKS.json absent; earlier measurement on "
-            "this B200 pool): of fallback")
+    return (f"{what}{key} = {value} (MEASURED_PEAKS.json absent; an earlier measurement on "
+            "B200): of fallback")
 
 
 def hbm_roof(achieved, peaks, kernel, traffic=None, unit_note=""):
