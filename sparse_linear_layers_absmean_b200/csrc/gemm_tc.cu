@@ -700,7 +700,8 @@ __device__ __forceinline__ bool bar_any(int id, int n, bool pred) {
 // stages at 208 tokens).  Ring 1 (shared memory) is filled by the producers and freed by
 // the MMA's commit of the stage; ring 2 (TMEM) is filled by the expanders, which wait for
 // stage kg - S2's commit before they write stage kg's ring-2 slot.  The tile width 208 puts
-// a 2048-token batch in 10 token tiles (six rounds of tiles on 74 pairs for 11008 rows).
+// a 2048-token batch in 10 token tiles (six rounds of tiles on 74 pairs for 11008 rows); the
+// host takes 192 where that needs no more rounds (4096 rows x 4096 tokens: 5 either way).
 // ---------------------------------------------------------------------------------------
 // 12 warps: expanders 0-3, producers 4 and 10, MMA threads in warps 5 and 11, epilogue 6-9
 constexpr int kPairThreads = 384;
@@ -721,7 +722,9 @@ struct PairCfg {
   // (16 columns each, from the gap's start) and their metadata (4 columns each, after them)
   static constexpr int kAccStride = 256;
   static constexpr int kPerGap = (256 - BN) / 20;
-  static constexpr int kS2 = (2 * kPerGap) / kG;  // TMEM stages
+  // TMEM stages, even: the two MMA threads take alternate stages
+  static constexpr int kS2 = (2 * kPerGap) / kG / 2 * 2;
+  static_assert(kS2 % 2 == 0 && kS1 % 2 == 0, "rings of whole stage pairs");
   static_assert(kS2 >= 2, "at least two TMEM stages");
   static_assert(BN % 16 == 0 && BN <= 224, "pair tile width");
   static_assert(kBHalf % 8 == 0, "B tiles of whole 8-row swizzle atoms");
@@ -1239,9 +1242,18 @@ sbn_status launch_gemm_tc(const int8_t *Xq, const float *absmax, const uint8_t *
                           void *Y, int y_is_bf16, int32_t *acc_dbg, int32_t *err_flag,
                           cudaStream_t st) {
   const bool compact = (n == 2 && m == 4);
-  if (compact && tokens > 128)  // CTA pairs (every sm_100 device runs 2-CTA clusters)
+  if (compact && tokens > 128) {  // CTA pairs (every sm_100 device runs 2-CTA clusters)
+    // tile width: 208 tokens, or 192 where that takes no more rounds of tiles over the
+    // pairs (fewer activation bytes per tile; e.g. 4096 rows x 4096 tokens: 5 rounds either way)
+    const int64_t pairs = num_sms() / 2 > 0 ? num_sms() / 2 : 1;
+    const int64_t n_o = (out + 255) / 256;
+    auto span = [&](int64_t bn) { return (n_o * ((tokens + bn - 1) / bn) + pairs - 1) / pairs * bn; };
+    if (span(192) < span(208))
+      return gemm_sp24_pair_t<192>(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldx, ldc,
+                                   ldm, Y, y_is_bf16, acc_dbg, err_flag, st);
     return gemm_sp24_pair_t<208>(Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldx, ldc, ldm, Y,
                                  y_is_bf16, acc_dbg, err_flag, st);
+  }
   if (tokens > 128)
     return gemm_tc_bn<256>(compact, Xq, absmax, codes, meta, gamma_eff, tokens, out, in, ldx, ldc,
                            ldm, Y, y_is_bf16, acc_dbg, err_flag, st);

@@ -170,14 +170,22 @@ def test_linear_tensor_cores(T, O, K, n, m):
 
 
 @pytest.mark.parametrize("T,O,K", [(1500, 6000, 320), (1000, 8000, 128), (500, 12000, 64),
-                                   (1200, 5000, 1152), (700, 9000, 1664)])
+                                   (1200, 5000, 1152), (700, 9000, 1664), (2048, 11008, 640)])
 def test_linear_many_tiles_per_cta(T, O, K):
-    """Enough 256 x 208 output tiles that the persistent CTA-pair 2:4 kernel gives each pair
+    """Enough 256-row output tiles that the persistent CTA-pair 2:4 kernel gives each pair
     several, so both TMEM accumulators and the stage rings wrap across tiles (ragged rows,
-    tokens and K in each case).  Odd stage counts per tile (K = 128, 64, 1152, 1664: 1, 1, 5
-    and 7 stages of two K blocks) move the two MMA-issuing threads' share of stages from
-    one tile to the next."""
+    tokens and K in each case); 2048 x 11008 takes 208-token tiles, the others 192.  Odd
+    stage counts per tile (K = 128, 64, 1152, 1664, 640: 1, 1, 5, 7 and 3 stages of two K
+    blocks) move the two MMA-issuing threads' share of stages from one tile to the next."""
     check_linear(T, O, K, 2, 4, seed=T + O + K)
+
+
+@pytest.mark.parametrize("T,O,K", [(2048, 4096, 1152), (1500, 2000, 640), (4096, 4096, 512)])
+def test_linear_pair_192_token_tiles(T, O, K):
+    """Shapes where the CTA-pair kernel takes 192-token tiles (no more rounds of tiles over
+    the pairs than 208 would take): ragged last token tile, odd stage counts (K = 1152, 640:
+    5 and 3 stages of two K blocks), one or several tiles per pair."""
+    check_linear(T, O, K, 2, 4, seed=T + O + K + 7)
 
 
 @pytest.mark.parametrize("T,O,K", [(5, 4100, 4096), (16, 1000, 11008), (17, 300, 2048),
