@@ -1019,6 +1019,8 @@ def run_only(args):
     dev = torch.device("cuda", 0)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     calls = args.warmup + args.steps
+    if args.only == "backward" and args.workload != "prefill":
+        sys.exit("--only backward takes the prefill workload (W 11008x4096 2:4, 2048 tokens)")
     if args.workload == "stack":
         packed = build_stack(sbn, dev, 0, err)
         T = workloads.STACK_DECODE_T
@@ -1044,6 +1046,24 @@ def run_only(args):
         pg = sbn.PackGroup(Ws, ((6, 8), (2, 4)), device=dev)
         for _ in range(calls):
             pg.run(err)
+    elif args.only == "backward":
+        cfg = workloads.PREFILL_GEMM
+        O, K, T = cfg["O"], cfg["K"], cfg["T"]
+        W = workloads.masters_device(O, K, device=dev, config=6, tensor=0)
+        X = workloads.torch_bf16(workloads.activations(T, K, seed=0, config=6, tensor=1), dev)
+        g = torch.Generator(device=dev)
+        g.manual_seed(6)
+        dY = torch.randn((T, O), device=dev, generator=g).bfloat16()
+        w = sbn.pack_weights(W, 2, 4, err_flag=err)
+        Xq, s = sbn.quantize_acts(X, err_flag=err)
+        dX = torch.empty((T, K), dtype=torch.float32, device=dev)
+        dW = torch.empty((O, K), dtype=torch.float32, device=dev)
+        ws = torch.empty(sbn.sbn_backward_workspace_bytes(T, O, K), dtype=torch.uint8, device=dev)
+        for _ in range(calls):
+            sbn.sbn_backward(dY, Xq, s, w.codes, w.meta, W, w.gamma_eff, O, K, 2, 4, dX, None, ws,
+                             err)
+            sbn.sbn_backward(dY, Xq, s, w.codes, w.meta, W, w.gamma_eff, O, K, 2, 4, None, dW, ws,
+                             err)
     else:
         cfg = {"decode": workloads.DECODE_GEMV, "prefill": workloads.PREFILL_GEMM}[args.workload]
         O, K, T, n, m = cfg["O"], cfg["K"], cfg["T"], cfg["n"], cfg["m"]
@@ -1087,9 +1107,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub", action="store_true", help="headline only, no sub-records")
-    ap.add_argument("--only", choices=["pack", "act", "linear"],
+    ap.add_argument("--only", choices=["pack", "act", "linear", "backward"],
                     help="profiling aid: one kind of C-ABI call, untimed (decode, prefill, stack; "
-                         "train-step: pack)")
+                         "train-step: pack; prefill: backward, dX then dW)")
     ap.add_argument("--train-layers", type=int, default=workloads.TRAIN_LAYERS,
                     help="profiling aid with --only: decoder layers of the training step "
                          "(default 26)")

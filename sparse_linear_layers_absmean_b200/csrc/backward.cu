@@ -293,100 +293,168 @@ __device__ __forceinline__ uint16_t bf16_of_code(uint32_t c) {
   return c == 1u ? (uint16_t)0x3f80u : c == 3u ? (uint16_t)0xbf80u : (uint16_t)0u;
 }
 
-// Ws^T [K][ldw] bf16 from the packed planes: thread (o, 16-input chunk) decodes 16 weights of
-// row o and writes them down column o (consecutive threads take consecutive rows, so each
-// 16-bit store of a warp is one contiguous 64-byte segment).
+// The operands of the two GEMMs are transposes of the inputs (Ws^T, dY'^T, Xq^T).  Each is
+// built in tiles through shared memory: 8-byte loads along the rows of the input and 8-byte
+// stores along the rows of the output, so both sides move whole 128-byte lines.
+
+// 16 weights of row o, inputs 16c .. 16c + 15, as bf16 {-1, 0, +1} from the packed planes.
+__device__ __forceinline__ void decode_chunk(const uint8_t *__restrict__ codes,
+                                             const uint8_t *__restrict__ meta, int64_t o,
+                                             int64_t c, int64_t ldc, int64_t ldm, int compact,
+                                             uint16_t (&v)[16]) {
+  if (!compact) {
+    // stored element e = k: word e / 16, byte e % 4, bits 6 - 2j .. 7 - 2j, j = (e % 16) / 4
+    const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(codes + o * ldc) + c);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] = bf16_of_code((w >> (8 * (e % 4) + 6 - 2 * (e / 4))) & 3u);
+  } else {
+    // 2:4: the 8 kept codes of these 4 groups are stored elements 8c .. 8c + 7 (word c / 2,
+    // half c % 2); group q's pair of positions is the nibble i0 | i1 << 2 of meta
+    const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(codes + o * ldc) + c / 2);
+    const uint32_t mw = __ldg(reinterpret_cast<const uint16_t *>(meta + o * ldm) + c);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const uint32_t nib = (mw >> (4 * g)) & 15u;
+      const uint32_t i0 = nib & 3u, i1 = nib >> 2;
+      const int se0 = 8 * (int)(c % 2) + 2 * g;  // stored elements se0, se0 + 1 of the word
+      const uint16_t c0 = bf16_of_code((w >> (8 * (se0 % 4) + 6 - 2 * (se0 / 4))) & 3u);
+      const uint16_t c1 = bf16_of_code((w >> (8 * ((se0 + 1) % 4) + 6 - 2 * ((se0 + 1) / 4))) & 3u);
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+        v[4 * g + p] = (uint32_t)p == i0 ? c0 : (uint32_t)p == i1 ? c1 : (uint16_t)0u;
+    }
+  }
+}
+
+// Ws^T [K][ldw] bf16 from the packed planes, in tiles of 64 rows o x 128 inputs: thread
+// (row r, quarter q) decodes the row's 16-input chunks 2q and 2q + 1 of the tile (8
+// contiguous bytes of codes), the tile is transposed through shared memory, and each of its
+// 128 input rows is stored as 64 contiguous bf16.  K is a multiple of 64; O of 8.
 __global__ void __launch_bounds__(256)
     k_bwd_expand_wt(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ meta,
                     int64_t O, int64_t K, int64_t ldc, int64_t ldm, int compact,
                     uint16_t *__restrict__ wt, int64_t ldw) {
+  __shared__ __align__(16) uint16_t tile[128][64 + 4];  // [k][o]; rows 136 bytes apart
   ptx::grid_dep_launch();
   ptx::grid_dep_wait();
-  const int64_t chunks = K / 16, total = O * chunks;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t o = i % O, c = i / O;  // 16 inputs k = 16c .. 16c + 15
+  const int64_t o0 = (int64_t)blockIdx.x * 64, k0 = (int64_t)blockIdx.y * 128;
+  const int r = threadIdx.x >> 2, q = threadIdx.x & 3;
+  const int64_t o = o0 + r, nch = K / 16;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int64_t c = k0 / 16 + 2 * q + h;
     uint16_t v[16];
-    if (!compact) {
-      // stored element e = k: word e / 16, byte e % 4, bits 6 - 2j .. 7 - 2j, j = (e % 16) / 4
-      const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(codes + o * ldc) + c);
-#pragma unroll
-      for (int e = 0; e < 16; ++e)
-        v[e] = bf16_of_code((w >> (8 * (e % 4) + 6 - 2 * (e / 4))) & 3u);
+    if (o < O && c < nch) {
+      decode_chunk(codes, meta, o, c, ldc, ldm, compact, v);
     } else {
-      // 2:4: the 8 kept codes of these 4 groups are stored elements 8c .. 8c + 7 (word c / 2,
-      // half c % 2); group q's pair of positions is the nibble i0 | i1 << 2 of meta
-      const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(codes + o * ldc) + c / 2);
-      const uint32_t mw = __ldg(reinterpret_cast<const uint16_t *>(meta + o * ldm) + c);
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const uint32_t nib = (mw >> (4 * g)) & 15u;
-        const uint32_t i0 = nib & 3u, i1 = nib >> 2;
-        const int se0 = 8 * (int)(c % 2) + 2 * g;  // stored elements se0, se0 + 1 of the word
-        const uint16_t c0 = bf16_of_code((w >> (8 * (se0 % 4) + 6 - 2 * (se0 / 4))) & 3u);
-        const uint16_t c1 = bf16_of_code((w >> (8 * ((se0 + 1) % 4) + 6 - 2 * ((se0 + 1) / 4))) & 3u);
-#pragma unroll
-        for (int p = 0; p < 4; ++p)
-          v[4 * g + p] = (uint32_t)p == i0 ? c0 : (uint32_t)p == i1 ? c1 : (uint16_t)0u;
-      }
+      for (int e = 0; e < 16; ++e) v[e] = 0;
     }
 #pragma unroll
-    for (int e = 0; e < 16; ++e) wt[(16 * c + e) * ldw + o] = v[e];
+    for (int e = 0; e < 16; ++e) tile[(2 * q + h) * 16 + e][r] = v[e];
+  }
+  __syncthreads();
+  const int oc = 4 * (threadIdx.x & 15);
+#pragma unroll
+  for (int pass = 0; pass < 8; ++pass) {
+    const int kk = pass * 16 + (threadIdx.x >> 4);
+    const int64_t k = k0 + kk, oo = o0 + oc;
+    if (k < K && oo < O)
+      *reinterpret_cast<uint2 *>(wt + k * ldw + oo) =
+          *reinterpret_cast<const uint2 *>(&tile[kk][oc]);
   }
 }
 
 // dY'^T as two bf16 terms side by side: out[o][t] = hi, out[o][Tp + t] = lo, where
 // dY' = fp32(dY[t][o] * fp32(s_t / 127)), hi = bf16(dY'), lo = bf16(dY' - hi); zero for
-// t >= T.  32 x 32 tiles through shared memory (coalesced reads along o, writes along t).
+// t >= T.  Tiles of 64 tokens x 64 outputs: 4 bf16 per thread loaded along o, the scale of
+// each token computed once per tile, 4 tokens per thread stored along t (O is a multiple of
+// 8, Tp of 32).
 __global__ void __launch_bounds__(256)
     k_bwd_scale_dy(const uint16_t *__restrict__ dY, const float *__restrict__ absmax, int64_t T,
                    int64_t O, int64_t Tp, uint16_t *__restrict__ out) {
-  __shared__ float tile[32][33];
+  __shared__ float tile[64][64 + 1];  // [t][o]
+  __shared__ float s_c[64];
   ptx::grid_dep_launch();
   ptx::grid_dep_wait();
-  const int64_t o0 = (int64_t)blockIdx.x * 32, t0 = (int64_t)blockIdx.y * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
-  for (int r = ty; r < 32; r += 8) {
-    const int64_t t = t0 + r, o = o0 + tx;
-    float v = 0.0f;
-    if (t < T && o < O) {
-      const float c = __fdiv_rn(__ldg(absmax + t), 127.0f);
-      v = __fmul_rn(__uint_as_float((uint32_t)dY[t * O + o] << 16), c);
-    }
-    tile[r][tx] = v;
+  const int64_t o0 = (int64_t)blockIdx.x * 64, t0 = (int64_t)blockIdx.y * 64;
+  if (threadIdx.x < 64) {
+    const int64_t t = t0 + threadIdx.x;
+    s_c[threadIdx.x] = t < T ? __fdiv_rn(__ldg(absmax + t), 127.0f) : 0.0f;
   }
   __syncthreads();
-  for (int r = ty; r < 32; r += 8) {
-    const int64_t o = o0 + r, t = t0 + tx;
+  const int c4 = 4 * (threadIdx.x & 15);
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {
+    const int tt = pass * 16 + (threadIdx.x >> 4);
+    const int64_t t = t0 + tt, o = o0 + c4;
+    uint2 w = make_uint2(0u, 0u);
+    if (t < T && o < O) w = __ldg(reinterpret_cast<const uint2 *>(dY + t * O + o));
+    const float c = s_c[tt];
+    tile[tt][c4 + 0] = __fmul_rn(__uint_as_float(w.x << 16), c);
+    tile[tt][c4 + 1] = __fmul_rn(__uint_as_float(w.x & 0xffff0000u), c);
+    tile[tt][c4 + 2] = __fmul_rn(__uint_as_float(w.y << 16), c);
+    tile[tt][c4 + 3] = __fmul_rn(__uint_as_float(w.y & 0xffff0000u), c);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {
+    const int oo = pass * 16 + (threadIdx.x >> 4);
+    const int64_t o = o0 + oo, t = t0 + c4;
     if (o >= O || t >= Tp) continue;
-    const float v = tile[tx][r];
-    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(hi)));
-    out[o * (2 * Tp) + t] = __bfloat16_as_ushort(hi);
-    out[o * (2 * Tp) + Tp + t] = __bfloat16_as_ushort(lo);
+    uint32_t hi[2], lo[2];
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      uint32_t h2 = 0, l2 = 0;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const float v = tile[c4 + 2 * p + u][oo];
+        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+        const __nv_bfloat16 l = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(h)));
+        h2 |= (uint32_t)__bfloat16_as_ushort(h) << (16 * u);
+        l2 |= (uint32_t)__bfloat16_as_ushort(l) << (16 * u);
+      }
+      hi[p] = h2;
+      lo[p] = l2;
+    }
+    *reinterpret_cast<uint2 *>(out + o * (2 * Tp) + t) = make_uint2(hi[0], hi[1]);
+    *reinterpret_cast<uint2 *>(out + o * (2 * Tp) + Tp + t) = make_uint2(lo[0], lo[1]);
   }
 }
 
 // Xq^T twice side by side as bf16: out[k][t] = out[k][Tp + t] = Xq[t][k]; zero for t >= T.
+// Tiles of 64 tokens x 64 inputs: 4 int8 per thread loaded along k, 4 tokens per thread
+// stored along t (K is a multiple of 64, Tp of 32).
 __global__ void __launch_bounds__(256)
     k_bwd_transpose_xq(const int8_t *__restrict__ Xq, int64_t T, int64_t K, int64_t Tp,
                        uint16_t *__restrict__ out) {
-  __shared__ float tile[32][33];
+  __shared__ float tile[64][64 + 1];  // [t][k]
   ptx::grid_dep_launch();
   ptx::grid_dep_wait();
-  const int64_t k0 = (int64_t)blockIdx.x * 32, t0 = (int64_t)blockIdx.y * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  for (int r = ty; r < 32; r += 8) {
-    const int64_t t = t0 + r, k = k0 + tx;
-    tile[r][tx] = (t < T && k < K) ? (float)Xq[t * K + k] : 0.0f;
+  const int64_t k0 = (int64_t)blockIdx.x * 64, t0 = (int64_t)blockIdx.y * 64;
+  const int c4 = 4 * (threadIdx.x & 15);
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {
+    const int tt = pass * 16 + (threadIdx.x >> 4);
+    const int64_t t = t0 + tt, k = k0 + c4;
+    uint32_t w = 0;
+    if (t < T && k < K) w = __ldg(reinterpret_cast<const uint32_t *>(Xq + t * K + k));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) tile[tt][c4 + u] = (float)(int8_t)(w >> (8 * u));
   }
   __syncthreads();
-  for (int r = ty; r < 32; r += 8) {
-    const int64_t k = k0 + r, t = t0 + tx;
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {
+    const int kk = pass * 16 + (threadIdx.x >> 4);
+    const int64_t k = k0 + kk, t = t0 + c4;
     if (k >= K || t >= Tp) continue;
-    const uint16_t b = __bfloat16_as_ushort(__float2bfloat16_rn(tile[tx][r]));
-    out[k * (2 * Tp) + t] = b;
-    out[k * (2 * Tp) + Tp + t] = b;
+    uint32_t b[2];
+#pragma unroll
+    for (int p = 0; p < 2; ++p)
+      b[p] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(tile[c4 + 2 * p][kk])) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(tile[c4 + 2 * p + 1][kk])) << 16);
+    *reinterpret_cast<uint2 *>(out + k * (2 * Tp) + t) = make_uint2(b[0], b[1]);
+    *reinterpret_cast<uint2 *>(out + k * (2 * Tp) + Tp + t) = make_uint2(b[0], b[1]);
   }
 }
 
@@ -434,15 +502,11 @@ sbn_status launch_backward(const void *dY, const int8_t *Xq, const float *absmax
   uint16_t *dyt = reinterpret_cast<uint16_t *>(ws + (K * ldw * 2 + 255) / 256 * 256);
   uint16_t *xqt = reinterpret_cast<uint16_t *>(reinterpret_cast<uint8_t *>(dyt) +
                                                (O * 2 * Tp * 2 + 255) / 256 * 256);
-  const int64_t cap = (int64_t)num_sms() * 8;
   EpiArgs e{gamma_eff, static_cast<const uint16_t *>(W)};
   sbn_status s = SBN_OK;
   if (dX) {
-    const int64_t total = O * (K / 16);
-    int64_t grid = (total + 255) / 256;
-    if (grid > cap) grid = cap;
-    s = launch_pdl(k_bwd_expand_wt, dim3((unsigned)grid), dim3(256), 0, st, codes, meta, O, K, ldc,
-                   ldm, (int)(n == 2 && m == 4), wt, ldw);
+    s = launch_pdl(k_bwd_expand_wt, dim3((unsigned)((O + 63) / 64), (unsigned)((K + 127) / 128)),
+                   dim3(256), 0, st, codes, meta, O, K, ldc, ldm, (int)(n == 2 && m == 4), wt, ldw);
     if (s != SBN_OK) return s;
     CUtensorMap ta, tb;
     if (!encode_bf16(&ta, dY, O, T, O, kBwBM) || !encode_bf16(&tb, wt, O, K, ldw, kBwBN / 2))
@@ -451,10 +515,10 @@ sbn_status launch_backward(const void *dY, const int8_t *Xq, const float *absmax
     if (s != SBN_OK) return s;
   }
   if (dW) {
-    s = launch_pdl(k_bwd_scale_dy, dim3((unsigned)((O + 31) / 32), (unsigned)(Tp / 32)), dim3(256),
-                   0, st, static_cast<const uint16_t *>(dY), absmax, T, O, Tp, dyt);
+    s = launch_pdl(k_bwd_scale_dy, dim3((unsigned)((O + 63) / 64), (unsigned)((Tp + 63) / 64)),
+                   dim3(256), 0, st, static_cast<const uint16_t *>(dY), absmax, T, O, Tp, dyt);
     if (s != SBN_OK) return s;
-    s = launch_pdl(k_bwd_transpose_xq, dim3((unsigned)((K + 31) / 32), (unsigned)(Tp / 32)),
+    s = launch_pdl(k_bwd_transpose_xq, dim3((unsigned)((K + 63) / 64), (unsigned)((Tp + 63) / 64)),
                    dim3(256), 0, st, Xq, T, K, Tp, xqt);
     if (s != SBN_OK) return s;
     CUtensorMap ta, tb;
