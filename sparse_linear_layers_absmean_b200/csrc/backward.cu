@@ -297,19 +297,26 @@ __device__ __forceinline__ uint16_t bf16_of_code(uint32_t c) {
 // built in tiles through shared memory: 8-byte loads along the rows of the input and 8-byte
 // stores along the rows of the output, so both sides move whole 128-byte lines.
 
-// 16 weights of row o, inputs 16c .. 16c + 15, as bf16 {-1, 0, +1} from the packed planes.
+// 16 weights of row o, inputs 16c .. 16c + 15, as bf16 {-1, 0, +1} from the packed planes,
+// two per word: v[j] holds inputs 16c + 2j (low half) and 16c + 2j + 1 (high half).
 __device__ __forceinline__ void decode_chunk(const uint8_t *__restrict__ codes,
                                              const uint8_t *__restrict__ meta, int64_t o,
                                              int64_t c, int64_t ldc, int64_t ldm, int compact,
-                                             uint16_t (&v)[16]) {
+                                             uint32_t (&v)[8]) {
   if (!compact) {
     // stored element e = k: word e / 16, byte e % 4, bits 6 - 2j .. 7 - 2j, j = (e % 16) / 4
     const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(codes + o * ldc) + c);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) v[e] = bf16_of_code((w >> (8 * (e % 4) + 6 - 2 * (e / 4))) & 3u);
+    for (int j = 0; j < 8; ++j) {
+      const int e0 = 2 * j, e1 = 2 * j + 1;
+      v[j] = (uint32_t)bf16_of_code((w >> (8 * (e0 % 4) + 6 - 2 * (e0 / 4))) & 3u) |
+             ((uint32_t)bf16_of_code((w >> (8 * (e1 % 4) + 6 - 2 * (e1 / 4))) & 3u) << 16);
+    }
   } else {
     // 2:4: the 8 kept codes of these 4 groups are stored elements 8c .. 8c + 7 (word c / 2,
-    // half c % 2); group q's pair of positions is the nibble i0 | i1 << 2 of meta
+    // half c % 2); group g's pair of positions is the nibble i0 | i1 << 2 of meta.  The
+    // group's four bf16 are one 64-bit word: code 0 at position i0, code 1 at i1 (i0 wins
+    // if the two are equal)
     const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(codes + o * ldc) + c / 2);
     const uint32_t mw = __ldg(reinterpret_cast<const uint16_t *>(meta + o * ldm) + c);
 #pragma unroll
@@ -317,48 +324,56 @@ __device__ __forceinline__ void decode_chunk(const uint8_t *__restrict__ codes,
       const uint32_t nib = (mw >> (4 * g)) & 15u;
       const uint32_t i0 = nib & 3u, i1 = nib >> 2;
       const int se0 = 8 * (int)(c % 2) + 2 * g;  // stored elements se0, se0 + 1 of the word
-      const uint16_t c0 = bf16_of_code((w >> (8 * (se0 % 4) + 6 - 2 * (se0 / 4))) & 3u);
-      const uint16_t c1 = bf16_of_code((w >> (8 * ((se0 + 1) % 4) + 6 - 2 * ((se0 + 1) / 4))) & 3u);
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-        v[4 * g + p] = (uint32_t)p == i0 ? c0 : (uint32_t)p == i1 ? c1 : (uint16_t)0u;
+      const uint64_t c0 = bf16_of_code((w >> (8 * (se0 % 4) + 6 - 2 * (se0 / 4))) & 3u);
+      const uint64_t c1 = bf16_of_code((w >> (8 * ((se0 + 1) % 4) + 6 - 2 * ((se0 + 1) / 4))) & 3u);
+      const uint64_t q = (c0 << (16 * i0)) | (i1 != i0 ? c1 << (16 * i1) : 0ull);
+      v[2 * g] = (uint32_t)q;
+      v[2 * g + 1] = (uint32_t)(q >> 32);
     }
   }
 }
 
 // Ws^T [K][ldw] bf16 from the packed planes, in tiles of 64 rows o x 128 inputs: thread
-// (row r, quarter q) decodes the row's 16-input chunks 2q and 2q + 1 of the tile (8
-// contiguous bytes of codes), the tile is transposed through shared memory, and each of its
-// 128 input rows is stored as 64 contiguous bf16.  K is a multiple of 64; O of 8.
+// (row pair p, chunk q) decodes the tile's 16-input chunk q of rows 2p and 2p + 1 (8
+// threads read a row's 32 contiguous bytes of codes), writes each input's two bf16 as one
+// 32-bit word into the tile, and each of the tile's 128 input rows is stored as 64
+// contiguous bf16.  K is a multiple of 64; O of 8.
 __global__ void __launch_bounds__(256)
     k_bwd_expand_wt(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ meta,
                     int64_t O, int64_t K, int64_t ldc, int64_t ldm, int compact,
                     uint16_t *__restrict__ wt, int64_t ldw) {
-  __shared__ __align__(16) uint16_t tile[128][64 + 4];  // [k][o]; rows 136 bytes apart
+  __shared__ __align__(16) uint32_t tile[128][32 + 2];  // [k][o / 2]; rows 136 bytes apart
   ptx::grid_dep_launch();
   ptx::grid_dep_wait();
   const int64_t o0 = (int64_t)blockIdx.x * 64, k0 = (int64_t)blockIdx.y * 128;
-  const int r = threadIdx.x >> 2, q = threadIdx.x & 3;
-  const int64_t o = o0 + r, nch = K / 16;
+  const int p = threadIdx.x >> 3, q = threadIdx.x & 7;
+  const int64_t o = o0 + 2 * p, c = k0 / 16 + q;
+  uint32_t va[8], vb[8];
+  const bool cin = c < K / 16;
+  if (cin && o < O) {
+    decode_chunk(codes, meta, o, c, ldc, ldm, compact, va);
+  } else {
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int64_t c = k0 / 16 + 2 * q + h;
-    uint16_t v[16];
-    if (o < O && c < nch) {
-      decode_chunk(codes, meta, o, c, ldc, ldm, compact, v);
-    } else {
+    for (int j = 0; j < 8; ++j) va[j] = 0;
+  }
+  if (cin && o + 1 < O) {
+    decode_chunk(codes, meta, o + 1, c, ldc, ldm, compact, vb);
+  } else {
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = 0;
-    }
+    for (int j = 0; j < 8; ++j) vb[j] = 0;
+  }
 #pragma unroll
-    for (int e = 0; e < 16; ++e) tile[(2 * q + h) * 16 + e][r] = v[e];
+  for (int j = 0; j < 8; ++j) {
+    // inputs 16q + 2j (low halves) and 16q + 2j + 1 (high halves) of rows o, o + 1
+    tile[16 * q + 2 * j][p] = (va[j] & 0xffffu) | (vb[j] << 16);
+    tile[16 * q + 2 * j + 1][p] = (va[j] >> 16) | (vb[j] & 0xffff0000u);
   }
   __syncthreads();
-  const int oc = 4 * (threadIdx.x & 15);
+  const int oc = 2 * (threadIdx.x & 15);  // word column: outputs 2 oc .. 2 oc + 3
 #pragma unroll
   for (int pass = 0; pass < 8; ++pass) {
     const int kk = pass * 16 + (threadIdx.x >> 4);
-    const int64_t k = k0 + kk, oo = o0 + oc;
+    const int64_t k = k0 + kk, oo = o0 + 2 * oc;
     if (k < K && oo < O)
       *reinterpret_cast<uint2 *>(wt + k * ldw + oo) =
           *reinterpret_cast<const uint2 *>(&tile[kk][oc]);
