@@ -551,14 +551,21 @@ def bench_train(args, sbn, dev, local, rank, world, peaks, timer, err):
     pg_prev.Ws = []
     del Wp
     cnt = torch.zeros((len(Ws), 3), dtype=torch.int64, device=dev)
+    # the 390 calls are independent (a counter each): four streams, forked from and joined
+    # back to the timed stream, so that the small launches overlap
+    sstreams = [torch.cuda.Stream(device=dev) for _ in range(4)]
 
     def step_stats(i, ev):
         cnt.zero_()
+        for s_ in sstreams:
+            s_.wait_stream(st)
         for k, (W, pw, pp) in enumerate(zip(Ws, pg.packed, pg_prev.packed)):
-            sbn.sbn_count_zero_codes(W, pw[0].gamma_eff, cnt[k, 0:1], st)
+            sbn.sbn_count_zero_codes(W, pw[0].gamma_eff, cnt[k, 0:1], sstreams[k % 2])
             for j in range(2):
                 sbn.sbn_count_mask_flips(pp[j].meta, pw[j].meta, pw[j].out, pw[j].in_, pw[j].n,
-                                         pw[j].m, cnt[k, 1 + j:2 + j], st)
+                                         pw[j].m, cnt[k, 1 + j:2 + j], sstreams[2 + j])
+        for s_ in sstreams:
+            st.wait_stream(s_)
 
     ms_stats, _, _ = timer.run(step_stats, steps, min(args.warmup, 3))
     tot = cnt.sum(dim=0).tolist()
@@ -570,7 +577,8 @@ def bench_train(args, sbn, dev, local, rank, world, peaks, timer, err):
              "flips_2of4": tot[2] / weights, "launches_per_step": 3 * len(Ws),
              "bytes_per_step": stats_bytes,
              "what": "k_count_zero_codes on W (2 B/w) + k_count_mask_flips on both patterns' "
-                     "meta planes of two steps (2 x 0.125 B/w each)"}
+                     "meta planes of two steps (2 x 0.125 B/w each); the per-tensor calls on "
+                     "four streams"}
     moved = weights * 2 * 2 + weights * 3 // 8 + weights // 4  # per pattern: read W + planes
     gbs = moved / (ms * 1e-3) / 1e9
     return {"value": gbs * world, "unit": "GB/s", "ms_per_step": ms, "steps": steps,
@@ -1003,6 +1011,10 @@ def run_cuda(args):
             "bytes_per_step": head.get("bytes_per_step"), "sub": subs,
             "peaks": {k: peaks[k] for k in ("hbm", "bf16", "bf16_sustained", "source")},
         }
+        # the top record's own side measurements (per-tensor calls, mask statistics, ...)
+        for key in ("per_tensor_calls", "mask_stats", "one_layer_calls"):
+            if key in head:
+                line[key] = head[key]
         print(json.dumps(line))
     dist.barrier(dev)
     dist.shutdown()
